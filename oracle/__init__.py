@@ -1,0 +1,250 @@
+"""Python access to the CPU oracle ``libict_oracle.so`` (test infrastructure only).
+
+The oracle is the plain int64 C implementation in ``ict_oracle.c``.  Only the tests,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` import this
+module; the CUDA library never does.  Inputs and outputs are
+``integer_only_nn_02_b200.workloads.CE`` containers (numpy arrays).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+from integer_only_nn_02_b200.workloads import CE, empty_ce
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "ict_oracle.c")
+LIB = os.path.join(HERE, "libict_oracle.so")
+
+ORC_OK, ORC_ERR_ARG, ORC_ERR_LAYOUT, ORC_ERR_EXP_RANGE = 0, 1, 2, 8
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code, what):
+        super().__init__(f"oracle {what} failed with status {code}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (OpenMP over independent output rows)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=gnu11", "-o", tmp, SRC],
+            check=True,
+        )
+        os.replace(tmp, LIB)
+    return LIB
+
+
+class _OT(ctypes.Structure):
+    _fields_ = [
+        ("mant", ctypes.c_void_p),
+        ("exp", ctypes.c_void_p),
+        ("rows", ctypes.c_int64),
+        ("cols", ctypes.c_int64),
+        ("ld", ctypes.c_int64),
+        ("g_rows", ctypes.c_int32),
+        ("g_cols", ctypes.c_int32),
+    ]
+
+
+class _Conv(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")]
+
+
+class _Sgd(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("mom_mul", "mom_shift", "lr_mul", "lr_shift")]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.POINTER
+        L = _lib
+        L.oracle_requant.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                     ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, P(_OT)]
+        L.oracle_align.argtypes = [P(_OT), ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
+                                   ctypes.c_int, ctypes.c_void_p]
+        for name in ("oracle_linear_fwd", "oracle_linear_bwd_data", "oracle_linear_bwd_weight",
+                     "oracle_gelu_bwd"):
+            getattr(L, name).argtypes = [P(_OT), P(_OT), P(_OT)]
+        for name in ("oracle_linear_fwd_acc", "oracle_linear_bwd_data_acc",
+                     "oracle_linear_bwd_weight_acc"):
+            getattr(L, name).argtypes = [P(_OT), P(_OT), ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_gelu_fwd.argtypes = [P(_OT), P(_OT)]
+        L.oracle_conv.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), P(_OT)]
+        L.oracle_conv_acc.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), ctypes.c_void_p,
+                                      ctypes.c_void_p]
+        L.oracle_sgd_step.argtypes = [P(_OT), P(_OT), P(_OT), P(_Sgd)]
+        L.oracle_need64.argtypes = [ctypes.c_int64, ctypes.c_int32]
+        L.oracle_rne_shift64.argtypes = [ctypes.c_int64, ctypes.c_int32]
+        L.oracle_rne_shift64.restype = ctypes.c_int64
+        L.oracle_fit_two_term.argtypes = [ctypes.c_int64] + [ctypes.c_void_p] * 5
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _ot(t: CE) -> _OT:
+    assert t.mant.dtype == np.int8 and t.exp.dtype == np.int8
+    assert t.mant.flags.c_contiguous and t.exp.flags.c_contiguous
+    return _OT(_ptr(t.mant), _ptr(t.exp), t.rows, t.cols, t.cols, t.g_rows, t.g_cols)
+
+
+def _check(code, what):
+    if code != ORC_OK:
+        raise OracleError(code, what)
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+# ------------------------------------------------------------------ primitives
+
+
+def need(x: int, r: int) -> int:
+    """Smallest exponent at which RNE(x * 2^(r-e)) fits in [-127, 127]; -128 for x = 0."""
+    return int(lib().oracle_need64(int(x), int(r)))
+
+
+def rne_shift(x: int, k: int) -> int:
+    """RNE(x * 2^k)."""
+    return int(lib().oracle_rne_shift64(int(x), int(k)))
+
+
+def fit_two_term(a, pa, b, pb):
+    """FIT of one group of values a*2^pa + b*2^pb; returns (mantissas, exponent)."""
+    a = np.ascontiguousarray(a, np.int64)
+    b = np.ascontiguousarray(b, np.int64)
+    pa = np.ascontiguousarray(pa, np.int32)
+    pb = np.ascontiguousarray(pb, np.int32)
+    out = np.zeros(a.shape[0], np.int8)
+    e = lib().oracle_fit_two_term(a.shape[0], _ptr(a), _ptr(pa), _ptr(b), _ptr(pb), _ptr(out))
+    return out, int(e)
+
+
+def requant(x: np.ndarray, g_rows: int, g_cols: int, base_exp: int = 0,
+            row_exp: np.ndarray | None = None, col_exp: np.ndarray | None = None) -> CE:
+    x = np.ascontiguousarray(x, np.int64)
+    rows, cols = x.shape
+    out = empty_ce(rows, cols, g_rows, g_cols)
+    re = None if row_exp is None else np.ascontiguousarray(row_exp, np.int8)
+    ce = None if col_exp is None else np.ascontiguousarray(col_exp, np.int8)
+    code = lib().oracle_requant(rows, cols, _ptr(x), cols, base_exp,
+                                None if re is None else _ptr(re),
+                                None if ce is None else _ptr(ce), ctypes.byref(_ot(out)))
+    _check(code, "requant")
+    return out
+
+
+def align(t: CE, axis: int, transpose: bool = False):
+    """ALIGN_MAX; returns (aligned mantissas, exponent vector)."""
+    shape = (t.cols, t.rows) if transpose else (t.rows, t.cols)
+    out = np.zeros(shape, np.int8)
+    e = np.zeros(t.rows if axis == 1 else t.cols, np.int8)
+    code = lib().oracle_align(ctypes.byref(_ot(t)), axis, _ptr(out), shape[1], int(transpose), _ptr(e))
+    _check(code, "align")
+    return out, e
+
+
+def _product(name, a, b, rows, cols, g_rows, g_cols):
+    out = empty_ce(rows, cols, g_rows, g_cols)
+    _check(getattr(lib(), name)(ctypes.byref(_ot(a)), ctypes.byref(_ot(b)), ctypes.byref(_ot(out))), name)
+    return out
+
+
+def linear_fwd(X: CE, W: CE, g_rows=1, g_cols=32) -> CE:
+    """Y = X * W^T, requantised into (g_rows, g_cols) groups."""
+    return _product("oracle_linear_fwd", X, W, X.rows, W.rows, g_rows, g_cols)
+
+
+def linear_bwd_data(dY: CE, W: CE, g_rows=1, g_cols=32) -> CE:
+    """dX = dY * W."""
+    return _product("oracle_linear_bwd_data", dY, W, dY.rows, W.cols, g_rows, g_cols)
+
+
+def linear_bwd_weight(dY: CE, X: CE, g_rows=1, g_cols=None) -> CE:
+    """dW = dY^T * X (default groups: one per row)."""
+    cols = X.cols
+    return _product("oracle_linear_bwd_weight", dY, X, dY.cols, cols, g_rows, g_cols or cols)
+
+
+def _acc(name, a, b, rows, cols):
+    acc = np.zeros((rows, cols), np.int64)
+    r = np.zeros((rows, cols), np.int32)
+    _check(getattr(lib(), name)(ctypes.byref(_ot(a)), ctypes.byref(_ot(b)), _ptr(acc), _ptr(r)), name)
+    return acc, r
+
+
+def linear_fwd_acc(X, W):
+    return _acc("oracle_linear_fwd_acc", X, W, X.rows, W.rows)
+
+
+def linear_bwd_data_acc(dY, W):
+    return _acc("oracle_linear_bwd_data_acc", dY, W, dY.rows, W.cols)
+
+
+def linear_bwd_weight_acc(dY, X):
+    return _acc("oracle_linear_bwd_weight_acc", dY, X, dY.cols, X.cols)
+
+
+CONV_FWD, CONV_BWD_DATA, CONV_BWD_WEIGHT = 0, 1, 2
+
+
+def _conv_out_shape(direction, d):
+    P = (d["h"] + 2 * d["pad"] - d["r"]) // d["stride"] + 1
+    Q = (d["w"] + 2 * d["pad"] - d["s"]) // d["stride"] + 1
+    if direction == CONV_FWD:
+        return d["n"] * P * Q, d["k"]
+    if direction == CONV_BWD_DATA:
+        return d["n"] * d["h"] * d["w"], d["c"]
+    return d["k"], d["r"] * d["s"] * d["c"]
+
+
+def conv(direction: int, d: dict, a: CE, b: CE, g_rows: int, g_cols: int) -> CE:
+    rows, cols = _conv_out_shape(direction, d)
+    out = empty_ce(rows, cols, g_rows, g_cols)
+    cd = _Conv(*[int(d[k]) for k in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")])
+    _check(lib().oracle_conv(direction, ctypes.byref(cd), ctypes.byref(_ot(a)), ctypes.byref(_ot(b)),
+                             ctypes.byref(_ot(out))), "conv")
+    return out
+
+
+def conv_acc(direction: int, d: dict, a: CE, b: CE):
+    rows, cols = _conv_out_shape(direction, d)
+    acc = np.zeros((rows, cols), np.int64)
+    r = np.zeros((rows, cols), np.int32)
+    cd = _Conv(*[int(d[k]) for k in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")])
+    _check(lib().oracle_conv_acc(direction, ctypes.byref(cd), ctypes.byref(_ot(a)), ctypes.byref(_ot(b)),
+                                 _ptr(acc), _ptr(r)), "conv_acc")
+    return acc, r
+
+
+def sgd_step(W: CE, V: CE, G: CE, mom=(230, 8), lr=(1, 4)):
+    """One integer SGD-momentum step; returns new (W, V) (inputs untouched)."""
+    W2, V2 = W.copy(), V.copy()
+    p = _Sgd(mom[0], mom[1], lr[0], lr[1])
+    _check(lib().oracle_sgd_step(ctypes.byref(_ot(W2)), ctypes.byref(_ot(V2)), ctypes.byref(_ot(G)),
+                                 ctypes.byref(p)), "sgd_step")
+    return W2, V2
+
+
+def gelu_fwd(H: CE) -> CE:
+    out = empty_ce(H.rows, H.cols, H.g_rows, H.g_cols)
+    _check(lib().oracle_gelu_fwd(ctypes.byref(_ot(H)), ctypes.byref(_ot(out))), "gelu_fwd")
+    return out
+
+
+def gelu_bwd(H: CE, dG: CE, g_rows=1, g_cols=32) -> CE:
+    return _product("oracle_gelu_bwd", H, dG, H.rows, H.cols, g_rows, g_cols)

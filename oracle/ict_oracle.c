@@ -1,0 +1,746 @@
+/*
+ * ict_oracle.c -- plain CPU oracle for the integer-only (C,e) training hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is the slow, obviously-correct reference that the
+ * CUDA library is checked against, element by element.  Only the test suite, the
+ * smoke check and the CPU-baseline leg of the benchmark load it.  It shares no code,
+ * header, table or helper with the CUDA library, and the library never calls it.
+ *
+ * Source: "Memory-Efficient Integer-Only Training of Deep Neural Networks"
+ * (Shalby, Pittorino, Roveri).  The page prints the abstract, the Figure 1 caption and
+ * Tables 1-11 but not the equations those cite (Eq. 1, 3, 5, 6, 19), so each routine
+ * below states the passage it follows and the reading it takes where the page is silent.
+ *
+ * Arithmetic is integer only: int64 everywhere, __int128 where a two-term sum needs the
+ * range.  No floating point is used anywhere in this file.
+ *
+ * Representation (Abstract: "signed integer mantissas paired with explicit power-of-two
+ * exponents"; Figure 1 caption: every tensor is a (C,e) pair; Table 7: symmetric clip
+ * bound q_max; Table 5: one exponent byte per group):
+ *   value = C * 2^e,  C in [-127, 127],  e an int8 in [-127, 127],
+ *   e = E_ZERO = -128 marks a group whose mantissas are all zero.
+ *
+ * Parity pins: every public routine is checked in tests/ against closed forms,
+ * hand-derived examples, brute force on tiny inputs and library primitives (numpy
+ * matmul / convolution on the aligned mantissas); see tests/test_oracle_*.py.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define E_ZERO (-128)
+#define QMAX 127
+/* Two-term sums whose exponents are further apart than this are reduced to a sticky
+ * unit (see two_term below); below it they are exact in __int128. */
+#define EXACT_SPAN 100
+
+enum { ORC_OK = 0, ORC_ERR_ARG = 1, ORC_ERR_LAYOUT = 2, ORC_ERR_EXP_RANGE = 8 };
+
+typedef __int128 i128;
+typedef unsigned __int128 u128;
+
+/* A (C,e) matrix view: mantissas row-major with leading dimension ld; exponents on a
+ * grid of groups of g_rows x g_cols elements, row-major, ceil(rows/g_rows) x
+ * ceil(cols/g_cols) bytes.  Groups at the bottom/right edge may be short. */
+typedef struct {
+    int8_t *mant;
+    int8_t *exp;
+    int64_t rows, cols, ld;
+    int32_t g_rows, g_cols;
+} o_tensor;
+
+typedef struct { int32_t n, h, w, c, k, r, s, stride, pad; } o_conv;
+typedef struct { int32_t mom_mul, mom_shift, lr_mul, lr_shift; } o_sgd;
+
+/* ------------------------------------------------------------------------------------ */
+/* Group geometry                                                                        */
+/* ------------------------------------------------------------------------------------ */
+
+static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static int64_t n_grp_rows(const o_tensor *t) { return cdiv(t->rows, t->g_rows); }
+static int64_t n_grp_cols(const o_tensor *t) { return cdiv(t->cols, t->g_cols); }
+
+/* exponent of the group holding element (i, j) */
+static int exp_at(const o_tensor *t, int64_t i, int64_t j) {
+    return t->exp[(i / t->g_rows) * n_grp_cols(t) + (j / t->g_cols)];
+}
+static int mant_at(const o_tensor *t, int64_t i, int64_t j) { return t->mant[i * t->ld + j]; }
+
+/* Checks the input invariants: |C| <= 127 and E_ZERO groups hold only zeros. */
+static int check_input(const o_tensor *t) {
+    if (!t || !t->mant || !t->exp || t->rows < 0 || t->cols < 0 || t->g_rows < 1 ||
+        t->g_cols < 1 || t->ld < t->cols)
+        return ORC_ERR_ARG;
+    for (int64_t i = 0; i < t->rows; i++)
+        for (int64_t j = 0; j < t->cols; j++) {
+            int c = mant_at(t, i, j);
+            if (c < -QMAX || c > QMAX) return ORC_ERR_ARG;
+            if (exp_at(t, i, j) == E_ZERO && c != 0) return ORC_ERR_ARG;
+        }
+    return ORC_OK;
+}
+static int check_output(const o_tensor *t, int64_t rows, int64_t cols) {
+    if (!t || !t->mant || !t->exp || t->g_rows < 1 || t->g_cols < 1) return ORC_ERR_ARG;
+    if (t->rows != rows || t->cols != cols || t->ld < cols) return ORC_ERR_ARG;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Rounding and exponent selection (the requantisation step that follows every Product)  */
+/* ------------------------------------------------------------------------------------ */
+
+/* RNE(x * 2^k): exact for k >= 0; for k < 0 a right shift by s = -k that rounds to the
+ * nearest integer, ties to even.  Reading: the page prints no rounding rule, so
+ * round-half-to-even is taken. */
+static i128 rne_scale(i128 x, int k) {
+    if (k >= 0) return x * ((i128)1 << k); /* callers keep |x| * 2^k far below 2^126 */
+    int s = -k;
+    if (s >= 126) return 0; /* |x| < 2^120 here, so |x| / 2^s < 1/2 */
+    i128 p = (i128)1 << s;
+    /* floor division by 2^s */
+    i128 q = x / p;
+    if (x % p != 0 && x < 0) q -= 1;
+    i128 rem = x - q * p; /* 0 <= rem < 2^s */
+    i128 twice = 2 * rem;
+    if (twice > p || (twice == p && (q & 1))) q += 1;
+    return q;
+}
+
+static int fits_at(i128 x, int r, int e) {
+    i128 q = rne_scale(x, r - e);
+    return q >= -QMAX && q <= QMAX;
+}
+
+static int bitlen(i128 x) {
+    u128 a = x < 0 ? (u128)(-x) : (u128)x;
+    int b = 0;
+    while (a) { a >>= 1; b++; }
+    return b;
+}
+
+/* need(x, r): the smallest exponent e at which RNE(x * 2^(r-e)) fits in [-127, 127], for
+ * x != 0.  Written as the definition: start where it surely does not fit (|x| scaled to
+ * at least 128) and step up until it does.  Reading of the spec requant rule
+ * "smallest exponent that fits the group maximum". */
+static int need(i128 x, int r) {
+    int e = r + bitlen(x) - 8; /* here |x| * 2^(r-e) >= 2^7: does not fit */
+    while (!fits_at(x, r, e)) e++;
+    return e;
+}
+
+/* FIT of one group of n values x[i] at exponents r[i]: the group exponent is the max of
+ * need over the nonzero members (E_ZERO when all are zero), clamped below at -127; each
+ * mantissa is RNE(x[i] * 2^(r[i] - e)).  Returns the exponent, or a value > 127 when the
+ * group cannot be represented (ORC_ERR_EXP_RANGE). */
+static int fit_group(int64_t n, const i128 *x, const int *r, int8_t *c_out) {
+    int have = 0, e = 0;
+    for (int64_t i = 0; i < n; i++) {
+        if (x[i] == 0) continue;
+        int ni = need(x[i], r[i]);
+        if (!have || ni > e) e = ni;
+        have = 1;
+    }
+    if (!have) {
+        for (int64_t i = 0; i < n; i++) c_out[i] = 0;
+        return E_ZERO;
+    }
+    if (e < -127) e = -127;
+    if (e > 127) {
+        for (int64_t i = 0; i < n; i++) c_out[i] = 0;
+        return 1000;
+    }
+    for (int64_t i = 0; i < n; i++) {
+        i128 q = x[i] == 0 ? 0 : rne_scale(x[i], r[i] - e);
+        if (q < -QMAX) q = -QMAX; /* never taken: e fits every member */
+        if (q > QMAX) q = QMAX;
+        c_out[i] = (int8_t)q;
+    }
+    return e;
+}
+
+/* FIT of a whole matrix of values (x at exponent r, element (i,j) at i*cols+j) into the
+ * groups of `out`. */
+static int fit_matrix(const i128 *x, const int *r, o_tensor *out) {
+    int64_t ngr = n_grp_rows(out), ngc = n_grp_cols(out);
+    int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t gi = 0; gi < ngr; gi++) {
+        int64_t i0 = gi * out->g_rows, i1 = i0 + out->g_rows;
+        if (i1 > out->rows) i1 = out->rows;
+        int64_t maxn = (int64_t)out->g_rows * out->g_cols;
+        i128 *gx = malloc(sizeof(i128) * maxn);
+        int *gr = malloc(sizeof(int) * maxn);
+        int8_t *gc = malloc(maxn);
+        for (int64_t gj = 0; gj < ngc; gj++) {
+            int64_t j0 = gj * out->g_cols, j1 = j0 + out->g_cols;
+            if (j1 > out->cols) j1 = out->cols;
+            int64_t n = 0;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++) {
+                    gx[n] = x[i * out->cols + j];
+                    gr[n] = r[i * out->cols + j];
+                    n++;
+                }
+            int e = fit_group(n, gx, gr, gc);
+            if (e > 127) {
+#pragma omp atomic write
+                status = ORC_ERR_EXP_RANGE;
+                e = 127;
+            }
+            out->exp[gi * ngc + gj] = (int8_t)e;
+            n = 0;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++) out->mant[i * out->ld + j] = gc[n++];
+        }
+        free(gx);
+        free(gr);
+        free(gc);
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Sum primitive: exact sum of two (C,e) terms                                          */
+/* ------------------------------------------------------------------------------------ */
+
+/* a*2^pa + b*2^pb as one integer x at exponent r.  Exact (Table 6: "Sum", Eq. 6, read as
+ * an exact integer sum at the smaller exponent) while the exponents are at most
+ * EXACT_SPAN apart.  Beyond that the smaller term is replaced by a one-unit sticky,
+ * sign(b) * 2^(e_hi - EXACT_SPAN): the requantisation of the sum is unchanged, because
+ * its exponent is at least e_hi - 7, every rounding and fitting threshold it compares
+ * against is a multiple of 2^(e_hi - 8), and both the true small term (|b| < 2^16,
+ * so below 2^(e_hi - 84)) and the sticky lie strictly inside the same gap between two
+ * such thresholds next to a * 2^e_hi.  tests/test_oracle_pins.py checks this against
+ * unbounded Python integers. */
+static void two_term(int64_t a, int pa, int64_t b, int pb, i128 *x, int *r) {
+    if (a == 0 && b == 0) { *x = 0; *r = 0; return; }
+    if (a == 0) { *x = b; *r = pb; return; }
+    if (b == 0) { *x = a; *r = pa; return; }
+    if (pa < pb) { int64_t t = a; a = b; b = t; int tp = pa; pa = pb; pb = tp; }
+    /* now pa >= pb: a is the term with the larger exponent */
+    int d = pa - pb;
+    if (d <= EXACT_SPAN) {
+        *x = (i128)a * ((i128)1 << d) + b;
+        *r = pb;
+    } else {
+        *x = (i128)a * ((i128)1 << EXACT_SPAN) + (b > 0 ? 1 : -1);
+        *r = pa - EXACT_SPAN;
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: requantisation                                                                */
+/* ------------------------------------------------------------------------------------ */
+
+/* FIT of int64 values x[i][j] whose exponent is base + row_exp[i] + col_exp[j]
+ * (either vector may be NULL) into the caller-chosen groups of `out`.  This is the
+ * requantisation that closes every Product (Table 6, Eqs. 5 and 3, read as: exact
+ * integer product, exponent addition, then requant to INT8 per group). */
+int oracle_requant(int64_t rows, int64_t cols, const int64_t *x, int64_t ldx, int32_t base_exp,
+                   const int8_t *row_exp, const int8_t *col_exp, o_tensor *out) {
+    if (!x || ldx < cols || check_output(out, rows, cols)) return ORC_ERR_ARG;
+    i128 *v = malloc(sizeof(i128) * (rows * cols + 1));
+    int *r = malloc(sizeof(int) * (rows * cols + 1));
+    int status = ORC_OK;
+    for (int64_t i = 0; i < rows; i++)
+        for (int64_t j = 0; j < cols; j++) {
+            int64_t val = x[i * ldx + j];
+            int re = row_exp ? row_exp[i] : 0, ce = col_exp ? col_exp[j] : 0;
+            if ((re == E_ZERO || ce == E_ZERO) && val != 0) status = ORC_ERR_ARG;
+            v[i * cols + j] = val;
+            r[i * cols + j] = base_exp + re + ce;
+        }
+    if (status == ORC_OK) status = fit_matrix(v, r, out);
+    free(v);
+    free(r);
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: exponent alignment along the contracted index                                 */
+/* ------------------------------------------------------------------------------------ */
+
+/* ALIGN_MAX.  Before an integer contraction every operand whose exponent varies along
+ * the contracted index is brought to one exponent per non-contracted index: the largest
+ * of the group exponents it meets (E_ZERO groups ignored), each mantissa shifted right
+ * to it with RNE.  Reading of the Sum primitive (Table 6, Eq. 6): integer terms are
+ * added at a common exponent, the larger one, so the aligned mantissas stay INT8.
+ *   axis = 1: contracted index runs along columns -> one exponent per row (rows entries)
+ *   axis = 0: contracted index runs along rows    -> one exponent per column
+ * out (ld_out) receives the aligned mantissas, transposed when `transpose` is set. */
+int oracle_align(const o_tensor *in, int axis, int8_t *out, int64_t ld_out, int transpose,
+                 int8_t *e_star) {
+    int st = check_input(in);
+    if (st) return st;
+    if (!out || !e_star || (axis != 0 && axis != 1)) return ORC_ERR_ARG;
+    int64_t n_keep = axis == 1 ? in->rows : in->cols;
+    int64_t n_red = axis == 1 ? in->cols : in->rows;
+    for (int64_t a = 0; a < n_keep; a++) {
+        int have = 0, m = E_ZERO;
+        for (int64_t b = 0; b < n_red; b++) {
+            int64_t i = axis == 1 ? a : b, j = axis == 1 ? b : a;
+            int e = exp_at(in, i, j);
+            if (e == E_ZERO) continue;
+            if (!have || e > m) m = e;
+            have = 1;
+        }
+        e_star[a] = (int8_t)m;
+        for (int64_t b = 0; b < n_red; b++) {
+            int64_t i = axis == 1 ? a : b, j = axis == 1 ? b : a;
+            int c = mant_at(in, i, j);
+            int q = 0;
+            if (c != 0) q = (int)rne_scale(c, exp_at(in, i, j) - m);
+            if (transpose) out[j * ld_out + i] = (int8_t)q;
+            else out[i * ld_out + j] = (int8_t)q;
+        }
+    }
+    return ORC_OK;
+}
+
+/* dense aligned copy (rows x cols, ld = cols) + exponent vector */
+static int align_dense(const o_tensor *t, int axis, int8_t **m, int8_t **e) {
+    *m = malloc(t->rows * t->cols + 1);
+    *e = malloc((axis == 1 ? t->rows : t->cols) + 1);
+    return oracle_align(t, axis, *m, t->cols, 0, *e);
+}
+
+static int sum_exp(int a, int b) { return (a == E_ZERO || b == E_ZERO) ? 0 : a + b; }
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: linear layer, three training directions                                      */
+/* ------------------------------------------------------------------------------------ */
+
+/* Pre-requant accumulators of the forward product Y = X * W^T (Figure 1a; Table 6:
+ * "Linear / fully-connected: Product"): align X per row and W per row (both contract
+ * along their columns), exact int64 dot products, exponents added. */
+int oracle_linear_fwd_acc(const o_tensor *X, const o_tensor *W, int64_t *acc, int32_t *r) {
+    int st;
+    if ((st = check_input(X)) || (st = check_input(W))) return st;
+    if (X->cols != W->cols) return ORC_ERR_ARG;
+    int8_t *xa, *xe, *wa, *we;
+    align_dense(X, 1, &xa, &xe);
+    align_dense(W, 1, &wa, &we);
+    int64_t M = X->rows, N = W->rows, K = X->cols;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; k++) s += (int64_t)xa[m * K + k] * wa[n * K + k];
+            acc[m * N + n] = s;
+            r[m * N + n] = sum_exp(xe[m], we[n]);
+        }
+    free(xa); free(xe); free(wa); free(we);
+    return ORC_OK;
+}
+
+/* Pre-requant accumulators of dX = dY * W: dY aligned per row, W per column (its
+ * contracted index, the output feature, runs along W's rows). */
+int oracle_linear_bwd_data_acc(const o_tensor *dY, const o_tensor *W, int64_t *acc, int32_t *r) {
+    int st;
+    if ((st = check_input(dY)) || (st = check_input(W))) return st;
+    if (dY->cols != W->rows) return ORC_ERR_ARG;
+    int8_t *ya, *ye, *wa, *we;
+    align_dense(dY, 1, &ya, &ye);
+    align_dense(W, 0, &wa, &we);
+    int64_t M = dY->rows, N = W->rows, K = W->cols;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t k = 0; k < K; k++) {
+            int64_t s = 0;
+            for (int64_t n = 0; n < N; n++) s += (int64_t)ya[m * N + n] * wa[n * K + k];
+            acc[m * K + k] = s;
+            r[m * K + k] = sum_exp(ye[m], we[k]);
+        }
+    free(ya); free(ye); free(wa); free(we);
+    return ORC_OK;
+}
+
+/* Pre-requant accumulators of dW = dY^T * X: both aligned per column (the contracted
+ * index, the token, runs along their rows). */
+int oracle_linear_bwd_weight_acc(const o_tensor *dY, const o_tensor *X, int64_t *acc, int32_t *r) {
+    int st;
+    if ((st = check_input(dY)) || (st = check_input(X))) return st;
+    if (dY->rows != X->rows) return ORC_ERR_ARG;
+    int8_t *ya, *ye, *xa, *xe;
+    align_dense(dY, 0, &ya, &ye);
+    align_dense(X, 0, &xa, &xe);
+    int64_t M = dY->rows, N = dY->cols, K = X->cols;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            int64_t s = 0;
+            for (int64_t m = 0; m < M; m++) s += (int64_t)ya[m * N + n] * xa[m * K + k];
+            acc[n * K + k] = s;
+            r[n * K + k] = sum_exp(ye[n], xe[k]);
+        }
+    free(ya); free(ye); free(xa); free(xe);
+    return ORC_OK;
+}
+
+static int fit_acc(const int64_t *acc, const int32_t *r, o_tensor *out) {
+    int64_t n = out->rows * out->cols;
+    i128 *v = malloc(sizeof(i128) * (n + 1));
+    int *rr = malloc(sizeof(int) * (n + 1));
+    for (int64_t i = 0; i < n; i++) { v[i] = acc[i]; rr[i] = r[i]; }
+    int st = fit_matrix(v, rr, out);
+    free(v);
+    free(rr);
+    return st;
+}
+
+typedef int (*acc_fn)(const o_tensor *, const o_tensor *, int64_t *, int32_t *);
+static int product(acc_fn f, const o_tensor *a, const o_tensor *b, o_tensor *out,
+                   int64_t rows, int64_t cols) {
+    if (check_output(out, rows, cols)) return ORC_ERR_ARG;
+    int64_t *acc = malloc(sizeof(int64_t) * (rows * cols + 1));
+    int32_t *r = malloc(sizeof(int32_t) * (rows * cols + 1));
+    int st = f(a, b, acc, r);
+    if (!st) st = fit_acc(acc, r, out);
+    free(acc);
+    free(r);
+    return st;
+}
+
+int oracle_linear_fwd(const o_tensor *X, const o_tensor *W, o_tensor *Y) {
+    return product(oracle_linear_fwd_acc, X, W, Y, X->rows, W->rows);
+}
+int oracle_linear_bwd_data(const o_tensor *dY, const o_tensor *W, o_tensor *dX) {
+    return product(oracle_linear_bwd_data_acc, dY, W, dX, dY->rows, W->cols);
+}
+int oracle_linear_bwd_weight(const o_tensor *dY, const o_tensor *X, o_tensor *dW) {
+    return product(oracle_linear_bwd_weight_acc, dY, X, dW, dY->cols, X->cols);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: convolution (Table 6: "Convolution (incl. 1x1, depthwise): Product")          */
+/* ------------------------------------------------------------------------------------ */
+
+/* NHWC activations viewed as [n*h*w][c] (C,e) matrices whose exponent groups span all
+ * pixels (g_rows >= rows: one exponent per channel group, uniform over pixels);
+ * KRSC weights viewed as [k][r*s*c].  Directions:
+ *   dir 0 forward      a = X  [N*H*W][C], b = W [K][R*S*C], out = Y  [N*P*Q][K]
+ *   dir 1 bwd-data     a = dY [N*P*Q][K], b = W [K][R*S*C], out = dX [N*H*W][C]
+ *   dir 2 bwd-weight   a = dY [N*P*Q][K], b = X [N*H*W][C], out = dW [K][R*S*C]
+ * with P = (H + 2 pad - R) / stride + 1, zero padding.  Alignment: fwd aligns the
+ * activation to the largest channel-group exponent and W per output channel; bwd-data
+ * aligns dY the same way and W per input channel c (max over k, r, s); bwd-weight
+ * aligns dY and X per channel over all pixels. */
+static int64_t out_dim(int64_t in, int pad, int ker, int stride) {
+    return (in + 2 * pad - ker) / stride + 1;
+}
+
+int oracle_conv_acc(int dir, const o_conv *d, const o_tensor *a, const o_tensor *b, int64_t *acc,
+                    int32_t *rexp) {
+    int st;
+    if (!d || d->stride < 1 || d->pad < 0 || d->r < 1 || d->s < 1) return ORC_ERR_ARG;
+    if ((st = check_input(a)) || (st = check_input(b))) return st;
+    int64_t N = d->n, H = d->h, Wd = d->w, C = d->c, K = d->k, R = d->r, S = d->s;
+    int64_t P = out_dim(H, d->pad, R, d->stride), Q = out_dim(Wd, d->pad, S, d->stride);
+    if (P < 1 || Q < 1) return ORC_ERR_ARG;
+    int64_t npix_in = N * H * Wd, npix_out = N * P * Q, RSC = R * S * C;
+
+    if (dir == 0 || dir == 1) {
+        /* activation operand: X (fwd) or dY (bwd-data); exponent uniform over pixels */
+        const o_tensor *act = a;
+        int64_t act_rows = dir == 0 ? npix_in : npix_out, act_cols = dir == 0 ? C : K;
+        if (act->rows != act_rows || act->cols != act_cols) return ORC_ERR_ARG;
+        if (act->g_rows < act->rows) return ORC_ERR_LAYOUT;
+        if (b->rows != K || b->cols != RSC) return ORC_ERR_ARG;
+        int8_t *aa = malloc(act_rows * act_cols + 1), *ae = malloc(act_rows + 1);
+        oracle_align(act, 1, aa, act_cols, 0, ae); /* every row gets the same e* */
+        int ea = act_rows ? ae[0] : E_ZERO;
+        int8_t *wa = malloc(K * RSC + 1);
+        int8_t *we;
+        if (dir == 0) {
+            we = malloc(K + 1);
+            oracle_align(b, 1, wa, RSC, 0, we); /* per output channel k */
+        } else {
+            /* per input channel c: max over k, r, s of the group exponent */
+            we = malloc(C + 1);
+            for (int64_t c = 0; c < C; c++) {
+                int have = 0, m = E_ZERO;
+                for (int64_t k = 0; k < K; k++)
+                    for (int64_t rs = 0; rs < R * S; rs++) {
+                        int e = exp_at(b, k, rs * C + c);
+                        if (e == E_ZERO) continue;
+                        if (!have || e > m) m = e;
+                        have = 1;
+                    }
+                we[c] = (int8_t)m;
+                for (int64_t k = 0; k < K; k++)
+                    for (int64_t rs = 0; rs < R * S; rs++) {
+                        int v = mant_at(b, k, rs * C + c);
+                        wa[k * RSC + rs * C + c] =
+                            v ? (int8_t)rne_scale(v, exp_at(b, k, rs * C + c) - m) : 0;
+                    }
+            }
+        }
+        if (dir == 0) {
+#pragma omp parallel for schedule(static)
+            for (int64_t op = 0; op < npix_out; op++) {
+                int64_t n = op / (P * Q), p = (op / Q) % P, q = op % Q;
+                for (int64_t k = 0; k < K; k++) {
+                    int64_t s = 0;
+                    for (int64_t r = 0; r < R; r++)
+                        for (int64_t ss = 0; ss < S; ss++) {
+                            int64_t h = p * d->stride + r - d->pad, w = q * d->stride + ss - d->pad;
+                            if (h < 0 || h >= H || w < 0 || w >= Wd) continue;
+                            const int8_t *xr = aa + ((n * H + h) * Wd + w) * C;
+                            const int8_t *wr = wa + k * RSC + (r * S + ss) * C;
+                            for (int64_t c = 0; c < C; c++) s += (int64_t)xr[c] * wr[c];
+                        }
+                    acc[op * K + k] = s;
+                    rexp[op * K + k] = sum_exp(ea, we[k]);
+                }
+            }
+        } else {
+#pragma omp parallel for schedule(static)
+            for (int64_t ip = 0; ip < npix_in; ip++) {
+                int64_t n = ip / (H * Wd), h = (ip / Wd) % H, w = ip % Wd;
+                for (int64_t c = 0; c < C; c++) {
+                    int64_t s = 0;
+                    for (int64_t r = 0; r < R; r++)
+                        for (int64_t ss = 0; ss < S; ss++) {
+                            int64_t ph = h + d->pad - r, qw = w + d->pad - ss;
+                            if (ph < 0 || qw < 0 || ph % d->stride || qw % d->stride) continue;
+                            int64_t p = ph / d->stride, q = qw / d->stride;
+                            if (p >= P || q >= Q) continue;
+                            const int8_t *yr = aa + ((n * P + p) * Q + q) * K;
+                            for (int64_t k = 0; k < K; k++)
+                                s += (int64_t)yr[k] * wa[k * RSC + (r * S + ss) * C + c];
+                        }
+                    acc[ip * C + c] = s;
+                    rexp[ip * C + c] = sum_exp(ea, we[c]);
+                }
+            }
+        }
+        free(aa); free(ae); free(wa); free(we);
+        return ORC_OK;
+    }
+    if (dir == 2) {
+        if (a->rows != npix_out || a->cols != K || b->rows != npix_in || b->cols != C)
+            return ORC_ERR_ARG;
+        int8_t *ya, *ye, *xa, *xe;
+        align_dense(a, 0, &ya, &ye); /* per output channel k, over all pixels */
+        align_dense(b, 0, &xa, &xe); /* per input channel c, over all pixels */
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < K; k++)
+            for (int64_t rs = 0; rs < R * S; rs++) {
+                int64_t r = rs / S, ss = rs % S;
+                for (int64_t c = 0; c < C; c++) {
+                    int64_t s = 0;
+                    for (int64_t n = 0; n < N; n++)
+                        for (int64_t p = 0; p < P; p++)
+                            for (int64_t q = 0; q < Q; q++) {
+                                int64_t h = p * d->stride + r - d->pad, w = q * d->stride + ss - d->pad;
+                                if (h < 0 || h >= H || w < 0 || w >= Wd) continue;
+                                s += (int64_t)ya[((n * P + p) * Q + q) * K + k] *
+                                     xa[((n * H + h) * Wd + w) * C + c];
+                            }
+                    acc[k * RSC + rs * C + c] = s;
+                    rexp[k * RSC + rs * C + c] = sum_exp(ye[k], xe[c]);
+                }
+            }
+        free(ya); free(ye); free(xa); free(xe);
+        return ORC_OK;
+    }
+    return ORC_ERR_ARG;
+}
+
+int oracle_conv(int dir, const o_conv *d, const o_tensor *a, const o_tensor *b, o_tensor *out) {
+    if (!d || d->stride < 1) return ORC_ERR_ARG;
+    int64_t P = out_dim(d->h, d->pad, d->r, d->stride), Q = out_dim(d->w, d->pad, d->s, d->stride);
+    int64_t rows, cols;
+    if (dir == 0) { rows = (int64_t)d->n * P * Q; cols = d->k; }
+    else if (dir == 1) { rows = (int64_t)d->n * d->h * d->w; cols = d->c; }
+    else if (dir == 2) { rows = d->k; cols = (int64_t)d->r * d->s * d->c; }
+    else return ORC_ERR_ARG;
+    if (check_output(out, rows, cols)) return ORC_ERR_ARG;
+    int64_t *acc = malloc(sizeof(int64_t) * (rows * cols + 1));
+    int32_t *r = malloc(sizeof(int32_t) * (rows * cols + 1));
+    int st = oracle_conv_acc(dir, d, a, b, acc, r);
+    if (!st) st = fit_acc(acc, r, out);
+    free(acc);
+    free(r);
+    return st;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: integer SGD with momentum and per-group velocity (Figure 1b)                  */
+/* ------------------------------------------------------------------------------------ */
+
+/* One step of SGD with momentum, every tensor a (C,e) pair with its own exponent per
+ * group (Abstract: "per-group velocity mechanism with independent exponent tracking";
+ * Figure 1b; Table 10: SGD with momentum beta = 0.9).  Reading: the usual form
+ *     v <- beta * v + g ;   w <- w - lr * v
+ * with beta = mom_mul * 2^-mom_shift and lr = lr_mul * 2^-lr_shift as integer
+ * multiply-shifts, each right-hand side an exact two-term Sum requantised once by FIT
+ * into the group (so both exponents are chosen afresh every step).  W, V and G share
+ * one group partition; W and V are updated in place. */
+int oracle_sgd_step(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p) {
+    int st;
+    if (!p) return ORC_ERR_ARG;
+    if ((st = check_input(W)) || (st = check_input(V)) || (st = check_input(G))) return st;
+    if (W->rows != V->rows || W->rows != G->rows || W->cols != V->cols || W->cols != G->cols ||
+        W->g_rows != V->g_rows || W->g_rows != G->g_rows || W->g_cols != V->g_cols ||
+        W->g_cols != G->g_cols)
+        return ORC_ERR_ARG;
+    if (p->mom_shift < 0 || p->lr_shift < 0) return ORC_ERR_ARG;
+    int64_t ngr = n_grp_rows(W), ngc = n_grp_cols(W);
+    int status = ORC_OK;
+#pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < ngr; gi++) {
+        int64_t maxn = (int64_t)W->g_rows * W->g_cols;
+        i128 *x = malloc(sizeof(i128) * maxn);
+        int *r = malloc(sizeof(int) * maxn);
+        int8_t *cv = malloc(maxn), *cw = malloc(maxn);
+        for (int64_t gj = 0; gj < ngc; gj++) {
+            int64_t i0 = gi * W->g_rows, i1 = i0 + W->g_rows, j0 = gj * W->g_cols,
+                    j1 = j0 + W->g_cols;
+            if (i1 > W->rows) i1 = W->rows;
+            if (j1 > W->cols) j1 = W->cols;
+            int64_t ge = gi * ngc + gj;
+            int ev = V->exp[ge], eg = G->exp[ge], ew = W->exp[ge];
+            /* velocity: mom_mul * Cv * 2^(ev - mom_shift) + Cg * 2^eg */
+            int64_t n = 0;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++, n++)
+                    two_term((int64_t)p->mom_mul * mant_at(V, i, j), ev - p->mom_shift,
+                             mant_at(G, i, j), eg, &x[n], &r[n]);
+            int ev2 = fit_group(n, x, r, cv);
+            /* weight: Cw * 2^ew - lr_mul * Cv' * 2^(ev' - lr_shift) */
+            n = 0;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++, n++)
+                    two_term(mant_at(W, i, j), ew, -(int64_t)p->lr_mul * cv[n],
+                             ev2 - p->lr_shift, &x[n], &r[n]);
+            int ew2 = fit_group(n, x, r, cw);
+            if (ev2 > 127 || ew2 > 127) {
+#pragma omp atomic write
+                status = ORC_ERR_EXP_RANGE;
+                if (ev2 > 127) ev2 = 127;
+                if (ew2 > 127) ew2 = 127;
+            }
+            V->exp[ge] = (int8_t)ev2;
+            W->exp[ge] = (int8_t)ew2;
+            n = 0;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++, n++) {
+                    V->mant[i * V->ld + j] = cv[n];
+                    W->mant[i * W->ld + j] = cw[n];
+                }
+        }
+        free(x); free(r); free(cv); free(cw);
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: integer GELU                                                                  */
+/* ------------------------------------------------------------------------------------ */
+
+/* C * 2^e >= 2, decided exactly */
+static int at_least_two(int64_t c, int e) {
+    if (e >= 1) return c >= 1;
+    if (1 - e > 100) return 0;
+    return (i128)c >= ((i128)1 << (1 - e));
+}
+
+/* Forward of the piecewise GELU h(x) = x * clip((x + 2) / 4, 0, 1) on (C,e), the
+ * exponent carried through unchanged (Table 7 caption: pointwise activations act on the
+ * mantissa and keep e).  Reading: the page's own GELU is a lookup table (Table 7, Eq. 19)
+ * whose contents are not printed; this shift-friendly curve stands in for it.
+ *   x <= -2: 0;  x >= 2: x;  otherwise x (x + 2) / 4 = C^2 2^(2e-2) + C 2^(e-1),
+ * rounded RNE to the input exponent.  E_ZERO groups stay zero. */
+int oracle_gelu_fwd(const o_tensor *H, o_tensor *out) {
+    int st;
+    if ((st = check_input(H))) return st;
+    if (check_output(out, H->rows, H->cols) || out->g_rows != H->g_rows ||
+        out->g_cols != H->g_cols)
+        return ORC_ERR_ARG;
+    int64_t ne = n_grp_rows(H) * n_grp_cols(H);
+    memcpy(out->exp, H->exp, ne);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < H->rows; i++)
+        for (int64_t j = 0; j < H->cols; j++) {
+            int c = mant_at(H, i, j), e = exp_at(H, i, j);
+            int o;
+            if (c == 0 || e == E_ZERO) o = 0;
+            else if (at_least_two(-c, e)) o = 0;
+            else if (at_least_two(c, e)) o = c;
+            else {
+                i128 x;
+                int r;
+                two_term((int64_t)c * c, 2 * e - 2, c, e - 1, &x, &r);
+                o = (int)rne_scale(x, r - e);
+            }
+            out->mant[i * out->ld + j] = (int8_t)o;
+        }
+    return ORC_OK;
+}
+
+/* Backward of the same curve: dH = dG * h'(x) with h'(x) = 0 for x <= -2, 1 for x >= 2
+ * and (x + 1) / 2 in between, i.e. dG * x / 2 + dG / 2 as an exact two-term Sum, then
+ * FIT into the groups of dH.  H and dG share one shape. */
+int oracle_gelu_bwd(const o_tensor *H, const o_tensor *dG, o_tensor *dH) {
+    int st;
+    if ((st = check_input(H)) || (st = check_input(dG))) return st;
+    if (H->rows != dG->rows || H->cols != dG->cols) return ORC_ERR_ARG;
+    int64_t rows = H->rows, cols = H->cols;
+    if (check_output(dH, rows, cols)) return ORC_ERR_ARG;
+    i128 *x = malloc(sizeof(i128) * (rows * cols + 1));
+    int *r = malloc(sizeof(int) * (rows * cols + 1));
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < rows; i++)
+        for (int64_t j = 0; j < cols; j++) {
+            int ch = mant_at(H, i, j), eh = exp_at(H, i, j);
+            int cd = mant_at(dG, i, j), ed = exp_at(dG, i, j);
+            i128 v = 0;
+            int rr = 0;
+            if (cd != 0) {
+                if (eh == E_ZERO) ch = 0;
+                if (ch != 0 && at_least_two(-ch, eh)) { v = 0; }
+                else if (ch != 0 && at_least_two(ch, eh)) { v = cd; rr = ed; }
+                else two_term((int64_t)cd * ch, ed + eh - 1, cd, ed - 1, &v, &rr);
+            }
+            x[i * cols + j] = v;
+            r[i * cols + j] = rr;
+        }
+    st = fit_matrix(x, r, dH);
+    free(x);
+    free(r);
+    return st;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Introspection for the tests                                                           */
+/* ------------------------------------------------------------------------------------ */
+
+/* need() and RNE on int64 inputs, exported so the tests can pin them by brute force. */
+int oracle_need64(int64_t x, int32_t r) { return x == 0 ? E_ZERO : need(x, r); }
+int64_t oracle_rne_shift64(int64_t x, int32_t k) { return (int64_t)rne_scale(x, k); }
+
+/* FIT of one group of two-term values (a[i] * 2^pa[i] + b[i] * 2^pb[i]), exported so the
+ * tests can compare the sticky reduction against unbounded integers. */
+int oracle_fit_two_term(int64_t n, const int64_t *a, const int32_t *pa, const int64_t *b,
+                        const int32_t *pb, int8_t *c_out) {
+    i128 *x = malloc(sizeof(i128) * (n + 1));
+    int *r = malloc(sizeof(int) * (n + 1));
+    for (int64_t i = 0; i < n; i++) two_term(a[i], pa[i], b[i], pb[i], &x[i], &r[i]);
+    int e = fit_group(n, x, r, c_out);
+    free(x);
+    free(r);
+    return e;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
