@@ -1,0 +1,205 @@
+/*
+ * ict.h -- C ABI of libict.so: the integer-only (C,e) training hot path on B200 (sm_100a).
+ *
+ * Method: "Memory-Efficient Integer-Only Training of Deep Neural Networks" (Shalby,
+ * Pittorino, Roveri).  Every training tensor is a pair (C,e): INT8 signed mantissas C
+ * with an explicit power-of-two exponent e per tensor or per group (Abstract; Figure 1
+ * caption).  Layers are built from integer primitives (Abstract: products, sums,
+ * divide-by-constant, nonlinear functions, weight updates; Table 6 maps convolution and
+ * linear layers onto the Product primitive).  The page prints neither the equations nor
+ * a rounding rule; the readings this library implements are:
+ *
+ *   value(C, e)   = C * 2^e,  C in [-127, 127],  e an int8 in [-127, 127];
+ *                   e = ICT_E_ZERO (-128) marks a group whose mantissas are all zero.
+ *   need(x, r)    = the smallest exponent e at which RNE(x * 2^(r - e)) lies in
+ *                   [-127, 127] (x an exact integer at exponent r; RNE = round half
+ *                   to even).
+ *   FIT(group)    = requantisation after every product: the group exponent is the
+ *                   largest need() of its nonzero members (ICT_E_ZERO when all are
+ *                   zero), raised to at least -127; each mantissa is
+ *                   RNE(x * 2^(r - e)).
+ *   ALIGN_MAX     = before a contraction, an operand whose exponent varies along the
+ *                   contracted index is brought, per non-contracted index, to the
+ *                   largest group exponent it meets (ICT_E_ZERO groups ignored), each
+ *                   mantissa shifted right with RNE (reading of the Sum primitive,
+ *                   Table 6 Eq. 6).
+ *   Product       = exact integer dot product of aligned mantissas (int32, int64 where a
+ *                   long contraction needs it), exponents added, then FIT into the
+ *                   caller's output groups.  No int32 result is ever visible to the
+ *                   caller.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are allocated and owned by the caller.  The library allocates no
+ *     memory; scratch space is the caller's `ws` buffer, sized by the matching
+ *     *_workspace() query.  ws must be 256-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void *; NULL is
+ *     the legacy default stream) and never synchronises, except
+ *     ict_get_device_status().
+ *   - Argument errors are returned before anything is launched.  Conditions found on the
+ *     device (an exponent above 127, a bounded wait that ran out) are OR-ed into a sticky
+ *     device status word read by ict_get_device_status().
+ *   - Unsupported geometry returns ICT_ERR_LAYOUT; there is no fallback path.
+ *   - Mantissa matrices are row-major with a leading dimension `ld` (elements = bytes);
+ *     outputs never alias inputs, except that the SGD step updates W and V in place.
+ *   - Inputs must satisfy |C| <= 127 and have all-zero mantissas in ICT_E_ZERO groups
+ *     (every output of this library does).  Other inputs give unspecified (but
+ *     memory-safe) results.
+ */
+#ifndef ICT_H
+#define ICT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ICT_E_ZERO (-128)
+#define ICT_QMAX 127
+
+typedef enum {
+    ICT_OK = 0,
+    ICT_ERR_INVALID_ARG = 1,    /* null pointer, bad size, inconsistent shapes */
+    ICT_ERR_LAYOUT = 2,         /* group geometry or shape this build does not support */
+    ICT_ERR_ALIGNMENT = 3,      /* pointer or leading dimension not 16-byte aligned */
+    ICT_ERR_WORKSPACE = 4,      /* ws too small or not 256-byte aligned */
+    ICT_ERR_UNSUPPORTED_ARCH = 5, /* current device is not sm_100 */
+    ICT_ERR_CUDA = 6,           /* a CUDA runtime or driver call failed */
+    ICT_ERR_DEVICE_TIMEOUT = 7, /* (device word) a bounded wait inside a kernel ran out */
+    ICT_ERR_EXP_RANGE = 8       /* (device word) a result needed an exponent above 127 */
+} ict_status;
+
+/* One (C,e) matrix view.
+ *   mant   [rows][ld] int8, |C| <= 127
+ *   exp    [ceil(rows/g_rows)][ceil(cols/g_cols)] int8, row-major, contiguous;
+ *          group (i, j) covers rows [i*g_rows, ...) and columns [j*g_cols, ...);
+ *          edge groups may be short.  g_rows >= rows means one group row (uniform over
+ *          rows), g_cols >= cols one group column.
+ *   For outputs the caller chooses g_rows/g_cols and the library writes mant and exp. */
+typedef struct {
+    int8_t *mant;
+    int8_t *exp;
+    int64_t rows, cols, ld;
+    int32_t g_rows, g_cols;
+} ict_tensor;
+
+/* SGD with momentum as integer multiply-shifts: beta = mom_mul * 2^-mom_shift,
+ * lr = lr_mul * 2^-lr_shift (Table 10: momentum 0.9 -> 230, 8). */
+typedef struct {
+    int32_t mom_mul, mom_shift, lr_mul, lr_shift;
+} ict_sgd_params;
+
+/* NHWC activations, KRSC weights.  Activations are ict_tensor views
+ * [n*h*w][c] (or [n*p*q][k]); weights are [k][r*s*c]. */
+typedef struct {
+    int32_t n, h, w, c, k, r, s, stride, pad;
+} ict_conv_desc;
+
+typedef enum { ICT_CONV_FWD = 0, ICT_CONV_BWD_DATA = 1, ICT_CONV_BWD_WEIGHT = 2 } ict_conv_dir;
+
+typedef enum { ICT_OP_LINEAR_FWD = 0, ICT_OP_LINEAR_BWD_DATA = 1, ICT_OP_LINEAR_BWD_WEIGHT = 2 } ict_linear_op;
+
+/* Human-readable name of a status code (static string). */
+const char *ict_status_string(int32_t status);
+
+/* Reads the sticky device status word into *host_out and clears it.  Synchronises
+ * `stream`.  ICT_OK means no device-side condition was raised since the last call. */
+int32_t ict_get_device_status(int32_t *host_out, void *stream);
+
+/* Library build identification: returns a static string. */
+const char *ict_version(void);
+
+/* Number of kernels this process has launched through the library so far (all devices,
+ * all threads).  Lets a caller count the device work a sequence of calls issues. */
+uint64_t ict_launch_count(void);
+
+/* Bound, in nanoseconds, of every wait inside a kernel (0 restores the default, 2 s).
+ * A wait that runs out raises ICT_ERR_DEVICE_TIMEOUT in the device status word; the
+ * kernel then lets its in-flight copies and tensor-core operations finish (again with a
+ * bound), releases its tensor memory and exits, leaving the context usable and the
+ * outputs unspecified.  Process-wide; meant for tests of that path. */
+int32_t ict_set_wait_limit_ns(uint64_t ns);
+
+/* --------------------------------------------------------------------------------- */
+/* Requantisation (FIT) of integer values, the step that closes every Product         */
+/* (Table 6, Eqs. 5 and 3; Figure 1a).                                                 */
+/*   vals      device [rows][ld_vals] of int32 (val_bits = 32) or int64 (64)            */
+/*   element (i, j) has exponent base_exp + row_exp[i] + col_exp[j]                      */
+/*   (row_exp / col_exp: device int8 vectors, either may be NULL = 0; an ICT_E_ZERO      */
+/*   entry requires the value to be 0)                                                  */
+/*   out       groups chosen by the caller; rows/cols must match                        */
+int32_t ict_requant(const void *vals, int32_t val_bits, int64_t rows, int64_t cols,
+                    int64_t ld_vals, int32_t base_exp, const int8_t *row_exp,
+                    const int8_t *col_exp, ict_tensor *out, void *stream);
+
+/* ALIGN_MAX of one operand (reading of the Sum primitive, Table 6 Eq. 6).
+ *   axis = 1: the contracted index runs along columns -> e_star[rows]
+ *   axis = 0: the contracted index runs along rows    -> e_star[cols]
+ *   out_mant  device, [rows][ld_out] (or [cols][ld_out] when transpose = 1)
+ *   e_star    device int8 vector of the aligned exponents                           */
+int32_t ict_align(const ict_tensor *in, int32_t axis, int32_t transpose, int8_t *out_mant,
+                  int64_t ld_out, int8_t *e_star, void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* Linear layer Product in the three training directions (Figure 1a; Table 6          */
+/* "Linear / fully-connected").  Operands whose exponent varies along the contracted   */
+/* index are aligned (ALIGN_MAX) into `ws` first; the int8 x int8 -> int32 contraction */
+/* runs on the tensor cores and the FIT requant is fused into its epilogue where the   */
+/* output groups lie inside one tile.                                                 */
+/*   fwd          Y[M][N]  = X[M][K] * W[N][K]^T                                       */
+/*   bwd_data     dX[M][K] = dY[M][N] * W[N][K]                                        */
+/*   bwd_weight   dW[N][K] = dY[M][N]^T * X[M][K]                                      */
+/* Output groups must be row-local (g_rows = 1).  Leading dimensions and pointers must */
+/* be 16-byte aligned.                                                                 */
+size_t ict_linear_workspace(int32_t op, const ict_tensor *a, const ict_tensor *b,
+                            const ict_tensor *out);
+int32_t ict_linear_fwd(const ict_tensor *X, const ict_tensor *W, ict_tensor *Y, void *ws,
+                       size_t ws_bytes, void *stream);
+int32_t ict_linear_bwd_data(const ict_tensor *dY, const ict_tensor *W, ict_tensor *dX,
+                            void *ws, size_t ws_bytes, void *stream);
+int32_t ict_linear_bwd_weight(const ict_tensor *dY, const ict_tensor *X, ict_tensor *dW,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* Convolution as implicit GEMM (Table 6: "Convolution ... Product").                  */
+/*   dir FWD         a = X  [n*h*w][c], b = W [k][r*s*c] -> out = Y  [n*p*q][k]        */
+/*   dir BWD_DATA    a = dY [n*p*q][k], b = W [k][r*s*c] -> out = dX [n*h*w][c]        */
+/*   dir BWD_WEIGHT  a = dY [n*p*q][k], b = X [n*h*w][c] -> out = dW [k][r*s*c]        */
+/* Activation exponents must be uniform over pixels (g_rows >= rows); activation       */
+/* output groups likewise (g_rows >= rows, g_cols a multiple of 16); dW groups are     */
+/* per row.  This build supports 3x3, stride 1, pad 1, c and k multiples of 64 up to   */
+/* 256, w <= 128.                                                                      */
+size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d);
+int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_tensor *a,
+                               const ict_tensor *b, ict_tensor *out, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* Integer SGD with momentum and per-group velocity (Figure 1b; Abstract: "per-group   */
+/* velocity mechanism with independent exponent tracking").  Per group:                */
+/*   v <- FIT(beta * v + g)      w <- FIT(w - lr * v)                                  */
+/* each right-hand side an exact two-term Sum.  W, V, G share one shape and one        */
+/* row-local group partition (g_rows = 1); W and V are updated in place.               */
+int32_t ict_sgd_momentum_step(ict_tensor *W, ict_tensor *V, const ict_tensor *G,
+                              const ict_sgd_params *p, void *stream);
+/* The same update over n_tensors independent (W, V, G) triples in one launch
+ * (n_tensors <= 128). */
+int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W,
+                                    ict_tensor *const *V, const ict_tensor *const *G,
+                                    const ict_sgd_params *p, void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* Integer GELU stand-in h(x) = x * clip((x + 2) / 4, 0, 1) (the page's GELU is a      */
+/* lookup table, Table 7 / Eq. 19, whose contents are not printed).                    */
+/*   fwd: exponent carried through unchanged (Table 7 caption); out has H's groups.    */
+/*   bwd: dH = FIT(dG * h'(H)) into dH's groups; H, dG, dH share one row-local group   */
+/*        partition.                                                                    */
+int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream);
+int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ICT_H */

@@ -1,0 +1,890 @@
+// ict_api.cu -- the C ABI of libict.so (declared in include/ict.h).
+//
+// Host side only: argument validation, workspace planning, TMA descriptor encoding and
+// the composition align -> tensor-core Product -> FIT of each entry point.  Every step
+// of the arithmetic runs in the kernels of ict_elementwise.cuh and ict_gemm.cuh.
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "ict_device.cuh"
+#include "ict_elementwise.cuh"
+#include "ict_gemm.cuh"
+
+using namespace ict;
+
+namespace {
+
+// ------------------------------------------------------------------ device checks
+
+struct DeviceInfo {
+    bool checked = false;
+    int status = ICT_OK;
+    int sms = 0;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+uint64_t g_wait_ns = 2000000000ull;  // bound of every mbarrier wait inside a kernel
+const uint64_t kDrainNs = 1000000000ull;
+
+int device_info(int *sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ICT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return ICT_ERR_CUDA;
+        d.status = (major == 10 && minor == 0) ? ICT_OK : ICT_ERR_UNSUPPORTED_ARCH;
+        d.sms = n;
+        d.checked = true;
+    }
+    if (sms) *sms = d.sms;
+    return d.status;
+}
+// SM count for planning; 148 (B200) when no device is visible (workspace queries only)
+int planning_sms() {
+    int sms = 0;
+    if (device_info(&sms) != ICT_OK || sms <= 0) return 148;
+    return sms;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? ICT_OK : ICT_ERR_CUDA; }
+
+// number of kernels launched through this library (process-wide)
+std::atomic<uint64_t> g_launches{0};
+void counted(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// ------------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)ptr;
+    }
+    return fn;
+}
+
+// int8 matrix [outer][inner] with row stride `stride` bytes; box inner x outer.
+int tmap_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t stride,
+            uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return ICT_ERR_CUDA;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {stride};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ICT_OK : ICT_ERR_CUDA;
+}
+
+// Dense NHWC int8 activations [n][h][w][c]; box 64 channels x w x rows x 1 image,
+// 64-byte swizzle (one K block of the implicit GEMM).
+int tmap_nhwc(CUtensorMap *m, const void *base, int n, int h, int w, int c, uint32_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return ICT_ERR_CUDA;
+    cuuint64_t dims[4] = {(cuuint64_t)c, (cuuint64_t)w, (cuuint64_t)h, (cuuint64_t)n};
+    cuuint64_t strides[3] = {(cuuint64_t)c, (cuuint64_t)w * c, (cuuint64_t)h * w * c};
+    cuuint32_t box[4] = {64, (cuuint32_t)w, rows, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ICT_OK : ICT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ tensors
+
+int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
+int64_t n_grp_rows(const ict_tensor *t) { return cdiv64(t->rows, t->g_rows); }
+int64_t n_grp_cols(const ict_tensor *t) { return cdiv64(t->cols, t->g_cols); }
+bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+int clamp_div(int64_t g, int64_t n) { return (int)(g < n ? g : (n > 0 ? n : 1)); }
+
+int check_tensor(const ict_tensor *t) {
+    if (!t || t->rows < 0 || t->cols < 0 || t->g_rows < 1 || t->g_cols < 1 || t->ld < t->cols)
+        return ICT_ERR_INVALID_ARG;
+    if (t->rows > 0 && t->cols > 0 && (!t->mant || !t->exp)) return ICT_ERR_INVALID_ARG;
+    if (t->rows >= (1ll << 31) || t->cols >= (1ll << 31)) return ICT_ERR_LAYOUT;
+    return ICT_OK;
+}
+// tensors read or written by 16-byte vectors / TMA
+int check_vec(const ict_tensor *t) {
+    if (!aligned16(t->mant) || (t->ld & 15)) return ICT_ERR_ALIGNMENT;
+    if (t->cols & 15) return ICT_ERR_LAYOUT;
+    if (t->g_cols < t->cols && (t->g_cols & 15)) return ICT_ERR_LAYOUT;
+    return ICT_OK;
+}
+bool uniform_along_cols(const ict_tensor *t) { return t->g_cols >= t->cols; }
+
+// ------------------------------------------------------------------ workspace
+
+struct Ws {
+    uint8_t *base;
+    size_t cap, used;
+    bool dry;
+    void *take(size_t bytes) {
+        used = (size_t)round_up((int64_t)used, 256);
+        void *p = dry ? nullptr : base + used;
+        used += bytes;
+        return p;
+    }
+};
+Ws make_ws(void *ws, size_t bytes, bool dry) { return Ws{(uint8_t *)ws, bytes, 0, dry}; }
+
+// ------------------------------------------------------------------ kernel launchers
+
+struct AlignJob {
+    const ict_tensor *t;
+    int axis;
+    bool transpose;
+    int8_t *out;
+    int64_t ld;
+    int8_t *e_star;
+};
+
+int launch_align(const AlignJob &j, cudaStream_t s) {
+    const ict_tensor *in = j.t;
+    if (in->rows == 0 || in->cols == 0) return ICT_OK;
+    AlignArgs a;
+    a.in = in->mant;
+    a.in_exp = in->exp;
+    a.rows = in->rows;
+    a.cols = in->cols;
+    a.ld = in->ld;
+    a.g_rows = clamp_div(in->g_rows, in->rows);
+    a.g_cols = clamp_div(in->g_cols, in->cols);
+    a.ngc = n_grp_cols(in);
+    a.axis = j.axis;
+    a.out = j.out;
+    a.out_ld = j.ld;
+    a.e_star = j.e_star;
+    if (j.axis == 1)
+        estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
+    else
+        estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
+    dim3 grid((unsigned)cdiv64(in->cols, 64), (unsigned)cdiv64(in->rows, 64));
+    if (j.transpose)
+        align_tile_kernel<true><<<grid, 256, 0, s>>>(a);
+    else
+        align_tile_kernel<false><<<grid, 256, 0, s>>>(a);
+    counted(2);
+    return launch_status();
+}
+
+int launch_requant_rows(RequantArgs a, cudaStream_t s) {
+    const int64_t groups = a.rows * a.ngc;
+    if (groups == 0) return ICT_OK;
+    requant_rows_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+int launch_zero(const ict_tensor *out, cudaStream_t s) {
+    const int64_t n = out->rows * out->cols, ne = n_grp_rows(out) * n_grp_cols(out);
+    const int64_t m = n > ne ? n : ne;
+    if (m == 0) return ICT_OK;
+    zero_ce_kernel<<<(unsigned)cdiv64(m, 256), 256, 0, s>>>(out->mant, out->rows, out->cols, out->ld,
+                                                           out->exp, ne);
+    counted(1);
+    return launch_status();
+}
+
+// ---- tensor-core Product
+
+constexpr int stages_for(int bn, int bk) {
+    return bk == 128 ? (bn <= 64 ? 8 : bn <= 128 ? 6 : bn <= 192 ? 5 : 4)
+                     : (bn <= 64 ? 12 : bn <= 128 ? 10 : 8);
+}
+
+template <int BN, int BK, int LOAD>
+int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid,
+                  cudaStream_t s) {
+    constexpr int ST = stages_for(BN, BK);
+    using L = GemmSmem<BN, BK, ST>;
+    auto k = gemm_ce_kernel<BN, BK, ST, LOAD>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+        return ICT_ERR_CUDA;
+    k<<<grid, 256, L::kBytes, s>>>(ta, tb, p);
+    counted(1);
+    return launch_status();
+}
+
+int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
+                const GemmParams &p, int grid, cudaStream_t s) {
+#define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
+    if (bn == BN_ && bk == BK_ && load == LOAD_) \
+        return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s);
+    ICT_GEMM_CASE(64, 128, LOAD_2D)
+    ICT_GEMM_CASE(128, 128, LOAD_2D)
+    ICT_GEMM_CASE(192, 128, LOAD_2D)
+    ICT_GEMM_CASE(256, 128, LOAD_2D)
+    ICT_GEMM_CASE(64, 64, LOAD_CONV)
+    ICT_GEMM_CASE(128, 64, LOAD_CONV)
+    ICT_GEMM_CASE(192, 64, LOAD_CONV)
+    ICT_GEMM_CASE(256, 64, LOAD_CONV)
+#undef ICT_GEMM_CASE
+    return ICT_ERR_LAYOUT;
+}
+
+int pick_bn(int64_t n) {
+    if (n <= 64) return 64;
+    if (n <= 128) return 128;
+    if (n <= 192) return 192;
+    if (n % 256 == 0) return 256;
+    if (n % 192 == 0) return 192;
+    if (n % 128 == 0) return 128;
+    return 256;
+}
+
+// A K-major operand of the Product: rows of int8, K contiguous, an exponent per row.
+struct Operand {
+    const int8_t *mant;
+    int64_t rows, k, ld;
+    const int8_t *exp;
+    int exp_div;  // exponent of row i is exp[i / exp_div]
+};
+
+// Operand whose contracted index runs along the tensor's columns.
+Operand operand_rows(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
+    if (uniform_along_cols(t))
+        return Operand{t->mant, t->rows, t->cols, t->ld, t->exp, clamp_div(t->g_rows, t->rows)};
+    const int64_t ld = round_up(t->cols, 16);
+    int8_t *m = (int8_t *)ws.take((size_t)t->rows * ld);
+    int8_t *e = (int8_t *)ws.take((size_t)t->rows);
+    jobs[(*njobs)++] = AlignJob{t, 1, false, m, ld, e};
+    return Operand{m, t->rows, t->cols, ld, e, 1};
+}
+// Operand whose contracted index runs along the tensor's rows: aligned per column and
+// transposed into K-major rows.
+Operand operand_cols(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
+    const int64_t ld = round_up(t->rows, 16);
+    int8_t *m = (int8_t *)ws.take((size_t)t->cols * ld);
+    int8_t *e = (int8_t *)ws.take((size_t)t->cols);
+    jobs[(*njobs)++] = AlignJob{t, 0, true, m, ld, e};
+    return Operand{m, t->cols, t->rows, ld, e, 1};
+}
+
+struct ProductPlan {
+    int bn, splits, kblk_per_split, n_kblk, n_mtiles, n_ntiles, units, grid;
+    bool fused;
+    int32_t *ws32;
+    int64_t ws_ld;
+};
+
+// Tiling of D[M][N] = A[M][K] B[N][K]^T with FIT into the row-local groups of `out`.
+ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out, int sms,
+                         bool allow_split, Ws &ws) {
+    ProductPlan pl;
+    pl.bn = pick_bn(N);
+    pl.n_kblk = (int)cdiv64(K, 128);
+    pl.n_mtiles = (int)cdiv64(M, 128);
+    pl.n_ntiles = (int)cdiv64(N, pl.bn);
+    const int tiles = pl.n_mtiles * pl.n_ntiles;
+    int splits = 1;
+    if (allow_split && tiles < sms && pl.n_kblk >= 8) {
+        splits = (int)std::min<int64_t>(cdiv64(sms, tiles), pl.n_kblk / 4);
+        if (splits < 1) splits = 1;
+    }
+    // int32 partial sums stay exact: at most 2^17 products of magnitude <= 127^2 each
+    const int max_kblk = (1 << 17) / 128;
+    if (cdiv64(pl.n_kblk, splits) > max_kblk) splits = (int)cdiv64(pl.n_kblk, max_kblk);
+    pl.kblk_per_split = (int)cdiv64(pl.n_kblk, splits);
+    pl.splits = (int)cdiv64(pl.n_kblk, pl.kblk_per_split);
+    pl.units = tiles * pl.splits;
+    pl.grid = std::min(pl.units, sms);
+    const int64_t G = out->g_cols;
+    const bool groups_in_tile = (G >= N) ? (N <= pl.bn) : (pl.bn % G == 0 && G % 32 == 0);
+    pl.fused = pl.splits == 1 && groups_in_tile;
+    pl.ws_ld = round_up(N, 32);
+    pl.ws32 = pl.fused ? nullptr : (int32_t *)ws.take((size_t)pl.splits * M * pl.ws_ld * 4);
+    return pl;
+}
+
+int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const ProductPlan &pl,
+                cudaStream_t s) {
+    const int64_t M = A.rows, N = B.rows, K = A.k;
+    CUtensorMap ta, tb;
+    int st;
+    if ((st = tmap_2d(&ta, A.mant, K, M, A.ld, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return st;
+    if ((st = tmap_2d(&tb, B.mant, K, N, B.ld, 128, pl.bn, CU_TENSOR_MAP_SWIZZLE_128B))) return st;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = (int)M;
+    p.N = (int)N;
+    p.n_kblk = pl.n_kblk;
+    p.n_mtiles = pl.n_mtiles;
+    p.n_ntiles = pl.n_ntiles;
+    p.splits = pl.splits;
+    p.kblk_per_split = pl.kblk_per_split;
+    p.num_units = pl.units;
+    p.eA = A.exp;
+    p.eA_div = A.exp_div;
+    p.eB = B.exp;
+    p.eB_div = B.exp_div;
+    p.G = (int)std::min<int64_t>(out->g_cols, N);
+    p.out = out->mant;
+    p.out_ld = out->ld;
+    p.out_exp = out->exp;
+    p.out_exp_ld = n_grp_cols(out);
+    p.ws32 = pl.ws32;
+    p.ws_ld = pl.ws_ld;
+    p.ws_split_stride = M * pl.ws_ld;
+    p.stage_tx_bytes = (uint32_t)(128 * 128 + pl.bn * 128);
+    p.wait_ns = g_wait_ns;
+    p.drain_ns = kDrainNs;
+    p.epi = pl.fused ? EPI_FIT_ROW : EPI_I32;
+    if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s))) return st;
+    if (pl.fused) return ICT_OK;
+    RequantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.v32 = pl.ws32;
+    a.nsplit = pl.splits;
+    a.split_stride = M * pl.ws_ld;
+    a.rows = M;
+    a.cols = N;
+    a.ld = pl.ws_ld;
+    a.row_exp = A.exp;
+    a.row_div = A.exp_div;
+    a.col_exp = B.exp;
+    a.col_div = B.exp_div;
+    a.out = out->mant;
+    a.out_ld = out->ld;
+    a.out_exp = out->exp;
+    a.G = (int)std::min<int64_t>(out->g_cols, N);
+    a.ngc = n_grp_cols(out);
+    return launch_requant_rows(a, s);
+}
+
+// ---- linear layer
+
+struct LinearPlan {
+    AlignJob jobs[2];
+    int njobs;
+    Operand A, B;
+    ProductPlan pp;
+    const ict_tensor *out;
+    bool empty;  // K == 0: the result is zero
+};
+
+int plan_linear(int op, const ict_tensor *a, const ict_tensor *b, const ict_tensor *out, Ws &ws,
+                LinearPlan *lp) {
+    int st;
+    if ((st = check_tensor(a)) || (st = check_tensor(b)) || (st = check_tensor(out))) return st;
+    int64_t M, N, K;
+    if (op == ICT_OP_LINEAR_FWD) {  // Y = X W^T
+        if (a->cols != b->cols) return ICT_ERR_INVALID_ARG;
+        M = a->rows, N = b->rows, K = a->cols;
+    } else if (op == ICT_OP_LINEAR_BWD_DATA) {  // dX = dY W
+        if (a->cols != b->rows) return ICT_ERR_INVALID_ARG;
+        M = a->rows, N = b->cols, K = a->cols;
+    } else if (op == ICT_OP_LINEAR_BWD_WEIGHT) {  // dW = dY^T X
+        if (a->rows != b->rows) return ICT_ERR_INVALID_ARG;
+        M = a->cols, N = b->cols, K = a->rows;
+    } else {
+        return ICT_ERR_INVALID_ARG;
+    }
+    if (out->rows != M || out->cols != N) return ICT_ERR_INVALID_ARG;
+    if (out->g_rows != 1 && M > 1) return ICT_ERR_LAYOUT;
+    if ((st = check_vec(out))) return st;
+    if ((st = check_vec(a)) || (st = check_vec(b))) return st;
+    lp->out = out;
+    lp->njobs = 0;
+    lp->empty = (K == 0);
+    if (M == 0 || N == 0 || K == 0) return ICT_OK;
+    if (op == ICT_OP_LINEAR_FWD) {
+        lp->A = operand_rows(a, ws, lp->jobs, &lp->njobs);
+        lp->B = operand_rows(b, ws, lp->jobs, &lp->njobs);
+    } else if (op == ICT_OP_LINEAR_BWD_DATA) {
+        lp->A = operand_rows(a, ws, lp->jobs, &lp->njobs);
+        lp->B = operand_cols(b, ws, lp->jobs, &lp->njobs);
+    } else {
+        lp->A = operand_cols(a, ws, lp->jobs, &lp->njobs);
+        lp->B = operand_cols(b, ws, lp->jobs, &lp->njobs);
+    }
+    lp->pp = plan_product(M, N, K, out, planning_sms(), op == ICT_OP_LINEAR_BWD_WEIGHT, ws);
+    return ICT_OK;
+}
+
+int run_linear(const LinearPlan &lp, cudaStream_t s) {
+    if (lp.empty) return launch_zero(lp.out, s);
+    if (lp.out->rows == 0 || lp.out->cols == 0) return ICT_OK;
+    int st;
+    for (int i = 0; i < lp.njobs; ++i)
+        if ((st = launch_align(lp.jobs[i], s))) return st;
+    return run_product(lp.A, lp.B, lp.out, lp.pp, s);
+}
+
+int linear_entry(int op, const ict_tensor *a, const ict_tensor *b, ict_tensor *out, void *ws,
+                 size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    LinearPlan lp;
+    Ws w = make_ws(ws, ws_bytes, false);
+    if ((st = plan_linear(op, a, b, out, w, &lp))) return st;
+    if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
+    return run_linear(lp, (cudaStream_t)stream);
+}
+
+// ---- convolution (implicit GEMM, NHWC / KRSC, "same" 3x3-style, stride 1)
+
+struct ConvPlan {
+    AlignJob jobs[2];
+    int njobs;
+    bool weight_prep;      // backward-data: W'[c][(r,s,k)] aligned per input channel
+    ConvWeightArgs wprep;
+    const int8_t *a_mant;  // dense NHWC activation operand fed to TMA
+    int a_c;               // its channel count (the contracted channels)
+    const int8_t *eA;
+    int eA_div;
+    const int8_t *b_mant;  // K-major weight operand [N][taps * a_c]
+    int64_t b_ld;
+    const int8_t *eB;
+    int eB_div;
+    int64_t out_rows, out_cols;
+    int bn, rows_per_tile, tiles_per_img;
+    bool global_groups;
+    int32_t *gmax;
+    int n_gcols;
+};
+
+int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
+              const ict_tensor *out, Ws &ws, ConvPlan *cp) {
+    int st;
+    if (!d) return ICT_ERR_INVALID_ARG;
+    if ((st = check_tensor(a)) || (st = check_tensor(b)) || (st = check_tensor(out))) return st;
+    if (d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1 || d->k < 1 || d->r < 1 || d->s < 1 ||
+        d->stride < 1 || d->pad < 0)
+        return ICT_ERR_INVALID_ARG;
+    if (d->stride != 1 || d->r != d->s || 2 * d->pad != d->r - 1) return ICT_ERR_LAYOUT;
+    if (d->c % 64 || d->k % 64 || d->c > 256 || d->k > 256 || d->w > 128) return ICT_ERR_LAYOUT;
+    const int64_t npix = (int64_t)d->n * d->h * d->w, RS = (int64_t)d->r * d->s;
+    if (dir == ICT_CONV_BWD_WEIGHT) return ICT_ERR_LAYOUT;
+    if (dir != ICT_CONV_FWD && dir != ICT_CONV_BWD_DATA) return ICT_ERR_INVALID_ARG;
+    const int64_t act_c = dir == ICT_CONV_FWD ? d->c : d->k;  // contracted channels
+    const int64_t out_c = dir == ICT_CONV_FWD ? d->k : d->c;
+    if (a->rows != npix || a->cols != act_c) return ICT_ERR_INVALID_ARG;
+    if (b->rows != d->k || b->cols != RS * d->c) return ICT_ERR_INVALID_ARG;
+    if (out->rows != npix || out->cols != out_c) return ICT_ERR_INVALID_ARG;
+    if (a->g_rows < a->rows) return ICT_ERR_LAYOUT;  // activation exponents uniform over pixels
+    if ((st = check_vec(a)) || (st = check_vec(b)) || (st = check_vec(out))) return st;
+    cp->global_groups = out->g_rows >= out->rows;
+    if (!cp->global_groups && out->g_rows != 1) return ICT_ERR_LAYOUT;
+    cp->bn = pick_bn(out_c);
+    const int64_t G = out->g_cols;
+    if (!(G >= out_c ? out_c <= cp->bn : (cp->bn % G == 0 && G % 32 == 0))) return ICT_ERR_LAYOUT;
+    cp->out_rows = npix;
+    cp->out_cols = out_c;
+    cp->rows_per_tile = std::min(128 / d->w, d->h);
+    cp->tiles_per_img = (int)cdiv64(d->h, cp->rows_per_tile);
+    cp->a_c = (int)act_c;
+    cp->njobs = 0;
+    // activation operand: aligned along channels unless already uniform; dense NHWC
+    if (uniform_along_cols(a) && a->ld == act_c) {
+        cp->a_mant = a->mant;
+        cp->eA = a->exp;
+        cp->eA_div = clamp_div(a->g_rows, a->rows);
+    } else {
+        int8_t *m = (int8_t *)ws.take((size_t)npix * act_c);
+        int8_t *e = (int8_t *)ws.take((size_t)npix);
+        cp->jobs[cp->njobs++] = AlignJob{a, 1, false, m, act_c, e};
+        cp->a_mant = m;
+        cp->eA = e;
+        cp->eA_div = 1;
+    }
+    // weight operand
+    cp->weight_prep = false;
+    if (dir == ICT_CONV_FWD) {  // contracted (r, s, c) runs along W's rows: align per k
+        if (uniform_along_cols(b)) {
+            cp->b_mant = b->mant;
+            cp->b_ld = b->ld;
+            cp->eB = b->exp;
+            cp->eB_div = clamp_div(b->g_rows, b->rows);
+        } else {
+            int8_t *m = (int8_t *)ws.take((size_t)b->rows * b->cols);
+            int8_t *e = (int8_t *)ws.take((size_t)b->rows);
+            cp->jobs[cp->njobs++] = AlignJob{b, 1, false, m, b->cols, e};
+            cp->b_mant = m;
+            cp->b_ld = b->cols;
+            cp->eB = e;
+            cp->eB_div = 1;
+        }
+    } else {
+        const int64_t ld = round_up(RS * d->k, 16);
+        int8_t *m = (int8_t *)ws.take((size_t)d->c * ld);
+        int8_t *e = (int8_t *)ws.take((size_t)d->c);
+        ConvWeightArgs w;
+        w.w = b->mant;
+        w.w_exp = b->exp;
+        w.ld = b->ld;
+        w.ngc = n_grp_cols(b);
+        w.g_rows = clamp_div(b->g_rows, b->rows);
+        w.g_cols = clamp_div(b->g_cols, b->cols);
+        w.K = d->k;
+        w.RS = (int)RS;
+        w.C = d->c;
+        w.e_star = e;
+        w.out = m;
+        w.out_ld = ld;
+        cp->wprep = w;
+        cp->weight_prep = true;
+        cp->b_mant = m;
+        cp->b_ld = ld;
+        cp->eB = e;
+        cp->eB_div = 1;
+    }
+    cp->n_gcols = (int)n_grp_cols(out);
+    cp->gmax = cp->global_groups ? (int32_t *)ws.take((size_t)cp->n_gcols * 4) : nullptr;
+    return ICT_OK;
+}
+
+int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvPlan &cp, int sms,
+             cudaStream_t s) {
+    int st;
+    for (int i = 0; i < cp.njobs; ++i)
+        if ((st = launch_align(cp.jobs[i], s))) return st;
+    if (cp.weight_prep) {
+        conv_wt_estar_kernel<<<d->c, 256, 0, s>>>(cp.wprep);
+        const int64_t n = (int64_t)d->c * d->r * d->s * d->k;
+        conv_wt_prep_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(cp.wprep);
+        counted(2);
+        if ((st = launch_status())) return st;
+    }
+    CUtensorMap ta, tb;
+    if ((st = tmap_nhwc(&ta, cp.a_mant, d->n, d->h, d->w, cp.a_c, cp.rows_per_tile))) return st;
+    const int64_t ktot = (int64_t)d->r * d->s * cp.a_c;
+    if ((st = tmap_2d(&tb, cp.b_mant, ktot, cp.out_cols, cp.b_ld, 64, cp.bn, CU_TENSOR_MAP_SWIZZLE_64B)))
+        return st;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = (int)cp.out_rows;
+    p.N = (int)cp.out_cols;
+    p.n_kblk = (int)(ktot / 64);
+    p.n_mtiles = d->n * cp.tiles_per_img;
+    p.n_ntiles = (int)cdiv64(cp.out_cols, cp.bn);
+    p.splits = 1;
+    p.kblk_per_split = p.n_kblk;
+    p.num_units = p.n_mtiles * p.n_ntiles;
+    p.eA = cp.eA;
+    p.eA_div = cp.eA_div;
+    p.eB = cp.eB;
+    p.eB_div = cp.eB_div;
+    p.G = (int)std::min<int64_t>(out->g_cols, cp.out_cols);
+    p.out = out->mant;
+    p.out_ld = out->ld;
+    p.out_exp = out->exp;
+    p.out_exp_ld = cp.n_gcols;
+    p.gmax = cp.gmax;
+    p.cv_W = d->w;
+    p.cv_P = d->h;
+    p.cv_rows = cp.rows_per_tile;
+    p.cv_tiles_per_img = cp.tiles_per_img;
+    p.cv_cblk = cp.a_c / 64;
+    p.cv_S = d->s;
+    p.cv_pad = d->pad;
+    p.cv_sign = dir == ICT_CONV_FWD ? 1 : -1;
+    p.stage_tx_bytes = (uint32_t)(64 * d->w * cp.rows_per_tile + 64 * cp.bn);
+    p.wait_ns = g_wait_ns;
+    p.drain_ns = kDrainNs;
+    const int grid = std::min(p.num_units, sms);
+    if (!cp.global_groups) {
+        p.epi = EPI_FIT_ROW;
+        return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s);
+    }
+    fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
+    counted(1);
+    p.epi = EPI_NEED_GLOBAL;
+    if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s))) return st;
+    p.epi = EPI_FIT_GLOBAL;
+    return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s);
+}
+
+// ---- SGD
+
+int fill_sgd_tensor(ict_tensor *W, ict_tensor *V, const ict_tensor *G, SgdTensor *t) {
+    int st;
+    if ((st = check_tensor(W)) || (st = check_tensor(V)) || (st = check_tensor(G))) return st;
+    if (W->rows != V->rows || W->rows != G->rows || W->cols != V->cols || W->cols != G->cols)
+        return ICT_ERR_INVALID_ARG;
+    if (W->g_cols != V->g_cols || W->g_cols != G->g_cols) return ICT_ERR_INVALID_ARG;
+    if ((W->g_rows != 1 || V->g_rows != 1 || G->g_rows != 1) && W->rows > 1) return ICT_ERR_LAYOUT;
+    if (W->ld != V->ld || W->ld != G->ld) return ICT_ERR_LAYOUT;
+    t->w = W->mant;
+    t->w_exp = W->exp;
+    t->v = V->mant;
+    t->v_exp = V->exp;
+    t->g = G->mant;
+    t->g_exp = G->exp;
+    t->rows = W->rows;
+    t->cols = W->cols;
+    t->ld = W->ld;
+    t->G = clamp_div(W->g_cols, W->cols);
+    t->ngc = n_grp_cols(W);
+    return ICT_OK;
+}
+
+int check_sgd_params(const ict_sgd_params *p) {
+    if (!p) return ICT_ERR_INVALID_ARG;
+    if (p->mom_shift < 0 || p->mom_shift > 62 || p->lr_shift < 0 || p->lr_shift > 62) return ICT_ERR_INVALID_ARG;
+    if (p->mom_mul < -65535 || p->mom_mul > 65535 || p->lr_mul < -65535 || p->lr_mul > 65535)
+        return ICT_ERR_INVALID_ARG;
+    return ICT_OK;
+}
+
+int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
+    if (a.total_groups == 0) return ICT_OK;
+    const int64_t blocks = std::min<int64_t>(cdiv64(a.total_groups, 8), (int64_t)sms * 16);
+    sgd_warp_kernel<<<(unsigned)blocks, 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char *ict_status_string(int32_t status) {
+    switch (status) {
+        case ICT_OK: return "ICT_OK";
+        case ICT_ERR_INVALID_ARG: return "ICT_ERR_INVALID_ARG";
+        case ICT_ERR_LAYOUT: return "ICT_ERR_LAYOUT";
+        case ICT_ERR_ALIGNMENT: return "ICT_ERR_ALIGNMENT";
+        case ICT_ERR_WORKSPACE: return "ICT_ERR_WORKSPACE";
+        case ICT_ERR_UNSUPPORTED_ARCH: return "ICT_ERR_UNSUPPORTED_ARCH";
+        case ICT_ERR_CUDA: return "ICT_ERR_CUDA";
+        case ICT_ERR_DEVICE_TIMEOUT: return "ICT_ERR_DEVICE_TIMEOUT";
+        case ICT_ERR_EXP_RANGE: return "ICT_ERR_EXP_RANGE";
+        default: return "ICT_ERR_UNKNOWN";
+    }
+}
+
+const char *ict_version(void) { return "libict 0.1 sm_100a"; }
+
+uint64_t ict_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t ict_get_device_status(int32_t *host_out, void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ICT_ERR_CUDA;
+    int32_t v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return ICT_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return ICT_ERR_CUDA;
+    if (host_out) *host_out = v;
+    if (v & (1 << ICT_ERR_DEVICE_TIMEOUT)) return ICT_ERR_DEVICE_TIMEOUT;
+    if (v & (1 << ICT_ERR_EXP_RANGE)) return ICT_ERR_EXP_RANGE;
+    return ICT_OK;
+}
+
+int32_t ict_set_wait_limit_ns(uint64_t ns) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_wait_ns = ns ? ns : 2000000000ull;
+    return ICT_OK;
+}
+
+int32_t ict_requant(const void *vals, int32_t val_bits, int64_t rows, int64_t cols, int64_t ld_vals,
+                    int32_t base_exp, const int8_t *row_exp, const int8_t *col_exp,
+                    ict_tensor *out, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_tensor(out))) return st;
+    if (val_bits != 32 && val_bits != 64) return ICT_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld_vals < cols || out->rows != rows || out->cols != cols)
+        return ICT_ERR_INVALID_ARG;
+    if (rows && cols && !vals) return ICT_ERR_INVALID_ARG;
+    if (out->g_rows != 1 && rows > 1) return ICT_ERR_LAYOUT;
+    RequantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.v32 = val_bits == 32 ? (const int32_t *)vals : nullptr;
+    a.v64 = val_bits == 64 ? (const int64_t *)vals : nullptr;
+    a.nsplit = 1;
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld_vals;
+    a.base = base_exp;
+    a.row_exp = row_exp;
+    a.row_div = 1;
+    a.col_exp = col_exp;
+    a.col_div = 1;
+    a.out = out->mant;
+    a.out_ld = out->ld;
+    a.out_exp = out->exp;
+    a.G = clamp_div(out->g_cols, cols);
+    a.ngc = n_grp_cols(out);
+    return launch_requant_rows(a, (cudaStream_t)stream);
+}
+
+int32_t ict_align(const ict_tensor *in, int32_t axis, int32_t transpose, int8_t *out_mant,
+                  int64_t ld_out, int8_t *e_star, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_tensor(in))) return st;
+    if ((axis != 0 && axis != 1) || !out_mant || !e_star) return ICT_ERR_INVALID_ARG;
+    if ((st = check_vec(in))) return st;
+    if (!aligned16(out_mant) || (ld_out & 15)) return ICT_ERR_ALIGNMENT;
+    if (ld_out < (transpose ? round_up(in->rows, 16) : in->cols)) return ICT_ERR_INVALID_ARG;
+    return launch_align(AlignJob{in, axis, transpose != 0, out_mant, ld_out, e_star}, (cudaStream_t)stream);
+}
+
+size_t ict_linear_workspace(int32_t op, const ict_tensor *a, const ict_tensor *b,
+                            const ict_tensor *out) {
+    LinearPlan lp;
+    Ws w = make_ws(nullptr, 0, true);
+    if (plan_linear(op, a, b, out, w, &lp) != ICT_OK) return 0;
+    return w.used;
+}
+
+int32_t ict_linear_fwd(const ict_tensor *X, const ict_tensor *W, ict_tensor *Y, void *ws,
+                       size_t ws_bytes, void *stream) {
+    return linear_entry(ICT_OP_LINEAR_FWD, X, W, Y, ws, ws_bytes, stream);
+}
+int32_t ict_linear_bwd_data(const ict_tensor *dY, const ict_tensor *W, ict_tensor *dX, void *ws,
+                            size_t ws_bytes, void *stream) {
+    return linear_entry(ICT_OP_LINEAR_BWD_DATA, dY, W, dX, ws, ws_bytes, stream);
+}
+int32_t ict_linear_bwd_weight(const ict_tensor *dY, const ict_tensor *X, ict_tensor *dW, void *ws,
+                              size_t ws_bytes, void *stream) {
+    return linear_entry(ICT_OP_LINEAR_BWD_WEIGHT, dY, X, dW, ws, ws_bytes, stream);
+}
+
+size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d) {
+    if (!d || d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1 || d->k < 1 || d->r < 1 || d->s < 1)
+        return 0;
+    // worst case: activation aligned copy + its exponents, the prepared weight, gmax
+    const int64_t npix = (int64_t)d->n * d->h * d->w;
+    const int64_t act_c = dir == ICT_CONV_FWD ? d->c : d->k;
+    const int64_t RS = (int64_t)d->r * d->s;
+    Ws w = make_ws(nullptr, 0, true);
+    w.take((size_t)npix * act_c);
+    w.take((size_t)npix);
+    w.take((size_t)std::max<int64_t>(d->k * RS * d->c, d->c * round_up(RS * d->k, 16)));
+    w.take((size_t)std::max(d->k, d->c));
+    w.take((size_t)std::max(d->k, d->c) * 4);
+    return w.used;
+}
+
+int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_tensor *a,
+                               const ict_tensor *b, ict_tensor *out, void *ws, size_t ws_bytes,
+                               void *stream) {
+    int st, sms = 0;
+    if ((st = device_info(&sms))) return st;
+    if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    ConvPlan cp;
+    Ws w = make_ws(ws, ws_bytes, false);
+    if ((st = plan_conv(dir, d, a, b, out, w, &cp))) return st;
+    if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
+    return run_conv(dir, d, out, cp, sms, (cudaStream_t)stream);
+}
+
+int32_t ict_sgd_momentum_step(ict_tensor *W, ict_tensor *V, const ict_tensor *G,
+                              const ict_sgd_params *p, void *stream) {
+    ict_tensor *Ws_[1] = {W}, *Vs_[1] = {V};
+    const ict_tensor *Gs_[1] = {G};
+    return ict_sgd_momentum_step_multi(1, Ws_, Vs_, Gs_, p, stream);
+}
+
+int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W, ict_tensor *const *V,
+                                    const ict_tensor *const *G, const ict_sgd_params *p,
+                                    void *stream) {
+    int st, sms = 0;
+    if ((st = device_info(&sms))) return st;
+    if (n_tensors < 1 || n_tensors > kSgdMaxTensors || !W || !V || !G) return ICT_ERR_INVALID_ARG;
+    if ((st = check_sgd_params(p))) return st;
+    SgdArgs a;  // passed whole as the kernel's parameter block (about 12 KB)
+    memset(&a, 0, sizeof(a));
+    a.n = n_tensors;
+    a.mom_mul = p->mom_mul;
+    a.mom_shift = p->mom_shift;
+    a.lr_mul = p->lr_mul;
+    a.lr_shift = p->lr_shift;
+    int64_t total = 0;
+    for (int i = 0; i < n_tensors; ++i) {
+        if ((st = fill_sgd_tensor(W[i], V[i], G[i], &a.t[i]))) return st;
+        a.t[i].first_group = total;
+        total += a.t[i].rows * a.t[i].ngc;
+    }
+    a.total_groups = total;
+    return run_sgd(a, sms, (cudaStream_t)stream);
+}
+
+int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_tensor(H)) || (st = check_tensor(out))) return st;
+    if (out->rows != H->rows || out->cols != H->cols || out->g_rows != H->g_rows ||
+        out->g_cols != H->g_cols)
+        return ICT_ERR_INVALID_ARG;
+    if ((st = check_vec(H)) || (st = check_vec(out))) return st;
+    if (H->rows == 0 || H->cols == 0) return ICT_OK;
+    GeluArgs a;
+    memset(&a, 0, sizeof(a));
+    a.h = H->mant;
+    a.h_exp = H->exp;
+    a.out = out->mant;
+    a.rows = H->rows;
+    a.cols = H->cols;
+    a.ld_h = H->ld;
+    a.ld_out = out->ld;
+    a.g_rows = clamp_div(H->g_rows, H->rows);
+    a.g_cols = clamp_div(H->g_cols, H->cols);
+    a.ngc = n_grp_cols(H);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t ne = (size_t)(n_grp_rows(H) * n_grp_cols(H));
+    if (cudaMemcpyAsync(out->exp, H->exp, ne, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return ICT_ERR_CUDA;
+    const int64_t vecs = H->rows * (H->cols / 16);
+    gelu_fwd_kernel<<<(unsigned)cdiv64(vecs, 256), 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_tensor(H)) || (st = check_tensor(dG)) || (st = check_tensor(dH))) return st;
+    if (dG->rows != H->rows || dG->cols != H->cols || dH->rows != H->rows || dH->cols != H->cols)
+        return ICT_ERR_INVALID_ARG;
+    if ((H->g_rows != 1 || dG->g_rows != 1 || dH->g_rows != 1) && H->rows > 1) return ICT_ERR_LAYOUT;
+    if (H->g_cols != dG->g_cols || H->g_cols != dH->g_cols) return ICT_ERR_LAYOUT;
+    if (H->rows == 0 || H->cols == 0) return ICT_OK;
+    GeluArgs a;
+    memset(&a, 0, sizeof(a));
+    a.h = H->mant;
+    a.h_exp = H->exp;
+    a.dg = dG->mant;
+    a.dg_exp = dG->exp;
+    a.out = dH->mant;
+    a.out_exp = dH->exp;
+    a.rows = H->rows;
+    a.cols = H->cols;
+    a.ld_h = H->ld;
+    a.ld_dg = dG->ld;
+    a.ld_out = dH->ld;
+    a.g_rows = 1;
+    a.g_cols = clamp_div(H->g_cols, H->cols);
+    a.ngc = n_grp_cols(H);
+    const int64_t groups = H->rows * a.ngc;
+    gelu_bwd_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, (cudaStream_t)stream>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+}  // extern "C"

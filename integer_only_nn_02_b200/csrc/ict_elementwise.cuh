@@ -1,0 +1,405 @@
+// ict_elementwise.cuh -- memory-bound kernels of the (C,e) training path:
+//   requant (FIT of integer values into row-local groups),
+//   ALIGN_MAX of an operand along its contracted index (optionally transposed),
+//   the integer GELU stand-in (forward and backward),
+//   the integer SGD-with-momentum update with per-group velocity.
+// Source: "Memory-Efficient Integer-Only Training of Deep Neural Networks",
+// Abstract (five integer building blocks), Figure 1b (integer SGD with momentum and
+// per-group velocity), Table 6 (Product / Sum), Table 7 (pointwise activations keep
+// the exponent).
+#pragma once
+
+#include "ict_device.cuh"
+
+namespace ict {
+
+// ------------------------------------------------------------------ two-term sums
+
+// a * 2^pa + b * 2^pb as one integer x at exponent r (the Sum primitive, Table 6).
+// Exact while the exponents are at most 32 apart (|a|, |b| < 2^16, so x < 2^48).
+// Beyond that the smaller term becomes a one-unit sticky below the larger one; the
+// requantised result is unchanged because the group exponent is at least pa - 7 and
+// both the true small term (< 2^(pa-16)) and the sticky (2^(pa-32)) sit strictly
+// inside the same gap between consecutive multiples of 2^(pa-8) next to a * 2^pa.
+struct TwoTerm {
+    int64_t x;
+    int r;
+};
+__device__ __forceinline__ TwoTerm two_term(int64_t a, int pa, int64_t b, int pb) {
+    if (a == 0) return TwoTerm{b, pb};
+    if (b == 0) return TwoTerm{a, pa};
+    if (pa < pb) {
+        int64_t t = a; a = b; b = t;
+        int tp = pa; pa = pb; pb = tp;
+    }
+    const int d = pa - pb;
+    if (d <= 32) return TwoTerm{a * (1ll << d) + b, pb};
+    return TwoTerm{a * (1ll << 32) + (b > 0 ? 1 : -1), pa - 32};
+}
+__device__ __forceinline__ int need64(int64_t x, int r) {
+    return x == 0 ? kNoExp : r + need_off64((uint64_t)(x < 0 ? -x : x));
+}
+
+// ------------------------------------------------------------------ requant (FIT)
+
+// FIT of int32 (optionally the int64 sum of `nsplit` int32 slices) or int64 values
+// into row-local groups (1, G).  One warp per group; element (i, j) has exponent
+// base + row_exp[i] + col_exp[j].
+struct RequantArgs {
+    const int32_t *v32;
+    const int64_t *v64;
+    int nsplit;
+    int64_t split_stride;
+    int64_t rows, cols, ld;
+    int32_t base;
+    const int8_t *row_exp;  // exponent of row i: row_exp[i / row_div] (NULL = 0)
+    int row_div;
+    const int8_t *col_exp;  // exponent of column j: col_exp[j / col_div] (NULL = 0)
+    int col_div;
+    int8_t *out;
+    int64_t out_ld;
+    int8_t *out_exp;
+    int G;
+    int64_t ngc;  // groups per row
+};
+
+__device__ __forceinline__ int64_t rq_value(const RequantArgs &a, int64_t i, int64_t j) {
+    if (a.v64) return a.v64[i * a.ld + j];
+    int64_t s = 0;
+    for (int k = 0; k < a.nsplit; ++k) s += a.v32[k * a.split_stride + i * a.ld + j];
+    return s;
+}
+
+__global__ void __launch_bounds__(256) requant_rows_kernel(RequantArgs a) {
+    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (gw >= a.rows * a.ngc) return;
+    const int64_t i = gw / a.ngc, g = gw % a.ngc;
+    const int64_t j0 = g * a.G, j1 = min(a.cols, j0 + a.G);
+    const int re = a.base + (a.row_exp ? a.row_exp[i / a.row_div] : 0);
+    int emax = kNoExp;
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const int64_t x = rq_value(a, i, j);
+        if (x) emax = max(emax, need64(x, re + (a.col_exp ? a.col_exp[j / a.col_div] : 0)));
+    }
+    const int e = finalize_exp(warp_max(emax));
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const int64_t x = rq_value(a, i, j);
+        a.out[i * a.out_ld + j] = (int8_t)requant64(x, re + (a.col_exp ? a.col_exp[j / a.col_div] : 0), e);
+    }
+    if (lane == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+}
+
+// ------------------------------------------------------------------ ALIGN_MAX
+
+struct AlignArgs {
+    const int8_t *in;
+    const int8_t *in_exp;
+    int64_t rows, cols, ld;
+    int g_rows, g_cols;
+    int64_t ngc;
+    int axis;  // 1: per-row e*, 0: per-column e*
+    int8_t *out;
+    int64_t out_ld;
+    int8_t *e_star;  // [rows] (axis 1) or [cols] (axis 0)
+};
+
+// e* per row: max over the row's group exponents, E_ZERO groups ignored.
+__global__ void estar_rows_kernel(AlignArgs a) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.rows) return;
+    const int8_t *e = a.in_exp + (i / a.g_rows) * a.ngc;
+    int m = kNoExp;
+    for (int64_t g = 0; g < a.ngc; ++g)
+        if (e[g] != kEZero) m = max(m, (int)e[g]);
+    a.e_star[i] = (int8_t)(m <= kNoExp ? kEZero : m);
+}
+
+// e* per column: one block per group column, max over all group rows.
+__global__ void __launch_bounds__(256) estar_cols_kernel(AlignArgs a) {
+    const int64_t gj = blockIdx.x;
+    const int64_t ngr = (a.rows + a.g_rows - 1) / a.g_rows;
+    int m = kNoExp;
+    for (int64_t gi = threadIdx.x; gi < ngr; gi += blockDim.x) {
+        const int e = a.in_exp[gi * a.ngc + gj];
+        if (e != kEZero) m = max(m, e);
+    }
+    m = warp_max(m);
+    __shared__ int red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int v = threadIdx.x < 8 ? red[threadIdx.x] : kNoExp;
+        v = warp_max(v);
+        const int8_t es = (int8_t)(v <= kNoExp ? kEZero : v);
+        const int64_t j1 = min(a.cols, (gj + 1) * a.g_cols);
+        for (int64_t j = gj * a.g_cols + threadIdx.x; j < j1; j += 32) a.e_star[j] = es;
+    }
+}
+
+// Aligned mantissas, 64 x 64 tiles of 16-byte vectors (cols and, when transposed,
+// rows are multiples of 16; g_cols is a multiple of 16 or spans all columns).
+template <bool TRANSPOSE>
+__global__ void __launch_bounds__(256) align_tile_kernel(AlignArgs a) {
+    __shared__ uint8_t tile[64][64 + 4];
+    const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+    const int tr = threadIdx.x >> 2, tc = (threadIdx.x & 3) * 16;
+    const int64_t i = r0 + tr, j = c0 + tc;
+    uint32_t w[4] = {0, 0, 0, 0};
+    if (i < a.rows && j < a.cols) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
+        const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
+        const int eg = a.in_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            const int es = a.axis == 1 ? a.e_star[i] : a.e_star[j + b];
+            const int c = sx8(src[b >> 2], b & 3);
+            int q = 0;
+            if (eg != kEZero && c != 0) q = es == eg ? c : rne_shr32(c, es - eg);
+            w[b >> 2] |= (uint32_t)(q & 0xff) << (8 * (b & 3));
+        }
+    }
+    if constexpr (!TRANSPOSE) {
+        if (i < a.rows && j < a.cols)
+            *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+#pragma unroll
+        for (int b = 0; b < 16; ++b) tile[tc + b][tr] = (uint8_t)(w[b >> 2] >> (8 * (b & 3)));
+        __syncthreads();
+        // output row = input column c0 + tr, output columns = input rows r0 + tc .. + 15
+        const int64_t oi = c0 + tr, oj = r0 + tc;
+        if (oi < a.cols && oj < a.rows) {
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o[q] = (uint32_t)tile[tr][tc + 4 * q] | ((uint32_t)tile[tr][tc + 4 * q + 1] << 8) |
+                       ((uint32_t)tile[tr][tc + 4 * q + 2] << 16) |
+                       ((uint32_t)tile[tr][tc + 4 * q + 3] << 24);
+            *reinterpret_cast<uint4 *>(a.out + oi * a.out_ld + oj) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ integer GELU
+
+struct GeluArgs {
+    const int8_t *h;
+    const int8_t *h_exp;
+    const int8_t *dg;
+    const int8_t *dg_exp;
+    int8_t *out;
+    int8_t *out_exp;
+    int64_t rows, cols, ld_h, ld_dg, ld_out;
+    int g_rows, g_cols;
+    int64_t ngc;
+};
+
+// h(x) = x * clip((x + 2) / 4, 0, 1) on one mantissa C at exponent e, result at e.
+__device__ __forceinline__ int gelu_fwd_elem(int c, int e) {
+    if (c == 0 || e == kEZero) return 0;
+    if (e >= 2) return c > 0 ? c : 0;
+    const int s = 2 - e;  // >= 1; T = 2^(1 - e) = 2^(s - 1)
+    if (s - 1 <= 7) {
+        const int t = 1 << (s - 1);
+        if (c <= -t) return 0;
+        if (c >= t) return c;
+    }
+    // interior: x (x + 2) / 4 at exponent e = RNE((C^2 + C * 2^(s-1)) / 2^s)
+    if (s <= 24) return rne_shr32(c * c + c * (1 << (s - 1)), s);
+    // C^2 / 2^s < 1/2: RNE(C / 2 + positive tiny) = floor((C + 1) / 2)
+    return (c + 1) >> 1;
+}
+
+__global__ void __launch_bounds__(256) gelu_fwd_kernel(GeluArgs a) {
+    const int64_t vecs_per_row = a.cols / 16;
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= a.rows * vecs_per_row) return;
+    const int64_t i = v / vecs_per_row, j = (v % vecs_per_row) * 16;
+    const int e = a.h_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+    const uint4 raw = *reinterpret_cast<const uint4 *>(a.h + i * a.ld_h + j);
+    const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        o[q] = pack4(gelu_fwd_elem(sx8(src[q], 0), e), gelu_fwd_elem(sx8(src[q], 1), e),
+                     gelu_fwd_elem(sx8(src[q], 2), e), gelu_fwd_elem(sx8(src[q], 3), e));
+    *reinterpret_cast<uint4 *>(a.out + i * a.ld_out + j) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// dG * h'(x): h' = 0 for x <= -2, 1 for x >= 2, (x + 1) / 2 between; as a two-term
+// value dG * C_h * 2^(e_d + e_h - 1) + dG * 2^(e_d - 1).
+__device__ __forceinline__ TwoTerm gelu_bwd_elem(int ch, int eh, int cd, int ed) {
+    if (cd == 0) return TwoTerm{0, 0};
+    if (eh == kEZero) ch = 0;
+    if (ch != 0) {
+        if (eh >= 1) return ch > 0 ? TwoTerm{cd, ed} : TwoTerm{0, 0};  // |x| >= 2
+        if (1 - eh <= 7) {
+            const int t = 1 << (1 - eh);
+            if (ch <= -t) return TwoTerm{0, 0};
+            if (ch >= t) return TwoTerm{cd, ed};
+        }
+    }
+    return two_term((int64_t)cd * ch, ed + eh - 1, cd, ed - 1);
+}
+
+__global__ void __launch_bounds__(256) gelu_bwd_kernel(GeluArgs a) {
+    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (gw >= a.rows * a.ngc) return;
+    const int64_t i = gw / a.ngc, g = gw % a.ngc;
+    const int64_t j0 = g * a.g_cols, j1 = min(a.cols, j0 + a.g_cols);
+    const int eh = a.h_exp[i * a.ngc + g], ed = a.dg_exp[i * a.ngc + g];
+    int emax = kNoExp;
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const TwoTerm t = gelu_bwd_elem(a.h[i * a.ld_h + j], eh, a.dg[i * a.ld_dg + j], ed);
+        if (t.x) emax = max(emax, need64(t.x, t.r));
+    }
+    const int e = finalize_exp(warp_max(emax));
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const TwoTerm t = gelu_bwd_elem(a.h[i * a.ld_h + j], eh, a.dg[i * a.ld_dg + j], ed);
+        a.out[i * a.ld_out + j] = (int8_t)requant64(t.x, t.r, e);
+    }
+    if (lane == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+}
+
+// ------------------------------------------------------------------ integer SGD
+
+struct SgdTensor {
+    int8_t *w, *w_exp, *v, *v_exp;
+    const int8_t *g, *g_exp;
+    int64_t rows, cols, ld;
+    int G;
+    int64_t ngc;
+    int64_t first_group;  // prefix sum of group counts over the tensor list
+};
+
+constexpr int kSgdMaxTensors = 128;
+
+struct SgdArgs {
+    int n;
+    int64_t total_groups;
+    int mom_mul, mom_shift, lr_mul, lr_shift;
+    SgdTensor t[kSgdMaxTensors];
+};
+
+// One warp per group: v <- FIT(mom * v + g), w <- FIT(w - lr * v).
+__device__ __forceinline__ void sgd_group(const SgdArgs &p, const SgdTensor &t, int64_t local,
+                                          int lane) {
+    const int64_t i = local / t.ngc, g = local % t.ngc;
+    const int64_t ge = i * t.ngc + g;
+    const int64_t j0 = g * t.G, j1 = min(t.cols, j0 + t.G);
+    const int ev = t.v_exp[ge], eg = t.g_exp[ge], ew = t.w_exp[ge];
+    const int pv = ev - p.mom_shift;
+    // velocity
+    int emax = kNoExp;
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const TwoTerm s = two_term((int64_t)p.mom_mul * t.v[i * t.ld + j], pv, t.g[i * t.ld + j], eg);
+        if (s.x) emax = max(emax, need64(s.x, s.r));
+    }
+    const int ev2 = finalize_exp(warp_max(emax));
+    // weight (recompute the new velocity mantissas element by element)
+    const int pu = ev2 - p.lr_shift;
+    emax = kNoExp;
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const TwoTerm s = two_term((int64_t)p.mom_mul * t.v[i * t.ld + j], pv, t.g[i * t.ld + j], eg);
+        const int cv = requant64(s.x, s.r, ev2);
+        const TwoTerm w = two_term(t.w[i * t.ld + j], ew, -(int64_t)p.lr_mul * cv, pu);
+        if (w.x) emax = max(emax, need64(w.x, w.r));
+    }
+    const int ew2 = finalize_exp(warp_max(emax));
+    __syncwarp();
+    for (int64_t j = j0 + lane; j < j1; j += 32) {
+        const TwoTerm s = two_term((int64_t)p.mom_mul * t.v[i * t.ld + j], pv, t.g[i * t.ld + j], eg);
+        const int cv = requant64(s.x, s.r, ev2);
+        const TwoTerm w = two_term(t.w[i * t.ld + j], ew, -(int64_t)p.lr_mul * cv, pu);
+        const int cw = requant64(w.x, w.r, ew2);
+        t.v[i * t.ld + j] = (int8_t)cv;  // each lane rewrites only the elements it read
+        t.w[i * t.ld + j] = (int8_t)cw;
+    }
+    if (lane == 0) {
+        t.v_exp[ge] = (int8_t)ev2;
+        t.w_exp[ge] = (int8_t)ew2;
+    }
+}
+
+__global__ void __launch_bounds__(256) sgd_warp_kernel(const __grid_constant__ SgdArgs p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * 8;
+    for (int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); gw < p.total_groups; gw += warps) {
+        int lo = 0, hi = p.n - 1;  // tensor holding global group gw
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.t[mid].first_group <= gw) lo = mid;
+            else hi = mid - 1;
+        }
+        sgd_group(p, p.t[lo], gw - p.t[lo].first_group, lane);
+    }
+}
+
+}  // namespace ict
+
+namespace ict {
+
+// ------------------------------------------------------------------ conv weight prep
+
+// Backward-data of a convolution contracts over (k, r, s) for each input channel c, so
+// the KRSC weight is aligned per c (max over k, r, s of its group exponents) and laid
+// out K-major as W'[c][(r*S + s)*K + k].
+struct ConvWeightArgs {
+    const int8_t *w;
+    const int8_t *w_exp;
+    int64_t ld, ngc;
+    int g_rows, g_cols;
+    int K, RS, C;
+    int8_t *e_star;  // [C]
+    int8_t *out;     // [C][out_ld]
+    int64_t out_ld;
+};
+
+__global__ void __launch_bounds__(256) conv_wt_estar_kernel(ConvWeightArgs a) {
+    const int c = blockIdx.x;
+    int m = kNoExp;
+    for (int idx = threadIdx.x; idx < a.K * a.RS; idx += blockDim.x) {
+        const int k = idx / a.RS, rs = idx % a.RS;
+        const int e = a.w_exp[(k / a.g_rows) * a.ngc + (rs * a.C + c) / a.g_cols];
+        if (e != kEZero) m = max(m, e);
+    }
+    m = warp_max(m);
+    __shared__ int red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int v = red[0];
+        for (int i = 1; i < 8; ++i) v = max(v, red[i]);
+        a.e_star[c] = (int8_t)(v <= kNoExp ? kEZero : v);
+    }
+}
+
+__global__ void __launch_bounds__(256) conv_wt_prep_kernel(ConvWeightArgs a) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_c = (int64_t)a.RS * a.K;
+    if (idx >= per_c * a.C) return;
+    const int c = (int)(idx / per_c), rem = (int)(idx % per_c);
+    const int rs = rem / a.K, k = rem % a.K;
+    const int e = a.w_exp[(k / a.g_rows) * a.ngc + (rs * a.C + c) / a.g_cols];
+    const int v = a.w[k * a.ld + rs * a.C + c];
+    const int es = a.e_star[c];
+    int q = 0;
+    if (e != kEZero && v != 0) q = es == e ? v : rne_shr32(v, es - e);
+    a.out[c * a.out_ld + rem] = (int8_t)q;
+}
+
+__global__ void fill_i32_kernel(int32_t *p, int n, int32_t v) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) p[i] = v;
+}
+
+// zero result of an empty contraction: mantissas 0, every group E_ZERO
+__global__ void zero_ce_kernel(int8_t *mant, int64_t rows, int64_t cols, int64_t ld, int8_t *exp,
+                               int64_t n_exp) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < rows * cols) mant[(i / cols) * ld + i % cols] = 0;
+    if (i < n_exp) exp[i] = (int8_t)kEZero;
+}
+
+}  // namespace ict

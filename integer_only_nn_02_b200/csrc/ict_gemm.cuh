@@ -1,0 +1,325 @@
+// ict_gemm.cuh -- the (C,e) Product on the 5th-generation tensor cores.
+//
+//   D[m][n] = sum_k A[m][k] * B[n][k]     (int8 x int8 -> int32 in TMEM)
+//   exponent(m, n) = eA[m] + eB[n]        (exponent addition of the Product)
+//   then FIT into the caller's output groups, fused into the epilogue.
+//
+// Source: "Memory-Efficient Integer-Only Training of Deep Neural Networks", Table 6
+// (convolution, linear and patch embedding are instances of the Product primitive)
+// and Figure 1a (forward and backward of every layer in integer arithmetic).
+//
+// Structure (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: A and B K-major tiles into a STAGES-deep ring of
+//               swizzled shared-memory buffers (mbarrier full/empty pairs)
+//   warp 1      MMA issuer: one thread issues tcgen05.mma kind::i8 (M = 128) into a
+//               double-buffered TMEM accumulator; tcgen05.commit frees smem stages
+//   warp 2      TMEM allocation / release
+//   warps 4..7  epilogue: tcgen05.ld (thread = output row), group max of need(),
+//               RNE shift, int8 stores of mantissas and group exponents
+// Every wait is bounded; on expiry the CTA raises ICT_ERR_DEVICE_TIMEOUT, drains its
+// in-flight copies and MMAs (again with a bound), frees TMEM and exits.
+#pragma once
+
+#include "ict_device.cuh"
+
+namespace ict {
+
+enum EpiMode : int {
+    EPI_FIT_ROW = 0,      // row-local groups (1, G) inside one tile -> int8 + exps
+    EPI_I32 = 1,          // raw int32 partials to a workspace slice (split-K / wide groups)
+    EPI_NEED_GLOBAL = 2,  // pass 1 of groups spanning all rows: max need per column group
+    EPI_FIT_GLOBAL = 3,   // pass 2: requantise with the global group exponents
+};
+enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1 };
+
+struct GemmParams {
+    int M, N;       // output rows (MMA M side) and columns (MMA N side)
+    int n_kblk;     // number of BK-wide K blocks
+    int n_mtiles, n_ntiles, splits, kblk_per_split, num_units;
+    const int8_t *eA;
+    int eA_div;     // exponent of output row m: eA[m / eA_div]
+    const int8_t *eB;
+    int eB_div;     // exponent of output column n: eB[n / eB_div]
+    int G;          // output group width along N
+    int8_t *out;
+    int64_t out_ld;
+    int8_t *out_exp;
+    int64_t out_exp_ld;
+    int32_t *ws32;
+    int64_t ws_ld, ws_split_stride;
+    int32_t *gmax;  // [column groups] running max of need() (global groups)
+    // implicit-GEMM convolution: output tile = cv_rows image rows of width cv_W
+    int cv_W, cv_P, cv_rows, cv_tiles_per_img, cv_cblk, cv_S, cv_pad, cv_sign;
+    uint32_t stage_tx_bytes;
+    uint64_t wait_ns, drain_ns;
+    int epi;
+};
+
+template <int BN, int BK, int STAGES>
+struct GemmSmem {
+    static constexpr int kABytes = 128 * BK;
+    static constexpr int kBBytes = BN * BK;
+    static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+    static constexpr int kOffB = STAGES * kABytes;
+    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 5 mbarriers
+    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 5) * 8;
+    static constexpr int kOffEB = kOffMisc + 16;
+    static constexpr int kBytes = kOffEB + 4 * BN + 1024;  // + alignment slack
+};
+
+template <int BN, int BK, int STAGES, int LOAD>
+__global__ void __launch_bounds__(256, 1)
+    gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ GemmParams p) {
+    using L = GemmSmem<BN, BK, STAGES>;
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    static_assert(BK == 128 || BK == 64, "BK");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + L::kOffBar;           // [STAGES]
+    const uint32_t bar_empty = bar_full + 8 * STAGES;       // [STAGES]
+    const uint32_t bar_tfull = bar_empty + 8 * STAGES;      // [2]
+    const uint32_t bar_tempty = bar_tfull + 16;             // [2]
+    const uint32_t bar_drain = bar_tempty + 16;             // [1]
+    volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
+    int *sEB = (int *)(smem + L::kOffEB);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar_tfull + 8 * a, 1);
+            mbar_init(bar_tempty + 8 * a, 128);
+        }
+        mbar_init(bar_drain, 1);
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32((const void *)&misc[0]), L::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = (uint32_t)misc[0];
+    volatile int *abort_flag = &misc[1];
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        raise_status(ICT_ERR_DEVICE_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[STAGES];
+            uint32_t issued_phase[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = 0, issued_phase[s] = 0;
+            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+                const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
+                const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
+                const int kb0 = split * p.kblk_per_split;
+                const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
+                int img = 0, h0 = 0;
+                if (LOAD == LOAD_CONV) {
+                    img = mt / p.cv_tiles_per_img;
+                    h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
+                }
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, p.wait_ns, abort_flag)) {
+                        fail();
+                        break;
+                    }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    mbar_expect_tx(fb, p.stage_tx_bytes);
+                    const uint32_t sa = sbase + stage * L::kABytes;
+                    const uint32_t sb = sbase + L::kOffB + stage * L::kBBytes;
+                    if (LOAD == LOAD_2D) {
+                        tma_load_2d(sa, &tmA, fb, kb * BK, mt * 128);
+                    } else {
+                        const int tap = kb / p.cv_cblk, cb = kb % p.cv_cblk;
+                        const int r = tap / p.cv_S, s = tap % p.cv_S;
+                        tma_load_4d(sa, &tmA, fb, cb * 64, p.cv_sign * (s - p.cv_pad),
+                                    h0 + p.cv_sign * (r - p.cv_pad), img);
+                    }
+                    tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
+                    issued[stage] = 1;
+                    issued_phase[stage] = phase;
+                    if (++stage == STAGES) stage = 0, phase ^= 1;
+                }
+            }
+            // drain: every issued copy must land before the CTA may exit
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s]) mbar_wait(bar_full + 8 * s, issued_phase[s], p.drain_ns, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = idesc_i8(128, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool any = false;
+            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x, ++it) {
+                const int split = u / (p.n_mtiles * p.n_ntiles);
+                const int kb0 = split * p.kblk_per_split;
+                const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
+                const int acc = it & 1;
+                if (!mbar_wait(bar_tempty + 8 * acc, ((it >> 1) & 1) ^ 1, p.wait_ns, abort_flag)) {
+                    fail();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tmem_d = tmem_base + acc * BN;
+                bool ok = true;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, p.wait_ns, abort_flag)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = smem_desc_kmajor(sbase + stage * L::kABytes, BK);
+                    const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + stage * L::kBBytes, BK);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                    any = true;
+                    umma_commit(bar_empty + 8 * stage);
+                    if (++stage == STAGES) stage = 0, phase ^= 1;
+                }
+                if (!ok) break;
+                umma_commit(bar_tfull + 8 * acc);
+            }
+            if (any) {  // drain: all issued MMAs complete before TMEM is released
+                umma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, p.drain_ns, nullptr);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 128;  // output row within the tile = TMEM lane
+        const int quarter = warp & 3;
+        int it = 0;
+        // The loop never tests the abort flag on its own: the 128 threads decide together
+        // through a barrier reduction, so none of them can be left waiting at a barrier.
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++it) {
+            const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
+            const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
+            const int acc = it & 1;
+            int64_t row_base;
+            int valid_rows;
+            if (LOAD == LOAD_CONV) {
+                const int img = mt / p.cv_tiles_per_img;
+                const int h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
+                row_base = ((int64_t)img * p.cv_P + h0) * p.cv_W;
+                valid_rows = min(p.cv_rows, p.cv_P - h0) * p.cv_W;
+            } else {
+                row_base = (int64_t)mt * 128;
+                valid_rows = min(128, p.M - mt * 128);
+            }
+            const int n0 = nt * BN;
+            for (int j = et; j < BN; j += 128) {
+                const int n = n0 + j;
+                sEB[j] = n < p.N ? (int)p.eB[n / p.eB_div] : 0;
+            }
+            const bool ok = mbar_wait(bar_tfull + 8 * acc, (it >> 1) & 1, p.wait_ns, abort_flag);
+            if (!ok) fail();
+            if (named_bar_or(1, 128, !ok || *abort_flag)) break;
+            tc_fence_after();
+
+            const bool valid = et < valid_rows;
+            const int64_t grow = row_base + et;
+            const int ea = valid ? (int)p.eA[grow / p.eA_div] : 0;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+            uint32_t v[32];
+
+            if (p.epi == EPI_I32) {
+                int32_t *dst = p.ws32 + split * p.ws_split_stride + grow * p.ws_ld + n0;
+                for (int c = 0; c < BN; c += 32) {
+                    tmem_ld32(taddr + c, v);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            if (n0 + c + 4 * q < p.N)
+                                *reinterpret_cast<uint4 *>(dst + c + 4 * q) =
+                                    make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                }
+            } else {
+                // groups wider than the output (whole rows) are one tile-wide group; the
+                // host guarantees G % 32 == 0 and BN % G == 0 otherwise
+                const int G = p.G >= p.N ? BN : p.G;
+                for (int g0 = 0; g0 < BN; g0 += G) {
+                    int emax = kNoExp;
+                    for (int c = g0; c < g0 + G; c += 32) {
+                        tmem_ld32(taddr + c, v);
+                        tmem_ld_wait();
+                        if (valid) {
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) {
+                                const int32_t x = (int32_t)v[q];
+                                if (x) emax = max(emax, ea + sEB[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
+                            }
+                        }
+                    }
+                    const int gcol = (n0 + g0) / p.G;
+                    if (p.epi == EPI_NEED_GLOBAL) {
+                        const int m = warp_max(emax);
+                        if (lane == 0 && m > kNoExp && n0 + g0 < p.N) atomicMax(p.gmax + gcol, m);
+                        continue;
+                    }
+                    const int e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : emax);
+                    for (int c = g0; c < g0 + G; c += 32) {
+                        if (G > 32) {
+                            tmem_ld32(taddr + c, v);
+                            tmem_ld_wait();
+                        }
+                        if (valid) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                w[q] = pack4(requant32((int32_t)v[4 * q], ea + sEB[c + 4 * q], e),
+                                             requant32((int32_t)v[4 * q + 1], ea + sEB[c + 4 * q + 1], e),
+                                             requant32((int32_t)v[4 * q + 2], ea + sEB[c + 4 * q + 2], e),
+                                             requant32((int32_t)v[4 * q + 3], ea + sEB[c + 4 * q + 3], e));
+                            int8_t *dst = p.out + grow * p.out_ld + n0 + c;
+                            if (n0 + c < p.N)
+                                *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                            if (n0 + c + 16 < p.N)
+                                *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                        }
+                    }
+                    if (n0 + g0 < p.N) {
+                        if (p.epi == EPI_FIT_ROW && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
+                        if (p.epi == EPI_FIT_GLOBAL && et == 0) p.out_exp[gcol] = (int8_t)e;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_tempty + 8 * acc);
+            named_bar_sync(1, 128);  // sEB is rewritten for the next tile
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tmem_base, L::kTmemCols);
+}
+
+}  // namespace ict

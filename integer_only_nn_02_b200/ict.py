@@ -1,0 +1,315 @@
+"""Thin Python binding of libict.so (argument marshalling only).
+
+Every entry point of ``include/ict.h`` is exposed under the same name and takes the
+same arguments, with :class:`DevCE` (a (C,e) tensor on the GPU: torch int8 mantissas
+plus an int8 exponent grid) in place of ``ict_tensor``.  PyTorch supplies device memory
+and streams; all arithmetic runs in the library's kernels.  Importing this module
+loads ``libict.so`` and raises if it has not been built; there is no other code path.
+
+Convenience wrappers (``linear_fwd`` ...) allocate outputs and workspace with torch
+and then make exactly one library call.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+from .workloads import CE, cdiv
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libict.so")
+
+ICT_OK = 0
+STATUS_NAMES = {
+    0: "ICT_OK", 1: "ICT_ERR_INVALID_ARG", 2: "ICT_ERR_LAYOUT", 3: "ICT_ERR_ALIGNMENT",
+    4: "ICT_ERR_WORKSPACE", 5: "ICT_ERR_UNSUPPORTED_ARCH", 6: "ICT_ERR_CUDA",
+    7: "ICT_ERR_DEVICE_TIMEOUT", 8: "ICT_ERR_EXP_RANGE",
+}
+OP_LINEAR_FWD, OP_LINEAR_BWD_DATA, OP_LINEAR_BWD_WEIGHT = 0, 1, 2
+CONV_FWD, CONV_BWD_DATA, CONV_BWD_WEIGHT = 0, 1, 2
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libict.so not found at {LIB_PATH}: build it with "
+        "`python -m integer_only_nn_02_b200.csrc.build` (nvcc, sm_100a)")
+lib = ctypes.CDLL(LIB_PATH)
+
+
+class ict_tensor(ctypes.Structure):
+    _fields_ = [("mant", ctypes.c_void_p), ("exp", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("ld", ctypes.c_int64), ("g_rows", ctypes.c_int32),
+                ("g_cols", ctypes.c_int32)]
+
+
+class ict_sgd_params(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("mom_mul", "mom_shift", "lr_mul", "lr_shift")]
+
+
+class ict_conv_desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")]
+
+
+_P = ctypes.POINTER
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "ict_status_string": ([_i32], ctypes.c_char_p),
+    "ict_version": ([], ctypes.c_char_p),
+    "ict_get_device_status": ([_P(_i32), _vp], _i32),
+    "ict_set_wait_limit_ns": ([ctypes.c_uint64], _i32),
+    "ict_launch_count": ([], ctypes.c_uint64),
+    "ict_requant": ([_vp, _i32, _i64, _i64, _i64, _i32, _vp, _vp, _P(ict_tensor), _vp], _i32),
+    "ict_align": ([_P(ict_tensor), _i32, _i32, _vp, _i64, _vp, _vp], _i32),
+    "ict_linear_workspace": ([_i32, _P(ict_tensor), _P(ict_tensor), _P(ict_tensor)], _sz),
+    "ict_linear_fwd": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_linear_bwd_data": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_linear_bwd_weight": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_conv_workspace": ([_i32, _P(ict_conv_desc)], _sz),
+    "ict_conv_implicit_gemm": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_sgd_momentum_step": ([_P(ict_tensor), _P(ict_tensor), _P(ict_tensor), _P(ict_sgd_params), _vp], _i32),
+    "ict_sgd_momentum_step_multi": ([_i32, _P(_P(ict_tensor)), _P(_P(ict_tensor)), _P(_P(ict_tensor)),
+                                     _P(ict_sgd_params), _vp], _i32),
+    "ict_gelu_fwd": ([_P(ict_tensor), _P(ict_tensor), _vp], _i32),
+    "ict_gelu_bwd": ([_P(ict_tensor)] * 3 + [_vp], _i32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class IctError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+def _check(code: int, what: str) -> None:
+    if code != ICT_OK:
+        raise IctError(code, what)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+class DevCE:
+    """A (C,e) tensor on the GPU: int8 mantissas [rows, ld] (first ``cols`` used) and an
+    int8 exponent grid [cdiv(rows, g_rows), cdiv(cols, g_cols)]."""
+
+    def __init__(self, mant: torch.Tensor, exp: torch.Tensor, g_rows: int, g_cols: int, cols=None):
+        assert mant.dtype == torch.int8 and exp.dtype == torch.int8 and mant.is_cuda
+        self.mant, self.exp = mant, exp
+        self.rows = int(mant.shape[0])
+        self.cols = int(cols if cols is not None else mant.shape[1])
+        self.ld = int(mant.stride(0)) if mant.dim() == 2 and self.rows > 1 else int(mant.shape[1])
+        self.g_rows, self.g_cols = int(g_rows), int(g_cols)
+
+    @staticmethod
+    def empty(rows, cols, g_rows, g_cols, device="cuda"):
+        g_rows = max(1, min(g_rows, rows)) if rows else max(1, g_rows)
+        g_cols = max(1, min(g_cols, cols)) if cols else max(1, g_cols)
+        ld = -(-cols // 16) * 16 if cols else 16
+        mant = torch.empty((rows, ld), dtype=torch.int8, device=device)
+        exp = torch.empty((cdiv(rows, g_rows), cdiv(cols, g_cols)), dtype=torch.int8, device=device)
+        return DevCE(mant, exp, g_rows, g_cols, cols=cols)
+
+    @staticmethod
+    def from_host(t: CE, device="cuda", pin=False):
+        rows, cols = t.rows, t.cols
+        ld = -(-cols // 16) * 16 if cols else 16
+        m = np.zeros((rows, ld), np.int8)
+        m[:, :cols] = t.mant
+        mt = torch.from_numpy(m)
+        et = torch.from_numpy(np.ascontiguousarray(t.exp))
+        if pin:
+            mt, et = mt.pin_memory(), et.pin_memory()
+        return DevCE(mt.to(device, non_blocking=pin), et.to(device, non_blocking=pin),
+                     t.g_rows, t.g_cols, cols=cols)
+
+    def to_host(self) -> CE:
+        m = self.mant[:, : self.cols].cpu().numpy().copy()
+        return CE(np.ascontiguousarray(m), self.exp.cpu().numpy().copy(), self.g_rows, self.g_cols)
+
+    def c(self) -> ict_tensor:
+        return ict_tensor(self.mant.data_ptr(), self.exp.data_ptr(), self.rows, self.cols, self.ld,
+                          self.g_rows, self.g_cols)
+
+
+def _ws(nbytes: int, device="cuda") -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)  # 256-aligned by torch
+
+
+# ----------------------------------------------------------------- raw entry points
+
+def ict_status_string(code: int) -> str:
+    return lib.ict_status_string(code).decode()
+
+
+def ict_version() -> str:
+    return lib.ict_version().decode()
+
+
+def ict_get_device_status(stream=None):
+    v = ctypes.c_int32(0)
+    code = lib.ict_get_device_status(ctypes.byref(v), _stream(stream))
+    return code, v.value
+
+
+def ict_launch_count() -> int:
+    return int(lib.ict_launch_count())
+
+
+def ict_set_wait_limit_ns(ns: int) -> None:
+    _check(lib.ict_set_wait_limit_ns(int(ns)), "ict_set_wait_limit_ns")
+
+
+def ict_requant(vals: torch.Tensor, out: DevCE, base_exp=0, row_exp=None, col_exp=None, stream=None):
+    bits = {torch.int32: 32, torch.int64: 64}[vals.dtype]
+    rows, cols = vals.shape
+    o = out.c()
+    _check(lib.ict_requant(_ptr(vals), bits, rows, cols, vals.stride(0), base_exp, _ptr(row_exp),
+                           _ptr(col_exp), ctypes.byref(o), _stream(stream)), "ict_requant")
+
+
+def ict_align(t: DevCE, axis: int, transpose: bool, out: torch.Tensor, e_star: torch.Tensor, stream=None):
+    c = t.c()
+    _check(lib.ict_align(ctypes.byref(c), axis, int(transpose), _ptr(out), out.stride(0), _ptr(e_star),
+                         _stream(stream)), "ict_align")
+
+
+def ict_linear_workspace(op: int, a: DevCE, b: DevCE, out: DevCE) -> int:
+    ca, cb, co = a.c(), b.c(), out.c()
+    return int(lib.ict_linear_workspace(op, ctypes.byref(ca), ctypes.byref(cb), ctypes.byref(co)))
+
+
+def _linear(fn, name, a, b, out, ws, stream):
+    ca, cb, co = a.c(), b.c(), out.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(fn(ctypes.byref(ca), ctypes.byref(cb), ctypes.byref(co), _ptr(ws), nbytes, _stream(stream)), name)
+
+
+def ict_linear_fwd(X: DevCE, W: DevCE, Y: DevCE, ws=None, stream=None):
+    _linear(lib.ict_linear_fwd, "ict_linear_fwd", X, W, Y, ws, stream)
+
+
+def ict_linear_bwd_data(dY: DevCE, W: DevCE, dX: DevCE, ws=None, stream=None):
+    _linear(lib.ict_linear_bwd_data, "ict_linear_bwd_data", dY, W, dX, ws, stream)
+
+
+def ict_linear_bwd_weight(dY: DevCE, X: DevCE, dW: DevCE, ws=None, stream=None):
+    _linear(lib.ict_linear_bwd_weight, "ict_linear_bwd_weight", dY, X, dW, ws, stream)
+
+
+def conv_desc(d: dict) -> ict_conv_desc:
+    return ict_conv_desc(*[int(d[k]) for k in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")])
+
+
+def ict_conv_workspace(direction: int, d: dict) -> int:
+    cd = conv_desc(d)
+    return int(lib.ict_conv_workspace(direction, ctypes.byref(cd)))
+
+
+def ict_conv_implicit_gemm(direction: int, d: dict, a: DevCE, b: DevCE, out: DevCE, ws=None, stream=None):
+    cd, ca, cb, co = conv_desc(d), a.c(), b.c(), out.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib.ict_conv_implicit_gemm(direction, ctypes.byref(cd), ctypes.byref(ca), ctypes.byref(cb),
+                                      ctypes.byref(co), _ptr(ws), nbytes, _stream(stream)),
+           "ict_conv_implicit_gemm")
+
+
+def sgd_params(mom=(230, 8), lr=(1, 4)) -> ict_sgd_params:
+    return ict_sgd_params(int(mom[0]), int(mom[1]), int(lr[0]), int(lr[1]))
+
+
+def ict_sgd_momentum_step(W: DevCE, V: DevCE, G: DevCE, mom=(230, 8), lr=(1, 4), stream=None):
+    cw, cv, cg, p = W.c(), V.c(), G.c(), sgd_params(mom, lr)
+    _check(lib.ict_sgd_momentum_step(ctypes.byref(cw), ctypes.byref(cv), ctypes.byref(cg), ctypes.byref(p),
+                                      _stream(stream)), "ict_sgd_momentum_step")
+
+
+def ict_sgd_momentum_step_multi(Ws, Vs, Gs, mom=(230, 8), lr=(1, 4), stream=None):
+    n = len(Ws)
+    cw = [w.c() for w in Ws]
+    cv = [v.c() for v in Vs]
+    cg = [g.c() for g in Gs]
+    arr = _P(ict_tensor) * n
+    pw = arr(*[ctypes.pointer(x) for x in cw])
+    pv = arr(*[ctypes.pointer(x) for x in cv])
+    pg = arr(*[ctypes.pointer(x) for x in cg])
+    p = sgd_params(mom, lr)
+    _check(lib.ict_sgd_momentum_step_multi(n, pw, pv, pg, ctypes.byref(p), _stream(stream)),
+           "ict_sgd_momentum_step_multi")
+
+
+def ict_gelu_fwd(H: DevCE, out: DevCE, stream=None):
+    ch, co = H.c(), out.c()
+    _check(lib.ict_gelu_fwd(ctypes.byref(ch), ctypes.byref(co), _stream(stream)), "ict_gelu_fwd")
+
+
+def ict_gelu_bwd(H: DevCE, dG: DevCE, dH: DevCE, stream=None):
+    ch, cd, co = H.c(), dG.c(), dH.c()
+    _check(lib.ict_gelu_bwd(ctypes.byref(ch), ctypes.byref(cd), ctypes.byref(co), _stream(stream)),
+           "ict_gelu_bwd")
+
+
+# ----------------------------------------------------------------- conveniences
+
+def linear_fwd(X: DevCE, W: DevCE, g_cols=32, stream=None) -> DevCE:
+    Y = DevCE.empty(X.rows, W.rows, 1, g_cols)
+    ict_linear_fwd(X, W, Y, _ws(ict_linear_workspace(OP_LINEAR_FWD, X, W, Y)), stream)
+    return Y
+
+
+def linear_bwd_data(dY: DevCE, W: DevCE, g_cols=32, stream=None) -> DevCE:
+    dX = DevCE.empty(dY.rows, W.cols, 1, g_cols)
+    ict_linear_bwd_data(dY, W, dX, _ws(ict_linear_workspace(OP_LINEAR_BWD_DATA, dY, W, dX)), stream)
+    return dX
+
+
+def linear_bwd_weight(dY: DevCE, X: DevCE, g_cols=None, stream=None) -> DevCE:
+    dW = DevCE.empty(dY.cols, X.cols, 1, g_cols or X.cols)
+    ict_linear_bwd_weight(dY, X, dW, _ws(ict_linear_workspace(OP_LINEAR_BWD_WEIGHT, dY, X, dW)), stream)
+    return dW
+
+
+def conv(direction: int, d: dict, a: DevCE, b: DevCE, g_rows: int, g_cols: int, stream=None) -> DevCE:
+    P = (d["h"] + 2 * d["pad"] - d["r"]) // d["stride"] + 1
+    Q = (d["w"] + 2 * d["pad"] - d["s"]) // d["stride"] + 1
+    if direction == CONV_FWD:
+        rows, cols = d["n"] * P * Q, d["k"]
+    elif direction == CONV_BWD_DATA:
+        rows, cols = d["n"] * d["h"] * d["w"], d["c"]
+    else:
+        rows, cols = d["k"], d["r"] * d["s"] * d["c"]
+    out = DevCE.empty(rows, cols, g_rows, g_cols)
+    ict_conv_implicit_gemm(direction, d, a, b, out, _ws(ict_conv_workspace(direction, d)), stream)
+    return out
+
+
+def gelu_fwd(H: DevCE, stream=None) -> DevCE:
+    out = DevCE.empty(H.rows, H.cols, H.g_rows, H.g_cols)
+    ict_gelu_fwd(H, out, stream)
+    return out
+
+
+def gelu_bwd(H: DevCE, dG: DevCE, stream=None) -> DevCE:
+    dH = DevCE.empty(H.rows, H.cols, 1, H.g_cols)
+    ict_gelu_bwd(H, dG, dH, stream)
+    return dH
+
+
+def device_status(stream=None) -> int:
+    code, _ = ict_get_device_status(stream)
+    return code

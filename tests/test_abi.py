@@ -1,0 +1,51 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every entry
+point that include/ict.h declares (no compute calls here)."""
+import ctypes
+import os
+import re
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ict.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ict_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("ict_linear_fwd", "ict_linear_bwd_data", "ict_linear_bwd_weight",
+                     "ict_conv_implicit_gemm", "ict_requant", "ict_sgd_momentum_step"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    from integer_only_nn_02_b200.csrc.build import build
+
+    path = build()
+    lib = ctypes.CDLL(path)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    lib.ict_status_string.restype = ctypes.c_char_p
+    assert lib.ict_status_string(0) == b"ICT_OK"
+    assert lib.ict_status_string(7) == b"ICT_ERR_DEVICE_TIMEOUT"
+
+
+def test_binding_names_match_header():
+    from integer_only_nn_02_b200 import ict
+
+    assert sorted(ict.EXPORTED) == declared_functions()
+    for name in ict.EXPORTED:
+        assert callable(getattr(ict, name))
+
+
+def test_library_shares_nothing_with_oracle():
+    """The oracle and the CUDA path share no source: no include of one by the other."""
+    csrc = os.path.join(ROOT, "integer_only_nn_02_b200", "csrc")
+    for f in os.listdir(csrc):
+        text = open(os.path.join(csrc, f)).read()
+        assert "oracle" not in text.lower() or f == "build.py" and "oracle" not in text
+    oracle_src = open(os.path.join(ROOT, "oracle", "ict_oracle.c")).read()
+    assert "#include \"" not in oracle_src

@@ -1,0 +1,248 @@
+"""GPU parity: every entry point of libict.so against the CPU oracle, bit for bit.
+
+Sizes span several 128-row tiles with ragged tails; group geometries cover per-tensor,
+per-row, row-local (1, G) and pixel-uniform channel groups.  All arithmetic is integer,
+so the comparison is exact equality of mantissas and exponent bytes.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from integer_only_nn_02_b200.workloads import CE, E_ZERO, clipped_laplace, with_groups
+from tests.test_oracle_pins import rand_ce
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ict():
+    from integer_only_nn_02_b200 import ict as _ict
+
+    return _ict
+
+
+def same(gpu_ce: CE, ref: CE, what=""):
+    assert gpu_ce.mant.shape == ref.mant.shape, what
+    bad = np.argwhere(gpu_ce.mant != ref.mant)
+    assert bad.size == 0, f"{what}: {len(bad)} mantissas differ, first {bad[:5].tolist()}"
+    bad = np.argwhere(gpu_ce.exp != ref.exp)
+    assert bad.size == 0, f"{what}: {len(bad)} exponents differ, first {bad[:5].tolist()}"
+
+
+def status_ok(ict):
+    code, raw = ict.ict_get_device_status()
+    assert code == 0, (code, raw)
+
+
+# ------------------------------------------------------------------ requant / align
+
+
+@pytest.mark.parametrize("rows,cols,G", [(5, 32, 32), (130, 96, 32), (64, 192, 64), (33, 768, 768), (7, 48, 16)])
+def test_requant(ict, rows, cols, G):
+    import torch
+
+    rng = np.random.default_rng(rows + cols)
+    for bits in (10, 24, 31):
+        x = rng.integers(-(2 ** bits), 2 ** bits, size=(rows, cols)).astype(np.int64)
+        x[rng.random(x.shape) < 0.1] = 0
+        x[3 % rows] = 0  # an all-zero row -> E_ZERO groups
+        re = rng.integers(-40, 20, size=rows).astype(np.int8)
+        ce = rng.integers(-40, 20, size=cols).astype(np.int8)
+        ref = oracle.requant(x, 1, G, base_exp=-5, row_exp=re, col_exp=ce)
+        for dt in (torch.int32, torch.int64):
+            if dt == torch.int32 and bits > 30:
+                continue
+            out = ict.DevCE.empty(rows, cols, 1, G)
+            ict.ict_requant(torch.tensor(x, dtype=dt, device="cuda"), out, -5,
+                            torch.tensor(re, device="cuda"), torch.tensor(ce, device="cuda"))
+            same(out.to_host(), ref, f"requant {dt} bits={bits}")
+    status_ok(ict)
+
+
+@pytest.mark.parametrize("rows,cols,g", [(64, 128, (1, 32)), (200, 96, (1, 16)), (130, 64, (130, 32)),
+                                         (48, 768, (1, 64)), (144, 32, (16, 32)), (100, 48, (1, 48))])
+@pytest.mark.parametrize("axis,transpose", [(1, False), (0, True), (0, False), (1, True)])
+def test_align(ict, rows, cols, g, axis, transpose):
+    import torch
+
+    rng = np.random.default_rng(rows * 3 + cols)
+    t = rand_ce(rng, rows, cols, *g, elo=-20, ehi=5, zero_groups=0.1)
+    ref_m, ref_e = oracle.align(t, axis, transpose)
+    d = ict.DevCE.from_host(t)
+    out_rows = cols if transpose else rows
+    ld = -(-(rows if transpose else cols) // 16) * 16
+    out = torch.zeros((out_rows, ld), dtype=torch.int8, device="cuda")
+    e = torch.zeros(rows if axis == 1 else cols, dtype=torch.int8, device="cuda")
+    ict.ict_align(d, axis, transpose, out, e)
+    got = out.cpu().numpy()[:, : ref_m.shape[1]]
+    assert (got == ref_m).all()
+    assert (e.cpu().numpy() == ref_e).all()
+
+
+# ------------------------------------------------------------------ linear
+
+LINEAR_CASES = [
+    # M, N, K, X groups, W groups, out group
+    (64, 64, 128, (64, 128), (1, 128), 32),      # the single-layer config shapes
+    (200, 192, 96, (1, 96), (1, 32), 32),
+    (300, 320, 256, (1, 64), (1, 256), 64),
+    (129, 256, 384, (1, 128), (4, 64), 256),
+    (512, 448, 192, (1, 192), (1, 192), 64),
+    (1000, 768, 768, (1, 64), (1, 64), 64),
+]
+
+
+def _linear_inputs(M, N, K, gx, gw, seed):
+    rng = np.random.default_rng(seed)
+    X = rand_ce(rng, M, K, *gx, elo=-10, ehi=-4, zero_groups=0.05)
+    W = rand_ce(rng, N, K, *gw, elo=-12, ehi=-6, zero_groups=0.05)
+    dY = with_groups(clipped_laplace(rng, (M, N)), 1, 32, lambda g: rng.integers(-16, -10, size=g))
+    return X, W, dY
+
+
+@pytest.mark.parametrize("case", LINEAR_CASES)
+def test_linear_fwd(ict, case):
+    M, N, K, gx, gw, G = case
+    X, W, _ = _linear_inputs(M, N, K, gx, gw, M + N + K)
+    ref = oracle.linear_fwd(X, W, 1, G)
+    got = ict.linear_fwd(ict.DevCE.from_host(X), ict.DevCE.from_host(W), G).to_host()
+    same(got, ref, f"fwd {case}")
+    status_ok(ict)
+
+
+@pytest.mark.parametrize("case", LINEAR_CASES)
+def test_linear_bwd_data(ict, case):
+    M, N, K, gx, gw, G = case
+    X, W, dY = _linear_inputs(M, N, K, gx, gw, M + 2 * N + K)
+    ref = oracle.linear_bwd_data(dY, W, 1, G)
+    got = ict.linear_bwd_data(ict.DevCE.from_host(dY), ict.DevCE.from_host(W), G).to_host()
+    same(got, ref, f"bwd_data {case}")
+    status_ok(ict)
+
+
+@pytest.mark.parametrize("case", LINEAR_CASES)
+@pytest.mark.parametrize("per_row", [True, False])
+def test_linear_bwd_weight(ict, case, per_row):
+    M, N, K, gx, gw, G = case
+    X, W, dY = _linear_inputs(M, N, K, gx, gw, M + 3 * N + K)
+    g = K if per_row else G
+    ref = oracle.linear_bwd_weight(dY, X, 1, g)
+    got = ict.linear_bwd_weight(ict.DevCE.from_host(dY), ict.DevCE.from_host(X), g).to_host()
+    same(got, ref, f"bwd_weight {case} per_row={per_row}")
+    status_ok(ict)
+
+
+def test_linear_long_contraction_int64(ict):
+    """K far beyond 2^17 products of 127^2: split-K int32 partials, int64 combine."""
+    rng = np.random.default_rng(77)
+    M, N, K = 160000, 64, 32
+    dY = CE(np.full((M, N), 127, np.int8), np.zeros((1, 1), np.int8), M, N)
+    X = CE(np.full((M, K), -127, np.int8), np.zeros((1, 1), np.int8), M, K)
+    dY.mant[rng.random((M, N)) < 0.01] = -127
+    ref = oracle.linear_bwd_weight(dY, X, 1, K)
+    got = ict.linear_bwd_weight(ict.DevCE.from_host(dY), ict.DevCE.from_host(X), K).to_host()
+    same(got, ref, "long K")
+    status_ok(ict)
+
+
+# ------------------------------------------------------------------ conv
+
+
+def _conv_inputs(seed, n, h, w, c, k, gx=32):
+    rng = np.random.default_rng(seed)
+    npix = n * h * w
+    X = with_groups(np.where(rng.random((npix, c)) < 0.5, 0, rng.integers(1, 128, size=(npix, c))).astype(np.int8),
+                    npix, gx, lambda g: rng.integers(-8, -5, size=g))
+    W = rand_ce(rng, k, 9 * c, 1, 9 * c, elo=-10, ehi=-6)
+    dY = with_groups(clipped_laplace(rng, (npix, k)), npix, gx, lambda g: rng.integers(-14, -11, size=g))
+    return X, W, dY, dict(n=n, h=h, w=w, c=c, k=k, r=3, s=3, stride=1, pad=1)
+
+
+@pytest.mark.parametrize("shape", [(2, 8, 8, 64, 64), (3, 7, 56, 64, 64), (1, 9, 20, 128, 64),
+                                   (2, 5, 12, 64, 128)])
+@pytest.mark.parametrize("global_groups", [True, False])
+def test_conv_fwd_and_bwd_data(ict, shape, global_groups):
+    X, W, dY, d = _conv_inputs(sum(shape), *shape)
+    npix = X.rows
+    g_rows = npix if global_groups else 1
+    for direction, a, b in ((ict.CONV_FWD, X, W), (ict.CONV_BWD_DATA, dY, W)):
+        ref = oracle.conv(direction, d, a, b, g_rows, 32)
+        got = ict.conv(direction, d, ict.DevCE.from_host(a), ict.DevCE.from_host(b), g_rows, 32).to_host()
+        same(got, ref, f"conv dir={direction} {shape} global={global_groups}")
+    status_ok(ict)
+
+
+# ------------------------------------------------------------------ GELU
+
+
+@pytest.mark.parametrize("rows,cols,G,erange", [(64, 768, 32, (-9, -5)), (130, 96, 32, (-30, 3)),
+                                                (17, 64, 64, (-127, -100)), (40, 32, 32, (-3, 4))])
+def test_gelu(ict, rows, cols, G, erange):
+    rng = np.random.default_rng(rows + cols + G)
+    H = rand_ce(rng, rows, cols, 1, G, elo=erange[0], ehi=erange[1], zero_groups=0.05)
+    dG = rand_ce(rng, rows, cols, 1, G, elo=-16, ehi=-8, zero_groups=0.05)
+    dHd, dGd = ict.DevCE.from_host(H), ict.DevCE.from_host(dG)
+    same(ict.gelu_fwd(dHd).to_host(), oracle.gelu_fwd(H), "gelu fwd")
+    same(ict.gelu_bwd(dHd, dGd).to_host(), oracle.gelu_bwd(H, dG, 1, G), "gelu bwd")
+    status_ok(ict)
+
+
+# ------------------------------------------------------------------ SGD
+
+
+@pytest.mark.parametrize("rows,cols,G", [(64, 128, 128), (100, 64, 64), (12, 768, 768), (40, 192, 192),
+                                         (9, 64, 16), (30, 200, 64)])
+@pytest.mark.parametrize("erange", [(-16, -4), (-100, 40)])
+def test_sgd(ict, rows, cols, G, erange):
+    rng = np.random.default_rng(rows * cols + G + erange[0] + 200)
+    W = rand_ce(rng, rows, cols, 1, G, *erange, zero_groups=0.05)
+    V = rand_ce(rng, rows, cols, 1, G, *erange, zero_groups=0.3)
+    Gr = rand_ce(rng, rows, cols, 1, G, *erange, zero_groups=0.05)
+    for mom, lr in (((230, 8), (1, 4)), ((230, 8), (205, 11))):
+        try:
+            W2, V2 = oracle.sgd_step(W, V, Gr, mom, lr)
+        except oracle.OracleError:
+            continue
+        dW, dV, dG = ict.DevCE.from_host(W), ict.DevCE.from_host(V), ict.DevCE.from_host(Gr)
+        ict.ict_sgd_momentum_step(dW, dV, dG, mom, lr)
+        same(dV.to_host(), V2, "velocity")
+        same(dW.to_host(), W2, "weight")
+    status_ok(ict)
+
+
+def test_sgd_multi_matches_single(ict):
+    rng = np.random.default_rng(5)
+    shapes = [(64, 128, 128), (10, 64, 64), (3, 768, 64)]
+    Ws, Vs, Gs, refs = [], [], [], []
+    for r, c, g in shapes:
+        W, V, G = (rand_ce(rng, r, c, 1, g, -16, -4) for _ in range(3))
+        refs.append(oracle.sgd_step(W, V, G))
+        Ws.append(ict.DevCE.from_host(W))
+        Vs.append(ict.DevCE.from_host(V))
+        Gs.append(ict.DevCE.from_host(G))
+    ict.ict_sgd_momentum_step_multi(Ws, Vs, Gs)
+    for (W2, V2), dW, dV in zip(refs, Ws, Vs):
+        same(dW.to_host(), W2, "multi W")
+        same(dV.to_host(), V2, "multi V")
+    status_ok(ict)
+
+
+# ------------------------------------------------------------------ errors
+
+
+def test_argument_errors_return_before_launch(ict):
+    X = ict.DevCE.from_host(CE(np.zeros((64, 128), np.int8), np.zeros((1, 1), np.int8), 64, 128))
+    W = ict.DevCE.from_host(CE(np.zeros((64, 96), np.int8), np.zeros((64, 1), np.int8), 1, 96))
+    Y = ict.DevCE.empty(64, 64, 1, 32)
+    with pytest.raises(ict.IctError) as ei:
+        ict.ict_linear_fwd(X, W, Y)
+    assert ei.value.code == 1
+    Yb = ict.DevCE.empty(64, 64, 2, 32)  # 2-row output groups are not row-local
+    W2 = ict.DevCE.from_host(CE(np.zeros((64, 128), np.int8), np.zeros((64, 1), np.int8), 1, 128))
+    with pytest.raises(ict.IctError) as ei:
+        ict.ict_linear_fwd(X, W2, Yb)
+    assert ei.value.code == 2
+    Y = ict.DevCE.empty(64, 64, 1, 32)
+    need = ict.ict_linear_workspace(ict.OP_LINEAR_FWD, X, W2, Y)
+    assert need == 0  # both operands uniform along K, fused epilogue
+    status_ok(ict)
