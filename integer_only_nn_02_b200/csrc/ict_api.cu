@@ -223,7 +223,7 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
     auto k = gemm_ce_kernel<BN, BK, ST, LOAD>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
         return ICT_ERR_CUDA;
-    k<<<grid, 256, L::kBytes, s>>>(ta, tb, p);
+    k<<<grid, 384, L::kBytes, s>>>(ta, tb, p);
     counted(1);
     return launch_status();
 }
@@ -253,6 +253,34 @@ int pick_bn(int64_t n) {
     if (n % 192 == 0) return 192;
     if (n % 128 == 0) return 128;
     return 256;
+}
+
+// Tile width for an M x N output on `sms` SMs: among the widths that keep the output
+// groups inside a tile, the one whose last wave of tiles is fullest (ties: wider).
+int pick_bn_waves(int64_t M, int64_t N, int64_t G, int sms) {
+    if (N <= 256) return pick_bn(N);
+    int best = 0;
+    double best_score = -1.0;
+    const int cands[3] = {256, 192, 128};
+    for (int bn : cands) {
+        const bool fits = G >= N ? false : (bn % G == 0 && G % 32 == 0);
+        if (!fits && G < N) continue;
+        const int64_t tiles = cdiv64(M, 128) * cdiv64(N, bn);
+        const int64_t waves = cdiv64(tiles, sms);
+        const double eff = (double)(M * N) / (double)(waves * sms * 128 * bn);
+        const double score = eff * (1.0 + 0.03 * bn / 64.0);
+        if (score > best_score) best_score = score, best = bn;
+    }
+    return best ? best : pick_bn(N);
+}
+
+// groups whose column exponents differ by at most this take the fast epilogue:
+// |acc| <= K * 127^2 shifted left by the spread must stay below 2^30
+int fast_slack_for(int64_t K) {
+    const uint64_t bound = (uint64_t)K * 127u * 127u;
+    int bits = 0;
+    while ((bound >> bits) != 0) ++bits;
+    return 30 - bits;
 }
 
 // A K-major operand of the Product: rows of int8, K contiguous, an exponent per row.
@@ -294,14 +322,15 @@ struct ProductPlan {
 ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out, int sms,
                          bool allow_split, Ws &ws) {
     ProductPlan pl;
-    pl.bn = pick_bn(N);
+    pl.bn = pick_bn_waves(M, N, out->g_cols, sms);
     pl.n_kblk = (int)cdiv64(K, 128);
     pl.n_mtiles = (int)cdiv64(M, 128);
     pl.n_ntiles = (int)cdiv64(N, pl.bn);
     const int tiles = pl.n_mtiles * pl.n_ntiles;
     int splits = 1;
     if (allow_split && tiles < sms && pl.n_kblk >= 8) {
-        splits = (int)std::min<int64_t>(cdiv64(sms, tiles), pl.n_kblk / 4);
+        // whole waves: as many K slices as fit next to the tiles on the SMs
+        splits = (int)std::min<int64_t>(sms / tiles, pl.n_kblk / 4);
         if (splits < 1) splits = 1;
     }
     // int32 partial sums stay exact: at most 2^17 products of magnitude <= 127^2 each
@@ -341,6 +370,7 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     p.eB = B.exp;
     p.eB_div = B.exp_div;
     p.G = (int)std::min<int64_t>(out->g_cols, N);
+    p.fast_slack = fast_slack_for(K);
     p.out = out->mant;
     p.out_ld = out->ld;
     p.out_exp = out->exp;
@@ -589,6 +619,7 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     p.eB = cp.eB;
     p.eB_div = cp.eB_div;
     p.G = (int)std::min<int64_t>(out->g_cols, cp.out_cols);
+    p.fast_slack = fast_slack_for(ktot);
     p.out = out->mant;
     p.out_ld = out->ld;
     p.out_exp = out->exp;
@@ -650,8 +681,36 @@ int check_sgd_params(const ict_sgd_params *p) {
     return ICT_OK;
 }
 
+template <int L, int CPL>
+int launch_sgd_vec(const SgdArgs &a, int sms, cudaStream_t s) {
+    constexpr int gpb = 8 * (32 / L);  // groups per block and pass
+    const int64_t blocks = std::min<int64_t>(cdiv64(a.total_groups, gpb), (int64_t)sms * 8);
+    sgd_vec_kernel<L, CPL><<<(unsigned)blocks, 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+// Vectorised kernel when every tensor shares one group width G (a multiple of 16, at
+// most 2048): L lanes per group, CPL 16-byte chunks per lane; else one warp per group.
 int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
     if (a.total_groups == 0) return ICT_OK;
+    bool vec = true;
+    const int G = a.t[0].G;
+    for (int i = 0; i < a.n; ++i)
+        vec = vec && a.t[i].G == G && (a.t[i].ld & 15) == 0 && aligned16(a.t[i].w) && aligned16(a.t[i].v) &&
+              aligned16(a.t[i].g);
+    vec = vec && G % 16 == 0 && G <= 2048;
+    if (vec) {
+        const int chunks = G / 16;
+        if (chunks <= 1) return launch_sgd_vec<1, 1>(a, sms, s);
+        if (chunks <= 2) return launch_sgd_vec<2, 1>(a, sms, s);
+        if (chunks <= 4) return launch_sgd_vec<4, 1>(a, sms, s);
+        if (chunks <= 8) return launch_sgd_vec<8, 1>(a, sms, s);
+        if (chunks <= 16) return launch_sgd_vec<16, 1>(a, sms, s);
+        if (chunks <= 32) return launch_sgd_vec<32, 1>(a, sms, s);
+        if (chunks <= 64) return launch_sgd_vec<32, 2>(a, sms, s);
+        if (chunks <= 128) return launch_sgd_vec<32, 4>(a, sms, s);
+    }
     const int64_t blocks = std::min<int64_t>(cdiv64(a.total_groups, 8), (int64_t)sms * 16);
     sgd_warp_kernel<<<(unsigned)blocks, 256, 0, s>>>(a);
     counted(1);

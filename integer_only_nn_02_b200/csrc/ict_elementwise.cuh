@@ -322,6 +322,242 @@ __device__ __forceinline__ void sgd_group(const SgdArgs &p, const SgdTensor &t, 
     }
 }
 
+// ---- vectorised SGD: L lanes per group, each lane holds CPL 16-byte chunks of W, V, G.
+
+template <int L>
+__device__ __forceinline__ int group_max(int v, unsigned mask) {
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(mask, v, o));
+    return v;
+}
+
+// Locates global group `gw` in the tensor list.
+__device__ __forceinline__ int sgd_find(const SgdArgs &p, int64_t gw) {
+    int lo = 0, hi = p.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.t[mid].first_group <= gw) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Two terms a_i * 2^pa + b_i * 2^pb of one group at the common exponent r0 = min(pa, pb):
+// x_i = a_i * ma + b_i * mb with ma = 2^(pa - r0), mb = 2^(pb - r0).  An exponent whose
+// term is absent (E_ZERO, all mantissas zero) takes the other one's value.
+struct GroupSum {
+    int r0;
+    int64_t ma, mb;
+    bool small;  // every |x_i| < 2^30 (int32 arithmetic is exact)
+    bool exact;  // exponents at most 32 apart (int64 arithmetic is exact)
+};
+__device__ __forceinline__ GroupSum group_sum(int pa, bool za, int64_t amax, int pb, bool zb, int64_t bmax) {
+    GroupSum g;
+    if (za && zb) za = false, pa = pb = 0;
+    if (za) pa = pb;
+    if (zb) pb = pa;
+    g.r0 = min(pa, pb);
+    const int da = pa - g.r0, db = pb - g.r0;
+    g.exact = da <= 32 && db <= 32;
+    g.ma = g.exact ? (1ll << da) : 0;
+    g.mb = g.exact ? (1ll << db) : 0;
+    g.small = g.exact && (amax << da) + (bmax << db) < (1ll << 30);
+    return g;
+}
+
+// RNE(x * 2^-S) for a group-uniform S with |x| < 2^30 (S < 0: exact left shift).
+struct Shift {
+    int ls, rs, bias, om;
+};
+__device__ __forceinline__ Shift make_shift(int S) {
+    Shift h;
+    h.ls = S < 0 ? -S : 0;
+    h.rs = S > 0 ? min(S, 31) : 0;
+    h.bias = h.rs ? (1 << (h.rs - 1)) - 1 : 0;
+    h.om = h.rs ? 1 : 0;
+    return h;
+}
+__device__ __forceinline__ int apply_shift(int x, const Shift &h) {
+    x <<= h.ls;
+    return (x + h.bias + ((x >> h.rs) & h.om)) >> h.rs;
+}
+
+// Exact FIT of the group values a_mul * A_i * 2^pa + b_mul * B_i * 2^pb element by element
+// in int64 (two_term: exact up to a 32-bit exponent gap, sticky beyond), for groups whose
+// values do not fit the int32 fast path.  Kept out of line: it is rare and register-hungry.
+// Exact SGD update of one group, element by element in int64 (two_term: exact up to a
+// 32-bit exponent gap, sticky beyond), for groups whose values do not fit the int32 fast
+// path.  Reads W, V, G from memory again and writes the results; each lane handles the
+// elements li, li + L, ... of the group.  Out of line with rolled loops: it is rare and
+// must not cost the fast path registers.
+template <int L>
+__device__ __noinline__ void sgd_group_exact(const SgdArgs &p, const SgdTensor &t, int64_t row0,
+                                             int64_t ge, int glen, int li, unsigned gmask) {
+    const int ev = t.v_exp[ge], eg = t.g_exp[ge], ew = t.w_exp[ge];
+    const int pv = ev - p.mom_shift;
+    int emax = kNoExp;
+    for (int j = li; j < glen; j += L) {
+        const TwoTerm x = two_term((int64_t)p.mom_mul * t.v[row0 + j], pv, t.g[row0 + j], eg);
+        if (x.x) emax = max(emax, need64(x.x, x.r));
+    }
+    const int ev2 = finalize_exp(group_max<L>(emax, gmask));
+    const int pu = ev2 - p.lr_shift;
+    emax = kNoExp;
+    for (int j = li; j < glen; j += L) {
+        const TwoTerm x = two_term((int64_t)p.mom_mul * t.v[row0 + j], pv, t.g[row0 + j], eg);
+        const int cv = requant64(x.x, x.r, ev2);
+        const TwoTerm w = two_term(t.w[row0 + j], ew, -(int64_t)p.lr_mul * cv, pu);
+        if (w.x) emax = max(emax, need64(w.x, w.r));
+    }
+    const int ew2 = finalize_exp(group_max<L>(emax, gmask));
+    for (int j = li; j < glen; j += L) {
+        const TwoTerm x = two_term((int64_t)p.mom_mul * t.v[row0 + j], pv, t.g[row0 + j], eg);
+        const int cv = requant64(x.x, x.r, ev2);
+        const TwoTerm w = two_term(t.w[row0 + j], ew, -(int64_t)p.lr_mul * cv, pu);
+        t.v[row0 + j] = (int8_t)cv;
+        t.w[row0 + j] = (int8_t)requant64(w.x, w.r, ew2);
+    }
+    if (li == 0) {
+        t.v_exp[ge] = (int8_t)ev2;
+        t.w_exp[ge] = (int8_t)ew2;
+    }
+}
+
+template <int L, int CPL>
+__global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ SgdArgs p) {
+    constexpr int GPW = 32 / L;  // groups per warp and pass
+    const int lane = threadIdx.x & 31, sub = lane / L, li = lane % L;
+    const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (sub * L));
+    const int64_t nwarps = (int64_t)gridDim.x * 8;
+    for (int64_t base = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * GPW; base < p.total_groups;
+         base += nwarps * GPW) {
+        const int64_t gw = base + sub;
+        if (gw >= p.total_groups) continue;  // whole groups only: lanes of a group agree
+        const SgdTensor &t = p.t[sgd_find(p, gw)];
+        const int64_t local = gw - t.first_group;
+        const int64_t i = local / t.ngc, gi = local % t.ngc;
+        const int64_t ge = i * t.ngc + gi;
+        const int64_t j0 = gi * t.G;
+        const int glen = (int)min((int64_t)t.G, t.cols - j0);
+        const int ev = t.v_exp[ge], eg = t.g_exp[ge], ew = t.w_exp[ge];
+
+        uint32_t wv[CPL][4], vv[CPL][4], gv[CPL][4];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            const int off = (k * L + li) * 16;
+            if (off < glen) {
+                const int64_t at = i * t.ld + j0 + off;
+                const uint4 a = *reinterpret_cast<const uint4 *>(t.w + at);
+                const uint4 b = *reinterpret_cast<const uint4 *>(t.v + at);
+                const uint4 c = *reinterpret_cast<const uint4 *>(t.g + at);
+                wv[k][0] = a.x, wv[k][1] = a.y, wv[k][2] = a.z, wv[k][3] = a.w;
+                vv[k][0] = b.x, vv[k][1] = b.y, vv[k][2] = b.z, vv[k][3] = b.w;
+                gv[k][0] = c.x, gv[k][1] = c.y, gv[k][2] = c.z, gv[k][3] = c.w;
+                const int rem = glen - off;  // mask columns past the group's end
+                if (rem < 16) {
+#pragma unroll
+                    for (int b2 = 0; b2 < 16; ++b2)
+                        if (b2 >= rem) {
+                            const uint32_t m = ~(0xffu << (8 * (b2 & 3)));
+                            wv[k][b2 >> 2] &= m, vv[k][b2 >> 2] &= m, gv[k][b2 >> 2] &= m;
+                        }
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) wv[k][q] = vv[k][q] = gv[k][q] = 0;
+            }
+        }
+
+        // ---- velocity: v = mom * V + G
+        const GroupSum s1 = group_sum(ev - p.mom_shift, ev == kEZero, 127ll * abs(p.mom_mul), eg,
+                                      eg == kEZero, 127);
+        uint32_t nv[CPL][4];  // new velocity mantissas (packed)
+        int ev2;
+        if (s1.small) {
+            const int ma = (int)s1.ma * p.mom_mul, mb = (int)s1.mb;
+            int amax = 0;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int b2 = 0; b2 < 16; ++b2) {
+                    const int x = sx8(vv[k][b2 >> 2], b2 & 3) * ma + sx8(gv[k][b2 >> 2], b2 & 3) * mb;
+                    amax = max(amax, abs(x));
+                }
+            amax = group_max<L>(amax, gmask);
+            ev2 = finalize_exp(amax ? s1.r0 + need_off32((uint32_t)amax) : kNoExp);
+            const Shift h = make_shift(ev2 == kEZero ? 0 : ev2 - s1.r0);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    int r[4];
+#pragma unroll
+                    for (int b2 = 0; b2 < 4; ++b2)
+                        r[b2] = apply_shift(sx8(vv[k][q], b2) * ma + sx8(gv[k][q], b2) * mb, h);
+                    nv[k][q] = pack4(r[0], r[1], r[2], r[3]);
+                }
+        } else {
+            sgd_group_exact<L>(p, t, i * t.ld + j0, ge, glen, li, gmask);
+            continue;
+        }
+
+        // ---- weight: w = W - lr * v'
+        const GroupSum s2 = group_sum(ew, ew == kEZero, 127, ev2 - p.lr_shift, ev2 == kEZero,
+                                      127ll * abs(p.lr_mul));
+        uint32_t nw[CPL][4];
+        int ew2;
+        if (s2.small) {
+            const int ma = (int)s2.ma, mb = -(int)s2.mb * p.lr_mul;
+            int amax = 0;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int b2 = 0; b2 < 16; ++b2) {
+                    const int x = sx8(wv[k][b2 >> 2], b2 & 3) * ma + sx8(nv[k][b2 >> 2], b2 & 3) * mb;
+                    amax = max(amax, abs(x));
+                }
+            amax = group_max<L>(amax, gmask);
+            ew2 = finalize_exp(amax ? s2.r0 + need_off32((uint32_t)amax) : kNoExp);
+            const Shift h = make_shift(ew2 == kEZero ? 0 : ew2 - s2.r0);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    int r[4];
+#pragma unroll
+                    for (int b2 = 0; b2 < 4; ++b2)
+                        r[b2] = apply_shift(sx8(wv[k][q], b2) * ma + sx8(nv[k][q], b2) * mb, h);
+                    nw[k][q] = pack4(r[0], r[1], r[2], r[3]);
+                }
+        } else {
+            sgd_group_exact<L>(p, t, i * t.ld + j0, ge, glen, li, gmask);
+            continue;
+        }
+
+        // ---- store (masked columns past the group's end are left untouched)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            const int off = (k * L + li) * 16;
+            if (off < glen) {
+                const int64_t at = i * t.ld + j0 + off;
+                if (glen - off >= 16) {
+                    *reinterpret_cast<uint4 *>(t.v + at) = make_uint4(nv[k][0], nv[k][1], nv[k][2], nv[k][3]);
+                    *reinterpret_cast<uint4 *>(t.w + at) = make_uint4(nw[k][0], nw[k][1], nw[k][2], nw[k][3]);
+                } else {
+                    for (int b2 = 0; b2 < glen - off; ++b2) {
+                        t.v[at + b2] = (int8_t)(nv[k][b2 >> 2] >> (8 * (b2 & 3)));
+                        t.w[at + b2] = (int8_t)(nw[k][b2 >> 2] >> (8 * (b2 & 3)));
+                    }
+                }
+            }
+        }
+        if (li == 0) {
+            t.v_exp[ge] = (int8_t)ev2;
+            t.w_exp[ge] = (int8_t)ew2;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256) sgd_warp_kernel(const __grid_constant__ SgdArgs p) {
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * 8;

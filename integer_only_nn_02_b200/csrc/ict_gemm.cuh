@@ -8,14 +8,21 @@
 // (convolution, linear and patch embedding are instances of the Product primitive)
 // and Figure 1a (forward and backward of every layer in integer arithmetic).
 //
-// Structure (one CTA per SM, persistent over output tiles):
-//   warp 0      TMA producer: A and B K-major tiles into a STAGES-deep ring of
-//               swizzled shared-memory buffers (mbarrier full/empty pairs)
-//   warp 1      MMA issuer: one thread issues tcgen05.mma kind::i8 (M = 128) into a
-//               double-buffered TMEM accumulator; tcgen05.commit frees smem stages
-//   warp 2      TMEM allocation / release
-//   warps 4..7  epilogue: tcgen05.ld (thread = output row), group max of need(),
-//               RNE shift, int8 stores of mantissas and group exponents
+// Structure (one CTA per SM, persistent over output tiles, 384 threads):
+//   warp 0       TMA producer: A and B K-major tiles into a STAGES-deep ring of
+//                swizzled shared-memory buffers (mbarrier full/empty pairs)
+//   warp 1       MMA issuer: one thread issues tcgen05.mma kind::i8 (M = 128) into a
+//                double-buffered TMEM accumulator; tcgen05.commit frees smem stages
+//   warp 2       TMEM allocation / release
+//   warps 4..7   epilogue warpgroup 0 (tiles using accumulator 0)
+//   warps 8..11  epilogue warpgroup 1 (tiles using accumulator 1)
+//                tcgen05.ld (thread = output row), group exponent, RNE shift, int8
+//                stores of mantissas and group exponents.
+// Epilogue fast path: within one output group the exponent of element (m, n) is
+// eA[m] + eB[n]; with d_n = eB[n] - min_group(eB) every accumulator shifted left by d_n
+// is exact below 2^30 when the group's spread is small, so the group exponent is
+// need(max |x << d_n|) and every mantissa is one RNE shift of x << d_n by a per-row
+// amount.  Groups with a larger spread take the exact per-element path.
 // Every wait is bounded; on expiry the CTA raises ICT_ERR_DEVICE_TIMEOUT, drains its
 // in-flight copies and MMAs (again with a bound), frees TMEM and exits.
 #pragma once
@@ -41,6 +48,7 @@ struct GemmParams {
     const int8_t *eB;
     int eB_div;     // exponent of output column n: eB[n / eB_div]
     int G;          // output group width along N
+    int fast_slack; // groups whose eB spread is at most this take the fast epilogue
     int8_t *out;
     int64_t out_ld;
     int8_t *out_exp;
@@ -63,13 +71,23 @@ struct GemmSmem {
                                    : (2 * BN <= 256) ? 256 : 512;
     static constexpr int kOffB = STAGES * kABytes;
     static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 5 mbarriers
-    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 5) * 8;
-    static constexpr int kOffEB = kOffMisc + 16;
-    static constexpr int kBytes = kOffEB + 4 * BN + 1024;  // + alignment slack
+    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 5) * 8 + 15) / 16 * 16;
+    static constexpr int kColInts = 2 * BN + 16;               // per epilogue warpgroup
+    static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
+    static constexpr int kBytes = kOffCol + 2 * kColInts * 4 + 1024;  // + alignment slack
+    static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
+                  "column tables are read as int4");
+    static_assert(kABytes % 1024 == 0 && kBBytes % 512 == 0 && kOffB % 1024 == 0,
+                  "operand tiles must sit on their swizzle-atom boundaries");
+    static_assert(kBytes <= 232448, "shared memory per block");
 };
 
+__device__ __forceinline__ uint32_t pack4b(int a, int b, int c, int d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 template <int BN, int BK, int STAGES, int LOAD>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
     using L = GemmSmem<BN, BK, STAGES>;
@@ -84,7 +102,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t bar_tempty = bar_tfull + 16;             // [2]
     const uint32_t bar_drain = bar_tempty + 16;             // [1]
     volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
-    int *sEB = (int *)(smem + L::kOffEB);
+    int *sCol = (int *)(smem + L::kOffCol);  // per epilogue warpgroup column tables
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -211,12 +229,20 @@ __global__ void __launch_bounds__(256, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - 128;  // output row within the tile = TMEM lane
-        const int quarter = warp & 3;
-        int it = 0;
+        const int wg = (warp - 4) >> 2;           // warpgroup: owns accumulator buffer wg
+        const int et = (threadIdx.x & 127);       // output row within the tile = TMEM lane
+        const int quarter = warp & 3, wq = (warp - 4) & 3;
+        const int bar_id = 1 + wg;
+        int *colE = sCol + wg * L::kColInts;       // [BN] exponent of B row (output column)
+        int *colD = colE + BN;                     // [BN] shift of the column in its group
+        int *gmin = colD + BN;                     // [8]  min column exponent of each group
+        int *gfast = gmin + 8;                     // [8]  group takes the fast path
+        const int Gt = p.G >= p.N ? BN : p.G;      // group width inside the tile
+        const int ngroups = BN / Gt;
+        int it = wg;
         // The loop never tests the abort flag on its own: the 128 threads decide together
         // through a barrier reduction, so none of them can be left waiting at a barrier.
-        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++it) {
+        for (int u = blockIdx.x + wg * gridDim.x; u < p.num_units; u += 2 * gridDim.x, it += 2) {
             const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
             const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
             const int acc = it & 1;
@@ -232,13 +258,36 @@ __global__ void __launch_bounds__(256, 1)
                 valid_rows = min(128, p.M - mt * 128);
             }
             const int n0 = nt * BN;
+            // column tables of this tile (independent of the accumulator: built before waiting)
             for (int j = et; j < BN; j += 128) {
                 const int n = n0 + j;
-                sEB[j] = n < p.N ? (int)p.eB[n / p.eB_div] : 0;
+                colE[j] = n < p.N ? (int)p.eB[n / p.eB_div] : kEZero;
+            }
+            named_bar_sync(bar_id, 128);
+            for (int g = wq; g < ngroups; g += 4) {
+                int lo = 0x7fffffff, hi = kNoExp;
+                for (int j = g * Gt + lane; j < (g + 1) * Gt; j += 32) {
+                    const int e = colE[j];
+                    if (e != kEZero) lo = min(lo, e), hi = max(hi, e);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                }
+                if (lane == 0) {
+                    gmin[g] = hi <= kNoExp ? 0 : lo;
+                    gfast[g] = hi <= kNoExp || hi - lo <= p.fast_slack;
+                }
+            }
+            named_bar_sync(bar_id, 128);
+            for (int j = et; j < BN; j += 128) {
+                const int e = colE[j];
+                colD[j] = e == kEZero ? 0 : e - gmin[j / Gt];
             }
             const bool ok = mbar_wait(bar_tfull + 8 * acc, (it >> 1) & 1, p.wait_ns, abort_flag);
             if (!ok) fail();
-            if (named_bar_or(1, 128, !ok || *abort_flag)) break;
+            if (named_bar_or(bar_id, 128, !ok || *abort_flag)) break;  // also publishes colD
             tc_fence_after();
 
             const bool valid = et < valid_rows;
@@ -261,47 +310,107 @@ __global__ void __launch_bounds__(256, 1)
                     }
                 }
             } else {
-                // groups wider than the output (whole rows) are one tile-wide group; the
-                // host guarantees G % 32 == 0 and BN % G == 0 otherwise
-                const int G = p.G >= p.N ? BN : p.G;
-                for (int g0 = 0; g0 < BN; g0 += G) {
-                    int emax = kNoExp;
-                    for (int c = g0; c < g0 + G; c += 32) {
-                        tmem_ld32(taddr + c, v);
-                        tmem_ld_wait();
-                        if (valid) {
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) {
-                                const int32_t x = (int32_t)v[q];
-                                if (x) emax = max(emax, ea + sEB[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
-                            }
-                        }
-                    }
+                for (int g = 0; g < ngroups; ++g) {
+                    const int g0 = g * Gt;
                     const int gcol = (n0 + g0) / p.G;
-                    if (p.epi == EPI_NEED_GLOBAL) {
-                        const int m = warp_max(emax);
-                        if (lane == 0 && m > kNoExp && n0 + g0 < p.N) atomicMax(p.gmax + gcol, m);
-                        continue;
-                    }
-                    const int e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : emax);
-                    for (int c = g0; c < g0 + G; c += 32) {
-                        if (G > 32) {
+                    const int gm = gmin[g];
+                    int e;
+                    if (gfast[g]) {
+                        // |x << d| < 2^30: the group exponent follows from the largest magnitude
+                        int ymax = 0, ymin = 0;
+                        for (int c = g0; c < g0 + Gt; c += 32) {
                             tmem_ld32(taddr + c, v);
                             tmem_ld_wait();
-                        }
-                        if (valid) {
-                            uint32_t w[8];
+                            if (valid) {
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                w[q] = pack4(requant32((int32_t)v[4 * q], ea + sEB[c + 4 * q], e),
-                                             requant32((int32_t)v[4 * q + 1], ea + sEB[c + 4 * q + 1], e),
-                                             requant32((int32_t)v[4 * q + 2], ea + sEB[c + 4 * q + 2], e),
-                                             requant32((int32_t)v[4 * q + 3], ea + sEB[c + 4 * q + 3], e));
-                            int8_t *dst = p.out + grow * p.out_ld + n0 + c;
-                            if (n0 + c < p.N)
-                                *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-                            if (n0 + c + 16 < p.N)
-                                *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                                for (int q = 0; q < 32; q += 4) {
+                                    const int4 d4 = *reinterpret_cast<const int4 *>(colD + c + q);
+                                    const int y0 = (int)v[q] << d4.x, y1 = (int)v[q + 1] << d4.y;
+                                    const int y2 = (int)v[q + 2] << d4.z, y3 = (int)v[q + 3] << d4.w;
+                                    ymax = max(ymax, max(max(y0, y1), max(y2, y3)));
+                                    ymin = min(ymin, min(min(y0, y1), min(y2, y3)));
+                                }
+                            }
+                        }
+                        const int amax = max(ymax, -ymin);
+                        const int need = amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp;
+                        if (p.epi == EPI_NEED_GLOBAL) {
+                            const int m = warp_max(need);
+                            if (lane == 0 && m > kNoExp && n0 + g0 < p.N) atomicMax(p.gmax + gcol, m);
+                            continue;
+                        }
+                        e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : need);
+                        // mantissa = RNE((x << d) * 2^-S), S = e - ea - gm uniform over the row
+                        const int S = (e == kEZero) ? 0 : e - ea - gm;
+                        const int ls = S < 0 ? -S : 0;
+                        const int rs = S > 0 ? min(S, 31) : 0;
+                        const int bias = rs ? (1 << (rs - 1)) - 1 : 0;
+                        const int om = rs ? 1 : 0;
+                        const bool any_ls = __any_sync(0xffffffffu, valid && ls != 0);
+                        for (int c = g0; c < g0 + Gt; c += 32) {
+                            if (Gt > 32) {
+                                tmem_ld32(taddr + c, v);
+                                tmem_ld_wait();
+                            }
+                            if (valid) {
+                                uint32_t w[8];
+#pragma unroll
+                                for (int q = 0; q < 32; q += 4) {
+                                    const int4 d4 = *reinterpret_cast<const int4 *>(colD + c + q);
+                                    int y[4] = {(int)v[q] << d4.x, (int)v[q + 1] << d4.y,
+                                                (int)v[q + 2] << d4.z, (int)v[q + 3] << d4.w};
+                                    if (any_ls) {
+#pragma unroll
+                                        for (int t = 0; t < 4; ++t) y[t] <<= ls;
+                                    }
+#pragma unroll
+                                    for (int t = 0; t < 4; ++t) y[t] = (y[t] + bias + ((y[t] >> rs) & om)) >> rs;
+                                    w[q >> 2] = pack4b(y[0], y[1], y[2], y[3]);
+                                }
+                                int8_t *dst = p.out + grow * p.out_ld + n0 + c;
+                                if (n0 + c < p.N)
+                                    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                                if (n0 + c + 16 < p.N)
+                                    *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                            }
+                        }
+                    } else {
+                        // exact per-element path: exponent eA + eB[n] per element
+                        int emax = kNoExp;
+                        for (int c = g0; c < g0 + Gt; c += 32) {
+                            tmem_ld32(taddr + c, v);
+                            tmem_ld_wait();
+                            if (valid) {
+#pragma unroll
+                                for (int q = 0; q < 32; ++q) {
+                                    const int32_t x = (int32_t)v[q];
+                                    if (x) emax = max(emax, ea + colE[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
+                                }
+                            }
+                        }
+                        if (p.epi == EPI_NEED_GLOBAL) {
+                            const int m = warp_max(emax);
+                            if (lane == 0 && m > kNoExp && n0 + g0 < p.N) atomicMax(p.gmax + gcol, m);
+                            continue;
+                        }
+                        e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : emax);
+                        for (int c = g0; c < g0 + Gt; c += 32) {
+                            tmem_ld32(taddr + c, v);
+                            tmem_ld_wait();
+                            if (valid) {
+                                uint32_t w[8];
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    w[q] = pack4b(requant32((int32_t)v[4 * q], ea + colE[c + 4 * q], e),
+                                                  requant32((int32_t)v[4 * q + 1], ea + colE[c + 4 * q + 1], e),
+                                                  requant32((int32_t)v[4 * q + 2], ea + colE[c + 4 * q + 2], e),
+                                                  requant32((int32_t)v[4 * q + 3], ea + colE[c + 4 * q + 3], e));
+                                int8_t *dst = p.out + grow * p.out_ld + n0 + c;
+                                if (n0 + c < p.N)
+                                    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                                if (n0 + c + 16 < p.N)
+                                    *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                            }
                         }
                     }
                     if (n0 + g0 < p.N) {
@@ -312,7 +421,7 @@ __global__ void __launch_bounds__(256, 1)
             }
             tc_fence_before();
             mbar_arrive(bar_tempty + 8 * acc);
-            named_bar_sync(1, 128);  // sEB is rewritten for the next tile
+            named_bar_sync(bar_id, 128);  // the column tables are rewritten for the next tile
         }
     }
 
