@@ -161,6 +161,26 @@ int32_t ict_linear_bwd_data(const ict_tensor *dY, const ict_tensor *W, ict_tenso
 int32_t ict_linear_bwd_weight(const ict_tensor *dY, const ict_tensor *X, ict_tensor *dW,
                               void *ws, size_t ws_bytes, void *stream);
 
+/* Allocation-free forward Product.  The paper has no counterpart to this entry point;
+ * it exists for callers that cannot hand the library a device workspace: integrations
+ * whose device memory is reserved up front by a host framework that exposes no
+ * allocator, statically budgeted deployments, and code paths that must not call
+ * cudaMalloc/cudaFree because those calls can block or synchronise the device.
+ * Same arguments and result as ict_linear_fwd, without ws: the scratch it needs (the
+ * aligned copies of X and/or W and, when the output groups span several tiles, int32
+ * partial sums) lives in one fixed array of ICT_NOALLOC_SCRATCH_BYTES bytes inside the
+ * library, which every GPU that loads the library holds until the process exits.
+ *   - Problems whose scratch need (ict_linear_workspace for the same arguments) exceeds
+ *     ICT_NOALLOC_SCRATCH_BYTES are rejected with ICT_ERR_WORKSPACE before any launch.
+ *   - It never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - The first call on a device looks up that device's copy of the array (with the
+ *     device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents: calls that
+ *     can overlap on the GPU (other streams, other threads) race on it and must be
+ *     serialised by the caller. */
+#define ICT_NOALLOC_SCRATCH_BYTES (16u << 20)
+int32_t ict_linear_fwd_noalloc(const ict_tensor *X, const ict_tensor *W, ict_tensor *Y, void *stream);
+
 /* --------------------------------------------------------------------------------- */
 /* Convolution as implicit GEMM (Table 6: "Convolution ... Product").                  */
 /*   dir FWD         a = X  [n*h*w][c], b = W [k][r*s*c] -> out = Y  [n*p*q][k]        */

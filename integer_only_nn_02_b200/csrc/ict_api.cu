@@ -717,6 +717,27 @@ int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
     return launch_status();
 }
 
+// ---- allocation-free forward Product: fixed scratch inside the library
+
+// One array per device that loads the library; host code must not pass its name to a
+// kernel (on the host it is only a stand-in), so its device address is looked up once
+// per device with cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ICT_NOALLOC_SCRATCH_BYTES];
+void *g_noalloc_addr[64];
+
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ICT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ICT_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return ICT_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -815,6 +836,18 @@ int32_t ict_linear_fwd(const ict_tensor *X, const ict_tensor *W, ict_tensor *Y, 
                        size_t ws_bytes, void *stream) {
     return linear_entry(ICT_OP_LINEAR_FWD, X, W, Y, ws, ws_bytes, stream);
 }
+int32_t ict_linear_fwd_noalloc(const ict_tensor *X, const ict_tensor *W, ict_tensor *Y, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    LinearPlan lp;
+    Ws dry = make_ws(nullptr, 0, true);
+    if ((st = plan_linear(ICT_OP_LINEAR_FWD, X, W, Y, dry, &lp))) return st;
+    if (dry.used > ICT_NOALLOC_SCRATCH_BYTES) return ICT_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch))) return st;
+    return linear_entry(ICT_OP_LINEAR_FWD, X, W, Y, scratch, ICT_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 int32_t ict_linear_bwd_data(const ict_tensor *dY, const ict_tensor *W, ict_tensor *dX, void *ws,
                             size_t ws_bytes, void *stream) {
     return linear_entry(ICT_OP_LINEAR_BWD_DATA, dY, W, dX, ws, ws_bytes, stream);

@@ -23,6 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libict.so")
 
 ICT_OK = 0
+NOALLOC_SCRATCH_BYTES = 16 << 20  # ICT_NOALLOC_SCRATCH_BYTES in include/ict.h
 STATUS_NAMES = {
     0: "ICT_OK", 1: "ICT_ERR_INVALID_ARG", 2: "ICT_ERR_LAYOUT", 3: "ICT_ERR_ALIGNMENT",
     4: "ICT_ERR_WORKSPACE", 5: "ICT_ERR_UNSUPPORTED_ARCH", 6: "ICT_ERR_CUDA",
@@ -64,6 +65,7 @@ _SIGS = {
     "ict_align": ([_P(ict_tensor), _i32, _i32, _vp, _i64, _vp, _vp], _i32),
     "ict_linear_workspace": ([_i32, _P(ict_tensor), _P(ict_tensor), _P(ict_tensor)], _sz),
     "ict_linear_fwd": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_linear_fwd_noalloc": ([_P(ict_tensor)] * 3 + [_vp], _i32),
     "ict_linear_bwd_data": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
     "ict_linear_bwd_weight": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
     "ict_conv_workspace": ([_i32, _P(ict_conv_desc)], _sz),
@@ -202,6 +204,13 @@ def _linear(fn, name, a, b, out, ws, stream):
 
 def ict_linear_fwd(X: DevCE, W: DevCE, Y: DevCE, ws=None, stream=None):
     _linear(lib.ict_linear_fwd, "ict_linear_fwd", X, W, Y, ws, stream)
+
+
+def ict_linear_fwd_noalloc(X: DevCE, W: DevCE, Y: DevCE, stream=None):
+    """Forward Product with the library's fixed internal scratch instead of a workspace."""
+    cx, cw, cy = X.c(), W.c(), Y.c()
+    _check(lib.ict_linear_fwd_noalloc(ctypes.byref(cx), ctypes.byref(cw), ctypes.byref(cy), _stream(stream)),
+           "ict_linear_fwd_noalloc")
 
 
 def ict_linear_bwd_data(dY: DevCE, W: DevCE, dX: DevCE, ws=None, stream=None):
