@@ -159,12 +159,14 @@ struct AlignJob {
     int8_t *out;
     int64_t ld;
     int8_t *e_star;
+    int32_t *col_max;  // axis 0: int32 scratch [group columns] for a parallel column max
 };
 
 int launch_align(const AlignJob &j, cudaStream_t s) {
     const ict_tensor *in = j.t;
     if (in->rows == 0 || in->cols == 0) return ICT_OK;
     AlignArgs a;
+    memset(&a, 0, sizeof(a));
     a.in = in->mant;
     a.in_exp = in->exp;
     a.rows = in->rows;
@@ -177,10 +179,25 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     a.out = j.out;
     a.out_ld = j.ld;
     a.e_star = j.e_star;
-    if (j.axis == 1)
+    int sms = 148;
+    device_info(&sms);
+    const int64_t n_exp = n_grp_rows(in) * a.ngc;
+    if (j.axis == 1) {
         estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
-    else
+    } else if (j.col_max && a.ngc <= 8192) {
+        // every thread keeps one group column: a stride that is a multiple of ngc
+        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(n_exp, 256 * 8), (int64_t)sms * 4));
+        const int64_t used = (blocks * 256) / a.ngc * a.ngc;
+        if (used >= a.ngc) {
+            if (cudaMemsetAsync(j.col_max, 0x80, (size_t)a.ngc * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
+            estar_cols_scratch_kernel<<<(unsigned)blocks, 256, (size_t)a.ngc * 4, s>>>(a, j.col_max, used);
+            a.col_max = j.col_max;
+        } else {
+            estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
+        }
+    } else {
         estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
+    }
     dim3 grid((unsigned)cdiv64(in->cols, 64), (unsigned)cdiv64(in->rows, 64));
     if (j.transpose)
         align_tile_kernel<true><<<grid, 256, 0, s>>>(a);
@@ -190,10 +207,29 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     return launch_status();
 }
 
+template <int T, int EPT>
+void launch_requant_block(const RequantArgs &a, int64_t groups, cudaStream_t s) {
+    requant_group_block_kernel<T, EPT><<<(unsigned)groups, T, 0, s>>>(a);
+}
+
+// FIT into row-local groups: one warp per group up to 127 elements, one block per
+// group (values held in registers) for wider groups up to 4096.
 int launch_requant_rows(RequantArgs a, cudaStream_t s) {
     const int64_t groups = a.rows * a.ngc;
     if (groups == 0) return ICT_OK;
-    requant_rows_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, s>>>(a);
+    const int G = a.G;
+    if (G >= 128 && G <= 4096) {
+        const int T = G >= 256 ? 256 : 128;
+        const int ept = (G + T - 1) / T;
+        if (T == 128) launch_requant_block<128, 1>(a, groups, s);
+        else if (ept <= 1) launch_requant_block<256, 1>(a, groups, s);
+        else if (ept <= 2) launch_requant_block<256, 2>(a, groups, s);
+        else if (ept <= 4) launch_requant_block<256, 4>(a, groups, s);
+        else if (ept <= 8) launch_requant_block<256, 8>(a, groups, s);
+        else launch_requant_block<256, 16>(a, groups, s);
+    } else {
+        requant_rows_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, s>>>(a);
+    }
     counted(1);
     return launch_status();
 }
@@ -298,7 +334,7 @@ Operand operand_rows(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
     const int64_t ld = round_up(t->cols, 16);
     int8_t *m = (int8_t *)ws.take((size_t)t->rows * ld);
     int8_t *e = (int8_t *)ws.take((size_t)t->rows);
-    jobs[(*njobs)++] = AlignJob{t, 1, false, m, ld, e};
+    jobs[(*njobs)++] = AlignJob{t, 1, false, m, ld, e, nullptr};
     return Operand{m, t->rows, t->cols, ld, e, 1};
 }
 // Operand whose contracted index runs along the tensor's rows: aligned per column and
@@ -306,8 +342,9 @@ Operand operand_rows(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
 Operand operand_cols(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
     const int64_t ld = round_up(t->rows, 16);
     int8_t *m = (int8_t *)ws.take((size_t)t->cols * ld);
-    int8_t *e = (int8_t *)ws.take((size_t)t->cols);
-    jobs[(*njobs)++] = AlignJob{t, 0, true, m, ld, e};
+    int8_t *e = (int8_t *)ws.take((size_t)round_up(t->cols, 16));
+    int32_t *cm = (int32_t *)ws.take((size_t)n_grp_cols(t) * 4);
+    jobs[(*njobs)++] = AlignJob{t, 0, true, m, ld, e, cm};
     return Operand{m, t->cols, t->rows, ld, e, 1};
 }
 
@@ -536,7 +573,7 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
     } else {
         int8_t *m = (int8_t *)ws.take((size_t)npix * act_c);
         int8_t *e = (int8_t *)ws.take((size_t)npix);
-        cp->jobs[cp->njobs++] = AlignJob{a, 1, false, m, act_c, e};
+        cp->jobs[cp->njobs++] = AlignJob{a, 1, false, m, act_c, e, nullptr};
         cp->a_mant = m;
         cp->eA = e;
         cp->eA_div = 1;
@@ -552,7 +589,7 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
         } else {
             int8_t *m = (int8_t *)ws.take((size_t)b->rows * b->cols);
             int8_t *e = (int8_t *)ws.take((size_t)b->rows);
-            cp->jobs[cp->njobs++] = AlignJob{b, 1, false, m, b->cols, e};
+            cp->jobs[cp->njobs++] = AlignJob{b, 1, false, m, b->cols, e, nullptr};
             cp->b_mant = m;
             cp->b_ld = b->cols;
             cp->eB = e;
@@ -821,7 +858,8 @@ int32_t ict_align(const ict_tensor *in, int32_t axis, int32_t transpose, int8_t 
     if ((st = check_vec(in))) return st;
     if (!aligned16(out_mant) || (ld_out & 15)) return ICT_ERR_ALIGNMENT;
     if (ld_out < (transpose ? round_up(in->rows, 16) : in->cols)) return ICT_ERR_INVALID_ARG;
-    return launch_align(AlignJob{in, axis, transpose != 0, out_mant, ld_out, e_star}, (cudaStream_t)stream);
+    return launch_align(AlignJob{in, axis, transpose != 0, out_mant, ld_out, e_star, nullptr},
+                        (cudaStream_t)stream);
 }
 
 size_t ict_linear_workspace(int32_t op, const ict_tensor *a, const ict_tensor *b,
@@ -974,7 +1012,26 @@ int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, 
     a.g_cols = clamp_div(H->g_cols, H->cols);
     a.ngc = n_grp_cols(H);
     const int64_t groups = H->rows * a.ngc;
-    gelu_bwd_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, (cudaStream_t)stream>>>(a);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int G = a.g_cols;
+    const bool vec = check_vec(H) == ICT_OK && check_vec(dG) == ICT_OK && check_vec(dH) == ICT_OK &&
+                     G % 16 == 0 && G <= 512 && ((G / 16) & (G / 16 - 1)) == 0;
+    if (vec) {
+        int sms = 148;
+        device_info(&sms);
+        const int L = G / 16, gpb = 8 * (32 / L);
+        const unsigned blocks = (unsigned)std::min<int64_t>(cdiv64(groups, gpb), (int64_t)sms * 8);
+        switch (L) {
+            case 1: gelu_bwd_vec_kernel<1><<<blocks, 256, 0, s>>>(a); break;
+            case 2: gelu_bwd_vec_kernel<2><<<blocks, 256, 0, s>>>(a); break;
+            case 4: gelu_bwd_vec_kernel<4><<<blocks, 256, 0, s>>>(a); break;
+            case 8: gelu_bwd_vec_kernel<8><<<blocks, 256, 0, s>>>(a); break;
+            case 16: gelu_bwd_vec_kernel<16><<<blocks, 256, 0, s>>>(a); break;
+            default: gelu_bwd_vec_kernel<32><<<blocks, 256, 0, s>>>(a); break;
+        }
+    } else {
+        gelu_bwd_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, s>>>(a);
+    }
     counted(1);
     return launch_status();
 }

@@ -40,6 +40,33 @@ __device__ __forceinline__ int need64(int64_t x, int r) {
     return x == 0 ? kNoExp : r + need_off64((uint64_t)(x < 0 ? -x : x));
 }
 
+template <int L>
+__device__ __forceinline__ int group_max(int v, unsigned mask) {
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(mask, v, o));
+    return v;
+}
+
+// RNE(x * 2^-S) for a group-uniform S with |x| < 2^30 (S < 0: exact left shift).
+struct Shift {
+    int ls, rs, bias, om;
+};
+__device__ __forceinline__ Shift make_shift(int S) {
+    Shift h;
+    h.ls = S < 0 ? -S : 0;
+    h.rs = S > 0 ? min(S, 31) : 0;
+    h.bias = h.rs ? (1 << (h.rs - 1)) - 1 : 0;
+    h.om = h.rs ? 1 : 0;
+    return h;
+}
+__device__ __forceinline__ int apply_shift(int x, const Shift &h) {
+    x <<= h.ls;
+    return (x + h.bias + ((x >> h.rs) & h.om)) >> h.rs;
+}
+
+// Exact FIT of the group values a_mul * A_i * 2^pa + b_mul * B_i * 2^pb element by element
+// in int64 (two_term: exact up to a 32-bit exponent gap, sticky beyond), for groups whose
+// values do not fit the int32 fast path.  Kept out of line: it is rare and register-hungry.
 // ------------------------------------------------------------------ requant (FIT)
 
 // FIT of int32 (optionally the int64 sum of `nsplit` int32 slices) or int64 values
@@ -101,8 +128,11 @@ struct AlignArgs {
     int axis;  // 1: per-row e*, 0: per-column e*
     int8_t *out;
     int64_t out_ld;
-    int8_t *e_star;  // [rows] (axis 1) or [cols] (axis 0)
+    int8_t *e_star;           // [rows] (axis 1) or [cols] (axis 0)
+    const int32_t *col_max;   // axis 0 with scratch: max per group column (<= kNoExp: none)
 };
+
+__device__ __forceinline__ int estar_of(int m) { return m <= kNoExp ? kEZero : m; }
 
 // e* per row: max over the row's group exponents, E_ZERO groups ignored.
 __global__ void estar_rows_kernel(AlignArgs a) {
@@ -112,10 +142,10 @@ __global__ void estar_rows_kernel(AlignArgs a) {
     int m = kNoExp;
     for (int64_t g = 0; g < a.ngc; ++g)
         if (e[g] != kEZero) m = max(m, (int)e[g]);
-    a.e_star[i] = (int8_t)(m <= kNoExp ? kEZero : m);
+    a.e_star[i] = (int8_t)estar_of(m);
 }
 
-// e* per column: one block per group column, max over all group rows.
+// e* per column without scratch: one block per group column, max over all group rows.
 __global__ void __launch_bounds__(256) estar_cols_kernel(AlignArgs a) {
     const int64_t gj = blockIdx.x;
     const int64_t ngr = (a.rows + a.g_rows - 1) / a.g_rows;
@@ -131,14 +161,39 @@ __global__ void __launch_bounds__(256) estar_cols_kernel(AlignArgs a) {
     if (threadIdx.x < 32) {
         int v = threadIdx.x < 8 ? red[threadIdx.x] : kNoExp;
         v = warp_max(v);
-        const int8_t es = (int8_t)(v <= kNoExp ? kEZero : v);
+        const int8_t es = (int8_t)estar_of(v);
         const int64_t j1 = min(a.cols, (gj + 1) * a.g_cols);
         for (int64_t j = gj * a.g_cols + threadIdx.x; j < j1; j += 32) a.e_star[j] = es;
     }
 }
 
+// e* per column with an int32 scratch (pre-set to 0x80808080): every thread keeps one
+// group column (the grid stride is a multiple of the group-column count), reduces its
+// strided slice of the exponent grid in a register, then one atomicMax in shared and
+// one in global memory.
+__global__ void __launch_bounds__(256) estar_cols_scratch_kernel(AlignArgs a, int32_t *col_max,
+                                                                 int64_t used_threads) {
+    extern __shared__ int sm[];  // [ngc]
+    for (int64_t g = threadIdx.x; g < a.ngc; g += blockDim.x) sm[g] = kNoExp;
+    __syncthreads();
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t n = ((a.rows + a.g_rows - 1) / a.g_rows) * a.ngc;
+    if (tid < used_threads) {
+        int m = kNoExp;
+        for (int64_t idx = tid; idx < n; idx += used_threads) {
+            const int e = a.in_exp[idx];
+            if (e != kEZero) m = max(m, e);
+        }
+        if (m > kNoExp) atomicMax(&sm[tid % a.ngc], m);
+    }
+    __syncthreads();
+    for (int64_t g = threadIdx.x; g < a.ngc; g += blockDim.x)
+        if (sm[g] > kNoExp) atomicMax(&col_max[g], sm[g]);
+}
+
 // Aligned mantissas, 64 x 64 tiles of 16-byte vectors (cols and, when transposed,
-// rows are multiples of 16; g_cols is a multiple of 16 or spans all columns).
+// rows are multiples of 16; g_cols is a multiple of 16 or spans all columns, so every
+// 16-byte vector has one group exponent and one target exponent).
 template <bool TRANSPOSE>
 __global__ void __launch_bounds__(256) align_tile_kernel(AlignArgs a) {
     __shared__ uint8_t tile[64][64 + 4];
@@ -146,17 +201,39 @@ __global__ void __launch_bounds__(256) align_tile_kernel(AlignArgs a) {
     const int tr = threadIdx.x >> 2, tc = (threadIdx.x & 3) * 16;
     const int64_t i = r0 + tr, j = c0 + tc;
     uint32_t w[4] = {0, 0, 0, 0};
-    if (i < a.rows && j < a.cols) {
-        const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
-        const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
-        const int eg = a.in_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+    if (j < a.cols) {
+        int es;
+        if (a.axis == 1) {
+            es = i < a.rows ? a.e_star[i] : kEZero;
+        } else if (a.col_max) {
+            es = estar_of(a.col_max[j / a.g_cols]);
+            if (blockIdx.y == 0 && tr == 0)
+                for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
+        } else {
+            es = a.e_star[j];
+        }
+        if (i < a.rows) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
+            const int eg = a.in_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+            if (eg != kEZero) {
+                const int d = min(es - eg, 8);  // |C| <= 127: shifts of 8 or more give 0
+                if (d == 0) {
+                    w[0] = raw.x, w[1] = raw.y, w[2] = raw.z, w[3] = raw.w;
+                } else {
+                    const int bias = (1 << (d - 1)) - 1;
+                    const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int b = 0; b < 16; ++b) {
-            const int es = a.axis == 1 ? a.e_star[i] : a.e_star[j + b];
-            const int c = sx8(src[b >> 2], b & 3);
-            int q = 0;
-            if (eg != kEZero && c != 0) q = es == eg ? c : rne_shr32(c, es - eg);
-            w[b >> 2] |= (uint32_t)(q & 0xff) << (8 * (b & 3));
+                    for (int q = 0; q < 4; ++q) {
+                        int r[4];
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            const int c = sx8(src[q], b);
+                            r[b] = (c + bias + ((c >> d) & 1)) >> d;
+                        }
+                        w[q] = pack4(r[0], r[1], r[2], r[3]);
+                    }
+                }
+            }
         }
     }
     if constexpr (!TRANSPOSE) {
@@ -210,6 +287,8 @@ __device__ __forceinline__ int gelu_fwd_elem(int c, int e) {
     return (c + 1) >> 1;
 }
 
+// One 16-byte vector per thread; the vector's group exponent fixes the curve's
+// thresholds and the interior rounding shift for all 16 mantissas.
 __global__ void __launch_bounds__(256) gelu_fwd_kernel(GeluArgs a) {
     const int64_t vecs_per_row = a.cols / 16;
     const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -218,11 +297,38 @@ __global__ void __launch_bounds__(256) gelu_fwd_kernel(GeluArgs a) {
     const int e = a.h_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
     const uint4 raw = *reinterpret_cast<const uint4 *>(a.h + i * a.ld_h + j);
     const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t o[4];
+    uint32_t o[4] = {0, 0, 0, 0};
+    if (e != kEZero) {
+        if (e >= 2) {  // |x| >= 4 for every nonzero C: h(x) = max(x, 0)
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-        o[q] = pack4(gelu_fwd_elem(sx8(src[q], 0), e), gelu_fwd_elem(sx8(src[q], 1), e),
-                     gelu_fwd_elem(sx8(src[q], 2), e), gelu_fwd_elem(sx8(src[q], 3), e));
+            for (int q = 0; q < 4; ++q)
+                o[q] = pack4(max(sx8(src[q], 0), 0), max(sx8(src[q], 1), 0), max(sx8(src[q], 2), 0),
+                             max(sx8(src[q], 3), 0));
+        } else {
+            const int s = 2 - e;                           // interior: RNE(C (C + T) / 2^s)
+            const int t = s - 1 >= 8 ? 256 : (1 << (s - 1));  // T = 2^(1-e); |C| < 256
+            if (s <= 24) {
+                const int T = 1 << (s - 1), bias = T - 1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    int r[4];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const int c = sx8(src[q], b);
+                        const int x = c * (c + T);
+                        const int in = (x + bias + ((x >> s) & 1)) >> s;
+                        r[b] = c <= -t ? 0 : (c >= t ? c : in);
+                    }
+                    o[q] = pack4(r[0], r[1], r[2], r[3]);
+                }
+            } else {  // C^2 / 2^s < 1/2: RNE(C / 2 + a positive tiny term) = floor((C + 1) / 2)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    o[q] = pack4((sx8(src[q], 0) + 1) >> 1, (sx8(src[q], 1) + 1) >> 1,
+                                 (sx8(src[q], 2) + 1) >> 1, (sx8(src[q], 3) + 1) >> 1);
+            }
+        }
+    }
     *reinterpret_cast<uint4 *>(a.out + i * a.ld_out + j) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -260,6 +366,139 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(GeluArgs a) {
         a.out[i * a.ld_out + j] = (int8_t)requant64(t.x, t.r, e);
     }
     if (lane == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+}
+
+// Exact GELU backward of one group element by element (int64 two-term sums), for
+// groups whose hidden exponent is so small that the int32 path would overflow.  Re-reads
+// the inputs; lane li handles elements li, li + L, ...
+template <int L>
+__device__ __noinline__ void gelu_bwd_group_exact(const GeluArgs &a, int64_t i, int64_t g, int glen,
+                                                  int li, unsigned gmask) {
+    const int64_t j0 = g * a.g_cols;
+    const int eh = a.h_exp[i * a.ngc + g], ed = a.dg_exp[i * a.ngc + g];
+    int emax = kNoExp;
+    for (int j = li; j < glen; j += L) {
+        const TwoTerm t = gelu_bwd_elem(a.h[i * a.ld_h + j0 + j], eh, a.dg[i * a.ld_dg + j0 + j], ed);
+        if (t.x) emax = max(emax, need64(t.x, t.r));
+    }
+    const int e = finalize_exp(group_max<L>(emax, gmask));
+    for (int j = li; j < glen; j += L) {
+        const TwoTerm t = gelu_bwd_elem(a.h[i * a.ld_h + j0 + j], eh, a.dg[i * a.ld_dg + j0 + j], ed);
+        a.out[i * a.ld_out + j0 + j] = (int8_t)requant64(t.x, t.r, e);
+    }
+    if (li == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+}
+
+// GELU backward, L lanes per row-local group of 16 * L elements, one 16-byte chunk of H
+// and dG per lane.  Per group: dG * h'(x) = hi * 2^(e_d - 1) + lo * 2^(e_d + e_h - 1) with
+// hi in {0, C_d, 2 C_d} and lo = C_d * C_h inside (-2, 2); at the common exponent
+// r0 = e_d - 1 - sh (sh = max(0, -e_h)) every value is hi * 2^sh + lo, exact in int32
+// while sh <= 21.
+template <int L>
+__global__ void __launch_bounds__(256) gelu_bwd_vec_kernel(const __grid_constant__ GeluArgs a) {
+    constexpr int GPW = 32 / L;
+    const int lane = threadIdx.x & 31, sub = lane / L, li = lane % L;
+    const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (sub * L));
+    const int64_t total = a.rows * a.ngc;
+    const int64_t nwarps = (int64_t)gridDim.x * 8;
+    for (int64_t base = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * GPW; base < total;
+         base += nwarps * GPW) {
+        const int64_t gw = base + sub;
+        if (gw >= total) continue;
+        const int64_t i = gw / a.ngc, g = gw % a.ngc;
+        const int64_t j0 = g * a.g_cols;
+        const int glen = (int)min((int64_t)a.g_cols, a.cols - j0);
+        const int eh = a.h_exp[gw], ed = a.dg_exp[gw];
+        const int sh = (eh < 0 && eh != kEZero) ? -eh : 0;
+        if (sh > 21) {
+            gelu_bwd_group_exact<L>(a, i, g, glen, li, gmask);
+            continue;
+        }
+        const int off = li * 16;
+        uint32_t hv[4] = {0, 0, 0, 0}, dv[4] = {0, 0, 0, 0};
+        if (off < glen) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(a.h + i * a.ld_h + j0 + off);
+            const uint4 y = *reinterpret_cast<const uint4 *>(a.dg + i * a.ld_dg + j0 + off);
+            hv[0] = x.x, hv[1] = x.y, hv[2] = x.z, hv[3] = x.w;
+            dv[0] = y.x, dv[1] = y.y, dv[2] = y.z, dv[3] = y.w;
+            const int rem = glen - off;
+            if (rem < 16)
+                for (int b = rem; b < 16; ++b) dv[b >> 2] &= ~(0xffu << (8 * (b & 3)));
+        }
+        // |C_h| < T is the interior; e_h >= 1 (or E_ZERO) leaves only C_h = 0 inside
+        const int T = (eh >= 1 || eh == kEZero) ? 1 : (1 - eh >= 8 ? 256 : (1 << (1 - eh)));
+        int xv[16];
+        int amax = 0;
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            const int ch = sx8(hv[b >> 2], b & 3), cd = sx8(dv[b >> 2], b & 3);
+            const bool inside = ch > -T && ch < T;
+            const int hi = ch <= -T ? 0 : (inside ? cd : 2 * cd);
+            const int x = (hi << sh) + (inside ? cd * ch : 0);
+            xv[b] = x;
+            amax = max(amax, abs(x));
+        }
+        amax = group_max<L>(amax, gmask);
+        const int r0 = ed - 1 - sh;
+        const int e = finalize_exp(amax ? r0 + need_off32((uint32_t)amax) : kNoExp);
+        const Shift h = make_shift(e == kEZero ? 0 : e - r0);
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            o[q] = pack4(apply_shift(xv[4 * q], h), apply_shift(xv[4 * q + 1], h), apply_shift(xv[4 * q + 2], h),
+                         apply_shift(xv[4 * q + 3], h));
+        if (off < glen) {
+            int8_t *dst = a.out + i * a.ld_out + j0 + off;
+            if (glen - off >= 16) {
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+            } else {
+                for (int b = 0; b < glen - off; ++b) dst[b] = (int8_t)(o[b >> 2] >> (8 * (b & 3)));
+            }
+        }
+        if (li == 0) a.out_exp[gw] = (int8_t)e;
+    }
+}
+
+// ------------------------------------------------------------------ requant, wide groups
+
+// FIT of row-local groups wider than a warp can hold: one block of T threads per group,
+// EPT elements per thread kept in registers between the max and the rounding pass.
+template <int T, int EPT>
+__global__ void __launch_bounds__(T) requant_group_block_kernel(RequantArgs a) {
+    const int64_t gidx = blockIdx.x;
+    const int64_t i = gidx / a.ngc, g = gidx % a.ngc;
+    const int64_t j0 = g * a.G;
+    const int glen = (int)min((int64_t)a.G, a.cols - j0);
+    const int re = a.base + (a.row_exp ? a.row_exp[i / a.row_div] : 0);
+    int64_t x[EPT];
+    int r[EPT];
+    int emax = kNoExp;
+#pragma unroll
+    for (int k = 0; k < EPT; ++k) {
+        const int jj = threadIdx.x + k * T;
+        x[k] = 0;
+        r[k] = re;
+        if (jj < glen) {
+            const int64_t j = j0 + jj;
+            x[k] = rq_value(a, i, j);
+            r[k] = re + (a.col_exp ? a.col_exp[j / a.col_div] : 0);
+            if (x[k]) emax = max(emax, need64(x[k], r[k]));
+        }
+    }
+    __shared__ int red[T / 32];
+    emax = warp_max(emax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = emax;
+    __syncthreads();
+    int m = red[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) m = max(m, red[w]);
+    const int e = finalize_exp(m);
+#pragma unroll
+    for (int k = 0; k < EPT; ++k) {
+        const int jj = threadIdx.x + k * T;
+        if (jj < glen) a.out[i * a.out_ld + j0 + jj] = (int8_t)requant64(x[k], r[k], e);
+    }
+    if (threadIdx.x == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
 }
 
 // ------------------------------------------------------------------ integer SGD
@@ -324,13 +563,6 @@ __device__ __forceinline__ void sgd_group(const SgdArgs &p, const SgdTensor &t, 
 
 // ---- vectorised SGD: L lanes per group, each lane holds CPL 16-byte chunks of W, V, G.
 
-template <int L>
-__device__ __forceinline__ int group_max(int v, unsigned mask) {
-#pragma unroll
-    for (int o = L / 2; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(mask, v, o));
-    return v;
-}
-
 // Locates global group `gw` in the tensor list.
 __device__ __forceinline__ int sgd_find(const SgdArgs &p, int64_t gw) {
     int lo = 0, hi = p.n - 1;
@@ -365,26 +597,6 @@ __device__ __forceinline__ GroupSum group_sum(int pa, bool za, int64_t amax, int
     return g;
 }
 
-// RNE(x * 2^-S) for a group-uniform S with |x| < 2^30 (S < 0: exact left shift).
-struct Shift {
-    int ls, rs, bias, om;
-};
-__device__ __forceinline__ Shift make_shift(int S) {
-    Shift h;
-    h.ls = S < 0 ? -S : 0;
-    h.rs = S > 0 ? min(S, 31) : 0;
-    h.bias = h.rs ? (1 << (h.rs - 1)) - 1 : 0;
-    h.om = h.rs ? 1 : 0;
-    return h;
-}
-__device__ __forceinline__ int apply_shift(int x, const Shift &h) {
-    x <<= h.ls;
-    return (x + h.bias + ((x >> h.rs) & h.om)) >> h.rs;
-}
-
-// Exact FIT of the group values a_mul * A_i * 2^pa + b_mul * B_i * 2^pb element by element
-// in int64 (two_term: exact up to a 32-bit exponent gap, sticky beyond), for groups whose
-// values do not fit the int32 fast path.  Kept out of line: it is rare and register-hungry.
 // Exact SGD update of one group, element by element in int64 (two_term: exact up to a
 // 32-bit exponent gap, sticky beyond), for groups whose values do not fit the int32 fast
 // path.  Reads W, V, G from memory again and writes the results; each lane handles the
