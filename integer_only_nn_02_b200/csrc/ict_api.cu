@@ -247,8 +247,9 @@ int launch_zero(const ict_tensor *out, cudaStream_t s) {
 // ---- tensor-core Product
 
 constexpr int stages_for(int bn, int bk) {
-    return bk == 128 ? (bn <= 64 ? 8 : bn <= 128 ? 6 : bn <= 192 ? 5 : 4)
-                     : (bn <= 64 ? 12 : bn <= 128 ? 10 : 8);
+    return bk == 256 ? 4
+           : bk == 128 ? (bn <= 64 ? 8 : bn <= 128 ? 6 : bn <= 192 ? 5 : 4)
+                       : (bn <= 64 ? 12 : bn <= 128 ? 10 : 8);
 }
 
 template <int BN, int BK, int LOAD>
@@ -277,6 +278,7 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     ICT_GEMM_CASE(128, 64, LOAD_CONV)
     ICT_GEMM_CASE(192, 64, LOAD_CONV)
     ICT_GEMM_CASE(256, 64, LOAD_CONV)
+    ICT_GEMM_CASE(64, 256, LOAD_CONV_WGRAD)
 #undef ICT_GEMM_CASE
     return ICT_ERR_LAYOUT;
 }
@@ -429,6 +431,7 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     a.rows = M;
     a.cols = N;
     a.ld = pl.ws_ld;
+    a.cs = 1;
     a.row_exp = A.exp;
     a.row_div = A.exp_div;
     a.col_exp = B.exp;
@@ -545,7 +548,6 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
     if (d->stride != 1 || d->r != d->s || 2 * d->pad != d->r - 1) return ICT_ERR_LAYOUT;
     if (d->c % 64 || d->k % 64 || d->c > 256 || d->k > 256 || d->w > 128) return ICT_ERR_LAYOUT;
     const int64_t npix = (int64_t)d->n * d->h * d->w, RS = (int64_t)d->r * d->s;
-    if (dir == ICT_CONV_BWD_WEIGHT) return ICT_ERR_LAYOUT;
     if (dir != ICT_CONV_FWD && dir != ICT_CONV_BWD_DATA) return ICT_ERR_INVALID_ARG;
     const int64_t act_c = dir == ICT_CONV_FWD ? d->c : d->k;  // contracted channels
     const int64_t out_c = dir == ICT_CONV_FWD ? d->k : d->c;
@@ -684,6 +686,120 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s))) return st;
     p.epi = EPI_FIT_GLOBAL;
     return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s);
+}
+
+// ---- convolution backward-weight: dW[k][(r,s,c)] = sum over output pixels of
+// dY[pix][k] * X[pix shifted by (r,s)][c], both NHWC operands read MN-major by TMA
+
+struct WgradPlan {
+    int hrows, hblk, kpix, atoms, mtiles, ntiles, splits, kblk_per_split, n_kblk, units;
+    int64_t M, N, ws_ld;
+    int32_t *partial;
+    int8_t *e_rows, *e_cols;
+};
+
+int plan_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X, const ict_tensor *dW,
+               int sms, Ws &ws, WgradPlan *wp) {
+    int st;
+    if ((st = check_tensor(dY)) || (st = check_tensor(X)) || (st = check_tensor(dW))) return st;
+    if (d->stride != 1 || d->r != d->s || 2 * d->pad != d->r - 1) return ICT_ERR_LAYOUT;
+    if (d->c % 64 || d->k % 64 || d->w > 256) return ICT_ERR_LAYOUT;
+    const int64_t npix = (int64_t)d->n * d->h * d->w, RS = (int64_t)d->r * d->s;
+    if (dY->rows != npix || dY->cols != d->k || X->rows != npix || X->cols != d->c) return ICT_ERR_INVALID_ARG;
+    if (dW->rows != d->k || dW->cols != RS * d->c) return ICT_ERR_INVALID_ARG;
+    if (dY->g_rows < dY->rows || X->g_rows < X->rows) return ICT_ERR_LAYOUT;  // uniform over pixels
+    if (dY->ld != d->k || X->ld != d->c) return ICT_ERR_LAYOUT;                // dense NHWC
+    if (dW->g_rows != 1 && dW->rows > 1) return ICT_ERR_LAYOUT;
+    if ((st = check_vec(dY)) || (st = check_vec(X)) || (st = check_vec(dW))) return st;
+    // K block: whole image rows, a multiple of 32 pixels, at most 256
+    wp->hrows = 0;
+    for (int h = 1; d->w * h <= 256; ++h)  // rows past the image end are zero-filled
+        if ((d->w * h) % 32 == 0) { wp->hrows = h; break; }
+    if (!wp->hrows) return ICT_ERR_LAYOUT;
+    wp->kpix = d->w * wp->hrows;
+    wp->hblk = (int)cdiv64(d->h, wp->hrows);
+    wp->n_kblk = d->n * wp->hblk;
+    wp->atoms = (int)(RS * d->c / 64);
+    wp->mtiles = (wp->atoms + 1) / 2;
+    wp->ntiles = d->k / 64;
+    const int tiles = wp->mtiles * wp->ntiles;
+    int splits = std::max(1, std::min(sms / tiles, wp->n_kblk / 4));
+    // int32 partials stay exact: pixels per slice times 127^2 below 2^31
+    const int max_kblk = std::max(1, (int)(((1ll << 31) - 1) / (16129ll * wp->kpix)));
+    if (cdiv64(wp->n_kblk, splits) > max_kblk) splits = (int)cdiv64(wp->n_kblk, max_kblk);
+    wp->kblk_per_split = (int)cdiv64(wp->n_kblk, splits);
+    wp->splits = (int)cdiv64(wp->n_kblk, wp->kblk_per_split);
+    wp->units = tiles * wp->splits;
+    wp->M = RS * d->c;
+    wp->N = d->k;
+    wp->ws_ld = round_up(wp->N, 32);
+    wp->partial = (int32_t *)ws.take((size_t)wp->splits * wp->M * wp->ws_ld * 4);
+    wp->e_rows = (int8_t *)ws.take((size_t)wp->M);
+    wp->e_cols = (int8_t *)ws.take((size_t)wp->N);
+    return ICT_OK;
+}
+
+int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X, const ict_tensor *dW,
+              const WgradPlan &wp, int sms, cudaStream_t s) {
+    int st;
+    const int RS = d->r * d->s;
+    conv_wgrad_exp_kernel<<<(unsigned)cdiv64(std::max<int64_t>(wp.M, wp.N), 256), 256, 0, s>>>(
+        X->exp, clamp_div(X->g_cols, X->cols), dY->exp, clamp_div(dY->g_cols, dY->cols), d->c, RS, d->k,
+        wp.e_rows, wp.e_cols);
+    counted(1);
+    if ((st = launch_status())) return st;
+    CUtensorMap ta, tb;
+    if ((st = tmap_nhwc(&ta, X->mant, d->n, d->h, d->w, d->c, wp.hrows))) return st;
+    if ((st = tmap_nhwc(&tb, dY->mant, d->n, d->h, d->w, d->k, wp.hrows))) return st;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = (int)wp.M;
+    p.N = (int)wp.N;
+    p.n_kblk = wp.n_kblk;
+    p.n_mtiles = wp.mtiles;
+    p.n_ntiles = wp.ntiles;
+    p.splits = wp.splits;
+    p.kblk_per_split = wp.kblk_per_split;
+    p.num_units = wp.units;
+    p.eA = wp.e_rows;
+    p.eA_div = 1;
+    p.eB = wp.e_cols;
+    p.eB_div = 1;
+    p.G = (int)wp.N;
+    p.ws32 = wp.partial;
+    p.ws_ld = wp.ws_ld;
+    p.ws_split_stride = wp.M * wp.ws_ld;
+    p.cv_cblk = d->c / 64;
+    p.cv_S = d->s;
+    p.cv_pad = d->pad;
+    p.wg_hrows = wp.hrows;
+    p.wg_hblk = wp.hblk;
+    p.wg_kpix = wp.kpix;
+    p.wg_atoms = wp.atoms;
+    p.wait_ns = g_wait_ns;
+    p.drain_ns = kDrainNs;
+    p.epi = EPI_I32;
+    if ((st = launch_gemm(64, 256, LOAD_CONV_WGRAD, ta, tb, p, std::min(wp.units, sms), s))) return st;
+    // dW[k][j] = sum over slices of partial[j][k]: FIT per row k, exponent e_cols[k] + e_rows[j]
+    RequantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.v32 = wp.partial;
+    a.nsplit = wp.splits;
+    a.split_stride = wp.M * wp.ws_ld;
+    a.rows = wp.N;
+    a.cols = wp.M;
+    a.ld = 1;
+    a.cs = wp.ws_ld;
+    a.row_exp = wp.e_cols;
+    a.row_div = 1;
+    a.col_exp = wp.e_rows;
+    a.col_div = 1;
+    a.out = dW->mant;
+    a.out_ld = dW->ld;
+    a.out_exp = dW->exp;
+    a.G = clamp_div(dW->g_cols, dW->cols);
+    a.ngc = n_grp_cols(dW);
+    return launch_requant_rows(a, s);
 }
 
 // ---- SGD
@@ -836,6 +952,7 @@ int32_t ict_requant(const void *vals, int32_t val_bits, int64_t rows, int64_t co
     a.rows = rows;
     a.cols = cols;
     a.ld = ld_vals;
+    a.cs = 1;
     a.base = base_exp;
     a.row_exp = row_exp;
     a.row_div = 1;
@@ -898,6 +1015,20 @@ int32_t ict_linear_bwd_weight(const ict_tensor *dY, const ict_tensor *X, ict_ten
 size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d) {
     if (!d || d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1 || d->k < 1 || d->r < 1 || d->s < 1)
         return 0;
+    if (dir == ICT_CONV_BWD_WEIGHT) {
+        // the plan's own sizes: int32 partial slices and the exponent tables
+        ict_tensor dY{nullptr, nullptr, (int64_t)d->n * d->h * d->w, d->k, d->k, INT32_MAX, 32};
+        ict_tensor X{nullptr, nullptr, (int64_t)d->n * d->h * d->w, d->c, d->c, INT32_MAX, 32};
+        ict_tensor dW{nullptr, nullptr, d->k, (int64_t)d->r * d->s * d->c, (int64_t)d->r * d->s * d->c, 1,
+                      d->r * d->s * d->c};
+        static int8_t dummy[16] __attribute__((aligned(16)));
+        dY.mant = X.mant = dW.mant = dummy;
+        dY.exp = X.exp = dW.exp = dummy;
+        WgradPlan wp;
+        Ws w = make_ws(nullptr, 0, true);
+        if (plan_wgrad(d, &dY, &X, &dW, planning_sms(), w, &wp) != ICT_OK) return 0;
+        return w.used;
+    }
     // worst case: activation aligned copy + its exponents, the prepared weight, gmax
     const int64_t npix = (int64_t)d->n * d->h * d->w;
     const int64_t act_c = dir == ICT_CONV_FWD ? d->c : d->k;
@@ -917,8 +1048,15 @@ int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_te
     int st, sms = 0;
     if ((st = device_info(&sms))) return st;
     if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
-    ConvPlan cp;
     Ws w = make_ws(ws, ws_bytes, false);
+    if (dir == ICT_CONV_BWD_WEIGHT) {
+        if (!d) return ICT_ERR_INVALID_ARG;
+        WgradPlan wp;
+        if ((st = plan_wgrad(d, a, b, out, sms, w, &wp))) return st;
+        if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
+        return run_wgrad(d, a, b, out, wp, sms, (cudaStream_t)stream);
+    }
+    ConvPlan cp;
     if ((st = plan_conv(dir, d, a, b, out, w, &cp))) return st;
     if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
     return run_conv(dir, d, out, cp, sms, (cudaStream_t)stream);

@@ -77,7 +77,8 @@ struct RequantArgs {
     const int64_t *v64;
     int nsplit;
     int64_t split_stride;
-    int64_t rows, cols, ld;
+    int64_t rows, cols, ld;  // value (i, j) at v[i * ld + j * cs] (cs = 1 unless transposed)
+    int64_t cs;
     int32_t base;
     const int8_t *row_exp;  // exponent of row i: row_exp[i / row_div] (NULL = 0)
     int row_div;
@@ -91,9 +92,10 @@ struct RequantArgs {
 };
 
 __device__ __forceinline__ int64_t rq_value(const RequantArgs &a, int64_t i, int64_t j) {
-    if (a.v64) return a.v64[i * a.ld + j];
+    const int64_t at = i * a.ld + j * a.cs;
+    if (a.v64) return a.v64[at];
     int64_t s = 0;
-    for (int k = 0; k < a.nsplit; ++k) s += a.v32[k * a.split_stride + i * a.ld + j];
+    for (int k = 0; k < a.nsplit; ++k) s += a.v32[k * a.split_stride + at];
     return s;
 }
 
@@ -835,6 +837,15 @@ __global__ void __launch_bounds__(256) conv_wt_prep_kernel(ConvWeightArgs a) {
     int q = 0;
     if (e != kEZero && v != 0) q = es == e ? v : rne_shr32(v, es - e);
     a.out[c * a.out_ld + rem] = (int8_t)q;
+}
+
+// Exponent tables of a convolution's backward-weight Product: row m = tap * C + c of the
+// MMA output takes X's exponent of channel c, column k takes dY's exponent of channel k.
+__global__ void conv_wgrad_exp_kernel(const int8_t *x_exp, int gx, const int8_t *y_exp, int gy, int C,
+                                      int RS, int K, int8_t *e_rows, int8_t *e_cols) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < RS * C) e_rows[i] = x_exp[(i % C) / gx];
+    if (i < K) e_cols[i] = y_exp[i / gy];
 }
 
 __global__ void fill_i32_kernel(int32_t *p, int n, int32_t v) {

@@ -37,7 +37,13 @@ enum EpiMode : int {
     EPI_NEED_GLOBAL = 2,  // pass 1 of groups spanning all rows: max need per column group
     EPI_FIT_GLOBAL = 3,   // pass 2: requantise with the global group exponents
 };
-enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1 };
+// LOAD_2D         A, B: K-major rows from 2-D tensor maps (linear layers)
+// LOAD_CONV       A: one filter tap of NHWC activations per K block (4-D box), B: K-major
+//                 weight rows (convolution forward / backward-data)
+// LOAD_CONV_WGRAD A: two (tap, 64-channel) slices of the shifted NHWC input X, B: 64
+//                 channels of dY, both MN-major with output pixels as K (convolution
+//                 backward-weight); BK is the largest number of pixels per K block
+enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1, LOAD_CONV_WGRAD = 2 };
 
 struct GemmParams {
     int M, N;       // output rows (MMA M side) and columns (MMA N side)
@@ -58,6 +64,9 @@ struct GemmParams {
     int32_t *gmax;  // [column groups] running max of need() (global groups)
     // implicit-GEMM convolution: output tile = cv_rows image rows of width cv_W
     int cv_W, cv_P, cv_rows, cv_tiles_per_img, cv_cblk, cv_S, cv_pad, cv_sign;
+    // backward-weight: K block = wg_hrows image rows of every image (wg_kpix pixels), M rows
+    // (tap, channel) in 64-row atoms (wg_atoms in total)
+    int wg_hrows, wg_hblk, wg_kpix, wg_atoms;
     uint32_t stage_tx_bytes;
     uint64_t wait_ns, drain_ns;
     int epi;
@@ -77,7 +86,7 @@ struct GemmSmem {
     static constexpr int kBytes = kOffCol + 2 * kColInts * 4 + 1024;  // + alignment slack
     static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
                   "column tables are read as int4");
-    static_assert(kABytes % 1024 == 0 && kBBytes % 512 == 0 && kOffB % 1024 == 0,
+    static_assert(kABytes % 1024 == 0 && kBBytes % 512 == 0 && kOffB % 1024 == 0 && kABytes / 2 <= 16383 * 16,
                   "operand tiles must sit on their swizzle-atom boundaries");
     static_assert(kBytes <= 232448, "shared memory per block");
 };
@@ -92,7 +101,7 @@ __global__ void __launch_bounds__(384, 1)
                    const __grid_constant__ GemmParams p) {
     using L = GemmSmem<BN, BK, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
-    static_assert(BK == 128 || BK == 64, "BK");
+    static_assert(BK == 128 || BK == 64 || (BK == 256 && LOAD == LOAD_CONV_WGRAD), "BK");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
@@ -162,18 +171,32 @@ __global__ void __launch_bounds__(384, 1)
                         break;
                     }
                     const uint32_t fb = bar_full + 8 * stage;
-                    mbar_expect_tx(fb, p.stage_tx_bytes);
                     const uint32_t sa = sbase + stage * L::kABytes;
                     const uint32_t sb = sbase + L::kOffB + stage * L::kBBytes;
                     if (LOAD == LOAD_2D) {
+                        mbar_expect_tx(fb, p.stage_tx_bytes);
                         tma_load_2d(sa, &tmA, fb, kb * BK, mt * 128);
-                    } else {
+                        tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
+                    } else if (LOAD == LOAD_CONV) {
+                        mbar_expect_tx(fb, p.stage_tx_bytes);
                         const int tap = kb / p.cv_cblk, cb = kb % p.cv_cblk;
                         const int r = tap / p.cv_S, s = tap % p.cv_S;
                         tma_load_4d(sa, &tmA, fb, cb * 64, p.cv_sign * (s - p.cv_pad),
                                     h0 + p.cv_sign * (r - p.cv_pad), img);
+                        tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
+                    } else {
+                        // pixels of this K block: rows h1 .. h1 + hrows - 1 of image img1
+                        const int img1 = kb / p.wg_hblk, h1 = (kb % p.wg_hblk) * p.wg_hrows;
+                        const int a0 = 2 * mt, na = a0 + 1 < p.wg_atoms ? 2 : 1;
+                        mbar_expect_tx(fb, (uint32_t)((na + 1) * p.wg_kpix * 64));
+                        for (int q = 0; q < na; ++q) {
+                            const int tap = (a0 + q) / p.cv_cblk, cb = (a0 + q) % p.cv_cblk;
+                            const int r = tap / p.cv_S, s = tap % p.cv_S;
+                            tma_load_4d(sa + q * (L::kABytes / 2), &tmA, fb, cb * 64, s - p.cv_pad,
+                                        h1 + r - p.cv_pad, img1);
+                        }
+                        tma_load_4d(sb, &tmB, fb, nt * 64, 0, h1, img1);
                     }
-                    tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
                     issued[stage] = 1;
                     issued_phase[stage] = phase;
                     if (++stage == STAGES) stage = 0, phase ^= 1;
@@ -186,7 +209,9 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t kIdesc = idesc_i8(128, BN);
+            constexpr bool kMN = LOAD == LOAD_CONV_WGRAD;  // both operands MN-major
+            constexpr uint32_t kIdesc = idesc_i8(128, BN, kMN, kMN);
+            const int kk_per_blk = kMN ? p.wg_kpix / 32 : BK / 32;
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -210,11 +235,19 @@ __global__ void __launch_bounds__(384, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t da = smem_desc_kmajor(sbase + stage * L::kABytes, BK);
-                    const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + stage * L::kBBytes, BK);
+                    if constexpr (kMN) {
+                        // 32 pixels per MMA = four 8-row atoms of 64 bytes = 2048 bytes
+                        const uint64_t da = smem_desc_mnmajor64(sbase + stage * L::kABytes, L::kABytes / 2);
+                        const uint64_t db = smem_desc_mnmajor64(sbase + L::kOffB + stage * L::kBBytes, L::kABytes / 2);
+                        for (int kk = 0; kk < kk_per_blk; ++kk)
+                            umma_i8(tmem_d, da + 128 * kk, db + 128 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        const uint64_t da = smem_desc_kmajor(sbase + stage * L::kABytes, BK);
+                        const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + stage * L::kBBytes, BK);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 32; ++kk)
-                        umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 32; ++kk)
+                            umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                    }
                     any = true;
                     umma_commit(bar_empty + 8 * stage);
                     if (++stage == STAGES) stage = 0, phase ^= 1;

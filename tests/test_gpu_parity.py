@@ -169,6 +169,11 @@ def test_conv_fwd_and_bwd_data(ict, shape, global_groups):
         ref = oracle.conv(direction, d, a, b, g_rows, 32)
         got = ict.conv(direction, d, ict.DevCE.from_host(a), ict.DevCE.from_host(b), g_rows, 32).to_host()
         same(got, ref, f"conv dir={direction} {shape} global={global_groups}")
+    # backward-weight: dW rows of r*s*c, per-row groups (or 64-wide groups)
+    g = 9 * d["c"] if global_groups else 64
+    ref = oracle.conv(ict.CONV_BWD_WEIGHT, d, dY, X, 1, g)
+    got = ict.conv(ict.CONV_BWD_WEIGHT, d, ict.DevCE.from_host(dY), ict.DevCE.from_host(X), 1, g).to_host()
+    same(got, ref, f"conv bwd-weight {shape} g={g}")
     status_ok(ict)
 
 
