@@ -221,7 +221,8 @@ int launch_requant_rows(RequantArgs a, cudaStream_t s) {
     if (G >= 128 && G <= 4096) {
         const int T = G >= 256 ? 256 : 128;
         const int ept = (G + T - 1) / T;
-        if (T == 128) launch_requant_block<128, 1>(a, groups, s);
+        if (T == 128 && ept <= 1) launch_requant_block<128, 1>(a, groups, s);
+        else if (T == 128) launch_requant_block<128, 2>(a, groups, s);
         else if (ept <= 1) launch_requant_block<256, 1>(a, groups, s);
         else if (ept <= 2) launch_requant_block<256, 2>(a, groups, s);
         else if (ept <= 4) launch_requant_block<256, 4>(a, groups, s);
@@ -838,9 +839,18 @@ template <int L, int CPL>
 int launch_sgd_vec(const SgdArgs &a, int sms, cudaStream_t s) {
     constexpr int gpb = 8 * (32 / L);  // groups per block and pass
     const int64_t blocks = std::min<int64_t>(cdiv64(a.total_groups, gpb), (int64_t)sms * 8);
-    sgd_vec_kernel<L, CPL><<<(unsigned)blocks, 256, 0, s>>>(a);
+    if (a.n == 1)
+        sgd_vec_kernel<L, CPL, true><<<(unsigned)blocks, 256, 0, s>>>(a);
+    else
+        sgd_vec_kernel<L, CPL, false><<<(unsigned)blocks, 256, 0, s>>>(a);
     counted(1);
     return launch_status();
+}
+
+int bitlen_u64(uint64_t v) {
+    int b = 0;
+    while (v >> b) ++b;
+    return b;
 }
 
 // Vectorised kernel when every tensor shares one group width G (a multiple of 16, at
@@ -853,6 +863,29 @@ int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
         vec = vec && a.t[i].G == G && (a.t[i].ld & 15) == 0 && aligned16(a.t[i].w) && aligned16(a.t[i].v) &&
               aligned16(a.t[i].g);
     vec = vec && G % 16 == 0 && G <= 2048;
+    // one dense tensor, one group per row of 16 * L elements: the prefetching kernel
+    const SgdTensor &t0 = a.t[0];
+    const int Lr = G / 16;
+    if (vec && a.n == 1 && t0.ngc == 1 && t0.cols == t0.G && t0.ld == t0.G && Lr >= 1 && Lr <= 32 &&
+        (Lr & (Lr - 1)) == 0) {
+        const int L = Lr;
+        const int64_t gpb = 8 * (32 / L);
+        const unsigned blocks = (unsigned)std::min<int64_t>(cdiv64(a.total_groups, gpb), (int64_t)sms * 8);
+        bool done = true;
+        switch (L) {
+            case 1: sgd_rows_kernel<1><<<blocks, 256, 0, s>>>(a); break;
+            case 2: sgd_rows_kernel<2><<<blocks, 256, 0, s>>>(a); break;
+            case 4: sgd_rows_kernel<4><<<blocks, 256, 0, s>>>(a); break;
+            case 8: sgd_rows_kernel<8><<<blocks, 256, 0, s>>>(a); break;
+            case 16: sgd_rows_kernel<16><<<blocks, 256, 0, s>>>(a); break;
+            case 32: sgd_rows_kernel<32><<<blocks, 256, 0, s>>>(a); break;
+            default: done = false;
+        }
+        if (done) {
+            counted(1);
+            return launch_status();
+        }
+    }
     if (vec) {
         const int chunks = G / 16;
         if (chunks <= 1) return launch_sgd_vec<1, 1>(a, sms, s);
@@ -1083,6 +1116,8 @@ int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W, ict
     a.mom_shift = p->mom_shift;
     a.lr_mul = p->lr_mul;
     a.lr_shift = p->lr_shift;
+    a.cap_mom = 29 - bitlen_u64(127ull * (uint64_t)std::abs(p->mom_mul));
+    a.cap_lr = 29 - bitlen_u64(127ull * (uint64_t)std::abs(p->lr_mul));
     int64_t total = 0;
     for (int i = 0; i < n_tensors; ++i) {
         if ((st = fill_sgd_tensor(W[i], V[i], G[i], &a.t[i]))) return st;

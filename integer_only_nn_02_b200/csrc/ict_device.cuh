@@ -59,6 +59,13 @@ __device__ __forceinline__ int64_t rne_shr64(int64_t x, int s) {
     return q + ((rem > half) || (rem == half && (q & 1)));
 }
 
+// bits [pos, pos + len) of x (len 0 gives 0)
+__device__ __forceinline__ uint32_t bfe_u32(uint32_t x, uint32_t pos, uint32_t len) {
+    uint32_t r;
+    asm("bfe.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(pos), "r"(len));
+    return r;
+}
+
 __device__ __forceinline__ int sat127(int64_t q) {
     return q > 127 ? 127 : (q < -127 ? -127 : (int)q);
 }
@@ -91,8 +98,14 @@ __device__ __forceinline__ int finalize_exp(int emax) {
     return emax;
 }
 
-__device__ __forceinline__ int sx8(uint32_t w, int byte) {  // sign-extended byte of a word
-    return (int)(int8_t)(w >> (8 * byte));
+// sign-extended byte of a word: one prmt whose upper three selectors replicate the sign
+// bit of the selected byte (PTX prmt, default mode: selector msb = sign replicate)
+__device__ __forceinline__ int sx8(uint32_t w, int byte) {
+    const uint32_t sel = (uint32_t)byte | ((uint32_t)(byte | 8) << 4) | ((uint32_t)(byte | 8) << 8) |
+                         ((uint32_t)(byte | 8) << 12);
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));
+    return (int)r;
 }
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |

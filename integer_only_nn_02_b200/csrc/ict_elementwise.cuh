@@ -520,6 +520,9 @@ struct SgdArgs {
     int n;
     int64_t total_groups;
     int mom_mul, mom_shift, lr_mul, lr_shift;
+    // largest shift of each term at which |term| stays below 2^29 (so every two-term sum
+    // is below 2^30): 29 - bitlen(127 |multiplier|)
+    int cap_mom, cap_lr;
     SgdTensor t[kSgdMaxTensors];
 };
 
@@ -576,29 +579,6 @@ __device__ __forceinline__ int sgd_find(const SgdArgs &p, int64_t gw) {
     return lo;
 }
 
-// Two terms a_i * 2^pa + b_i * 2^pb of one group at the common exponent r0 = min(pa, pb):
-// x_i = a_i * ma + b_i * mb with ma = 2^(pa - r0), mb = 2^(pb - r0).  An exponent whose
-// term is absent (E_ZERO, all mantissas zero) takes the other one's value.
-struct GroupSum {
-    int r0;
-    int64_t ma, mb;
-    bool small;  // every |x_i| < 2^30 (int32 arithmetic is exact)
-    bool exact;  // exponents at most 32 apart (int64 arithmetic is exact)
-};
-__device__ __forceinline__ GroupSum group_sum(int pa, bool za, int64_t amax, int pb, bool zb, int64_t bmax) {
-    GroupSum g;
-    if (za && zb) za = false, pa = pb = 0;
-    if (za) pa = pb;
-    if (zb) pb = pa;
-    g.r0 = min(pa, pb);
-    const int da = pa - g.r0, db = pb - g.r0;
-    g.exact = da <= 32 && db <= 32;
-    g.ma = g.exact ? (1ll << da) : 0;
-    g.mb = g.exact ? (1ll << db) : 0;
-    g.small = g.exact && (amax << da) + (bmax << db) < (1ll << 30);
-    return g;
-}
-
 // Exact SGD update of one group, element by element in int64 (two_term: exact up to a
 // 32-bit exponent gap, sticky beyond), for groups whose values do not fit the int32 fast
 // path.  Reads W, V, G from memory again and writes the results; each lane handles the
@@ -637,33 +617,71 @@ __device__ __noinline__ void sgd_group_exact(const SgdArgs &p, const SgdTensor &
     }
 }
 
-template <int L, int CPL>
+// Common exponent of two group terms a * 2^pa + b * 2^pb: r0 = min(pa, pb), shifts sa, sb;
+// an absent term (E_ZERO, all mantissas zero) takes the other's exponent.  `small` when
+// both shifted terms stay below 2^29 (int32 sums are exact and leave room for rounding).
+__device__ __forceinline__ void common_exp(int pa, bool za, int pb, bool zb, int cap_a, int cap_b, int &r0,
+                                           int &sa, int &sb, bool &small) {
+    if (za) pa = pb;
+    if (zb) pb = pa;
+    r0 = min(pa, pb);
+    sa = pa - r0;
+    sb = pb - r0;
+    small = sa <= cap_a && sb <= cap_b;
+}
+
+template <int L, int CPL, bool SINGLE>
 __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ SgdArgs p) {
     constexpr int GPW = 32 / L;  // groups per warp and pass
     const int lane = threadIdx.x & 31, sub = lane / L, li = lane % L;
     const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (sub * L));
     const int64_t nwarps = (int64_t)gridDim.x * 8;
+    // a single tensor's fields live in registers for the whole kernel
+    const SgdTensor &t0 = p.t[0];
+    int8_t *const w0 = t0.w, *const v0 = t0.v, *const we0 = t0.w_exp, *const ve0 = t0.v_exp;
+    const int8_t *const g0 = t0.g, *const ge0 = t0.g_exp;
+    const int64_t ld0 = t0.ld, cols0 = t0.cols, ngc0 = t0.ngc;
+    const int G0 = t0.G;
     for (int64_t base = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * GPW; base < p.total_groups;
          base += nwarps * GPW) {
         const int64_t gw = base + sub;
         if (gw >= p.total_groups) continue;  // whole groups only: lanes of a group agree
-        const SgdTensor &t = p.t[sgd_find(p, gw)];
-        const int64_t local = gw - t.first_group;
-        const int64_t i = local / t.ngc, gi = local % t.ngc;
-        const int64_t ge = i * t.ngc + gi;
-        const int64_t j0 = gi * t.G;
-        const int glen = (int)min((int64_t)t.G, t.cols - j0);
-        const int ev = t.v_exp[ge], eg = t.g_exp[ge], ew = t.w_exp[ge];
+        int8_t *tw, *tv, *twe, *tve;
+        const int8_t *tg, *tge;
+        int64_t tld, tcols, tngc, local;
+        int tG;
+        if (SINGLE) {
+            tw = w0, tv = v0, twe = we0, tve = ve0, tg = g0, tge = ge0;
+            tld = ld0, tcols = cols0, tngc = ngc0, tG = G0, local = gw;
+        } else {
+            const SgdTensor &t = p.t[sgd_find(p, gw)];
+            tw = t.w, tv = t.v, twe = t.w_exp, tve = t.v_exp, tg = t.g, tge = t.g_exp;
+            tld = t.ld, tcols = t.cols, tngc = t.ngc, tG = t.G, local = gw - t.first_group;
+        }
+        // group (row i, column group gi); one column group per row needs no division
+        int64_t i, gi;
+        if (tngc == 1) {
+            i = local, gi = 0;
+        } else {
+            const uint32_t l32 = (uint32_t)local, n32 = (uint32_t)tngc;  // both < 2^31
+            i = l32 / n32, gi = l32 - (uint32_t)i * n32;
+        }
+        const int64_t ge = local;  // row-major exponent grid: i * ngc + gi
+        const int64_t j0 = gi * tG;
+        const int glen = (int)min((int64_t)tG, tcols - j0);
+        const int ev = tve[ge], eg = tge[ge], ew = twe[ge];
+        SgdTensor tt;  // for the exact path
+        if (!SINGLE) tt = p.t[sgd_find(p, gw)];
 
         uint32_t wv[CPL][4], vv[CPL][4], gv[CPL][4];
 #pragma unroll
         for (int k = 0; k < CPL; ++k) {
             const int off = (k * L + li) * 16;
             if (off < glen) {
-                const int64_t at = i * t.ld + j0 + off;
-                const uint4 a = *reinterpret_cast<const uint4 *>(t.w + at);
-                const uint4 b = *reinterpret_cast<const uint4 *>(t.v + at);
-                const uint4 c = *reinterpret_cast<const uint4 *>(t.g + at);
+                const int64_t at = i * tld + j0 + off;
+                const uint4 a = *reinterpret_cast<const uint4 *>(tw + at);
+                const uint4 b = *reinterpret_cast<const uint4 *>(tv + at);
+                const uint4 c = *reinterpret_cast<const uint4 *>(tg + at);
                 wv[k][0] = a.x, wv[k][1] = a.y, wv[k][2] = a.z, wv[k][3] = a.w;
                 vv[k][0] = b.x, vv[k][1] = b.y, vv[k][2] = b.z, vv[k][3] = b.w;
                 gv[k][0] = c.x, gv[k][1] = c.y, gv[k][2] = c.z, gv[k][3] = c.w;
@@ -682,70 +700,88 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
             }
         }
 
-        // ---- velocity: v = mom * V + G
-        const GroupSum s1 = group_sum(ev - p.mom_shift, ev == kEZero, 127ll * abs(p.mom_mul), eg,
-                                      eg == kEZero, 127);
-        uint32_t nv[CPL][4];  // new velocity mantissas (packed)
-        int ev2;
-        if (s1.small) {
-            const int ma = (int)s1.ma * p.mom_mul, mb = (int)s1.mb;
-            int amax = 0;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k)
-#pragma unroll
-                for (int b2 = 0; b2 < 16; ++b2) {
-                    const int x = sx8(vv[k][b2 >> 2], b2 & 3) * ma + sx8(gv[k][b2 >> 2], b2 & 3) * mb;
-                    amax = max(amax, abs(x));
-                }
-            amax = group_max<L>(amax, gmask);
-            ev2 = finalize_exp(amax ? s1.r0 + need_off32((uint32_t)amax) : kNoExp);
-            const Shift h = make_shift(ev2 == kEZero ? 0 : ev2 - s1.r0);
-#pragma unroll
-            for (int k = 0; k < CPL; ++k)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    int r[4];
-#pragma unroll
-                    for (int b2 = 0; b2 < 4; ++b2)
-                        r[b2] = apply_shift(sx8(vv[k][q], b2) * ma + sx8(gv[k][q], b2) * mb, h);
-                    nv[k][q] = pack4(r[0], r[1], r[2], r[3]);
-                }
-        } else {
-            sgd_group_exact<L>(p, t, i * t.ld + j0, ge, glen, li, gmask);
+        // ---- velocity: v = mom * V + G (every byte unpacked once; sums stay in registers)
+        constexpr int E = 16 * CPL;
+        int r1, sa1, sb1;
+        bool small1;
+        common_exp(ev - p.mom_shift, ev == kEZero, eg, eg == kEZero, p.cap_mom, 22, r1, sa1, sb1, small1);
+        if (!small1) {
+            sgd_group_exact<L>(p, SINGLE ? p.t[0] : tt, i * tld + j0, ge, glen, li, gmask);
             continue;
+        }
+        int x[E];
+        int ev2;
+        {
+            const int ma = p.mom_mul << sa1, mb = 1 << sb1;
+            int hi = 0, lo = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                x[e] = sx8(vv[e >> 4][(e >> 2) & 3], e & 3) * ma + sx8(gv[e >> 4][(e >> 2) & 3], e & 3) * mb;
+                hi = max(hi, x[e]);
+                lo = min(lo, x[e]);
+            }
+            const int amax = group_max<L>(max(hi, -lo), gmask);
+            ev2 = finalize_exp(amax ? r1 + need_off32((uint32_t)amax) : kNoExp);
+            const Shift h = make_shift(ev2 == kEZero ? 0 : ev2 - r1);
+            if (__any_sync(gmask, h.ls != 0)) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[e] <<= h.ls;
+            }
+            if (h.rs >= 2) {
+                // floor(v / 2^rs) = high word of v * 2^(32 - rs): the shifts run on the FMA pipe
+                const int m = 1 << (32 - h.rs);
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[e] = __mulhi(x[e] + h.bias + (__mulhi(x[e], m) & 1), m);  // v'
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[e] = (x[e] + h.bias + (int)bfe_u32((uint32_t)x[e], h.rs, h.om)) >> h.rs;
+            }
         }
 
         // ---- weight: w = W - lr * v'
-        const GroupSum s2 = group_sum(ew, ew == kEZero, 127, ev2 - p.lr_shift, ev2 == kEZero,
-                                      127ll * abs(p.lr_mul));
-        uint32_t nw[CPL][4];
-        int ew2;
-        if (s2.small) {
-            const int ma = (int)s2.ma, mb = -(int)s2.mb * p.lr_mul;
-            int amax = 0;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k)
-#pragma unroll
-                for (int b2 = 0; b2 < 16; ++b2) {
-                    const int x = sx8(wv[k][b2 >> 2], b2 & 3) * ma + sx8(nv[k][b2 >> 2], b2 & 3) * mb;
-                    amax = max(amax, abs(x));
-                }
-            amax = group_max<L>(amax, gmask);
-            ew2 = finalize_exp(amax ? s2.r0 + need_off32((uint32_t)amax) : kNoExp);
-            const Shift h = make_shift(ew2 == kEZero ? 0 : ew2 - s2.r0);
-#pragma unroll
-            for (int k = 0; k < CPL; ++k)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    int r[4];
-#pragma unroll
-                    for (int b2 = 0; b2 < 4; ++b2)
-                        r[b2] = apply_shift(sx8(wv[k][q], b2) * ma + sx8(nv[k][q], b2) * mb, h);
-                    nw[k][q] = pack4(r[0], r[1], r[2], r[3]);
-                }
-        } else {
-            sgd_group_exact<L>(p, t, i * t.ld + j0, ge, glen, li, gmask);
+        int r2, sa2, sb2;
+        bool small2;
+        common_exp(ew, ew == kEZero, ev2 - p.lr_shift, ev2 == kEZero, 22, p.cap_lr, r2, sa2, sb2, small2);
+        if (!small2) {
+            sgd_group_exact<L>(p, SINGLE ? p.t[0] : tt, i * tld + j0, ge, glen, li, gmask);
             continue;
+        }
+        uint32_t nv[CPL][4], nw[CPL][4];
+        int ew2;
+        {
+            const int ma = 1 << sa2, mb = -(p.lr_mul << sb2);
+            int y[E];
+            int hi = 0, lo = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                y[e] = sx8(wv[e >> 4][(e >> 2) & 3], e & 3) * ma + x[e] * mb;
+                hi = max(hi, y[e]);
+                lo = min(lo, y[e]);
+            }
+            const int amax = group_max<L>(max(hi, -lo), gmask);
+            ew2 = finalize_exp(amax ? r2 + need_off32((uint32_t)amax) : kNoExp);
+            const Shift h = make_shift(ew2 == kEZero ? 0 : ew2 - r2);
+            if (__any_sync(gmask, h.ls != 0)) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) y[e] <<= h.ls;
+            }
+            if (h.rs >= 2) {
+                const int m = 1 << (32 - h.rs);
+#pragma unroll
+                for (int e = 0; e < E; ++e) y[e] = __mulhi(y[e] + h.bias + (__mulhi(y[e], m) & 1), m);
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) y[e] = (y[e] + h.bias + (int)bfe_u32((uint32_t)y[e], h.rs, h.om)) >> h.rs;
+            }
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+                int r[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) r[q] = y[e + q];
+                nw[e >> 4][(e >> 2) & 3] = __byte_perm(__byte_perm(r[0], r[1], 0x0040), __byte_perm(r[2], r[3], 0x0040), 0x5410);
+                nv[e >> 4][(e >> 2) & 3] = __byte_perm(__byte_perm(x[e], x[e + 1], 0x0040),
+                                                       __byte_perm(x[e + 2], x[e + 3], 0x0040), 0x5410);
+            }
         }
 
         // ---- store (masked columns past the group's end are left untouched)
@@ -753,22 +789,140 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
         for (int k = 0; k < CPL; ++k) {
             const int off = (k * L + li) * 16;
             if (off < glen) {
-                const int64_t at = i * t.ld + j0 + off;
+                const int64_t at = i * tld + j0 + off;
                 if (glen - off >= 16) {
-                    *reinterpret_cast<uint4 *>(t.v + at) = make_uint4(nv[k][0], nv[k][1], nv[k][2], nv[k][3]);
-                    *reinterpret_cast<uint4 *>(t.w + at) = make_uint4(nw[k][0], nw[k][1], nw[k][2], nw[k][3]);
+                    *reinterpret_cast<uint4 *>(tv + at) = make_uint4(nv[k][0], nv[k][1], nv[k][2], nv[k][3]);
+                    *reinterpret_cast<uint4 *>(tw + at) = make_uint4(nw[k][0], nw[k][1], nw[k][2], nw[k][3]);
                 } else {
                     for (int b2 = 0; b2 < glen - off; ++b2) {
-                        t.v[at + b2] = (int8_t)(nv[k][b2 >> 2] >> (8 * (b2 & 3)));
-                        t.w[at + b2] = (int8_t)(nw[k][b2 >> 2] >> (8 * (b2 & 3)));
+                        tv[at + b2] = (int8_t)(nv[k][b2 >> 2] >> (8 * (b2 & 3)));
+                        tw[at + b2] = (int8_t)(nw[k][b2 >> 2] >> (8 * (b2 & 3)));
                     }
                 }
             }
         }
         if (li == 0) {
-            t.v_exp[ge] = (int8_t)ev2;
-            t.w_exp[ge] = (int8_t)ew2;
+            tve[ge] = (int8_t)ev2;
+            twe[ge] = (int8_t)ew2;
         }
+    }
+}
+
+// SGD over one dense tensor whose groups are whole rows of exactly 16 * L elements (a
+// parameter arena padded to its group width).  Same arithmetic as sgd_vec_kernel; the
+// next group's W, V, G chunks are loaded before the current group is computed, so each
+// warp keeps a load in flight while it computes.
+template <int L>
+__global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ SgdArgs p) {
+    constexpr int GPW = 32 / L;
+    const int lane = threadIdx.x & 31, sub = lane / L, li = lane % L;
+    const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (sub * L));
+    const SgdTensor &t0 = p.t[0];
+    int8_t *const tw = t0.w, *const tv = t0.v, *const twe = t0.w_exp, *const tve = t0.v_exp;
+    const int8_t *const tg = t0.g, *const tge = t0.g_exp;
+    const int64_t rows = t0.rows;
+    const int64_t step = (int64_t)gridDim.x * 8 * GPW;
+    int64_t r = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * GPW + sub;
+    uint4 cw = make_uint4(0, 0, 0, 0), cv = cw, cg = cw;
+    int ev = 0, eg = 0, ew = 0;
+    if (r < rows) {
+        const int64_t at = r * (16 * L) + li * 16;
+        cw = *reinterpret_cast<const uint4 *>(tw + at);
+        cv = *reinterpret_cast<const uint4 *>(tv + at);
+        cg = *reinterpret_cast<const uint4 *>(tg + at);
+        ev = tve[r], eg = tge[r], ew = twe[r];
+    }
+    for (; r < rows; r += step) {
+        const int64_t rn = r + step;
+        uint4 nw4 = make_uint4(0, 0, 0, 0), nv4 = nw4, ng4 = nw4;
+        int nev = 0, neg = 0, new_ = 0;
+        if (rn < rows) {  // prefetch the next group
+            const int64_t at = rn * (16 * L) + li * 16;
+            nw4 = *reinterpret_cast<const uint4 *>(tw + at);
+            nv4 = *reinterpret_cast<const uint4 *>(tv + at);
+            ng4 = *reinterpret_cast<const uint4 *>(tg + at);
+            nev = tve[rn], neg = tge[rn], new_ = twe[rn];
+        }
+        const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w}, vv[4] = {cv.x, cv.y, cv.z, cv.w},
+                       gv[4] = {cg.x, cg.y, cg.z, cg.w};
+        // velocity
+        int r1, sa1, sb1;
+        bool small1;
+        common_exp(ev - p.mom_shift, ev == kEZero, eg, eg == kEZero, p.cap_mom, 22, r1, sa1, sb1, small1);
+        int r2 = 0, sa2 = 0, sb2 = 0, ev2 = kEZero;
+        bool small2 = false;
+        int x[16];
+        if (small1) {
+            const int ma = p.mom_mul << sa1, mb = 1 << sb1;
+            int hi = 0, lo = 0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                x[e] = sx8(vv[e >> 2], e & 3) * ma + sx8(gv[e >> 2], e & 3) * mb;
+                hi = max(hi, x[e]);
+                lo = min(lo, x[e]);
+            }
+            const int amax = group_max<L>(max(hi, -lo), gmask);
+            ev2 = finalize_exp(amax ? r1 + need_off32((uint32_t)amax) : kNoExp);
+            const Shift h = make_shift(ev2 == kEZero ? 0 : ev2 - r1);
+            if (__any_sync(gmask, h.ls != 0)) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x[e] <<= h.ls;
+            }
+            if (h.rs >= 2) {
+                const int m = 1 << (32 - h.rs);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x[e] = __mulhi(x[e] + h.bias + (__mulhi(x[e], m) & 1), m);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x[e] = (x[e] + h.bias + (int)bfe_u32((uint32_t)x[e], h.rs, h.om)) >> h.rs;
+            }
+            common_exp(ew, ew == kEZero, ev2 - p.lr_shift, ev2 == kEZero, 22, p.cap_lr, r2, sa2, sb2, small2);
+        }
+        if (!(small1 && small2)) {
+            sgd_group_exact<L>(p, t0, r * (16 * L), r, 16 * L, li, gmask);
+        } else {
+            const int ma = 1 << sa2, mb = -(p.lr_mul << sb2);
+            int y[16];
+            int hi = 0, lo = 0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                y[e] = sx8(wv[e >> 2], e & 3) * ma + x[e] * mb;
+                hi = max(hi, y[e]);
+                lo = min(lo, y[e]);
+            }
+            const int amax = group_max<L>(max(hi, -lo), gmask);
+            const int ew2 = finalize_exp(amax ? r2 + need_off32((uint32_t)amax) : kNoExp);
+            const Shift h = make_shift(ew2 == kEZero ? 0 : ew2 - r2);
+            if (__any_sync(gmask, h.ls != 0)) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) y[e] <<= h.ls;
+            }
+            if (h.rs >= 2) {
+                const int m = 1 << (32 - h.rs);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) y[e] = __mulhi(y[e] + h.bias + (__mulhi(y[e], m) & 1), m);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) y[e] = (y[e] + h.bias + (int)bfe_u32((uint32_t)y[e], h.rs, h.om)) >> h.rs;
+            }
+            uint32_t ov[4], ow[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                ov[q] = __byte_perm(__byte_perm(x[4 * q], x[4 * q + 1], 0x0040),
+                                    __byte_perm(x[4 * q + 2], x[4 * q + 3], 0x0040), 0x5410);
+                ow[q] = __byte_perm(__byte_perm(y[4 * q], y[4 * q + 1], 0x0040),
+                                    __byte_perm(y[4 * q + 2], y[4 * q + 3], 0x0040), 0x5410);
+            }
+            const int64_t at = r * (16 * L) + li * 16;
+            *reinterpret_cast<uint4 *>(tv + at) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+            *reinterpret_cast<uint4 *>(tw + at) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            if (li == 0) {
+                tve[r] = (int8_t)ev2;
+                twe[r] = (int8_t)ew2;
+            }
+        }
+        cw = nw4, cv = nv4, cg = ng4;
+        ev = nev, eg = neg, ew = new_;
     }
 }
 

@@ -37,7 +37,8 @@ def status_ok(ict):
 # ------------------------------------------------------------------ requant / align
 
 
-@pytest.mark.parametrize("rows,cols,G", [(5, 32, 32), (130, 96, 32), (64, 192, 64), (33, 768, 768), (7, 48, 16)])
+@pytest.mark.parametrize("rows,cols,G", [(5, 32, 32), (130, 96, 32), (64, 192, 64), (33, 768, 768), (7, 48, 16),
+                                         (9, 192, 192), (4, 320, 160), (3, 3072, 3072), (6, 512, 256)])
 def test_requant(ict, rows, cols, G):
     import torch
 
@@ -89,6 +90,8 @@ LINEAR_CASES = [
     (129, 256, 384, (1, 128), (4, 64), 256),
     (512, 448, 192, (1, 192), (1, 192), 64),
     (1000, 768, 768, (1, 64), (1, 64), 64),
+    (2000, 64, 192, (1, 64), (1, 192), 64),       # long K: split-K slices, 192-wide dW rows
+    (3000, 128, 320, (1, 32), (1, 320), 32),      # split-K, 320-wide dW rows
 ]
 
 
