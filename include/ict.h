@@ -114,6 +114,25 @@ const char *ict_version(void);
  * all threads).  Lets a caller count the device work a sequence of calls issues. */
 uint64_t ict_launch_count(void);
 
+/* Device timing by kernel class, for measurement.  While enabled, every launch the
+ * library makes is bracketed by a pair of CUDA events recorded on its stream (events are
+ * created on first use and reused; no device memory is allocated).  ict_timing_read()
+ * synchronises the recorded events, adds their durations into per-class totals and
+ * returns, for one class, the summed device time (ms), the number of timed launches and
+ * their algorithmic work: multiply-add operations (2 M N K) for ICT_KC_GEMM, bytes read
+ * plus written for the memory-bound classes.  reset = 1 clears every class afterwards. */
+typedef enum {
+    ICT_KC_GEMM = 0,    /* tensor-core Product kernels (linear, conv) */
+    ICT_KC_SGD = 1,     /* integer SGD-with-momentum update */
+    ICT_KC_ALIGN = 2,   /* exponent alignment (ALIGN_MAX) and weight re-layout */
+    ICT_KC_REQUANT = 3, /* FIT of int32 / int64 values (split-K combine) */
+    ICT_KC_GELU = 4,    /* GELU forward / backward */
+    ICT_KC_OTHER = 5    /* fills and exponent tables */
+} ict_kernel_class;
+int32_t ict_timing_enable(int32_t on);
+int32_t ict_timing_read(int32_t kernel_class, double *ms_total, int64_t *launches, double *work,
+                        int32_t reset);
+
 /* Bound, in nanoseconds, of every wait inside a kernel (0 restores the default, 2 s).
  * A wait that runs out raises ICT_ERR_DEVICE_TIMEOUT in the device status word; the
  * kernel then lets its in-flight copies and tensor-core operations finish (again with a

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "ict_device.cuh"
 #include "ict_elementwise.cuh"
@@ -58,6 +59,55 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? ICT_OK : ICT_ER
 // number of kernels launched through this library (process-wide)
 std::atomic<uint64_t> g_launches{0};
 void counted(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// ---- optional per-kernel-class device timing (measurement only; off by default)
+enum { KC_GEMM = 0, KC_SGD = 1, KC_ALIGN = 2, KC_REQUANT = 3, KC_GELU = 4, KC_OTHER = 5, KC_N = 6 };
+struct TimedLaunch {
+    int kc;
+    cudaEvent_t a, b;
+    double work;
+};
+struct Timing {
+    bool on = false;
+    std::vector<TimedLaunch> pending;
+    std::vector<cudaEvent_t> pool;
+    double ms[KC_N] = {0}, work[KC_N] = {0};
+    int64_t n[KC_N] = {0};
+} g_timing;
+std::mutex g_timing_mu;
+
+cudaEvent_t timing_event() {
+    if (!g_timing.pool.empty()) {
+        cudaEvent_t e = g_timing.pool.back();
+        g_timing.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Brackets the launches issued during its lifetime with a pair of events on `s`.
+struct KTimer {
+    cudaEvent_t a = nullptr;
+    cudaStream_t s;
+    int kc;
+    double work;
+    KTimer(cudaStream_t s_, int kc_, double work_) : s(s_), kc(kc_), work(work_) {
+        std::lock_guard<std::mutex> lk(g_timing_mu);
+        if (!g_timing.on) return;
+        a = timing_event();
+        if (a) cudaEventRecord(a, s);
+    }
+    ~KTimer() {
+        if (!a) return;
+        std::lock_guard<std::mutex> lk(g_timing_mu);
+        cudaEvent_t b = timing_event();
+        if (!b) return;
+        cudaEventRecord(b, s);
+        g_timing.pending.push_back(TimedLaunch{kc, a, b, work});
+    }
+};
 
 // ------------------------------------------------------------------ TMA descriptors
 
@@ -182,6 +232,7 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     int sms = 148;
     device_info(&sms);
     const int64_t n_exp = n_grp_rows(in) * a.ngc;
+    KTimer kt(s, KC_ALIGN, 2.0 * (double)in->rows * (double)in->cols);
     if (j.axis == 1) {
         estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
     } else if (j.col_max && a.ngc <= 8192) {
@@ -218,6 +269,7 @@ int launch_requant_rows(RequantArgs a, cudaStream_t s) {
     const int64_t groups = a.rows * a.ngc;
     if (groups == 0) return ICT_OK;
     const int G = a.G;
+    KTimer kt(s, KC_REQUANT, (double)a.rows * (double)a.cols * (a.v64 ? 9.0 : 4.0 * a.nsplit + 1.0));
     if (G >= 128 && G <= 4096) {
         const int T = G >= 256 ? 256 : 128;
         const int ept = (G + T - 1) / T;
@@ -267,7 +319,8 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
 }
 
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
-                const GemmParams &p, int grid, cudaStream_t s) {
+                const GemmParams &p, int grid, cudaStream_t s, double ops) {
+    KTimer kt(s, KC_GEMM, ops);
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
     if (bn == BN_ && bk == BK_ && load == LOAD_) \
         return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s);
@@ -422,7 +475,8 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     p.epi = pl.fused ? EPI_FIT_ROW : EPI_I32;
-    if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s))) return st;
+    if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K)))
+        return st;
     if (pl.fused) return ICT_OK;
     RequantArgs a;
     memset(&a, 0, sizeof(a));
@@ -677,16 +731,17 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     const int grid = std::min(p.num_units, sms);
+    const double ops = 2.0 * (double)cp.out_rows * (double)cp.out_cols * (double)ktot;
     if (!cp.global_groups) {
         p.epi = EPI_FIT_ROW;
-        return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s);
+        return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
     }
     fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
     counted(1);
-    p.epi = EPI_NEED_GLOBAL;
-    if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s))) return st;
+    p.epi = EPI_NEED_GLOBAL;  // the first pass is recompute: its work is not counted again
+    if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
     p.epi = EPI_FIT_GLOBAL;
-    return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s);
+    return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
 }
 
 // ---- convolution backward-weight: dW[k][(r,s,c)] = sum over output pixels of
@@ -780,7 +835,9 @@ int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X,
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     p.epi = EPI_I32;
-    if ((st = launch_gemm(64, 256, LOAD_CONV_WGRAD, ta, tb, p, std::min(wp.units, sms), s))) return st;
+    if ((st = launch_gemm(64, 256, LOAD_CONV_WGRAD, ta, tb, p, std::min(wp.units, sms), s,
+                          2.0 * (double)wp.M * (double)wp.N * (double)d->n * d->h * d->w)))
+        return st;
     // dW[k][j] = sum over slices of partial[j][k]: FIT per row k, exponent e_cols[k] + e_rows[j]
     RequantArgs a;
     memset(&a, 0, sizeof(a));
@@ -857,6 +914,9 @@ int bitlen_u64(uint64_t v) {
 // most 2048): L lanes per group, CPL 16-byte chunks per lane; else one warp per group.
 int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
     if (a.total_groups == 0) return ICT_OK;
+    double elems = 0;
+    for (int i = 0; i < a.n; ++i) elems += (double)a.t[i].rows * (double)a.t[i].cols;
+    KTimer kt(s, KC_SGD, 5.0 * elems + 5.0 * (double)a.total_groups);
     bool vec = true;
     const int G = a.t[0].G;
     for (int i = 0; i < a.n; ++i)
@@ -948,6 +1008,36 @@ const char *ict_status_string(int32_t status) {
 const char *ict_version(void) { return "libict 0.1 sm_100a"; }
 
 uint64_t ict_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t ict_timing_enable(int32_t on) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timing.on = on != 0;
+    return ICT_OK;
+}
+
+int32_t ict_timing_read(int32_t kernel_class, double *ms_total, int64_t *launches, double *work,
+                        int32_t reset) {
+    if (kernel_class < 0 || kernel_class >= KC_N) return ICT_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    for (const TimedLaunch &t : g_timing.pending) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(t.b) != cudaSuccess || cudaEventElapsedTime(&ms, t.a, t.b) != cudaSuccess)
+            return ICT_ERR_CUDA;
+        g_timing.ms[t.kc] += ms;
+        g_timing.n[t.kc] += 1;
+        g_timing.work[t.kc] += t.work;
+        g_timing.pool.push_back(t.a);
+        g_timing.pool.push_back(t.b);
+    }
+    g_timing.pending.clear();
+    if (ms_total) *ms_total = g_timing.ms[kernel_class];
+    if (launches) *launches = g_timing.n[kernel_class];
+    if (work) *work = g_timing.work[kernel_class];
+    if (reset) {
+        for (int k = 0; k < KC_N; ++k) g_timing.ms[k] = g_timing.work[k] = 0, g_timing.n[k] = 0;
+    }
+    return ICT_OK;
+}
 
 int32_t ict_get_device_status(int32_t *host_out, void *stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ICT_ERR_CUDA;
@@ -1154,6 +1244,7 @@ int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream) {
     if (cudaMemcpyAsync(out->exp, H->exp, ne, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return ICT_ERR_CUDA;
     const int64_t vecs = H->rows * (H->cols / 16);
+    KTimer kt(s, KC_GELU, 2.0 * (double)H->rows * (double)H->cols + 2.0 * (double)ne);
     gelu_fwd_kernel<<<(unsigned)cdiv64(vecs, 256), 256, 0, s>>>(a);
     counted(1);
     return launch_status();
@@ -1187,6 +1278,7 @@ int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, 
     const int64_t groups = H->rows * a.ngc;
     cudaStream_t s = (cudaStream_t)stream;
     const int G = a.g_cols;
+    KTimer kt(s, KC_GELU, 3.0 * (double)H->rows * (double)H->cols + 3.0 * (double)groups);
     const bool vec = check_vec(H) == ICT_OK && check_vec(dG) == ICT_OK && check_vec(dH) == ICT_OK &&
                      G % 16 == 0 && G <= 512 && ((G / 16) & (G / 16 - 1)) == 0;
     if (vec) {

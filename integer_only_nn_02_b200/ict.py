@@ -61,6 +61,8 @@ _SIGS = {
     "ict_get_device_status": ([_P(_i32), _vp], _i32),
     "ict_set_wait_limit_ns": ([ctypes.c_uint64], _i32),
     "ict_launch_count": ([], ctypes.c_uint64),
+    "ict_timing_enable": ([_i32], _i32),
+    "ict_timing_read": ([_i32, _P(ctypes.c_double), _P(_i64), _P(ctypes.c_double), _i32], _i32),
     "ict_requant": ([_vp, _i32, _i64, _i64, _i64, _i32, _vp, _vp, _P(ict_tensor), _vp], _i32),
     "ict_align": ([_P(ict_tensor), _i32, _i32, _vp, _i64, _vp, _vp], _i32),
     "ict_linear_workspace": ([_i32, _P(ict_tensor), _P(ict_tensor), _P(ict_tensor)], _sz),
@@ -171,6 +173,21 @@ def ict_get_device_status(stream=None):
 
 def ict_launch_count() -> int:
     return int(lib.ict_launch_count())
+
+
+KERNEL_CLASSES = {"gemm": 0, "sgd": 1, "align": 2, "requant": 3, "gelu": 4, "other": 5}
+
+
+def ict_timing_enable(on: bool) -> None:
+    _check(lib.ict_timing_enable(int(bool(on))), "ict_timing_enable")
+
+
+def ict_timing_read(kernel_class: int, reset: bool = False):
+    """(device ms, launches, algorithmic work) accumulated for one kernel class."""
+    ms, n, w = ctypes.c_double(0), ctypes.c_int64(0), ctypes.c_double(0)
+    _check(lib.ict_timing_read(int(kernel_class), ctypes.byref(ms), ctypes.byref(n), ctypes.byref(w),
+                               int(bool(reset))), "ict_timing_read")
+    return ms.value, n.value, w.value
 
 
 def ict_set_wait_limit_ns(ns: int) -> None:
