@@ -1,21 +1,23 @@
 """Benchmark of the integer-only (C,e) training hot path on B200.
 
-One step = one training step of a ViT-Ti-shaped MLP block through libict.so:
-fc1 forward (12608x192 . 192x768), integer GELU, fc2 forward (12608x768 . 768x192),
-fc2 backward-data and backward-weight, GELU backward, fc1 backward-data and
-backward-weight, and the integer SGD-with-momentum update of both weight matrices
-(per-row velocity groups).  Synthetic seeded inputs of the paper's ViT-Ti shapes
-(64 images x 197 tokens; "Memory-Efficient Integer-Only Training of Deep Neural
+Default step (--config vit_ti_mlp): one training step of a ViT-Ti-shaped MLP block
+through libict.so: fc1 forward (12608x192 . 192x768), integer GELU, fc2 forward
+(12608x768 . 768x192), fc2 backward-data and backward-weight, GELU backward, fc1
+backward-data and backward-weight, and the integer SGD-with-momentum update of both
+weight matrices (per-row velocity groups).  Synthetic seeded inputs of the ViT-Ti layer
+shapes (64 images x 197 tokens; "Memory-Efficient Integer-Only Training of Deep Neural
 Networks", Abstract and Table 9).
 
-metric: (C,e) GEMM TOPS over the whole step (6 contractions = 22.31 GOP per step),
-plus the int-SGD update GB/s (ResNet-50 parameter arena) and the large-shape GEMM TOPS
-(ViT-B linear trio) as side measurements.
+metric: (C,e) GEMM TOPS over the step (6 contractions = 22.31 GOP per step).  The other
+configurations, each a step of its own with its own unit:
+  vit_b_linear_trio   the six ViT-B MLP contractions (357 GOP), TOPS
+  resnet18_conv3x3    3x3 conv fwd, bwd-data, bwd-weight on 128x56x56x64, TOPS
+  resnet50_sgd        int-SGD update of a ResNet-50-sized parameter arena, GB/s
+  single_linear       64x128 linear layer fwd+bwd+SGD, microseconds per step
 
-Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-For N > 1 run under torchrun: every rank runs the same single-GPU step on its own
-batch (independent replicas, no data-path collective); the reported time is the max
-over ranks.
+Usage:  python bench.py [--config C] [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 run under torchrun: every rank runs the same single-GPU step on its own batch
+(independent replicas, no data-path collective); the reported time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -34,18 +36,29 @@ import numpy as np  # noqa: E402
 
 from integer_only_nn_02_b200 import workloads as wl  # noqa: E402
 
-TOKENS, D, HID, GROUP = 64 * 197, 192, 768, 32
-STEP_OPS = 6 * 2 * TOKENS * D * HID  # six contractions per step
-L2_FLUSH_BYTES = 512 << 20          # larger than the 126 MB L2
+L2_FLUSH_BYTES = 512 << 20  # larger than the 126 MB L2
+METRIC = "(C,e) GEMM TOPS fwd+bwd vs INT8 tensor peak; int-SGD update GB/s vs HBM"
+CLASS_NAMES = ["gemm", "sgd", "align", "requant", "gelu", "estar", "other"]  # ict_kernel_class order
+CLASS_KERNELS = {
+    "gemm": "gemm_ce_kernel (tcgen05 kind::i8, fused FIT epilogue)",
+    "sgd": "sgd_rows_kernel / sgd_vec_kernel",
+    "align": "align_tile_kernel (ALIGN_MAX shifts, transposes)",
+    "requant": "requant_group_block_kernel / requant_rows_kernel",
+    "gelu": "gelu_fwd_kernel / gelu_bwd_vec_kernel",
+    "estar": "estar_rows_kernel / estar_cols_scratch_kernel",
+    "other": "fills, weight re-layout, exponent tables",
+}
 
 
 def parse():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--config", default="vit_ti_mlp", choices=list(STEPS))
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 20; 100 for resnet50_sgd)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-side", action="store_true", help="skip the side measurements")
+    ap.add_argument("--no-side", action="store_true", help="skip the other configurations' side numbers")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     return ap.parse_args()
 
 
@@ -80,7 +93,6 @@ class ClockSampler:
 
             pynvml.nvmlInit()
             self.nv = pynvml
-            h = None
             try:
                 uuid = str(torch.cuda.get_device_properties(torch_index).uuid)
                 uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
@@ -89,25 +101,22 @@ class ClockSampler:
                 h = pynvml.nvmlDeviceGetHandleByIndex(torch_index)
             self.handle = h
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-        except Exception as exc:  # pragma: no cover
-            self.error = str(exc)
+        except Exception:  # pragma: no cover
+            self.handle = None
 
     def _reasons(self):
-        nv = self.nv
-        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(self.nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
         return int(f(self.handle))
 
     def _loop(self):
-        import time as _t
-
         while not self.stop_flag:
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM))
                 self.reason_bits |= self._reasons()
             except Exception:
                 pass
-            _t.sleep(0.002)
+            time.sleep(0.002)
 
     def start(self):
         import threading
@@ -127,48 +136,24 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
 
 
-# --------------------------------------------------------------------- the step
+# --------------------------------------------------------------------- steps
 
 
-class MlpStep:
-    """Device state of one ViT-Ti MLP block training step (all buffers preallocated)."""
+class Step:
+    """A configuration's step: device state, the library calls of one step, its work."""
 
-    def __init__(self, ict, seed: int):
-        import torch
+    unit = "TOPS"
+    higher_is_better = True
+    sample_arg = None
 
+    def __init__(self, ict, torch):
         self.ict, self.torch = ict, torch
-        cfg = wl.vit_ti_mlp(seed=seed)
-        self.cfg = cfg
-        E = ict.DevCE
-        self.X, self.W1, self.W2, self.dY2 = (E.from_host(cfg[k]) for k in ("X", "W1", "W2", "dY2"))
-        self.V1, self.V2 = E.from_host(cfg["V1"]), E.from_host(cfg["V2"])
-        M = TOKENS
-        self.H = E.empty(M, HID, 1, GROUP)
-        self.G = E.empty(M, HID, 1, GROUP)
-        self.Y = E.empty(M, D, 1, GROUP)
-        self.dG = E.empty(M, HID, 1, GROUP)
-        self.dH = E.empty(M, HID, 1, GROUP)
-        self.dX = E.empty(M, D, 1, GROUP)
-        self.dW2 = E.empty(D, HID, 1, HID)
-        self.dW1 = E.empty(HID, D, 1, D)
-        ws = ict.ict_linear_workspace
-        need = max(ws(0, self.X, self.W1, self.H), ws(0, self.G, self.W2, self.Y),
-                   ws(1, self.dY2, self.W2, self.dG), ws(2, self.dY2, self.G, self.dW2),
-                   ws(1, self.dH, self.W1, self.dX), ws(2, self.dH, self.X, self.dW1))
-        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
-        self.mom, self.lr = cfg["sgd"]["mom"], cfg["sgd"]["lr"]
-        self.calls = [
-            ("fc1_fwd", lambda: ict.ict_linear_fwd(self.X, self.W1, self.H, self.ws)),
-            ("gelu_fwd", lambda: ict.ict_gelu_fwd(self.H, self.G)),
-            ("fc2_fwd", lambda: ict.ict_linear_fwd(self.G, self.W2, self.Y, self.ws)),
-            ("fc2_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY2, self.W2, self.dG, self.ws)),
-            ("fc2_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY2, self.G, self.dW2, self.ws)),
-            ("gelu_bwd", lambda: ict.ict_gelu_bwd(self.H, self.dG, self.dH)),
-            ("fc1_bwd_data", lambda: ict.ict_linear_bwd_data(self.dH, self.W1, self.dX, self.ws)),
-            ("fc1_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dH, self.X, self.dW1, self.ws)),
-            ("sgd_w1", lambda: ict.ict_sgd_momentum_step(self.W1, self.V1, self.dW1, self.mom, self.lr)),
-            ("sgd_w2", lambda: ict.ict_sgd_momentum_step(self.W2, self.V2, self.dW2, self.mom, self.lr)),
-        ]
+        self.calls = []
+        self.h2d = []  # device tensors refreshed from pinned host copies every e2e step
+        self.d2h = []  # device tensors read back every e2e step
+
+    def ws(self, nbytes):
+        return self.torch.empty(max(int(nbytes), 256), dtype=self.torch.uint8, device="cuda")
 
     def run(self, events=None):
         for i, (_, fn) in enumerate(self.calls):
@@ -178,9 +163,268 @@ class MlpStep:
             if events is not None:
                 events[i][1].record()
 
+    @classmethod
+    def value_of(cls, units, seconds):
+        """The metric from the step's work units and its time."""
+        if cls.unit == "us":
+            return seconds * 1e6
+        if cls.unit == "GB/s":
+            return units / seconds / 1e9
+        return units / seconds / 1e12
 
-def time_steps(step, K, W, flush):
-    """Per-step device time (ms) with an L2 flush between steps; per-call breakdown."""
+
+class MlpStep(Step):
+    TOKENS, D, HID, GROUP = 64 * 197, 192, 768, 32
+    sample_arg = 64 * 197
+    workload = {"workload": "vit_ti_mlp_block_step", "tokens": 12608, "d": 192, "hidden": 768, "group": 32,
+                "gop_per_step": 22.31}
+
+    def __init__(self, ict, torch, seed):
+        super().__init__(ict, torch)
+        E = ict.DevCE
+        cfg = wl.vit_ti_mlp(seed=seed)
+        self.X, self.W1, self.W2, self.dY2 = (E.from_host(cfg[k]) for k in ("X", "W1", "W2", "dY2"))
+        self.V1, self.V2 = E.from_host(cfg["V1"]), E.from_host(cfg["V2"])
+        M, D, H, G = self.TOKENS, self.D, self.HID, self.GROUP
+        self.H, self.G, self.dG, self.dH = (E.empty(M, H, 1, G) for _ in range(4))
+        self.Y, self.dX = E.empty(M, D, 1, G), E.empty(M, D, 1, G)
+        self.dW2, self.dW1 = E.empty(D, H, 1, H), E.empty(H, D, 1, D)
+        w = ict.ict_linear_workspace
+        ws = self.ws(max(w(0, self.X, self.W1, self.H), w(0, self.G, self.W2, self.Y),
+                         w(1, self.dY2, self.W2, self.dG), w(2, self.dY2, self.G, self.dW2),
+                         w(1, self.dH, self.W1, self.dX), w(2, self.dH, self.X, self.dW1)))
+        mom, lr = cfg["sgd"]["mom"], cfg["sgd"]["lr"]
+        self.calls = [
+            ("fc1_fwd", lambda: ict.ict_linear_fwd(self.X, self.W1, self.H, ws)),
+            ("gelu_fwd", lambda: ict.ict_gelu_fwd(self.H, self.G)),
+            ("fc2_fwd", lambda: ict.ict_linear_fwd(self.G, self.W2, self.Y, ws)),
+            ("fc2_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY2, self.W2, self.dG, ws)),
+            ("fc2_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY2, self.G, self.dW2, ws)),
+            ("gelu_bwd", lambda: ict.ict_gelu_bwd(self.H, self.dG, self.dH)),
+            ("fc1_bwd_data", lambda: ict.ict_linear_bwd_data(self.dH, self.W1, self.dX, ws)),
+            ("fc1_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dH, self.X, self.dW1, ws)),
+            ("sgd_w1", lambda: ict.ict_sgd_momentum_step(self.W1, self.V1, self.dW1, mom, lr)),
+            ("sgd_w2", lambda: ict.ict_sgd_momentum_step(self.W2, self.V2, self.dW2, mom, lr)),
+        ]
+        self.units = 6 * 2 * M * D * H
+        self.h2d = [self.X.mant, self.X.exp, self.dY2.mant, self.dY2.exp]
+        self.d2h = [self.W1.mant, self.W1.exp, self.W2.mant, self.W2.exp]
+
+    @staticmethod
+    def oracle_step(tokens):
+        import oracle
+
+        cfg = wl.vit_ti_mlp(seed=0, tokens=tokens)
+        X, W1, W2, dY2 = cfg["X"], cfg["W1"], cfg["W2"], cfg["dY2"]
+        G = MlpStep.GROUP
+        mom, lr = cfg["sgd"]["mom"], cfg["sgd"]["lr"]
+        t0 = time.perf_counter()
+        H = oracle.linear_fwd(X, W1, 1, G)
+        Gl = oracle.gelu_fwd(H)
+        oracle.linear_fwd(Gl, W2, 1, G)
+        dG = oracle.linear_bwd_data(dY2, W2, 1, G)
+        dW2 = oracle.linear_bwd_weight(dY2, Gl, 1, W2.cols)
+        dH = oracle.gelu_bwd(H, dG, 1, G)
+        oracle.linear_bwd_data(dH, W1, 1, G)
+        dW1 = oracle.linear_bwd_weight(dH, X, 1, W1.cols)
+        oracle.sgd_step(W1, cfg["V1"], dW1, mom, lr)
+        oracle.sgd_step(W2, cfg["V2"], dW2, mom, lr)
+        dt = time.perf_counter() - t0
+        return dt, 6 * 2 * tokens * MlpStep.D * MlpStep.HID, f"one full step ({tokens} tokens)"
+
+
+class LinearStep(Step):
+    unit = "us"
+    higher_is_better = False
+    workload = {"workload": "single_linear_step", "m": 64, "k": 128, "n": 64, "group": 32}
+
+    def __init__(self, ict, torch, seed):
+        super().__init__(ict, torch)
+        E = ict.DevCE
+        cfg = wl.single_linear(seed=seed)
+        self.X, self.W, self.dY, self.V = (E.from_host(cfg[k]) for k in ("X", "W", "dY", "V"))
+        G = cfg["out_group"]
+        self.Y, self.dX, self.dW = E.empty(64, 64, 1, G), E.empty(64, 128, 1, G), E.empty(64, 128, 1, 128)
+        w = ict.ict_linear_workspace
+        ws = self.ws(max(w(0, self.X, self.W, self.Y), w(1, self.dY, self.W, self.dX),
+                         w(2, self.dY, self.X, self.dW)))
+        mom, lr = cfg["sgd"]["mom"], cfg["sgd"]["lr"]
+        self.calls = [
+            ("fwd", lambda: ict.ict_linear_fwd(self.X, self.W, self.Y, ws)),
+            ("bwd_data", lambda: ict.ict_linear_bwd_data(self.dY, self.W, self.dX, ws)),
+            ("bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY, self.X, self.dW, ws)),
+            ("sgd", lambda: ict.ict_sgd_momentum_step(self.W, self.V, self.dW, mom, lr)),
+        ]
+        self.units = 1
+        self.h2d = [self.X.mant, self.X.exp, self.dY.mant, self.dY.exp]
+        self.d2h = [self.W.mant, self.W.exp]
+
+    @staticmethod
+    def oracle_step(_):
+        import oracle
+
+        cfg = wl.single_linear(seed=0)
+        X, W, dY, V = cfg["X"], cfg["W"], cfg["dY"], cfg["V"]
+        t0 = time.perf_counter()
+        oracle.linear_fwd(X, W, 1, 32)
+        oracle.linear_bwd_data(dY, W, 1, 32)
+        dW = oracle.linear_bwd_weight(dY, X, 1, 128)
+        oracle.sgd_step(W, V, dW, cfg["sgd"]["mom"], cfg["sgd"]["lr"])
+        return time.perf_counter() - t0, 1, "one full step"
+
+
+class ConvStep(Step):
+    sample_arg = 32
+    workload = {"workload": "resnet18_conv3x3_fwd_bwd", "n": 128, "h": 56, "w": 56, "c": 64, "k": 64,
+                "group": 32, "gop_per_step": 88.785}
+
+    def __init__(self, ict, torch, seed):
+        super().__init__(ict, torch)
+        E = ict.DevCE
+        cfg = wl.resnet18_conv3x3(seed=seed)
+        d, G = cfg["conv"], cfg["out_group"]
+        self.X, self.W, self.dY = (E.from_host(cfg[k]) for k in ("X", "W", "dY"))
+        npix = self.X.rows
+        self.Y, self.dX = E.empty(npix, 64, npix, G), E.empty(npix, 64, npix, G)
+        self.dW = E.empty(64, 576, 1, 576)
+        cw = ict.ict_conv_workspace
+        ws = self.ws(max(cw(0, d), cw(1, d), cw(2, d)))
+        self.calls = [
+            ("fwd", lambda: ict.ict_conv_implicit_gemm(0, d, self.X, self.W, self.Y, ws)),
+            ("bwd_data", lambda: ict.ict_conv_implicit_gemm(1, d, self.dY, self.W, self.dX, ws)),
+            ("bwd_weight", lambda: ict.ict_conv_implicit_gemm(2, d, self.dY, self.X, self.dW, ws)),
+        ]
+        self.units = 3 * 2 * npix * 64 * 576
+        self.h2d = [self.X.mant, self.X.exp, self.dY.mant, self.dY.exp]
+        self.d2h = [self.dW.mant, self.dW.exp]
+
+    @staticmethod
+    def oracle_step(images):
+        import oracle
+
+        cfg = wl.resnet18_conv3x3(seed=0, n=images)
+        X, W, dY, d = cfg["X"], cfg["W"], cfg["dY"], cfg["conv"]
+        t0 = time.perf_counter()
+        oracle.conv(oracle.CONV_FWD, d, X, W, X.rows, 32)
+        oracle.conv(oracle.CONV_BWD_DATA, d, dY, W, X.rows, 32)
+        oracle.conv(oracle.CONV_BWD_WEIGHT, d, dY, X, 1, W.cols)
+        dt = time.perf_counter() - t0
+        return dt, 3 * 2 * X.rows * 64 * 576, f"fwd+bwd-data+bwd-weight on {images} of the 128 images"
+
+
+class TrioStep(Step):
+    sample_arg = 2048
+    workload = {"workload": "vit_b_linear_trio", "tokens": 12608, "d": 768, "hidden": 3072, "group": 64,
+                "gop_per_step": 356.952}
+
+    def __init__(self, ict, torch, seed):
+        super().__init__(ict, torch)
+        E = ict.DevCE
+        cfg = wl.vit_b_linear_trio(seed=seed)
+        self.X, self.W1, self.W2, self.dY1, self.dY2 = (E.from_host(cfg[k]) for k in ("X", "W1", "W2", "dY1", "dY2"))
+        M, G = self.X.rows, cfg["out_group"]
+        self.H1, self.Y2 = E.empty(M, 3072, 1, G), E.empty(M, 768, 1, G)
+        self.dXo, self.dHo = E.empty(M, 768, 1, G), E.empty(M, 3072, 1, G)
+        self.dW1, self.dW2 = E.empty(3072, 768, 1, 768), E.empty(768, 3072, 1, 3072)
+        w = ict.ict_linear_workspace
+        ws = self.ws(max(w(0, self.X, self.W1, self.H1), w(0, self.H1, self.W2, self.Y2),
+                         w(1, self.dY2, self.W2, self.dHo), w(1, self.dY1, self.W1, self.dXo),
+                         w(2, self.dY1, self.X, self.dW1), w(2, self.dY2, self.H1, self.dW2)))
+        self.calls = [
+            ("fc1_fwd", lambda: ict.ict_linear_fwd(self.X, self.W1, self.H1, ws)),
+            ("fc2_fwd", lambda: ict.ict_linear_fwd(self.H1, self.W2, self.Y2, ws)),
+            ("fc2_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY2, self.W2, self.dHo, ws)),
+            ("fc1_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY1, self.W1, self.dXo, ws)),
+            ("fc1_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY1, self.X, self.dW1, ws)),
+            ("fc2_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY2, self.H1, self.dW2, ws)),
+        ]
+        self.units = 6 * 2 * M * 768 * 3072
+        self.h2d = [self.X.mant, self.X.exp, self.dY1.mant, self.dY1.exp, self.dY2.mant, self.dY2.exp]
+        self.d2h = [self.dW1.mant, self.dW1.exp, self.dW2.mant, self.dW2.exp]
+
+    @staticmethod
+    def oracle_step(tokens):
+        import oracle
+
+        cfg = wl.vit_b_linear_trio(seed=0, tokens=tokens)
+        X, W1, W2, dY1, dY2 = (cfg[k] for k in ("X", "W1", "W2", "dY1", "dY2"))
+        t0 = time.perf_counter()
+        H1 = oracle.linear_fwd(X, W1, 1, 64)
+        oracle.linear_fwd(H1, W2, 1, 64)
+        oracle.linear_bwd_data(dY2, W2, 1, 64)
+        oracle.linear_bwd_data(dY1, W1, 1, 64)
+        oracle.linear_bwd_weight(dY1, X, 1, X.cols)
+        oracle.linear_bwd_weight(dY2, H1, 1, H1.cols)
+        dt = time.perf_counter() - t0
+        return dt, 6 * 2 * tokens * 768 * 3072, f"the six contractions on {tokens} of the 12608 tokens"
+
+
+class SgdStep(Step):
+    unit = "GB/s"
+    workload = {"workload": "resnet50_sgd_arena", "params": 25557032, "tensors": 161, "groups": 399329,
+                "group": 64, "bytes_per_step": 5 * 25557032 + 5 * 399329}
+
+    def __init__(self, ict, torch, seed):
+        super().__init__(ict, torch)
+        E = ict.DevCE
+        c5 = wl.resnet50_sgd_arena(seed=seed)
+        self.W, self.V, self.G = (E.from_host(c5[k]) for k in ("W", "V", "G"))
+        mom, lr = c5["sgd"]["mom"], c5["sgd"]["lr"]
+        self.calls = [("sgd", lambda: ict.ict_sgd_momentum_step(self.W, self.V, self.G, mom, lr))]
+        # algorithmic bytes: W, V, G mantissas read, W, V mantissas written (5 B per
+        # parameter) and the same for the per-group exponents (5 B per group)
+        self.units = 5 * c5["numel"] + 5 * self.W.rows
+        self.h2d = [self.G.mant, self.G.exp]
+        self.d2h = [self.W.mant, self.W.exp]
+
+    @staticmethod
+    def oracle_step(_):
+        import oracle
+
+        c5 = wl.resnet50_sgd_arena(seed=0)
+        t0 = time.perf_counter()
+        oracle.sgd_step(c5["W"], c5["V"], c5["G"], c5["sgd"]["mom"], c5["sgd"]["lr"])
+        dt = time.perf_counter() - t0
+        return dt, 5 * c5["numel"] + 5 * c5["W"].rows, "one full update of the 25.6 M-parameter arena"
+
+
+STEPS = {"vit_ti_mlp": MlpStep, "vit_b_linear_trio": TrioStep, "resnet18_conv3x3": ConvStep,
+         "resnet50_sgd": SgdStep, "single_linear": LinearStep}
+
+
+# --------------------------------------------------------------------- timing
+
+
+def backlog(torch, ms):
+    """Hold the stream with a spin kernel for about `ms` so that the host enqueues the
+    launches that follow before the GPU reaches them: events between them then time the
+    kernels, not the host's launch rate."""
+    torch.cuda._sleep(int(ms * 2.0e6))
+
+
+def time_graph(step, graph, K, W, flush):
+    """Mean device time per step (ms): one graph replay per step, CUDA events on the
+    replay stream, L2 flushed (512 MB write) before every step."""
+    torch = step.torch
+    for _ in range(W):
+        flush.fill_(1)
+        graph.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        flush.fill_(1)
+        a.record()
+        graph.replay()
+        b.record()
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+
+def time_eager(step, K, W, flush, backlogged):
+    """Mean device time per step (ms) with the calls launched one by one from Python,
+    and the per-call breakdown.  backlogged=True holds the stream first, so the events
+    time the kernels; False measures what a plain Python loop gets (host launch rate
+    included)."""
     torch = step.torch
     for _ in range(W):
         step.run()
@@ -190,34 +434,53 @@ def time_steps(step, K, W, flush):
     totals = []
     for _ in range(K):
         flush.fill_(1)
+        if backlogged:
+            backlog(torch, 1.0 + 0.1 * n)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         step.run(ev)
         torch.cuda.synchronize()
-        ms = [a.elapsed_time(b) for a, b in ev]
-        per_call += ms
+        per_call += [a.elapsed_time(b) for a, b in ev]
         totals.append(ev[0][0].elapsed_time(ev[-1][1]))
     return float(np.mean(totals)), per_call / K
 
 
-def time_e2e(step, K, W):
-    """Same step through the public API with host buffers: pinned H2D of the batch
-    (X, dY2 mantissas and exponents), the step, D2H of the updated weights."""
-    torch, ict = step.torch, step.ict
-    host_in = []
-    for t in (step.X, step.dY2):
-        host_in.append((t.mant.cpu().pin_memory(), t.mant))
-        host_in.append((t.exp.cpu().pin_memory(), t.exp))
-    host_out = []
-    for t in (step.W1, step.W2):
-        host_out.append((torch.empty_like(t.mant, device="cpu").pin_memory(), t.mant))
-        host_out.append((torch.empty_like(t.exp, device="cpu").pin_memory(), t.exp))
-    h2d = sum(h.numel() for h, _ in host_in)
-    d2h = sum(h.numel() for h, _ in host_out)
+def time_classes(step, K, flush):
+    """Device time per kernel class inside K steps: the library brackets each of its
+    kernels with CUDA events on the launch's stream while timing is enabled; the stream
+    is held first so that the events time kernels, not launch gaps."""
+    ict, torch = step.ict, step.torch
+    torch.cuda.synchronize()
+    ict.ict_timing_read(0, reset=True)
+    ict.ict_timing_enable(True)
+    for _ in range(K):
+        flush.fill_(1)
+        backlog(torch, 1.0 + 0.1 * len(step.calls))
+        step.run()
+    torch.cuda.synchronize()
+    ict.ict_timing_enable(False)
+    out = {}
+    for i, name in enumerate(CLASS_NAMES):
+        ms, n, work = ict.ict_timing_read(i, reset=False)
+        if n:
+            out[name] = {"ms_per_step": ms / K, "launches_per_step": n / K, "work_per_step": work / K}
+    ict.ict_timing_read(0, reset=True)
+    return out
+
+
+def time_e2e(step, graph, K, W):
+    """The same step through the public API with host buffers: pinned H2D copies of the
+    step's inputs, the step's graph, D2H copies of its results, all inside the timed
+    region."""
+    torch = step.torch
+    host_in = [(t.cpu().pin_memory(), t) for t in step.h2d]
+    host_out = [(torch.empty_like(t, device="cpu").pin_memory(), t) for t in step.d2h]
+    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
+    d2h = sum(h.numel() * h.element_size() for h, _ in host_out)
 
     def one():
         for h, d in host_in:
             d.copy_(h, non_blocking=True)
-        step.run()
+        graph.replay()
         for h, d in host_out:
             h.copy_(d, non_blocking=True)
 
@@ -233,138 +496,154 @@ def time_e2e(step, K, W):
     return a.elapsed_time(b) / K, h2d, d2h
 
 
-# --------------------------------------------------------------------- side measurements
+def class_rate(name, c, peaks):
+    """(achieved, peak, unit, bound) of one kernel class over its own device time."""
+    if name == "gemm":
+        return c["work_per_step"] / (c["ms_per_step"] * 1e-3) / 1e12, 2.0 * peaks["bf16"], "TFLOP/s", "tensor"
+    return c["work_per_step"] / (c["ms_per_step"] * 1e-3) / 1e9, peaks["hbm"], "GB/s", "hbm"
 
 
-def side_measurements(ict, torch, peaks):
+def kernel_source_digest():
+    """sha256 over the CUDA sources of libict.so (the kernels the counters describe)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "integer_only_nn_02_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(src, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(config, kernel_class):
+    """DRAM bytes per launch (read + write) of a kernel class in a configuration, from
+    the committed ncu summary, or None when the summary was taken on other kernel
+    sources or does not cover the class."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_sha256") != kernel_source_digest():
+        return None
+    e = t.get("configs", {}).get(config, {}).get(kernel_class)
+    return None if e is None else e["dram_bytes_per_launch"]
+
+
+def roofline(classes, peaks, config):
+    """Roofline of the kernel class with the most device time in the step: the
+    tensor-core Product against the INT8 peak (measured dense bf16 x 2, the nominal
+    int8/bf16 ratio), the memory-bound classes against the measured HBM copy rate."""
+    name = max(classes, key=lambda k: classes[k]["ms_per_step"])
+    c = classes[name]
+    achieved, peak, unit, bound = class_rate(name, c, peaks)
+    note = (f"INT8 = 2 x {peaks['source']} dense bf16 {peaks['bf16']} TF/s (burst)" if bound == "tensor"
+            else f"{peaks['source']} HBM copy bandwidth")
+    return {"kernel": CLASS_KERNELS[name], "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
+            "unit": unit, "frac": round(achieved / peak, 4), "peak_note": note,
+            "traffic": measured_traffic(config, name),
+            "launches_per_step": c["launches_per_step"],
+            "us_per_launch": round(1e3 * c["ms_per_step"] / c["launches_per_step"], 2)}
+
+
+def class_summary(classes, peaks):
     out = {}
-    E = ict.DevCE
-
-    def ev_time(fn, n=10, warm=3, flush=None):
-        for _ in range(warm):
-            fn()
-        ts = []
-        for _ in range(n):
-            if flush is not None:
-                flush.fill_(1)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return float(np.median(ts))
-
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    # ViT-B linear trio: six contractions of 59.49 GOP
-    c4 = wl.vit_b_linear_trio(seed=0)
-    X, W1, W2, dY1, dY2 = (E.from_host(c4[k]) for k in ("X", "W1", "W2", "dY1", "dY2"))
-    M = X.rows
-    H1 = E.empty(M, 3072, 1, 64)
-    Y2 = E.empty(M, 768, 1, 64)
-    dXa = E.empty(M, 768, 1, 64)
-    dHa = E.empty(M, 3072, 1, 64)
-    dW1 = E.empty(3072, 768, 1, 768)
-    dW2 = E.empty(768, 3072, 1, 3072)
-    wsz = max(ict.ict_linear_workspace(0, X, W1, H1), ict.ict_linear_workspace(0, H1, W2, Y2),
-              ict.ict_linear_workspace(1, dY2, W2, dHa), ict.ict_linear_workspace(1, dY1, W1, dXa),
-              ict.ict_linear_workspace(2, dY1, X, dW1), ict.ict_linear_workspace(2, dY2, H1, dW2))
-    ws = torch.empty(max(wsz, 256), dtype=torch.uint8, device="cuda")
-    gop = 2 * M * 768 * 3072 / 1e9
-    trio = {
-        "fc1_fwd": lambda: ict.ict_linear_fwd(X, W1, H1, ws),
-        "fc2_fwd": lambda: ict.ict_linear_fwd(H1, W2, Y2, ws),
-        "fc2_bwd_data": lambda: ict.ict_linear_bwd_data(dY2, W2, dHa, ws),
-        "fc1_bwd_data": lambda: ict.ict_linear_bwd_data(dY1, W1, dXa, ws),
-        "fc1_bwd_weight": lambda: ict.ict_linear_bwd_weight(dY1, X, dW1, ws),
-        "fc2_bwd_weight": lambda: ict.ict_linear_bwd_weight(dY2, H1, dW2, ws),
-    }
-    ms = {k: ev_time(f, flush=flush) for k, f in trio.items()}
-    tot = sum(ms.values())
-    out["vit_b_linear_trio"] = {
-        "tops": round(6 * gop / tot, 1), "ms_total": round(tot, 4),
-        "tops_each": {k: round(gop / v, 1) for k, v in ms.items()},
-        "note": "each call includes its exponent-alignment passes; 357.0 GOP per trio",
-    }
-    del X, W1, W2, dY1, dY2, H1, Y2, dXa, dHa, dW1, dW2, ws
-    # ResNet-50 SGD arena: 5 B per element + 5 B per group of 64
-    c5 = wl.resnet50_sgd_arena(seed=0)
-    Wd, Vd, Gd = (E.from_host(c5[k]) for k in ("W", "V", "G"))
-    nbytes = 5 * c5["numel"] + 5 * Wd.rows
-    t = ev_time(lambda: ict.ict_sgd_momentum_step(Wd, Vd, Gd, (230, 8), (205, 11)), n=20, flush=flush)
-    out["resnet50_sgd"] = {"gbs": round(nbytes / t / 1e6, 1), "us": round(t * 1e3, 2),
-                           "frac_hbm": round(nbytes / t / 1e6 / peaks["hbm"], 3),
-                           "bytes_per_step": nbytes}
-    del Wd, Vd, Gd
-    torch.cuda.empty_cache()
+    for name, c in classes.items():
+        d = {"ms_per_step": round(c["ms_per_step"], 4), "launches_per_step": c["launches_per_step"]}
+        if c["work_per_step"] > 0:
+            achieved, peak, unit, _ = class_rate(name, c, peaks)
+            d[unit] = round(achieved, 1)
+            d["frac"] = round(achieved / peak, 4)
+        out[name] = d
     return out
 
 
-# --------------------------------------------------------------------- oracle arm
+# --------------------------------------------------------------------- side measurements
 
 
-def oracle_step_time(tokens: int):
-    """The CPU oracle on the same step with `tokens` of the 12608 tokens."""
-    import oracle
-
-    cfg = wl.vit_ti_mlp(seed=0, tokens=tokens)
-    X, W1, W2, dY2 = cfg["X"], cfg["W1"], cfg["W2"], cfg["dY2"]
-    t0 = time.perf_counter()
-    H = oracle.linear_fwd(X, W1, 1, GROUP)
-    G = oracle.gelu_fwd(H)
-    oracle.linear_fwd(G, W2, 1, GROUP)
-    dG = oracle.linear_bwd_data(dY2, W2, 1, GROUP)
-    dW2 = oracle.linear_bwd_weight(dY2, G, 1, HID)
-    dH = oracle.gelu_bwd(H, dG, 1, GROUP)
-    oracle.linear_bwd_data(dH, W1, 1, GROUP)
-    dW1 = oracle.linear_bwd_weight(dH, X, 1, D)
-    oracle.sgd_step(W1, cfg["V1"], dW1, *cfg["sgd"].values())
-    oracle.sgd_step(W2, cfg["V2"], dW2, *cfg["sgd"].values())
-    dt = time.perf_counter() - t0
-    ops = 6 * 2 * tokens * D * HID
-    return dt, ops, oracle.num_threads()
+def side_int_mm(torch):
+    """torch._int_mm on 8192^3 (the library INT8 GEMM on this GPU), for context."""
+    try:
+        a = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device="cuda")
+        b = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device="cuda")
+        for _ in range(3):
+            torch._int_mm(a, b)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        return round(10 * 2 * 8192 ** 3 / (e0.elapsed_time(e1) * 1e-3) / 1e12, 1)
+    except Exception as exc:  # pragma: no cover
+        return f"unavailable: {exc}"
 
 
-def base_line(args, n_gpus):
+def side_measurements(ict, torch, peaks, flush, steps):
+    """The other configurations' step values (a few steps each), for context."""
+    out = {}
+    for name in ("vit_b_linear_trio", "resnet18_conv3x3", "resnet50_sgd", "single_linear"):
+        st = STEPS[name](ict, torch, 0)
+        graph = ict.StepGraph(st.run)
+        ms = time_graph(st, graph, steps, 3, flush)
+        _, per_call = time_eager(st, steps, 3, flush, backlogged=True)
+        classes = time_classes(st, steps, flush)
+        del graph
+        out[name] = {"value": round(st.value_of(st.units, ms * 1e-3), 2), "unit": st.unit,
+                     "ms_per_step": round(ms, 4),
+                     "breakdown_ms": {n: round(float(v), 4) for (n, _), v in zip(st.calls, per_call)},
+                     "kernel_classes": class_summary(classes, peaks)}
+        del st
+        torch.cuda.empty_cache()
+    out["torch_int_mm_8192_tops"] = side_int_mm(torch)
+    return out
+
+
+# --------------------------------------------------------------------- lines
+
+
+def base_line(args, step_cls, n_gpus):
+    cfg = dict(step_cls.workload)
+    cfg.update(parallelism=f"replicas{n_gpus}" if n_gpus > 1 else "single",
+               l2="flushed between steps (512 MB write)")
     return {
-        "metric": "(C,e) GEMM TOPS fwd+bwd vs INT8 tensor peak; int-SGD update GB/s vs HBM",
-        "unit": "TOPS", "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded; ViT-Ti layer shapes)",
-        "config": {"workload": "vit_ti_mlp_block_step", "tokens": TOKENS, "d": D, "hidden": HID,
-                   "group": GROUP, "gop_per_step": round(STEP_OPS / 1e9, 3),
-                   "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single",
-                   "l2": "flushed between steps (512 MB write)"},
+        "metric": METRIC, "unit": step_cls.unit, "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": step_cls.higher_is_better, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded; layer shapes of the paper's networks)", "config": cfg,
     }
 
 
+def cpu_baseline(step_cls):
+    import oracle
+
+    dt, units, sample = step_cls.oracle_step(step_cls.sample_arg)
+    return {"value": step_cls.value_of(units, dt), "unit": step_cls.unit, "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": sample, "seconds": round(dt, 3)}
+
+
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    """The oracle as it stands, timed on the host cores on a bounded sample of the
+    configuration's step (rank 0 only)."""
+    if int(os.environ.get("RANK", "0")) != 0:
         return
-    tokens = TOKENS
-    times = []
-    for _ in range(max(1, args.warmup // 3)):
-        oracle_step_time(tokens)
-    for _ in range(max(1, min(args.steps, 3))):
-        dt, ops, cores = oracle_step_time(tokens)
-        times.append(dt)
-    dt = float(np.mean(times))
-    value = ops / dt / 1e12
-    line = base_line(args, args.gpus)
+    step_cls = STEPS[args.config]
+    runs = [cpu_baseline(step_cls) for _ in range(max(1, min(args.steps, 3)))]
+    value = float(np.mean([r["value"] for r in runs]))
+    cb = dict(runs[-1], value=value, sample=runs[-1]["sample"] + f", mean of {len(runs)} runs")
+    line = base_line(args, step_cls, args.gpus)
     line.update({
-        "impl": "reference", "value": value, "ms_per_step": dt * 1e3 * TOKENS / tokens,
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
-                         "sample": f"{tokens} of {TOKENS} tokens per step, {len(times)} steps"},
-        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "impl": "reference", "value": value, "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": step_cls.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     })
     print(json.dumps(line))
 
 
 def main():
     args = parse()
-    if args.warmup < 3:
-        args.warmup = 3
+    args.warmup = max(args.warmup, 3)
+    if args.steps is None:
+        args.steps = 100 if args.config == "resnet50_sgd" else 20
     if args.impl == "reference":
         run_reference(args)
         return
@@ -384,7 +663,8 @@ def main():
     from integer_only_nn_02_b200 import ict
 
     peaks = load_peaks()
-    step = MlpStep(ict, seed=rank)
+    step_cls = STEPS[args.config]
+    step = step_cls(ict, torch, rank)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     step.run()
     torch.cuda.synchronize()
@@ -392,25 +672,23 @@ def main():
     if code != 0:
         raise SystemExit(f"device status {code} ({raw:#x})")
 
+    graph = ict.StepGraph(step.run)
     clocks = ClockSampler(torch.cuda.current_device())
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    launches0 = ict.ict_launch_count()
     clocks.start()
-    t0 = time.perf_counter()
-    ms, per_call = time_steps(step, args.steps, args.warmup, flush)
-    wall = time.perf_counter() - t0
+    ms = time_graph(step, graph, args.steps, args.warmup, flush)
     clk = clocks.stop()
-    launches = ict.ict_launch_count() - launches0
-    launches_per_step = launches / (args.steps + args.warmup)
-    torch.cuda.synchronize()
     if dist:
         t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
         dist.barrier()
-    e2e_ms, h2d, d2h = time_e2e(step, args.steps, args.warmup)
+    eager_ms, _ = time_eager(step, args.steps, args.warmup, flush, backlogged=False)
+    _, per_call = time_eager(step, args.steps, args.warmup, flush, backlogged=True)
+    classes = time_classes(step, args.steps, flush)
+    e2e_ms, h2d, d2h = time_e2e(step, graph, args.steps, args.warmup)
     if dist:
         t = torch.tensor([e2e_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -419,55 +697,32 @@ def main():
     if code != 0:
         raise SystemExit(f"device status {code} ({raw:#x})")
 
-    names = [n for n, _ in step.calls]
-    breakdown = {n: round(float(v), 4) for n, v in zip(names, per_call)}
-    # dominant kernel: fc1 forward is exactly one tensor-core launch (both operands are
-    # uniform along K), so its event time is the kernel's own duration
-    gemm_ms = breakdown["fc1_fwd"]
-    int8_peak = 2.0 * peaks["bf16"]  # measured bf16 dense x nominal int8/bf16 ratio (2)
-    achieved = (2 * TOKENS * D * HID) / (gemm_ms * 1e-3) / 1e12
-    value = STEP_OPS / (ms * 1e-3) / 1e12 * world
-    line = base_line(args, world)
+    agg = world if step.higher_is_better else 1  # rates add over independent replicas
+    line = base_line(args, step_cls, world)
     line.update({
-        "value": round(value, 2), "ms_per_step": round(ms, 4),
-        "e2e": {"value": round(STEP_OPS / (e2e_ms * 1e-3) / 1e12 * world, 2), "unit": "TOPS",
+        "value": round(step.value_of(step.units, ms * 1e-3) * agg, 3), "ms_per_step": round(ms, 4),
+        "e2e": {"value": round(step.value_of(step.units, e2e_ms * 1e-3) * agg, 3), "unit": step.unit,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": int(round(launches_per_step * args.steps)),
-        "gpu_launches_per_step": round(launches_per_step, 2),
-        "breakdown_ms": breakdown,
-        "roofline": {"kernel": "gemm_ce_kernel (fc1 forward, 12608x192 . 192x768)", "bound": "tensor",
-                     "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / int8_peak, 4),
-                     "peak_note": f"int8 = 2 x {peaks['source']} bf16 dense {peaks['bf16']} TF/s",
-                     "traffic": None},
+        "gpu_launches": int(graph.launches * args.steps),
+        "gpu_launches_per_step": graph.launches,
+        "launch": "one CUDA graph replay per step",
+        "eager_ms_per_step": round(eager_ms, 4),
+        "breakdown_ms": {n: round(float(v), 4) for (n, _), v in zip(step.calls, per_call)},
+        "kernel_classes": class_summary(classes, peaks),
+        "roofline": roofline(classes, peaks, args.config),
         "clocks": clk,
-        "wall_s_timed": round(wall, 3),
     })
-    if rank == 0 and not args.no_side:
-        line["side"] = side_measurements(ict, torch, peaks)
-        try:
-            a = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device="cuda")
-            b = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device="cuda")
-            for _ in range(3):
-                torch._int_mm(a, b)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(10):
-                torch._int_mm(a, b)
-            e1.record()
-            torch.cuda.synchronize()
-            line["side"]["torch_int_mm_8192_tops"] = round(10 * 2 * 8192 ** 3 / (e0.elapsed_time(e1) * 1e-3) / 1e12, 1)
-        except Exception as exc:  # pragma: no cover
-            line["side"]["torch_int_mm_8192_tops"] = f"unavailable: {exc}"
+    if rank == 0 and not args.no_side and args.config == "vit_ti_mlp":
+        del graph, step
+        torch.cuda.empty_cache()
+        line["side"] = side_measurements(ict, torch, peaks, flush, max(5, args.steps // 2))
     if rank == 0:
-        try:
-            dt, ops, cores = oracle_step_time(TOKENS)
-            line["cpu_baseline"] = {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": cores,
-                                    "kind": "oracle", "sample": f"one full step ({TOKENS} tokens)",
-                                    "seconds": round(dt, 2)}
-        except Exception as exc:  # pragma: no cover
-            line["cpu_baseline"] = {"value": None, "unit": "TOPS", "cores": None, "kind": "oracle",
-                                    "sample": f"failed: {exc}"}
+        if not args.no_cpu:
+            try:
+                line["cpu_baseline"] = cpu_baseline(step_cls)
+            except Exception as exc:  # pragma: no cover
+                line["cpu_baseline"] = {"value": None, "unit": step_cls.unit, "cores": None, "kind": "oracle",
+                                        "sample": f"failed: {exc}"}
         print(json.dumps(line))
     if dist:
         dist.barrier()

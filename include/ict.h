@@ -124,10 +124,11 @@ uint64_t ict_launch_count(void);
 typedef enum {
     ICT_KC_GEMM = 0,    /* tensor-core Product kernels (linear, conv) */
     ICT_KC_SGD = 1,     /* integer SGD-with-momentum update */
-    ICT_KC_ALIGN = 2,   /* exponent alignment (ALIGN_MAX) and weight re-layout */
+    ICT_KC_ALIGN = 2,   /* ALIGN_MAX mantissa shifts (and transposes) */
     ICT_KC_REQUANT = 3, /* FIT of int32 / int64 values (split-K combine) */
     ICT_KC_GELU = 4,    /* GELU forward / backward */
-    ICT_KC_OTHER = 5    /* fills and exponent tables */
+    ICT_KC_ESTAR = 5,   /* target exponents e* of ALIGN_MAX (maxima of group exponents) */
+    ICT_KC_OTHER = 6    /* fills, weight re-layout and exponent tables */
 } ict_kernel_class;
 int32_t ict_timing_enable(int32_t on);
 int32_t ict_timing_read(int32_t kernel_class, double *ms_total, int64_t *launches, double *work,

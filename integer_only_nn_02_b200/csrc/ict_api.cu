@@ -61,7 +61,7 @@ std::atomic<uint64_t> g_launches{0};
 void counted(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 // ---- optional per-kernel-class device timing (measurement only; off by default)
-enum { KC_GEMM = 0, KC_SGD = 1, KC_ALIGN = 2, KC_REQUANT = 3, KC_GELU = 4, KC_OTHER = 5, KC_N = 6 };
+enum { KC_GEMM = 0, KC_SGD = 1, KC_ALIGN = 2, KC_REQUANT = 3, KC_GELU = 4, KC_ESTAR = 5, KC_OTHER = 6, KC_N = 7 };
 struct TimedLaunch {
     int kc;
     cudaEvent_t a, b;
@@ -96,6 +96,8 @@ struct KTimer {
     KTimer(cudaStream_t s_, int kc_, double work_) : s(s_), kc(kc_), work(work_) {
         std::lock_guard<std::mutex> lk(g_timing_mu);
         if (!g_timing.on) return;
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
         a = timing_event();
         if (a) cudaEventRecord(a, s);
     }
@@ -232,23 +234,25 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     int sms = 148;
     device_info(&sms);
     const int64_t n_exp = n_grp_rows(in) * a.ngc;
-    KTimer kt(s, KC_ALIGN, 2.0 * (double)in->rows * (double)in->cols);
     if (j.axis == 1) {
+        KTimer kt(s, KC_ESTAR, (double)n_exp + (double)in->rows);
         estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
-    } else if (j.col_max && a.ngc <= 8192) {
-        // every thread keeps one group column: a stride that is a multiple of ngc
+    } else {
+        // every thread of the scratch form keeps one group column: a stride that is a
+        // multiple of ngc
         const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(n_exp, 256 * 8), (int64_t)sms * 4));
         const int64_t used = (blocks * 256) / a.ngc * a.ngc;
-        if (used >= a.ngc) {
+        if (j.col_max && a.ngc <= 8192 && used >= a.ngc) {
             if (cudaMemsetAsync(j.col_max, 0x80, (size_t)a.ngc * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
+            KTimer kt(s, KC_ESTAR, (double)n_exp + 8.0 * (double)a.ngc);
             estar_cols_scratch_kernel<<<(unsigned)blocks, 256, (size_t)a.ngc * 4, s>>>(a, j.col_max, used);
             a.col_max = j.col_max;
         } else {
+            KTimer kt(s, KC_ESTAR, (double)n_exp + (double)in->cols);
             estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
         }
-    } else {
-        estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
     }
+    KTimer kt(s, KC_ALIGN, 2.0 * (double)in->rows * (double)in->cols + (double)n_exp);
     dim3 grid((unsigned)cdiv64(in->cols, 64), (unsigned)cdiv64(in->rows, 64));
     if (j.transpose)
         align_tile_kernel<true><<<grid, 256, 0, s>>>(a);
@@ -291,6 +295,7 @@ int launch_zero(const ict_tensor *out, cudaStream_t s) {
     const int64_t n = out->rows * out->cols, ne = n_grp_rows(out) * n_grp_cols(out);
     const int64_t m = n > ne ? n : ne;
     if (m == 0) return ICT_OK;
+    KTimer kt(s, KC_OTHER, (double)n + (double)ne);
     zero_ce_kernel<<<(unsigned)cdiv64(m, 256), 256, 0, s>>>(out->mant, out->rows, out->cols, out->ld,
                                                            out->exp, ne);
     counted(1);
@@ -687,8 +692,12 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     for (int i = 0; i < cp.njobs; ++i)
         if ((st = launch_align(cp.jobs[i], s))) return st;
     if (cp.weight_prep) {
-        conv_wt_estar_kernel<<<d->c, 256, 0, s>>>(cp.wprep);
         const int64_t n = (int64_t)d->c * d->r * d->s * d->k;
+        {
+            KTimer kt(s, KC_ESTAR, (double)n);
+            conv_wt_estar_kernel<<<d->c, 256, 0, s>>>(cp.wprep);
+        }
+        KTimer kt(s, KC_OTHER, 2.0 * (double)n);
         conv_wt_prep_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(cp.wprep);
         counted(2);
         if ((st = launch_status())) return st;
@@ -736,7 +745,10 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         p.epi = EPI_FIT_ROW;
         return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
     }
-    fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
+    {
+        KTimer kt(s, KC_OTHER, 4.0 * (double)cp.n_gcols);
+        fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
+    }
     counted(1);
     p.epi = EPI_NEED_GLOBAL;  // the first pass is recompute: its work is not counted again
     if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
@@ -799,9 +811,12 @@ int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X,
               const WgradPlan &wp, int sms, cudaStream_t s) {
     int st;
     const int RS = d->r * d->s;
-    conv_wgrad_exp_kernel<<<(unsigned)cdiv64(std::max<int64_t>(wp.M, wp.N), 256), 256, 0, s>>>(
-        X->exp, clamp_div(X->g_cols, X->cols), dY->exp, clamp_div(dY->g_cols, dY->cols), d->c, RS, d->k,
-        wp.e_rows, wp.e_cols);
+    {
+        KTimer kt(s, KC_OTHER, 2.0 * (double)(wp.M + wp.N));
+        conv_wgrad_exp_kernel<<<(unsigned)cdiv64(std::max<int64_t>(wp.M, wp.N), 256), 256, 0, s>>>(
+            X->exp, clamp_div(X->g_cols, X->cols), dY->exp, clamp_div(dY->g_cols, dY->cols), d->c, RS, d->k,
+            wp.e_rows, wp.e_cols);
+    }
     counted(1);
     if ((st = launch_status())) return st;
     CUtensorMap ta, tb;

@@ -175,7 +175,7 @@ def ict_launch_count() -> int:
     return int(lib.ict_launch_count())
 
 
-KERNEL_CLASSES = {"gemm": 0, "sgd": 1, "align": 2, "requant": 3, "gelu": 4, "other": 5}
+KERNEL_CLASSES = {"gemm": 0, "sgd": 1, "align": 2, "requant": 3, "gelu": 4, "estar": 5, "other": 6}
 
 
 def ict_timing_enable(on: bool) -> None:
@@ -339,3 +339,32 @@ def gelu_bwd(H: DevCE, dG: DevCE, stream=None) -> DevCE:
 def device_status(stream=None) -> int:
     code, _ = ict_get_device_status(stream)
     return code
+
+
+class StepGraph:
+    """A fixed sequence of library calls (for instance one training step) captured into
+    one CUDA graph and replayed with a single launch.
+
+    ``fn`` issues the calls on torch's current stream.  It runs ``warmup`` times eagerly
+    on a side stream first (one-time host setup such as kernel attributes happens
+    there), then once under capture.  Every tensor and workspace ``fn`` touches must
+    stay alive, at the same address, for the life of the graph; each replay reruns all
+    calls, including in-place updates (an SGD step advances the weights every replay).
+    """
+
+    def __init__(self, fn, warmup: int = 1):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        n0 = ict_launch_count()
+        with torch.cuda.graph(self.graph, capture_error_mode="relaxed"):
+            fn()
+        self.launches = ict_launch_count() - n0  # kernels in one replay
+
+    def replay(self) -> None:
+        self.graph.replay()
