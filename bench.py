@@ -42,7 +42,7 @@ CLASS_NAMES = ["gemm", "sgd", "align", "requant", "gelu", "estar", "other"]  # i
 CLASS_KERNELS = {
     "gemm": "gemm_ce_kernel (tcgen05 kind::i8, fused FIT epilogue)",
     "sgd": "sgd_rows_kernel / sgd_vec_kernel",
-    "align": "align_tile_kernel (ALIGN_MAX shifts, transposes)",
+    "align": "align_rows_kernel / align_transpose_kernel (ALIGN_MAX shifts)",
     "requant": "requant_group_block_kernel / requant_rows_kernel",
     "gelu": "gelu_fwd_kernel / gelu_bwd_vec_kernel",
     "estar": "estar_rows_kernel / estar_cols_scratch_kernel",

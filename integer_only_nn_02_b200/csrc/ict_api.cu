@@ -235,8 +235,12 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     device_info(&sms);
     const int64_t n_exp = n_grp_rows(in) * a.ngc;
     if (j.axis == 1) {
-        KTimer kt(s, KC_ESTAR, (double)n_exp + (double)in->rows);
-        estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
+        if (j.transpose) {
+            KTimer kt(s, KC_ESTAR, (double)n_exp + (double)in->rows);
+            estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
+        } else {
+            a.row_estar = 1;  // computed inside align_rows_kernel
+        }
     } else {
         // every thread of the scratch form keeps one group column: a stride that is a
         // multiple of ngc
@@ -253,12 +257,11 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
         }
     }
     KTimer kt(s, KC_ALIGN, 2.0 * (double)in->rows * (double)in->cols + (double)n_exp);
-    dim3 grid((unsigned)cdiv64(in->cols, 64), (unsigned)cdiv64(in->rows, 64));
     if (j.transpose)
-        align_tile_kernel<true><<<grid, 256, 0, s>>>(a);
+        align_transpose_kernel<<<dim3((unsigned)cdiv64(in->cols, 128), (unsigned)cdiv64(in->rows, 128)), 256, 0, s>>>(a);
     else
-        align_tile_kernel<false><<<grid, 256, 0, s>>>(a);
-    counted(2);
+        align_rows_kernel<<<dim3((unsigned)cdiv64(in->cols, 64), (unsigned)cdiv64(in->rows, 64)), 256, 0, s>>>(a);
+    counted(a.row_estar ? 1 : 2);
     return launch_status();
 }
 
@@ -324,8 +327,13 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
 }
 
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
-                const GemmParams &p, int grid, cudaStream_t s, double ops) {
+                const GemmParams &p_in, int grid, cudaStream_t s, double ops) {
     KTimer kt(s, KC_GEMM, ops);
+    // both epilogue warpgroups take every tile (one column half each) when no output
+    // group straddles the halves
+    GemmParams p = p_in;
+    const int gt = p.G >= p.N ? bn : p.G;
+    p.epi_split = p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0);
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
     if (bn == BN_ && bk == BK_ && load == LOAD_) \
         return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s);
@@ -365,7 +373,9 @@ int pick_bn_waves(int64_t M, int64_t N, int64_t G, int sms) {
         const int64_t tiles = cdiv64(M, 128) * cdiv64(N, bn);
         const int64_t waves = cdiv64(tiles, sms);
         const double eff = (double)(M * N) / (double)(waves * sms * 128 * bn);
-        const double score = eff * (1.0 + 0.03 * bn / 64.0);
+        // widths whose halves hold whole groups let both epilogue warpgroups share a tile
+        const bool halves = G >= N || (bn / 2) % G == 0;
+        const double score = eff * (1.0 + 0.05 * bn / 64.0) * (halves ? 1.15 : 1.0);
         if (score > best_score) best_score = score, best = bn;
     }
     return best ? best : pick_bn(N);

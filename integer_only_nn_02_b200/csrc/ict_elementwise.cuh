@@ -132,6 +132,7 @@ struct AlignArgs {
     int64_t out_ld;
     int8_t *e_star;           // [rows] (axis 1) or [cols] (axis 0)
     const int32_t *col_max;   // axis 0 with scratch: max per group column (<= kNoExp: none)
+    int row_estar;            // axis 1: the alignment kernel computes and stores e* itself
 };
 
 __device__ __forceinline__ int estar_of(int m) { return m <= kNoExp ? kEZero : m; }
@@ -193,69 +194,125 @@ __global__ void __launch_bounds__(256) estar_cols_scratch_kernel(AlignArgs a, in
         if (sm[g] > kNoExp) atomicMax(&col_max[g], sm[g]);
 }
 
-// Aligned mantissas, 64 x 64 tiles of 16-byte vectors (cols and, when transposed,
-// rows are multiples of 16; g_cols is a multiple of 16 or spans all columns, so every
-// 16-byte vector has one group exponent and one target exponent).
-template <bool TRANSPOSE>
-__global__ void __launch_bounds__(256) align_tile_kernel(AlignArgs a) {
-    __shared__ uint8_t tile[64][64 + 4];
-    const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
-    const int tr = threadIdx.x >> 2, tc = (threadIdx.x & 3) * 16;
-    const int64_t i = r0 + tr, j = c0 + tc;
-    uint32_t w[4] = {0, 0, 0, 0};
+// RNE(C / 2^d) of 16 signed int8 mantissas (|C| <= 127), d >= 0.  d = 0 is a copy and
+// d >= 8 gives 0.  For 1 <= d <= 7 one fp32 FMA per byte computes it exactly:
+//   f = 2^23 + (C + 128)                      (bits 0x4B0000uu, uu = C ^ 0x80)
+//   f * 2^-d + (1.5 * 2^23 - 2^(23-d) - 2^(7-d)) = 1.5 * 2^23 + C * 2^-d
+// Every operand is exact in fp32.  The FMA rounds once, to the nearest integer with
+// ties to even, since its result lies in [2^23, 2^24) where the spacing is 1.  So the
+// low byte of the result's bits is RNE(C / 2^d) in two's complement.  The work runs on
+// the FMA pipe; the ALU only builds the operands and packs the bytes.
+__device__ __forceinline__ uint4 rne_shift16(uint4 raw, int d) {
+    if (d == 0) return raw;
+    if (d >= 8) return make_uint4(0, 0, 0, 0);
+    const float sc = __int_as_float((127 - d) << 23);
+    const float k = 12582912.0f - (float)(1 << (23 - d)) - (float)(1 << (7 - d));
+    const uint32_t src[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t r[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            r[b] = __float_as_uint(__fmaf_rn(__uint_as_float(__byte_perm(src[q], 0x4B000000u, 0x7650 | b)), sc, k));
+        o[q] = __byte_perm(__byte_perm(r[0], r[1], 0x0040), __byte_perm(r[2], r[3], 0x0040), 0x5410);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Target exponent of the 16-byte vector at column j of row i (axis 1: per row; axis 0:
+// per column, from the column-max scratch or the e* vector).
+__device__ __forceinline__ int align_target(const AlignArgs &a, int64_t i, int64_t j) {
+    if (a.axis == 1) return i < a.rows ? a.e_star[i] : kEZero;
+    if (a.col_max) return estar_of(a.col_max[j / a.g_cols]);
+    return a.e_star[j];
+}
+
+// The aligned 16-byte vector at (i, j): each vector has one group exponent and one target.
+__device__ __forceinline__ uint4 align_vec(const AlignArgs &a, int64_t i, int64_t j, int es) {
+    if (i >= a.rows) return make_uint4(0, 0, 0, 0);
+    const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
+    const int eg = a.in_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+    if (eg == kEZero) return make_uint4(0, 0, 0, 0);
+    return rne_shift16(raw, min(es - eg, 8));  // |C| <= 127: shifts of 8 or more give 0
+}
+
+// Aligned mantissas in place of layout, 64 x 64 tiles of 16-byte vectors (cols are a
+// multiple of 16; g_cols is a multiple of 16 or spans all columns).
+// With axis 1 and no precomputed e*, the four threads of a row compute the row's e*
+// themselves (a quarter of its group exponents each, then two shuffles) and the first
+// of them stores it.
+__global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
+    const int64_t i = (int64_t)blockIdx.y * 64 + (threadIdx.x >> 2);
+    const int64_t j = (int64_t)blockIdx.x * 64 + (threadIdx.x & 3) * 16;
+    if (i >= a.rows) return;  // whole 4-thread row groups leave together
+    int es;
+    if (a.axis == 1 && a.row_estar) {
+        const int8_t *e = a.in_exp + (i / a.g_rows) * a.ngc;
+        int m = kNoExp;
+        for (int64_t g = threadIdx.x & 3; g < a.ngc; g += 4)
+            if (e[g] != kEZero) m = max(m, (int)e[g]);
+        const unsigned quad = 0xfu << (threadIdx.x & 28);
+        m = max(m, __shfl_xor_sync(quad, m, 1));
+        m = max(m, __shfl_xor_sync(quad, m, 2));
+        es = estar_of(m);
+        if (blockIdx.x == 0 && (threadIdx.x & 3) == 0) a.e_star[i] = (int8_t)es;
+    } else {
+        es = align_target(a, i, j);
+    }
+    if (j >= a.cols) return;
+    if (a.axis == 0 && a.col_max && i == 0)
+        for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
+    *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) = align_vec(a, i, j, es);
+}
+
+// Aligned and transposed, 128 x 128 tiles (rows and cols are multiples of 16).  Thread
+// (warp w, lane l) aligns rows 16 w + 4 (l & 3) .. + 3 at columns 16 (l >> 2) .. + 15,
+// transposes the 4 x 4 byte blocks in registers (8 byte permutes per 16 bytes) and
+// stores 32-bit words into a shared tile whose 16-byte chunks are XOR-swizzled by the
+// output row's 16-row band, so that both the word stores and the 16-byte reads that
+// feed the coalesced global stores are free of bank conflicts.
+__global__ void __launch_bounds__(256) align_transpose_kernel(AlignArgs a) {
+    __shared__ uint4 tile[128][8];  // [output row = input column][16-byte chunk, swizzled]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r0 = (int64_t)blockIdx.y * 128, c0 = (int64_t)blockIdx.x * 128;
+    const int rq = 4 * warp + (lane & 3), cc = lane >> 2;  // row quad 0..31, column chunk 0..7
+    const int64_t j = c0 + 16 * cc;
     if (j < a.cols) {
-        int es;
-        if (a.axis == 1) {
-            es = i < a.rows ? a.e_star[i] : kEZero;
-        } else if (a.col_max) {
-            es = estar_of(a.col_max[j / a.g_cols]);
-            if (blockIdx.y == 0 && tr == 0)
-                for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
-        } else {
-            es = a.e_star[j];
+        if (a.axis == 0 && a.col_max && blockIdx.y == 0 && rq == 0) {
+            const int es = align_target(a, 0, j);
+            for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
         }
-        if (i < a.rows) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
-            const int eg = a.in_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
-            if (eg != kEZero) {
-                const int d = min(es - eg, 8);  // |C| <= 127: shifts of 8 or more give 0
-                if (d == 0) {
-                    w[0] = raw.x, w[1] = raw.y, w[2] = raw.z, w[3] = raw.w;
-                } else {
-                    const int bias = (1 << (d - 1)) - 1;
-                    const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint4 v[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        int r[4];
+        for (int t = 0; t < 4; ++t) {
+            const int64_t i = r0 + 4 * rq + t;
+            v[t] = align_vec(a, i, j, align_target(a, i, j));
+        }
+        const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w}, {v[1].x, v[1].y, v[1].z, v[1].w},
+                                  {v[2].x, v[2].y, v[2].z, v[2].w}, {v[3].x, v[3].y, v[3].z, v[3].w}};
+        uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
 #pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            const int c = sx8(src[q], b);
-                            r[b] = (c + bias + ((c >> d) & 1)) >> d;
-                        }
-                        w[q] = pack4(r[0], r[1], r[2], r[3]);
-                    }
-                }
+        for (int q = 0; q < 4; ++q) {  // columns 16 cc + 4 q .. + 3
+            const uint32_t t0 = __byte_perm(w[0][q], w[1][q], 0x5140), t1 = __byte_perm(w[0][q], w[1][q], 0x7362);
+            const uint32_t t2 = __byte_perm(w[2][q], w[3][q], 0x5140), t3 = __byte_perm(w[2][q], w[3][q], 0x7362);
+            const uint32_t col[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
+                                     __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632)};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int orow = 16 * cc + 4 * q + k;                 // output row in the tile
+                const int chunk = (rq >> 2) ^ cc;                     // swizzled 16-byte chunk
+                tw[orow * 32 + chunk * 4 + (rq & 3)] = col[k];
             }
         }
     }
-    if constexpr (!TRANSPOSE) {
-        if (i < a.rows && j < a.cols)
-            *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
+    __syncthreads();
 #pragma unroll
-        for (int b = 0; b < 16; ++b) tile[tc + b][tr] = (uint8_t)(w[b >> 2] >> (8 * (b & 3)));
-        __syncthreads();
-        // output row = input column c0 + tr, output columns = input rows r0 + tc .. + 15
-        const int64_t oi = c0 + tr, oj = r0 + tc;
-        if (oi < a.cols && oj < a.rows) {
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                o[q] = (uint32_t)tile[tr][tc + 4 * q] | ((uint32_t)tile[tr][tc + 4 * q + 1] << 8) |
-                       ((uint32_t)tile[tr][tc + 4 * q + 2] << 16) |
-                       ((uint32_t)tile[tr][tc + 4 * q + 3] << 24);
-            *reinterpret_cast<uint4 *>(a.out + oi * a.out_ld + oj) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
+    for (int pass = 0; pass < 4; ++pass) {
+        const int orow = pass * 32 + (threadIdx.x >> 3), m = threadIdx.x & 7;
+        const int64_t oi = c0 + orow, oj = r0 + 16 * m;
+        if (oi < a.cols && oj < a.rows)
+            *reinterpret_cast<uint4 *>(a.out + oi * a.out_ld + oj) = tile[orow][m ^ (orow >> 4)];
     }
 }
 

@@ -70,6 +70,7 @@ struct GemmParams {
     uint32_t stage_tx_bytes;
     uint64_t wait_ns, drain_ns;
     int epi;
+    int epi_split;  // 1: both epilogue warpgroups share every tile, one half of its columns each
 };
 
 template <int BN, int BK, int STAGES>
@@ -93,6 +94,76 @@ struct GemmSmem {
 
 __device__ __forceinline__ uint32_t pack4b(int a, int b, int c, int d) {
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Fast epilogue of one output group of 32 columns of an accumulator row, the group on
+// the fast path: y = acc * 2^d_n (d_n = column shift inside the group, |y| < 2^30), the
+// group exponent from max |y|, then one RNE shift.  The multiplies and the high-half
+// multiplies of the rounding shift run on the FMA pipe, leaving compares, the rounding
+// bit and the byte packing to the ALU pipe; TMEM is read once.
+template <bool MUL>  // MUL = false: every column of the group has the same exponent
+__device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
+                                           bool valid, int ea, int64_t grow, int ncol, int gcol, int et) {
+    uint32_t v[32];
+    tmem_ld32(taddr, v);
+    tmem_ld_wait();
+    int hi = 0, lo = 0;
+#pragma unroll
+    for (int q = 0; q < 32; q += 4) {
+        int y0 = (int)v[q], y1 = (int)v[q + 1], y2 = (int)v[q + 2], y3 = (int)v[q + 3];
+        if (MUL) {
+            const int4 m4 = *reinterpret_cast<const int4 *>(colM + q);
+            y0 *= m4.x, y1 *= m4.y, y2 *= m4.z, y3 *= m4.w;
+            v[q] = (uint32_t)y0, v[q + 1] = (uint32_t)y1, v[q + 2] = (uint32_t)y2, v[q + 3] = (uint32_t)y3;
+        }
+        hi = max(hi, max(max(y0, y1), max(y2, y3)));
+        lo = min(lo, min(min(y0, y1), min(y2, y3)));
+    }
+    const int amax = valid ? max(hi, -lo) : 0;
+    const int need = amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp;
+    if (p.epi == EPI_NEED_GLOBAL) {
+        const int m = warp_max(need);
+        if ((threadIdx.x & 31) == 0 && m > kNoExp && ncol < p.N) atomicMax(p.gmax + gcol, m);
+        return;
+    }
+    const int e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : need);
+    // mantissa = RNE(y * 2^-S), S = e - ea - gm uniform over the row's group
+    const int S = (e == kEZero) ? 0 : e - ea - gm;
+    if (__any_sync(0xffffffffu, valid && S < 0)) {
+        const int lm = S < 0 ? (1 << min(-S, 30)) : 1;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = (uint32_t)((int)v[q] * lm);
+    }
+    const int rs = S > 0 ? min(S, 31) : 0;
+    if (rs >= 2) {
+        const int m = 1 << (32 - rs), bias = (1 << (rs - 1)) - 1;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int y = (int)v[q];
+            v[q] = (uint32_t)__mulhi(y + bias + (__mulhi(y, m) & 1), m);
+        }
+    } else if (rs == 1) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int y = (int)v[q];
+            v[q] = (uint32_t)((y + ((y >> 1) & 1)) >> 1);
+        }
+    }
+    if (ncol < p.N) {
+        if (p.epi == EPI_FIT_ROW && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
+        if (p.epi == EPI_FIT_GLOBAL && et == 0) p.out_exp[gcol] = (int8_t)e;
+    }
+    if (valid) {
+        int8_t *dst = p.out + grow * p.out_ld + ncol;
+#pragma unroll
+        for (int q = 0; q < 32; q += 16)
+            if (ncol + q < p.N)
+                *reinterpret_cast<uint4 *>(dst + q) = make_uint4(
+                    pack4b((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
+                    pack4b((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
+                    pack4b((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
+                    pack4b((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+    }
 }
 
 template <int BN, int BK, int STAGES, int LOAD>
@@ -122,7 +193,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
-            mbar_init(bar_tempty + 8 * a, 128);
+            mbar_init(bar_tempty + 8 * a, p.epi_split ? 256 : 128);
         }
         mbar_init(bar_drain, 1);
         misc[1] = 0;
@@ -262,7 +333,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
-        const int wg = (warp - 4) >> 2;           // warpgroup: owns accumulator buffer wg
+        const int wg = (warp - 4) >> 2;           // warpgroup (alternating tiles, or one column half)
         const int et = (threadIdx.x & 127);       // output row within the tile = TMEM lane
         const int quarter = warp & 3, wq = (warp - 4) & 3;
         const int bar_id = 1 + wg;
@@ -272,15 +343,18 @@ __global__ void __launch_bounds__(384, 1)
         int *gfast = gmin + 8;                     // [8]  group takes the fast path
         const int Gt = p.G >= p.N ? BN : p.G;      // group width inside the tile
         const int ngroups = BN / Gt;
-        int it = wg;
+        // split: every tile, groups [g_lo, g_hi) of it; else every other tile, all groups
+        const int g_lo = p.epi_split ? wg * (ngroups >> 1) : 0;
+        const int g_hi = p.epi_split ? g_lo + (ngroups >> 1) : ngroups;
+        const int c_lo = p.epi_split ? wg * (BN / 2) : 0, c_hi = p.epi_split ? c_lo + BN / 2 : BN;
+        const int u_step = p.epi_split ? gridDim.x : 2 * gridDim.x, it_step = p.epi_split ? 1 : 2;
+        int it = p.epi_split ? 0 : wg;
         // The loop never tests the abort flag on its own: the 128 threads decide together
         // through a barrier reduction, so none of them can be left waiting at a barrier.
-        for (int u = blockIdx.x + wg * gridDim.x; u < p.num_units; u += 2 * gridDim.x, it += 2) {
-            const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
+        // Geometry of unit u: first output row, valid rows, first output column.
+        auto geometry = [&](int u, int64_t &row_base, int &valid_rows, int &n0) {
+            const int tile = u % (p.n_mtiles * p.n_ntiles);
             const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
-            const int acc = it & 1;
-            int64_t row_base;
-            int valid_rows;
             if (LOAD == LOAD_CONV) {
                 const int img = mt / p.cv_tiles_per_img;
                 const int h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
@@ -290,12 +364,36 @@ __global__ void __launch_bounds__(384, 1)
                 row_base = (int64_t)mt * 128;
                 valid_rows = min(128, p.M - mt * 128);
             }
-            const int n0 = nt * BN;
+            n0 = nt * BN;
+        };
+        // The exponents a tile needs (two column exponents and one row exponent per
+        // thread) are loaded one tile ahead, so their latency hides behind the previous
+        // tile's epilogue.
+        int pf_e0 = kEZero, pf_e1 = kEZero, pf_ea = 0;
+        auto prefetch = [&](int u) {
+            if (u >= p.num_units) return;
+            int64_t rb;
+            int vr, c0;
+            geometry(u, rb, vr, c0);
+            const int n_a = c0 + et, n_b = c0 + et + 128;
+            pf_e0 = n_a < p.N ? (int)p.eB[p.eB_div == 1 ? n_a : n_a / p.eB_div] : kEZero;
+            pf_e1 = (et + 128 < BN && n_b < p.N) ? (int)p.eB[p.eB_div == 1 ? n_b : n_b / p.eB_div] : kEZero;
+            const int64_t r = rb + et;
+            pf_ea = et < vr ? (int)p.eA[p.eA_div == 1 ? r : r / p.eA_div] : 0;
+        };
+        const int u0 = blockIdx.x + (p.epi_split ? 0 : wg * gridDim.x);
+        prefetch(u0);
+        for (int u = u0; u < p.num_units; u += u_step, it += it_step) {
+            const int split = u / (p.n_mtiles * p.n_ntiles);
+            const int acc = it & 1;
+            int64_t row_base;
+            int valid_rows, n0;
+            geometry(u, row_base, valid_rows, n0);
             // column tables of this tile (independent of the accumulator: built before waiting)
-            for (int j = et; j < BN; j += 128) {
-                const int n = n0 + j;
-                colE[j] = n < p.N ? (int)p.eB[n / p.eB_div] : kEZero;
-            }
+            colE[et] = pf_e0;
+            if (et + 128 < BN) colE[et + 128] = pf_e1;
+            const int ea_pf = pf_ea;
+            prefetch(u + u_step);
             named_bar_sync(bar_id, 128);
             for (int g = wq; g < ngroups; g += 4) {
                 int lo = 0x7fffffff, hi = kNoExp;
@@ -310,13 +408,15 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 if (lane == 0) {
                     gmin[g] = hi <= kNoExp ? 0 : lo;
-                    gfast[g] = hi <= kNoExp || hi - lo <= p.fast_slack;
+                    // 2: every column has the same exponent (no column shifts); 1: fast path
+                    gfast[g] = (hi <= kNoExp || hi == lo) ? 2 : (hi - lo <= p.fast_slack ? 1 : 0);
                 }
             }
             named_bar_sync(bar_id, 128);
-            for (int j = et; j < BN; j += 128) {
+            for (int j = et; j < BN; j += 128) {  // 2^d of each column (fast groups: d <= 30)
                 const int e = colE[j];
-                colD[j] = e == kEZero ? 0 : e - gmin[j / Gt];
+                const int d = e == kEZero ? 0 : e - gmin[j / Gt];
+                colD[j] = d <= 30 ? 1 << d : 0;
             }
             const bool ok = mbar_wait(bar_tfull + 8 * acc, (it >> 1) & 1, p.wait_ns, abort_flag);
             if (!ok) fail();
@@ -325,13 +425,14 @@ __global__ void __launch_bounds__(384, 1)
 
             const bool valid = et < valid_rows;
             const int64_t grow = row_base + et;
-            const int ea = valid ? (int)p.eA[grow / p.eA_div] : 0;
+            const int ea = valid ? ea_pf : 0;
+            const int gcol0 = n0 / p.G;  // output group of the tile's first column
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
             uint32_t v[32];
 
             if (p.epi == EPI_I32) {
                 int32_t *dst = p.ws32 + split * p.ws_split_stride + grow * p.ws_ld + n0;
-                for (int c = 0; c < BN; c += 32) {
+                for (int c = c_lo; c < c_hi; c += 32) {
                     tmem_ld32(taddr + c, v);
                     tmem_ld_wait();
                     if (valid) {
@@ -343,12 +444,20 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
             } else {
-                for (int g = 0; g < ngroups; ++g) {
+                for (int g = g_lo; g < g_hi; ++g) {
                     const int g0 = g * Gt;
-                    const int gcol = (n0 + g0) / p.G;
+                    const int gcol = gcol0 + g;
+                    const int gf = gfast[g];
+                    if (Gt == 32 && gf) {
+                        if (gf == 2)
+                            epi_fast32<false>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol, et);
+                        else
+                            epi_fast32<true>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol, et);
+                        continue;
+                    }
                     const int gm = gmin[g];
                     int e;
-                    if (gfast[g]) {
+                    if (gf) {
                         // |x << d| < 2^30: the group exponent follows from the largest magnitude
                         int ymax = 0, ymin = 0;
                         for (int c = g0; c < g0 + Gt; c += 32) {
@@ -357,9 +466,9 @@ __global__ void __launch_bounds__(384, 1)
                             if (valid) {
 #pragma unroll
                                 for (int q = 0; q < 32; q += 4) {
-                                    const int4 d4 = *reinterpret_cast<const int4 *>(colD + c + q);
-                                    const int y0 = (int)v[q] << d4.x, y1 = (int)v[q + 1] << d4.y;
-                                    const int y2 = (int)v[q + 2] << d4.z, y3 = (int)v[q + 3] << d4.w;
+                                    const int4 d4 = gf == 2 ? make_int4(1, 1, 1, 1) : *reinterpret_cast<const int4 *>(colD + c + q);
+                                    const int y0 = (int)v[q] * d4.x, y1 = (int)v[q + 1] * d4.y;
+                                    const int y2 = (int)v[q + 2] * d4.z, y3 = (int)v[q + 3] * d4.w;
                                     ymax = max(ymax, max(max(y0, y1), max(y2, y3)));
                                     ymin = min(ymin, min(min(y0, y1), min(y2, y3)));
                                 }
@@ -387,17 +496,24 @@ __global__ void __launch_bounds__(384, 1)
                             }
                             if (valid) {
                                 uint32_t w[8];
+                                const int hm = rs >= 2 ? 1 << (32 - rs) : 0;  // high-half multiplier
 #pragma unroll
                                 for (int q = 0; q < 32; q += 4) {
-                                    const int4 d4 = *reinterpret_cast<const int4 *>(colD + c + q);
-                                    int y[4] = {(int)v[q] << d4.x, (int)v[q + 1] << d4.y,
-                                                (int)v[q + 2] << d4.z, (int)v[q + 3] << d4.w};
+                                    const int4 d4 = gf == 2 ? make_int4(1, 1, 1, 1) : *reinterpret_cast<const int4 *>(colD + c + q);
+                                    int y[4] = {(int)v[q] * d4.x, (int)v[q + 1] * d4.y,
+                                                (int)v[q + 2] * d4.z, (int)v[q + 3] * d4.w};
                                     if (any_ls) {
 #pragma unroll
                                         for (int t = 0; t < 4; ++t) y[t] <<= ls;
                                     }
+                                    if (hm) {
 #pragma unroll
-                                    for (int t = 0; t < 4; ++t) y[t] = (y[t] + bias + ((y[t] >> rs) & om)) >> rs;
+                                        for (int t = 0; t < 4; ++t)
+                                            y[t] = __mulhi(y[t] + bias + (__mulhi(y[t], hm) & 1), hm);
+                                    } else {
+#pragma unroll
+                                        for (int t = 0; t < 4; ++t) y[t] = (y[t] + bias + ((y[t] >> rs) & om)) >> rs;
+                                    }
                                     w[q >> 2] = pack4b(y[0], y[1], y[2], y[3]);
                                 }
                                 int8_t *dst = p.out + grow * p.out_ld + n0 + c;
