@@ -244,7 +244,7 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     } else {
         // every thread of the scratch form keeps one group column: a stride that is a
         // multiple of ngc
-        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(n_exp, 256 * 8), (int64_t)sms * 4));
+        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(n_exp, 256 * 4), (int64_t)sms * 4));
         const int64_t used = (blocks * 256) / a.ngc * a.ngc;
         if (j.col_max && a.ngc <= 8192 && used >= a.ngc) {
             if (cudaMemsetAsync(j.col_max, 0x80, (size_t)a.ngc * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
@@ -277,7 +277,22 @@ int launch_requant_rows(RequantArgs a, cudaStream_t s) {
     if (groups == 0) return ICT_OK;
     const int G = a.G;
     KTimer kt(s, KC_REQUANT, (double)a.rows * (double)a.cols * (a.v64 ? 9.0 : 4.0 * a.nsplit + 1.0));
-    if (G >= 128 && G <= 4096) {
+    const bool vec = !a.v64 && a.cs == 1 && G >= 64 && G <= 4096 && G % 4 == 0 && a.cols % 4 == 0 &&
+                     a.ld % 4 == 0 && a.out_ld % 4 == 0 && a.split_stride % 4 == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.v32) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 3) == 0;
+    if (vec) {
+        const unsigned b = (unsigned)groups;
+        const bool wide = a.nsplit > 1;
+#define ICT_RQ_VEC(T_, V_)                                                      \
+    (wide ? requant_vec_kernel<T_, V_, true><<<b, T_, 0, s>>>(a)               \
+          : requant_vec_kernel<T_, V_, false><<<b, T_, 0, s>>>(a))
+        if (G <= 256) ICT_RQ_VEC(64, 1);
+        else if (G <= 512) ICT_RQ_VEC(128, 1);
+        else if (G <= 1024) ICT_RQ_VEC(256, 1);
+        else if (G <= 2048) ICT_RQ_VEC(256, 2);
+        else ICT_RQ_VEC(256, 4);
+#undef ICT_RQ_VEC
+    } else if (G >= 128 && G <= 4096) {
         const int T = G >= 256 ? 256 : 128;
         const int ept = (G + T - 1) / T;
         if (T == 128 && ept <= 1) launch_requant_block<128, 1>(a, groups, s);
@@ -948,8 +963,8 @@ int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
         vec = vec && a.t[i].G == G && (a.t[i].ld & 15) == 0 && aligned16(a.t[i].w) && aligned16(a.t[i].v) &&
               aligned16(a.t[i].g);
     vec = vec && G % 16 == 0 && G <= 2048;
-    // one dense tensor, one group per row of 16 * L elements: the prefetching kernel
     const SgdTensor &t0 = a.t[0];
+    // one dense tensor, one group per row of 16 * L elements: the prefetching kernel
     const int Lr = G / 16;
     if (vec && a.n == 1 && t0.ngc == 1 && t0.cols == t0.G && t0.ld == t0.G && Lr >= 1 && Lr <= 32 &&
         (Lr & (Lr - 1)) == 0) {

@@ -11,6 +11,8 @@
 
 #include "ict_device.cuh"
 
+#include <type_traits>
+
 namespace ict {
 
 // ------------------------------------------------------------------ two-term sums
@@ -183,7 +185,16 @@ __global__ void __launch_bounds__(256) estar_cols_scratch_kernel(AlignArgs a, in
     const int64_t n = ((a.rows + a.g_rows - 1) / a.g_rows) * a.ngc;
     if (tid < used_threads) {
         int m = kNoExp;
-        for (int64_t idx = tid; idx < n; idx += used_threads) {
+        int64_t idx = tid;
+        for (; idx + 3 * used_threads < n; idx += 4 * used_threads) {  // four loads in flight
+            const int e0 = a.in_exp[idx], e1 = a.in_exp[idx + used_threads];
+            const int e2 = a.in_exp[idx + 2 * used_threads], e3 = a.in_exp[idx + 3 * used_threads];
+            if (e0 != kEZero) m = max(m, e0);
+            if (e1 != kEZero) m = max(m, e1);
+            if (e2 != kEZero) m = max(m, e2);
+            if (e3 != kEZero) m = max(m, e3);
+        }
+        for (; idx < n; idx += used_threads) {
             const int e = a.in_exp[idx];
             if (e != kEZero) m = max(m, e);
         }
@@ -556,6 +567,77 @@ __global__ void __launch_bounds__(T) requant_group_block_kernel(RequantArgs a) {
     for (int k = 0; k < EPT; ++k) {
         const int jj = threadIdx.x + k * T;
         if (jj < glen) a.out[i * a.out_ld + j0 + jj] = (int8_t)requant64(x[k], r[k], e);
+    }
+    if (threadIdx.x == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+}
+
+// FIT of row-local groups of int32 partial sums (one or more split-K slices), 4 columns
+// per thread with 16-byte loads and 4-byte stores: one block of T threads per group of
+// at most 16 T columns.  WIDE: more than one slice, summed in int64.  Requires cs = 1,
+// G, cols, ld and out_ld multiples of 4.
+template <int T, int V, bool WIDE>
+__global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
+    using X = typename std::conditional<WIDE, int64_t, int32_t>::type;
+    const int64_t gidx = blockIdx.x;
+    const int64_t i = gidx / a.ngc, g = gidx % a.ngc;
+    const int64_t j0 = g * a.G;
+    const int glen = (int)min((int64_t)a.G, a.cols - j0);
+    const int re = a.base + (a.row_exp ? a.row_exp[i / a.row_div] : 0);
+    const bool ce4 = a.col_exp && a.col_div == 1 && ((reinterpret_cast<uintptr_t>(a.col_exp) & 3) == 0);
+    X x[V][4];
+    int r[V][4];
+    int emax = kNoExp;
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        const int jj = 4 * (threadIdx.x + k * T);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) x[k][t] = 0, r[k][t] = re;
+        if (jj < glen) {
+            const int64_t at = i * a.ld + j0 + jj;
+            const int4 q = *reinterpret_cast<const int4 *>(a.v32 + at);
+            X s0 = q.x, s1 = q.y, s2 = q.z, s3 = q.w;
+            for (int sp = 1; sp < a.nsplit; ++sp) {
+                const int4 q2 = *reinterpret_cast<const int4 *>(a.v32 + sp * a.split_stride + at);
+                s0 += q2.x, s1 += q2.y, s2 += q2.z, s3 += q2.w;
+            }
+            x[k][0] = s0, x[k][1] = s1, x[k][2] = s2, x[k][3] = s3;
+            if (ce4) {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(a.col_exp + j0 + jj);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) r[k][t] = re + sx8(w, t);
+            } else if (a.col_exp) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) r[k][t] = re + a.col_exp[(j0 + jj + t) / a.col_div];
+            }
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                if (WIDE) {
+                    if (x[k][t]) emax = max(emax, need64((int64_t)x[k][t], r[k][t]));
+                } else {
+                    const int32_t v = (int32_t)x[k][t];
+                    if (v) emax = max(emax, r[k][t] + need_off32((uint32_t)(v < 0 ? -v : v)));
+                }
+            }
+        }
+    }
+    __shared__ int red[T / 32];
+    emax = warp_max(emax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = emax;
+    __syncthreads();
+    int m = red[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) m = max(m, red[w]);
+    const int e = finalize_exp(m);
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        const int jj = 4 * (threadIdx.x + k * T);
+        if (jj < glen) {
+            int o[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                o[t] = WIDE ? requant64((int64_t)x[k][t], r[k][t], e) : requant32((int32_t)x[k][t], r[k][t], e);
+            *reinterpret_cast<uint32_t *>(a.out + i * a.out_ld + j0 + jj) = pack4(o[0], o[1], o[2], o[3]);
+        }
     }
     if (threadIdx.x == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
 }

@@ -82,7 +82,7 @@ struct GemmSmem {
     static constexpr int kOffB = STAGES * kABytes;
     static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 5 mbarriers
     static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 5) * 8 + 15) / 16 * 16;
-    static constexpr int kColInts = 2 * BN + 16;               // per epilogue warpgroup
+    static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
     static constexpr int kBytes = kOffCol + 2 * kColInts * 4 + 1024;  // + alignment slack
     static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
@@ -351,76 +351,89 @@ __global__ void __launch_bounds__(384, 1)
         int it = p.epi_split ? 0 : wg;
         // The loop never tests the abort flag on its own: the 128 threads decide together
         // through a barrier reduction, so none of them can be left waiting at a barrier.
-        // Geometry of unit u: first output row, valid rows, first output column.
-        auto geometry = [&](int u, int64_t &row_base, int &valid_rows, int &n0) {
-            const int tile = u % (p.n_mtiles * p.n_ntiles);
-            const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
-            if (LOAD == LOAD_CONV) {
-                const int img = mt / p.cv_tiles_per_img;
-                const int h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
-                row_base = ((int64_t)img * p.cv_P + h0) * p.cv_W;
-                valid_rows = min(p.cv_rows, p.cv_P - h0) * p.cv_W;
-            } else {
-                row_base = (int64_t)mt * 128;
-                valid_rows = min(128, p.M - mt * 128);
-            }
-            n0 = nt * BN;
-        };
-        // The exponents a tile needs (two column exponents and one row exponent per
-        // thread) are loaded one tile ahead, so their latency hides behind the previous
-        // tile's epilogue.
-        int pf_e0 = kEZero, pf_e1 = kEZero, pf_ea = 0;
-        auto prefetch = [&](int u) {
-            if (u >= p.num_units) return;
-            int64_t rb;
-            int vr, c0;
-            geometry(u, rb, vr, c0);
-            const int n_a = c0 + et, n_b = c0 + et + 128;
-            pf_e0 = n_a < p.N ? (int)p.eB[p.eB_div == 1 ? n_a : n_a / p.eB_div] : kEZero;
-            pf_e1 = (et + 128 < BN && n_b < p.N) ? (int)p.eB[p.eB_div == 1 ? n_b : n_b / p.eB_div] : kEZero;
-            const int64_t r = rb + et;
-            pf_ea = et < vr ? (int)p.eA[p.eA_div == 1 ? r : r / p.eA_div] : 0;
-        };
+        // Units are visited as u0, u0 + u_step, ...: their (split, m tile, n tile) advance
+        // incrementally, with no division per tile.
+        const int NT = p.n_ntiles, MT = p.n_mtiles, T = MT * NT;
         const int u0 = blockIdx.x + (p.epi_split ? 0 : wg * gridDim.x);
-        prefetch(u0);
+        const int d_split = u_step / T, d_m = (u_step % T) / NT, d_n = (u_step % T) % NT;
+        int c_split = u0 / T, c_mt = (u0 % T) / NT, c_nt = (u0 % T) % NT;  // unit being prefetched
+        // group of a tile column: shift for power-of-two widths (Gt == BN: always group 0)
+        const int gsh = (Gt & (Gt - 1)) == 0 ? __ffs(Gt) - 1 : -1;
+        auto group_of = [&](int j) { return gsh >= 0 ? j >> gsh : j / Gt; };
+        // The exponents a tile needs (two column exponents and one row exponent per
+        // thread) are loaded one tile ahead, so that their latency hides behind the
+        // previous tile's epilogue.
+        int pf_e0 = kEZero, pf_e1 = kEZero, pf_ea = 0, pf_split = 0, pf_vr = 0, pf_n0 = 0;
+        int64_t pf_rb = 0;
+        auto prefetch = [&](bool have) {
+            if (!have) return;
+            if (LOAD == LOAD_CONV) {
+                const int img = c_mt / p.cv_tiles_per_img;
+                const int h0 = (c_mt % p.cv_tiles_per_img) * p.cv_rows;
+                pf_rb = ((int64_t)img * p.cv_P + h0) * p.cv_W;
+                pf_vr = min(p.cv_rows, p.cv_P - h0) * p.cv_W;
+            } else {
+                pf_rb = (int64_t)c_mt * 128;
+                pf_vr = min(128, p.M - c_mt * 128);
+            }
+            pf_n0 = c_nt * BN;
+            pf_split = c_split;
+            const int n_a = pf_n0 + et, n_b = pf_n0 + et + 128;
+            pf_e0 = (et < BN && n_a < p.N) ? (int)p.eB[p.eB_div == 1 ? n_a : n_a / p.eB_div] : kEZero;
+            pf_e1 = (et + 128 < BN && n_b < p.N) ? (int)p.eB[p.eB_div == 1 ? n_b : n_b / p.eB_div] : kEZero;
+            const int64_t r = pf_rb + et;
+            pf_ea = et < pf_vr ? (int)p.eA[p.eA_div == 1 ? r : r / p.eA_div] : 0;
+            // advance the cursor to the unit after this one
+            c_nt += d_n;
+            if (c_nt >= NT) c_nt -= NT, ++c_mt;
+            c_mt += d_m;
+            if (c_mt >= MT) c_mt -= MT, ++c_split;
+            c_split += d_split;
+        };
+        int *cmin = gfast + 8, *cmax = cmin + 8;  // [8] per 32-column chunk of the tile
+        prefetch(u0 < p.num_units);
         for (int u = u0; u < p.num_units; u += u_step, it += it_step) {
-            const int split = u / (p.n_mtiles * p.n_ntiles);
             const int acc = it & 1;
-            int64_t row_base;
-            int valid_rows, n0;
-            geometry(u, row_base, valid_rows, n0);
+            const int64_t row_base = pf_rb;
+            const int valid_rows = pf_vr, n0 = pf_n0, split = pf_split;
+            const int e0 = pf_e0, e1 = pf_e1, ea_pf = pf_ea;
+            prefetch(u + u_step < p.num_units);
             // column tables of this tile (independent of the accumulator: built before waiting)
-            colE[et] = pf_e0;
-            if (et + 128 < BN) colE[et + 128] = pf_e1;
-            const int ea_pf = pf_ea;
-            prefetch(u + u_step);
-            named_bar_sync(bar_id, 128);
-            for (int g = wq; g < ngroups; g += 4) {
-                int lo = 0x7fffffff, hi = kNoExp;
-                for (int j = g * Gt + lane; j < (g + 1) * Gt; j += 32) {
-                    const int e = colE[j];
-                    if (e != kEZero) lo = min(lo, e), hi = max(hi, e);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-                    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-                }
+            if (et < BN) colE[et] = e0;
+            if (et + 128 < BN) colE[et + 128] = e1;
+            {   // min / max column exponent of each 32-column chunk (E_ZERO columns ignored)
+                const int lo0 = __reduce_min_sync(0xffffffffu, e0 == kEZero ? 0x7fffffff : e0);
+                const int hi0 = __reduce_max_sync(0xffffffffu, e0 == kEZero ? kNoExp : e0);
+                const int lo1 = __reduce_min_sync(0xffffffffu, e1 == kEZero ? 0x7fffffff : e1);
+                const int hi1 = __reduce_max_sync(0xffffffffu, e1 == kEZero ? kNoExp : e1);
                 if (lane == 0) {
-                    gmin[g] = hi <= kNoExp ? 0 : lo;
-                    // 2: every column has the same exponent (no column shifts); 1: fast path
-                    gfast[g] = (hi <= kNoExp || hi == lo) ? 2 : (hi - lo <= p.fast_slack ? 1 : 0);
+                    cmin[wq] = lo0, cmax[wq] = hi0;
+                    if (BN > 128) cmin[4 + wq] = lo1, cmax[4 + wq] = hi1;
                 }
             }
             named_bar_sync(bar_id, 128);
+            auto group_range = [&](int g, int &lo, int &hi) {
+                lo = 0x7fffffff, hi = kNoExp;
+                const int k0 = (g * Gt) >> 5, k1 = ((g + 1) * Gt) >> 5;
+                for (int k = k0; k < k1; ++k) lo = min(lo, cmin[k]), hi = max(hi, cmax[k]);
+            };
+            if (et < ngroups) {
+                int lo, hi;
+                group_range(et, lo, hi);
+                gmin[et] = hi <= kNoExp ? 0 : lo;
+                // 2: every column has the same exponent (no column shifts); 1: fast path
+                gfast[et] = (hi <= kNoExp || hi == lo) ? 2 : (hi - lo <= p.fast_slack ? 1 : 0);
+            }
             for (int j = et; j < BN; j += 128) {  // 2^d of each column (fast groups: d <= 30)
-                const int e = colE[j];
-                const int d = e == kEZero ? 0 : e - gmin[j / Gt];
+                int lo, hi;
+                group_range(group_of(j), lo, hi);
+                const int e = j == et ? e0 : e1;
+                const int d = (e == kEZero || hi <= kNoExp) ? 0 : e - lo;
                 colD[j] = d <= 30 ? 1 << d : 0;
             }
             const bool ok = mbar_wait(bar_tfull + 8 * acc, (it >> 1) & 1, p.wait_ns, abort_flag);
             if (!ok) fail();
-            if (named_bar_or(bar_id, 128, !ok || *abort_flag)) break;  // also publishes colD
+            if (named_bar_or(bar_id, 128, !ok || *abort_flag)) break;  // also publishes the tables
             tc_fence_after();
 
             const bool valid = et < valid_rows;
