@@ -209,7 +209,10 @@ int32_t ict_linear_fwd_noalloc(const ict_tensor *X, const ict_tensor *W, ict_ten
 /* Activation exponents must be uniform over pixels (g_rows >= rows); activation       */
 /* output groups likewise (g_rows >= rows, g_cols a multiple of 16); dW groups are     */
 /* per row.  This build supports 3x3, stride 1, pad 1, c and k multiples of 64 up to   */
-/* 256, w <= 128.                                                                      */
+/* 256, w <= 128.  ict_conv_workspace() is an upper bound for the direction; for FWD   */
+/* and BWD_DATA it includes int32 sums of the whole output (4 bytes per element), used  */
+/* when the output groups span all pixels: one Product pass writes the sums and every  */
+/* group's largest need, a streaming pass rounds them.                                 */
 size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d);
 int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_tensor *a,
                                const ict_tensor *b, ict_tensor *out, void *ws,

@@ -620,6 +620,8 @@ struct ConvPlan {
     bool global_groups;
     int32_t *gmax;
     int n_gcols;
+    int32_t *acc32;  // int32 sums of the one-pass global-group plan (else NULL)
+    int64_t acc_ld;
 };
 
 int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
@@ -708,6 +710,13 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
     }
     cp->n_gcols = (int)n_grp_cols(out);
     cp->gmax = cp->global_groups ? (int32_t *)ws.take((size_t)cp->n_gcols * 4) : nullptr;
+    // groups spanning all pixels: one Product pass writes int32 sums and the groups'
+    // largest need; a streaming pass rounds (needs G a multiple of 16, at most 8 groups)
+    cp->acc32 = nullptr;
+    if (cp->global_groups && cp->n_gcols <= 8 && (G >= out_c || G % 16 == 0) && out_c % 16 == 0) {
+        cp->acc_ld = round_up(out_c, 32);
+        cp->acc32 = (int32_t *)ws.take((size_t)npix * cp->acc_ld * 4);
+    }
     return ICT_OK;
 }
 
@@ -775,6 +784,33 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
     }
     counted(1);
+    if (cp.acc32) {
+        p.epi = EPI_I32;
+        p.ws32 = cp.acc32;
+        p.ws_ld = cp.acc_ld;
+        p.ws_split_stride = 0;
+        if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
+        GlobalRequantArgs r;
+        r.v = cp.acc32;
+        r.rows = cp.out_rows;
+        r.cols = cp.out_cols;
+        r.ld = cp.acc_ld;
+        r.eA = cp.eA;
+        r.eA_div = cp.eA_div;
+        r.eB = cp.eB;
+        r.eB_div = cp.eB_div;
+        r.gmax = cp.gmax;
+        r.G = p.G;
+        r.ngc = cp.n_gcols;
+        r.out = out->mant;
+        r.out_ld = out->ld;
+        r.out_exp = out->exp;
+        const int64_t n = cp.out_rows * (cp.out_cols / 16);
+        KTimer kt(s, KC_REQUANT, 5.0 * (double)cp.out_rows * (double)cp.out_cols);
+        requant_global_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(r);
+        counted(1);
+        return launch_status();
+    }
     p.epi = EPI_NEED_GLOBAL;  // the first pass is recompute: its work is not counted again
     if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
     p.epi = EPI_FIT_GLOBAL;
@@ -1202,6 +1238,8 @@ size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d) {
     w.take((size_t)std::max<int64_t>(d->k * RS * d->c, d->c * round_up(RS * d->k, 16)));
     w.take((size_t)std::max(d->k, d->c));
     w.take((size_t)std::max(d->k, d->c) * 4);
+    const int64_t out_c = dir == ICT_CONV_FWD ? d->k : d->c;
+    w.take((size_t)npix * round_up(out_c, 32) * 4);  // int32 sums for groups spanning all pixels
     return w.used;
 }
 

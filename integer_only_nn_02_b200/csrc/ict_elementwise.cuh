@@ -642,6 +642,47 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
     if (threadIdx.x == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
 }
 
+// FIT into groups that span all rows (a block of G columns over every row): the group
+// exponents are final in gmax (largest need over the whole group, from the Product's
+// epilogue), so every element is rounded independently.  16 columns per thread: four
+// 16-byte loads of int32 partial sums, one 16-byte store of mantissas.  Requires cols,
+// ld and out_ld multiples of 16.
+struct GlobalRequantArgs {
+    const int32_t *v;
+    int64_t rows, cols, ld;
+    const int8_t *eA;
+    int eA_div;
+    const int8_t *eB;
+    int eB_div;
+    const int32_t *gmax;
+    int G;
+    int64_t ngc;
+    int8_t *out;
+    int64_t out_ld;
+    int8_t *out_exp;
+};
+__global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a) {
+    const int64_t cv = a.cols / 16;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= a.rows * cv) return;
+    const int64_t i = t / cv, j0 = (t % cv) * 16;
+    const int ea = a.eA[i / a.eA_div];
+    const int e = finalize_exp(a.gmax[j0 / a.G]);  // 16 | G, so one group per thread
+    if (i == 0 && j0 % a.G == 0) a.out_exp[j0 / a.G] = (int8_t)e;
+    const int32_t *src = a.v + i * a.ld + j0;
+    int eb[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) eb[q] = a.eB_div == 1 ? a.eB[j0 + q] : a.eB[(j0 + q) / a.eB_div];
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int4 x = *reinterpret_cast<const int4 *>(src + 4 * q);
+        o[q] = pack4(requant32(x.x, ea + eb[4 * q], e), requant32(x.y, ea + eb[4 * q + 1], e),
+                     requant32(x.z, ea + eb[4 * q + 2], e), requant32(x.w, ea + eb[4 * q + 3], e));
+    }
+    *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // ------------------------------------------------------------------ integer SGD
 
 struct SgdTensor {

@@ -84,7 +84,8 @@ struct GemmSmem {
     static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 5) * 8 + 15) / 16 * 16;
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
-    static constexpr int kBytes = kOffCol + 2 * kColInts * 4 + 1024;  // + alignment slack
+    static constexpr int kOffGacc = kOffCol + 2 * kColInts * 4;     // [8] group needs (I32 + global groups)
+    static constexpr int kBytes = kOffGacc + 8 * 4 + 1024;           // + alignment slack
     static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
                   "column tables are read as int4");
     static_assert(kABytes % 1024 == 0 && kBBytes % 512 == 0 && kOffB % 1024 == 0 && kABytes / 2 <= 16383 * 16,
@@ -183,9 +184,11 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t bar_drain = bar_tempty + 16;             // [1]
     volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
     int *sCol = (int *)(smem + L::kOffCol);  // per epilogue warpgroup column tables
+    int *gacc = (int *)(smem + L::kOffGacc);  // running max need per output group (I32 with gmax)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    if (threadIdx.x < 8) gacc[threadIdx.x] = kNoExp;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
@@ -455,6 +458,20 @@ __global__ void __launch_bounds__(384, 1)
                                 *reinterpret_cast<uint4 *>(dst + c + 4 * q) =
                                     make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
+                    if (p.gmax) {
+                        // groups spanning all rows: the largest need of each 32 columns,
+                        // exponent eA[m] + eB[n] per element, kept per CTA
+                        int emax = kNoExp;
+                        if (valid) {
+#pragma unroll 8
+                            for (int q = 0; q < 32; ++q) {
+                                const int32_t x = (int32_t)v[q];
+                                if (x) emax = max(emax, ea + colE[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
+                            }
+                        }
+                        emax = warp_max(emax);
+                        if (lane == 0 && emax > kNoExp) atomicMax(gacc + group_of(c) + gcol0, emax);
+                    }
                 }
             } else {
                 for (int g = g_lo; g < g_hi; ++g) {
@@ -590,6 +607,8 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (p.epi == EPI_I32 && p.gmax && threadIdx.x < 8 && gacc[threadIdx.x] > kNoExp)
+        atomicMax(p.gmax + threadIdx.x, gacc[threadIdx.x]);
     if (warp == 2) tmem_dealloc(tmem_base, L::kTmemCols);
 }
 
