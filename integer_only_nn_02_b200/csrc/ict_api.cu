@@ -333,12 +333,16 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
                   cudaStream_t s) {
     constexpr int ST = stages_for(BN, BK);
     using L = GemmSmem<BN, BK, ST>;
-    auto k = gemm_ce_kernel<BN, BK, ST, LOAD>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
-        return ICT_ERR_CUDA;
-    k<<<grid, 384, L::kBytes, s>>>(ta, tb, p);
-    counted(1);
-    return launch_status();
+    auto run = [&](auto k) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+            return (int)ICT_ERR_CUDA;
+        k<<<grid, 384, L::kBytes, s>>>(ta, tb, p);
+        counted(1);
+        return launch_status();
+    };
+    if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, true>);
+    if constexpr (LOAD == LOAD_CONV_WGRAD) return ICT_ERR_LAYOUT;  // backward-weight writes int32 only
+    else return run(gemm_ce_kernel<BN, BK, ST, LOAD, false>);
 }
 
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,

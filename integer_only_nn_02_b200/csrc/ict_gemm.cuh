@@ -167,7 +167,10 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     }
 }
 
-template <int BN, int BK, int STAGES, int LOAD>
+// I32 (compile time): the kernel writes int32 partial sums (EPI_I32) and contains no FIT
+// code, and the FIT kernels contain no int32 path, so that each keeps a small code
+// footprint in the instruction cache.
+template <int BN, int BK, int STAGES, int LOAD, bool I32>
 __global__ void __launch_bounds__(384, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
@@ -446,7 +449,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
             uint32_t v[32];
 
-            if (p.epi == EPI_I32) {
+            if constexpr (I32) {
                 int32_t *dst = p.ws32 + split * p.ws_split_stride + grow * p.ws_ld + n0;
                 for (int c = c_lo; c < c_hi; c += 32) {
                     tmem_ld32(taddr + c, v);
@@ -607,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (p.epi == EPI_I32 && p.gmax && threadIdx.x < 8 && gacc[threadIdx.x] > kNoExp)
+    if (I32 && p.gmax && threadIdx.x < 8 && gacc[threadIdx.x] > kNoExp)
         atomicMax(p.gmax + threadIdx.x, gacc[threadIdx.x]);
     if (warp == 2) tmem_dealloc(tmem_base, L::kTmemCols);
 }
