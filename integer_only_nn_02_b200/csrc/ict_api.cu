@@ -214,10 +214,18 @@ struct AlignJob {
     int32_t *col_max;  // axis 0: int32 scratch [group columns] for a parallel column max
 };
 
-int launch_align(const AlignJob &j, cudaStream_t s) {
-    const ict_tensor *in = j.t;
-    if (in->rows == 0 || in->cols == 0) return ICT_OK;
+// Arguments of one alignment job and how its target exponents are found.
+struct AlignLaunch {
     AlignArgs a;
+    int64_t n_exp;
+    int estar;             // 0: none (row e* inside the rows kernel), 1: rows, 2: column scratch, 3: column blocks
+    int64_t blocks, used;  // column scratch form
+};
+
+AlignLaunch plan_align(const AlignJob &j, int sms) {
+    const ict_tensor *in = j.t;
+    AlignLaunch L;
+    AlignArgs &a = L.a;
     memset(&a, 0, sizeof(a));
     a.in = in->mant;
     a.in_exp = in->exp;
@@ -231,38 +239,108 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
     a.out = j.out;
     a.out_ld = j.ld;
     a.e_star = j.e_star;
-    int sms = 148;
-    device_info(&sms);
-    const int64_t n_exp = n_grp_rows(in) * a.ngc;
+    L.n_exp = n_grp_rows(in) * a.ngc;
+    L.blocks = L.used = 0;
     if (j.axis == 1) {
-        if (j.transpose) {
-            KTimer kt(s, KC_ESTAR, (double)n_exp + (double)in->rows);
-            estar_rows_kernel<<<(unsigned)cdiv64(in->rows, 256), 256, 0, s>>>(a);
-        } else {
-            a.row_estar = 1;  // computed inside align_rows_kernel
-        }
+        L.estar = j.transpose ? 1 : 0;
+        a.row_estar = j.transpose ? 0 : 1;  // computed inside align_rows_kernel
     } else {
         // every thread of the scratch form keeps one group column: a stride that is a
         // multiple of ngc
-        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(n_exp, 256 * 4), (int64_t)sms * 4));
-        const int64_t used = (blocks * 256) / a.ngc * a.ngc;
-        if (j.col_max && a.ngc <= 8192 && used >= a.ngc) {
-            if (cudaMemsetAsync(j.col_max, 0x80, (size_t)a.ngc * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
-            KTimer kt(s, KC_ESTAR, (double)n_exp + 8.0 * (double)a.ngc);
-            estar_cols_scratch_kernel<<<(unsigned)blocks, 256, (size_t)a.ngc * 4, s>>>(a, j.col_max, used);
-            a.col_max = j.col_max;
+        L.blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(L.n_exp, 256 * 4), (int64_t)sms * 4));
+        L.used = (L.blocks * 256) / a.ngc * a.ngc;
+        L.estar = (j.col_max && a.ngc <= 8192 && L.used >= a.ngc) ? 2 : 3;
+        if (L.estar == 2) a.col_max = j.col_max;
+    }
+    return L;
+}
+
+// One or two alignment jobs; two jobs must both be transposing column alignments with
+// scratch (the operands of a backward-weight contraction): they share one launch of the
+// column e* kernel and one of the transposing kernel.
+int launch_align_n(const AlignJob *jobs, int n, cudaStream_t s) {
+    int sms = 148;
+    device_info(&sms);
+    AlignLaunch L[2];
+    AlignPair P;
+    memset(&P, 0, sizeof(P));
+    double estar_work = 0, align_work = 0;
+    for (int i = 0; i < n; ++i) {
+        L[i] = plan_align(jobs[i], sms);
+        P.a[i] = L[i].a;
+        P.cm[i] = jobs[i].col_max;
+        P.used[i] = L[i].used;
+        estar_work += (double)L[i].n_exp + 8.0 * (double)L[i].a.ngc;
+        align_work += 2.0 * (double)L[i].a.rows * (double)L[i].a.cols + (double)L[i].n_exp;
+    }
+    int launches = 0;
+    if (n == 2 && (L[0].estar != 2 || L[1].estar != 2)) {  // not pairable on this device: one by one
+        int st;
+        if ((st = launch_align_n(jobs, 1, s))) return st;
+        return launch_align_n(jobs + 1, 1, s);
+    }
+    if (n == 2) {
+        for (int i = 0; i < 2; ++i)
+            if (cudaMemsetAsync(jobs[i].col_max, 0x80, (size_t)L[i].a.ngc * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
+        {
+            KTimer kt(s, KC_ESTAR, estar_work);
+            const int64_t ngc = std::max(L[0].a.ngc, L[1].a.ngc);
+            estar_cols_scratch_kernel<<<dim3((unsigned)std::max(L[0].blocks, L[1].blocks), 2), 256,
+                                        (size_t)ngc * 4, s>>>(P);
+        }
+        KTimer kt(s, KC_ALIGN, align_work);
+        const int64_t cols = std::max(L[0].a.cols, L[1].a.cols), rows = std::max(L[0].a.rows, L[1].a.rows);
+        align_transpose_kernel<<<dim3((unsigned)cdiv64(cols, 128), (unsigned)cdiv64(rows, 128), 2), 256, 0, s>>>(P);
+        counted(2);
+        return launch_status();
+    }
+    const AlignLaunch &l = L[0];
+    const AlignArgs &a = l.a;
+    if (l.estar == 1) {
+        KTimer kt(s, KC_ESTAR, (double)l.n_exp + (double)a.rows);
+        estar_rows_kernel<<<(unsigned)cdiv64(a.rows, 256), 256, 0, s>>>(a);
+        ++launches;
+    } else if (l.estar == 2) {
+        if (cudaMemsetAsync(jobs[0].col_max, 0x80, (size_t)a.ngc * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
+        KTimer kt(s, KC_ESTAR, estar_work);
+        estar_cols_scratch_kernel<<<(unsigned)l.blocks, 256, (size_t)a.ngc * 4, s>>>(P);
+        ++launches;
+    } else if (l.estar == 3) {
+        KTimer kt(s, KC_ESTAR, (double)l.n_exp + (double)a.cols);
+        estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
+        ++launches;
+    }
+    KTimer kt(s, KC_ALIGN, align_work);
+    if (jobs[0].transpose)
+        align_transpose_kernel<<<dim3((unsigned)cdiv64(a.cols, 128), (unsigned)cdiv64(a.rows, 128)), 256, 0, s>>>(P);
+    else
+        align_rows_kernel<<<dim3((unsigned)cdiv64(a.cols, 64), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);
+    counted(launches + 1);
+    return launch_status();
+}
+
+int launch_align(const AlignJob &j, cudaStream_t s) {
+    if (j.t->rows == 0 || j.t->cols == 0) return ICT_OK;
+    return launch_align_n(&j, 1, s);
+}
+
+// The jobs of one call, pairing transposing column alignments with scratch.
+int launch_aligns(const AlignJob *jobs, int n, cudaStream_t s) {
+    auto pairable = [&](const AlignJob &j) {
+        return j.axis == 0 && j.transpose && j.col_max && j.t->rows > 0 && j.t->cols > 0 &&
+               plan_align(j, planning_sms()).estar == 2;
+    };
+    int st;
+    for (int i = 0; i < n;) {
+        if (i + 1 < n && pairable(jobs[i]) && pairable(jobs[i + 1])) {
+            if ((st = launch_align_n(jobs + i, 2, s))) return st;
+            i += 2;
         } else {
-            KTimer kt(s, KC_ESTAR, (double)n_exp + (double)in->cols);
-            estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
+            if ((st = launch_align(jobs[i], s))) return st;
+            ++i;
         }
     }
-    KTimer kt(s, KC_ALIGN, 2.0 * (double)in->rows * (double)in->cols + (double)n_exp);
-    if (j.transpose)
-        align_transpose_kernel<<<dim3((unsigned)cdiv64(in->cols, 128), (unsigned)cdiv64(in->rows, 128)), 256, 0, s>>>(a);
-    else
-        align_rows_kernel<<<dim3((unsigned)cdiv64(in->cols, 64), (unsigned)cdiv64(in->rows, 64)), 256, 0, s>>>(a);
-    counted(a.row_estar ? 1 : 2);
-    return launch_status();
+    return ICT_OK;
 }
 
 template <int T, int EPT>
@@ -341,8 +419,13 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
         return launch_status();
     };
     if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, true>);
-    if constexpr (LOAD == LOAD_CONV_WGRAD) return ICT_ERR_LAYOUT;  // backward-weight writes int32 only
-    else return run(gemm_ce_kernel<BN, BK, ST, LOAD, false>);
+    if constexpr (LOAD == LOAD_CONV_WGRAD) {
+        return ICT_ERR_LAYOUT;  // backward-weight writes int32 only
+    } else {
+        const int gt = p.G >= p.N ? BN : p.G;  // group width inside a tile
+        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, true>);
+        return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, false>);
+    }
 }
 
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
@@ -587,8 +670,7 @@ int run_linear(const LinearPlan &lp, cudaStream_t s) {
     if (lp.empty) return launch_zero(lp.out, s);
     if (lp.out->rows == 0 || lp.out->cols == 0) return ICT_OK;
     int st;
-    for (int i = 0; i < lp.njobs; ++i)
-        if ((st = launch_align(lp.jobs[i], s))) return st;
+    if ((st = launch_aligns(lp.jobs, lp.njobs, s))) return st;
     return run_product(lp.A, lp.B, lp.out, lp.pp, s);
 }
 

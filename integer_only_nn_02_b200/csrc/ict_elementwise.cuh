@@ -176,8 +176,18 @@ __global__ void __launch_bounds__(256) estar_cols_kernel(AlignArgs a) {
 // group column (the grid stride is a multiple of the group-column count), reduces its
 // strided slice of the exponent grid in a register, then one atomicMax in shared and
 // one in global memory.
-__global__ void __launch_bounds__(256) estar_cols_scratch_kernel(AlignArgs a, int32_t *col_max,
-                                                                 int64_t used_threads) {
+// Up to two alignment jobs per launch (blockIdx.y or blockIdx.z selects the job), so that
+// both operands of a contraction are prepared by one launch of each kernel.
+struct AlignPair {
+    AlignArgs a[2];
+    int32_t *cm[2];
+    int64_t used[2];
+};
+
+__global__ void __launch_bounds__(256) estar_cols_scratch_kernel(const __grid_constant__ AlignPair P) {
+    const AlignArgs &a = P.a[blockIdx.y];
+    int32_t *const col_max = P.cm[blockIdx.y];
+    const int64_t used_threads = P.used[blockIdx.y];
     extern __shared__ int sm[];  // [ngc]
     for (int64_t g = threadIdx.x; g < a.ngc; g += blockDim.x) sm[g] = kNoExp;
     __syncthreads();
@@ -283,7 +293,8 @@ __global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
 // stores 32-bit words into a shared tile whose 16-byte chunks are XOR-swizzled by the
 // output row's 16-row band, so that both the word stores and the 16-byte reads that
 // feed the coalesced global stores are free of bank conflicts.
-__global__ void __launch_bounds__(256) align_transpose_kernel(AlignArgs a) {
+__global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_constant__ AlignPair P) {
+    const AlignArgs &a = P.a[blockIdx.z];
     __shared__ uint4 tile[128][8];  // [output row = input column][16-byte chunk, swizzled]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r0 = (int64_t)blockIdx.y * 128, c0 = (int64_t)blockIdx.x * 128;

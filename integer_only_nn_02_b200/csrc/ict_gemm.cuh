@@ -170,7 +170,9 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
 // I32 (compile time): the kernel writes int32 partial sums (EPI_I32) and contains no FIT
 // code, and the FIT kernels contain no int32 path, so that each keeps a small code
 // footprint in the instruction cache.
-template <int BN, int BK, int STAGES, int LOAD, bool I32>
+// G32 (compile time, FIT kernels): output groups are 32 columns wide, so only the
+// 32-column fast path and the exact path are compiled in.
+template <int BN, int BK, int STAGES, int LOAD, bool I32, bool G32 = false>
 __global__ void __launch_bounds__(384, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
@@ -481,7 +483,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int g0 = g * Gt;
                     const int gcol = gcol0 + g;
                     const int gf = gfast[g];
-                    if (Gt == 32 && gf) {
+                    if (G32 && gf) {
                         if (gf == 2)
                             epi_fast32<false>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol, et);
                         else
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     const int gm = gmin[g];
                     int e;
-                    if (gf) {
+                    if (!G32 && gf) {
                         // |x << d| < 2^30: the group exponent follows from the largest magnitude
                         int ymax = 0, ymin = 0;
                         for (int c = g0; c < g0 + Gt; c += 32) {
