@@ -250,6 +250,10 @@ AlignLaunch plan_align(const AlignJob &j, int sms) {
         L.blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(L.n_exp, 256 * 4), (int64_t)sms * 4));
         L.used = (L.blocks * 256) / a.ngc * a.ngc;
         L.estar = (j.col_max && a.ngc <= 8192 && L.used >= a.ngc) ? 2 : 3;
+        if (j.transpose && in->rows <= 4096 && a.g_cols >= 16) {
+            L.estar = 0;  // few rows (a weight): each transposing block scans its columns' exponents
+            a.col_scan = 1;
+        }
         if (L.estar == 2) a.col_max = j.col_max;
     }
     return L;

@@ -31,6 +31,15 @@ __device__ __forceinline__ void raise_status(int code) { atomicOr(&g_status, 1 <
 // need(x, r) - r for a = |x| > 0: the offset s such that RNE(x * 2^-s) fits in
 // [-127, 127] and RNE(x * 2^-(s-1)) does not.  With b = bitlen(a), s = b - 7, plus one
 // when the top eight bits of a are all ones (a >= 127.5 * 2^s rounds to 128).
+// x / d for an index x >= 0 and d >= 1: a shift for powers of two, 32-bit division when
+// both fit (64-bit division is a long emulated sequence).
+__device__ __forceinline__ int64_t idiv(int64_t x, int64_t d) {
+    if (d == 1) return x;
+    if ((d & (d - 1)) == 0) return x >> (__ffsll(d) - 1);
+    if (x <= 0x7fffffff && d <= 0x7fffffff) return (int64_t)((uint32_t)x / (uint32_t)d);
+    return x / d;
+}
+
 __device__ __forceinline__ int need_off32(uint32_t a) {
     int s = 25 - __clz(a);  // bitlen - 7
     if (s > 0 && (a >> (s - 1)) == 255u) s += 1;

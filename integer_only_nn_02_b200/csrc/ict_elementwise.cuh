@@ -105,18 +105,18 @@ __global__ void __launch_bounds__(256) requant_rows_kernel(RequantArgs a) {
     const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (gw >= a.rows * a.ngc) return;
-    const int64_t i = gw / a.ngc, g = gw % a.ngc;
+    const int64_t i = idiv(gw, a.ngc), g = gw - i * a.ngc;
     const int64_t j0 = g * a.G, j1 = min(a.cols, j0 + a.G);
-    const int re = a.base + (a.row_exp ? a.row_exp[i / a.row_div] : 0);
+    const int re = a.base + (a.row_exp ? a.row_exp[idiv(i, a.row_div)] : 0);
     int emax = kNoExp;
     for (int64_t j = j0 + lane; j < j1; j += 32) {
         const int64_t x = rq_value(a, i, j);
-        if (x) emax = max(emax, need64(x, re + (a.col_exp ? a.col_exp[j / a.col_div] : 0)));
+        if (x) emax = max(emax, need64(x, re + (a.col_exp ? a.col_exp[idiv(j, a.col_div)] : 0)));
     }
     const int e = finalize_exp(warp_max(emax));
     for (int64_t j = j0 + lane; j < j1; j += 32) {
         const int64_t x = rq_value(a, i, j);
-        a.out[i * a.out_ld + j] = (int8_t)requant64(x, re + (a.col_exp ? a.col_exp[j / a.col_div] : 0), e);
+        a.out[i * a.out_ld + j] = (int8_t)requant64(x, re + (a.col_exp ? a.col_exp[idiv(j, a.col_div)] : 0), e);
     }
     if (lane == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
 }
@@ -135,6 +135,7 @@ struct AlignArgs {
     int8_t *e_star;           // [rows] (axis 1) or [cols] (axis 0)
     const int32_t *col_max;   // axis 0 with scratch: max per group column (<= kNoExp: none)
     int row_estar;            // axis 1: the alignment kernel computes and stores e* itself
+    int col_scan;             // axis 0, transposed: each block finds its columns' e* itself
 };
 
 __device__ __forceinline__ int estar_of(int m) { return m <= kNoExp ? kEZero : m; }
@@ -245,7 +246,7 @@ __device__ __forceinline__ uint4 rne_shift16(uint4 raw, int d) {
 // per column, from the column-max scratch or the e* vector).
 __device__ __forceinline__ int align_target(const AlignArgs &a, int64_t i, int64_t j) {
     if (a.axis == 1) return i < a.rows ? a.e_star[i] : kEZero;
-    if (a.col_max) return estar_of(a.col_max[j / a.g_cols]);
+    if (a.col_max) return estar_of(a.col_max[idiv(j, a.g_cols)]);
     return a.e_star[j];
 }
 
@@ -253,7 +254,7 @@ __device__ __forceinline__ int align_target(const AlignArgs &a, int64_t i, int64
 __device__ __forceinline__ uint4 align_vec(const AlignArgs &a, int64_t i, int64_t j, int es) {
     if (i >= a.rows) return make_uint4(0, 0, 0, 0);
     const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
-    const int eg = a.in_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+    const int eg = a.in_exp[idiv(i, a.g_rows) * a.ngc + idiv(j, a.g_cols)];
     if (eg == kEZero) return make_uint4(0, 0, 0, 0);
     return rne_shift16(raw, min(es - eg, 8));  // |C| <= 127: shifts of 8 or more give 0
 }
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
     if (i >= a.rows) return;  // whole 4-thread row groups leave together
     int es;
     if (a.axis == 1 && a.row_estar) {
-        const int8_t *e = a.in_exp + (i / a.g_rows) * a.ngc;
+        const int8_t *e = a.in_exp + idiv(i, a.g_rows) * a.ngc;
         int m = kNoExp;
         for (int64_t g = threadIdx.x & 3; g < a.ngc; g += 4)
             if (e[g] != kEZero) m = max(m, (int)e[g]);
@@ -300,16 +301,37 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
     const int64_t r0 = (int64_t)blockIdx.y * 128, c0 = (int64_t)blockIdx.x * 128;
     const int rq = 4 * warp + (lane & 3), cc = lane >> 2;  // row quad 0..31, column chunk 0..7
     const int64_t j = c0 + 16 * cc;
+    __shared__ int gmx[16];  // col_scan: e* of the column groups of this block's 128 columns
+    int64_t g_first = 0;
+    if (a.col_scan) {
+        // a strip of at most 128 columns spans at most 9 groups (groups are >= 16 wide)
+        g_first = idiv(c0, a.g_cols);
+        const int ng = (int)(idiv(min(c0 + 128, a.cols) - 1, a.g_cols) - g_first + 1);
+        if (threadIdx.x < 16) gmx[threadIdx.x] = kNoExp;
+        __syncthreads();
+        const int64_t ngr = idiv(a.rows + a.g_rows - 1, a.g_rows);
+        const int k = threadIdx.x % ng, per = 256 / ng;
+        if (threadIdx.x < per * ng) {
+            int m = kNoExp;
+            for (int64_t r = threadIdx.x / ng; r < ngr; r += per) {
+                const int e = a.in_exp[r * a.ngc + g_first + k];
+                if (e != kEZero) m = max(m, e);
+            }
+            if (m > kNoExp) atomicMax(&gmx[k], m);
+        }
+        __syncthreads();
+    }
     if (j < a.cols) {
-        if (a.axis == 0 && a.col_max && blockIdx.y == 0 && rq == 0) {
-            const int es = align_target(a, 0, j);
+        const int es_col = a.col_scan ? estar_of(gmx[idiv(j, a.g_cols) - g_first]) : 0;
+        if (a.axis == 0 && (a.col_max || a.col_scan) && blockIdx.y == 0 && rq == 0) {
+            const int es = a.col_scan ? es_col : align_target(a, 0, j);
             for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
         }
         uint4 v[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const int64_t i = r0 + 4 * rq + t;
-            v[t] = align_vec(a, i, j, align_target(a, i, j));
+            v[t] = align_vec(a, i, j, a.col_scan ? es_col : align_target(a, i, j));
         }
         const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w}, {v[1].x, v[1].y, v[1].z, v[1].w},
                                   {v[2].x, v[2].y, v[2].z, v[2].w}, {v[3].x, v[3].y, v[3].z, v[3].w}};
@@ -374,8 +396,8 @@ __global__ void __launch_bounds__(256) gelu_fwd_kernel(GeluArgs a) {
     const int64_t vecs_per_row = a.cols / 16;
     const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (v >= a.rows * vecs_per_row) return;
-    const int64_t i = v / vecs_per_row, j = (v % vecs_per_row) * 16;
-    const int e = a.h_exp[(i / a.g_rows) * a.ngc + j / a.g_cols];
+    const int64_t i = idiv(v, vecs_per_row), j = (v - i * vecs_per_row) * 16;
+    const int e = a.h_exp[idiv(i, a.g_rows) * a.ngc + idiv(j, a.g_cols)];
     const uint4 raw = *reinterpret_cast<const uint4 *>(a.h + i * a.ld_h + j);
     const uint32_t src[4] = {raw.x, raw.y, raw.z, raw.w};
     uint32_t o[4] = {0, 0, 0, 0};
@@ -433,7 +455,7 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(GeluArgs a) {
     const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (gw >= a.rows * a.ngc) return;
-    const int64_t i = gw / a.ngc, g = gw % a.ngc;
+    const int64_t i = idiv(gw, a.ngc), g = gw - i * a.ngc;
     const int64_t j0 = g * a.g_cols, j1 = min(a.cols, j0 + a.g_cols);
     const int eh = a.h_exp[i * a.ngc + g], ed = a.dg_exp[i * a.ngc + g];
     int emax = kNoExp;
@@ -486,7 +508,7 @@ __global__ void __launch_bounds__(256) gelu_bwd_vec_kernel(const __grid_constant
          base += nwarps * GPW) {
         const int64_t gw = base + sub;
         if (gw >= total) continue;
-        const int64_t i = gw / a.ngc, g = gw % a.ngc;
+        const int64_t i = idiv(gw, a.ngc), g = gw - i * a.ngc;
         const int64_t j0 = g * a.g_cols;
         const int glen = (int)min((int64_t)a.g_cols, a.cols - j0);
         const int eh = a.h_exp[gw], ed = a.dg_exp[gw];
@@ -550,7 +572,7 @@ __global__ void __launch_bounds__(T) requant_group_block_kernel(RequantArgs a) {
     const int64_t i = gidx / a.ngc, g = gidx % a.ngc;
     const int64_t j0 = g * a.G;
     const int glen = (int)min((int64_t)a.G, a.cols - j0);
-    const int re = a.base + (a.row_exp ? a.row_exp[i / a.row_div] : 0);
+    const int re = a.base + (a.row_exp ? a.row_exp[idiv(i, a.row_div)] : 0);
     int64_t x[EPT];
     int r[EPT];
     int emax = kNoExp;
@@ -562,7 +584,7 @@ __global__ void __launch_bounds__(T) requant_group_block_kernel(RequantArgs a) {
         if (jj < glen) {
             const int64_t j = j0 + jj;
             x[k] = rq_value(a, i, j);
-            r[k] = re + (a.col_exp ? a.col_exp[j / a.col_div] : 0);
+            r[k] = re + (a.col_exp ? a.col_exp[idiv(j, a.col_div)] : 0);
             if (x[k]) emax = max(emax, need64(x[k], r[k]));
         }
     }
@@ -593,7 +615,7 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
     const int64_t i = gidx / a.ngc, g = gidx % a.ngc;
     const int64_t j0 = g * a.G;
     const int glen = (int)min((int64_t)a.G, a.cols - j0);
-    const int re = a.base + (a.row_exp ? a.row_exp[i / a.row_div] : 0);
+    const int re = a.base + (a.row_exp ? a.row_exp[idiv(i, a.row_div)] : 0);
     const bool ce4 = a.col_exp && a.col_div == 1 && ((reinterpret_cast<uintptr_t>(a.col_exp) & 3) == 0);
     X x[V][4];
     int r[V][4];
@@ -676,10 +698,11 @@ __global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a
     const int64_t cv = a.cols / 16;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= a.rows * cv) return;
-    const int64_t i = t / cv, j0 = (t % cv) * 16;
-    const int ea = a.eA[i / a.eA_div];
-    const int e = finalize_exp(a.gmax[j0 / a.G]);  // 16 | G, so one group per thread
-    if (i == 0 && j0 % a.G == 0) a.out_exp[j0 / a.G] = (int8_t)e;
+    const int64_t i = idiv(t, cv), j0 = (t - i * cv) * 16;
+    const int ea = a.eA[idiv(i, a.eA_div)];
+    const int64_t g = idiv(j0, a.G);  // 16 | G, so one group per thread
+    const int e = finalize_exp(a.gmax[g]);
+    if (i == 0 && j0 == g * a.G) a.out_exp[g] = (int8_t)e;
     const int32_t *src = a.v + i * a.ld + j0;
     int eb[16];
 #pragma unroll
