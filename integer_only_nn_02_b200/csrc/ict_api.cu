@@ -860,7 +860,9 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     p.cv_S = d->s;
     p.cv_pad = d->pad;
     p.cv_sign = dir == ICT_CONV_FWD ? 1 : -1;
-    p.stage_tx_bytes = (uint32_t)(64 * d->w * cp.rows_per_tile + 64 * cp.bn);
+    // the weight operand stays in shared memory when all its K blocks fit the B ring
+    p.b_resident = p.n_ntiles == 1 && p.n_kblk <= stages_for(cp.bn, 64);
+    p.stage_tx_bytes = (uint32_t)(64 * d->w * cp.rows_per_tile + (p.b_resident ? 0 : 64 * cp.bn));
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     const int grid = std::min(p.num_units, sms);
@@ -914,6 +916,7 @@ struct WgradPlan {
     int hrows, hblk, kpix, atoms, mtiles, ntiles, splits, kblk_per_split, n_kblk, units;
     int64_t M, N, ws_ld;
     int32_t *partial;
+    int64_t *sums64;  // [N][M] slice sums
     int8_t *e_rows, *e_cols;
 };
 
@@ -953,6 +956,7 @@ int plan_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X
     wp->N = d->k;
     wp->ws_ld = round_up(wp->N, 32);
     wp->partial = (int32_t *)ws.take((size_t)wp->splits * wp->M * wp->ws_ld * 4);
+    wp->sums64 = (int64_t *)ws.take((size_t)wp->M * wp->N * 8);
     wp->e_rows = (int8_t *)ws.take((size_t)wp->M);
     wp->e_cols = (int8_t *)ws.take((size_t)wp->N);
     return ICT_OK;
@@ -1004,16 +1008,23 @@ int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X,
     if ((st = launch_gemm(64, 256, LOAD_CONV_WGRAD, ta, tb, p, std::min(wp.units, sms), s,
                           2.0 * (double)wp.M * (double)wp.N * (double)d->n * d->h * d->w)))
         return st;
-    // dW[k][j] = sum over slices of partial[j][k]: FIT per row k, exponent e_cols[k] + e_rows[j]
+    // dW[k][j] = sum over slices of partial[j][k]: the slices are summed and transposed
+    // into int64 sums64[k][j], then FIT per row k with exponent e_cols[k] + e_rows[j]
+    {
+        KTimer kt(s, KC_REQUANT, 4.0 * (double)wp.splits * (double)wp.M * (double)wp.N + 8.0 * (double)wp.M * wp.N);
+        sum_slices_t_kernel<<<dim3((unsigned)cdiv64(wp.N, 32), (unsigned)cdiv64(wp.M, 32)), 256, 0, s>>>(
+            wp.partial, wp.splits, wp.M * wp.ws_ld, wp.M, wp.N, wp.ws_ld, wp.sums64);
+        counted(1);
+        if ((st = launch_status())) return st;
+    }
     RequantArgs a;
     memset(&a, 0, sizeof(a));
-    a.v32 = wp.partial;
-    a.nsplit = wp.splits;
-    a.split_stride = wp.M * wp.ws_ld;
+    a.v64 = wp.sums64;
+    a.nsplit = 1;
     a.rows = wp.N;
     a.cols = wp.M;
-    a.ld = 1;
-    a.cs = wp.ws_ld;
+    a.ld = wp.M;
+    a.cs = 1;
     a.row_exp = wp.e_cols;
     a.row_div = 1;
     a.col_exp = wp.e_rows;

@@ -705,16 +705,55 @@ __global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a
     if (i == 0 && j0 == g * a.G) a.out_exp[g] = (int8_t)e;
     const int32_t *src = a.v + i * a.ld + j0;
     int eb[16];
+    if (a.eB_div == 1 && (reinterpret_cast<uintptr_t>(a.eB) & 15) == 0) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(a.eB + j0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int q = 0; q < 16; ++q) eb[q] = a.eB_div == 1 ? a.eB[j0 + q] : a.eB[(j0 + q) / a.eB_div];
+        for (int q = 0; q < 16; ++q) eb[q] = sx8(ww[q >> 2], q & 3);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) eb[q] = a.eB[idiv(j0 + q, a.eB_div)];
+    }
+    // element exponent ea + eb[q]; mantissa = RNE(x * 2^-(e - ea - eb[q])): a right shift
+    // of at least 2 by high-half multiplies, anything else by the general routine
+    auto rq = [&](int32_t x, int q) {
+        const int sft = e - ea - eb[q];
+        if (sft >= 2 && sft < 32) {
+            const int m = 1 << (32 - sft), bias = (1 << (sft - 1)) - 1;
+            return __mulhi(x + bias + (__mulhi(x, m) & 1), m);
+        }
+        return requant32(x, ea + eb[q], e);
+    };
     uint32_t o[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int4 x = *reinterpret_cast<const int4 *>(src + 4 * q);
-        o[q] = pack4(requant32(x.x, ea + eb[4 * q], e), requant32(x.y, ea + eb[4 * q + 1], e),
-                     requant32(x.z, ea + eb[4 * q + 2], e), requant32(x.w, ea + eb[4 * q + 3], e));
+        o[q] = pack4(rq(x.x, 4 * q), rq(x.y, 4 * q + 1), rq(x.z, 4 * q + 2), rq(x.w, 4 * q + 3));
     }
     *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Sum of split-K int32 slices, transposed: out[c][r] = sum_s in[s][r][c] (int64), through
+// 32 x 32 shared tiles so that both the slice reads and the output writes are coalesced.
+__global__ void __launch_bounds__(256) sum_slices_t_kernel(const int32_t *in, int nsplit, int64_t split_stride,
+                                                           int64_t rows, int64_t cols, int64_t ld, int64_t *out) {
+    __shared__ int64_t tile[32][33];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 threads
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t r = r0 + ty + 8 * k, c = c0 + tx;
+        int64_t acc = 0;
+        if (r < rows && c < cols)
+            for (int sp = 0; sp < nsplit; ++sp) acc += in[sp * split_stride + r * ld + c];
+        tile[ty + 8 * k][tx] = acc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t c = c0 + ty + 8 * k, r = r0 + tx;
+        if (c < cols && r < rows) out[c * rows + r] = tile[tx][ty + 8 * k];
+    }
 }
 
 // ------------------------------------------------------------------ integer SGD

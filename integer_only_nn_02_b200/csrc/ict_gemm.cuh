@@ -64,6 +64,9 @@ struct GemmParams {
     int32_t *gmax;  // [column groups] running max of need() (global groups)
     // implicit-GEMM convolution: output tile = cv_rows image rows of width cv_W
     int cv_W, cv_P, cv_rows, cv_tiles_per_img, cv_cblk, cv_S, cv_pad, cv_sign;
+    // conv: every K block of the weight operand held in shared memory for the whole kernel
+    // (block kb at the B ring's slot kb; needs n_kblk <= STAGES); stage_tx_bytes is then A only
+    int b_resident;
     // backward-weight: K block = wg_hrows image rows of every image (wg_kpix pixels), M rows
     // (tap, channel) in 64-row atoms (wg_atoms in total)
     int wg_hrows, wg_hblk, wg_kpix, wg_atoms;
@@ -80,8 +83,8 @@ struct GemmSmem {
     static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
     static constexpr int kOffB = STAGES * kABytes;
-    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 5 mbarriers
-    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 5) * 8 + 15) / 16 * 16;
+    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 6 mbarriers
+    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 6) * 8 + 15) / 16 * 16;
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
     static constexpr int kOffGacc = kOffCol + 2 * kColInts * 4;     // [8] group needs (I32 + global groups)
@@ -187,6 +190,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t bar_tfull = bar_empty + 8 * STAGES;      // [2]
     const uint32_t bar_tempty = bar_tfull + 16;             // [2]
     const uint32_t bar_drain = bar_tempty + 16;             // [1]
+    const uint32_t bar_bres = bar_drain + 8;                // [1] resident weight operand landed
     volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
     int *sCol = (int *)(smem + L::kOffCol);  // per epilogue warpgroup column tables
     int *gacc = (int *)(smem + L::kOffGacc);  // running max need per output group (I32 with gmax)
@@ -204,6 +208,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(bar_tempty + 8 * a, p.epi_split ? 256 : 128);
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_bres, 1);
         misc[1] = 0;
         fence_barrier_init();
     }
@@ -234,6 +239,12 @@ __global__ void __launch_bounds__(384, 1)
             int issued[STAGES];
             uint32_t issued_phase[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = 0, issued_phase[s] = 0;
+            const bool bres = LOAD == LOAD_CONV && p.b_resident;
+            if (bres && blockIdx.x < p.num_units) {  // the weight operand, once
+                mbar_expect_tx(bar_bres, (uint32_t)(p.n_kblk * L::kBBytes));
+                for (int kb = 0; kb < p.n_kblk; ++kb)
+                    tma_load_2d(sbase + L::kOffB + kb * L::kBBytes, &tmB, bar_bres, kb * BK, 0);
+            }
             for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
                 const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
                 const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
@@ -262,7 +273,7 @@ __global__ void __launch_bounds__(384, 1)
                         const int r = tap / p.cv_S, s = tap % p.cv_S;
                         tma_load_4d(sa, &tmA, fb, cb * 64, p.cv_sign * (s - p.cv_pad),
                                     h0 + p.cv_sign * (r - p.cv_pad), img);
-                        tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
+                        if (!bres) tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
                     } else {
                         // pixels of this K block: rows h1 .. h1 + hrows - 1 of image img1
                         const int img1 = kb / p.wg_hblk, h1 = (kb % p.wg_hblk) * p.wg_hrows;
@@ -284,6 +295,7 @@ __global__ void __launch_bounds__(384, 1)
             // drain: every issued copy must land before the CTA may exit
             for (int s = 0; s < STAGES; ++s)
                 if (issued[s]) mbar_wait(bar_full + 8 * s, issued_phase[s], p.drain_ns, nullptr);
+            if (bres && blockIdx.x < p.num_units) mbar_wait(bar_bres, 0, p.drain_ns, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -295,6 +307,9 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t phase = 0;
             int it = 0;
             bool any = false;
+            if (LOAD == LOAD_CONV && p.b_resident && blockIdx.x < p.num_units &&
+                !mbar_wait(bar_bres, 0, p.wait_ns, abort_flag))
+                fail();
             for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x, ++it) {
                 const int split = u / (p.n_mtiles * p.n_ntiles);
                 const int kb0 = split * p.kblk_per_split;
@@ -322,7 +337,8 @@ __global__ void __launch_bounds__(384, 1)
                             umma_i8(tmem_d, da + 128 * kk, db + 128 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
                     } else {
                         const uint64_t da = smem_desc_kmajor(sbase + stage * L::kABytes, BK);
-                        const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + stage * L::kBBytes, BK);
+                        const int bslot = (LOAD == LOAD_CONV && p.b_resident) ? kb : stage;
+                        const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + bslot * L::kBBytes, BK);
 #pragma unroll
                         for (int kk = 0; kk < BK / 32; ++kk)
                             umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
