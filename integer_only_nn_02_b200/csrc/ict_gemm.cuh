@@ -99,6 +99,14 @@ struct GemmSmem {
 __device__ __forceinline__ uint32_t pack4b(int a, int b, int c, int d) {
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
+// The same packing for values already within [-127, 127], in two conversion
+// instructions (each packs two values into bytes; the second merges the first's word).
+__device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {
+    uint32_t t, r;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(t) : "r"(d), "r"(c));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(b), "r"(a), "r"(t));
+    return r;
+}
 
 // Fast epilogue of one output group of 32 columns of an accumulator row, the group on
 // the fast path: y = acc * 2^d_n (d_n = column shift inside the group, |y| < 2^30), the
@@ -111,7 +119,8 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     uint32_t v[32];
     tmem_ld32(taddr, v);
     tmem_ld_wait();
-    int hi = 0, lo = 0;
+    // four independent max / min chains, so that the reductions overlap
+    int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int q = 0; q < 32; q += 4) {
         int y0 = (int)v[q], y1 = (int)v[q + 1], y2 = (int)v[q + 2], y3 = (int)v[q + 3];
@@ -120,10 +129,12 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
             y0 *= m4.x, y1 *= m4.y, y2 *= m4.z, y3 *= m4.w;
             v[q] = (uint32_t)y0, v[q + 1] = (uint32_t)y1, v[q + 2] = (uint32_t)y2, v[q + 3] = (uint32_t)y3;
         }
-        hi = max(hi, max(max(y0, y1), max(y2, y3)));
-        lo = min(lo, min(min(y0, y1), min(y2, y3)));
+        const int c = (q >> 2) & 3;
+        hi[c] = max(hi[c], max(max(y0, y1), max(y2, y3)));
+        lo[c] = min(lo[c], min(min(y0, y1), min(y2, y3)));
     }
-    const int amax = valid ? max(hi, -lo) : 0;
+    const int h = max(max(hi[0], hi[1]), max(hi[2], hi[3])), l = min(min(lo[0], lo[1]), min(lo[2], lo[3]));
+    const int amax = valid ? max(h, -l) : 0;
     const int need = amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp;
     if (p.epi == EPI_NEED_GLOBAL) {
         const int m = warp_max(need);
@@ -142,9 +153,14 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     if (rs >= 2) {
         const int m = 1 << (32 - rs), bias = (1 << (rs - 1)) - 1;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int y = (int)v[q];
-            v[q] = (uint32_t)__mulhi(y + bias + (__mulhi(y, m) & 1), m);
+        for (int q = 0; q < 32; q += 8) {  // eight elements per stage, stage by stage
+            int t[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = __mulhi((int)v[q + k], m);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = (int)v[q + k] + bias + (t[k] & 1);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[q + k] = (uint32_t)__mulhi(t[k], m);
         }
     } else if (rs == 1) {
 #pragma unroll
@@ -163,10 +179,10 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
         for (int q = 0; q < 32; q += 16)
             if (ncol + q < p.N)
                 *reinterpret_cast<uint4 *>(dst + q) = make_uint4(
-                    pack4b((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
-                    pack4b((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
-                    pack4b((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
-                    pack4b((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+                    pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
+                    pack4s((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
+                    pack4s((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
+                    pack4s((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
     }
 }
 
