@@ -327,12 +327,24 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
             const int es = a.col_scan ? es_col : align_target(a, 0, j);
             for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
         }
-        uint4 v[4];
+        // all loads first (rows beyond the tensor read nothing), then the shifts
+        uint4 raw[4];
+        int eg[4];
+        const int64_t gcol = idiv(j, a.g_cols);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const int64_t i = r0 + 4 * rq + t;
-            v[t] = align_vec(a, i, j, a.col_scan ? es_col : align_target(a, i, j));
+            const bool in = i < a.rows;
+            raw[t] = in ? *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j) : make_uint4(0, 0, 0, 0);
+            eg[t] = in ? (int)a.in_exp[idiv(i, a.g_rows) * a.ngc + gcol] : kEZero;
         }
+        int es[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) es[t] = a.col_scan ? es_col : align_target(a, r0 + 4 * rq + t, j);
+        uint4 v[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            v[t] = eg[t] == kEZero ? make_uint4(0, 0, 0, 0) : rne_shift16(raw[t], min(es[t] - eg[t], 8));
         const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w}, {v[1].x, v[1].y, v[1].z, v[1].w},
                                   {v[2].x, v[2].y, v[2].z, v[2].w}, {v[3].x, v[3].y, v[3].z, v[3].w}};
         uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
@@ -744,8 +756,17 @@ __global__ void __launch_bounds__(256) sum_slices_t_kernel(const int32_t *in, in
     for (int k = 0; k < 4; ++k) {
         const int64_t r = r0 + ty + 8 * k, c = c0 + tx;
         int64_t acc = 0;
-        if (r < rows && c < cols)
-            for (int sp = 0; sp < nsplit; ++sp) acc += in[sp * split_stride + r * ld + c];
+        if (r < rows && c < cols) {
+            const int32_t *src = in + r * ld + c;
+            int64_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;  // four loads in flight
+            int sp = 0;
+            for (; sp + 4 <= nsplit; sp += 4) {
+                a0 += src[sp * split_stride], a1 += src[(sp + 1) * split_stride];
+                a2 += src[(sp + 2) * split_stride], a3 += src[(sp + 3) * split_stride];
+            }
+            for (; sp < nsplit; ++sp) a0 += src[sp * split_stride];
+            acc = (a0 + a1) + (a2 + a3);
+        }
         tile[ty + 8 * k][tx] = acc;
     }
     __syncthreads();
