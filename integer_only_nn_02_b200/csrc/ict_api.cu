@@ -414,21 +414,28 @@ template <int BN, int BK, int LOAD>
 int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid,
                   cudaStream_t s) {
     constexpr int ST = stages_for(BN, BK);
-    using L = GemmSmem<BN, BK, ST>;
-    auto run = [&](auto k) {
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+    auto run = [&](auto k, int nwg, int smem_bytes) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
             return (int)ICT_ERR_CUDA;
-        k<<<grid, 384, L::kBytes, s>>>(ta, tb, p);
+        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, p);
         counted(1);
         return launch_status();
     };
-    if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, true>);
+    constexpr int kB2 = GemmSmem<BN, BK, ST, 2>::kBytes;
+    if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, true>, 2, kB2);
     if constexpr (LOAD == LOAD_CONV_WGRAD) {
         return ICT_ERR_LAYOUT;  // backward-weight writes int32 only
     } else {
         const int gt = p.G >= p.N ? BN : p.G;  // group width inside a tile
-        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, true>);
-        return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, false>);
+        if constexpr (LOAD == LOAD_2D && BN <= 128) {
+            if (p.nwg == 4) {  // four epilogue warpgroups, four accumulators
+                constexpr int kB4 = GemmSmem<BN, BK, ST, 4>::kBytes;
+                if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, true, 4>, 4, kB4);
+                return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, false, 4>, 4, kB4);
+            }
+        }
+        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, true>, 2, kB2);
+        return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, false>, 2, kB2);
     }
 }
 
@@ -439,7 +446,8 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     // group straddles the halves
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
-    p.epi_split = p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0);
+    if (p.nwg != 4 || p.epi == EPI_I32) p.nwg = 2;
+    p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0));
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
     if (bn == BN_ && bk == BK_ && load == LOAD_) \
         return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s);
@@ -526,7 +534,7 @@ Operand operand_cols(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
 }
 
 struct ProductPlan {
-    int bn, splits, kblk_per_split, n_kblk, n_mtiles, n_ntiles, units, grid;
+    int bn, nwg, splits, kblk_per_split, n_kblk, n_mtiles, n_ntiles, units, grid;
     bool fused;
     int32_t *ws32;
     int64_t ws_ld;
@@ -537,6 +545,12 @@ ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out,
                          bool allow_split, Ws &ws) {
     ProductPlan pl;
     pl.bn = pick_bn_waves(M, N, out->g_cols, sms);
+    pl.nwg = 2;
+    {   // short contractions are bound by the FIT epilogue: four epilogue warpgroups
+        // (four accumulators) on 128-wide tiles
+        const int64_t G = out->g_cols;
+        if (K <= 1024 && N % 128 == 0 && G < N && G % 32 == 0 && 128 % G == 0) pl.bn = 128, pl.nwg = 4;
+    }
     pl.n_kblk = (int)cdiv64(K, 128);
     pl.n_mtiles = (int)cdiv64(M, 128);
     pl.n_ntiles = (int)cdiv64(N, pl.bn);
@@ -596,6 +610,7 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     p.epi = pl.fused ? EPI_FIT_ROW : EPI_I32;
+    p.nwg = pl.nwg;
     if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K)))
         return st;
     if (pl.fused) return ICT_OK;

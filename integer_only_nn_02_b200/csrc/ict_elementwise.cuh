@@ -523,23 +523,22 @@ __global__ void __launch_bounds__(256) gelu_bwd_vec_kernel(const __grid_constant
         const int64_t i = idiv(gw, a.ngc), g = gw - i * a.ngc;
         const int64_t j0 = g * a.g_cols;
         const int glen = (int)min((int64_t)a.g_cols, a.cols - j0);
+        // the group's mantissas and exponents are loaded together (no dependent round trip)
+        const int off = li * 16;
+        uint4 x = make_uint4(0, 0, 0, 0), y = make_uint4(0, 0, 0, 0);
+        if (off < glen) {
+            x = *reinterpret_cast<const uint4 *>(a.h + i * a.ld_h + j0 + off);
+            y = *reinterpret_cast<const uint4 *>(a.dg + i * a.ld_dg + j0 + off);
+        }
         const int eh = a.h_exp[gw], ed = a.dg_exp[gw];
         const int sh = (eh < 0 && eh != kEZero) ? -eh : 0;
         if (sh > 21) {
             gelu_bwd_group_exact<L>(a, i, g, glen, li, gmask);
             continue;
         }
-        const int off = li * 16;
-        uint32_t hv[4] = {0, 0, 0, 0}, dv[4] = {0, 0, 0, 0};
-        if (off < glen) {
-            const uint4 x = *reinterpret_cast<const uint4 *>(a.h + i * a.ld_h + j0 + off);
-            const uint4 y = *reinterpret_cast<const uint4 *>(a.dg + i * a.ld_dg + j0 + off);
-            hv[0] = x.x, hv[1] = x.y, hv[2] = x.z, hv[3] = x.w;
-            dv[0] = y.x, dv[1] = y.y, dv[2] = y.z, dv[3] = y.w;
-            const int rem = glen - off;
-            if (rem < 16)
-                for (int b = rem; b < 16; ++b) dv[b >> 2] &= ~(0xffu << (8 * (b & 3)));
-        }
+        uint32_t hv[4] = {x.x, x.y, x.z, x.w}, dv[4] = {y.x, y.y, y.z, y.w};
+        if (off < glen && glen - off < 16)
+            for (int b = glen - off; b < 16; ++b) dv[b >> 2] &= ~(0xffu << (8 * (b & 3)));
         // |C_h| < T is the interior; e_h >= 1 (or E_ZERO) leaves only C_h = 0 inside
         const int T = (eh >= 1 || eh == kEZero) ? 1 : (1 - eh >= 8 ? 256 : (1 << (1 - eh)));
         int xv[16];
@@ -641,7 +640,13 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
             const int64_t at = i * a.ld + j0 + jj;
             const int4 q = *reinterpret_cast<const int4 *>(a.v32 + at);
             X s0 = q.x, s1 = q.y, s2 = q.z, s3 = q.w;
-            for (int sp = 1; sp < a.nsplit; ++sp) {
+            int sp = 1;
+            for (; sp + 2 <= a.nsplit; sp += 2) {  // two slices in flight
+                const int4 q2 = *reinterpret_cast<const int4 *>(a.v32 + sp * a.split_stride + at);
+                const int4 q3 = *reinterpret_cast<const int4 *>(a.v32 + (sp + 1) * a.split_stride + at);
+                s0 += (X)q2.x + q3.x, s1 += (X)q2.y + q3.y, s2 += (X)q2.z + q3.z, s3 += (X)q2.w + q3.w;
+            }
+            for (; sp < a.nsplit; ++sp) {
                 const int4 q2 = *reinterpret_cast<const int4 *>(a.v32 + sp * a.split_stride + at);
                 s0 += q2.x, s1 += q2.y, s2 += q2.z, s3 += q2.w;
             }

@@ -74,20 +74,23 @@ struct GemmParams {
     uint64_t wait_ns, drain_ns;
     int epi;
     int epi_split;  // 1: both epilogue warpgroups share every tile, one half of its columns each
+    int nwg;        // host only: epilogue warpgroups of the instantiation to launch (2 or 4)
 };
 
-template <int BN, int BK, int STAGES>
+template <int BN, int BK, int STAGES, int NWG = 2>
 struct GemmSmem {
     static constexpr int kABytes = 128 * BK;
     static constexpr int kBBytes = BN * BK;
-    static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
+    // one TMEM accumulator per epilogue warpgroup
+    static constexpr int kTmemCols = (NWG * BN <= 32) ? 32 : (NWG * BN <= 64) ? 64 : (NWG * BN <= 128) ? 128
+                                   : (NWG * BN <= 256) ? 256 : 512;
+    static_assert(NWG * BN <= 512, "accumulators must fit TMEM");
     static constexpr int kOffB = STAGES * kABytes;
-    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 6 mbarriers
-    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 6) * 8 + 15) / 16 * 16;
+    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 2*NWG + 2 mbarriers
+    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 2 * NWG + 2) * 8 + 15) / 16 * 16;
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
-    static constexpr int kOffGacc = kOffCol + 2 * kColInts * 4;     // [8] group needs (I32 + global groups)
+    static constexpr int kOffGacc = kOffCol + NWG * kColInts * 4;   // [8] group needs (I32 + global groups)
     static constexpr int kBytes = kOffGacc + 8 * 4 + 1024;           // + alignment slack
     static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
                   "column tables are read as int4");
@@ -191,11 +194,13 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
 // footprint in the instruction cache.
 // G32 (compile time, FIT kernels): output groups are 32 columns wide, so only the
 // 32-column fast path and the exact path are compiled in.
-template <int BN, int BK, int STAGES, int LOAD, bool I32, bool G32 = false>
-__global__ void __launch_bounds__(384, 1)
+// NWG (compile time): epilogue warpgroups, each owning one TMEM accumulator (2 or 4).
+template <int BN, int BK, int STAGES, int LOAD, bool I32, bool G32 = false, int NWG = 2>
+__global__ void __launch_bounds__(128 + 128 * NWG, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
-    using L = GemmSmem<BN, BK, STAGES>;
+    using L = GemmSmem<BN, BK, STAGES, NWG>;
+    constexpr int NACC = NWG;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(BK == 128 || BK == 64 || (BK == 256 && LOAD == LOAD_CONV_WGRAD), "BK");
     extern __shared__ uint8_t smem_raw[];
@@ -203,9 +208,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L::kOffBar;           // [STAGES]
     const uint32_t bar_empty = bar_full + 8 * STAGES;       // [STAGES]
-    const uint32_t bar_tfull = bar_empty + 8 * STAGES;      // [2]
-    const uint32_t bar_tempty = bar_tfull + 16;             // [2]
-    const uint32_t bar_drain = bar_tempty + 16;             // [1]
+    const uint32_t bar_tfull = bar_empty + 8 * STAGES;      // [NACC]
+    const uint32_t bar_tempty = bar_tfull + 8 * NACC;       // [NACC]
+    const uint32_t bar_drain = bar_tempty + 8 * NACC;       // [1]
     const uint32_t bar_bres = bar_drain + 8;                // [1] resident weight operand landed
     volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
     int *sCol = (int *)(smem + L::kOffCol);  // per epilogue warpgroup column tables
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < NACC; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
             mbar_init(bar_tempty + 8 * a, p.epi_split ? 256 : 128);
         }
@@ -330,8 +335,8 @@ __global__ void __launch_bounds__(384, 1)
                 const int split = u / (p.n_mtiles * p.n_ntiles);
                 const int kb0 = split * p.kblk_per_split;
                 const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
-                const int acc = it & 1;
-                if (!mbar_wait(bar_tempty + 8 * acc, ((it >> 1) & 1) ^ 1, p.wait_ns, abort_flag)) {
+                const int acc = it % NACC;
+                if (!mbar_wait(bar_tempty + 8 * acc, ((it / NACC) & 1) ^ 1, p.wait_ns, abort_flag)) {
                     fail();
                     break;
                 }
@@ -387,7 +392,7 @@ __global__ void __launch_bounds__(384, 1)
         const int g_lo = p.epi_split ? wg * (ngroups >> 1) : 0;
         const int g_hi = p.epi_split ? g_lo + (ngroups >> 1) : ngroups;
         const int c_lo = p.epi_split ? wg * (BN / 2) : 0, c_hi = p.epi_split ? c_lo + BN / 2 : BN;
-        const int u_step = p.epi_split ? gridDim.x : 2 * gridDim.x, it_step = p.epi_split ? 1 : 2;
+        const int u_step = p.epi_split ? gridDim.x : NWG * gridDim.x, it_step = p.epi_split ? 1 : NWG;
         int it = p.epi_split ? 0 : wg;
         // The loop never tests the abort flag on its own: the 128 threads decide together
         // through a barrier reduction, so none of them can be left waiting at a barrier.
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(384, 1)
         int *cmin = gfast + 8, *cmax = cmin + 8;  // [8] per 32-column chunk of the tile
         prefetch(u0 < p.num_units);
         for (int u = u0; u < p.num_units; u += u_step, it += it_step) {
-            const int acc = it & 1;
+            const int acc = it % NACC;
             const int64_t row_base = pf_rb;
             const int valid_rows = pf_vr, n0 = pf_n0, split = pf_split;
             const int e0 = pf_e0, e1 = pf_e1, ea_pf = pf_ea;
@@ -471,7 +476,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int d = (e == kEZero || hi <= kNoExp) ? 0 : e - lo;
                 colD[j] = d <= 30 ? 1 << d : 0;
             }
-            const bool ok = mbar_wait(bar_tfull + 8 * acc, (it >> 1) & 1, p.wait_ns, abort_flag);
+            const bool ok = mbar_wait(bar_tfull + 8 * acc, (it / NACC) & 1, p.wait_ns, abort_flag);
             if (!ok) fail();
             if (named_bar_or(bar_id, 128, !ok || *abort_flag)) break;  // also publishes the tables
             tc_fence_after();
