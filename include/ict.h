@@ -141,6 +141,12 @@ int32_t ict_timing_read(int32_t kernel_class, double *ms_total, int64_t *launche
  * outputs unspecified.  Process-wide; meant for tests of that path. */
 int32_t ict_set_wait_limit_ns(uint64_t ns);
 
+/* Self-test of the bounded-wait path: launches one block that waits on an mbarrier no
+ * one ever arrives on, bounded by limit_ns (nanoseconds, > 0).  When the bound runs out
+ * the block raises ICT_ERR_DEVICE_TIMEOUT in the device status word and exits; nothing
+ * faults, traps or hangs, and the context stays usable.  Asynchronous on `stream`. */
+int32_t ict_selftest_wait_timeout(uint64_t limit_ns, void *stream);
+
 /* --------------------------------------------------------------------------------- */
 /* Requantisation (FIT) of integer values, the step that closes every Product         */
 /* (Table 6, Eqs. 5 and 3; Figure 1a).                                                 */

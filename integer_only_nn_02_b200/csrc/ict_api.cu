@@ -1242,6 +1242,15 @@ int32_t ict_get_device_status(int32_t *host_out, void *stream) {
     return ICT_OK;
 }
 
+int32_t ict_selftest_wait_timeout(uint64_t limit_ns, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if (limit_ns == 0) return ICT_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+    counted(1);
+    return launch_status();
+}
+
 int32_t ict_set_wait_limit_ns(uint64_t ns) {
     std::lock_guard<std::mutex> lk(g_mu);
     g_wait_ns = ns ? ns : 2000000000ull;

@@ -782,6 +782,20 @@ __global__ void __launch_bounds__(256) sum_slices_t_kernel(const int32_t *in, in
     }
 }
 
+// A wait on an mbarrier that never completes, bounded by limit_ns: raises
+// ICT_ERR_DEVICE_TIMEOUT and returns (self-test of the bounded-wait path).
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(b, 0, limit_ns, nullptr)) raise_status(ICT_ERR_DEVICE_TIMEOUT);
+    __syncthreads();
+}
+
 // ------------------------------------------------------------------ integer SGD
 
 struct SgdTensor {

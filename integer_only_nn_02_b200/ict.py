@@ -60,6 +60,7 @@ _SIGS = {
     "ict_version": ([], ctypes.c_char_p),
     "ict_get_device_status": ([_P(_i32), _vp], _i32),
     "ict_set_wait_limit_ns": ([ctypes.c_uint64], _i32),
+    "ict_selftest_wait_timeout": ([ctypes.c_uint64, _vp], _i32),
     "ict_launch_count": ([], ctypes.c_uint64),
     "ict_timing_enable": ([_i32], _i32),
     "ict_timing_read": ([_i32, _P(ctypes.c_double), _P(_i64), _P(ctypes.c_double), _i32], _i32),
@@ -192,6 +193,10 @@ def ict_timing_read(kernel_class: int, reset: bool = False):
 
 def ict_set_wait_limit_ns(ns: int) -> None:
     _check(lib.ict_set_wait_limit_ns(int(ns)), "ict_set_wait_limit_ns")
+
+
+def ict_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(lib.ict_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ict_selftest_wait_timeout")
 
 
 def ict_requant(vals: torch.Tensor, out: DevCE, base_exp=0, row_exp=None, col_exp=None, stream=None):

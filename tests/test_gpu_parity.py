@@ -254,3 +254,21 @@ def test_argument_errors_return_before_launch(ict):
     need = ict.ict_linear_workspace(ict.OP_LINEAR_FWD, X, W2, Y)
     assert need == 0  # both operands uniform along K, fused epilogue
     status_ok(ict)
+
+
+def test_bounded_wait_timeout_leaves_context_usable(ict):
+    """A wait that nothing completes runs out its bound, raises ICT_ERR_DEVICE_TIMEOUT in
+    the status word and returns; the next calls run normally and bit-exact."""
+    ict.ict_get_device_status()  # clear
+    ict.ict_selftest_wait_timeout(2_000_000)  # 2 ms
+    code, raw = ict.ict_get_device_status()
+    assert code == 7, (code, raw)  # ICT_ERR_DEVICE_TIMEOUT
+    from integer_only_nn_02_b200 import workloads as wl
+    cfg = wl.single_linear(seed=3)
+    X, W = cfg["X"], cfg["W"]
+    Y = ict.linear_fwd(ict.DevCE.from_host(X), ict.DevCE.from_host(W), 32)
+    ref = oracle.linear_fwd(X, W, 1, 32)
+    h = Y.to_host()
+    assert np.array_equal(h.mant, ref.mant) and np.array_equal(h.exp, ref.exp)
+    code, raw = ict.ict_get_device_status()
+    assert code == 0, (code, raw)
