@@ -16,8 +16,12 @@ configurations, each a step of its own with its own unit:
   single_linear       64x128 linear layer fwd+bwd+SGD, microseconds per step
 
 Usage:  python bench.py [--config C] [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-For N > 1 run under torchrun: every rank runs the same single-GPU step on its own batch
-(independent replicas, no data-path collective); the reported time is the max over ranks.
+For N > 1 run under torchrun, one rank per GPU, each with its own batch of the
+configuration's size (weak scaling); the reported time is the max over ranks.  The linear
+configurations train data-parallel: every backward-weight Product exchanges its alignment
+targets (MAX) and exact integer sums (SUM) over NCCL, so all ranks apply the same update,
+the one a single GPU computes on the whole batch.  resnet18_conv3x3 and resnet50_sgd run
+as independent replicas.
 """
 from __future__ import annotations
 
@@ -155,6 +159,22 @@ class Step:
     def ws(self, nbytes):
         return self.torch.empty(max(int(nbytes), 256), dtype=self.torch.uint8, device="cuda")
 
+    data_parallel = False  # True: with several ranks the batch is split and dW all-reduced
+
+    def bwd_weight(self, dY, X, dW, ws):
+        """One linear layer's backward-weight call.  On one GPU, the library's single call;
+        with several ranks (each holding its own shard of the batch), the split-batch form
+        whose targets and integer sums are all-reduced over NCCL, bit-identical to one GPU
+        on the whole batch."""
+        from integer_only_nn_02_b200 import dp
+
+        world = dp.world_size()
+        if world == 1:
+            return lambda: self.ict.ict_linear_bwd_weight(dY, X, dW, ws)
+        g = dp.LinearWeightGrad(dY, X, total_rows=world * dY.rows)
+        self.exchanged_bytes = getattr(self, "exchanged_bytes", 0) + g.exchanged_bytes
+        return lambda: g(dY, X, dW)
+
     def run(self, events=None):
         for i, (_, fn) in enumerate(self.calls):
             if events is not None:
@@ -174,6 +194,7 @@ class Step:
 
 
 class MlpStep(Step):
+    data_parallel = True
     TOKENS, D, HID, GROUP = 64 * 197, 192, 768, 32
     sample_arg = 64 * 197
     workload = {"workload": "vit_ti_mlp_block_step", "tokens": 12608, "d": 192, "hidden": 768, "group": 32,
@@ -199,10 +220,10 @@ class MlpStep(Step):
             ("gelu_fwd", lambda: ict.ict_gelu_fwd(self.H, self.G)),
             ("fc2_fwd", lambda: ict.ict_linear_fwd(self.G, self.W2, self.Y, ws)),
             ("fc2_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY2, self.W2, self.dG, ws)),
-            ("fc2_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY2, self.G, self.dW2, ws)),
+            ("fc2_bwd_weight", self.bwd_weight(self.dY2, self.G, self.dW2, ws)),
             ("gelu_bwd", lambda: ict.ict_gelu_bwd(self.H, self.dG, self.dH)),
             ("fc1_bwd_data", lambda: ict.ict_linear_bwd_data(self.dH, self.W1, self.dX, ws)),
-            ("fc1_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dH, self.X, self.dW1, ws)),
+            ("fc1_bwd_weight", self.bwd_weight(self.dH, self.X, self.dW1, ws)),
             ("sgd_w1", lambda: ict.ict_sgd_momentum_step(self.W1, self.V1, self.dW1, mom, lr)),
             ("sgd_w2", lambda: ict.ict_sgd_momentum_step(self.W2, self.V2, self.dW2, mom, lr)),
         ]
@@ -234,6 +255,7 @@ class MlpStep(Step):
 
 
 class LinearStep(Step):
+    data_parallel = True
     unit = "us"
     higher_is_better = False
     workload = {"workload": "single_linear_step", "m": 64, "k": 128, "n": 64, "group": 32}
@@ -252,7 +274,7 @@ class LinearStep(Step):
         self.calls = [
             ("fwd", lambda: ict.ict_linear_fwd(self.X, self.W, self.Y, ws)),
             ("bwd_data", lambda: ict.ict_linear_bwd_data(self.dY, self.W, self.dX, ws)),
-            ("bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY, self.X, self.dW, ws)),
+            ("bwd_weight", self.bwd_weight(self.dY, self.X, self.dW, ws)),
             ("sgd", lambda: ict.ict_sgd_momentum_step(self.W, self.V, self.dW, mom, lr)),
         ]
         self.units = 1
@@ -313,6 +335,7 @@ class ConvStep(Step):
 
 
 class TrioStep(Step):
+    data_parallel = True
     sample_arg = 2048
     workload = {"workload": "vit_b_linear_trio", "tokens": 12608, "d": 768, "hidden": 3072, "group": 64,
                 "gop_per_step": 356.952}
@@ -335,8 +358,8 @@ class TrioStep(Step):
             ("fc2_fwd", lambda: ict.ict_linear_fwd(self.H1, self.W2, self.Y2, ws)),
             ("fc2_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY2, self.W2, self.dHo, ws)),
             ("fc1_bwd_data", lambda: ict.ict_linear_bwd_data(self.dY1, self.W1, self.dXo, ws)),
-            ("fc1_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY1, self.X, self.dW1, ws)),
-            ("fc2_bwd_weight", lambda: ict.ict_linear_bwd_weight(self.dY2, self.H1, self.dW2, ws)),
+            ("fc1_bwd_weight", self.bwd_weight(self.dY1, self.X, self.dW1, ws)),
+            ("fc2_bwd_weight", self.bwd_weight(self.dY2, self.H1, self.dW2, ws)),
         ]
         self.units = 6 * 2 * M * 768 * 3072
         self.h2d = [self.X.mant, self.X.exp, self.dY1.mant, self.dY1.exp, self.dY2.mant, self.dY2.exp]
@@ -605,7 +628,8 @@ def side_measurements(ict, torch, peaks, flush, steps):
 
 def base_line(args, step_cls, n_gpus):
     cfg = dict(step_cls.workload)
-    cfg.update(parallelism=f"replicas{n_gpus}" if n_gpus > 1 else "single",
+    mode = "dp" if step_cls.data_parallel else "replicas"
+    cfg.update(parallelism=f"{mode}{n_gpus}" if n_gpus > 1 else "single",
                l2="flushed between steps (512 MB write)")
     return {
         "metric": METRIC, "unit": step_cls.unit, "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
@@ -712,12 +736,14 @@ def main():
         "roofline": roofline(classes, peaks, args.config),
         "clocks": clk,
     })
-    if rank == 0 and not args.no_side and args.config == "vit_ti_mlp":
+    if world > 1 and getattr(step, "exchanged_bytes", 0):
+        line["allreduce_bytes_per_rank_per_step"] = int(step.exchanged_bytes)
+    if rank == 0 and world == 1 and not args.no_side and args.config == "vit_ti_mlp":
         del graph, step
         torch.cuda.empty_cache()
         line["side"] = side_measurements(ict, torch, peaks, flush, max(5, args.steps // 2))
     if rank == 0:
-        if not args.no_cpu:
+        if not args.no_cpu and world == 1:
             try:
                 line["cpu_baseline"] = cpu_baseline(step_cls)
             except Exception as exc:  # pragma: no cover
@@ -725,6 +751,8 @@ def main():
                                         "sample": f"failed: {exc}"}
         print(json.dumps(line))
     if dist:
+        graph = None  # a CUDA graph holding NCCL calls goes before its process group
+        torch.cuda.synchronize()
         dist.barrier()
         dist.destroy_process_group()
 

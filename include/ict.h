@@ -187,6 +187,45 @@ int32_t ict_linear_bwd_data(const ict_tensor *dY, const ict_tensor *W, ict_tenso
 int32_t ict_linear_bwd_weight(const ict_tensor *dY, const ict_tensor *X, ict_tensor *dW,
                               void *ws, size_t ws_bytes, void *stream);
 
+/* Backward-weight Product of a batch split across devices (data-parallel training, one
+ * process per GPU; Abstract: the method trains ResNet and ViT models on ImageNet, whose
+ * batches are split this way).  dW = dY^T X contracts over the batch, so its only
+ * exchange is there; the steps are, on every device with its shard dY_r [K_r][M],
+ * X_r [K_r][N] (K_r may differ, and may be 0):
+ *   1. ict_linear_bwd_weight_targets(dY_r, X_r, e_dy, e_x): the ALIGN_MAX targets of the
+ *      shard, the largest group exponent of each column (ICT_E_ZERO: all groups zero);
+ *   2. element-wise MAX of e_dy and e_x over the devices (an all-reduce on int8; the
+ *      ordering of int8 puts ICT_E_ZERO = -128 below every real exponent);
+ *   3. ict_linear_bwd_weight_partial(dY_r, X_r, e_dy, e_x, acc): the shard aligned to
+ *      those targets and contracted exactly,
+ *        acc[m][n] = sum_k A(dY_r)[k][m] * A(X_r)[k][n],  exponent e_dy[m] + e_x[n];
+ *   4. element-wise SUM of acc over the devices (an all-reduce on int32 / int64; integer
+ *      addition is exact in any order);
+ *   5. ict_requant(acc, bits, M, N, ld_acc, 0, e_dy, e_x, dW).
+ * The result equals ict_linear_bwd_weight on the whole batch bit for bit, whatever the
+ * split.  With one device, steps 2 and 4 are identities.
+ *   e_dy [M], e_x [N]   device int8 target vectors; outputs of step 1, inputs of step 3.
+ *                       Each target must be at least every group exponent of the shard's
+ *                       column, and equal across the columns of one group column, as the
+ *                       maxima of step 2 are when every device uses the same group
+ *                       widths; other values give unspecified, memory-safe results.
+ *   acc                 device, [M][ld_acc] row-major, int64 (acc_bits = 64) or int32
+ *                       (32: allowed only when K_r * 127^2 < 2^31, and the caller must
+ *                       keep the SUM of step 4 below 2^31 in magnitude, e.g. with
+ *                       (sum of all K_r) * 127^2 < 2^31).  16-byte aligned, ld_acc a
+ *                       multiple of 4 (ICT_ERR_ALIGNMENT otherwise).  Fully written.
+ *   ws                  both calls need ict_linear_bwd_weight_partial_workspace() bytes
+ *                       (256-byte aligned); returns 0 for invalid operands.
+ * Operands follow ict_linear_bwd_weight's rules (16-byte aligned, cols multiples of 16,
+ * row-local or uniform groups).  Asynchronous on `stream`. */
+size_t ict_linear_bwd_weight_partial_workspace(const ict_tensor *dY, const ict_tensor *X);
+int32_t ict_linear_bwd_weight_targets(const ict_tensor *dY, const ict_tensor *X, int8_t *e_dy,
+                                      int8_t *e_x, void *ws, size_t ws_bytes, void *stream);
+int32_t ict_linear_bwd_weight_partial(const ict_tensor *dY, const ict_tensor *X,
+                                      const int8_t *e_dy, const int8_t *e_x, void *acc,
+                                      int32_t acc_bits, int64_t ld_acc, void *ws,
+                                      size_t ws_bytes, void *stream);
+
 /* Allocation-free forward Product.  The paper has no counterpart to this entry point;
  * it exists for callers that cannot hand the library a device workspace: integrations
  * whose device memory is reserved up front by a host framework that exposes no

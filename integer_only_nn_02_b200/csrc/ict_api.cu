@@ -212,6 +212,7 @@ struct AlignJob {
     int64_t ld;
     int8_t *e_star;
     int32_t *col_max;  // axis 0: int32 scratch [group columns] for a parallel column max
+    bool given = false;  // the targets are read from e_star, not found from the tensor
 };
 
 // Arguments of one alignment job and how its target exponents are found.
@@ -241,6 +242,10 @@ AlignLaunch plan_align(const AlignJob &j, int sms) {
     a.e_star = j.e_star;
     L.n_exp = n_grp_rows(in) * a.ngc;
     L.blocks = L.used = 0;
+    if (j.given) {  // targets fixed by the caller: no e* pass, the shift kernel reads e_star
+        L.estar = 0;
+        return L;
+    }
     if (j.axis == 1) {
         L.estar = j.transpose ? 1 : 0;
         a.row_estar = j.transpose ? 0 : 1;  // computed inside align_rows_kernel
@@ -278,6 +283,13 @@ int launch_align_n(const AlignJob *jobs, int n, cudaStream_t s) {
         align_work += 2.0 * (double)L[i].a.rows * (double)L[i].a.cols + (double)L[i].n_exp;
     }
     int launches = 0;
+    if (n == 2 && jobs[0].given && jobs[1].given && jobs[0].transpose && jobs[1].transpose) {
+        KTimer kt(s, KC_ALIGN, align_work);
+        const int64_t cols = std::max(L[0].a.cols, L[1].a.cols), rows = std::max(L[0].a.rows, L[1].a.rows);
+        align_transpose_kernel<<<dim3((unsigned)cdiv64(cols, 128), (unsigned)cdiv64(rows, 128), 2), 256, 0, s>>>(P);
+        counted(1);
+        return launch_status();
+    }
     if (n == 2 && (L[0].estar != 2 || L[1].estar != 2)) {  // not pairable on this device: one by one
         int st;
         if ((st = launch_align_n(jobs, 1, s))) return st;
@@ -331,12 +343,13 @@ int launch_align(const AlignJob &j, cudaStream_t s) {
 // The jobs of one call, pairing transposing column alignments with scratch.
 int launch_aligns(const AlignJob *jobs, int n, cudaStream_t s) {
     auto pairable = [&](const AlignJob &j) {
-        return j.axis == 0 && j.transpose && j.col_max && j.t->rows > 0 && j.t->cols > 0 &&
+        return j.axis == 0 && j.transpose && j.col_max && !j.given && j.t->rows > 0 && j.t->cols > 0 &&
                plan_align(j, planning_sms()).estar == 2;
     };
+    auto given_t = [&](const AlignJob &j) { return j.given && j.transpose && j.t->rows > 0 && j.t->cols > 0; };
     int st;
     for (int i = 0; i < n;) {
-        if (i + 1 < n && pairable(jobs[i]) && pairable(jobs[i + 1])) {
+        if (i + 1 < n && ((pairable(jobs[i]) && pairable(jobs[i + 1])) || (given_t(jobs[i]) && given_t(jobs[i + 1])))) {
             if ((st = launch_align_n(jobs + i, 2, s))) return st;
             i += 2;
         } else {
@@ -541,8 +554,9 @@ struct ProductPlan {
 };
 
 // Tiling of D[M][N] = A[M][K] B[N][K]^T with FIT into the row-local groups of `out`.
+// raw: the int32 sums are the result (no FIT), so the product always writes them to ws32.
 ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out, int sms,
-                         bool allow_split, Ws &ws) {
+                         bool allow_split, Ws &ws, bool raw = false) {
     ProductPlan pl;
     pl.bn = pick_bn_waves(M, N, out->g_cols, sms);
     pl.nwg = 2;
@@ -570,14 +584,29 @@ ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out,
     pl.grid = std::min(pl.units, sms);
     const int64_t G = out->g_cols;
     const bool groups_in_tile = (G >= N) ? (N <= pl.bn) : (pl.bn % G == 0 && G % 32 == 0);
-    pl.fused = pl.splits == 1 && groups_in_tile;
+    pl.fused = !raw && pl.splits == 1 && groups_in_tile;
     pl.ws_ld = round_up(N, 32);
     pl.ws32 = pl.fused ? nullptr : (int32_t *)ws.take((size_t)pl.splits * M * pl.ws_ld * 4);
     return pl;
 }
 
+// Sums of the split-K int32 slices of a raw product into the caller's int32 / int64 buffer.
+int launch_sum_slices(const ProductPlan &pl, int64_t M, int64_t N, void *acc, int bits, int64_t ld_acc,
+                      cudaStream_t s) {
+    const int64_t vecs = M * (N / 4);
+    if (vecs == 0) return ICT_OK;
+    KTimer kt(s, KC_REQUANT, (double)M * (double)N * (4.0 * pl.splits + bits / 8.0));
+    const unsigned grid = (unsigned)cdiv64(vecs, 256);
+    if (bits == 64)
+        sum_slices_kernel<true><<<grid, 256, 0, s>>>(pl.ws32, pl.splits, M * pl.ws_ld, M, N, pl.ws_ld, acc, ld_acc);
+    else
+        sum_slices_kernel<false><<<grid, 256, 0, s>>>(pl.ws32, pl.splits, M * pl.ws_ld, M, N, pl.ws_ld, acc, ld_acc);
+    counted(1);
+    return launch_status();
+}
+
 int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const ProductPlan &pl,
-                cudaStream_t s) {
+                cudaStream_t s, void *raw_acc = nullptr, int raw_bits = 0, int64_t raw_ld = 0) {
     const int64_t M = A.rows, N = B.rows, K = A.k;
     CUtensorMap ta, tb;
     int st;
@@ -614,6 +643,7 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K)))
         return st;
     if (pl.fused) return ICT_OK;
+    if (raw_acc) return launch_sum_slices(pl, M, N, raw_acc, raw_bits, raw_ld, s);
     RequantArgs a;
     memset(&a, 0, sizeof(a));
     a.v32 = pl.ws32;
@@ -703,6 +733,114 @@ int linear_entry(int op, const ict_tensor *a, const ict_tensor *b, ict_tensor *o
     if ((st = plan_linear(op, a, b, out, w, &lp))) return st;
     if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
     return run_linear(lp, (cudaStream_t)stream);
+}
+
+// ---- backward weight of a batch split across devices
+//
+// dW = dY^T X contracts over the batch.  With the batch split, every device aligns its
+// shard to targets that hold for the whole batch (the maxima over all shards, found by
+// ict_linear_bwd_weight_targets on each device and a MAX reduction between them) and
+// contracts it exactly; the integer sums of all shards add up to the sums of the whole
+// batch, which one FIT (ict_requant) turns into the single-device result bit for bit.
+
+// Operand whose contracted index runs along the tensor's rows, aligned per column to
+// caller-given targets and transposed into K-major rows.
+Operand operand_cols_given(const ict_tensor *t, const int8_t *e_target, Ws &ws, AlignJob *jobs, int *njobs) {
+    const int64_t ld = round_up(t->rows, 16);
+    int8_t *m = (int8_t *)ws.take((size_t)t->cols * ld);
+    AlignJob j{t, 0, true, m, ld, const_cast<int8_t *>(e_target), nullptr};
+    j.given = true;
+    jobs[(*njobs)++] = j;
+    return Operand{m, t->cols, t->rows, ld, e_target, 1};
+}
+
+int check_split_operands(const ict_tensor *dY, const ict_tensor *X) {
+    int st;
+    if ((st = check_tensor(dY)) || (st = check_tensor(X))) return st;
+    if (dY->rows != X->rows) return ICT_ERR_INVALID_ARG;
+    if ((st = check_vec(dY)) || (st = check_vec(X))) return st;
+    return ICT_OK;
+}
+
+struct TargetsPlan {
+    AlignJob jobs[2];
+    AlignLaunch L[2];
+};
+
+int plan_targets(const ict_tensor *dY, const ict_tensor *X, int8_t *e_dy, int8_t *e_x, Ws &ws, TargetsPlan *tp) {
+    const ict_tensor *t[2] = {dY, X};
+    int8_t *e[2] = {e_dy, e_x};
+    for (int i = 0; i < 2; ++i) {
+        int32_t *cm = (int32_t *)ws.take((size_t)n_grp_cols(t[i]) * 4);
+        tp->jobs[i] = AlignJob{t[i], 0, false, nullptr, 0, e[i], cm};
+        tp->L[i] = plan_align(tp->jobs[i], planning_sms());
+    }
+    return ICT_OK;
+}
+
+int run_targets(const TargetsPlan &tp, cudaStream_t s) {
+    const int64_t K = tp.jobs[0].t->rows;
+    if (K == 0) {  // no rows: every target is E_ZERO
+        for (int i = 0; i < 2; ++i)
+            if (tp.jobs[i].t->cols &&
+                cudaMemsetAsync(tp.jobs[i].e_star, 0x80, (size_t)tp.jobs[i].t->cols, s) != cudaSuccess)
+                return ICT_ERR_CUDA;
+        return ICT_OK;
+    }
+    const bool paired = tp.L[0].estar == 2 && tp.L[1].estar == 2;
+    if (!paired) {  // one block per group column, no scratch
+        for (int i = 0; i < 2; ++i) {
+            const AlignArgs &a = tp.L[i].a;
+            KTimer kt(s, KC_ESTAR, (double)tp.L[i].n_exp + (double)a.cols);
+            estar_cols_kernel<<<(unsigned)a.ngc, 256, 0, s>>>(a);
+            counted(1);
+        }
+        return launch_status();
+    }
+    AlignPair P;
+    memset(&P, 0, sizeof(P));
+    double work = 0;
+    for (int i = 0; i < 2; ++i) {
+        P.a[i] = tp.L[i].a;
+        P.cm[i] = tp.jobs[i].col_max;
+        P.used[i] = tp.L[i].used;
+        work += (double)tp.L[i].n_exp + 8.0 * (double)tp.L[i].a.ngc + (double)tp.L[i].a.cols;
+        if (cudaMemsetAsync(tp.jobs[i].col_max, 0x80, (size_t)tp.L[i].a.ngc * 4, s) != cudaSuccess)
+            return ICT_ERR_CUDA;
+    }
+    KTimer kt(s, KC_ESTAR, work);
+    const int64_t ngc = std::max(P.a[0].ngc, P.a[1].ngc), cols = std::max(P.a[0].cols, P.a[1].cols);
+    estar_cols_scratch_kernel<<<dim3((unsigned)std::max(tp.L[0].blocks, tp.L[1].blocks), 2), 256, (size_t)ngc * 4,
+                                s>>>(P);
+    estar_expand_kernel<<<dim3((unsigned)cdiv64(cols, 256), 2), 256, 0, s>>>(P);
+    counted(2);
+    return launch_status();
+}
+
+struct PartialPlan {
+    AlignJob jobs[2];
+    int njobs;
+    Operand A, B;
+    ProductPlan pp;
+    ict_tensor shape;  // [N][K] with one group per row: tiling only, nothing is written to it
+    int64_t M, N, K;
+};
+
+int plan_partial(const ict_tensor *dY, const ict_tensor *X, const int8_t *e_dy, const int8_t *e_x, Ws &ws,
+                 PartialPlan *pp) {
+    pp->M = dY->cols, pp->N = X->cols, pp->K = dY->rows;
+    pp->njobs = 0;
+    if (pp->M == 0 || pp->N == 0 || pp->K == 0) return ICT_OK;
+    pp->A = operand_cols_given(dY, e_dy, ws, pp->jobs, &pp->njobs);
+    pp->B = operand_cols_given(X, e_x, ws, pp->jobs, &pp->njobs);
+    memset(&pp->shape, 0, sizeof(pp->shape));
+    pp->shape.rows = pp->M;
+    pp->shape.cols = pp->N;
+    pp->shape.ld = pp->N;
+    pp->shape.g_rows = 1;
+    pp->shape.g_cols = (int32_t)pp->N;
+    pp->pp = plan_product(pp->M, pp->N, pp->K, &pp->shape, planning_sms(), true, ws, true);
+    return ICT_OK;
 }
 
 // ---- convolution (implicit GEMM, NHWC / KRSC, "same" 3x3-style, stride 1)
@@ -1336,6 +1474,54 @@ int32_t ict_linear_bwd_weight(const ict_tensor *dY, const ict_tensor *X, ict_ten
     return linear_entry(ICT_OP_LINEAR_BWD_WEIGHT, dY, X, dW, ws, ws_bytes, stream);
 }
 
+size_t ict_linear_bwd_weight_partial_workspace(const ict_tensor *dY, const ict_tensor *X) {
+    if (check_split_operands(dY, X) != ICT_OK) return 0;
+    Ws wt = make_ws(nullptr, 0, true), wp = make_ws(nullptr, 0, true);
+    TargetsPlan tp;
+    PartialPlan pp;
+    plan_targets(dY, X, nullptr, nullptr, wt, &tp);
+    plan_partial(dY, X, nullptr, nullptr, wp, &pp);
+    return std::max<size_t>(std::max(wt.used, wp.used), 256);
+}
+int32_t ict_linear_bwd_weight_targets(const ict_tensor *dY, const ict_tensor *X, int8_t *e_dy, int8_t *e_x,
+                                      void *ws, size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_split_operands(dY, X))) return st;
+    if ((dY->cols && !e_dy) || (X->cols && !e_x)) return ICT_ERR_INVALID_ARG;
+    if (!ws || ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    Ws w = make_ws(ws, ws_bytes, false);
+    TargetsPlan tp;
+    plan_targets(dY, X, e_dy, e_x, w, &tp);
+    if (w.used > ws_bytes) return ICT_ERR_WORKSPACE;
+    return run_targets(tp, (cudaStream_t)stream);
+}
+int32_t ict_linear_bwd_weight_partial(const ict_tensor *dY, const ict_tensor *X, const int8_t *e_dy,
+                                      const int8_t *e_x, void *acc, int32_t acc_bits, int64_t ld_acc,
+                                      void *ws, size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_split_operands(dY, X))) return st;
+    const int64_t M = dY->cols, N = X->cols, K = dY->rows;
+    if (acc_bits != 32 && acc_bits != 64) return ICT_ERR_INVALID_ARG;
+    if (ld_acc < N || (M && N && !acc) || (M && !e_dy) || (N && !e_x)) return ICT_ERR_INVALID_ARG;
+    if (!aligned16(acc) || (ld_acc & 3)) return ICT_ERR_ALIGNMENT;
+    if (acc_bits == 32 && K * 127 * 127 >= (int64_t(1) << 31)) return ICT_ERR_LAYOUT;
+    if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    if (M == 0 || N == 0) return ICT_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (K == 0) {  // empty shard: its sums are zero
+        if (cudaMemsetAsync(acc, 0, (size_t)((M - 1) * ld_acc + N) * (acc_bits / 8), s) != cudaSuccess)
+            return ICT_ERR_CUDA;
+        return ICT_OK;
+    }
+    Ws w = make_ws(ws, ws_bytes, false);
+    PartialPlan pp;
+    plan_partial(dY, X, e_dy, e_x, w, &pp);
+    if (w.used > ws_bytes || !ws) return ICT_ERR_WORKSPACE;
+    if ((st = launch_aligns(pp.jobs, pp.njobs, s))) return st;
+    return run_product(pp.A, pp.B, &pp.shape, pp.pp, s, acc, acc_bits, ld_acc);
+}
 size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d) {
     if (!d || d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1 || d->k < 1 || d->r < 1 || d->s < 1)
         return 0;

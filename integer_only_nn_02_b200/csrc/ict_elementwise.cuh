@@ -786,6 +786,53 @@ __global__ void __launch_bounds__(256) sum_slices_t_kernel(const int32_t *in, in
     }
 }
 
+// Sum of split-K int32 slices in place of layout: out[r][c] = sum_s in[s][r][c], stored
+// as int64 (OUT64) or int32 (the caller guarantees the sums fit).  Each thread sums four
+// adjacent columns with 16-byte loads, four slices in flight (cols, ld and ld_out are
+// multiples of 4; in and out 16-byte aligned).
+template <bool OUT64>
+__global__ void __launch_bounds__(256) sum_slices_kernel(const int32_t *in, int nsplit, int64_t split_stride,
+                                                         int64_t rows, int64_t cols, int64_t ld, void *out,
+                                                         int64_t ld_out) {
+    const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 4-column vector
+    const int64_t qpr = cols >> 2;
+    if (q >= rows * qpr) return;
+    const int64_t r = idiv(q, qpr), c = (q - r * qpr) * 4;
+    const int32_t *src = in + r * ld + c;
+    int64_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+    int sp = 0;
+    for (; sp + 4 <= nsplit; sp += 4) {
+        const int4 a = *reinterpret_cast<const int4 *>(src + sp * split_stride);
+        const int4 b = *reinterpret_cast<const int4 *>(src + (sp + 1) * split_stride);
+        const int4 d = *reinterpret_cast<const int4 *>(src + (sp + 2) * split_stride);
+        const int4 e = *reinterpret_cast<const int4 *>(src + (sp + 3) * split_stride);
+        s0 += ((int64_t)a.x + b.x) + ((int64_t)d.x + e.x), s1 += ((int64_t)a.y + b.y) + ((int64_t)d.y + e.y);
+        s2 += ((int64_t)a.z + b.z) + ((int64_t)d.z + e.z), s3 += ((int64_t)a.w + b.w) + ((int64_t)d.w + e.w);
+    }
+    for (; sp < nsplit; ++sp) {
+        const int4 a = *reinterpret_cast<const int4 *>(src + sp * split_stride);
+        s0 += a.x, s1 += a.y, s2 += a.z, s3 += a.w;
+    }
+    if constexpr (OUT64) {
+        int64_t *o = static_cast<int64_t *>(out) + r * ld_out + c;
+        reinterpret_cast<longlong2 *>(o)[0] = make_longlong2(s0, s1);
+        reinterpret_cast<longlong2 *>(o)[1] = make_longlong2(s2, s3);
+    } else {
+        int32_t *o = static_cast<int32_t *>(out) + r * ld_out + c;
+        *reinterpret_cast<int4 *>(o) = make_int4((int)s0, (int)s1, (int)s2, (int)s3);
+    }
+}
+
+// Per-column e* from the per-group-column maxima of the column scratch form, for up to
+// two jobs (blockIdx.y): e_star[j] = the maximum of column j's group column, E_ZERO when
+// every group of it is zero.
+__global__ void estar_expand_kernel(const __grid_constant__ AlignPair P) {
+    const AlignArgs &a = P.a[blockIdx.y];
+    const int32_t *col_max = P.cm[blockIdx.y];
+    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j < a.cols) a.e_star[j] = (int8_t)estar_of(col_max[idiv(j, a.g_cols)]);
+}
+
 // A wait on an mbarrier that never completes, bounded by limit_ns: raises
 // ICT_ERR_DEVICE_TIMEOUT and returns (self-test of the bounded-wait path).
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {

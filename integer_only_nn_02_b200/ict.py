@@ -71,6 +71,9 @@ _SIGS = {
     "ict_linear_fwd_noalloc": ([_P(ict_tensor)] * 3 + [_vp], _i32),
     "ict_linear_bwd_data": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
     "ict_linear_bwd_weight": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_linear_bwd_weight_partial_workspace": ([_P(ict_tensor)] * 2, _sz),
+    "ict_linear_bwd_weight_targets": ([_P(ict_tensor)] * 2 + [_vp, _vp, _vp, _sz, _vp], _i32),
+    "ict_linear_bwd_weight_partial": ([_P(ict_tensor)] * 2 + [_vp, _vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
     "ict_conv_workspace": ([_i32, _P(ict_conv_desc)], _sz),
     "ict_conv_implicit_gemm": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
     "ict_sgd_momentum_step": ([_P(ict_tensor), _P(ict_tensor), _P(ict_tensor), _P(ict_sgd_params), _vp], _i32),
@@ -241,6 +244,26 @@ def ict_linear_bwd_data(dY: DevCE, W: DevCE, dX: DevCE, ws=None, stream=None):
 
 def ict_linear_bwd_weight(dY: DevCE, X: DevCE, dW: DevCE, ws=None, stream=None):
     _linear(lib.ict_linear_bwd_weight, "ict_linear_bwd_weight", dY, X, dW, ws, stream)
+
+
+def ict_linear_bwd_weight_partial_workspace(dY: DevCE, X: DevCE) -> int:
+    cy, cx = dY.c(), X.c()
+    return int(lib.ict_linear_bwd_weight_partial_workspace(ctypes.byref(cy), ctypes.byref(cx)))
+
+
+def ict_linear_bwd_weight_targets(dY: DevCE, X: DevCE, e_dy: torch.Tensor, e_x: torch.Tensor, ws, stream=None):
+    cy, cx = dY.c(), X.c()
+    _check(lib.ict_linear_bwd_weight_targets(ctypes.byref(cy), ctypes.byref(cx), _ptr(e_dy), _ptr(e_x), _ptr(ws),
+                                             ws.numel(), _stream(stream)), "ict_linear_bwd_weight_targets")
+
+
+def ict_linear_bwd_weight_partial(dY: DevCE, X: DevCE, e_dy: torch.Tensor, e_x: torch.Tensor, acc: torch.Tensor,
+                                  ws, stream=None):
+    bits = {torch.int32: 32, torch.int64: 64}[acc.dtype]
+    cy, cx = dY.c(), X.c()
+    _check(lib.ict_linear_bwd_weight_partial(ctypes.byref(cy), ctypes.byref(cx), _ptr(e_dy), _ptr(e_x), _ptr(acc),
+                                             bits, acc.stride(0), _ptr(ws), ws.numel(), _stream(stream)),
+           "ict_linear_bwd_weight_partial")
 
 
 def conv_desc(d: dict) -> ict_conv_desc:

@@ -71,6 +71,8 @@ def lib():
         L = _lib
         L.oracle_requant.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
                                      ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, P(_OT)]
+        L.oracle_align_to.argtypes = [P(_OT), ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_int64, ctypes.c_int]
         L.oracle_align.argtypes = [P(_OT), ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
                                    ctypes.c_int, ctypes.c_void_p]
         for name in ("oracle_linear_fwd", "oracle_linear_bwd_data", "oracle_linear_bwd_weight",
@@ -156,6 +158,18 @@ def align(t: CE, axis: int, transpose: bool = False):
     code = lib().oracle_align(ctypes.byref(_ot(t)), axis, _ptr(out), shape[1], int(transpose), _ptr(e))
     _check(code, "align")
     return out, e
+
+
+def align_to(t: CE, axis: int, e_target: np.ndarray, transpose: bool = False) -> np.ndarray:
+    """ALIGN_MAX to given target exponents (one per non-contracted index, each at least
+    the group exponents it covers); returns the aligned mantissas."""
+    shape = (t.cols, t.rows) if transpose else (t.rows, t.cols)
+    out = np.zeros(shape, np.int8)
+    e = np.ascontiguousarray(e_target, np.int8)
+    assert e.shape == ((t.rows if axis == 1 else t.cols),)
+    code = lib().oracle_align_to(ctypes.byref(_ot(t)), axis, _ptr(e), _ptr(out), shape[1], int(transpose))
+    _check(code, "align_to")
+    return out
 
 
 def _product(name, a, b, rows, cols, g_rows, g_cols):

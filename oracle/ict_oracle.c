@@ -301,6 +301,31 @@ int oracle_align(const o_tensor *in, int axis, int8_t *out, int64_t ld_out, int 
     return ORC_OK;
 }
 
+/* ALIGN_MAX to targets fixed elsewhere.  When a batch is split across devices, the
+ * exponent an operand is aligned to along the contracted (batch) index is the largest
+ * group exponent over ALL the shards, not only the local one (reading of the Sum
+ * primitive, Table 6 Eq. 6, applied to the whole batch: training on a split batch must
+ * compute what one device computes on all of it).  e_target has one entry per
+ * non-contracted index (rows for axis 1, cols for axis 0); every entry must be at least
+ * every non-E_ZERO group exponent it covers.  Each mantissa becomes
+ * RNE(C * 2^(e - target)); E_ZERO groups and zero mantissas give 0. */
+int oracle_align_to(const o_tensor *in, int axis, const int8_t *e_target, int8_t *out,
+                    int64_t ld_out, int transpose) {
+    int st = check_input(in);
+    if (st) return st;
+    if (!out || !e_target || (axis != 0 && axis != 1)) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < in->rows; i++)
+        for (int64_t j = 0; j < in->cols; j++) {
+            int t = e_target[axis == 1 ? i : j];
+            int e = exp_at(in, i, j), c = mant_at(in, i, j);
+            if (e != E_ZERO && (t == E_ZERO || t < e)) return ORC_ERR_ARG;
+            int q = (c == 0 || e == E_ZERO) ? 0 : (int)rne_scale(c, e - t);
+            if (transpose) out[j * ld_out + i] = (int8_t)q;
+            else out[i * ld_out + j] = (int8_t)q;
+        }
+    return ORC_OK;
+}
+
 /* dense aligned copy (rows x cols, ld = cols) + exponent vector */
 static int align_dense(const o_tensor *t, int axis, int8_t **m, int8_t **e) {
     *m = malloc(t->rows * t->cols + 1);

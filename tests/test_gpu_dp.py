@@ -1,0 +1,109 @@
+"""GPU parity of the data-parallel backward weight (ict_linear_bwd_weight_targets /
+_partial + ict_requant): a batch split into shards, each shard's steps run on the one
+GPU in turn, the MAX of the targets and the SUM of the integer sums taken by the test
+between them (what the all-reduces of integer_only_nn_02_b200.dp do across GPUs).  The
+result must equal the single-device oracle on the whole batch, bit for bit; at the
+ViT-B size, where the oracle is too slow, it must equal the single-device GPU call,
+which the parity suite checks against the oracle at that size."""
+import numpy as np
+import pytest
+
+import oracle
+from integer_only_nn_02_b200.workloads import CE
+from tests.test_oracle_pins import rand_ce
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ict():
+    from integer_only_nn_02_b200 import ict as _ict
+
+    return _ict
+
+
+def same(got: CE, ref: CE, what=""):
+    bad = np.argwhere(got.mant != ref.mant)
+    assert bad.size == 0, f"{what}: {len(bad)} mantissas differ, first {bad[:5].tolist()}"
+    bad = np.argwhere(got.exp != ref.exp)
+    assert bad.size == 0, f"{what}: {len(bad)} exponents differ, first {bad[:5].tolist()}"
+
+
+def shard(t: CE, a: int, b: int) -> CE:
+    return CE(t.mant[a:b].copy(), t.exp[a:b].copy(), 1, t.g_cols)
+
+
+def split_batch_dw(ict, dY: CE, X: CE, cuts, bits, check_targets=True):
+    """The five steps of the split-batch backward weight, shards run one after another."""
+    import torch
+
+    M, N = dY.cols, X.cols
+    parts = [(shard(dY, a, b), shard(X, a, b)) for a, b in zip(cuts[:-1], cuts[1:])]
+    devs = [(ict.DevCE.from_host(p), ict.DevCE.from_host(q)) for p, q in parts]
+    ws = torch.empty(max(ict.ict_linear_bwd_weight_partial_workspace(a, b) for a, b in devs), dtype=torch.uint8,
+                     device="cuda")
+    targets = []
+    for (hdy, hx), (ddy, dx) in zip(parts, devs):
+        e_dy = torch.empty(M, dtype=torch.int8, device="cuda")
+        e_x = torch.empty(N, dtype=torch.int8, device="cuda")
+        ict.ict_linear_bwd_weight_targets(ddy, dx, e_dy, e_x, ws)
+        if check_targets:
+            assert np.array_equal(e_dy.cpu().numpy(), oracle.align(hdy, 0)[1]), "targets of dY"
+            assert np.array_equal(e_x.cpu().numpy(), oracle.align(hx, 0)[1]), "targets of X"
+        targets.append(torch.cat([e_dy, e_x]))
+    e = torch.stack(targets).max(dim=0).values.contiguous()  # the MAX all-reduce
+    e_dy, e_x = e[:M], e[M:]
+    dt = torch.int32 if bits == 32 else torch.int64
+    acc = torch.zeros((M, N), dtype=dt, device="cuda")
+    part = torch.empty((M, N), dtype=dt, device="cuda")
+    for ddy, dx in devs:
+        part.fill_(0x5A5A)  # the call must write every element
+        ict.ict_linear_bwd_weight_partial(ddy, dx, e_dy, e_x, part, ws)
+        acc += part  # the SUM all-reduce
+    dW = ict.DevCE.empty(M, N, 1, N)
+    ict.ict_requant(acc, dW, 0, e_dy, e_x)
+    torch.cuda.synchronize()
+    code, raw = ict.ict_get_device_status()
+    assert code == 0, (code, raw)
+    return dW.to_host()
+
+
+@pytest.mark.parametrize("K,M,N,g,cuts,bits", [
+    (1000, 192, 768, 32, [0, 337, 337, 1000], 32),   # three shards, one of them empty
+    (1000, 192, 768, 32, [0, 500, 1000], 64),
+    (300, 64, 48, 16, [0, 7, 300], 64),              # a 7-row shard: one ragged tile
+    (2100, 128, 96, 32, [0, 1, 1024, 2100], 32),     # a one-row shard
+])
+def test_split_batch_matches_oracle(ict, K, M, N, g, cuts, bits):
+    rng = np.random.default_rng(K + M + N)
+    dY = rand_ce(rng, K, M, 1, g, elo=-14, ehi=-3, zero_groups=0.1)
+    X = rand_ce(rng, K, N, 1, g, elo=-9, ehi=-1, zero_groups=0.1)
+    got = split_batch_dw(ict, dY, X, cuts, bits)
+    same(got, oracle.linear_bwd_weight(dY, X), f"split {cuts}")
+
+
+def test_split_batch_vit_b_matches_single_device(ict):
+    """ViT-B fc1 backward weight (12 608 tokens, 3072 x 768) split over four shards."""
+    from integer_only_nn_02_b200 import workloads as wl
+
+    cfg = wl.vit_b_linear_trio(seed=3)
+    dH, X = cfg["dY1"], cfg["X"]
+    K = X.rows
+    got = split_batch_dw(ict, dH, X, [0, 3152, 6304, 9456, K], 32, check_targets=False)
+    dW = ict.linear_bwd_weight(ict.DevCE.from_host(dH), ict.DevCE.from_host(X))
+    same(got, dW.to_host(), "ViT-B fc1 dW")
+
+
+def test_linear_weight_grad_one_rank(ict):
+    """dp.LinearWeightGrad without a process group (one rank) is ict_linear_bwd_weight."""
+    from integer_only_nn_02_b200 import dp
+
+    rng = np.random.default_rng(5)
+    dY = ict.DevCE.from_host(rand_ce(rng, 777, 192, 1, 32, elo=-14, ehi=-3, zero_groups=0.05))
+    X = ict.DevCE.from_host(rand_ce(rng, 777, 768, 1, 32, elo=-9, ehi=-1, zero_groups=0.05))
+    for total in (777, None):
+        g = dp.LinearWeightGrad(dY, X, total_rows=total)
+        assert g.bits == (32 if total else 64)
+        dW = ict.DevCE.empty(192, 768, 1, 768)
+        g(dY, X, dW)
+        same(dW.to_host(), ict.linear_bwd_weight(dY, X).to_host(), f"bits {g.bits}")

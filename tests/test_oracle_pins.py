@@ -168,6 +168,62 @@ def test_align_rounds_to_max_group_exponent(axis, g):
             assert int(m[i, j]) == want
 
 
+@pytest.mark.parametrize("axis", [0, 1])
+@pytest.mark.parametrize("g", [(1, 4), (3, 5), (9, 1)])
+def test_align_to_raised_targets_matches_python_round(axis, g):
+    """ALIGN_MAX to targets above the tensor's own maxima (the maxima of a larger batch):
+    every mantissa is Python's half-to-even round of its exact value at the target."""
+    rng = np.random.default_rng(40 + axis)
+    t = rand_ce(rng, 9, 13, g[0], g[1], zero_groups=0.2)
+    _, e = oracle.align(t, axis=axis)
+    raise_by = rng.integers(0, 10, size=e.shape)
+    target = np.where(e == E_ZERO, rng.integers(-20, 0, size=e.shape), e.astype(np.int64) + raise_by).astype(np.int8)
+    target[0] = E_ZERO if e[0] == E_ZERO else target[0]  # an all-zero index may keep E_ZERO
+    m = oracle.align_to(t, axis, target)
+    assert (oracle.align_to(t, axis, target, transpose=True) == m.T).all()
+    vals = ce_values(t)
+    for i in range(t.rows):
+        for j in range(t.cols):
+            tg = int(target[i if axis == 1 else j])
+            want = 0 if vals[i][j] == 0 else round(vals[i][j] / pow2(tg))
+            assert int(m[i, j]) == want, (i, j)
+
+
+def test_align_to_own_maxima_equals_align():
+    rng = np.random.default_rng(43)
+    t = rand_ce(rng, 17, 24, 1, 8, zero_groups=0.1)
+    for axis in (0, 1):
+        m, e = oracle.align(t, axis=axis)
+        assert (oracle.align_to(t, axis, e) == m).all()
+
+
+def test_align_to_rejects_target_below_a_group():
+    t = CE(np.array([[3, 0], [5, 1]], np.int8), np.array([[-4], [-2]], np.int8), 1, 2)
+    with pytest.raises(oracle.OracleError):
+        oracle.align_to(t, 0, np.array([-3, -3], np.int8))  # row 1's group sits at -2
+
+
+def test_split_batch_sums_reproduce_whole_batch():
+    """Backward weight of a batch split in three (one shard empty): shard-wise alignment to
+    the MAX of the shards' targets, exact int64 sums added over the shards, one FIT.  This
+    is the whole-batch result, bit for bit (integer addition is exact in any order)."""
+    rng = np.random.default_rng(44)
+    K, M, N = 50, 24, 40
+    dY = rand_ce(rng, K, M, 1, 8, elo=-14, ehi=-3, zero_groups=0.1)
+    X = rand_ce(rng, K, N, 1, 8, elo=-9, ehi=-1, zero_groups=0.1)
+    cuts = [(0, 21), (21, 21), (21, K)]
+    shard = lambda t, a, b: CE(t.mant[a:b].copy(), t.exp[a:b].copy(), 1, t.g_cols)
+    parts = [(shard(dY, a, b), shard(X, a, b)) for a, b in cuts]
+    e_dy = np.max([oracle.align(p[0], 0)[1] for p in parts], axis=0).astype(np.int8)
+    e_x = np.max([oracle.align(p[1], 0)[1] for p in parts], axis=0).astype(np.int8)
+    acc = np.zeros((M, N), np.int64)
+    for pdy, px in parts:
+        acc += oracle.align_to(pdy, 0, e_dy).astype(np.int64).T @ oracle.align_to(px, 0, e_x).astype(np.int64)
+    got = oracle.requant(acc, 1, N, 0, row_exp=e_dy, col_exp=e_x)
+    ref = oracle.linear_bwd_weight(dY, X)
+    assert (got.mant == ref.mant).all() and (got.exp == ref.exp).all()
+
+
 # --------------------------------------------------------------------- linear
 
 
