@@ -82,6 +82,9 @@ def lib():
                      "oracle_linear_bwd_weight_acc"):
             getattr(L, name).argtypes = [P(_OT), P(_OT), ctypes.c_void_p, ctypes.c_void_p]
         L.oracle_gelu_fwd.argtypes = [P(_OT), P(_OT)]
+        L.oracle_sum.argtypes = [P(_OT), P(_OT), P(_OT)]
+        L.oracle_relu_fwd.argtypes = [P(_OT), ctypes.c_int, P(_OT)]
+        L.oracle_relu_bwd.argtypes = [P(_OT), P(_OT), ctypes.c_int, P(_OT)]
         L.oracle_conv.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), P(_OT)]
         L.oracle_conv_acc.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), ctypes.c_void_p,
                                       ctypes.c_void_p]
@@ -262,3 +265,25 @@ def gelu_fwd(H: CE) -> CE:
 
 def gelu_bwd(H: CE, dG: CE, g_rows=1, g_cols=32) -> CE:
     return _product("oracle_gelu_bwd", H, dG, H.rows, H.cols, g_rows, g_cols)
+
+
+def sum_(X: CE, Y: CE, g_rows: int, g_cols: int) -> CE:
+    """The Sum primitive: FIT(X + Y) into (g_rows, g_cols) groups."""
+    out = empty_ce(X.rows, X.cols, g_rows, g_cols)
+    _check(lib().oracle_sum(ctypes.byref(_ot(X)), ctypes.byref(_ot(Y)), ctypes.byref(_ot(out))), "sum")
+    return out
+
+
+def relu_fwd(X: CE, six: bool = False) -> CE:
+    """ReLU (or ReLU6) on the mantissas; the exponents are carried through."""
+    out = empty_ce(X.rows, X.cols, X.g_rows, X.g_cols)
+    _check(lib().oracle_relu_fwd(ctypes.byref(_ot(X)), int(six), ctypes.byref(_ot(out))), "relu_fwd")
+    return out
+
+
+def relu_bwd(X: CE, dY: CE, six: bool = False) -> CE:
+    """dY masked where the forward input passed the ReLU (ReLU6); dY's exponents."""
+    out = empty_ce(dY.rows, dY.cols, dY.g_rows, dY.g_cols)
+    _check(lib().oracle_relu_bwd(ctypes.byref(_ot(X)), ctypes.byref(_ot(dY)), int(six), ctypes.byref(_ot(out))),
+           "relu_bwd")
+    return out

@@ -742,6 +742,88 @@ int oracle_gelu_bwd(const o_tensor *H, const o_tensor *dG, o_tensor *dH) {
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Public: Sum (residual add, gradient merge)                                            */
+/* ------------------------------------------------------------------------------------ */
+
+/* Z = FIT(X + Y).  Table 6 lists "Residual add, gradient merge" under the Sum primitive
+ * (Eq. 6, whose text the page does not print).  Reading, the same as for the two-term
+ * sums of the SGD step: every element's two terms x * 2^ex + y * 2^ey are added exactly,
+ * then the result is requantised into Z's groups.  X, Y and Z share one shape; each has
+ * its own group geometry. */
+int oracle_sum(const o_tensor *X, const o_tensor *Y, o_tensor *Z) {
+    int st;
+    if ((st = check_input(X)) || (st = check_input(Y))) return st;
+    if (X->rows != Y->rows || X->cols != Y->cols) return ORC_ERR_ARG;
+    if ((st = check_output(Z, X->rows, X->cols))) return st;
+    int64_t n = X->rows * X->cols;
+    i128 *v = malloc(sizeof(i128) * (n + 1));
+    int *r = malloc(sizeof(int) * (n + 1));
+    for (int64_t i = 0; i < X->rows; i++)
+        for (int64_t j = 0; j < X->cols; j++)
+            two_term(mant_at(X, i, j), exp_at(X, i, j), mant_at(Y, i, j), exp_at(Y, i, j),
+                     &v[i * X->cols + j], &r[i * X->cols + j]);
+    st = fit_matrix(v, r, Z);
+    free(v);
+    free(r);
+    return st;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Public: ReLU / ReLU6 (the Clip primitive)                                             */
+/* ------------------------------------------------------------------------------------ */
+
+/* Clip bound of ReLU6 in a group at exponent e (Table 7: c = min(6 >> e, q_max)): the
+ * integer 6 shifted right by e, a left shift for negative e, then capped at q_max.
+ * Read literally, a right shift truncates, so e = 2 gives 1 and e >= 3 gives 0. */
+static int relu6_bound(int e) {
+    if (e >= 0) return e >= 3 ? 0 : (6 >> e);
+    if (-e >= 5) return QMAX; /* 6 << 5 = 192 already exceeds q_max */
+    int c = 6 << (-e);
+    return c > QMAX ? QMAX : c;
+}
+
+/* Forward ReLU (six = 0: max(C, 0)) or ReLU6 (six = 1: clip(C, 0, c)), Table 7: integer
+ * operations on the mantissas, the exponent carried through unchanged.  Z has X's
+ * shape and group geometry; its exponent grid is a copy of X's. */
+int oracle_relu_fwd(const o_tensor *X, int six, o_tensor *Z) {
+    int st;
+    if ((st = check_input(X))) return st;
+    if ((st = check_output(Z, X->rows, X->cols))) return st;
+    if (Z->g_rows != X->g_rows || Z->g_cols != X->g_cols || (six != 0 && six != 1)) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < X->rows; i++)
+        for (int64_t j = 0; j < X->cols; j++) {
+            int c = mant_at(X, i, j), e = exp_at(X, i, j);
+            int q = c > 0 ? c : 0;
+            if (six && e != E_ZERO) {
+                int b = relu6_bound(e);
+                if (q > b) q = b;
+            }
+            Z->mant[i * Z->ld + j] = (int8_t)q;
+        }
+    memcpy(Z->exp, X->exp, (size_t)(n_grp_rows(X) * n_grp_cols(X)));
+    return ORC_OK;
+}
+
+/* Backward ReLU / ReLU6 (Table 7): dX = dY * 1[C > 0] (ReLU) or dY * 1[0 < C < c]
+ * (ReLU6), C the forward input's mantissa and c the bound of its group.  dX has dY's
+ * shape and groups and dY's exponents (a mask changes no exponent). */
+int oracle_relu_bwd(const o_tensor *X, const o_tensor *dY, int six, o_tensor *dX) {
+    int st;
+    if ((st = check_input(X)) || (st = check_input(dY))) return st;
+    if (X->rows != dY->rows || X->cols != dY->cols || (six != 0 && six != 1)) return ORC_ERR_ARG;
+    if ((st = check_output(dX, dY->rows, dY->cols))) return st;
+    if (dX->g_rows != dY->g_rows || dX->g_cols != dY->g_cols) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < X->rows; i++)
+        for (int64_t j = 0; j < X->cols; j++) {
+            int c = mant_at(X, i, j), e = exp_at(X, i, j);
+            int pass = c > 0 && (!six || c < relu6_bound(e));
+            dX->mant[i * dX->ld + j] = pass ? (int8_t)mant_at(dY, i, j) : 0;
+        }
+    memcpy(dX->exp, dY->exp, (size_t)(n_grp_rows(dY) * n_grp_cols(dY)));
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Introspection for the tests                                                           */
 /* ------------------------------------------------------------------------------------ */
 

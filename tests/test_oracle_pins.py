@@ -488,3 +488,98 @@ def test_input_invariants_are_enforced():
     zero_bad = CE(np.array([[0, 3]], np.int8), np.array([[E_ZERO]], np.int8), 1, 2)
     with pytest.raises(oracle.OracleError):
         oracle.linear_fwd(zero_bad, ok, 1, 1)
+
+
+# --------------------------------------------------------------------- Sum (residual add)
+
+
+@pytest.mark.parametrize("gx,gy,gz", [((1, 4), (1, 4), (1, 4)), ((9, 5), (1, 13), (3, 4)), ((1, 13), (9, 1), (9, 13))])
+@pytest.mark.parametrize("erange", [((-12, -2), (-12, -2)), ((-30, -20), (-3, 5)), ((-127, -90), (10, 40))])
+def test_sum_matches_bruteforce(gx, gy, gz, erange):
+    """FIT(X + Y) against exact rational sums and the brute-force FIT, with exponent gaps
+    from 0 up to beyond the oracle's exact span (its sticky reduction)."""
+    rng = np.random.default_rng(60 + gx[0] + gy[1] + abs(erange[0][0]))
+    X = rand_ce(rng, 9, 13, *gx, *erange[0], zero_groups=0.15)
+    Y = rand_ce(rng, 9, 13, *gy, *erange[1], zero_groups=0.15)
+    Z = oracle.sum_(X, Y, *gz)
+    vx, vy = ce_values(X), ce_values(Y)
+    mant, exps = fit_matrix_brute([[vx[i][j] + vy[i][j] for j in range(13)] for i in range(9)], *gz)
+    assert Z.mant.tolist() == mant and Z.exp.tolist() == exps
+
+
+def test_sum_with_zero_is_requant_of_the_other_term():
+    rng = np.random.default_rng(61)
+    X = rand_ce(rng, 6, 32, 1, 16)
+    Zr = CE(np.zeros((6, 32), np.int8), np.full((6, 2), E_ZERO, np.int8), 1, 16)
+    # every group holds a mantissa of magnitude >= 64, so X is its own FIT
+    assert (np.abs(X.mant.astype(int)).reshape(6, 2, 16).max(axis=2) >= 64).all()
+    Z = oracle.sum_(X, Zr, 1, 16)
+    assert (Z.mant == X.mant).all() and (Z.exp == X.exp).all()
+    assert (oracle.sum_(Zr, Zr, 1, 16).exp == E_ZERO).all()
+
+
+def test_sum_of_equal_terms_doubles():
+    """x + x = 2x: the exponent rises by one exactly where the mantissa cannot double."""
+    rng = np.random.default_rng(62)
+    X = rand_ce(rng, 5, 48, 1, 16)
+    Z = oracle.sum_(X, X, 1, 16)
+    vx, vz = ce_values(X), ce_values(Z)
+    for i in range(5):
+        for j in range(48):
+            assert vz[i][j] == 2 * vx[i][j]  # doubling is exact in (C, e+1)
+
+
+# --------------------------------------------------------------------- ReLU / ReLU6
+
+
+def _all_mantissas_ce(e_list):
+    """One row per exponent, every mantissa -127..127 once: rows x 255, one group per row."""
+    m = np.tile(np.arange(-127, 128, dtype=np.int8), (len(e_list), 1))
+    return CE(m, np.array(e_list, np.int8).reshape(-1, 1), 1, 255)
+
+
+def test_relu_fwd_matches_torch():
+    import torch
+
+    X = _all_mantissas_ce(list(range(-127, 128, 3)))
+    vals = torch.tensor([[float(v) for v in row] for row in ce_values(X)], dtype=torch.float64)
+    for six in (False, True):
+        Z = oracle.relu_fwd(X, six)
+        assert (Z.exp == X.exp).all()
+        got = torch.tensor([[float(v) for v in row] for row in ce_values(Z)], dtype=torch.float64)
+        if not six:
+            assert torch.equal(got, torch.relu(vals))
+            continue
+        for r, e in enumerate(X.exp[:, 0].tolist()):
+            if e <= 1:  # the bound 6 >> e times 2^e is 6, or q_max * 2^e < 6: exactly relu6
+                assert torch.equal(got[r], torch.nn.functional.relu6(vals[r])), e
+            else:  # 6 >> e truncates: the largest multiple of 2^e not above 6 (0 for e >= 3)
+                cap = (6 >> e) * 2.0 ** e
+                assert torch.equal(got[r], torch.clamp(vals[r], 0.0, cap)), e
+
+
+def test_relu_bwd_matches_torch_autograd():
+    import torch
+
+    rng = np.random.default_rng(63)
+    X = _all_mantissas_ce(list(range(-12, 3)))
+    dY = CE(rng.integers(-127, 128, size=X.mant.shape).astype(np.int8),
+            rng.integers(-20, -5, size=(X.rows, 1)).astype(np.int8), 1, 255)
+    vals = torch.tensor([[float(v) for v in row] for row in ce_values(X)], dtype=torch.float64)
+    up = torch.tensor(dY.mant, dtype=torch.float64)
+    for six, fn in ((False, torch.relu), (True, torch.nn.functional.relu6)):
+        x = vals.clone().requires_grad_(True)
+        fn(x).backward(up)
+        dX = oracle.relu_bwd(X, dY, six)
+        assert (dX.exp == dY.exp).all()
+        got = torch.tensor(dX.mant, dtype=torch.float64)
+        for r, e in enumerate(X.exp[:, 0].tolist()):
+            if six and e <= -5:
+                # c = q_max: the page's mask 0 < C < c also drops C = q_max (value below 6)
+                want = x.grad[r].clone()
+                want[-1] = 0.0
+                assert torch.equal(got[r], want), e
+            elif six and e == 2:  # c = 1: no mantissa lies strictly between 0 and 1
+                assert (got[r] == 0).all()
+            else:
+                assert torch.equal(got[r], x.grad[r]), (six, e)
