@@ -14,6 +14,8 @@ configurations, each a step of its own with its own unit:
   resnet18_conv3x3    3x3 conv fwd, bwd-data, bwd-weight on 128x56x56x64, TOPS
   resnet50_sgd        int-SGD update of a ResNet-50-sized parameter arena, GB/s
   single_linear       64x128 linear layer fwd+bwd+SGD, microseconds per step
+  resnet18_block_tail residual add, ReLU, ReLU backward and gradient merge on the
+                      ResNet-18 stage-1 activations, GB/s
 
 Usage:  python bench.py [--config C] [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 run under torchrun, one rank per GPU, each with its own batch of the
@@ -42,7 +44,7 @@ from integer_only_nn_02_b200 import workloads as wl  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20  # larger than the 126 MB L2
 METRIC = "(C,e) GEMM TOPS fwd+bwd vs INT8 tensor peak; int-SGD update GB/s vs HBM"
-CLASS_NAMES = ["gemm", "sgd", "align", "requant", "gelu", "estar", "other"]  # ict_kernel_class order
+CLASS_NAMES = ["gemm", "sgd", "align", "requant", "gelu", "estar", "other", "pointwise"]  # ict_kernel_class order
 CLASS_KERNELS = {
     "gemm": "gemm_ce_kernel (tcgen05 kind::i8, fused FIT epilogue)",
     "sgd": "sgd_rows_kernel / sgd_vec_kernel",
@@ -51,6 +53,7 @@ CLASS_KERNELS = {
     "gelu": "gelu_fwd_kernel / gelu_bwd_vec_kernel",
     "estar": "estar_rows_kernel / estar_cols_scratch_kernel",
     "other": "fills, weight re-layout, exponent tables",
+    "pointwise": "clip_kernel / sum_rows_kernel / sum_global_*_kernel (ReLU, Sum)",
 }
 
 
@@ -160,6 +163,7 @@ class Step:
         return self.torch.empty(max(int(nbytes), 256), dtype=self.torch.uint8, device="cuda")
 
     data_parallel = False  # True: with several ranks the batch is split and dW all-reduced
+    gemm_bytes = 0  # algorithmic int8 bytes (operands read, results written) of the step's Products
 
     def bwd_weight(self, dY, X, dW, ws):
         """One linear layer's backward-weight call.  On one GPU, the library's single call;
@@ -228,6 +232,7 @@ class MlpStep(Step):
             ("sgd_w2", lambda: ict.ict_sgd_momentum_step(self.W2, self.V2, self.dW2, mom, lr)),
         ]
         self.units = 6 * 2 * M * D * H
+        self.gemm_bytes = 6 * (M * D + D * H + M * H)
         self.h2d = [self.X.mant, self.X.exp, self.dY2.mant, self.dY2.exp]
         self.d2h = [self.W1.mant, self.W1.exp, self.W2.mant, self.W2.exp]
 
@@ -317,6 +322,7 @@ class ConvStep(Step):
             ("bwd_weight", lambda: ict.ict_conv_implicit_gemm(2, d, self.dY, self.X, self.dW, ws)),
         ]
         self.units = 3 * 2 * npix * 64 * 576
+        self.gemm_bytes = 3 * (2 * npix * 64 + 64 * 576)
         self.h2d = [self.X.mant, self.X.exp, self.dY.mant, self.dY.exp]
         self.d2h = [self.dW.mant, self.dW.exp]
 
@@ -362,6 +368,7 @@ class TrioStep(Step):
             ("fc2_bwd_weight", self.bwd_weight(self.dY2, self.H1, self.dW2, ws)),
         ]
         self.units = 6 * 2 * M * 768 * 3072
+        self.gemm_bytes = 6 * (M * 768 + 768 * 3072 + M * 3072)
         self.h2d = [self.X.mant, self.X.exp, self.dY1.mant, self.dY1.exp, self.dY2.mant, self.dY2.exp]
         self.d2h = [self.dW1.mant, self.dW1.exp, self.dW2.mant, self.dW2.exp]
 
@@ -411,8 +418,57 @@ class SgdStep(Step):
         return dt, 5 * c5["numel"] + 5 * c5["W"].rows, "one full update of the 25.6 M-parameter arena"
 
 
+class BlockTailStep(Step):
+    """The pointwise steps around a ResNet-18 stage-1 basic block's convolutions, on its
+    128 x 56 x 56 x 64 activations (channel groups of 32 spanning all pixels): residual
+    add S = FIT(conv_out + identity), A = ReLU(S); backward dS = dA * 1[S > 0] and the
+    gradient merge dX = FIT(dX_conv + dS) at the block input."""
+
+    unit = "GB/s"
+    N_IMG, HW, C, GROUP = 128, 56, 64, 32
+    sample_arg = 128  # images in the oracle's sample: the whole workload, about 7 s
+    workload = {"workload": "resnet18_block_tail", "n": 128, "h": 56, "w": 56, "c": 64, "group": 32,
+                "ops": "sum, relu, relu_bwd, sum"}
+
+    def __init__(self, ict, torch, seed):
+        super().__init__(ict, torch)
+        E = ict.DevCE
+        cfg = wl.resnet18_block_tail(seed=seed, n=self.N_IMG)
+        npix = cfg["Y"].rows
+        self.Y, self.X, self.dA, self.dXc = (E.from_host(cfg[k]) for k in ("Y", "X", "dA", "dXc"))
+        G = self.GROUP
+        self.S, self.A = E.empty(npix, self.C, npix, G), E.empty(npix, self.C, npix, G)
+        self.dS, self.dX = E.empty(npix, self.C, npix, G), E.empty(npix, self.C, npix, G)
+        ws = self.ws(ict.ict_sum_workspace(self.Y, self.X, self.S))
+        self.calls = [
+            ("residual_add", lambda: ict.ict_sum(self.Y, self.X, self.S, ws)),
+            ("relu", lambda: ict.ict_relu_fwd(self.S, False, self.A)),
+            ("relu_bwd", lambda: ict.ict_relu_bwd(self.S, self.dA, False, self.dS)),
+            ("grad_merge", lambda: ict.ict_sum(self.dXc, self.dS, self.dX, ws)),
+        ]
+        n = npix * self.C
+        self.units = (3 + 2 + 3 + 3) * n  # algorithmic bytes: inputs read once, outputs written once
+        self.h2d = [self.Y.mant, self.Y.exp, self.dA.mant, self.dA.exp]
+        self.d2h = [self.dX.mant, self.dX.exp]
+
+    @staticmethod
+    def oracle_step(n_img):
+        import oracle
+
+        cfg = wl.resnet18_block_tail(seed=0, n=n_img)
+        g = (cfg["Y"].rows, BlockTailStep.GROUP)
+        t0 = time.perf_counter()
+        S = oracle.sum_(cfg["Y"], cfg["X"], *g)
+        oracle.relu_fwd(S)
+        dS = oracle.relu_bwd(S, cfg["dA"])
+        oracle.sum_(cfg["dXc"], dS, *g)
+        dt = time.perf_counter() - t0
+        n = cfg["Y"].rows * BlockTailStep.C
+        return dt, 11 * n, f"one full block tail on {n_img} images"
+
+
 STEPS = {"vit_ti_mlp": MlpStep, "vit_b_linear_trio": TrioStep, "resnet18_conv3x3": ConvStep,
-         "resnet50_sgd": SgdStep, "single_linear": LinearStep}
+         "resnet50_sgd": SgdStep, "single_linear": LinearStep, "resnet18_block_tail": BlockTailStep}
 
 
 # --------------------------------------------------------------------- timing
@@ -554,20 +610,40 @@ def measured_traffic(config, kernel_class):
     return None if e is None else e["dram_bytes_per_launch"]
 
 
-def roofline(classes, peaks, config):
+def roofline(classes, peaks, config, gemm_bytes=0):
     """Roofline of the kernel class with the most device time in the step: the
-    tensor-core Product against the INT8 peak (measured dense bf16 x 2, the nominal
-    int8/bf16 ratio), the memory-bound classes against the measured HBM copy rate."""
+    memory-bound classes against the measured HBM copy rate; the tensor-core Product
+    against whichever bound is binding for its shapes: the INT8 peak (measured dense
+    bf16 x 2, the nominal int8/bf16 ratio) for its multiply-adds, or the HBM copy rate
+    for its algorithmic bytes (int8 operands read once, int8 results written once) when
+    moving those takes longer than the multiply-adds (short contractions)."""
     name = max(classes, key=lambda k: classes[k]["ms_per_step"])
     c = classes[name]
     achieved, peak, unit, bound = class_rate(name, c, peaks)
+    alt = None
+    if name == "gemm" and gemm_bytes:
+        t_tensor = c["work_per_step"] / (2.0 * peaks["bf16"] * 1e12)
+        t_hbm = gemm_bytes / (peaks["hbm"] * 1e9)
+        hbm_rate = gemm_bytes / (c["ms_per_step"] * 1e-3) / 1e9
+        if t_hbm > t_tensor:
+            alt = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+                   "frac": round(achieved / peak, 4)}
+            achieved, peak, unit, bound = hbm_rate, peaks["hbm"], "GB/s", "hbm"
+        else:
+            alt = {"bound": "hbm", "achieved": round(hbm_rate, 1), "peak": round(peaks["hbm"], 1), "unit": "GB/s",
+                   "frac": round(hbm_rate / peaks["hbm"], 4)}
     note = (f"INT8 = 2 x {peaks['source']} dense bf16 {peaks['bf16']} TF/s (burst)" if bound == "tensor"
             else f"{peaks['source']} HBM copy bandwidth")
-    return {"kernel": CLASS_KERNELS[name], "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
-            "unit": unit, "frac": round(achieved / peak, 4), "peak_note": note,
-            "traffic": measured_traffic(config, name),
-            "launches_per_step": c["launches_per_step"],
-            "us_per_launch": round(1e3 * c["ms_per_step"] / c["launches_per_step"], 2)}
+    out = {"kernel": CLASS_KERNELS[name], "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1),
+           "unit": unit, "frac": round(achieved / peak, 4), "peak_note": note,
+           "traffic": measured_traffic(config, name),
+           "launches_per_step": c["launches_per_step"],
+           "us_per_launch": round(1e3 * c["ms_per_step"] / c["launches_per_step"], 2)}
+    if alt:
+        out["algorithmic_bytes_per_step" if bound == "hbm" else "ops_per_step"] = (
+            int(gemm_bytes) if bound == "hbm" else c["work_per_step"])
+        out["other_bound"] = alt
+    return out
 
 
 def class_summary(classes, peaks):
@@ -733,7 +809,7 @@ def main():
         "eager_ms_per_step": round(eager_ms, 4),
         "breakdown_ms": {n: round(float(v), 4) for (n, _), v in zip(step.calls, per_call)},
         "kernel_classes": class_summary(classes, peaks),
-        "roofline": roofline(classes, peaks, args.config),
+        "roofline": roofline(classes, peaks, args.config, step.gemm_bytes),
         "clocks": clk,
     })
     if world > 1 and getattr(step, "exchanged_bytes", 0):

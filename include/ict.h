@@ -128,7 +128,8 @@ typedef enum {
     ICT_KC_REQUANT = 3, /* FIT of int32 / int64 values (split-K combine) */
     ICT_KC_GELU = 4,    /* GELU forward / backward */
     ICT_KC_ESTAR = 5,   /* target exponents e* of ALIGN_MAX (maxima of group exponents) */
-    ICT_KC_OTHER = 6    /* fills, weight re-layout and exponent tables */
+    ICT_KC_OTHER = 6,   /* fills, weight re-layout and exponent tables */
+    ICT_KC_POINTWISE = 7 /* ReLU / ReLU6 and Sum (residual add) */
 } ict_kernel_class;
 int32_t ict_timing_enable(int32_t on);
 int32_t ict_timing_read(int32_t kernel_class, double *ms_total, int64_t *launches, double *work,
@@ -285,6 +286,36 @@ int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W,
 /*        partition.                                                                    */
 int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream);
 int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* ReLU / ReLU6, the Clip primitive (Table 6: "ReLU / ReLU6 -> Clip"; Table 7): integer  */
+/* operations on the mantissas C, the exponent carried through unchanged.              */
+/*   six = 0: ReLU    forward  Z = max(C, 0)          backward dX = dY * 1[C > 0]       */
+/*   six = 1: ReLU6   forward  Z = clip(C, 0, c)      backward dX = dY * 1[0 < C < c]   */
+/*   c = min(6 >> e, 127) for the group exponent e of C: 6 shifted right by e (left for  */
+/*   e < 0), truncating, so e = 2 gives 1 and e >= 3 gives 0; taken literally, the     */
+/*   backward mask also drops C = 127 where c = 127 (e <= -5).                          */
+/* Forward: Z has X's shape and group geometry and receives a copy of X's exponents.    */
+/* Backward: X is the forward input; dX has dY's shape and groups and receives a copy   */
+/* of dY's exponents.  Tensors: cols multiple of 16, mantissas and ld 16-byte aligned,  */
+/* group widths multiples of 16 (or one group per row).                                 */
+int32_t ict_relu_fwd(const ict_tensor *X, int32_t six, ict_tensor *Z, void *stream);
+int32_t ict_relu_bwd(const ict_tensor *X, const ict_tensor *dY, int32_t six, ict_tensor *dX,
+                     void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* Sum (Table 6: "Residual add, gradient merge -> Sum", Eq. 6): Z = FIT(X + Y), every   */
+/* element's two terms x * 2^ex + y * 2^ey added exactly, then requantised into Z's     */
+/* groups.  X, Y, Z share one shape and one group partition: row-local groups (g_rows  */
+/* = 1, as the linear layers produce) or groups spanning all rows (g_rows >= rows, the  */
+/* pixel-uniform channel groups of convolution activations; at most 8192 group        */
+/* columns).  Group widths are multiples of 16 or span the row; cols a multiple of 16;  */
+/* mantissas and ld 16-byte aligned.  Groups spanning all rows need an int32 per group  */
+/* column of workspace (ict_sum_workspace; 0 for row-local groups, where ws may be     */
+/* NULL); the result is written in two streaming passes.                              */
+size_t ict_sum_workspace(const ict_tensor *X, const ict_tensor *Y, const ict_tensor *Z);
+int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *ws,
+                size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

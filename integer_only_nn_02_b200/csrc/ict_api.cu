@@ -12,6 +12,7 @@
 #include "ict_device.cuh"
 #include "ict_elementwise.cuh"
 #include "ict_gemm.cuh"
+#include "ict_pointwise.cuh"
 
 using namespace ict;
 
@@ -61,7 +62,8 @@ std::atomic<uint64_t> g_launches{0};
 void counted(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 // ---- optional per-kernel-class device timing (measurement only; off by default)
-enum { KC_GEMM = 0, KC_SGD = 1, KC_ALIGN = 2, KC_REQUANT = 3, KC_GELU = 4, KC_ESTAR = 5, KC_OTHER = 6, KC_N = 7 };
+enum { KC_GEMM = 0, KC_SGD = 1, KC_ALIGN = 2, KC_REQUANT = 3, KC_GELU = 4, KC_ESTAR = 5, KC_OTHER = 6, KC_POINTWISE = 7,
+       KC_N = 8 };
 struct TimedLaunch {
     int kc;
     cudaEvent_t a, b;
@@ -1318,6 +1320,71 @@ int noalloc_scratch(void **out) {
 
 // ====================================================================== C ABI
 
+// ---- pointwise primitives (ReLU / ReLU6, Sum)
+
+// A tensor streamed by 16-byte vectors whose groups never straddle a vector.
+int check_pointwise(const ict_tensor *t) {
+    int st;
+    if ((st = check_tensor(t))) return st;
+    return check_vec(t);
+}
+bool same_groups(const ict_tensor *a, const ict_tensor *b) {
+    return a->rows == b->rows && a->cols == b->cols && clamp_div(a->g_rows, a->rows) == clamp_div(b->g_rows, b->rows) &&
+           clamp_div(a->g_cols, a->cols) == clamp_div(b->g_cols, b->cols);
+}
+unsigned stream_grid(int64_t nvec, int per_thread) {
+    int sms = 148;
+    device_info(&sms);
+    const int64_t want = cdiv64(nvec, 256 * (int64_t)per_thread);
+    return (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
+}
+
+int launch_clip(const ict_tensor *X, const ict_tensor *dY, int six, ict_tensor *out, cudaStream_t s) {
+    ClipArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = X->mant;
+    a.x_exp = X->exp;
+    a.ldx = X->ld;
+    a.gx_rows = clamp_div(X->g_rows, X->rows);
+    a.gx_cols = clamp_div(X->g_cols, X->cols);
+    a.ngcx = n_grp_cols(X);
+    if (dY) {
+        a.dy = dY->mant;
+        a.dy_exp = dY->exp;
+        a.ldy = dY->ld;
+    }
+    a.out = out->mant;
+    a.out_exp = out->exp;
+    a.ldo = out->ld;
+    a.rows = X->rows;
+    a.cols = X->cols;
+    a.six = six;
+    a.n_exp = n_grp_rows(out) * n_grp_cols(out);
+    const int64_t nvec = a.rows * (a.cols >> 4);
+    if (std::max(nvec, a.n_exp) == 0) return ICT_OK;
+    KTimer kt(s, KC_POINTWISE, (double)a.rows * (double)a.cols * (dY ? 3.0 : 2.0) + 2.0 * (double)a.n_exp);
+    const unsigned grid = stream_grid(std::max(nvec, a.n_exp), 4);
+    if (dY) clip_kernel<true><<<grid, 256, 0, s>>>(a);
+    else clip_kernel<false><<<grid, 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+// Sum operands: one shape and one group partition, row-local (g_rows = 1) or spanning
+// all rows; group columns a multiple of 16 wide unless one spans the row.
+int check_sum(const ict_tensor *X, const ict_tensor *Y, const ict_tensor *Z, bool *global) {
+    int st;
+    if ((st = check_pointwise(X)) || (st = check_pointwise(Y)) || (st = check_pointwise(Z))) return st;
+    if (X->rows != Y->rows || X->cols != Y->cols || X->rows != Z->rows || X->cols != Z->cols)
+        return ICT_ERR_INVALID_ARG;
+    if (!same_groups(X, Y) || !same_groups(X, Z)) return ICT_ERR_LAYOUT;
+    const int gr = clamp_div(X->g_rows, X->rows);
+    *global = X->rows > 1 && gr >= X->rows;
+    if (gr != 1 && !*global) return ICT_ERR_LAYOUT;
+    if (*global && n_grp_cols(X) > 8192) return ICT_ERR_LAYOUT;
+    return ICT_OK;
+}
+
 extern "C" {
 
 const char *ict_status_string(int32_t status) {
@@ -1686,6 +1753,80 @@ int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, 
     } else {
         gelu_bwd_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, s>>>(a);
     }
+    counted(1);
+    return launch_status();
+}
+
+int32_t ict_relu_fwd(const ict_tensor *X, int32_t six, ict_tensor *Z, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_pointwise(X)) || (st = check_pointwise(Z))) return st;
+    if (six != 0 && six != 1) return ICT_ERR_INVALID_ARG;
+    if (Z->rows != X->rows || Z->cols != X->cols) return ICT_ERR_INVALID_ARG;
+    if (!same_groups(X, Z)) return ICT_ERR_LAYOUT;
+    return launch_clip(X, nullptr, six, Z, (cudaStream_t)stream);
+}
+int32_t ict_relu_bwd(const ict_tensor *X, const ict_tensor *dY, int32_t six, ict_tensor *dX, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_pointwise(X)) || (st = check_pointwise(dY)) || (st = check_pointwise(dX))) return st;
+    if (six != 0 && six != 1) return ICT_ERR_INVALID_ARG;
+    if (dY->rows != X->rows || dY->cols != X->cols || dX->rows != X->rows || dX->cols != X->cols)
+        return ICT_ERR_INVALID_ARG;
+    if (!same_groups(dY, dX)) return ICT_ERR_LAYOUT;
+    return launch_clip(X, dY, six, dX, (cudaStream_t)stream);
+}
+size_t ict_sum_workspace(const ict_tensor *X, const ict_tensor *Y, const ict_tensor *Z) {
+    bool global = false;
+    if (check_sum(X, Y, Z, &global) != ICT_OK) return 0;
+    return global ? (size_t)round_up(n_grp_cols(X) * 4, 256) : 0;
+}
+int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *ws, size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    bool global = false;
+    if ((st = check_sum(X, Y, Z, &global))) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    SumArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = X->mant, a.x_exp = X->exp, a.ldx = X->ld;
+    a.y = Y->mant, a.y_exp = Y->exp, a.ldy = Y->ld;
+    a.z = Z->mant, a.z_exp = Z->exp, a.ldz = Z->ld;
+    a.rows = X->rows, a.cols = X->cols;
+    a.G = clamp_div(X->g_cols, X->cols);
+    a.ngc = n_grp_cols(X);
+    const int64_t n = a.rows * a.cols;
+    if (n == 0) return ICT_OK;
+    if (global) {
+        const size_t need = (size_t)a.ngc * 4;
+        if (!ws || ((uintptr_t)ws & 255) || ws_bytes < need) return ICT_ERR_WORKSPACE;
+        a.col_need = (int32_t *)ws;
+        if (cudaMemsetAsync(a.col_need, 0x80, need, s) != cudaSuccess) return ICT_ERR_CUDA;
+        KTimer kt(s, KC_POINTWISE, 5.0 * (double)n + 3.0 * (double)a.ngc);
+        const unsigned grid = stream_grid(a.rows * (a.cols >> 4), 2);
+        sum_global_need_kernel<<<grid, 256, (size_t)a.ngc * 4, s>>>(a);
+        sum_global_round_kernel<<<grid, 256, 0, s>>>(a);
+        counted(2);
+        return launch_status();
+    }
+    KTimer kt(s, KC_POINTWISE, 3.0 * (double)n + 3.0 * (double)(a.rows * a.ngc));
+    const int64_t nv = cdiv64(a.G, 16);  // vectors per group
+    const int64_t groups = a.rows * a.ngc;
+#define ICT_SUM_ROWS(L_, CPL_)                                                              \
+    {                                                                                       \
+        const int64_t blocks = cdiv64(groups, 8 * (32 / L_));                               \
+        sum_rows_kernel<L_, CPL_><<<(unsigned)std::min<int64_t>(blocks, 148 * 16), 256, 0, s>>>(a); \
+    }
+    if (nv <= 1) ICT_SUM_ROWS(1, 1)
+    else if (nv <= 2) ICT_SUM_ROWS(2, 1)
+    else if (nv <= 4) ICT_SUM_ROWS(4, 1)
+    else if (nv <= 8) ICT_SUM_ROWS(8, 1)
+    else if (nv <= 16) ICT_SUM_ROWS(16, 1)
+    else if (nv <= 32) ICT_SUM_ROWS(32, 1)
+    else if (nv <= 64) ICT_SUM_ROWS(32, 2)
+    else if (nv <= 128) ICT_SUM_ROWS(32, 4)
+    else ICT_SUM_ROWS(32, 0)
+#undef ICT_SUM_ROWS
     counted(1);
     return launch_status();
 }

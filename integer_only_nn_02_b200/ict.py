@@ -81,6 +81,10 @@ _SIGS = {
                                      _P(ict_sgd_params), _vp], _i32),
     "ict_gelu_fwd": ([_P(ict_tensor), _P(ict_tensor), _vp], _i32),
     "ict_gelu_bwd": ([_P(ict_tensor)] * 3 + [_vp], _i32),
+    "ict_relu_fwd": ([_P(ict_tensor), _i32, _P(ict_tensor), _vp], _i32),
+    "ict_relu_bwd": ([_P(ict_tensor), _P(ict_tensor), _i32, _P(ict_tensor), _vp], _i32),
+    "ict_sum_workspace": ([_P(ict_tensor)] * 3, _sz),
+    "ict_sum": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -179,7 +183,7 @@ def ict_launch_count() -> int:
     return int(lib.ict_launch_count())
 
 
-KERNEL_CLASSES = {"gemm": 0, "sgd": 1, "align": 2, "requant": 3, "gelu": 4, "estar": 5, "other": 6}
+KERNEL_CLASSES = {"gemm": 0, "sgd": 1, "align": 2, "requant": 3, "gelu": 4, "estar": 5, "other": 6, "pointwise": 7}
 
 
 def ict_timing_enable(on: bool) -> None:
@@ -320,6 +324,29 @@ def ict_gelu_bwd(H: DevCE, dG: DevCE, dH: DevCE, stream=None):
 
 # ----------------------------------------------------------------- conveniences
 
+def ict_relu_fwd(X: DevCE, six: bool, Z: DevCE, stream=None):
+    cx, cz = X.c(), Z.c()
+    _check(lib.ict_relu_fwd(ctypes.byref(cx), int(six), ctypes.byref(cz), _stream(stream)), "ict_relu_fwd")
+
+
+def ict_relu_bwd(X: DevCE, dY: DevCE, six: bool, dX: DevCE, stream=None):
+    cx, cy, cd = X.c(), dY.c(), dX.c()
+    _check(lib.ict_relu_bwd(ctypes.byref(cx), ctypes.byref(cy), int(six), ctypes.byref(cd), _stream(stream)),
+           "ict_relu_bwd")
+
+
+def ict_sum_workspace(X: DevCE, Y: DevCE, Z: DevCE) -> int:
+    cx, cy, cz = X.c(), Y.c(), Z.c()
+    return int(lib.ict_sum_workspace(ctypes.byref(cx), ctypes.byref(cy), ctypes.byref(cz)))
+
+
+def ict_sum(X: DevCE, Y: DevCE, Z: DevCE, ws=None, stream=None):
+    cx, cy, cz = X.c(), Y.c(), Z.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib.ict_sum(ctypes.byref(cx), ctypes.byref(cy), ctypes.byref(cz), _ptr(ws), nbytes, _stream(stream)),
+           "ict_sum")
+
+
 def linear_fwd(X: DevCE, W: DevCE, g_cols=32, stream=None) -> DevCE:
     Y = DevCE.empty(X.rows, W.rows, 1, g_cols)
     ict_linear_fwd(X, W, Y, _ws(ict_linear_workspace(OP_LINEAR_FWD, X, W, Y)), stream)
@@ -396,3 +423,22 @@ class StepGraph:
 
     def replay(self) -> None:
         self.graph.replay()
+
+
+def relu_fwd(X: DevCE, six=False, stream=None) -> DevCE:
+    Z = DevCE.empty(X.rows, X.cols, X.g_rows, X.g_cols)
+    ict_relu_fwd(X, six, Z, stream)
+    return Z
+
+
+def relu_bwd(X: DevCE, dY: DevCE, six=False, stream=None) -> DevCE:
+    dX = DevCE.empty(dY.rows, dY.cols, dY.g_rows, dY.g_cols)
+    ict_relu_bwd(X, dY, six, dX, stream)
+    return dX
+
+
+def sum_(X: DevCE, Y: DevCE, stream=None) -> DevCE:
+    """FIT(X + Y) into X's (and Y's) group partition."""
+    Z = DevCE.empty(X.rows, X.cols, X.g_rows, X.g_cols)
+    ict_sum(X, Y, Z, _ws(ict_sum_workspace(X, Y, Z)), stream)
+    return Z

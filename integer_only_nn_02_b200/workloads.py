@@ -149,6 +149,20 @@ def resnet18_conv3x3(seed=0, n=128, h=56, w=56, c=64, k=64, group=32):
     return dict(X=X, W=W, dY=dY, conv=conv, out_group=group)
 
 
+def resnet18_block_tail(seed=0, n=128, h=56, w=56, c=64, group=32):
+    """Tensors around a ResNet-18 stage-1 basic block's convolutions (NHWC, channel groups
+    spanning all pixels): the second conv's output Y (signed, before the residual add),
+    the block input X (post-ReLU), the upstream gradient dA and the conv branch's input
+    gradient dXc (signed)."""
+    rng = np.random.default_rng(seed)
+    npix = n * h * w
+    Y = with_groups(clipped_gaussian(rng, (npix, c), 32), npix, group, lambda g: exps(rng, g, -8, -6))
+    X = with_groups(relu_like(rng, (npix, c)), npix, group, lambda g: exps(rng, g, -8, -6))
+    dA = with_groups(clipped_laplace(rng, (npix, c)), npix, group, lambda g: exps(rng, g, -14, -12))
+    dXc = with_groups(clipped_laplace(rng, (npix, c)), npix, group, lambda g: exps(rng, g, -15, -12))
+    return dict(Y=Y, X=X, dA=dA, dXc=dXc, shape=dict(n=n, h=h, w=w, c=c), group=group)
+
+
 def vit_b_linear_trio(seed=0, tokens=64 * 197, d=768, hidden=3072, group=64):
     """ViT-B MLP linears 768 -> 3072 -> 768: fwd, bwd-data, bwd-weight for both."""
     rng = np.random.default_rng(seed)

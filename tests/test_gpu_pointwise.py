@@ -1,0 +1,134 @@
+"""GPU parity of the pointwise primitives against the CPU oracle, bit for bit: ReLU /
+ReLU6 forward and backward (the Clip primitive) and the Sum primitive (residual add),
+on row-local and all-row (pixel-uniform) group partitions, with exponents chosen to
+reach every ReLU6 bound case and every exponent-gap regime of the Sum (int32 fast path,
+exact int64 path, sticky path beyond a 32-bit gap)."""
+import numpy as np
+import pytest
+
+import oracle
+from integer_only_nn_02_b200.workloads import CE, E_ZERO
+from tests.test_oracle_pins import rand_ce
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ict():
+    from integer_only_nn_02_b200 import ict as _ict
+
+    return _ict
+
+
+def same(got: CE, ref: CE, what=""):
+    assert got.mant.shape == ref.mant.shape, what
+    bad = np.argwhere(got.mant != ref.mant)
+    assert bad.size == 0, f"{what}: {len(bad)} mantissas differ, first {bad[:5].tolist()}"
+    bad = np.argwhere(got.exp != ref.exp)
+    assert bad.size == 0, f"{what}: {len(bad)} exponents differ, first {bad[:5].tolist()}"
+
+
+def status_ok(ict):
+    code, raw = ict.ict_get_device_status()
+    assert code == 0, (code, raw)
+
+
+CLIP_CASES = [  # rows, cols, groups
+    (300, 192, (1, 32)),
+    (129, 768, (1, 768)),     # one group per row
+    (1000, 64, (1000, 16)),   # pixel-uniform channel groups
+    (7, 48, (7, 16)),
+    (2048, 256, (1, 64)),
+]
+
+
+@pytest.mark.parametrize("case", CLIP_CASES)
+@pytest.mark.parametrize("six", [False, True])
+def test_relu_fwd_bwd(ict, case, six):
+    rows, cols, g = case
+    rng = np.random.default_rng(rows + cols + six)
+    X = rand_ce(rng, rows, cols, *g, elo=-8, ehi=4, zero_groups=0.1)  # every ReLU6 bound case
+    dY = rand_ce(rng, rows, cols, 1, 32 if cols % 32 == 0 else 16, elo=-20, ehi=-8, zero_groups=0.05)
+    dX_ = ict.DevCE.from_host
+    got = ict.relu_fwd(dX_(X), six).to_host()
+    same(got, oracle.relu_fwd(X, six), f"fwd {case} six={six}")
+    got = ict.relu_bwd(dX_(X), dX_(dY), six).to_host()
+    same(got, oracle.relu_bwd(X, dY, six), f"bwd {case} six={six}")
+    status_ok(ict)
+
+
+SUM_CASES = [  # rows, cols, groups
+    (300, 192, (1, 32)),
+    (130, 768, (1, 64)),
+    (64, 3072, (1, 3072)),    # one group per row: 32 lanes per group
+    (5, 16, (1, 16)),
+    (60, 256, (1, 128)),      # 8 lanes per group
+    (70, 256, (1, 256)),      # 16 lanes
+    (50, 512, (1, 512)),      # 32 lanes, one vector each
+    (20, 1008, (1, 1008)),    # 32 lanes, two vectors each, the last lanes short
+    (33, 2048, (1, 2048)),    # 32 lanes, four vectors each
+    (2000, 64, (2000, 32)),   # pixel-uniform channel groups: two passes
+    (777, 256, (777, 16)),
+]
+GAPS = [((-12, -2), (-12, -2)), ((-40, -30), (-5, 5)), ((-127, -90), (10, 40))]
+
+
+@pytest.mark.parametrize("case", SUM_CASES)
+@pytest.mark.parametrize("gaps", GAPS)
+def test_sum(ict, case, gaps):
+    rows, cols, g = case
+    rng = np.random.default_rng(rows * 3 + cols + abs(gaps[0][0]))
+    X = rand_ce(rng, rows, cols, *g, *gaps[0], zero_groups=0.1)
+    Y = rand_ce(rng, rows, cols, *g, *gaps[1], zero_groups=0.1)
+    d = ict.DevCE.from_host
+    got = ict.sum_(d(X), d(Y)).to_host()
+    same(got, oracle.sum_(X, Y, *g), f"sum {case} gaps={gaps}")
+    got = ict.sum_(d(Y), d(X)).to_host()  # the Sum is symmetric
+    same(got, oracle.sum_(X, Y, *g), f"sum (swapped) {case} gaps={gaps}")
+    status_ok(ict)
+
+
+def test_sum_edge_cases(ict):
+    import torch
+
+    d = ict.DevCE.from_host
+    # both terms zero everywhere: E_ZERO groups
+    Z = CE(np.zeros((40, 64), np.int8), np.full((40, 2), E_ZERO, np.int8), 1, 32)
+    same(ict.sum_(d(Z), d(Z)).to_host(), oracle.sum_(Z, Z, 1, 32), "zeros")
+    # x + (-x) = 0
+    rng = np.random.default_rng(9)
+    X = rand_ce(rng, 40, 64, 1, 32)
+    N = CE((-X.mant.astype(np.int16)).astype(np.int8), X.exp.copy(), 1, 32)
+    got = ict.sum_(d(X), d(N)).to_host()
+    assert (got.mant == 0).all() and (got.exp == E_ZERO).all()
+    # an empty tensor is a no-op
+    E = ict.DevCE.empty(0, 64, 1, 32)
+    ict.ict_sum(E, E, ict.DevCE.empty(0, 64, 1, 32))
+    # mismatched partitions are refused
+    A = d(rand_ce(rng, 40, 64, 1, 32))
+    B = d(rand_ce(rng, 40, 64, 1, 16))
+    with pytest.raises(ict.IctError) as ei:
+        ict.ict_sum(A, B, ict.DevCE.empty(40, 64, 1, 32))
+    assert ei.value.code == 2  # ICT_ERR_LAYOUT
+    torch.cuda.synchronize()
+    status_ok(ict)
+
+
+def test_resnet_residual_and_relu_full_size(ict):
+    """The ResNet-18 stage-1 block tail at full size: residual add of two
+    128 x 56 x 56 x 64 activations (channel groups of 32 spanning all pixels), then ReLU,
+    then the backward mask."""
+    from integer_only_nn_02_b200 import workloads as wl
+
+    cfg = wl.resnet18_conv3x3(seed=4)
+    X, dY = cfg["X"], cfg["dY"]
+    rng = np.random.default_rng(12)
+    R = rand_ce(rng, X.rows, X.cols, X.rows, 32, elo=-9, ehi=-6)
+    d = ict.DevCE.from_host
+    S = ict.sum_(d(X), d(R))
+    same(S.to_host(), oracle.sum_(X, R, X.rows, 32), "residual add")
+    Sh = S.to_host()
+    A = ict.relu_fwd(S)
+    same(A.to_host(), oracle.relu_fwd(Sh), "relu")
+    same(ict.relu_bwd(S, d(dY)).to_host(), oracle.relu_bwd(Sh, dY), "relu bwd")
+    status_ok(ict)
