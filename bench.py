@@ -20,10 +20,11 @@ configurations, each a step of its own with its own unit:
 Usage:  python bench.py [--config C] [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 run under torchrun, one rank per GPU, each with its own batch of the
 configuration's size (weak scaling); the reported time is the max over ranks.  The linear
-configurations train data-parallel: every backward-weight Product exchanges its alignment
-targets (MAX) and exact integer sums (SUM) over NCCL, so all ranks apply the same update,
-the one a single GPU computes on the whole batch.  resnet18_conv3x3 and resnet50_sgd run
-as independent replicas.
+configurations and the convolution train data-parallel: every backward-weight Product
+exchanges exact integer sums (SUM, with the linear layers' alignment targets by MAX) and
+the convolution's all-pixel output groups exchange their needs (MAX) over NCCL, so all
+ranks compute what a single GPU computes on the whole batch.  resnet50_sgd and
+resnet18_block_tail run as independent replicas.
 """
 from __future__ import annotations
 
@@ -301,6 +302,7 @@ class LinearStep(Step):
 
 
 class ConvStep(Step):
+    data_parallel = True
     sample_arg = 32
     workload = {"workload": "resnet18_conv3x3_fwd_bwd", "n": 128, "h": 56, "w": 56, "c": 64, "k": 64,
                 "group": 32, "gop_per_step": 88.785}
@@ -314,13 +316,32 @@ class ConvStep(Step):
         npix = self.X.rows
         self.Y, self.dX = E.empty(npix, 64, npix, G), E.empty(npix, 64, npix, G)
         self.dW = E.empty(64, 576, 1, 576)
-        cw = ict.ict_conv_workspace
-        ws = self.ws(max(cw(0, d), cw(1, d), cw(2, d)))
-        self.calls = [
-            ("fwd", lambda: ict.ict_conv_implicit_gemm(0, d, self.X, self.W, self.Y, ws)),
-            ("bwd_data", lambda: ict.ict_conv_implicit_gemm(1, d, self.dY, self.W, self.dX, ws)),
-            ("bwd_weight", lambda: ict.ict_conv_implicit_gemm(2, d, self.dY, self.X, self.dW, ws)),
-        ]
+        from integer_only_nn_02_b200 import dp
+
+        if dp.world_size() > 1:
+            # data parallel: every rank holds its own 128 images; the ranks share the
+            # weights and the activations' pixel-uniform exponents (those of rank 0's draw)
+            c0 = wl.resnet18_conv3x3(seed=0)
+            for t, k in ((self.X, "X"), (self.dY, "dY")):
+                t.exp.copy_(torch.from_numpy(c0[k].exp))
+            self.W = E.from_host(c0["W"])
+            fwd = dp.ConvSplit(0, d, self.X, self.W, self.Y)
+            bwd = dp.ConvSplit(1, d, self.dY, self.W, self.dX)
+            wgt = dp.ConvWeightGrad(d)
+            self.exchanged_bytes = fwd.need.numel() * 4 + bwd.need.numel() * 4 + wgt.exchanged_bytes
+            self.calls = [
+                ("fwd", lambda: fwd(self.X, self.W, self.Y)),
+                ("bwd_data", lambda: bwd(self.dY, self.W, self.dX)),
+                ("bwd_weight", lambda: wgt(self.dY, self.X, self.dW)),
+            ]
+        else:
+            cw = ict.ict_conv_workspace
+            ws = self.ws(max(cw(0, d), cw(1, d), cw(2, d)))
+            self.calls = [
+                ("fwd", lambda: ict.ict_conv_implicit_gemm(0, d, self.X, self.W, self.Y, ws)),
+                ("bwd_data", lambda: ict.ict_conv_implicit_gemm(1, d, self.dY, self.W, self.dX, ws)),
+                ("bwd_weight", lambda: ict.ict_conv_implicit_gemm(2, d, self.dY, self.X, self.dW, ws)),
+            ]
         self.units = 3 * 2 * npix * 64 * 576
         self.gemm_bytes = 3 * (2 * npix * 64 + 64 * 576)
         self.h2d = [self.X.mant, self.X.exp, self.dY.mant, self.dY.exp]

@@ -264,6 +264,35 @@ int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_te
                                const ict_tensor *b, ict_tensor *out, void *ws,
                                size_t ws_bytes, void *stream);
 
+/* Convolution over a batch split across devices (images split between the ranks of a
+ * data-parallel run).  Every rank's activation operands must carry the exponents of the
+ * whole batch's tensor (true of outputs made by this split form); then:
+ *  - output groups local to each pixel (g_rows = 1): no exchange, each rank calls
+ *    ict_conv_implicit_gemm on its shard;
+ *  - FWD / BWD_DATA with output groups spanning all pixels: the group exponent depends
+ *    on every shard.  ict_conv_split_begin writes the shard's largest need() per output
+ *    group column into need[ceil(out_c / g_cols)] (int32; below -2^30 when the shard's
+ *    group is all zero) and keeps the int32 sums in ws; after an element-wise MAX of need
+ *    over the ranks, ict_conv_split_end writes the shard's rows of `out`.  Same
+ *    arguments and the same, untouched ws (ict_conv_workspace(dir, d) bytes, d the
+ *    shard's descriptor) in both calls;
+ *  - BWD_WEIGHT: ict_conv_bwd_weight_partial writes the shard's exact int64 sums
+ *    acc[k][(r,s,c)] (row stride ld_acc >= r*s*c) and the exponent vectors
+ *    e_k[k] (dY's channel exponents) and e_rsc[(r,s,c)] (X's, per filter tap); after an
+ *    element-wise SUM of acc over the ranks, ict_requant(acc, 64, k, r*s*c, ld_acc, 0,
+ *    e_k, e_rsc, dW) gives dW.
+ * The results equal ict_conv_implicit_gemm on the whole batch bit for bit. */
+int32_t ict_conv_split_begin(int32_t dir, const ict_conv_desc *d, const ict_tensor *a,
+                             const ict_tensor *b, ict_tensor *out, int32_t *need, void *ws,
+                             size_t ws_bytes, void *stream);
+int32_t ict_conv_split_end(int32_t dir, const ict_conv_desc *d, const ict_tensor *a,
+                           const ict_tensor *b, ict_tensor *out, const int32_t *need, void *ws,
+                           size_t ws_bytes, void *stream);
+int32_t ict_conv_bwd_weight_partial(const ict_conv_desc *d, const ict_tensor *dY,
+                                    const ict_tensor *X, int64_t *acc, int64_t ld_acc,
+                                    int8_t *e_k, int8_t *e_rsc, void *ws, size_t ws_bytes,
+                                    void *stream);
+
 /* --------------------------------------------------------------------------------- */
 /* Integer SGD with momentum and per-group velocity (Figure 1b; Abstract: "per-group   */
 /* velocity mechanism with independent exponent tracking").  Per group:                */

@@ -965,12 +965,14 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
     return ICT_OK;
 }
 
+// phase bit 1: operand preparation and the first Product pass; bit 2: the pass that
+// rounds with the groups' needs in cp.gmax (groups spanning all pixels).  3: both.
 int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvPlan &cp, int sms,
-             cudaStream_t s) {
+             cudaStream_t s, int phase = 3) {
     int st;
-    for (int i = 0; i < cp.njobs; ++i)
+    for (int i = 0; (phase & 1) && i < cp.njobs; ++i)
         if ((st = launch_align(cp.jobs[i], s))) return st;
-    if (cp.weight_prep) {
+    if ((phase & 1) && cp.weight_prep) {
         const int64_t n = (int64_t)d->c * d->r * d->s * d->k;
         {
             KTimer kt(s, KC_ESTAR, (double)n);
@@ -1026,17 +1028,20 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         p.epi = EPI_FIT_ROW;
         return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
     }
-    {
-        KTimer kt(s, KC_OTHER, 4.0 * (double)cp.n_gcols);
-        fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
+    if (phase & 1) {
+        {
+            KTimer kt(s, KC_OTHER, 4.0 * (double)cp.n_gcols);
+            fill_i32_kernel<<<(unsigned)cdiv64(cp.n_gcols, 256), 256, 0, s>>>(cp.gmax, cp.n_gcols, kNoExp);
+        }
+        counted(1);
     }
-    counted(1);
     if (cp.acc32) {
         p.epi = EPI_I32;
         p.ws32 = cp.acc32;
         p.ws_ld = cp.acc_ld;
         p.ws_split_stride = 0;
-        if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
+        if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
+        if (!(phase & 2)) return ICT_OK;
         GlobalRequantArgs r;
         r.v = cp.acc32;
         r.rows = cp.out_rows;
@@ -1059,7 +1064,8 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         return launch_status();
     }
     p.epi = EPI_NEED_GLOBAL;  // the first pass is recompute: its work is not counted again
-    if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
+    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
+    if (!(phase & 2)) return ICT_OK;
     p.epi = EPI_FIT_GLOBAL;
     return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
 }
@@ -1071,7 +1077,8 @@ struct WgradPlan {
     int hrows, hblk, kpix, atoms, mtiles, ntiles, splits, kblk_per_split, n_kblk, units;
     int64_t M, N, ws_ld;
     int32_t *partial;
-    int64_t *sums64;  // [N][M] slice sums
+    int64_t *sums64;  // [N][sums_ld] slice sums
+    int64_t sums_ld;
     int8_t *e_rows, *e_cols;
 };
 
@@ -1112,13 +1119,15 @@ int plan_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X
     wp->ws_ld = round_up(wp->N, 32);
     wp->partial = (int32_t *)ws.take((size_t)wp->splits * wp->M * wp->ws_ld * 4);
     wp->sums64 = (int64_t *)ws.take((size_t)wp->M * wp->N * 8);
+    wp->sums_ld = wp->M;
     wp->e_rows = (int8_t *)ws.take((size_t)wp->M);
     wp->e_cols = (int8_t *)ws.take((size_t)wp->N);
     return ICT_OK;
 }
 
+// sums_only: the int64 sums (and the exponent vectors) are the result; no FIT.
 int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X, const ict_tensor *dW,
-              const WgradPlan &wp, int sms, cudaStream_t s) {
+              const WgradPlan &wp, int sms, cudaStream_t s, bool sums_only = false) {
     int st;
     const int RS = d->r * d->s;
     {
@@ -1168,17 +1177,18 @@ int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X,
     {
         KTimer kt(s, KC_REQUANT, 4.0 * (double)wp.splits * (double)wp.M * (double)wp.N + 8.0 * (double)wp.M * wp.N);
         sum_slices_t_kernel<<<dim3((unsigned)cdiv64(wp.N, 32), (unsigned)cdiv64(wp.M, 32)), 256, 0, s>>>(
-            wp.partial, wp.splits, wp.M * wp.ws_ld, wp.M, wp.N, wp.ws_ld, wp.sums64);
+            wp.partial, wp.splits, wp.M * wp.ws_ld, wp.M, wp.N, wp.ws_ld, wp.sums64, wp.sums_ld);
         counted(1);
         if ((st = launch_status())) return st;
     }
+    if (sums_only) return ICT_OK;
     RequantArgs a;
     memset(&a, 0, sizeof(a));
     a.v64 = wp.sums64;
     a.nsplit = 1;
     a.rows = wp.N;
     a.cols = wp.M;
-    a.ld = wp.M;
+    a.ld = wp.sums_ld;
     a.cs = 1;
     a.row_exp = wp.e_cols;
     a.row_div = 1;
@@ -1319,6 +1329,24 @@ int noalloc_scratch(void **out) {
 }  // namespace
 
 // ====================================================================== C ABI
+
+// Split-batch convolution, forward and backward-data with groups spanning all pixels:
+// phase 1 writes this shard's largest need per group column into `need` (the int32 sums
+// stay in ws), phase 2 rounds with the needs given (after the MAX over the shards).
+int conv_split(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b, const ict_tensor *out,
+               int32_t *need, void *ws, size_t ws_bytes, void *stream, int phase) {
+    int st, sms = 0;
+    if ((st = device_info(&sms))) return st;
+    if ((dir != ICT_CONV_FWD && dir != ICT_CONV_BWD_DATA) || !need) return ICT_ERR_INVALID_ARG;
+    if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    Ws w = make_ws(ws, ws_bytes, false);
+    ConvPlan cp;
+    if ((st = plan_conv(dir, d, a, b, out, w, &cp))) return st;
+    if (!cp.global_groups) return ICT_ERR_LAYOUT;  // pixel-local groups: no exchange, call the whole Product
+    if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
+    cp.gmax = need;
+    return run_conv(dir, d, out, cp, sms, (cudaStream_t)stream, phase);
+}
 
 // ---- pointwise primitives (ReLU / ReLU6, Sum)
 
@@ -1639,6 +1667,36 @@ int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_te
     if ((st = plan_conv(dir, d, a, b, out, w, &cp))) return st;
     if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
     return run_conv(dir, d, out, cp, sms, (cudaStream_t)stream);
+}
+
+int32_t ict_conv_split_begin(int32_t dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
+                             ict_tensor *out, int32_t *need, void *ws, size_t ws_bytes, void *stream) {
+    return conv_split(dir, d, a, b, out, need, ws, ws_bytes, stream, 1);
+}
+int32_t ict_conv_split_end(int32_t dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
+                           ict_tensor *out, const int32_t *need, void *ws, size_t ws_bytes, void *stream) {
+    return conv_split(dir, d, a, b, out, const_cast<int32_t *>(need), ws, ws_bytes, stream, 2);
+}
+int32_t ict_conv_bwd_weight_partial(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X,
+                                    int64_t *acc, int64_t ld_acc, int8_t *e_k, int8_t *e_rsc, void *ws,
+                                    size_t ws_bytes, void *stream) {
+    int st, sms = 0;
+    if ((st = device_info(&sms))) return st;
+    if (!d || !acc || !e_k || !e_rsc) return ICT_ERR_INVALID_ARG;
+    if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    const int64_t RSC = (int64_t)d->r * d->s * d->c;
+    if (ld_acc < RSC || ((uintptr_t)acc & 7)) return ICT_ERR_INVALID_ARG;
+    static int8_t shape_only[16] __attribute__((aligned(16)));  // dW's shape for the plan; never written
+    ict_tensor dW{shape_only, shape_only, d->k, RSC, RSC, 1, (int32_t)RSC};
+    Ws w = make_ws(ws, ws_bytes, false);
+    WgradPlan wp;
+    if ((st = plan_wgrad(d, dY, X, &dW, sms, w, &wp))) return st;
+    if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
+    wp.sums64 = acc;
+    wp.sums_ld = ld_acc;
+    wp.e_rows = e_rsc;
+    wp.e_cols = e_k;
+    return run_wgrad(d, dY, X, &dW, wp, sms, (cudaStream_t)stream, true);
 }
 
 int32_t ict_sgd_momentum_step(ict_tensor *W, ict_tensor *V, const ict_tensor *G,

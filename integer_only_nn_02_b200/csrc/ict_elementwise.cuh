@@ -754,10 +754,12 @@ __global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a
     *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Sum of split-K int32 slices, transposed: out[c][r] = sum_s in[s][r][c] (int64), through
-// 32 x 32 shared tiles so that both the slice reads and the output writes are coalesced.
+// Sum of split-K int32 slices, transposed: out[c][r] = sum_s in[s][r][c] (int64, row
+// stride ld_out), through 32 x 32 shared tiles so that both the slice reads and the output
+// writes are coalesced.
 __global__ void __launch_bounds__(256) sum_slices_t_kernel(const int32_t *in, int nsplit, int64_t split_stride,
-                                                           int64_t rows, int64_t cols, int64_t ld, int64_t *out) {
+                                                           int64_t rows, int64_t cols, int64_t ld, int64_t *out,
+                                                           int64_t ld_out) {
     __shared__ int64_t tile[32][33];
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 threads
     const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
@@ -782,7 +784,7 @@ __global__ void __launch_bounds__(256) sum_slices_t_kernel(const int32_t *in, in
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int64_t c = c0 + ty + 8 * k, r = r0 + tx;
-        if (c < cols && r < rows) out[c * rows + r] = tile[tx][ty + 8 * k];
+        if (c < cols && r < rows) out[c * ld_out + r] = tile[tx][ty + 8 * k];
     }
 }
 

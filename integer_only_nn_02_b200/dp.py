@@ -1,6 +1,6 @@
-"""Data-parallel training of the integer-only (C,e) linear layers: one process per GPU,
-the batch (tokens) split over the ranks of a torch.distributed process group (NCCL over
-NVLink / NVSwitch between GPUs; gloo for CPU tests of the collectives).
+"""Data-parallel training of the integer-only (C,e) layers: one process per GPU, the
+batch (tokens or images) split over the ranks of a torch.distributed process group (NCCL
+over NVLink / NVSwitch between GPUs; gloo for CPU tests of the collectives).
 
 "Memory-Efficient Integer-Only Training of Deep Neural Networks" trains ResNets and
 ViTs on ImageNet (Abstract; Table 10 batch sizes), i.e. with batches that a
@@ -17,10 +17,15 @@ backward-weight Product dW = dY^T X, which contracts over the batch:
      else int64);
   5. every rank rounds the same sums (FIT) into dW.
 
+Convolutions (ConvSplit, ConvWeightGrad): activation exponents are uniform over
+pixels, so nothing is aligned across the batch.  Outputs whose channel groups span all
+pixels take one MAX all-reduce of the groups' needs between the Product pass and the
+rounding pass; dW takes one SUM all-reduce of int64 sums.
+
 Integer addition is exact in any order, so every rank ends with the single-device
 result on the whole batch, bit for bit, and the replicated SGD step keeps the weights
-identical on all ranks.  Steps 1, 3 and 5 are kernels of libict; this module only holds
-the buffers and issues the two collectives.
+identical on all ranks.  The arithmetic is in libict's kernels; this module only holds
+the buffers and issues the collectives.
 """
 from __future__ import annotations
 
@@ -37,7 +42,8 @@ def world_size(group=None) -> int:
 
 
 def merge_targets(e: torch.Tensor, group=None) -> None:
-    """Step 2: element-wise MAX of the int8 alignment targets over the ranks, in place."""
+    """Element-wise MAX over the ranks, in place: the int8 alignment targets of a
+    backward-weight Product, or the int32 group needs of a split convolution."""
     if world_size(group) > 1:
         dist.all_reduce(e, op=dist.ReduceOp.MAX, group=group)
 
@@ -92,3 +98,46 @@ class LinearWeightGrad:
         ict.ict_linear_bwd_weight_partial(dY, X, self.e_dy, self.e_x, self.acc, self.ws)
         merge_sums(self.acc_buf, self.group)
         ict.ict_requant(self.acc, dW, 0, self.e_dy, self.e_x)
+
+
+class ConvSplit:
+    """Forward or backward-data convolution over a batch split across the ranks of
+    `group`, with output groups spanning all pixels (the channel groups of convolution
+    activations): the shard's Product writes its int32 sums and each group's largest
+    need, a MAX all-reduce of the needs gives the whole batch's group exponents, and the
+    shard's rows are rounded with them.  Every rank's operands must carry the whole
+    batch's exponents (true of the outputs of this class)."""
+
+    def __init__(self, direction: int, d: dict, a: ict.DevCE, b: ict.DevCE, out: ict.DevCE, group=None):
+        self.direction, self.d, self.group = direction, dict(d), group
+        dev = a.mant.device
+        self.need = torch.empty(-(-out.cols // min(out.g_cols, out.cols)), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(256, ict.ict_conv_workspace(direction, d)), dtype=torch.uint8, device=dev)
+
+    def __call__(self, a: ict.DevCE, b: ict.DevCE, out: ict.DevCE) -> None:
+        ict.ict_conv_split_begin(self.direction, self.d, a, b, out, self.need, self.ws)
+        merge_targets(self.need, self.group)
+        ict.ict_conv_split_end(self.direction, self.d, a, b, out, self.need, self.ws)
+
+
+class ConvWeightGrad:
+    """Convolution dW over a batch split across the ranks of `group`: exact int64 sums of
+    the shard, a SUM all-reduce, one FIT (pixel-uniform operand exponents need no
+    alignment, and they are the same on every rank)."""
+
+    def __init__(self, d: dict, group=None, device="cuda"):
+        self.d, self.group = dict(d), group
+        K, RSC = d["k"], d["r"] * d["s"] * d["c"]
+        self.acc = torch.empty((K, RSC), dtype=torch.int64, device=device)
+        self.e_k = torch.empty(K, dtype=torch.int8, device=device)
+        self.e_rsc = torch.empty(RSC, dtype=torch.int8, device=device)
+        self.ws = torch.empty(max(256, ict.ict_conv_workspace(2, d)), dtype=torch.uint8, device=device)
+
+    @property
+    def exchanged_bytes(self) -> int:
+        return self.acc.numel() * 8
+
+    def __call__(self, dY: ict.DevCE, X: ict.DevCE, dW: ict.DevCE) -> None:
+        ict.ict_conv_bwd_weight_partial(self.d, dY, X, self.acc, self.e_k, self.e_rsc, self.ws)
+        merge_sums(self.acc, self.group)
+        ict.ict_requant(self.acc, dW, 0, self.e_k, self.e_rsc)

@@ -76,6 +76,10 @@ _SIGS = {
     "ict_linear_bwd_weight_partial": ([_P(ict_tensor)] * 2 + [_vp, _vp, _vp, _i32, _i64, _vp, _sz, _vp], _i32),
     "ict_conv_workspace": ([_i32, _P(ict_conv_desc)], _sz),
     "ict_conv_implicit_gemm": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_conv_split_begin": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _vp, _sz, _vp], _i32),
+    "ict_conv_split_end": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _vp, _sz, _vp], _i32),
+    "ict_conv_bwd_weight_partial": ([_P(ict_conv_desc)] + [_P(ict_tensor)] * 2 + [_vp, _i64, _vp, _vp, _vp, _sz,
+                                                                                   _vp], _i32),
     "ict_sgd_momentum_step": ([_P(ict_tensor), _P(ict_tensor), _P(ict_tensor), _P(ict_sgd_params), _vp], _i32),
     "ict_sgd_momentum_step_multi": ([_i32, _P(_P(ict_tensor)), _P(_P(ict_tensor)), _P(_P(ict_tensor)),
                                      _P(ict_sgd_params), _vp], _i32),
@@ -285,6 +289,30 @@ def ict_conv_implicit_gemm(direction: int, d: dict, a: DevCE, b: DevCE, out: Dev
     _check(lib.ict_conv_implicit_gemm(direction, ctypes.byref(cd), ctypes.byref(ca), ctypes.byref(cb),
                                       ctypes.byref(co), _ptr(ws), nbytes, _stream(stream)),
            "ict_conv_implicit_gemm")
+
+
+def _conv_split(fn, name, direction, d, a, b, out, need, ws, stream):
+    cd, ca, cb, co = conv_desc(d), a.c(), b.c(), out.c()
+    _check(fn(direction, ctypes.byref(cd), ctypes.byref(ca), ctypes.byref(cb), ctypes.byref(co), _ptr(need), _ptr(ws),
+              ws.numel(), _stream(stream)), name)
+
+
+def ict_conv_split_begin(direction: int, d: dict, a: DevCE, b: DevCE, out: DevCE, need: torch.Tensor, ws,
+                         stream=None):
+    _conv_split(lib.ict_conv_split_begin, "ict_conv_split_begin", direction, d, a, b, out, need, ws, stream)
+
+
+def ict_conv_split_end(direction: int, d: dict, a: DevCE, b: DevCE, out: DevCE, need: torch.Tensor, ws,
+                       stream=None):
+    _conv_split(lib.ict_conv_split_end, "ict_conv_split_end", direction, d, a, b, out, need, ws, stream)
+
+
+def ict_conv_bwd_weight_partial(d: dict, dY: DevCE, X: DevCE, acc: torch.Tensor, e_k: torch.Tensor,
+                                e_rsc: torch.Tensor, ws, stream=None):
+    cd, cy, cx = conv_desc(d), dY.c(), X.c()
+    _check(lib.ict_conv_bwd_weight_partial(ctypes.byref(cd), ctypes.byref(cy), ctypes.byref(cx), _ptr(acc),
+                                           acc.stride(0), _ptr(e_k), _ptr(e_rsc), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "ict_conv_bwd_weight_partial")
 
 
 def sgd_params(mom=(230, 8), lr=(1, 4)) -> ict_sgd_params:

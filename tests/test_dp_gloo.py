@@ -80,3 +80,56 @@ def test_sum_width():
     assert dp.sum_bits(8 * 12608) == 32  # 100 864 * 127^2 < 2^31
     assert dp.sum_bits(133_145) == 64    # 133 145 * 127^2 >= 2^31
     assert dp.sum_bits(133_144) == 32
+
+
+def _conv_batch(seed=5, n=2, h=4, w=4, c=64, k=64, G=32):
+    from integer_only_nn_02_b200.workloads import clipped_laplace, relu_like
+
+    rng = np.random.default_rng(seed)
+    npix = n * h * w
+    X = with_groups(relu_like(rng, (npix, c)), npix, G, lambda g: rng.integers(-9, -5, size=g))
+    W = with_groups(rng.integers(-127, 128, size=(k, 9 * c)).astype(np.int8), 1, 9 * c,
+                    lambda g: rng.integers(-11, -6, size=g))
+    dY = with_groups(clipped_laplace(rng, (npix, k)), npix, G, lambda g: rng.integers(-14, -11, size=g))
+    return X, W, dY, dict(n=n, h=h, w=w, c=c, k=k, r=3, s=3, stride=1, pad=1), G
+
+
+def _conv_rank(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        X, W, dY, d, G = _conv_batch()
+        hw = d["h"] * d["w"]
+        rows = slice(rank * hw, (rank + 1) * hw)  # one image per rank
+        Xr = CE(X.mant[rows].copy(), X.exp.copy(), hw, G)
+        dYr = CE(dY.mant[rows].copy(), dY.exp.copy(), hw, G)
+        dr = dict(d, n=1)
+        # forward: the shard's largest need per output group column, MAX over the ranks
+        acc, r = oracle.conv_acc(oracle.CONV_FWD, dr, Xr, W)
+        need = np.full(d["k"] // G, -(2 ** 30), np.int32)
+        for i, j in zip(*np.nonzero(acc)):
+            need[j // G] = max(need[j // G], oracle.need(int(acc[i, j]), int(r[i, j])))
+        t = torch.from_numpy(need)
+        dp.merge_targets(t)
+        # backward weight: exact int64 sums of the shard, SUM over the ranks
+        accw, _ = oracle.conv_acc(oracle.CONV_BWD_WEIGHT, dr, dYr, Xr)
+        s = torch.from_numpy(accw.copy())
+        dp.merge_sums(s)
+        np.savez(os.path.join(out_dir, f"c{rank}.npz"), need=t.numpy(), accw=s.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_conv_exchanges(tmp_path):
+    """Convolution split by images: the MAX of the ranks' group needs is the whole batch's
+    group exponent, and the SUM of their int64 dW sums is the whole batch's sums."""
+    mp.spawn(_conv_rank, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True)
+    X, W, dY, d, G = _conv_batch()
+    Y = oracle.conv(oracle.CONV_FWD, d, X, W, X.rows, G)
+    accw, _ = oracle.conv_acc(oracle.CONV_BWD_WEIGHT, d, dY, X)
+    for r in range(2):
+        got = np.load(tmp_path / f"c{r}.npz")
+        # the exponent FIT picks from the largest need: raised to -127, E_ZERO for none
+        exps = [E_ZERO if n < -(2 ** 29) else max(int(n), -127) for n in got["need"]]
+        assert exps == Y.exp[0].tolist(), f"rank {r}"
+        assert np.array_equal(got["accw"], accw), f"rank {r}"

@@ -107,3 +107,91 @@ def test_linear_weight_grad_one_rank(ict):
         dW = ict.DevCE.empty(192, 768, 1, 768)
         g(dY, X, dW)
         same(dW.to_host(), ict.linear_bwd_weight(dY, X).to_host(), f"bits {g.bits}")
+
+
+# ------------------------------------------------------------------ convolution
+
+
+def _rows(t: CE, a: int, b: int) -> CE:
+    """Pixel rows [a, b) of an activation whose groups span all pixels (one exponent row)."""
+    return CE(t.mant[a:b].copy(), t.exp.copy(), max(1, b - a), t.g_cols)
+
+
+@pytest.mark.parametrize("shape,G,cuts", [
+    ((3, 8, 8, 64, 64), 32, [0, 1, 3]),
+    ((4, 7, 20, 128, 256), 32, [0, 2, 3, 4]),       # eight output group columns
+    ((5, 6, 12, 64, 128), 64, [0, 1, 2, 5]),
+])
+def test_conv_split_batch_matches_oracle(ict, shape, G, cuts):
+    """Images split between shards: forward and backward-data rounding with the MAX of the
+    shards' group needs, backward weight from the SUM of their int64 sums."""
+    import torch
+
+    from integer_only_nn_02_b200 import dp
+    from integer_only_nn_02_b200.workloads import clipped_laplace, relu_like, with_groups
+
+    n, h, w, c, k = shape
+    rng = np.random.default_rng(sum(shape) + G)
+    npix = n * h * w
+    X = with_groups(relu_like(rng, (npix, c)), npix, G, lambda g: rng.integers(-9, -5, size=g))
+    W = rand_ce(rng, k, 9 * c, 1, 64, elo=-11, ehi=-6, zero_groups=0.05)
+    dY = with_groups(clipped_laplace(rng, (npix, k)), npix, G, lambda g: rng.integers(-14, -11, size=g))
+    d_full = dict(n=n, h=h, w=w, c=c, k=k, r=3, s=3, stride=1, pad=1)
+    hw = h * w
+    shards = list(zip(cuts[:-1], cuts[1:]))
+    Wd = ict.DevCE.from_host(W)
+    for direction, act, out_c in ((ict.CONV_FWD, X, k), (ict.CONV_BWD_DATA, dY, c)):
+        parts = []
+        for i0, i1 in shards:
+            d_r = dict(d_full, n=i1 - i0)
+            a_r = ict.DevCE.from_host(_rows(act, i0 * hw, i1 * hw))
+            out_r = ict.DevCE.empty((i1 - i0) * hw, out_c, (i1 - i0) * hw, G)
+            split = dp.ConvSplit(direction, d_r, a_r, Wd, out_r)
+            parts.append((d_r, a_r, out_r, split))
+        for d_r, a_r, out_r, split in parts:  # phase 1 on every shard
+            ict.ict_conv_split_begin(direction, d_r, a_r, Wd, out_r, split.need, split.ws)
+        need = torch.stack([p[3].need for p in parts]).max(dim=0).values  # the MAX all-reduce
+        for d_r, a_r, out_r, split in parts:  # phase 2 with the whole batch's needs
+            ict.ict_conv_split_end(direction, d_r, a_r, Wd, out_r, need, split.ws)
+        hosts = [p[2].to_host() for p in parts]
+        got = CE(np.concatenate([t.mant for t in hosts]), hosts[0].exp, npix, G)
+        for t in hosts[1:]:
+            assert np.array_equal(t.exp, hosts[0].exp), "every shard rounds with the same exponents"
+        same(got, oracle.conv(direction, d_full, act, W, npix, G), f"dir={direction} {shape} cuts={cuts}")
+    # backward weight
+    RSC = 9 * c
+    acc = torch.zeros((k, RSC), dtype=torch.int64, device="cuda")
+    for i0, i1 in shards:
+        d_r = dict(d_full, n=i1 - i0)
+        g = dp.ConvWeightGrad(d_r)
+        g.acc.fill_(77)  # the call must write every sum
+        ict.ict_conv_bwd_weight_partial(d_r, ict.DevCE.from_host(_rows(dY, i0 * hw, i1 * hw)),
+                                        ict.DevCE.from_host(_rows(X, i0 * hw, i1 * hw)), g.acc, g.e_k, g.e_rsc, g.ws)
+        acc += g.acc  # the SUM all-reduce
+    dW = ict.DevCE.empty(k, RSC, 1, RSC)
+    ict.ict_requant(acc, dW, 0, g.e_k, g.e_rsc)
+    same(dW.to_host(), oracle.conv(ict.CONV_BWD_WEIGHT, d_full, dY, X, 1, RSC), f"dW {shape} cuts={cuts}")
+    torch.cuda.synchronize()
+    code, raw = ict.ict_get_device_status()
+    assert code == 0, (code, raw)
+
+
+def test_conv_split_classes_one_rank(ict):
+    """dp.ConvSplit and dp.ConvWeightGrad without a process group equal the single calls."""
+    from integer_only_nn_02_b200 import dp
+    from integer_only_nn_02_b200.workloads import clipped_laplace, relu_like, with_groups
+
+    rng = np.random.default_rng(31)
+    n, h, w, c, k, G = 2, 8, 8, 64, 64, 32
+    npix = n * h * w
+    d = dict(n=n, h=h, w=w, c=c, k=k, r=3, s=3, stride=1, pad=1)
+    X = ict.DevCE.from_host(with_groups(relu_like(rng, (npix, c)), npix, G, lambda g: rng.integers(-9, -5, size=g)))
+    W = ict.DevCE.from_host(rand_ce(rng, k, 9 * c, 1, 64, elo=-11, ehi=-6))
+    dY = ict.DevCE.from_host(with_groups(clipped_laplace(rng, (npix, k)), npix, G,
+                                         lambda g: rng.integers(-14, -11, size=g)))
+    Y = ict.DevCE.empty(npix, k, npix, G)
+    dp.ConvSplit(ict.CONV_FWD, d, X, W, Y)(X, W, Y)
+    same(Y.to_host(), ict.conv(ict.CONV_FWD, d, X, W, npix, G).to_host(), "fwd")
+    dW = ict.DevCE.empty(k, 9 * c, 1, 9 * c)
+    dp.ConvWeightGrad(d)(dY, X, dW)
+    same(dW.to_host(), ict.conv(ict.CONV_BWD_WEIGHT, d, dY, X, 1, 9 * c).to_host(), "dW")
