@@ -83,6 +83,8 @@ def lib():
             getattr(L, name).argtypes = [P(_OT), P(_OT), ctypes.c_void_p, ctypes.c_void_p]
         L.oracle_gelu_fwd.argtypes = [P(_OT), P(_OT)]
         L.oracle_sum.argtypes = [P(_OT), P(_OT), P(_OT)]
+        L.oracle_sum_scaled.argtypes = [P(_OT), ctypes.c_int32, ctypes.c_int32, P(_OT), ctypes.c_int32,
+                                        ctypes.c_int32, P(_OT)]
         L.oracle_relu_fwd.argtypes = [P(_OT), ctypes.c_int, P(_OT)]
         L.oracle_relu_bwd.argtypes = [P(_OT), P(_OT), ctypes.c_int, P(_OT)]
         L.oracle_conv.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), P(_OT)]
@@ -271,6 +273,14 @@ def sum_(X: CE, Y: CE, g_rows: int, g_cols: int) -> CE:
     """The Sum primitive: FIT(X + Y) into (g_rows, g_cols) groups."""
     out = empty_ce(X.rows, X.cols, g_rows, g_cols)
     _check(lib().oracle_sum(ctypes.byref(_ot(X)), ctypes.byref(_ot(Y)), ctypes.byref(_ot(out))), "sum")
+    return out
+
+
+def sum_scaled(X: CE, xw, Y: CE, yw, g_rows: int, g_cols: int) -> CE:
+    """FIT(xm 2^-xs X + ym 2^-ys Y) for weights xw = (xm, xs), yw = (ym, ys)."""
+    out = empty_ce(X.rows, X.cols, g_rows, g_cols)
+    _check(lib().oracle_sum_scaled(ctypes.byref(_ot(X)), int(xw[0]), int(xw[1]), ctypes.byref(_ot(Y)), int(yw[0]),
+                                   int(yw[1]), ctypes.byref(_ot(out))), "sum_scaled")
     return out
 
 

@@ -749,23 +749,34 @@ int oracle_gelu_bwd(const o_tensor *H, const o_tensor *dG, o_tensor *dH) {
  * (Eq. 6, whose text the page does not print).  Reading, the same as for the two-term
  * sums of the SGD step: every element's two terms x * 2^ex + y * 2^ey are added exactly,
  * then the result is requantised into Z's groups.  X, Y and Z share one shape; each has
- * its own group geometry. */
-int oracle_sum(const o_tensor *X, const o_tensor *Y, o_tensor *Z) {
+ * its own group geometry.
+ * The scaled form weighs each term by an integer multiply-shift, m * 2^-s (the way the
+ * SGD step applies momentum and learning rate): Z = FIT(xm 2^-xs X + ym 2^-ys Y).  With
+ * weights (1, 0) it is the plain Sum; the weight decay of SGD (Table 10: 1e-4) is the
+ * Sum G + lambda W with lambda = ym 2^-ys. */
+int oracle_sum_scaled(const o_tensor *X, int32_t xm, int32_t xs, const o_tensor *Y, int32_t ym, int32_t ys,
+                      o_tensor *Z) {
     int st;
     if ((st = check_input(X)) || (st = check_input(Y))) return st;
     if (X->rows != Y->rows || X->cols != Y->cols) return ORC_ERR_ARG;
     if ((st = check_output(Z, X->rows, X->cols))) return st;
+    if (xm < -512 || xm > 512 || ym < -512 || ym > 512 || xs < 0 || ys < 0 || xs > 64 || ys > 64)
+        return ORC_ERR_ARG;
     int64_t n = X->rows * X->cols;
     i128 *v = malloc(sizeof(i128) * (n + 1));
     int *r = malloc(sizeof(int) * (n + 1));
     for (int64_t i = 0; i < X->rows; i++)
         for (int64_t j = 0; j < X->cols; j++)
-            two_term(mant_at(X, i, j), exp_at(X, i, j), mant_at(Y, i, j), exp_at(Y, i, j),
-                     &v[i * X->cols + j], &r[i * X->cols + j]);
+            two_term((int64_t)xm * mant_at(X, i, j), exp_at(X, i, j) - xs, (int64_t)ym * mant_at(Y, i, j),
+                     exp_at(Y, i, j) - ys, &v[i * X->cols + j], &r[i * X->cols + j]);
     st = fit_matrix(v, r, Z);
     free(v);
     free(r);
     return st;
+}
+
+int oracle_sum(const o_tensor *X, const o_tensor *Y, o_tensor *Z) {
+    return oracle_sum_scaled(X, 1, 0, Y, 1, 0, Z);
 }
 
 /* ------------------------------------------------------------------------------------ */

@@ -583,3 +583,29 @@ def test_relu_bwd_matches_torch_autograd():
                 assert (got[r] == 0).all()
             else:
                 assert torch.equal(got[r], x.grad[r]), (six, e)
+
+
+@pytest.mark.parametrize("xw,yw", [((1, 0), (105, 20)), ((-3, 1), (230, 8)), ((512, 0), (-512, 30)),
+                                   ((7, 64), (1, 0))])
+def test_sum_scaled_matches_bruteforce(xw, yw):
+    """FIT(xm 2^-xs X + ym 2^-ys Y) against exact rationals: the weight-decay form
+    G + lambda W (lambda = 105 * 2^-20, about 1e-4) among others."""
+    rng = np.random.default_rng(70 + xw[0] + yw[1])
+    X = rand_ce(rng, 7, 32, 1, 16, elo=-20, ehi=-8, zero_groups=0.15)
+    Y = rand_ce(rng, 7, 32, 1, 16, elo=-12, ehi=0, zero_groups=0.15)
+    Z = oracle.sum_scaled(X, xw, Y, yw, 1, 16)
+    vx, vy = ce_values(X), ce_values(Y)
+    wx = Fraction(xw[0]) * pow2(-xw[1])
+    wy = Fraction(yw[0]) * pow2(-yw[1])
+    mant, exps = fit_matrix_brute([[wx * vx[i][j] + wy * vy[i][j] for j in range(32)] for i in range(7)], 1, 16)
+    assert Z.mant.tolist() == mant and Z.exp.tolist() == exps
+
+
+def test_sum_scaled_unit_weights_is_sum():
+    rng = np.random.default_rng(71)
+    X = rand_ce(rng, 5, 48, 1, 16, zero_groups=0.1)
+    Y = rand_ce(rng, 5, 48, 1, 16, elo=-20, ehi=-5, zero_groups=0.1)
+    a, b = oracle.sum_scaled(X, (1, 0), Y, (1, 0), 1, 16), oracle.sum_(X, Y, 1, 16)
+    assert (a.mant == b.mant).all() and (a.exp == b.exp).all()
+    with pytest.raises(oracle.OracleError):
+        oracle.sum_scaled(X, (513, 0), Y, (1, 0), 1, 16)  # weights beyond 512 are refused
