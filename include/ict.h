@@ -342,9 +342,18 @@ int32_t ict_relu_bwd(const ict_tensor *X, const ict_tensor *dY, int32_t six, ict
 /* mantissas and ld 16-byte aligned.  Groups spanning all rows need an int32 per group  */
 /* column of workspace (ict_sum_workspace; 0 for row-local groups, where ws may be     */
 /* NULL); the result is written in two streaming passes.                              */
+/* Z must not alias X or Y. */
 size_t ict_sum_workspace(const ict_tensor *X, const ict_tensor *Y, const ict_tensor *Z);
 int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *ws,
                 size_t ws_bytes, void *stream);
+/* The weighted Sum Z = FIT(x_mul 2^-x_shift X + y_mul 2^-y_shift Y), weights as integer
+ * multiply-shifts like the SGD step's (|mul| <= 512, 0 <= shift <= 64; others
+ * ICT_ERR_INVALID_ARG).  Weights (1, 0), (1, 0) are ict_sum.  SGD's weight decay
+ * (Table 10: 1e-4) is G' = FIT(G + lambda W), lambda = y_mul 2^-y_shift (105 2^-20 for
+ * 1e-4), into G's groups, before ict_sgd_momentum_step.  Same rules as ict_sum. */
+int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y,
+                       int32_t y_mul, int32_t y_shift, ict_tensor *Z, void *ws, size_t ws_bytes,
+                       void *stream);
 
 #ifdef __cplusplus
 }

@@ -1840,8 +1840,15 @@ size_t ict_sum_workspace(const ict_tensor *X, const ict_tensor *Y, const ict_ten
     return global ? (size_t)round_up(n_grp_cols(X) * 4, 256) : 0;
 }
 int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *ws, size_t ws_bytes, void *stream) {
+    return ict_sum_scaled(X, 1, 0, Y, 1, 0, Z, ws, ws_bytes, stream);
+}
+int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y, int32_t y_mul,
+                       int32_t y_shift, ict_tensor *Z, void *ws, size_t ws_bytes, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if (x_mul < -512 || x_mul > 512 || y_mul < -512 || y_mul > 512 || x_shift < 0 || y_shift < 0 ||
+        x_shift > 64 || y_shift > 64)
+        return ICT_ERR_INVALID_ARG;
     bool global = false;
     if ((st = check_sum(X, Y, Z, &global))) return st;
     cudaStream_t s = (cudaStream_t)stream;
@@ -1853,6 +1860,14 @@ int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *w
     a.rows = X->rows, a.cols = X->cols;
     a.G = clamp_div(X->g_cols, X->cols);
     a.ngc = n_grp_cols(X);
+    a.xm = x_mul, a.xs = x_shift, a.ym = y_mul, a.ys = y_shift;
+    auto cap = [](int m) {
+        const uint32_t v = 127u * (uint32_t)(m < 0 ? -m : m);
+        int bits = 0;
+        while ((v >> bits) != 0) ++bits;
+        return 29 - bits;
+    };
+    a.cap_x = cap(x_mul), a.cap_y = cap(y_mul);
     const int64_t n = a.rows * a.cols;
     if (n == 0) return ICT_OK;
     if (global) {

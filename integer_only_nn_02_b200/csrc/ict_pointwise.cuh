@@ -98,26 +98,32 @@ struct SumArgs {
     int G;        // group width in columns (a multiple of 16, or the whole row)
     int64_t ngc;  // groups per row
     int32_t *col_need;
+    // term weights m * 2^-s (|m| <= 512), and the largest shift of each weighted term at
+    // which it stays below 2^29: 29 - bitlen(127 |m|)
+    int xm, xs, ym, ys, cap_x, cap_y;
 };
 
-// The group's two terms at a common exponent r0: x << sa + y << sb.  An E_ZERO term (all
-// its mantissas zero) takes the other's exponent.  fast: both shifts <= 22, so every sum
-// lies below 2^30 and int32 arithmetic is exact.
+// The group's two weighted terms (x xm) 2^pa + (y ym) 2^pb with pa = ex - xs, pb = ey - ys,
+// at a common exponent r0: x (xm << sa) + y (ym << sb).  An E_ZERO term (all its
+// mantissas zero) takes the other's exponent.  fast: each weighted, shifted term stays
+// below 2^29, so every sum lies below 2^30 and int32 arithmetic is exact.
 struct SumShape {
-    int pa, pb, r0, sa, sb, ma, mb;  // ma = 2^sa, mb = 2^sb (fast path)
+    int pa, pb, r0, sa, sb, ma, mb, xm, ym;  // ma = xm 2^sa, mb = ym 2^sb (fast path)
     bool fast;
 };
-__device__ __forceinline__ SumShape sum_shape(int ex, int ey) {
+__device__ __forceinline__ SumShape sum_shape(int ex, int ey, const SumArgs &a) {
     SumShape s;
-    s.pa = ex == kEZero ? ey : ex;
-    s.pb = ey == kEZero ? s.pa : ey;
+    s.xm = a.xm, s.ym = a.ym;
+    const int px = ex - a.xs, py = ey - a.ys;
+    s.pa = ex == kEZero ? py : px;
+    s.pb = ey == kEZero ? s.pa : py;
     if (ex == kEZero && ey == kEZero) s.pa = s.pb = 0;
     s.r0 = min(s.pa, s.pb);
     s.sa = s.pa - s.r0;
     s.sb = s.pb - s.r0;
-    s.fast = s.sa <= 22 && s.sb <= 22;
-    s.ma = s.fast ? 1 << s.sa : 0;
-    s.mb = s.fast ? 1 << s.sb : 0;
+    s.fast = s.sa <= a.cap_x && s.sb <= a.cap_y;
+    s.ma = s.fast ? s.xm * (1 << s.sa) : 0;
+    s.mb = s.fast ? s.ym * (1 << s.sb) : 0;
     return s;
 }
 
@@ -138,7 +144,7 @@ __device__ __forceinline__ int sum_need16(uint4 vx, uint4 vy, const SumShape &s)
     int emax = kNoExp;
     for (int q = 0; q < 4; ++q)
         for (int b = 0; b < 4; ++b) {
-            const TwoTerm t = two_term(sx8(wx[q], b), s.pa, sx8(wy[q], b), s.pb);
+            const TwoTerm t = two_term((int64_t)s.xm * sx8(wx[q], b), s.pa, (int64_t)s.ym * sx8(wy[q], b), s.pb);
             if (t.x) emax = max(emax, need64(t.x, t.r));
         }
     return emax;
@@ -162,7 +168,7 @@ __device__ __forceinline__ uint4 sum_round16(uint4 vx, uint4 vy, const SumShape 
         for (int q = 0; q < 4; ++q) {
             int c[4];
             for (int b = 0; b < 4; ++b) {
-                const TwoTerm t = two_term(sx8(wx[q], b), s.pa, sx8(wy[q], b), s.pb);
+                const TwoTerm t = two_term((int64_t)s.xm * sx8(wx[q], b), s.pa, (int64_t)s.ym * sx8(wy[q], b), s.pb);
                 c[b] = requant64(t.x, t.r, E);
             }
             o[q] = pack4(c[0], c[1], c[2], c[3]);
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(256) sum_rows_kernel(const __grid_constant__ S
         if (gidx >= groups) continue;  // the L lanes of a group leave together
         const int64_t i = idiv(gidx, a.ngc), j0 = (gidx - i * a.ngc) * a.G;
         const int nv = (int)(min((int64_t)a.G, a.cols - j0) >> 4);
-        const SumShape s = sum_shape(a.x_exp[gidx], a.y_exp[gidx]);
+        const SumShape s = sum_shape(a.x_exp[gidx], a.y_exp[gidx], a);
         const int8_t *xr = a.x + i * a.ldx + j0, *yr = a.y + i * a.ldy + j0;
         int8_t *zr = a.z + i * a.ldz + j0;
         int emax = kNoExp;
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(256) sum_global_need_kernel(const __grid_const
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
         const int64_t i = idiv(v, vpr), j = (v - i * vpr) << 4, g = idiv(j, a.G);
-        const SumShape s = sum_shape(a.x_exp[g], a.y_exp[g]);
+        const SumShape s = sum_shape(a.x_exp[g], a.y_exp[g], a);
         const int e = sum_need16(*reinterpret_cast<const uint4 *>(a.x + i * a.ldx + j),
                                  *reinterpret_cast<const uint4 *>(a.y + i * a.ldy + j), s);
         if (e > kNoExp) atomicMax(&smax[g], e);
@@ -264,8 +270,8 @@ __global__ void __launch_bounds__(256) sum_global_round_kernel(const __grid_cons
         uint4 r = make_uint4(0, 0, 0, 0);
         if (E != kEZero)
             r = sum_round16(*reinterpret_cast<const uint4 *>(a.x + i * a.ldx + j),
-                            *reinterpret_cast<const uint4 *>(a.y + i * a.ldy + j), sum_shape(a.x_exp[g], a.y_exp[g]),
-                            E);
+                            *reinterpret_cast<const uint4 *>(a.y + i * a.ldy + j),
+                            sum_shape(a.x_exp[g], a.y_exp[g], a), E);
         *reinterpret_cast<uint4 *>(a.z + i * a.ldz + j) = r;
     }
 }

@@ -89,6 +89,7 @@ _SIGS = {
     "ict_relu_bwd": ([_P(ict_tensor), _P(ict_tensor), _i32, _P(ict_tensor), _vp], _i32),
     "ict_sum_workspace": ([_P(ict_tensor)] * 3, _sz),
     "ict_sum": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_sum_scaled": ([_P(ict_tensor), _i32, _i32, _P(ict_tensor), _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -373,6 +374,22 @@ def ict_sum(X: DevCE, Y: DevCE, Z: DevCE, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel()
     _check(lib.ict_sum(ctypes.byref(cx), ctypes.byref(cy), ctypes.byref(cz), _ptr(ws), nbytes, _stream(stream)),
            "ict_sum")
+
+
+def ict_sum_scaled(X: DevCE, xw, Y: DevCE, yw, Z: DevCE, ws=None, stream=None):
+    """Z = FIT(xw[0] 2^-xw[1] X + yw[0] 2^-yw[1] Y)."""
+    cx, cy, cz = X.c(), Y.c(), Z.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib.ict_sum_scaled(ctypes.byref(cx), int(xw[0]), int(xw[1]), ctypes.byref(cy), int(yw[0]), int(yw[1]),
+                              ctypes.byref(cz), _ptr(ws), nbytes, _stream(stream)), "ict_sum_scaled")
+
+
+def ict_sgd_momentum_step_wd(W: DevCE, V: DevCE, G: DevCE, Gd: DevCE, wd=(105, 20), mom=(230, 8), lr=(1, 4),
+                             stream=None):
+    """SGD with momentum and weight decay: Gd = FIT(G + wd W) (the weighted Sum, into G's
+    groups; wd = 105 2^-20 is 1e-4), then the momentum step on Gd."""
+    ict_sum_scaled(G, (1, 0), W, wd, Gd, _ws(ict_sum_workspace(G, W, Gd)), stream)
+    ict_sgd_momentum_step(W, V, Gd, mom, lr, stream)
 
 
 def linear_fwd(X: DevCE, W: DevCE, g_cols=32, stream=None) -> DevCE:

@@ -132,3 +132,39 @@ def test_resnet_residual_and_relu_full_size(ict):
     same(A.to_host(), oracle.relu_fwd(Sh), "relu")
     same(ict.relu_bwd(S, d(dY)).to_host(), oracle.relu_bwd(Sh, dY), "relu bwd")
     status_ok(ict)
+
+
+@pytest.mark.parametrize("case", [(300, 192, (1, 32)), (2000, 64, (2000, 32)), (33, 2048, (1, 2048))])
+@pytest.mark.parametrize("xw,yw", [((1, 0), (105, 20)), ((-3, 1), (230, 8)), ((512, 0), (-512, 30)),
+                                   ((0, 0), (7, 3))])
+def test_sum_scaled(ict, case, xw, yw):
+    rows, cols, g = case
+    rng = np.random.default_rng(rows + cols + xw[0] + yw[1])
+    X = rand_ce(rng, rows, cols, *g, elo=-20, ehi=-8, zero_groups=0.1)
+    Y = rand_ce(rng, rows, cols, *g, elo=-12, ehi=0, zero_groups=0.1)
+    d = ict.DevCE.from_host
+    Z = ict.DevCE.empty(rows, cols, *g)
+    ict.ict_sum_scaled(d(X), xw, d(Y), yw, Z, ict._ws(ict.ict_sum_workspace(d(X), d(Y), Z)))
+    same(Z.to_host(), oracle.sum_scaled(X, xw, Y, yw, *g), f"sum_scaled {case} {xw} {yw}")
+    status_ok(ict)
+
+
+def test_sgd_with_weight_decay(ict):
+    """SGD with momentum and weight decay 1e-4 (105 2^-20): the weighted Sum G + lambda W
+    then the momentum step, two steps, against the oracle's composition."""
+    rng = np.random.default_rng(77)
+    rows, cols, G = 96, 256, 64
+    W = rand_ce(rng, rows, cols, 1, G, elo=-9, ehi=-6)
+    V = rand_ce(rng, rows, cols, 1, G, elo=-14, ehi=-10, zero_groups=0.2)
+    Gr = rand_ce(rng, rows, cols, 1, G, elo=-16, ehi=-12, zero_groups=0.05)
+    d = ict.DevCE.from_host
+    Wd, Vd, Gd = d(W), d(V), d(Gr)
+    Gw = ict.DevCE.empty(rows, cols, 1, G)
+    w_ref, v_ref = W, V
+    for _ in range(2):
+        ict.ict_sgd_momentum_step_wd(Wd, Vd, Gd, Gw, wd=(105, 20), mom=(230, 8), lr=(1, 4))
+        g_ref = oracle.sum_scaled(Gr, (1, 0), w_ref, (105, 20), 1, G)
+        w_ref, v_ref = oracle.sgd_step(w_ref, v_ref, g_ref, (230, 8), (1, 4))
+    same(Wd.to_host(), w_ref, "W")
+    same(Vd.to_host(), v_ref, "V")
+    status_ok(ict)
