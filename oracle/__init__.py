@@ -86,6 +86,8 @@ def lib():
         L.oracle_sum_scaled.argtypes = [P(_OT), ctypes.c_int32, ctypes.c_int32, P(_OT), ctypes.c_int32,
                                         ctypes.c_int32, P(_OT)]
         L.oracle_relu_fwd.argtypes = [P(_OT), ctypes.c_int, P(_OT)]
+        L.oracle_avgpool_fwd.argtypes = [P(_OT)] + [ctypes.c_int] * 4 + [P(_OT)]
+        L.oracle_avgpool_bwd.argtypes = [P(_OT)] + [ctypes.c_int] * 4 + [P(_OT)]
         L.oracle_relu_bwd.argtypes = [P(_OT), P(_OT), ctypes.c_int, P(_OT)]
         L.oracle_conv.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), P(_OT)]
         L.oracle_conv_acc.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), ctypes.c_void_p,
@@ -296,4 +298,18 @@ def relu_bwd(X: CE, dY: CE, six: bool = False) -> CE:
     out = empty_ce(dY.rows, dY.cols, dY.g_rows, dY.g_cols)
     _check(lib().oracle_relu_bwd(ctypes.byref(_ot(X)), ctypes.byref(_ot(dY)), int(six), ctypes.byref(_ot(out))),
            "relu_bwd")
+    return out
+
+
+def avgpool_fwd(X: CE, n: int, h: int, w: int, K: int, g_rows: int, g_cols: int) -> CE:
+    """K x K average pool, stride K, of NHWC X [n*h*w][c]: FIT(window sum / K^2)."""
+    out = empty_ce(n * (h // K) * (w // K), X.cols, g_rows, g_cols)
+    _check(lib().oracle_avgpool_fwd(ctypes.byref(_ot(X)), n, h, w, K, ctypes.byref(_ot(out))), "avgpool_fwd")
+    return out
+
+
+def avgpool_bwd(dY: CE, n: int, h: int, w: int, K: int, g_rows: int, g_cols: int) -> CE:
+    """Backward of the K x K average pool: FIT(dY of the window / K^2) at every pixel."""
+    out = empty_ce(n * h * w, dY.cols, g_rows, g_cols)
+    _check(lib().oracle_avgpool_bwd(ctypes.byref(_ot(dY)), n, h, w, K, ctypes.byref(_ot(out))), "avgpool_bwd")
     return out

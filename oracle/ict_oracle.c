@@ -835,6 +835,129 @@ int oracle_relu_bwd(const o_tensor *X, const o_tensor *dY, int six, o_tensor *dX
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Public: average pool (the Divide-by-constant primitive)                               */
+/* ------------------------------------------------------------------------------------ */
+
+/* RNE(x * 2^k / D) for D >= 1, exactly: the numerator and denominator as integers, then
+ * floor division and a remainder test (ties to even). */
+static i128 rne_div(i128 x, int k, int64_t D) {
+    i128 num = x, den = D;
+    if (k >= 0) num = x * ((i128)1 << k);
+    else den = (i128)D << (-k);
+    i128 q = num / den, rem = num % den;
+    if (rem != 0 && num < 0) { q -= 1; rem += den; } /* floor division, 0 <= rem < den */
+    if (2 * rem > den || (2 * rem == den && (q & 1))) q += 1;
+    return q;
+}
+
+/* The smallest exponent at which RNE(x * 2^(r - e) / D) fits in [-127, 127] (x != 0). */
+static int need_div(i128 x, int r, int64_t D) {
+    int e = r + bitlen(x) - bitlen(D) - 8; /* |x| 2^(r-e) / D > 2^7 here: does not fit */
+    for (;;) {
+        i128 q = rne_div(x, r - e, D);
+        if (q >= -QMAX && q <= QMAX) return e;
+        e++;
+    }
+}
+
+/* FIT of values x[i] * 2^r[i] / D into the groups of `out` (the divided counterpart of
+ * fit_matrix: the group exponent is the largest need over its nonzero members, raised to
+ * -127, E_ZERO for an all-zero group; each mantissa RNE(x 2^(r - e) / D)). */
+static int fit_matrix_div(const i128 *x, const int *r, int64_t D, o_tensor *out) {
+    int64_t ngc = n_grp_cols(out);
+    int status = ORC_OK;
+    for (int64_t gi = 0; gi < n_grp_rows(out); gi++)
+        for (int64_t gj = 0; gj < ngc; gj++) {
+            int64_t i0 = gi * out->g_rows, i1 = i0 + out->g_rows, j0 = gj * out->g_cols, j1 = j0 + out->g_cols;
+            if (i1 > out->rows) i1 = out->rows;
+            if (j1 > out->cols) j1 = out->cols;
+            int have = 0, e = 0;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++) {
+                    i128 v = x[i * out->cols + j];
+                    if (v == 0) continue;
+                    int ni = need_div(v, r[i * out->cols + j], D);
+                    if (!have || ni > e) e = ni;
+                    have = 1;
+                }
+            if (!have) e = E_ZERO;
+            else if (e < -127) e = -127;
+            if (e > 127) { status = ORC_ERR_EXP_RANGE; e = 127; }
+            out->exp[gi * ngc + gj] = (int8_t)e;
+            for (int64_t i = i0; i < i1; i++)
+                for (int64_t j = j0; j < j1; j++) {
+                    i128 v = x[i * out->cols + j];
+                    i128 q = (v == 0 || e == E_ZERO) ? 0 : rne_div(v, r[i * out->cols + j] - e, D);
+                    if (q < -QMAX) q = -QMAX;
+                    if (q > QMAX) q = QMAX;
+                    out->mant[i * out->ld + j] = (int8_t)q;
+                }
+        }
+    return status;
+}
+
+/* Average pool K x K with stride K over NHWC activations X [n*h*w][c] (Table 6: "Average
+ * pool (K x K)" -> Divide-by-constant, Eqs. 7-8, whose text the page does not print).
+ * Reading: the exact integer sum S of the window's mantissas (one exponent e: activation
+ * groups are uniform over pixels) divided by the constant D = K^2, the quotient S 2^e / D
+ * rounded once by FIT into Y's groups.  h and w are multiples of K;
+ * Y is [n*(h/K)*(w/K)][c]. */
+int oracle_avgpool_fwd(const o_tensor *X, int n, int h, int w, int K, o_tensor *Y) {
+    int st;
+    if ((st = check_input(X))) return st;
+    if (n < 1 || h < 1 || w < 1 || K < 1 || h % K || w % K || X->rows != (int64_t)n * h * w) return ORC_ERR_ARG;
+    if (X->g_rows < X->rows) return ORC_ERR_LAYOUT; /* exponents uniform over pixels */
+    int64_t P = h / K, Q = w / K, C = X->cols, rows = (int64_t)n * P * Q;
+    if ((st = check_output(Y, rows, C))) return st;
+    i128 *v = malloc(sizeof(i128) * (rows * C + 1));
+    int *r = malloc(sizeof(int) * (rows * C + 1));
+    for (int64_t img = 0; img < n; img++)
+        for (int64_t p = 0; p < P; p++)
+            for (int64_t q = 0; q < Q; q++)
+                for (int64_t ch = 0; ch < C; ch++) {
+                    i128 sum = 0;
+                    for (int dy = 0; dy < K; dy++)
+                        for (int dx = 0; dx < K; dx++)
+                            sum += mant_at(X, (img * h + p * K + dy) * w + q * K + dx, ch);
+                    int64_t o = ((img * P + p) * Q + q) * C + ch;
+                    v[o] = sum;
+                    r[o] = exp_at(X, 0, ch);
+                }
+    st = fit_matrix_div(v, r, (int64_t)K * K, Y);
+    free(v);
+    free(r);
+    return st;
+}
+
+/* Backward of the K x K average pool: every input pixel of a window receives the window's
+ * upstream gradient divided by D = K^2, dX = FIT(dY 2^e / D) into dX's groups.
+ * dY [n*(h/K)*(w/K)][c] may have any group geometry; dX is [n*h*w][c]. */
+int oracle_avgpool_bwd(const o_tensor *dY, int n, int h, int w, int K, o_tensor *dX) {
+    int st;
+    if ((st = check_input(dY))) return st;
+    if (n < 1 || h < 1 || w < 1 || K < 1 || h % K || w % K) return ORC_ERR_ARG;
+    int64_t P = h / K, Q = w / K, C = dY->cols;
+    if (dY->rows != (int64_t)n * P * Q) return ORC_ERR_ARG;
+    int64_t rows = (int64_t)n * h * w;
+    if ((st = check_output(dX, rows, C))) return st;
+    i128 *v = malloc(sizeof(i128) * (rows * C + 1));
+    int *r = malloc(sizeof(int) * (rows * C + 1));
+    for (int64_t img = 0; img < n; img++)
+        for (int64_t y = 0; y < h; y++)
+            for (int64_t x = 0; x < w; x++)
+                for (int64_t ch = 0; ch < C; ch++) {
+                    int64_t o = (img * P + y / K) * Q + x / K;
+                    int64_t i = ((img * h + y) * w + x) * C + ch;
+                    v[i] = mant_at(dY, o, ch);
+                    r[i] = exp_at(dY, o, ch);
+                }
+    st = fit_matrix_div(v, r, (int64_t)K * K, dX);
+    free(v);
+    free(r);
+    return st;
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Introspection for the tests                                                           */
 /* ------------------------------------------------------------------------------------ */
 

@@ -609,3 +609,55 @@ def test_sum_scaled_unit_weights_is_sum():
     assert (a.mant == b.mant).all() and (a.exp == b.exp).all()
     with pytest.raises(oracle.OracleError):
         oracle.sum_scaled(X, (513, 0), Y, (1, 0), 1, 16)  # weights beyond 512 are refused
+
+
+# --------------------------------------------------------------------- average pool
+
+
+def _act(rng, n, h, w, c, g, elo=-9, ehi=-5):
+    """NHWC activations with channel groups of g spanning all pixels."""
+    npix = n * h * w
+    m = rng.integers(-127, 128, size=(npix, c)).astype(np.int8)
+    return with_groups(m, npix, g, lambda s: rng.integers(elo, ehi + 1, size=s))
+
+
+@pytest.mark.parametrize("n,h,w,c,K,og", [(2, 4, 6, 32, 2, (1, 16)), (1, 6, 6, 16, 3, (4, 16)), (3, 7, 7, 32, 7, (1, 32)),
+                                          (2, 5, 5, 16, 5, (2, 16)), (1, 4, 4, 16, 1, (16, 16))])
+def test_avgpool_fwd_matches_bruteforce(n, h, w, c, K, og):
+    rng = np.random.default_rng(80 + K + c)
+    X = _act(rng, n, h, w, c, 16)
+    g_rows = og[0] if og[0] != 16 else n * (h // K) * (w // K)
+    Y = oracle.avgpool_fwd(X, n, h, w, K, g_rows, og[1])
+    vx = ce_values(X)
+    P, Q = h // K, w // K
+    vals = [[sum(vx[(img * h + p * K + dy) * w + q * K + dx][ch] for dy in range(K) for dx in range(K)) / (K * K)
+             for ch in range(c)] for img in range(n) for p in range(P) for q in range(Q)]
+    mant, exps = fit_matrix_brute(vals, g_rows, og[1])
+    assert Y.mant.tolist() == mant and Y.exp.tolist() == exps
+
+
+def test_avgpool_power_of_two_window_is_a_requant():
+    """D = 4: the average is the dyadic S 2^(e-2), so the pool equals the integer FIT of
+    the window sums at exponent e - 2."""
+    rng = np.random.default_rng(85)
+    n, h, w, c = 2, 6, 4, 32
+    X = _act(rng, n, h, w, c, 32)
+    Y = oracle.avgpool_fwd(X, n, h, w, 2, 1, 16)
+    S = X.mant.astype(np.int64).reshape(n, h // 2, 2, w // 2, 2, c).sum(axis=(2, 4)).reshape(-1, c)
+    ref = oracle.requant(S, 1, 16, base_exp=-2, col_exp=np.repeat(X.exp[0], 32))
+    assert (Y.mant == ref.mant).all() and (Y.exp == ref.exp).all()
+
+
+@pytest.mark.parametrize("n,h,w,c,K,dyg,dxg", [(2, 4, 6, 32, 2, (1, 16), (48, 16)), (1, 6, 6, 16, 3, (4, 16), (1, 16)),
+                                               (3, 7, 7, 32, 7, (1, 32), (147, 32))])
+def test_avgpool_bwd_matches_bruteforce(n, h, w, c, K, dyg, dxg):
+    rng = np.random.default_rng(90 + K)
+    rows = n * (h // K) * (w // K)
+    dY = rand_ce(rng, rows, c, *dyg, elo=-16, ehi=-8, zero_groups=0.1)
+    dX = oracle.avgpool_bwd(dY, n, h, w, K, *dxg)
+    vy = ce_values(dY)
+    P, Q = h // K, w // K
+    vals = [[vy[(img * P + y // K) * Q + x // K][ch] / (K * K) for ch in range(c)]
+            for img in range(n) for y in range(h) for x in range(w)]
+    mant, exps = fit_matrix_brute(vals, *dxg)
+    assert dX.mant.tolist() == mant and dX.exp.tolist() == exps
