@@ -355,6 +355,26 @@ int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, cons
                        int32_t y_mul, int32_t y_shift, ict_tensor *Z, void *ws, size_t ws_bytes,
                        void *stream);
 
+/* --------------------------------------------------------------------------------- */
+/* Average pool K x K, stride K (Table 6: "Average pool (K x K) -> Divide-by-constant",   */
+/* Eqs. 7-8, whose text the page does not print).  Reading: every output element is an   */
+/* exact integer S at exponent e divided by the constant D = K*K, rounded once by FIT    */
+/* into the output's groups: mantissa RNE(S 2^(e - E) / D), E the smallest exponent at   */
+/* which every member of the group fits (raised to -127; ICT_E_ZERO for all zero).       */
+/*   forward   X [n*h*w][c] NHWC, exponents uniform over pixels (g_rows >= rows);        */
+/*             S = the window's mantissa sum.  Y [n*(h/K)*(w/K)][c].                     */
+/*   backward  dY [n*(h/K)*(w/K)][c], any group geometry; every pixel of a window takes  */
+/*             S = the window's dY mantissa at dY's exponent.  dX [n*h*w][c].            */
+/* h and w multiples of K, 1 <= K <= 16.  Output groups: any geometry.  Two passes (the   */
+/* groups' needs into ws, int32 per output group: ict_avgpool_workspace, dir 0 = forward, */
+/* 1 = backward, then the rounding).  No alignment requirements.                         */
+size_t ict_avgpool_workspace(int32_t dir, const ict_tensor *in, int32_t n, int32_t h, int32_t w,
+                             int32_t K, const ict_tensor *out);
+int32_t ict_avgpool_fwd(const ict_tensor *X, int32_t n, int32_t h, int32_t w, int32_t K,
+                        ict_tensor *Y, void *ws, size_t ws_bytes, void *stream);
+int32_t ict_avgpool_bwd(const ict_tensor *dY, int32_t n, int32_t h, int32_t w, int32_t K,
+                        ict_tensor *dX, void *ws, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

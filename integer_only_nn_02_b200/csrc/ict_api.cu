@@ -1413,6 +1413,42 @@ int check_sum(const ict_tensor *X, const ict_tensor *Y, const ict_tensor *Z, boo
     return ICT_OK;
 }
 
+// Average pool K x K, stride K: geometry checks and the arguments of both directions.
+int plan_pool(bool bwd, const ict_tensor *in, int n, int h, int w, int K, const ict_tensor *out, PoolArgs *a) {
+    int st;
+    if ((st = check_tensor(in)) || (st = check_tensor(out))) return st;
+    if (n < 1 || h < 1 || w < 1 || K < 1 || K > 16 || h % K || w % K) return ICT_ERR_INVALID_ARG;
+    const int64_t P = h / K, Q = w / K, big = (int64_t)n * h * w, small = (int64_t)n * P * Q;
+    if (in->rows != (bwd ? small : big) || out->rows != (bwd ? big : small) || in->cols != out->cols)
+        return ICT_ERR_INVALID_ARG;
+    if (!bwd && in->rows > 0 && in->g_rows < in->rows) return ICT_ERR_LAYOUT;  // pixel-uniform exponents
+    memset(a, 0, sizeof(*a));
+    a->in = in->mant, a->in_exp = in->exp, a->ld_in = in->ld, a->in_ngc = n_grp_cols(in);
+    a->in_g_rows = clamp_div(in->g_rows, in->rows), a->in_g_cols = clamp_div(in->g_cols, in->cols);
+    a->out = out->mant, a->out_exp = out->exp, a->ld_out = out->ld, a->out_ngc = n_grp_cols(out);
+    a->out_g_rows = clamp_div(out->g_rows, out->rows), a->out_g_cols = clamp_div(out->g_cols, out->cols);
+    a->out_rows = out->rows, a->C = out->cols;
+    a->h = h, a->w = w, a->K = K, a->P = (int)P, a->Q = (int)Q, a->D = K * K, a->bwd = bwd;
+    return ICT_OK;
+}
+int64_t pool_groups(const PoolArgs &a) { return cdiv64(a.out_rows, a.out_g_rows) * a.out_ngc; }
+
+int run_pool(PoolArgs a, void *ws, size_t ws_bytes, cudaStream_t s) {
+    const int64_t n = a.out_rows * a.C, groups = pool_groups(a);
+    if (n == 0) return ICT_OK;
+    if (!ws || ((uintptr_t)ws & 255) || ws_bytes < (size_t)groups * 4) return ICT_ERR_WORKSPACE;
+    a.need = (int32_t *)ws;
+    if (cudaMemsetAsync(a.need, 0x80, (size_t)groups * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
+    // algorithmic bytes: every input mantissa read once, every output written once
+    const double bytes = a.bwd ? (double)n + (double)n / a.D : (double)n * (a.D + 1.0);
+    KTimer kt(s, KC_POINTWISE, bytes);
+    const unsigned grid = stream_grid(n, 1);
+    pool_need_kernel<<<grid, 256, 0, s>>>(a);
+    pool_round_kernel<<<grid, 256, 0, s>>>(a);
+    counted(2);
+    return launch_status();
+}
+
 extern "C" {
 
 const char *ict_status_string(int32_t status) {
@@ -1902,6 +1938,29 @@ int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, cons
 #undef ICT_SUM_ROWS
     counted(1);
     return launch_status();
+}
+
+size_t ict_avgpool_workspace(int32_t dir, const ict_tensor *in, int32_t n, int32_t h, int32_t w, int32_t K,
+                             const ict_tensor *out) {
+    PoolArgs a;
+    if (plan_pool(dir == 1, in, n, h, w, K, out, &a) != ICT_OK) return 0;
+    return (size_t)round_up(std::max<int64_t>(pool_groups(a) * 4, 1), 256);
+}
+int32_t ict_avgpool_fwd(const ict_tensor *X, int32_t n, int32_t h, int32_t w, int32_t K, ict_tensor *Y, void *ws,
+                        size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    PoolArgs a;
+    if ((st = plan_pool(false, X, n, h, w, K, Y, &a))) return st;
+    return run_pool(a, ws, ws_bytes, (cudaStream_t)stream);
+}
+int32_t ict_avgpool_bwd(const ict_tensor *dY, int32_t n, int32_t h, int32_t w, int32_t K, ict_tensor *dX, void *ws,
+                        size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    PoolArgs a;
+    if ((st = plan_pool(true, dY, n, h, w, K, dX, &a))) return st;
+    return run_pool(a, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -276,4 +276,102 @@ __global__ void __launch_bounds__(256) sum_global_round_kernel(const __grid_cons
     }
 }
 
+// ------------------------------------------------------------------ Divide-by-constant (average pool)
+
+// K x K average pool with stride K over NHWC activations (Table 6: "Average pool" ->
+// Divide-by-constant): every output element is an exact integer S at exponent r divided
+// by D = K^2 (forward: S the window's mantissa sum at the pixel-uniform exponent;
+// backward: S the window's upstream gradient mantissa), rounded once by FIT into the
+// output's groups.  Two passes: the largest need of every output group (int32 per
+// group, pre-set to 0x80808080), then the rounding.  One thread per output element.
+struct PoolArgs {
+    const int8_t *in, *in_exp;
+    int64_t ld_in, in_ngc;
+    int in_g_rows, in_g_cols;
+    int8_t *out, *out_exp;
+    int64_t ld_out, out_ngc, out_rows, C;
+    int out_g_rows, out_g_cols;
+    int h, w, K, P, Q, D, bwd;
+    int32_t *need;
+};
+
+// RNE(x 2^-t / D), exactly, for |x| < 2^16, 1 <= D <= 256 and -17 <= t <= 40.
+__device__ __forceinline__ int64_t rne_div64(int64_t x, int t, int64_t D) {
+    if (t > 40) return 0;  // |x| 2^-t / D < 2^-24: rounds to 0
+    int64_t num = x, den = D;
+    if (t <= 0) num = x * (1ll << (-t));
+    else den = D << t;
+    int64_t q = num / den, rem = num - q * den;  // truncating division
+    if (rem < 0) q -= 1, rem += den;             // floor, 0 <= rem < den
+    if (2 * rem > den || (2 * rem == den && (q & 1))) q += 1;
+    return q;
+}
+// The smallest exponent at which RNE(x 2^(r - e) / D) fits in [-127, 127] (x != 0): from
+// an exponent where the quotient still exceeds 127, step up until it fits.
+__device__ __forceinline__ int need_div(int64_t x, int r, int D) {
+    const int bx = 64 - __clzll(x < 0 ? -x : x), bd = 32 - __clz(D);
+    for (int t = bx - bd - 8;; ++t) {
+        const int64_t q = rne_div64(x, t, D);
+        if (q >= -127 && q <= 127) return r + t;
+    }
+}
+
+__device__ __forceinline__ void pool_value(const PoolArgs &a, int64_t i, int64_t ch, int64_t &S, int &r) {
+    if (a.bwd) {  // input pixel i of image img receives its window's gradient
+        const int64_t hw = (int64_t)a.h * a.w, img = i / hw, y = (i - img * hw) / a.w, x = i - img * hw - y * a.w;
+        const int64_t o = (img * a.P + y / a.K) * a.Q + x / a.K;
+        S = a.in[o * a.ld_in + ch];
+        r = a.in_exp[(o / a.in_g_rows) * a.in_ngc + ch / a.in_g_cols];
+        return;
+    }
+    const int64_t pq = (int64_t)a.P * a.Q, img = i / pq, p = (i - img * pq) / a.Q, q = i - img * pq - p * a.Q;
+    const int8_t *src = a.in + ((img * a.h + p * a.K) * a.w + q * a.K) * a.ld_in + ch;
+    int64_t sum = 0;
+    for (int dy = 0; dy < a.K; ++dy)
+        for (int dx = 0; dx < a.K; ++dx) sum += src[((int64_t)dy * a.w + dx) * a.ld_in];
+    S = sum;
+    r = a.in_exp[ch / a.in_g_cols];  // pixel-uniform exponents: one exponent row
+}
+
+__global__ void __launch_bounds__(256) pool_need_kernel(const __grid_constant__ PoolArgs a) {
+    const int64_t n = a.out_rows * a.C, stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t0 = (int64_t)blockIdx.x * blockDim.x; t0 < n; t0 += stride) {  // whole warps iterate together
+        const int64_t t = t0 + threadIdx.x;
+        int e = kNoExp;
+        int64_t g = -1;
+        if (t < n) {
+            const int64_t i = t / a.C, ch = t - i * a.C;
+            int64_t S;
+            int r;
+            pool_value(a, i, ch, S, r);
+            if (S) e = need_div(S, r, a.D);
+            g = (i / a.out_g_rows) * a.out_ngc + ch / a.out_g_cols;
+        }
+        // lanes of one output group reduce together; one atomic per group and warp
+        const unsigned peers = __match_any_sync(0xffffffffu, (long long)g);
+        const int m = __reduce_max_sync(peers, e);
+        if (g >= 0 && m > kNoExp && (threadIdx.x & 31) == __ffs(peers) - 1) atomicMax(&a.need[g], m);
+    }
+}
+
+__global__ void __launch_bounds__(256) pool_round_kernel(const __grid_constant__ PoolArgs a) {
+    const int64_t n = a.out_rows * a.C, stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += stride) {
+        const int64_t i = t / a.C, ch = t - i * a.C;
+        const int64_t g = (i / a.out_g_rows) * a.out_ngc + ch / a.out_g_cols;
+        const int m = a.need[g];
+        const int E = finalize_exp(m <= kNoExp ? kNoExp : m);
+        if (i % a.out_g_rows == 0 && ch % a.out_g_cols == 0) a.out_exp[g] = (int8_t)E;
+        int64_t S;
+        int r;
+        pool_value(a, i, ch, S, r);
+        int c = 0;
+        if (S && E != kEZero) {
+            const int64_t q = rne_div64(S, E - r, a.D);
+            c = q > 127 ? 127 : (q < -127 ? -127 : (int)q);
+        }
+        a.out[i * a.ld_out + ch] = (int8_t)c;
+    }
+}
+
 }  // namespace ict

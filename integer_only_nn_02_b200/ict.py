@@ -89,6 +89,9 @@ _SIGS = {
     "ict_relu_bwd": ([_P(ict_tensor), _P(ict_tensor), _i32, _P(ict_tensor), _vp], _i32),
     "ict_sum_workspace": ([_P(ict_tensor)] * 3, _sz),
     "ict_sum": ([_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
+    "ict_avgpool_workspace": ([_i32, _P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor)], _sz),
+    "ict_avgpool_fwd": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
+    "ict_avgpool_bwd": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
     "ict_sum_scaled": ([_P(ict_tensor), _i32, _i32, _P(ict_tensor), _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -487,3 +490,39 @@ def sum_(X: DevCE, Y: DevCE, stream=None) -> DevCE:
     Z = DevCE.empty(X.rows, X.cols, X.g_rows, X.g_cols)
     ict_sum(X, Y, Z, _ws(ict_sum_workspace(X, Y, Z)), stream)
     return Z
+
+
+def ict_avgpool_workspace(direction: int, src: DevCE, n, h, w, K, out: DevCE) -> int:
+    ci, co = src.c(), out.c()
+    return int(lib.ict_avgpool_workspace(direction, ctypes.byref(ci), n, h, w, K, ctypes.byref(co)))
+
+
+def ict_avgpool_fwd(X: DevCE, n, h, w, K, Y: DevCE, ws, stream=None):
+    cx, cy = X.c(), Y.c()
+    _check(lib.ict_avgpool_fwd(ctypes.byref(cx), n, h, w, K, ctypes.byref(cy), _ptr(ws), 0 if ws is None else ws.numel(),
+                               _stream(stream)), "ict_avgpool_fwd")
+
+
+def ict_avgpool_bwd(dY: DevCE, n, h, w, K, dX: DevCE, ws, stream=None):
+    cy, cx = dY.c(), dX.c()
+    _check(lib.ict_avgpool_bwd(ctypes.byref(cy), n, h, w, K, ctypes.byref(cx), _ptr(ws), 0 if ws is None else ws.numel(),
+                               _stream(stream)), "ict_avgpool_bwd")
+
+
+def _avgpool(direction, src: DevCE, n, h, w, K, out: DevCE, stream):
+    ws = _ws(ict_avgpool_workspace(direction, src, n, h, w, K, out))
+    (ict_avgpool_fwd if direction == 0 else ict_avgpool_bwd)(src, n, h, w, K, out, ws, stream)
+
+
+def avgpool_fwd(X: DevCE, n, h, w, K, g_rows, g_cols, stream=None) -> DevCE:
+    """K x K average pool, stride K, of NHWC X [n*h*w][c]: FIT(window sum / K^2)."""
+    Y = DevCE.empty(n * (h // K) * (w // K), X.cols, g_rows, g_cols)
+    _avgpool(0, X, n, h, w, K, Y, stream)
+    return Y
+
+
+def avgpool_bwd(dY: DevCE, n, h, w, K, g_rows, g_cols, stream=None) -> DevCE:
+    """Backward of the K x K average pool: FIT(window gradient / K^2) at every pixel."""
+    dX = DevCE.empty(n * h * w, dY.cols, g_rows, g_cols)
+    _avgpool(1, dY, n, h, w, K, dX, stream)
+    return dX

@@ -168,3 +168,30 @@ def test_sgd_with_weight_decay(ict):
     same(Wd.to_host(), w_ref, "W")
     same(Vd.to_host(), v_ref, "V")
     status_ok(ict)
+
+
+POOL_CASES = [  # n, h, w, c, K, input groups (forward), output groups
+    (2, 4, 6, 32, 2, 16, (1, 16)),
+    (1, 6, 6, 16, 3, 16, (4, 16)),
+    (3, 7, 7, 32, 7, 32, (1, 32)),
+    (32, 7, 7, 512, 7, 32, (1, 32)),      # ResNet-18 head: global pool into the classifier's rows
+    (4, 14, 14, 64, 2, 32, ("all", 32)),  # output groups spanning all pixels
+]
+
+
+@pytest.mark.parametrize("case", POOL_CASES)
+def test_avgpool(ict, case):
+    n, h, w, c, K, gin, og = case
+    rng = np.random.default_rng(n + h + c + K)
+    npix, nout = n * h * w, n * (h // K) * (w // K)
+    X = rand_ce(rng, npix, c, npix, gin, elo=-9, ehi=-5, zero_groups=0.1)
+    g_rows = nout if og[0] == "all" else og[0]
+    d = ict.DevCE.from_host
+    got = ict.avgpool_fwd(d(X), n, h, w, K, g_rows, og[1]).to_host()
+    same(got, oracle.avgpool_fwd(X, n, h, w, K, g_rows, og[1]), f"avgpool fwd {case}")
+    # backward: dY with the output's geometry, dX with pixel-uniform or row-local groups
+    dY = rand_ce(rng, nout, c, g_rows, og[1], elo=-16, ehi=-8, zero_groups=0.1)
+    for dxg in ((npix, gin), (1, gin)):
+        got = ict.avgpool_bwd(d(dY), n, h, w, K, *dxg).to_host()
+        same(got, oracle.avgpool_bwd(dY, n, h, w, K, *dxg), f"avgpool bwd {case} {dxg}")
+    status_ok(ict)
