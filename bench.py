@@ -441,15 +441,16 @@ class SgdStep(Step):
 
 class BlockTailStep(Step):
     """The pointwise steps around a ResNet-18 stage-1 basic block's convolutions, on its
-    128 x 56 x 56 x 64 activations (channel groups of 32 spanning all pixels): residual
-    add S = FIT(conv_out + identity), A = ReLU(S); backward dS = dA * 1[S > 0] and the
-    gradient merge dX = FIT(dX_conv + dS) at the block input."""
+    128 x 56 x 56 x 64 activations (channel groups of 32 spanning all pixels): the
+    residual add and the ReLU after it in one rounding pass, A = ReLU(FIT(conv_out +
+    identity)); backward dS = dA * 1[A > 0] (the same mask as 1[S > 0]) and the gradient
+    merge dX = FIT(dX_conv + dS) at the block input."""
 
     unit = "GB/s"
     N_IMG, HW, C, GROUP = 128, 56, 64, 32
     sample_arg = 128  # images in the oracle's sample: the whole workload, about 7 s
     workload = {"workload": "resnet18_block_tail", "n": 128, "h": 56, "w": 56, "c": 64, "group": 32,
-                "ops": "sum, relu, relu_bwd, sum"}
+                "ops": "sum+relu (fused), relu_bwd, sum"}
 
     def __init__(self, ict, torch, seed):
         super().__init__(ict, torch)
@@ -458,17 +459,16 @@ class BlockTailStep(Step):
         npix = cfg["Y"].rows
         self.Y, self.X, self.dA, self.dXc = (E.from_host(cfg[k]) for k in ("Y", "X", "dA", "dXc"))
         G = self.GROUP
-        self.S, self.A = E.empty(npix, self.C, npix, G), E.empty(npix, self.C, npix, G)
+        self.A = E.empty(npix, self.C, npix, G)
         self.dS, self.dX = E.empty(npix, self.C, npix, G), E.empty(npix, self.C, npix, G)
-        ws = self.ws(ict.ict_sum_workspace(self.Y, self.X, self.S))
+        ws = self.ws(ict.ict_sum_workspace(self.Y, self.X, self.A))
         self.calls = [
-            ("residual_add", lambda: ict.ict_sum(self.Y, self.X, self.S, ws)),
-            ("relu", lambda: ict.ict_relu_fwd(self.S, False, self.A)),
-            ("relu_bwd", lambda: ict.ict_relu_bwd(self.S, self.dA, False, self.dS)),
+            ("residual_add_relu", lambda: ict.ict_sum_act(self.Y, self.X, self.A, ict.ACT_RELU, ws)),
+            ("relu_bwd", lambda: ict.ict_relu_bwd(self.A, self.dA, False, self.dS)),
             ("grad_merge", lambda: ict.ict_sum(self.dXc, self.dS, self.dX, ws)),
         ]
         n = npix * self.C
-        self.units = (3 + 2 + 3 + 3) * n  # algorithmic bytes: inputs read once, outputs written once
+        self.units = (3 + 3 + 3) * n  # algorithmic bytes: inputs read once, outputs written once
         self.h2d = [self.Y.mant, self.Y.exp, self.dA.mant, self.dA.exp]
         self.d2h = [self.dX.mant, self.dX.exp]
 
@@ -480,12 +480,12 @@ class BlockTailStep(Step):
         g = (cfg["Y"].rows, BlockTailStep.GROUP)
         t0 = time.perf_counter()
         S = oracle.sum_(cfg["Y"], cfg["X"], *g)
-        oracle.relu_fwd(S)
-        dS = oracle.relu_bwd(S, cfg["dA"])
+        A = oracle.relu_fwd(S)
+        dS = oracle.relu_bwd(A, cfg["dA"])
         oracle.sum_(cfg["dXc"], dS, *g)
         dt = time.perf_counter() - t0
         n = cfg["Y"].rows * BlockTailStep.C
-        return dt, 11 * n, f"one full block tail on {n_img} images"
+        return dt, 9 * n, f"one full block tail on {n_img} images"
 
 
 STEPS = {"vit_ti_mlp": MlpStep, "vit_b_linear_trio": TrioStep, "resnet18_conv3x3": ConvStep,

@@ -354,6 +354,18 @@ int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *w
 int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y,
                        int32_t y_mul, int32_t y_shift, ict_tensor *Z, void *ws, size_t ws_bytes,
                        void *stream);
+/* Activations fused into a rounding pass (Table 7: integer operations on C, exponents
+ * unchanged): act 0 none, 1 ReLU, 2 ReLU6 (bound from the output group's exponent).
+ * ict_sum_act: Z = act(FIT(X + Y)), the residual add and the ReLU after it in one pass;
+ *   the ReLU backward mask can be taken from Z (Z > 0 exactly where FIT(X + Y) > 0,
+ *   and Z < c where it is below the ReLU6 bound c).
+ * ict_conv_fwd_act: Y = act(conv forward), fused into the streaming rounding pass when
+ *   Y's groups span all pixels, else a clip pass over Y in place.  Same arguments and
+ *   workspace as ict_conv_implicit_gemm with ICT_CONV_FWD. */
+int32_t ict_sum_act(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, int32_t act, void *ws,
+                    size_t ws_bytes, void *stream);
+int32_t ict_conv_fwd_act(const ict_conv_desc *d, const ict_tensor *X, const ict_tensor *W,
+                         ict_tensor *Y, int32_t act, void *ws, size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------------- */
 /* Average pool K x K, stride K (Table 6: "Average pool (K x K) -> Divide-by-constant",   */

@@ -16,6 +16,8 @@
 
 using namespace ict;
 
+int launch_clip(const ict_tensor *X, const ict_tensor *dY, int six, ict_tensor *out, cudaStream_t s);
+
 namespace {
 
 // ------------------------------------------------------------------ device checks
@@ -967,8 +969,11 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
 
 // phase bit 1: operand preparation and the first Product pass; bit 2: the pass that
 // rounds with the groups' needs in cp.gmax (groups spanning all pixels).  3: both.
+
+// act (ACT_*): an activation applied to the rounded output, fused into the streaming
+// rounding pass of all-pixel groups, else a clip pass over the output in place.
 int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvPlan &cp, int sms,
-             cudaStream_t s, int phase = 3) {
+             cudaStream_t s, int phase = 3, int act = ACT_NONE) {
     int st;
     for (int i = 0; (phase & 1) && i < cp.njobs; ++i)
         if ((st = launch_align(cp.jobs[i], s))) return st;
@@ -1026,7 +1031,8 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     const double ops = 2.0 * (double)cp.out_rows * (double)cp.out_cols * (double)ktot;
     if (!cp.global_groups) {
         p.epi = EPI_FIT_ROW;
-        return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
+        if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
+        return act == ACT_NONE ? ICT_OK : launch_clip(out, nullptr, act == ACT_RELU6, const_cast<ict_tensor *>(out), s);
     }
     if (phase & 1) {
         {
@@ -1057,6 +1063,7 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         r.out = out->mant;
         r.out_ld = out->ld;
         r.out_exp = out->exp;
+        r.act = act;
         const int64_t n = cp.out_rows * (cp.out_cols / 16);
         KTimer kt(s, KC_REQUANT, 5.0 * (double)cp.out_rows * (double)cp.out_cols);
         requant_global_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(r);
@@ -1067,7 +1074,8 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
     if (!(phase & 2)) return ICT_OK;
     p.epi = EPI_FIT_GLOBAL;
-    return launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops);
+    if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
+    return act == ACT_NONE ? ICT_OK : launch_clip(out, nullptr, act == ACT_RELU6, const_cast<ict_tensor *>(out), s);
 }
 
 // ---- convolution backward-weight: dW[k][(r,s,c)] = sum over output pixels of
@@ -1449,6 +1457,9 @@ int run_pool(PoolArgs a, void *ws, size_t ws_bytes, cudaStream_t s) {
     return launch_status();
 }
 
+int sum_entry(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y, int32_t y_mul,
+              int32_t y_shift, ict_tensor *Z, int act, void *ws, size_t ws_bytes, void *stream);
+
 extern "C" {
 
 const char *ict_status_string(int32_t status) {
@@ -1705,6 +1716,18 @@ int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_te
     return run_conv(dir, d, out, cp, sms, (cudaStream_t)stream);
 }
 
+int32_t ict_conv_fwd_act(const ict_conv_desc *d, const ict_tensor *X, const ict_tensor *W, ict_tensor *Y,
+                         int32_t act, void *ws, size_t ws_bytes, void *stream) {
+    int st, sms = 0;
+    if ((st = device_info(&sms))) return st;
+    if (act < ACT_NONE || act > ACT_RELU6) return ICT_ERR_INVALID_ARG;
+    if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
+    Ws w = make_ws(ws, ws_bytes, false);
+    ConvPlan cp;
+    if ((st = plan_conv(ICT_CONV_FWD, d, X, W, Y, w, &cp))) return st;
+    if (w.used > ws_bytes || (w.used && !ws)) return ICT_ERR_WORKSPACE;
+    return run_conv(ICT_CONV_FWD, d, Y, cp, sms, (cudaStream_t)stream, 3, act);
+}
 int32_t ict_conv_split_begin(int32_t dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
                              ict_tensor *out, int32_t *need, void *ws, size_t ws_bytes, void *stream) {
     return conv_split(dir, d, a, b, out, need, ws, ws_bytes, stream, 1);
@@ -1876,10 +1899,21 @@ size_t ict_sum_workspace(const ict_tensor *X, const ict_tensor *Y, const ict_ten
     return global ? (size_t)round_up(n_grp_cols(X) * 4, 256) : 0;
 }
 int32_t ict_sum(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, void *ws, size_t ws_bytes, void *stream) {
-    return ict_sum_scaled(X, 1, 0, Y, 1, 0, Z, ws, ws_bytes, stream);
+    return sum_entry(X, 1, 0, Y, 1, 0, Z, ACT_NONE, ws, ws_bytes, stream);
+}
+int32_t ict_sum_act(const ict_tensor *X, const ict_tensor *Y, ict_tensor *Z, int32_t act, void *ws,
+                    size_t ws_bytes, void *stream) {
+    if (act < ACT_NONE || act > ACT_RELU6) return ICT_ERR_INVALID_ARG;
+    return sum_entry(X, 1, 0, Y, 1, 0, Z, act, ws, ws_bytes, stream);
 }
 int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y, int32_t y_mul,
                        int32_t y_shift, ict_tensor *Z, void *ws, size_t ws_bytes, void *stream) {
+    return sum_entry(X, x_mul, x_shift, Y, y_mul, y_shift, Z, ACT_NONE, ws, ws_bytes, stream);
+}
+}  // extern "C"
+
+int sum_entry(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y, int32_t y_mul,
+              int32_t y_shift, ict_tensor *Z, int act, void *ws, size_t ws_bytes, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
     if (x_mul < -512 || x_mul > 512 || y_mul < -512 || y_mul > 512 || x_shift < 0 || y_shift < 0 ||
@@ -1897,6 +1931,7 @@ int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, cons
     a.G = clamp_div(X->g_cols, X->cols);
     a.ngc = n_grp_cols(X);
     a.xm = x_mul, a.xs = x_shift, a.ym = y_mul, a.ys = y_shift;
+    a.act = act;
     auto cap = [](int m) {
         const uint32_t v = 127u * (uint32_t)(m < 0 ? -m : m);
         int bits = 0;
@@ -1939,6 +1974,8 @@ int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, cons
     counted(1);
     return launch_status();
 }
+
+extern "C" {
 
 size_t ict_avgpool_workspace(int32_t dir, const ict_tensor *in, int32_t n, int32_t h, int32_t w, int32_t K,
                              const ict_tensor *out) {

@@ -701,6 +701,31 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
 // epilogue), so every element is rounded independently.  16 columns per thread: four
 // 16-byte loads of int32 partial sums, one 16-byte store of mantissas.  Requires cols,
 // ld and out_ld multiples of 16.
+// ------------------------------------------------------------------ fused activations
+
+// ReLU6's clip bound in a group at exponent e, min(6 >> e, q_max) (Table 7): the integer
+// 6 shifted right by e (left for e < 0, where 6 << 5 already exceeds q_max); the right
+// shift truncates, so e = 2 gives 1 and e >= 3 gives 0.  E_ZERO groups hold zeros only.
+__device__ __forceinline__ uint32_t relu6_bound4(int e) {
+    int c;
+    if (e == kEZero || e <= -5) c = 127;
+    else if (e < 0) c = min(6 << (-e), 127);
+    else c = e >= 3 ? 0 : (6 >> e);
+    return (uint32_t)c * 0x01010101u;
+}
+
+__device__ __forceinline__ uint32_t relu_word(uint32_t w, uint32_t hi) { return __vmins4(__vmaxs4(w, 0u), hi); }
+
+// An activation fused into a rounding pass (Table 7: integer operations on C, the
+// exponent unchanged): act 0 none, 1 ReLU max(C, 0), 2 ReLU6 clip(C, 0, c) with c the
+// bound of the output group's exponent e.
+enum { ACT_NONE = 0, ACT_RELU = 1, ACT_RELU6 = 2 };
+__device__ __forceinline__ uint4 apply_act(uint4 v, int act, int e) {
+    if (act == ACT_NONE) return v;
+    const uint32_t hi = act == ACT_RELU6 ? relu6_bound4(e) : 0x7f7f7f7fu;
+    return make_uint4(relu_word(v.x, hi), relu_word(v.y, hi), relu_word(v.z, hi), relu_word(v.w, hi));
+}
+
 struct GlobalRequantArgs {
     const int32_t *v;
     int64_t rows, cols, ld;
@@ -714,6 +739,7 @@ struct GlobalRequantArgs {
     int8_t *out;
     int64_t out_ld;
     int8_t *out_exp;
+    int act;  // fused activation (ACT_*)
 };
 __global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a) {
     const int64_t cv = a.cols / 16;
@@ -751,7 +777,7 @@ __global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a
         const int4 x = *reinterpret_cast<const int4 *>(src + 4 * q);
         o[q] = pack4(rq(x.x, 4 * q), rq(x.y, 4 * q + 1), rq(x.z, 4 * q + 2), rq(x.w, 4 * q + 3));
     }
-    *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = apply_act(make_uint4(o[0], o[1], o[2], o[3]), a.act, e);
 }
 
 // Sum of split-K int32 slices, transposed: out[c][r] = sum_s in[s][r][c] (int64, row

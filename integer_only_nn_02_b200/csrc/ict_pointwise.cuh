@@ -15,17 +15,6 @@ namespace ict {
 
 // ------------------------------------------------------------------ Clip (ReLU / ReLU6)
 
-// ReLU6's clip bound in a group at exponent e, min(6 >> e, q_max) (Table 7): the integer
-// 6 shifted right by e (left for e < 0, where 6 << 5 already exceeds q_max); the right
-// shift truncates, so e = 2 gives 1 and e >= 3 gives 0.  E_ZERO groups hold zeros only.
-__device__ __forceinline__ uint32_t relu6_bound4(int e) {
-    int c;
-    if (e == kEZero || e <= -5) c = 127;
-    else if (e < 0) c = min(6 << (-e), 127);
-    else c = e >= 3 ? 0 : (6 >> e);
-    return (uint32_t)c * 0x01010101u;
-}
-
 struct ClipArgs {
     const int8_t *x, *x_exp;  // forward input C and its exponents
     int64_t ldx;
@@ -40,7 +29,6 @@ struct ClipArgs {
     int64_t n_exp;  // exponent bytes copied to out_exp (from x_exp forward, dy_exp backward)
 };
 
-__device__ __forceinline__ uint32_t relu_word(uint32_t w, uint32_t hi) { return __vmins4(__vmaxs4(w, 0u), hi); }
 __device__ __forceinline__ uint32_t relu_mask(uint32_t w, uint32_t hi) {
     return __vcmpgts4(w, 0u) & __vcmplts4(w, hi);
 }
@@ -101,6 +89,7 @@ struct SumArgs {
     // term weights m * 2^-s (|m| <= 512), and the largest shift of each weighted term at
     // which it stays below 2^29: 29 - bitlen(127 |m|)
     int xm, xs, ym, ys, cap_x, cap_y;
+    int act;  // activation fused into the rounding (ACT_*)
 };
 
 // The group's two weighted terms (x xm) 2^pa + (y ym) 2^pb with pa = ex - xs, pb = ey - ys,
@@ -217,7 +206,7 @@ __global__ void __launch_bounds__(256) sum_rows_kernel(const __grid_constant__ S
                 const int c = li + k * L;
                 if (c < nv)
                     *reinterpret_cast<uint4 *>(zr + 16 * c) =
-                        E == kEZero ? make_uint4(0, 0, 0, 0) : sum_round16(vx[k], vy[k], s, E);
+                        E == kEZero ? make_uint4(0, 0, 0, 0) : apply_act(sum_round16(vx[k], vy[k], s, E), a.act, E);
             }
         } else {
             for (int c = li; c < nv; c += L)
@@ -228,8 +217,9 @@ __global__ void __launch_bounds__(256) sum_rows_kernel(const __grid_constant__ S
             for (int c = li; c < nv; c += L) {
                 uint4 r = make_uint4(0, 0, 0, 0);
                 if (E != kEZero)
-                    r = sum_round16(*reinterpret_cast<const uint4 *>(xr + 16 * c),
-                                    *reinterpret_cast<const uint4 *>(yr + 16 * c), s, E);
+                    r = apply_act(sum_round16(*reinterpret_cast<const uint4 *>(xr + 16 * c),
+                                              *reinterpret_cast<const uint4 *>(yr + 16 * c), s, E),
+                                  a.act, E);
                 *reinterpret_cast<uint4 *>(zr + 16 * c) = r;
             }
         }
@@ -269,9 +259,10 @@ __global__ void __launch_bounds__(256) sum_global_round_kernel(const __grid_cons
         if (i == 0 && j == g * a.G) a.z_exp[g] = (int8_t)E;
         uint4 r = make_uint4(0, 0, 0, 0);
         if (E != kEZero)
-            r = sum_round16(*reinterpret_cast<const uint4 *>(a.x + i * a.ldx + j),
-                            *reinterpret_cast<const uint4 *>(a.y + i * a.ldy + j),
-                            sum_shape(a.x_exp[g], a.y_exp[g], a), E);
+            r = apply_act(sum_round16(*reinterpret_cast<const uint4 *>(a.x + i * a.ldx + j),
+                                      *reinterpret_cast<const uint4 *>(a.y + i * a.ldy + j),
+                                      sum_shape(a.x_exp[g], a.y_exp[g], a), E),
+                          a.act, E);
         *reinterpret_cast<uint4 *>(a.z + i * a.ldz + j) = r;
     }
 }

@@ -92,6 +92,8 @@ _SIGS = {
     "ict_avgpool_workspace": ([_i32, _P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor)], _sz),
     "ict_avgpool_fwd": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
     "ict_avgpool_bwd": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
+    "ict_sum_act": ([_P(ict_tensor)] * 3 + [_i32, _vp, _sz, _vp], _i32),
+    "ict_conv_fwd_act": ([_P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_i32, _vp, _sz, _vp], _i32),
     "ict_sum_scaled": ([_P(ict_tensor), _i32, _i32, _P(ict_tensor), _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -385,6 +387,23 @@ def ict_sum_scaled(X: DevCE, xw, Y: DevCE, yw, Z: DevCE, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel()
     _check(lib.ict_sum_scaled(ctypes.byref(cx), int(xw[0]), int(xw[1]), ctypes.byref(cy), int(yw[0]), int(yw[1]),
                               ctypes.byref(cz), _ptr(ws), nbytes, _stream(stream)), "ict_sum_scaled")
+
+
+ACT_NONE, ACT_RELU, ACT_RELU6 = 0, 1, 2
+
+
+def ict_sum_act(X: DevCE, Y: DevCE, Z: DevCE, act: int, ws=None, stream=None):
+    cx, cy, cz = X.c(), Y.c(), Z.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib.ict_sum_act(ctypes.byref(cx), ctypes.byref(cy), ctypes.byref(cz), int(act), _ptr(ws), nbytes,
+                           _stream(stream)), "ict_sum_act")
+
+
+def ict_conv_fwd_act(d: dict, X: DevCE, W: DevCE, Y: DevCE, act: int, ws=None, stream=None):
+    cd, cx, cw, cy = conv_desc(d), X.c(), W.c(), Y.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib.ict_conv_fwd_act(ctypes.byref(cd), ctypes.byref(cx), ctypes.byref(cw), ctypes.byref(cy), int(act),
+                                _ptr(ws), nbytes, _stream(stream)), "ict_conv_fwd_act")
 
 
 def ict_sgd_momentum_step_wd(W: DevCE, V: DevCE, G: DevCE, Gd: DevCE, wd=(105, 20), mom=(230, 8), lr=(1, 4),

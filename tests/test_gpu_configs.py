@@ -10,7 +10,7 @@ bench.py times (same shapes and group geometries, hence the same tiling plans).
   gradients on whole-group column slices of dY (column alignment per column over all
   tokens is unchanged by taking whole groups).
 * ResNet-50 SGD arena (25 557 032 parameters): the whole update.
-* ResNet-18 block tail (residual add, ReLU, ReLU backward, gradient merge on
+* ResNet-18 block tail (residual add fused with ReLU, ReLU backward, gradient merge on
   128x56x56x64): every output.
 """
 import numpy as np
@@ -161,17 +161,19 @@ def test_resnet50_sgd_full(ict):
 
 
 def test_resnet18_block_tail_full(ict):
-    """The block tail bench.py times (residual add, ReLU, ReLU backward, gradient merge on
-    128 x 56 x 56 x 64 with all-pixel channel groups of 32), every output."""
+    """The block tail bench.py times (residual add fused with ReLU, ReLU backward from the
+    fused output, gradient merge on 128 x 56 x 56 x 64 with all-pixel channel groups of
+    32), every output, against the oracle's unfused composition."""
     cfg = wl.resnet18_block_tail(seed=0)
     d = ict.DevCE.from_host
     Y, X, dA, dXc = (cfg[k] for k in ("Y", "X", "dA", "dXc"))
     g = (Y.rows, cfg["group"])
-    S = ict.sum_(d(Y), d(X))
+    A = ict.DevCE.empty(Y.rows, Y.cols, *g)
+    Yd, Xd = d(Y), d(X)
+    ict.ict_sum_act(Yd, Xd, A, ict.ACT_RELU, ict._ws(ict.ict_sum_workspace(Yd, Xd, A)))
     Sr = oracle.sum_(Y, X, *g)
-    same(S.to_host(), Sr, "residual add")
-    same(ict.relu_fwd(S).to_host(), oracle.relu_fwd(Sr), "relu")
-    dS = ict.relu_bwd(S, d(dA))
+    same(A.to_host(), oracle.relu_fwd(Sr), "residual add + relu")
+    dS = ict.relu_bwd(A, d(dA))
     dSr = oracle.relu_bwd(Sr, dA)
     same(dS.to_host(), dSr, "relu backward")
     same(ict.sum_(d(dXc), dS).to_host(), oracle.sum_(dXc, dSr, *g), "gradient merge")

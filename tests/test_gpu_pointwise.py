@@ -195,3 +195,46 @@ def test_avgpool(ict, case):
         got = ict.avgpool_bwd(d(dY), n, h, w, K, *dxg).to_host()
         same(got, oracle.avgpool_bwd(dY, n, h, w, K, *dxg), f"avgpool bwd {case} {dxg}")
     status_ok(ict)
+
+
+@pytest.mark.parametrize("case", [(300, 192, (1, 32)), (2000, 64, (2000, 32)), (33, 2048, (1, 2048))])
+@pytest.mark.parametrize("act", [1, 2])
+def test_sum_act_fused(ict, case, act):
+    """Residual add and ReLU / ReLU6 in one rounding pass; the backward mask taken from the
+    fused output equals the one taken from the Sum before the activation."""
+    rows, cols, g = case
+    rng = np.random.default_rng(rows + cols + act)
+    X = rand_ce(rng, rows, cols, *g, elo=-6, ehi=3, zero_groups=0.1)  # every ReLU6 bound case
+    Y = rand_ce(rng, rows, cols, *g, elo=-8, ehi=1, zero_groups=0.1)
+    dA = rand_ce(rng, rows, cols, 1, 16, elo=-16, ehi=-8)
+    d = ict.DevCE.from_host
+    Z = ict.DevCE.empty(rows, cols, *g)
+    ict.ict_sum_act(d(X), d(Y), Z, act, ict._ws(ict.ict_sum_workspace(d(X), d(Y), Z)))
+    S = oracle.sum_(X, Y, *g)
+    six = act == 2
+    same(Z.to_host(), oracle.relu_fwd(S, six), f"sum_act {case} act={act}")
+    same(ict.relu_bwd(Z, d(dA), six).to_host(), oracle.relu_bwd(S, dA, six), f"mask from fused output {case}")
+    status_ok(ict)
+
+
+@pytest.mark.parametrize("global_groups", [True, False])
+@pytest.mark.parametrize("act", [0, 1, 2])
+def test_conv_fwd_act_fused(ict, global_groups, act):
+    from integer_only_nn_02_b200.workloads import with_groups
+
+    rng = np.random.default_rng(40 + act + global_groups)
+    n, h, w, c, k, G = 2, 8, 8, 64, 64, 32
+    npix = n * h * w
+    X = with_groups(rng.integers(-127, 128, size=(npix, c)).astype(np.int8), npix, G,
+                    lambda s: rng.integers(-6, -2, size=s))
+    W = rand_ce(rng, k, 9 * c, 1, 9 * c, elo=-9, ehi=-6)
+    d = dict(n=n, h=h, w=w, c=c, k=k, r=3, s=3, stride=1, pad=1)
+    g_rows = npix if global_groups else 1
+    Y = ict.DevCE.empty(npix, k, g_rows, G)
+    ws = ict._ws(ict.ict_conv_workspace(0, d))
+    ict.ict_conv_fwd_act(d, ict.DevCE.from_host(X), ict.DevCE.from_host(W), Y, act, ws)
+    ref = oracle.conv(0, d, X, W, g_rows, G)
+    if act:
+        ref = oracle.relu_fwd(ref, act == 2)
+    same(Y.to_host(), ref, f"conv fwd act={act} global={global_groups}")
+    status_ok(ict)
