@@ -334,7 +334,7 @@ int launch_align_n(const AlignJob *jobs, int n, cudaStream_t s) {
     if (jobs[0].transpose)
         align_transpose_kernel<<<dim3((unsigned)cdiv64(a.cols, 128), (unsigned)cdiv64(a.rows, 128)), 256, 0, s>>>(P);
     else
-        align_rows_kernel<<<dim3((unsigned)cdiv64(a.cols, 64), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);
+        align_rows_kernel<<<dim3((unsigned)cdiv64(a.cols, 256), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);
     counted(launches + 1);
     return launch_status();
 }

@@ -250,26 +250,30 @@ __device__ __forceinline__ int align_target(const AlignArgs &a, int64_t i, int64
     return a.e_star[j];
 }
 
-// The aligned 16-byte vector at (i, j): each vector has one group exponent and one target.
-__device__ __forceinline__ uint4 align_vec(const AlignArgs &a, int64_t i, int64_t j, int es) {
-    if (i >= a.rows) return make_uint4(0, 0, 0, 0);
-    const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
-    const int eg = a.in_exp[idiv(i, a.g_rows) * a.ngc + idiv(j, a.g_cols)];
-    if (eg == kEZero) return make_uint4(0, 0, 0, 0);
-    return rne_shift16(raw, min(es - eg, 8));  // |C| <= 127: shifts of 8 or more give 0
-}
-
-// Aligned mantissas in place of layout, 64 x 64 tiles of 16-byte vectors (cols are a
-// multiple of 16; g_cols is a multiple of 16 or spans all columns).
+// Aligned mantissas in place of layout, 64 x 256 tiles: four threads per row, each with
+// four 16-byte vectors (columns j, j + 64, j + 128, j + 192; cols are a multiple of 16,
+// g_cols a multiple of 16 or spanning all columns), loaded before the row's target is
+// known.
 // With axis 1 and no precomputed e*, the four threads of a row compute the row's e*
 // themselves (a quarter of its group exponents each, then two shuffles) and the first
 // of them stores it.
 __global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
     const int64_t i = (int64_t)blockIdx.y * 64 + (threadIdx.x >> 2);
-    const int64_t j = (int64_t)blockIdx.x * 64 + (threadIdx.x & 3) * 16;
+    const int64_t j0 = (int64_t)blockIdx.x * 256 + (threadIdx.x & 3) * 16;
     if (i >= a.rows) return;  // whole 4-thread row groups leave together
-    int es;
-    if (a.axis == 1 && a.row_estar) {
+    uint4 raw[4];
+    int eg[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {  // the loads first
+        const int64_t j = j0 + 64 * v;
+        if (j < a.cols) {
+            raw[v] = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j);
+            eg[v] = a.in_exp[idiv(i, a.g_rows) * a.ngc + idiv(j, a.g_cols)];
+        }
+    }
+    int es_row = 0;
+    const bool row_e = a.axis == 1 && a.row_estar;
+    if (row_e) {
         const int8_t *e = a.in_exp + idiv(i, a.g_rows) * a.ngc;
         int m = kNoExp;
         for (int64_t g = threadIdx.x & 3; g < a.ngc; g += 4)
@@ -277,15 +281,19 @@ __global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
         const unsigned quad = 0xfu << (threadIdx.x & 28);
         m = max(m, __shfl_xor_sync(quad, m, 1));
         m = max(m, __shfl_xor_sync(quad, m, 2));
-        es = estar_of(m);
-        if (blockIdx.x == 0 && (threadIdx.x & 3) == 0) a.e_star[i] = (int8_t)es;
-    } else {
-        es = align_target(a, i, j);
+        es_row = estar_of(m);
+        if (blockIdx.x == 0 && (threadIdx.x & 3) == 0) a.e_star[i] = (int8_t)es_row;
     }
-    if (j >= a.cols) return;
-    if (a.axis == 0 && a.col_max && i == 0)
-        for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
-    *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) = align_vec(a, i, j, es);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const int64_t j = j0 + 64 * v;
+        if (j >= a.cols) continue;
+        const int es = row_e ? es_row : align_target(a, i, j);
+        if (a.axis == 0 && a.col_max && i == 0)
+            for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
+        *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) =
+            eg[v] == kEZero ? make_uint4(0, 0, 0, 0) : rne_shift16(raw[v], min(es - eg[v], 8));
+    }
 }
 
 // Aligned and transposed, 128 x 128 tiles (rows and cols are multiples of 16).  Thread
