@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
     ICT_OK = 0,
     ICT_ERR_INVALID_ARG = 1,    /* null pointer, bad size, inconsistent shapes */
-    ICT_ERR_LAYOUT = 2,         /* group geometry or shape this build does not support */
+    ICT_ERR_LAYOUT = 2,         /* group geometry or shape the library does not support */
     ICT_ERR_ALIGNMENT = 3,      /* pointer or leading dimension not 16-byte aligned */
     ICT_ERR_WORKSPACE = 4,      /* ws too small or not 256-byte aligned */
     ICT_ERR_UNSUPPORTED_ARCH = 5, /* current device is not sm_100 */
@@ -254,7 +254,7 @@ int32_t ict_linear_fwd_noalloc(const ict_tensor *X, const ict_tensor *W, ict_ten
 /*   dir BWD_WEIGHT  a = dY [n*p*q][k], b = X [n*h*w][c] -> out = dW [k][r*s*c]        */
 /* Activation exponents must be uniform over pixels (g_rows >= rows); activation       */
 /* output groups likewise (g_rows >= rows, g_cols a multiple of 16); dW groups are     */
-/* per row.  This build supports 3x3, stride 1, pad 1, c and k multiples of 64 up to   */
+/* per row.  The library supports 3x3, stride 1, pad 1, c and k multiples of 64 up to */
 /* 256, w <= 128.  ict_conv_workspace() is an upper bound for the direction; for FWD   */
 /* and BWD_DATA it includes int32 sums of the whole output (4 bytes per element), used  */
 /* when the output groups span all pixels: one Product pass writes the sums and every  */
