@@ -49,3 +49,20 @@ def test_library_shares_nothing_with_oracle():
         assert "oracle" not in text.lower() or f == "build.py" and "oracle" not in text
     oracle_src = open(os.path.join(ROOT, "oracle", "ict_oracle.c")).read()
     assert "#include \"" not in oracle_src
+
+
+def test_header_is_plain_c():
+    """The boundary is a C ABI: the header compiles as C99 and as C++ without warnings,
+    names no torch or CUDA type, and every entry point takes plain pointers and sizes."""
+    import shutil
+    import subprocess
+
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for banned in ("torch", "at::", "cudaStream_t", "std::", "Tensor"):
+        assert banned not in text, banned
+    for compiler, lang, std in (("gcc", "c", "-std=c99"), ("g++", "c++", "-std=c++11")):
+        if shutil.which(compiler) is None:
+            continue
+        r = subprocess.run([compiler, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang, std, HEADER],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
