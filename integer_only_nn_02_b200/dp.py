@@ -54,6 +54,25 @@ def merge_sums(acc: torch.Tensor, group=None) -> None:
         dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
 
 
+def scatter_row_sums(sums: torch.Tensor, shard: torch.Tensor, group=None) -> None:
+    """SUM over the ranks of `sums` ([world * c] rows), rank r keeping rows [r c, (r+1) c)
+    in `shard` ([c] rows).  With one rank the shard is the whole tensor."""
+    if world_size(group) > 1:
+        dist.reduce_scatter_tensor(shard, sums, op=dist.ReduceOp.SUM, group=group)
+    else:
+        shard.copy_(sums)
+
+
+def gather_rows(t: torch.Tensor, group=None) -> None:
+    """Every rank's block of rows of `t` ([world * c] rows, rank r owning [r c, (r+1) c))
+    copied to every rank, in place."""
+    world = world_size(group)
+    if world > 1:
+        c = t.shape[0] // world
+        r = dist.get_rank(group)
+        dist.all_gather_into_tensor(t, t[r * c:(r + 1) * c], group=group)
+
+
 def sum_bits(total_rows: int | None) -> int:
     """Width of the sums: 32 bits when every sum of the whole batch stays below 2^31
     (total_rows * 127^2 < 2^31), else 64; 64 when the batch size is not known."""
@@ -141,3 +160,76 @@ class ConvWeightGrad:
         ict.ict_conv_bwd_weight_partial(self.d, dY, X, self.acc, self.e_k, self.e_rsc, self.ws)
         merge_sums(self.acc, self.group)
         ict.ict_requant(self.acc, dW, 0, self.e_k, self.e_rsc)
+
+
+class ShardedLinearUpdate:
+    """Backward weight and SGD step of one linear layer with the optimizer state sharded
+    over the ranks (reduce-scatter form).  The weight has row-local groups, so rows are
+    independent through the FIT of dW and the SGD step:
+
+      1. targets and their MAX all-reduce, the shard's exact sums (as LinearWeightGrad);
+      2. reduce-scatter of the sums over rows: rank r receives the summed rows
+         [r c, (r + 1) c) of dW, c = ceil(M / world);
+      3. FIT of those rows into its dW rows, the SGD step on its rows of W and of the
+         velocity V (V is only held for those rows);
+      4. all-gather of the updated W rows (mantissas and exponents) into every rank's W.
+
+    Every rank ends with the W a single device computes on the whole batch, bit for bit;
+    each rank sends about half the bytes of the all-reduce form and holds 1/world of V.
+    The object owns W (rows padded to a multiple of world) and the velocity shard; use
+    `self.W` as the layer's weight.
+    """
+
+    def __init__(self, dY: ict.DevCE, X: ict.DevCE, W: ict.DevCE, V: ict.DevCE, group=None,
+                 total_rows: int | None = None, mom=(230, 8), lr=(1, 4)):
+        if W.g_rows != 1 and W.rows > 1:
+            raise ValueError("the weight's groups must be row-local")
+        self.group, self.mom, self.lr = group, mom, lr
+        self.world = world_size(group)
+        self.rank = dist.get_rank(group) if self.world > 1 else 0
+        self.grad = LinearWeightGrad(dY, X, group, total_rows)
+        M, N, G = W.rows, W.cols, W.g_cols
+        self.M, self.chunk = M, -(-M // self.world)
+        Mp = self.chunk * self.world
+        dev = W.mant.device
+        ngc = W.exp.shape[1]
+        # the weight, rows padded to Mp so that each rank's rows are one equal block
+        self.w_mant = torch.zeros((Mp, W.mant.shape[1]), dtype=torch.int8, device=dev)
+        self.w_exp = torch.full((Mp, ngc), -128, dtype=torch.int8, device=dev)
+        self.w_mant[:M].copy_(W.mant)
+        self.w_exp[:M].copy_(W.exp)
+        self.W = ict.DevCE(self.w_mant[:M], self.w_exp[:M], 1, G, cols=N)
+        r0, r1 = self.rank * self.chunk, min(M, (self.rank + 1) * self.chunk)
+        self.r0, self.r1 = r0, r1
+        self.W_shard = ict.DevCE(self.w_mant[r0:r1], self.w_exp[r0:r1], 1, G, cols=N) if r1 > r0 else None
+        self.V_shard = None
+        if r1 > r0:
+            vm = V.mant[r0:r1].clone()
+            ve = V.exp[r0:r1].clone()
+            self.V_shard = ict.DevCE(vm, ve, 1, G, cols=N)
+            self.dW_shard = ict.DevCE.empty(r1 - r0, N, 1, G)
+        acc = self.grad.acc_buf
+        self.sums = torch.zeros((Mp, acc.shape[1]), dtype=acc.dtype, device=dev)  # padded rows stay 0
+        self.sums_shard = torch.empty((self.chunk, acc.shape[1]), dtype=acc.dtype, device=dev)
+
+    @property
+    def exchanged_bytes(self) -> int:
+        """Bytes each rank contributes per call: targets, one row block of sums, W rows."""
+        g = self.grad
+        return (g.e.numel() + self.sums_shard.numel() * self.sums_shard.element_size()
+                + self.chunk * (self.w_mant.shape[1] + self.w_exp.shape[1]))
+
+    def __call__(self, dY: ict.DevCE, X: ict.DevCE) -> None:
+        g = self.grad
+        ict.ict_linear_bwd_weight_targets(dY, X, g.e_dy, g.e_x, g.ws)
+        merge_targets(g.e, self.group)
+        ict.ict_linear_bwd_weight_partial(dY, X, g.e_dy, g.e_x, self.sums[: self.M, : g.N], g.ws)
+        mine = self.sums[: self.M]
+        if self.world > 1:
+            scatter_row_sums(self.sums, self.sums_shard, self.group)
+            mine = self.sums_shard[: self.r1 - self.r0]
+        if self.r1 > self.r0:
+            ict.ict_requant(mine[:, : g.N], self.dW_shard, 0, g.e_dy[self.r0:self.r1], g.e_x)
+            ict.ict_sgd_momentum_step(self.W_shard, self.V_shard, self.dW_shard, self.mom, self.lr)
+        gather_rows(self.w_mant, self.group)
+        gather_rows(self.w_exp, self.group)

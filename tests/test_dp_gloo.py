@@ -133,3 +133,53 @@ def test_two_ranks_conv_exchanges(tmp_path):
         exps = [E_ZERO if n < -(2 ** 29) else max(int(n), -127) for n in got["need"]]
         assert exps == Y.exp[0].tolist(), f"rank {r}"
         assert np.array_equal(got["accw"], accw), f"rank {r}"
+
+
+def _sharded_rank(rank, world, port, out_dir):
+    """Reduce-scatter form on the oracle: each rank rounds and updates only its rows of
+    W and V, then the rows are gathered."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        K, M, N, G = 90, 24, 40, 40
+        dY, X = _batch(K, M, N, seed=9)
+        rng = np.random.default_rng(10)
+        W = with_groups(rng.integers(-127, 128, size=(M, N)).astype(np.int8), 1, G, lambda s: rng.integers(-9, -6, size=s))
+        V = with_groups(rng.integers(-127, 128, size=(M, N)).astype(np.int8), 1, G, lambda s: rng.integers(-14, -10, size=s))
+        a, b = [(0, 40), (40, 90)][rank]
+        sdy, sx = _shard(dY, a, b), _shard(X, a, b)
+        e = torch.from_numpy(np.concatenate([oracle.align(sdy, 0)[1], oracle.align(sx, 0)[1]]))
+        dp.merge_targets(e)
+        e_dy, e_x = e[:M].numpy(), e[M:].numpy()
+        acc = oracle.align_to(sdy, 0, e_dy).astype(np.int64).T @ oracle.align_to(sx, 0, e_x).astype(np.int64)
+        c = -(-M // world)
+        sums = torch.zeros((c * world, N), dtype=torch.int64)
+        sums[:M] = torch.from_numpy(acc)
+        shard = torch.empty((c, N), dtype=torch.int64)
+        dp.scatter_row_sums(sums, shard)
+        r0, r1 = rank * c, min(M, (rank + 1) * c)
+        dW = oracle.requant(shard[: r1 - r0].numpy(), 1, G, 0, row_exp=e_dy[r0:r1], col_exp=e_x)
+        rows = lambda t: CE(t.mant[r0:r1].copy(), t.exp[r0:r1].copy(), 1, G)
+        Wn, _ = oracle.sgd_step(rows(W), rows(V), dW)
+        wm = torch.zeros((c * world, N), dtype=torch.int8)
+        we = torch.zeros((c * world, 1), dtype=torch.int8)
+        wm[r0:r1] = torch.from_numpy(Wn.mant)
+        we[r0:r1] = torch.from_numpy(Wn.exp)
+        dp.gather_rows(wm)
+        dp.gather_rows(we)
+        np.savez(os.path.join(out_dir, f"s{rank}.npz"), mant=wm[:M].numpy(), exp=we[:M].numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_sharded_update_matches_single_device(tmp_path):
+    mp.spawn(_sharded_rank, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True)
+    K, M, N, G = 90, 24, 40, 40
+    dY, X = _batch(K, M, N, seed=9)
+    rng = np.random.default_rng(10)
+    W = with_groups(rng.integers(-127, 128, size=(M, N)).astype(np.int8), 1, G, lambda s: rng.integers(-9, -6, size=s))
+    V = with_groups(rng.integers(-127, 128, size=(M, N)).astype(np.int8), 1, G, lambda s: rng.integers(-14, -10, size=s))
+    Wn, _ = oracle.sgd_step(W, V, oracle.linear_bwd_weight(dY, X, 1, G))
+    for r in range(2):
+        got = np.load(tmp_path / f"s{r}.npz")
+        assert np.array_equal(got["mant"], Wn.mant) and np.array_equal(got["exp"], Wn.exp), f"rank {r}"

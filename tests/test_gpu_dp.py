@@ -195,3 +195,41 @@ def test_conv_split_classes_one_rank(ict):
     dW = ict.DevCE.empty(k, 9 * c, 1, 9 * c)
     dp.ConvWeightGrad(d)(dY, X, dW)
     same(dW.to_host(), ict.conv(ict.CONV_BWD_WEIGHT, d, dY, X, 1, 9 * c).to_host(), "dW")
+
+
+def test_sharded_update_one_rank_and_row_blocks(ict):
+    """dp.ShardedLinearUpdate on one rank equals ict_linear_bwd_weight + the SGD step; the
+    per-rank pieces it runs (FIT of a block of rows of the sums, SGD on a block of rows of
+    W and V) run here on two row blocks of one GPU and give the same W and V."""
+    import torch
+
+    from integer_only_nn_02_b200 import dp
+
+    rng = np.random.default_rng(21)
+    K, M, N, G = 777, 192, 768, 768
+    dYh = rand_ce(rng, K, M, 1, 32, elo=-14, ehi=-3, zero_groups=0.05)
+    Xh = rand_ce(rng, K, N, 1, 32, elo=-9, ehi=-1, zero_groups=0.05)
+    Wh = rand_ce(rng, M, N, 1, G, elo=-9, ehi=-6)
+    Vh = rand_ce(rng, M, N, 1, G, elo=-14, ehi=-10)
+    d = ict.DevCE.from_host
+    dY, X = d(dYh), d(Xh)
+    upd = dp.ShardedLinearUpdate(dY, X, d(Wh), d(Vh), total_rows=K)
+    upd(dY, X)
+    W2, V2 = oracle.sgd_step(Wh, Vh, oracle.linear_bwd_weight(dYh, Xh, 1, G))
+    same(upd.W.to_host(), W2, "W, one rank")
+    same(upd.V_shard.to_host(), V2, "V, one rank")
+    # the same rounds on two row blocks
+    g = dp.LinearWeightGrad(dY, X, total_rows=K)
+    ict.ict_linear_bwd_weight_targets(dY, X, g.e_dy, g.e_x, g.ws)
+    ict.ict_linear_bwd_weight_partial(dY, X, g.e_dy, g.e_x, g.acc, g.ws)
+    Wd, Vd = d(Wh), d(Vh)
+    for r0, r1 in ((0, 96), (96, M)):
+        rows = lambda t: ict.DevCE(t.mant[r0:r1], t.exp[r0:r1], 1, G, cols=N)
+        dWs = ict.DevCE.empty(r1 - r0, N, 1, G)
+        ict.ict_requant(g.acc[r0:r1], dWs, 0, g.e_dy[r0:r1], g.e_x)
+        ict.ict_sgd_momentum_step(rows(Wd), rows(Vd), dWs)
+    torch.cuda.synchronize()
+    same(Wd.to_host(), W2, "W, two row blocks")
+    same(Vd.to_host(), V2, "V, two row blocks")
+    code, raw = ict.ict_get_device_status()
+    assert code == 0, (code, raw)
