@@ -254,7 +254,8 @@ int32_t ict_linear_fwd_noalloc(const ict_tensor *X, const ict_tensor *W, ict_ten
 /*   dir BWD_WEIGHT  a = dY [n*p*q][k], b = X [n*h*w][c] -> out = dW [k][r*s*c]        */
 /* Activation exponents must be uniform over pixels (g_rows >= rows); activation       */
 /* output groups likewise (g_rows >= rows, g_cols a multiple of 16); dW groups are     */
-/* per row.  The library supports 3x3, stride 1, pad 1, c and k multiples of 64 up to */
+/* per row.  The library supports square odd filters with "same" padding and stride 1 */
+/* (r = s, pad = (r - 1) / 2: 1x1, 3x3, 5x5, 7x7, ...), c and k multiples of 64 up to   */
 /* 256, w <= 128.  ict_conv_workspace() is an upper bound for the direction; for FWD   */
 /* and BWD_DATA it includes int32 sums of the whole output (4 bytes per element), used  */
 /* when the output groups span all pixels: one Product pass writes the sums and every  */

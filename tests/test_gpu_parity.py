@@ -272,3 +272,27 @@ def test_bounded_wait_timeout_leaves_context_usable(ict):
     assert np.array_equal(h.mant, ref.mant) and np.array_equal(h.exp, ref.exp)
     code, raw = ict.ict_get_device_status()
     assert code == 0, (code, raw)
+
+
+@pytest.mark.parametrize("r", [1, 5, 7])
+@pytest.mark.parametrize("global_groups", [True, False])
+def test_conv_other_odd_filters(ict, r, global_groups):
+    """'Same' convolutions with other odd square filters (1x1: pad 0; 5x5: pad 2; 7x7:
+    pad 3), all three directions, through the same implicit-GEMM kernels."""
+    rng = np.random.default_rng(50 + r + global_groups)
+    n, h, w, c, k = 2, 9, 12, 64, 128
+    npix = n * h * w
+    X = with_groups(np.where(rng.random((npix, c)) < 0.5, 0, rng.integers(1, 128, size=(npix, c))).astype(np.int8),
+                    npix, 32, lambda g: rng.integers(-8, -5, size=g))
+    W = rand_ce(rng, k, r * r * c, 1, r * r * c, elo=-10, ehi=-6)
+    dY = with_groups(clipped_laplace(rng, (npix, k)), npix, 32, lambda g: rng.integers(-14, -11, size=g))
+    d = dict(n=n, h=h, w=w, c=c, k=k, r=r, s=r, stride=1, pad=(r - 1) // 2)
+    g_rows = npix if global_groups else 1
+    for direction, a, b in ((ict.CONV_FWD, X, W), (ict.CONV_BWD_DATA, dY, W)):
+        ref = oracle.conv(direction, d, a, b, g_rows, 32)
+        got = ict.conv(direction, d, ict.DevCE.from_host(a), ict.DevCE.from_host(b), g_rows, 32).to_host()
+        same(got, ref, f"conv {r}x{r} dir={direction} global={global_groups}")
+    ref = oracle.conv(ict.CONV_BWD_WEIGHT, d, dY, X, 1, r * r * c)
+    got = ict.conv(ict.CONV_BWD_WEIGHT, d, ict.DevCE.from_host(dY), ict.DevCE.from_host(X), 1, r * r * c).to_host()
+    same(got, ref, f"conv {r}x{r} bwd-weight")
+    status_ok(ict)
