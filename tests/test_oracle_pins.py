@@ -319,7 +319,8 @@ def _conv_case(rng, n=2, h=5, w=6, c=8, k=12, g=4, r=3, s=3, pad=1, stride=1):
     return X, W, dY, d, P, Q
 
 
-@pytest.mark.parametrize("geom", [dict(), dict(stride=2), dict(r=1, s=1, pad=0), dict(h=3, w=3, pad=2)])
+@pytest.mark.parametrize("geom", [dict(), dict(stride=2), dict(r=1, s=1, pad=0), dict(h=3, w=3, pad=2),
+                                  dict(h=4, w=6, r=2, s=2, pad=0, stride=2)])  # non-overlapping patches
 def test_conv_acc_matches_torch_conv(geom):
     torch = pytest.importorskip("torch")
     F = torch.nn.functional
