@@ -294,6 +294,19 @@ int32_t ict_conv_bwd_weight_partial(const ict_conv_desc *d, const ict_tensor *dY
                                     int8_t *e_k, int8_t *e_rsc, void *ws, size_t ws_bytes,
                                     void *stream);
 
+/* Patch embedding (a P x P convolution with stride P, as a ViT's first layer): the     */
+/* non-overlapping patches of NHWC X [n*h*w][c] gathered into the rows of             */
+/* out [n*(h/P)*(w/P)][P*P*c] in (dy, dx, channel) order, ALIGN_MAX-ed to one exponent */
+/* (the largest of X's channel-group exponents, which are uniform over pixels; out has */
+/* one group: g_rows >= rows, g_cols >= cols).  ict_linear_fwd(out, W [k][P*P*c]) is   */
+/* then the patch-embedding forward, equal to the convolution's (stride P, pad 0)      */
+/* result; ict_linear_bwd_weight(dY, out) its weight gradient.  h and w multiples of P,  */
+/* P*c a multiple of 16; X's groups either one per tensor (then c may be narrow, e.g.  */
+/* 3 RGB channels, with pixels packed: ld = c) or 16-aligned channel groups with c a   */
+/* multiple of 16.                                                                      */
+int32_t ict_patchify(const ict_tensor *X, int32_t n, int32_t h, int32_t w, int32_t P,
+                     ict_tensor *out, void *stream);
+
 /* --------------------------------------------------------------------------------- */
 /* Integer SGD with momentum and per-group velocity (Figure 1b; Abstract: "per-group   */
 /* velocity mechanism with independent exponent tracking").  Per group:                */

@@ -1910,6 +1910,36 @@ int32_t ict_sum_scaled(const ict_tensor *X, int32_t x_mul, int32_t x_shift, cons
                        int32_t y_shift, ict_tensor *Z, void *ws, size_t ws_bytes, void *stream) {
     return sum_entry(X, x_mul, x_shift, Y, y_mul, y_shift, Z, ACT_NONE, ws, ws_bytes, stream);
 }
+int32_t ict_patchify(const ict_tensor *X, int32_t n, int32_t h, int32_t w, int32_t P, ict_tensor *out,
+                     void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_tensor(X)) || (st = check_tensor(out))) return st;
+    if (n < 1 || h < 1 || w < 1 || P < 1 || h % P || w % P) return ICT_ERR_INVALID_ARG;
+    const int64_t c = X->cols, rows = (int64_t)n * (h / P) * (w / P), K = (int64_t)P * P * c;
+    if (X->rows != (int64_t)n * h * w || out->rows != rows || out->cols != K) return ICT_ERR_INVALID_ARG;
+    if (X->g_rows < X->rows) return ICT_ERR_LAYOUT;  // exponents uniform over pixels
+    const int g_cols = clamp_div(X->g_cols, X->cols);
+    // 16-byte vectors: each inside one channel group and one row segment
+    if ((P * c) % 16 || !(g_cols >= c || (c % 16 == 0 && g_cols % 16 == 0))) return ICT_ERR_LAYOUT;
+    if (out->g_rows < out->rows || out->g_cols < out->cols) return ICT_ERR_LAYOUT;  // one exponent
+    if (c % 16 && X->ld != c) return ICT_ERR_LAYOUT;  // narrow channels: pixels must be packed
+    if (!aligned16(X->mant) || (c % 16 == 0 && (X->ld & 15)) || !aligned16(out->mant) || (out->ld & 15))
+        return ICT_ERR_ALIGNMENT;
+    PatchArgs a;
+    memset(&a, 0, sizeof(a));
+    a.in = X->mant, a.in_exp = X->exp, a.ld_in = X->ld, a.g_cols = g_cols, a.ngc = n_grp_cols(X);
+    a.out = out->mant, a.out_exp = out->exp, a.ld_out = out->ld, a.rows = rows;
+    a.h = h, a.w = w, a.c = (int)c, a.P = P, a.Hp = h / P, a.Wp = w / P;
+    const int64_t vecs = rows * (K / 16);
+    if (vecs == 0) return ICT_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    KTimer kt(s, KC_ALIGN, 2.0 * (double)rows * (double)K);
+    patchify_kernel<<<(unsigned)cdiv64(vecs, 256), 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
 }  // extern "C"
 
 int sum_entry(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y, int32_t y_mul,

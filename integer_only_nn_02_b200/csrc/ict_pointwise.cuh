@@ -365,4 +365,41 @@ __global__ void __launch_bounds__(256) pool_round_kernel(const __grid_constant__
     }
 }
 
+// ------------------------------------------------------------------ patch embedding
+
+// Non-overlapping P x P patches of NHWC activations gathered into rows, (dy, dx, ch)
+// order, ALIGN_MAX-ed to one exponent: the largest of the activation's channel-group
+// exponents (they are uniform over pixels).  The rows are the K-major operand of the
+// patch-embedding Product (a P x P, stride P convolution), which then needs no
+// alignment.  One thread per 16-byte output vector: P * c is a multiple of 16, so a
+// vector lies inside one (dy) row segment, and it spans one channel group.
+struct PatchArgs {
+    const int8_t *in, *in_exp;
+    int64_t ld_in;
+    int g_cols;
+    int64_t ngc;
+    int8_t *out, *out_exp;
+    int64_t ld_out, rows;
+    int h, w, c, P, Hp, Wp;
+};
+__global__ void __launch_bounds__(256) patchify_kernel(const __grid_constant__ PatchArgs a) {
+    const int64_t vpr = (int64_t)a.P * a.P * a.c / 16;  // vectors per output row
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= a.rows * vpr) return;
+    const int64_t o = v / vpr, t = v - o * vpr;
+    const int64_t seg = (int64_t)a.P * a.c;  // bytes of one (dy) row segment
+    const int64_t dy = (16 * t) / seg, off = 16 * t - dy * seg;
+    const int64_t per_img = (int64_t)a.Hp * a.Wp, img = o / per_img, pq = o - img * per_img;
+    const int64_t pp = pq / a.Wp, qq = pq - pp * a.Wp;
+    const int64_t pix = (img * a.h + pp * a.P + dy) * a.w + qq * a.P + off / a.c;
+    const int ch = (int)(off % a.c);
+    const uint4 raw = *reinterpret_cast<const uint4 *>(a.in + pix * a.ld_in + ch);
+    int es = kEZero;  // the target: E_ZERO (-128) is the smallest byte
+    for (int64_t g = 0; g < a.ngc; ++g) es = max(es, (int)a.in_exp[g]);
+    const int eg = a.in_exp[ch / a.g_cols];
+    if (v == 0) a.out_exp[0] = (int8_t)es;
+    *reinterpret_cast<uint4 *>(a.out + o * a.ld_out + 16 * t) =
+        eg == kEZero ? make_uint4(0, 0, 0, 0) : rne_shift16(raw, min(es - eg, 8));
+}
+
 }  // namespace ict

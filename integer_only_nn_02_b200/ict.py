@@ -94,6 +94,7 @@ _SIGS = {
     "ict_avgpool_bwd": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
     "ict_sum_act": ([_P(ict_tensor)] * 3 + [_i32, _vp, _sz, _vp], _i32),
     "ict_conv_fwd_act": ([_P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_i32, _vp, _sz, _vp], _i32),
+    "ict_patchify": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp], _i32),
     "ict_sum_scaled": ([_P(ict_tensor), _i32, _i32, _P(ict_tensor), _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -545,3 +546,16 @@ def avgpool_bwd(dY: DevCE, n, h, w, K, g_rows, g_cols, stream=None) -> DevCE:
     dX = DevCE.empty(n * h * w, dY.cols, g_rows, g_cols)
     _avgpool(1, dY, n, h, w, K, dX, stream)
     return dX
+
+
+def ict_patchify(X: DevCE, n, h, w, P, out: DevCE, stream=None):
+    cx, co = X.c(), out.c()
+    _check(lib.ict_patchify(ctypes.byref(cx), n, h, w, P, ctypes.byref(co), _stream(stream)), "ict_patchify")
+
+
+def patchify(X: DevCE, n, h, w, P, stream=None) -> DevCE:
+    """Non-overlapping P x P patches as the aligned rows of one (C,e) tensor."""
+    rows, K = n * (h // P) * (w // P), P * P * X.cols
+    out = DevCE.empty(rows, K, rows, K)
+    ict_patchify(X, n, h, w, P, out, stream)
+    return out

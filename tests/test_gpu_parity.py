@@ -296,3 +296,41 @@ def test_conv_other_odd_filters(ict, r, global_groups):
     got = ict.conv(ict.CONV_BWD_WEIGHT, d, ict.DevCE.from_host(dY), ict.DevCE.from_host(X), 1, r * r * c).to_host()
     same(got, ref, f"conv {r}x{r} bwd-weight")
     status_ok(ict)
+
+
+@pytest.mark.parametrize("n,h,w,c,P,G,k", [
+    (2, 32, 32, 16, 16, 16, 64),     # channel groups of 16
+    (2, 16, 48, 64, 8, 32, 96),      # two channel groups
+    (2, 32, 32, 3, 16, 3, 64),       # RGB, one exponent, pixels packed (ld = 3)
+])
+def test_patch_embedding(ict, n, h, w, c, P, G, k):
+    """ict_patchify then ict_linear_fwd equals the oracle's P x P, stride P convolution,
+    and ict_linear_bwd_weight on the patches equals the convolution's weight gradient."""
+    import torch
+
+    rng = np.random.default_rng(n + h + c + P)
+    npix = n * h * w
+    X = with_groups(rng.integers(-127, 128, size=(npix, c)).astype(np.int8), npix, G,
+                    lambda s: rng.integers(-9, -5, size=s))
+    W = rand_ce(rng, k, P * P * c, 1, P * P * c, elo=-10, ehi=-6)
+    d = dict(n=n, h=h, w=w, c=c, k=k, r=P, s=P, stride=P, pad=0)
+    if c % 16:
+        Xd = ict.DevCE(torch.from_numpy(X.mant.copy()).cuda(), torch.from_numpy(X.exp.copy()).cuda(), npix, G, cols=c)
+    else:
+        Xd = ict.DevCE.from_host(X)
+    patches = ict.patchify(Xd, n, h, w, P)
+    Y = ict.linear_fwd(patches, ict.DevCE.from_host(W), 32)
+    same(Y.to_host(), oracle.conv(0, d, X, W, 1, 32), f"patch embedding {n}x{h}x{w}x{c} P={P}")
+    # the patches themselves: the oracle's row alignment of X (one target for every
+    # pixel), gathered into (dy, dx, channel) rows by reshaping
+    xa, xe = oracle.align(X, axis=1)
+    rows = n * (h // P) * (w // P)
+    ref_m = xa.reshape(n, h // P, P, w // P, P, c).transpose(0, 1, 3, 2, 4, 5).reshape(rows, P * P * c)
+    got = patches.to_host()
+    assert np.array_equal(got.mant, ref_m) and int(got.exp[0, 0]) == int(xe[0]), "patches"
+    # weight gradient on the patches
+    dY = rand_ce(rng, rows, k, 1, 32, elo=-14, ehi=-10)
+    ref_p = CE(np.ascontiguousarray(ref_m), np.array([[xe[0]]], np.int8), rows, P * P * c)
+    dW = ict.linear_bwd_weight(ict.DevCE.from_host(dY), patches)
+    same(dW.to_host(), oracle.linear_bwd_weight(dY, ref_p, 1, P * P * c), "patch embedding dW")
+    status_ok(ict)
