@@ -66,3 +66,43 @@ def test_header_is_plain_c():
         r = subprocess.run([compiler, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang, std, HEADER],
                            capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_c_program_links_and_gets_errors_without_a_gpu(tmp_path):
+    """A plain C program includes ict.h, links libict.so and calls it.  The build host has
+    no GPU: the version and status strings work, and a Product call returns an error
+    code (no crash, no CPU fallback)."""
+    import shutil
+    import subprocess
+
+    import pytest
+    import torch
+
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    if torch.cuda.is_available():  # the call below passes host buffers: never on a GPU host
+        pytest.skip("meant for a host without a GPU")
+    from integer_only_nn_02_b200.csrc.build import build
+
+    lib = build()
+    src = tmp_path / "use_ict.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "ict.h"
+int main(void) {
+    int8_t m[64 * 64], e[64];
+    ict_tensor X = {m, e, 64, 64, 64, 1, 64}, W = X, Y = X;
+    int32_t st = ict_linear_fwd(&X, &W, &Y, NULL, 0, NULL);
+    printf("%s|%s|%d\n", ict_version(), ict_status_string(st), st != ICT_OK);
+    return 0;
+}
+""")
+    exe = tmp_path / "use_ict"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        lib, "-o", str(exe), f"-Wl,-rpath,{os.path.dirname(lib)}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    version, status, failed = out.stdout.strip().split("|")
+    assert version.startswith("libict") and status.startswith("ICT_ERR") and failed == "1"
