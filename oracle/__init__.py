@@ -87,6 +87,9 @@ def lib():
                                         ctypes.c_int32, P(_OT)]
         L.oracle_relu_fwd.argtypes = [P(_OT), ctypes.c_int, P(_OT)]
         L.oracle_avgpool_fwd.argtypes = [P(_OT)] + [ctypes.c_int] * 4 + [P(_OT)]
+        L.oracle_depthwise.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), P(_OT)]
+        L.oracle_depthwise_acc.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), ctypes.c_void_p,
+                                           ctypes.c_void_p]
         L.oracle_avgpool_bwd.argtypes = [P(_OT)] + [ctypes.c_int] * 4 + [P(_OT)]
         L.oracle_relu_bwd.argtypes = [P(_OT), P(_OT), ctypes.c_int, P(_OT)]
         L.oracle_conv.argtypes = [ctypes.c_int, P(_Conv), P(_OT), P(_OT), P(_OT)]
@@ -313,3 +316,33 @@ def avgpool_bwd(dY: CE, n: int, h: int, w: int, K: int, g_rows: int, g_cols: int
     out = empty_ce(n * h * w, dY.cols, g_rows, g_cols)
     _check(lib().oracle_avgpool_bwd(ctypes.byref(_ot(dY)), n, h, w, K, ctypes.byref(_ot(out))), "avgpool_bwd")
     return out
+
+
+def _dw_shape(direction, d):
+    P = (d["h"] + 2 * d["pad"] - d["r"]) // d["stride"] + 1
+    Q = (d["w"] + 2 * d["pad"] - d["s"]) // d["stride"] + 1
+    if direction == CONV_FWD:
+        return d["n"] * P * Q, d["c"]
+    if direction == CONV_BWD_DATA:
+        return d["n"] * d["h"] * d["w"], d["c"]
+    return d["c"], d["r"] * d["s"]
+
+
+def depthwise(direction: int, d: dict, a: CE, b: CE, g_rows: int, g_cols: int) -> CE:
+    """Depthwise convolution (one filter per channel, d["k"] == d["c"]), FIT into groups."""
+    rows, cols = _dw_shape(direction, d)
+    out = empty_ce(rows, cols, g_rows, g_cols)
+    cd = _Conv(*[int(d[k]) for k in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")])
+    _check(lib().oracle_depthwise(direction, ctypes.byref(cd), ctypes.byref(_ot(a)), ctypes.byref(_ot(b)),
+                                  ctypes.byref(_ot(out))), "depthwise")
+    return out
+
+
+def depthwise_acc(direction: int, d: dict, a: CE, b: CE):
+    rows, cols = _dw_shape(direction, d)
+    acc = np.zeros((rows, cols), np.int64)
+    r = np.zeros((rows, cols), np.int32)
+    cd = _Conv(*[int(d[k]) for k in ("n", "h", "w", "c", "k", "r", "s", "stride", "pad")])
+    _check(lib().oracle_depthwise_acc(direction, ctypes.byref(cd), ctypes.byref(_ot(a)), ctypes.byref(_ot(b)),
+                                      _ptr(acc), _ptr(r)), "depthwise_acc")
+    return acc, r

@@ -595,6 +595,112 @@ int oracle_conv(int dir, const o_conv *d, const o_tensor *a, const o_tensor *b, 
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Public: depthwise convolution (Table 6: "Convolution (incl. 1 x 1, depthwise)" ->      */
+/* Product)                                                                               */
+/* ------------------------------------------------------------------------------------ */
+
+/* Depthwise convolution, one R x S filter per channel (MobileNetV2's 3x3 depthwise
+ * layers; Table 3 trains MobileNetV2).  NHWC activations with exponents uniform over
+ * pixels; W [C][R*S].  The contraction of output channel ch runs over (r, s) of that one
+ * channel, so the activation keeps its per-channel exponent (no alignment across
+ * channels); W is aligned per row (ALIGN_MAX along (r, s)).  Exact int64 sums, exponents
+ * added:
+ *   dir 0  Y [n*P*Q][C]   = sum_(r,s) X[pixel(p,q,r,s)][ch] * W[ch][r,s]
+ *   dir 1  dX [n*h*w][C]  = sum over (p,q,r,s) reaching the pixel of dY[(p,q)][ch] * W[ch][r,s]
+ *   dir 2  dW [C][R*S]    = sum_(p,q) dY[(p,q)][ch] * X[pixel(p,q,r,s)][ch]
+ * d->k must equal d->c. */
+int oracle_depthwise_acc(int dir, const o_conv *d, const o_tensor *a, const o_tensor *b, int64_t *acc,
+                         int32_t *rexp) {
+    int st;
+    if (!d || d->stride < 1 || d->pad < 0 || d->r < 1 || d->s < 1 || d->k != d->c) return ORC_ERR_ARG;
+    if ((st = check_input(a)) || (st = check_input(b))) return st;
+    int64_t N = d->n, H = d->h, Wd = d->w, C = d->c, R = d->r, S = d->s, RS = R * S;
+    int64_t P = out_dim(H, d->pad, R, d->stride), Q = out_dim(Wd, d->pad, S, d->stride);
+    if (P < 1 || Q < 1) return ORC_ERR_ARG;
+    int64_t npix_in = N * H * Wd, npix_out = N * P * Q;
+    if (dir == 0 || dir == 1) {
+        if (a->rows != (dir == 0 ? npix_in : npix_out) || a->cols != C) return ORC_ERR_ARG;
+        if (a->g_rows < a->rows) return ORC_ERR_LAYOUT;
+        if (b->rows != C || b->cols != RS) return ORC_ERR_ARG;
+        int8_t *wa = malloc(C * RS + 1), *we = malloc(C + 1);
+        oracle_align(b, 1, wa, RS, 0, we);
+        if (dir == 0) {
+            for (int64_t op = 0; op < npix_out; op++) {
+                int64_t n = op / (P * Q), p = (op / Q) % P, q = op % Q;
+                for (int64_t ch = 0; ch < C; ch++) {
+                    int64_t sum = 0;
+                    for (int64_t r = 0; r < R; r++)
+                        for (int64_t ss = 0; ss < S; ss++) {
+                            int64_t h = p * d->stride + r - d->pad, w = q * d->stride + ss - d->pad;
+                            if (h < 0 || h >= H || w < 0 || w >= Wd) continue;
+                            sum += (int64_t)mant_at(a, (n * H + h) * Wd + w, ch) * wa[ch * RS + r * S + ss];
+                        }
+                    acc[op * C + ch] = sum;
+                    rexp[op * C + ch] = sum_exp(exp_at(a, 0, ch), we[ch]);
+                }
+            }
+        } else {
+            for (int64_t ip = 0; ip < npix_in; ip++) {
+                int64_t n = ip / (H * Wd), h = (ip / Wd) % H, w = ip % Wd;
+                for (int64_t ch = 0; ch < C; ch++) {
+                    int64_t sum = 0;
+                    for (int64_t r = 0; r < R; r++)
+                        for (int64_t ss = 0; ss < S; ss++) {
+                            int64_t ph = h + d->pad - r, qw = w + d->pad - ss;
+                            if (ph < 0 || qw < 0 || ph % d->stride || qw % d->stride) continue;
+                            int64_t p = ph / d->stride, q = qw / d->stride;
+                            if (p >= P || q >= Q) continue;
+                            sum += (int64_t)mant_at(a, (n * P + p) * Q + q, ch) * wa[ch * RS + r * S + ss];
+                        }
+                    acc[ip * C + ch] = sum;
+                    rexp[ip * C + ch] = sum_exp(exp_at(a, 0, ch), we[ch]);
+                }
+            }
+        }
+        free(wa);
+        free(we);
+        return ORC_OK;
+    }
+    if (dir == 2) {
+        if (a->rows != npix_out || a->cols != C || b->rows != npix_in || b->cols != C) return ORC_ERR_ARG;
+        if (a->g_rows < a->rows || b->g_rows < b->rows) return ORC_ERR_LAYOUT;
+        for (int64_t ch = 0; ch < C; ch++)
+            for (int64_t r = 0; r < R; r++)
+                for (int64_t ss = 0; ss < S; ss++) {
+                    int64_t sum = 0;
+                    for (int64_t op = 0; op < npix_out; op++) {
+                        int64_t n = op / (P * Q), p = (op / Q) % P, q = op % Q;
+                        int64_t h = p * d->stride + r - d->pad, w = q * d->stride + ss - d->pad;
+                        if (h < 0 || h >= H || w < 0 || w >= Wd) continue;
+                        sum += (int64_t)mant_at(a, op, ch) * mant_at(b, (n * H + h) * Wd + w, ch);
+                    }
+                    acc[ch * RS + r * S + ss] = sum;
+                    rexp[ch * RS + r * S + ss] = sum_exp(exp_at(a, 0, ch), exp_at(b, 0, ch));
+                }
+        return ORC_OK;
+    }
+    return ORC_ERR_ARG;
+}
+
+int oracle_depthwise(int dir, const o_conv *d, const o_tensor *a, const o_tensor *b, o_tensor *out) {
+    if (!d || d->stride < 1) return ORC_ERR_ARG;
+    int64_t P = out_dim(d->h, d->pad, d->r, d->stride), Q = out_dim(d->w, d->pad, d->s, d->stride);
+    int64_t rows, cols = d->c;
+    if (dir == 0) rows = (int64_t)d->n * P * Q;
+    else if (dir == 1) rows = (int64_t)d->n * d->h * d->w;
+    else if (dir == 2) { rows = d->c; cols = (int64_t)d->r * d->s; }
+    else return ORC_ERR_ARG;
+    if (check_output(out, rows, cols)) return ORC_ERR_ARG;
+    int64_t *acc = malloc(sizeof(int64_t) * (rows * cols + 1));
+    int32_t *r = malloc(sizeof(int32_t) * (rows * cols + 1));
+    int st = oracle_depthwise_acc(dir, d, a, b, acc, r);
+    if (!st) st = fit_acc(acc, r, out);
+    free(acc);
+    free(r);
+    return st;
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Public: integer SGD with momentum and per-group velocity (Figure 1b)                  */
 /* ------------------------------------------------------------------------------------ */
 

@@ -662,3 +662,60 @@ def test_avgpool_bwd_matches_bruteforce(n, h, w, c, K, dyg, dxg):
             for img in range(n) for y in range(h) for x in range(w)]
     mant, exps = fit_matrix_brute(vals, *dxg)
     assert dX.mant.tolist() == mant and dX.exp.tolist() == exps
+
+
+# --------------------------------------------------------------------- depthwise convolution
+
+
+@pytest.mark.parametrize("geom", [dict(), dict(stride=2), dict(r=5, s=5, pad=2), dict(h=4, w=4, r=1, s=1, pad=0)])
+def test_depthwise_acc_matches_torch_grouped_conv(geom):
+    """Depthwise sums against torch's grouped convolution (groups = channels) in float64
+    on the exact mantissas, all three directions, and the exponents each sum carries."""
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    rng = np.random.default_rng(95)
+    n, h, w, c = geom.get("n", 2), geom.get("h", 6), geom.get("w", 5), 8
+    r, s, pad, stride = geom.get("r", 3), geom.get("s", 3), geom.get("pad", 1), geom.get("stride", 1)
+    P, Q = (h + 2 * pad - r) // stride + 1, (w + 2 * pad - s) // stride + 1
+    X = rand_ce(rng, n * h * w, c, n * h * w, 4, zero_groups=0.2)
+    W = rand_ce(rng, c, r * s, 1, r * s)
+    dY = rand_ce(rng, n * P * Q, c, n * P * Q, 2, zero_groups=0.2)
+    d = dict(n=n, h=h, w=w, c=c, k=c, r=r, s=s, stride=stride, pad=pad)
+    xt = torch.tensor(X.mant, dtype=torch.float64).reshape(n, h, w, c).permute(0, 3, 1, 2)
+    wt = torch.tensor(W.mant, dtype=torch.float64).reshape(c, 1, r, s)
+    yt = torch.tensor(dY.mant, dtype=torch.float64).reshape(n, P, Q, c).permute(0, 3, 1, 2)
+    ex = np.repeat(X.exp[0], 4)[:c].astype(np.int32)
+    ey = np.repeat(dY.exp[0], 2)[:c].astype(np.int32)
+    ew = W.exp[:, 0].astype(np.int32)
+
+    def esum(a, b):
+        return np.where((a == E_ZERO) | (b == E_ZERO), 0, a + b)
+
+    acc, rx = oracle.depthwise_acc(0, d, X, W)
+    ref = F.conv2d(xt, wt, stride=stride, padding=pad, groups=c).permute(0, 2, 3, 1).reshape(-1, c)
+    assert (acc == ref.numpy().astype(np.int64)).all()
+    assert (rx == esum(ex, ew)[None, :]).all()
+    acc, rx = oracle.depthwise_acc(1, d, dY, W)
+    op = ((h + 2 * pad - r) % stride, (w + 2 * pad - s) % stride)
+    ref = F.conv_transpose2d(yt, wt, stride=stride, padding=pad, output_padding=op, groups=c)
+    assert (acc == ref.permute(0, 2, 3, 1).reshape(-1, c).numpy().astype(np.int64)).all()
+    assert (rx == esum(ey, ew)[None, :]).all()
+    acc, rx = oracle.depthwise_acc(2, d, dY, X)
+    ref = torch.nn.grad.conv2d_weight(xt, (c, 1, r, s), yt, stride=stride, padding=pad, groups=c)
+    assert (acc == ref.reshape(c, r * s).numpy().astype(np.int64)).all()
+    assert (rx == esum(ey, ex)[:, None]).all()
+
+
+def test_depthwise_outputs_match_bruteforce_fit():
+    rng = np.random.default_rng(96)
+    n, h, w, c, r = 1, 4, 4, 4, 3
+    X = rand_ce(rng, n * h * w, c, n * h * w, 2)
+    W = rand_ce(rng, c, r * r, 1, r * r)
+    d = dict(n=n, h=h, w=w, c=c, k=c, r=r, s=r, stride=1, pad=1)
+    Y = oracle.depthwise(0, d, X, W, n * h * w, 2)
+    vx, vw = ce_values(X), ce_values(W)
+    vals = [[sum(vx[(y + dy - 1) * w + (x + dx - 1)][ch] * vw[ch][dy * r + dx]
+                 for dy in range(r) for dx in range(r) if 0 <= y + dy - 1 < h and 0 <= x + dx - 1 < w)
+             for ch in range(c)] for y in range(h) for x in range(w)]
+    mant, exps = fit_matrix_brute(vals, n * h * w, 2)
+    assert Y.mant.tolist() == mant and Y.exp.tolist() == exps
