@@ -71,6 +71,8 @@ def lib():
         L = _lib
         L.oracle_requant.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
                                      ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, P(_OT)]
+        L.oracle_requant_bits.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                          ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, P(_OT)]
         L.oracle_align_to.argtypes = [P(_OT), ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_int64, ctypes.c_int]
         L.oracle_align.argtypes = [P(_OT), ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
@@ -157,6 +159,16 @@ def requant(x: np.ndarray, g_rows: int, g_cols: int, base_exp: int = 0,
                                 None if re is None else _ptr(re),
                                 None if ce is None else _ptr(ce), ctypes.byref(_ot(out)))
     _check(code, "requant")
+    return out
+
+
+def requant_bits(x: np.ndarray, bits: int, g_rows: int, g_cols: int, base_exp: int = 0) -> CE:
+    """FIT with B-bit mantissas (clip bound 2^(bits-1) - 1)."""
+    x = np.ascontiguousarray(x, np.int64)
+    rows, cols = x.shape
+    out = empty_ce(rows, cols, g_rows, g_cols)
+    _check(lib().oracle_requant_bits(rows, cols, _ptr(x), cols, base_exp, None, None, int(bits),
+                                     ctypes.byref(_ot(out))), "requant_bits")
     return out
 
 

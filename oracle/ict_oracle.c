@@ -110,9 +110,9 @@ static i128 rne_scale(i128 x, int k) {
     return q;
 }
 
-static int fits_at(i128 x, int r, int e) {
+static int fits_at_q(i128 x, int r, int e, int qmax) {
     i128 q = rne_scale(x, r - e);
-    return q >= -QMAX && q <= QMAX;
+    return q >= -qmax && q <= qmax;
 }
 
 static int bitlen(i128 x) {
@@ -126,21 +126,23 @@ static int bitlen(i128 x) {
  * x != 0.  Written as the definition: start where it surely does not fit (|x| scaled to
  * at least 128) and step up until it does.  Reading of the spec requant rule
  * "smallest exponent that fits the group maximum". */
-static int need(i128 x, int r) {
-    int e = r + bitlen(x) - 8; /* here |x| * 2^(r-e) >= 2^7: does not fit */
-    while (!fits_at(x, r, e)) e++;
+static int need_q(i128 x, int r, int qmax) {
+    int e = r + bitlen(x) - 8; /* here |x| * 2^(r-e) >= 2^7 > qmax: does not fit */
+    while (!fits_at_q(x, r, e, qmax)) e++;
     return e;
 }
+static int need(i128 x, int r) { return need_q(x, r, QMAX); }
 
 /* FIT of one group of n values x[i] at exponents r[i]: the group exponent is the max of
  * need over the nonzero members (E_ZERO when all are zero), clamped below at -127; each
  * mantissa is RNE(x[i] * 2^(r[i] - e)).  Returns the exponent, or a value > 127 when the
  * group cannot be represented (ORC_ERR_EXP_RANGE). */
-static int fit_group(int64_t n, const i128 *x, const int *r, int8_t *c_out) {
+/* (the same with a clip bound qmax below 127: the B-bit variants of Table 4) */
+static int fit_group_q(int64_t n, const i128 *x, const int *r, int8_t *c_out, int qmax) {
     int have = 0, e = 0;
     for (int64_t i = 0; i < n; i++) {
         if (x[i] == 0) continue;
-        int ni = need(x[i], r[i]);
+        int ni = need_q(x[i], r[i], qmax);
         if (!have || ni > e) e = ni;
         have = 1;
     }
@@ -155,16 +157,19 @@ static int fit_group(int64_t n, const i128 *x, const int *r, int8_t *c_out) {
     }
     for (int64_t i = 0; i < n; i++) {
         i128 q = x[i] == 0 ? 0 : rne_scale(x[i], r[i] - e);
-        if (q < -QMAX) q = -QMAX; /* never taken: e fits every member */
-        if (q > QMAX) q = QMAX;
+        if (q < -qmax) q = -qmax; /* never taken: e fits every member */
+        if (q > qmax) q = qmax;
         c_out[i] = (int8_t)q;
     }
     return e;
 }
+static int fit_group(int64_t n, const i128 *x, const int *r, int8_t *c_out) {
+    return fit_group_q(n, x, r, c_out, QMAX);
+}
 
 /* FIT of a whole matrix of values (x at exponent r, element (i,j) at i*cols+j) into the
  * groups of `out`. */
-static int fit_matrix(const i128 *x, const int *r, o_tensor *out) {
+static int fit_matrix_q(const i128 *x, const int *r, o_tensor *out, int qmax) {
     int64_t ngr = n_grp_rows(out), ngc = n_grp_cols(out);
     int status = ORC_OK;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -185,7 +190,7 @@ static int fit_matrix(const i128 *x, const int *r, o_tensor *out) {
                     gr[n] = r[i * out->cols + j];
                     n++;
                 }
-            int e = fit_group(n, gx, gr, gc);
+            int e = fit_group_q(n, gx, gr, gc, qmax);
             if (e > 127) {
 #pragma omp atomic write
                 status = ORC_ERR_EXP_RANGE;
@@ -202,6 +207,7 @@ static int fit_matrix(const i128 *x, const int *r, o_tensor *out) {
     }
     return status;
 }
+static int fit_matrix(const i128 *x, const int *r, o_tensor *out) { return fit_matrix_q(x, r, out, QMAX); }
 
 /* ------------------------------------------------------------------------------------ */
 /* Sum primitive: exact sum of two (C,e) terms                                          */
@@ -255,6 +261,29 @@ int oracle_requant(int64_t rows, int64_t cols, const int64_t *x, int64_t ldx, in
             r[i * cols + j] = base_exp + re + ce;
         }
     if (status == ORC_OK) status = fit_matrix(v, r, out);
+    free(v);
+    free(r);
+    return status;
+}
+
+/* FIT with B-bit mantissas (Table 4 sweeps B = 4..8): the clip bound is
+ * q_max = 2^(B-1) - 1 instead of 127 (Table 7's q_max); everything else as in
+ * oracle_requant.  Mantissas are stored one per byte. */
+int oracle_requant_bits(int64_t rows, int64_t cols, const int64_t *x, int64_t ldx, int32_t base_exp,
+                        const int8_t *row_exp, const int8_t *col_exp, int32_t bits, o_tensor *out) {
+    if (!x || ldx < cols || bits < 2 || bits > 8 || check_output(out, rows, cols)) return ORC_ERR_ARG;
+    i128 *v = malloc(sizeof(i128) * (rows * cols + 1));
+    int *r = malloc(sizeof(int) * (rows * cols + 1));
+    int status = ORC_OK;
+    for (int64_t i = 0; i < rows; i++)
+        for (int64_t j = 0; j < cols; j++) {
+            int64_t val = x[i * ldx + j];
+            int re = row_exp ? row_exp[i] : 0, ce = col_exp ? col_exp[j] : 0;
+            if ((re == E_ZERO || ce == E_ZERO) && val != 0) status = ORC_ERR_ARG;
+            v[i * cols + j] = val;
+            r[i * cols + j] = base_exp + re + ce;
+        }
+    if (status == ORC_OK) status = fit_matrix_q(v, r, out, (1 << (bits - 1)) - 1);
     free(v);
     free(r);
     return status;

@@ -18,18 +18,18 @@ def value(c: int, e: int) -> Fraction:
     return Fraction(c) * pow2(e)
 
 
-def fits(v: Fraction, e: int) -> bool:
-    return abs(round(v / pow2(e))) <= 127
+def fits(v: Fraction, e: int, qmax: int = 127) -> bool:
+    return abs(round(v / pow2(e))) <= qmax
 
 
-def fit_brute(values):
+def fit_brute(values, qmax: int = 127):
     """Group exponent and mantissas for exact rational values (scan from below)."""
     nz = [v for v in values if v != 0]
     if not nz:
         return [0] * len(values), E_ZERO
     m = max(abs(v) for v in nz)
     e = m.numerator.bit_length() - m.denominator.bit_length() - 12  # m / 2^e >= 2^10
-    while not all(fits(v, e) for v in nz):
+    while not all(fits(v, e, qmax) for v in nz):
         e += 1
     e = max(e, -127)
     return [round(v / pow2(e)) for v in values], e

@@ -719,3 +719,32 @@ def test_depthwise_outputs_match_bruteforce_fit():
              for ch in range(c)] for y in range(h) for x in range(w)]
     mant, exps = fit_matrix_brute(vals, n * h * w, 2)
     assert Y.mant.tolist() == mant and Y.exp.tolist() == exps
+
+
+# --------------------------------------------------------------------- B-bit mantissas (Table 4)
+
+
+@pytest.mark.parametrize("bits", [4, 5, 6, 7, 8])
+def test_requant_bits_matches_bruteforce(bits):
+    rng = np.random.default_rng(100 + bits)
+    x = rng.integers(-(2 ** 20), 2 ** 20, size=(6, 24)).astype(np.int64)
+    x[rng.random(x.shape) < 0.15] = 0
+    x[2] = 0  # an all-zero row: E_ZERO groups
+    qmax = 2 ** (bits - 1) - 1
+    out = oracle.requant_bits(x, bits, 1, 8, base_exp=-5)
+    assert np.abs(out.mant).max() <= qmax
+    mant = [[0] * 24 for _ in range(6)]
+    exps = [[E_ZERO] * 3 for _ in range(6)]
+    for gi, gj, cells in groups_of(6, 24, 1, 8):
+        c, e = fit_brute([value(int(x[i, j]), -5) for i, j in cells], qmax=qmax)
+        exps[gi][gj] = e
+        for (i, j), cc in zip(cells, c):
+            mant[i][j] = cc
+    assert out.mant.tolist() == mant and out.exp.tolist() == exps
+
+
+def test_requant_bits_8_is_requant():
+    rng = np.random.default_rng(110)
+    x = rng.integers(-(2 ** 30), 2 ** 30, size=(9, 40)).astype(np.int64)
+    a, b = oracle.requant_bits(x, 8, 1, 8, base_exp=3), oracle.requant(x, 1, 8, base_exp=3)
+    assert (a.mant == b.mant).all() and (a.exp == b.exp).all()
