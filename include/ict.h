@@ -294,6 +294,21 @@ int32_t ict_conv_bwd_weight_partial(const ict_conv_desc *d, const ict_tensor *dY
                                     int8_t *e_k, int8_t *e_rsc, void *ws, size_t ws_bytes,
                                     void *stream);
 
+/* Depthwise convolution, one R x S filter per channel (Table 6: "Convolution (incl.    */
+/* 1 x 1, depthwise)" -> Product; MobileNetV2).  d->k must equal d->c; any stride and    */
+/* padding, R * S <= 49.  The contraction of channel ch runs over its own taps, so the    */
+/* sums keep the activation's per-channel exponent: element exponent e_act[ch] + e_w[ch].*/
+/*   dir FWD         a = X  [n*h*w][c], b = W [c][r*s] -> out = Y  [n*P*Q][c]          */
+/*   dir BWD_DATA    a = dY [n*P*Q][c], b = W [c][r*s] -> out = dX [n*h*w][c]          */
+/*   dir BWD_WEIGHT  a = dY [n*P*Q][c], b = X [n*h*w][c] -> out = dW [c][r*s]          */
+/* Activation exponents uniform over pixels (g_rows >= rows); W and dW one group per row */
+/* (g_rows = 1, g_cols >= r*s).  FWD / BWD_DATA outputs: any group geometry, rounded in  */
+/* two passes with an int32 per output group of workspace (ict_depthwise_workspace).     */
+/* Byte accesses on CUDA cores (the contraction has 9-49 terms per output).              */
+size_t ict_depthwise_workspace(int32_t dir, const ict_conv_desc *d, const ict_tensor *out);
+int32_t ict_depthwise(int32_t dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
+                      ict_tensor *out, void *ws, size_t ws_bytes, void *stream);
+
 /* Patch embedding (a P x P convolution with stride P, as a ViT's first layer): the     */
 /* non-overlapping patches of NHWC X [n*h*w][c] gathered into the rows of             */
 /* out [n*(h/P)*(w/P)][P*P*c] in (dy, dx, channel) order, ALIGN_MAX-ed to one exponent */

@@ -1940,6 +1940,69 @@ int32_t ict_patchify(const ict_tensor *X, int32_t n, int32_t h, int32_t w, int32
     return launch_status();
 }
 
+size_t ict_depthwise_workspace(int32_t dir, const ict_conv_desc *d, const ict_tensor *out) {
+    if (!d || !out || dir == ICT_CONV_BWD_WEIGHT) return 256;
+    return (size_t)round_up(std::max<int64_t>(n_grp_rows(out) * n_grp_cols(out) * 4, 1), 256);
+}
+int32_t ict_depthwise(int32_t dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
+                      ict_tensor *out, void *ws, size_t ws_bytes, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if (!d || (st = check_tensor(a)) || (st = check_tensor(b)) || (st = check_tensor(out)))
+        return d ? st : ICT_ERR_INVALID_ARG;
+    if (d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1 || d->k != d->c || d->r < 1 || d->s < 1 || d->stride < 1 ||
+        d->pad < 0 || d->r * d->s > kDwMaxTaps)
+        return ICT_ERR_INVALID_ARG;
+    const int64_t P = (d->h + 2 * d->pad - d->r) / d->stride + 1, Q = (d->w + 2 * d->pad - d->s) / d->stride + 1;
+    if (P < 1 || Q < 1) return ICT_ERR_INVALID_ARG;
+    const int64_t C = d->c, RS = (int64_t)d->r * d->s;
+    const int64_t npix_in = (int64_t)d->n * d->h * d->w, npix_out = (int64_t)d->n * P * Q;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dir == ICT_CONV_BWD_WEIGHT) {  // a = dY, b = X, out = dW [C][R*S]
+        if (a->rows != npix_out || a->cols != C || b->rows != npix_in || b->cols != C) return ICT_ERR_INVALID_ARG;
+        if (out->rows != C || out->cols != RS) return ICT_ERR_INVALID_ARG;
+        if (a->g_rows < a->rows || b->g_rows < b->rows) return ICT_ERR_LAYOUT;  // pixel-uniform exponents
+        if ((out->g_rows != 1 && C > 1) || out->g_cols < RS) return ICT_ERR_LAYOUT;  // one group per row
+        DwWgradArgs w;
+        memset(&w, 0, sizeof(w));
+        w.dy = a->mant, w.dy_exp = a->exp, w.ldy = a->ld, w.dy_gcols = clamp_div(a->g_cols, a->cols);
+        w.x = b->mant, w.x_exp = b->exp, w.ldx = b->ld, w.x_gcols = clamp_div(b->g_cols, b->cols);
+        w.out = out->mant, w.out_exp = out->exp, w.ldo = out->ld;
+        w.n = d->n, w.h = d->h, w.w_ = d->w, w.C = (int)C, w.R = d->r, w.S = d->s, w.pad = d->pad;
+        w.stride = d->stride, w.P = (int)P, w.Q = (int)Q;
+        KTimer kt(s, KC_OTHER, (double)npix_out * C + (double)npix_in * C + (double)C * RS);
+        dw_wgrad_kernel<<<(unsigned)C, 256, 0, s>>>(w);
+        counted(1);
+        return launch_status();
+    }
+    if (dir != ICT_CONV_FWD && dir != ICT_CONV_BWD_DATA) return ICT_ERR_INVALID_ARG;
+    const bool bwd = dir == ICT_CONV_BWD_DATA;
+    if (a->rows != (bwd ? npix_out : npix_in) || a->cols != C) return ICT_ERR_INVALID_ARG;
+    if (b->rows != C || b->cols != RS) return ICT_ERR_INVALID_ARG;
+    if (out->rows != (bwd ? npix_in : npix_out) || out->cols != C) return ICT_ERR_INVALID_ARG;
+    if (a->g_rows < a->rows) return ICT_ERR_LAYOUT;                 // pixel-uniform exponents
+    if ((b->g_rows != 1 && C > 1) || b->g_cols < RS) return ICT_ERR_LAYOUT;  // one exponent per filter
+    DwArgs x;
+    memset(&x, 0, sizeof(x));
+    x.a = a->mant, x.a_exp = a->exp, x.lda = a->ld, x.a_gcols = clamp_div(a->g_cols, a->cols);
+    x.w = b->mant, x.w_exp = b->exp, x.ldw = b->ld;
+    x.out = out->mant, x.out_exp = out->exp, x.ldo = out->ld, x.out_rows = out->rows, x.out_ngc = n_grp_cols(out);
+    x.out_g_rows = clamp_div(out->g_rows, out->rows), x.out_g_cols = clamp_div(out->g_cols, out->cols);
+    x.h = d->h, x.w_ = d->w, x.C = (int)C, x.R = d->r, x.S = d->s, x.pad = d->pad, x.stride = d->stride;
+    x.P = (int)P, x.Q = (int)Q, x.bwd = bwd;
+    const int64_t groups = n_grp_rows(out) * n_grp_cols(out), n = out->rows * C;
+    if (n == 0) return ICT_OK;
+    if (!ws || ((uintptr_t)ws & 255) || ws_bytes < (size_t)groups * 4) return ICT_ERR_WORKSPACE;
+    x.need = (int32_t *)ws;
+    if (cudaMemsetAsync(x.need, 0x80, (size_t)groups * 4, s) != cudaSuccess) return ICT_ERR_CUDA;
+    KTimer kt(s, KC_OTHER, (double)(bwd ? npix_out : npix_in) * C + (double)n + (double)C * RS);
+    const unsigned grid = stream_grid(n, 1);
+    dw_need_kernel<<<grid, 256, 0, s>>>(x);
+    dw_round_kernel<<<grid, 256, 0, s>>>(x);
+    counted(2);
+    return launch_status();
+}
+
 }  // extern "C"
 
 int sum_entry(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_tensor *Y, int32_t y_mul,

@@ -402,4 +402,152 @@ __global__ void __launch_bounds__(256) patchify_kernel(const __grid_constant__ P
         eg == kEZero ? make_uint4(0, 0, 0, 0) : rne_shift16(raw, min(es - eg, 8));
 }
 
+// ------------------------------------------------------------------ depthwise convolution
+
+// One R x S filter per channel (Table 6: "Convolution (incl. 1 x 1, depthwise)" ->
+// Product; MobileNetV2's depthwise layers).  The contraction of channel ch runs over
+// (r, s) of that channel only, so each sum keeps the activation's per-channel exponent:
+// every output element is an exact integer S at exponent e_act[ch] + e_w[ch], rounded by
+// FIT into the output's groups in two passes (the groups' needs, then the rounding).
+// Activations are NHWC with exponents uniform over pixels; W [C][R*S] has one exponent
+// per row.
+struct DwArgs {
+    const int8_t *a, *a_exp;  // X (forward) or dY (backward-data), [rows][C]
+    int64_t lda;
+    int a_gcols;
+    const int8_t *w, *w_exp;  // W [C][R*S], w_exp[ch]
+    int64_t ldw;
+    int8_t *out, *out_exp;
+    int64_t ldo, out_rows, out_ngc;
+    int out_g_rows, out_g_cols;
+    int h, w_, C, R, S, pad, stride, P, Q, bwd;
+    int32_t *need;
+};
+
+__device__ __forceinline__ void dw_value(const DwArgs &a, int64_t i, int ch, int64_t &sum, int &r) {
+    sum = 0;
+    const int8_t *wr = a.w + (int64_t)ch * a.ldw;
+    if (!a.bwd) {  // output pixel i = (img, p, q)
+        const int64_t pq = (int64_t)a.P * a.Q, img = i / pq, p = (i - img * pq) / a.Q, q = i - img * pq - p * a.Q;
+        for (int rr = 0; rr < a.R; ++rr) {
+            const int64_t y = p * a.stride + rr - a.pad;
+            if (y < 0 || y >= a.h) continue;
+            for (int ss = 0; ss < a.S; ++ss) {
+                const int64_t x = q * a.stride + ss - a.pad;
+                if (x < 0 || x >= a.w_) continue;
+                sum += (int64_t)a.a[((img * a.h + y) * a.w_ + x) * a.lda + ch] * wr[rr * a.S + ss];
+            }
+        }
+    } else {  // input pixel i = (img, y, x) gathers every (p, q, r, s) that reads it
+        const int64_t hw = (int64_t)a.h * a.w_, img = i / hw, y = (i - img * hw) / a.w_, x = i - img * hw - y * a.w_;
+        for (int rr = 0; rr < a.R; ++rr) {
+            const int64_t ph = y + a.pad - rr;
+            if (ph < 0 || ph % a.stride) continue;
+            const int64_t p = ph / a.stride;
+            if (p >= a.P) continue;
+            for (int ss = 0; ss < a.S; ++ss) {
+                const int64_t qw = x + a.pad - ss;
+                if (qw < 0 || qw % a.stride) continue;
+                const int64_t q = qw / a.stride;
+                if (q >= a.Q) continue;
+                sum += (int64_t)a.a[((img * a.P + p) * a.Q + q) * a.lda + ch] * wr[rr * a.S + ss];
+            }
+        }
+    }
+    const int ea = a.a_exp[ch / a.a_gcols], ew = a.w_exp[ch];
+    r = (ea == kEZero || ew == kEZero) ? 0 : ea + ew;
+}
+
+__global__ void __launch_bounds__(256) dw_need_kernel(const __grid_constant__ DwArgs a) {
+    const int64_t n = a.out_rows * a.C, stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t0 = (int64_t)blockIdx.x * blockDim.x; t0 < n; t0 += stride) {  // whole warps iterate together
+        const int64_t t = t0 + threadIdx.x;
+        int e = kNoExp;
+        int64_t g = -1;
+        if (t < n) {
+            const int64_t i = t / a.C;
+            const int ch = (int)(t - i * a.C);
+            int64_t sum;
+            int r;
+            dw_value(a, i, ch, sum, r);
+            if (sum) e = need64(sum, r);
+            g = (i / a.out_g_rows) * a.out_ngc + ch / a.out_g_cols;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, (long long)g);
+        const int m = __reduce_max_sync(peers, e);
+        if (g >= 0 && m > kNoExp && (threadIdx.x & 31) == __ffs(peers) - 1) atomicMax(&a.need[g], m);
+    }
+}
+
+__global__ void __launch_bounds__(256) dw_round_kernel(const __grid_constant__ DwArgs a) {
+    const int64_t n = a.out_rows * a.C, stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += stride) {
+        const int64_t i = t / a.C;
+        const int ch = (int)(t - i * a.C);
+        const int64_t g = (i / a.out_g_rows) * a.out_ngc + ch / a.out_g_cols;
+        const int m = a.need[g];
+        const int E = finalize_exp(m <= kNoExp ? kNoExp : m);
+        if (i % a.out_g_rows == 0 && ch % a.out_g_cols == 0) a.out_exp[g] = (int8_t)E;
+        int64_t sum;
+        int r;
+        dw_value(a, i, ch, sum, r);
+        a.out[i * a.ldo + ch] = (int8_t)(sum && E != kEZero ? requant64(sum, r, E) : 0);
+    }
+}
+
+// Backward weight: one block per channel sums dY[(p,q)][ch] * X[pixel(p,q,r,s)][ch] over
+// every output pixel for each of the R*S taps (int64, exact), then rounds the row of R*S
+// sums by FIT (one group per row) and writes it with its exponent.
+struct DwWgradArgs {
+    const int8_t *dy, *dy_exp, *x, *x_exp;
+    int64_t ldy, ldx;
+    int dy_gcols, x_gcols;
+    int8_t *out, *out_exp;
+    int64_t ldo;
+    int n, h, w_, C, R, S, pad, stride, P, Q;
+};
+constexpr int kDwMaxTaps = 49;
+__global__ void __launch_bounds__(256) dw_wgrad_kernel(const __grid_constant__ DwWgradArgs a) {
+    const int ch = blockIdx.x, taps = a.R * a.S;
+    __shared__ long long part[8][kDwMaxTaps];
+    __shared__ int emax_s;
+    long long acc[kDwMaxTaps];
+    for (int k = 0; k < taps; ++k) acc[k] = 0;
+    const int64_t pq = (int64_t)a.P * a.Q, nout = (int64_t)a.n * pq;
+    for (int64_t op = threadIdx.x; op < nout; op += blockDim.x) {
+        const int dyv = a.dy[op * a.ldy + ch];
+        if (!dyv) continue;
+        const int64_t img = op / pq, p = (op - img * pq) / a.Q, q = op - img * pq - p * a.Q;
+        for (int rr = 0; rr < a.R; ++rr) {
+            const int64_t y = p * a.stride + rr - a.pad;
+            if (y < 0 || y >= a.h) continue;
+            for (int ss = 0; ss < a.S; ++ss) {
+                const int64_t x = q * a.stride + ss - a.pad;
+                if (x < 0 || x >= a.w_) continue;
+                acc[rr * a.S + ss] += (long long)dyv * a.x[((img * a.h + y) * a.w_ + x) * a.ldx + ch];
+            }
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int k = 0; k < taps; ++k) {
+        long long v = acc[k];
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) part[warp][k] = v;
+    }
+    if (threadIdx.x == 0) emax_s = kNoExp;
+    __syncthreads();
+    const int ey = a.dy_exp[ch / a.dy_gcols], ex = a.x_exp[ch / a.x_gcols];
+    const int r = (ey == kEZero || ex == kEZero) ? 0 : ey + ex;
+    long long total = 0;
+    if (threadIdx.x < taps) {
+        for (int wi = 0; wi < (int)(blockDim.x >> 5); ++wi) total += part[wi][threadIdx.x];
+        if (total) atomicMax(&emax_s, need64(total, r));
+    }
+    __syncthreads();
+    const int E = finalize_exp(emax_s);
+    if (threadIdx.x < taps)
+        a.out[(int64_t)ch * a.ldo + threadIdx.x] = (int8_t)(total && E != kEZero ? requant64(total, r, E) : 0);
+    if (threadIdx.x == 0) a.out_exp[ch] = (int8_t)E;
+}
+
 }  // namespace ict

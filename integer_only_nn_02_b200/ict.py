@@ -94,6 +94,8 @@ _SIGS = {
     "ict_avgpool_bwd": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
     "ict_sum_act": ([_P(ict_tensor)] * 3 + [_i32, _vp, _sz, _vp], _i32),
     "ict_conv_fwd_act": ([_P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_i32, _vp, _sz, _vp], _i32),
+    "ict_depthwise_workspace": ([_i32, _P(ict_conv_desc), _P(ict_tensor)], _sz),
+    "ict_depthwise": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
     "ict_patchify": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp], _i32),
     "ict_sum_scaled": ([_P(ict_tensor), _i32, _i32, _P(ict_tensor), _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
 }
@@ -558,4 +560,30 @@ def patchify(X: DevCE, n, h, w, P, stream=None) -> DevCE:
     rows, K = n * (h // P) * (w // P), P * P * X.cols
     out = DevCE.empty(rows, K, rows, K)
     ict_patchify(X, n, h, w, P, out, stream)
+    return out
+
+
+def ict_depthwise_workspace(direction: int, d: dict, out: DevCE) -> int:
+    cd, co = conv_desc(d), out.c()
+    return int(lib.ict_depthwise_workspace(direction, ctypes.byref(cd), ctypes.byref(co)))
+
+
+def ict_depthwise(direction: int, d: dict, a: DevCE, b: DevCE, out: DevCE, ws=None, stream=None):
+    cd, ca, cb, co = conv_desc(d), a.c(), b.c(), out.c()
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib.ict_depthwise(direction, ctypes.byref(cd), ctypes.byref(ca), ctypes.byref(cb), ctypes.byref(co),
+                             _ptr(ws), nbytes, _stream(stream)), "ict_depthwise")
+
+
+def depthwise(direction: int, d: dict, a: DevCE, b: DevCE, g_rows: int, g_cols: int, stream=None) -> DevCE:
+    P = (d["h"] + 2 * d["pad"] - d["r"]) // d["stride"] + 1
+    Q = (d["w"] + 2 * d["pad"] - d["s"]) // d["stride"] + 1
+    if direction == CONV_FWD:
+        rows, cols = d["n"] * P * Q, d["c"]
+    elif direction == CONV_BWD_DATA:
+        rows, cols = d["n"] * d["h"] * d["w"], d["c"]
+    else:
+        rows, cols = d["c"], d["r"] * d["s"]
+    out = DevCE.empty(rows, cols, g_rows, g_cols)
+    ict_depthwise(direction, d, a, b, out, _ws(max(256, ict_depthwise_workspace(direction, d, out))), stream)
     return out

@@ -334,3 +334,26 @@ def test_patch_embedding(ict, n, h, w, c, P, G, k):
     dW = ict.linear_bwd_weight(ict.DevCE.from_host(dY), patches)
     same(dW.to_host(), oracle.linear_bwd_weight(dY, ref_p, 1, P * P * c), "patch embedding dW")
     status_ok(ict)
+
+
+@pytest.mark.parametrize("geom", [dict(), dict(stride=2), dict(r=5, pad=2), dict(r=1, pad=0)])
+@pytest.mark.parametrize("global_groups", [True, False])
+def test_depthwise(ict, geom, global_groups):
+    """Depthwise convolution (one filter per channel) in the three directions against the
+    oracle, bit for bit."""
+    rng = np.random.default_rng(60 + geom.get("r", 3) + geom.get("stride", 1) + global_groups)
+    n, h, w, c = 2, 9, 10, 96
+    r, pad, stride = geom.get("r", 3), geom.get("pad", 1), geom.get("stride", 1)
+    P, Q = (h + 2 * pad - r) // stride + 1, (w + 2 * pad - r) // stride + 1
+    X = rand_ce(rng, n * h * w, c, n * h * w, 32, elo=-8, ehi=-5, zero_groups=0.1)
+    W = rand_ce(rng, c, r * r, 1, r * r, elo=-9, ehi=-6)
+    dY = rand_ce(rng, n * P * Q, c, n * P * Q, 32, elo=-14, ehi=-11, zero_groups=0.1)
+    d = dict(n=n, h=h, w=w, c=c, k=c, r=r, s=r, stride=stride, pad=pad)
+    dev = ict.DevCE.from_host
+    for direction, a, rows in ((0, X, n * P * Q), (1, dY, n * h * w)):
+        g_rows = rows if global_groups else 1
+        got = ict.depthwise(direction, d, dev(a), dev(W), g_rows, 32).to_host()
+        same(got, oracle.depthwise(direction, d, a, W, g_rows, 32), f"depthwise dir={direction} {geom}")
+    got = ict.depthwise(2, d, dev(dY), dev(X), 1, r * r).to_host()
+    same(got, oracle.depthwise(2, d, dY, X, 1, r * r), f"depthwise dW {geom}")
+    status_ok(ict)
