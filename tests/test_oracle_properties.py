@@ -89,3 +89,49 @@ def test_relu_keeps_exponents_and_sign(t, six):
     assert (z.mant >= 0).all() and (z.mant <= np.maximum(t.mant, 0)).all()
     if not six:
         assert (z.mant == np.maximum(t.mant, 0)).all()
+
+
+@SETTINGS
+@given(st.data())
+def test_sum_scaled_is_fit_of_weighted_exact_sums(data):
+    from fractions import Fraction
+
+    X = data.draw(ce_tensors())
+    Y = data.draw(ce_tensors(X.rows, X.cols))
+    xw = (data.draw(st.integers(-512, 512)), data.draw(st.integers(0, 24)))
+    yw = (data.draw(st.integers(-512, 512)), data.draw(st.integers(0, 24)))
+    g = (data.draw(st.integers(1, X.rows)), data.draw(st.integers(1, X.cols)))
+    Z = oracle.sum_scaled(X, xw, Y, yw, *g)
+    vx, vy = values(X), values(Y)
+    wx, wy = Fraction(xw[0]) * pow2(-xw[1]), Fraction(yw[0]) * pow2(-yw[1])
+    mant, exps = fit_matrix_brute([[wx * vx[i][j] + wy * vy[i][j] for j in range(X.cols)]
+                                   for i in range(X.rows)], *g)
+    assert Z.mant.tolist() == mant and Z.exp.tolist() == exps
+
+
+@SETTINGS
+@given(st.data())
+def test_avgpool_is_fit_of_exact_window_means(data):
+    from fractions import Fraction
+
+    K = data.draw(st.integers(1, 4))
+    n, hp, wp, c = data.draw(st.integers(1, 2)), data.draw(st.integers(1, 3)), data.draw(st.integers(1, 3)), 4
+    h, w = hp * K, wp * K
+    npix = n * h * w
+    g_in = data.draw(st.sampled_from([1, 2, 4]))  # channel groups spanning all pixels
+    m = np.array(data.draw(st.lists(st.integers(-127, 127), min_size=npix * c, max_size=npix * c)),
+                 np.int8).reshape(npix, c)
+    e = np.array([data.draw(st.sampled_from([E_ZERO] + list(range(-30, 20)))) for _ in range(c // g_in)],
+                 np.int8).reshape(1, -1)
+    for gj in range(e.shape[1]):  # E_ZERO groups hold zeros only
+        if e[0, gj] == E_ZERO:
+            m[:, gj * g_in:(gj + 1) * g_in] = 0
+    X = CE(m, e, npix, g_in)
+    og = (data.draw(st.integers(1, n * hp * wp)), data.draw(st.sampled_from([1, 2, 4])))
+    Y = oracle.avgpool_fwd(X, n, h, w, K, *og)
+    vx = values(X)
+    vals = [[sum((vx[(img * h + p * K + dy) * w + q * K + dx][ch] for dy in range(K) for dx in range(K)),
+                 Fraction(0)) / (K * K) for ch in range(c)]
+            for img in range(n) for p in range(hp) for q in range(wp)]
+    mant, exps = fit_matrix_brute(vals, *og)
+    assert Y.mant.tolist() == mant and Y.exp.tolist() == exps
