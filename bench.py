@@ -14,8 +14,8 @@ configurations, each a step of its own with its own unit:
   resnet18_conv3x3    3x3 conv fwd, bwd-data, bwd-weight on 128x56x56x64, TOPS
   resnet50_sgd        int-SGD update of a ResNet-50-sized parameter arena, GB/s
   single_linear       64x128 linear layer fwd+bwd+SGD, microseconds per step
-  resnet18_block_tail residual add, ReLU, ReLU backward and gradient merge on the
-                      ResNet-18 stage-1 activations, GB/s
+  resnet18_block_tail residual add fused with ReLU, ReLU backward and gradient merge on
+                      the ResNet-18 stage-1 activations, GB/s
 
 Usage:  python bench.py [--config C] [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 run under torchrun, one rank per GPU, each with its own batch of the
