@@ -1,16 +1,16 @@
 """Benchmark of the integer-only (C,e) training hot path on B200.
 
-Default step (--config vit_ti_mlp): one training step of a ViT-Ti-shaped MLP block
-through libict.so: fc1 forward (12608x192 . 192x768), integer GELU, fc2 forward
-(12608x768 . 768x192), fc2 backward-data and backward-weight, GELU backward, fc1
-backward-data and backward-weight, and the integer SGD-with-momentum update of both
-weight matrices (per-row velocity groups).  Synthetic seeded inputs of the ViT-Ti layer
-shapes (64 images x 197 tokens; "Memory-Efficient Integer-Only Training of Deep Neural
-Networks", Abstract and Table 9).
+Default step (--config vit_b_linear_trio): the six contractions of a ViT-B-shaped MLP
+block through libict.so on synthetic seeded inputs (12608 tokens = 64 images x 197
+tokens; d = 768, hidden 3072; (1, 64) exponent groups): fc1 forward (12608x768 .
+768x3072), fc2 forward (12608x3072 . 3072x768), both backward-data Products and both
+backward-weight Products ("Memory-Efficient Integer-Only Training of Deep Neural
+Networks", Table 6: linear layer = Product; Figure 1a: forward and backward in integer
+arithmetic).  metric: (C,e) GEMM TOPS over the step (356.95 GOP per step).
 
-metric: (C,e) GEMM TOPS over the step (6 contractions = 22.31 GOP per step).  The other
-configurations, each a step of its own with its own unit:
-  vit_b_linear_trio   the six ViT-B MLP contractions (357 GOP), TOPS
+The same run measures every other configuration as a side entry with its own value,
+roofline, end-to-end number and oracle baseline:
+  vit_ti_mlp          ViT-Ti MLP block training step (22.31 GOP), TOPS
   resnet18_conv3x3    3x3 conv fwd, bwd-data, bwd-weight on 128x56x56x64, TOPS
   resnet50_sgd        int-SGD update of a ResNet-50-sized parameter arena, GB/s
   single_linear       64x128 linear layer fwd+bwd+SGD, microseconds per step
@@ -60,7 +60,7 @@ CLASS_KERNELS = {
 
 def parse():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--config", default="vit_ti_mlp", choices=list(STEPS))
+    ap.add_argument("--config", default="vit_b_linear_trio", choices=list(STEPS))
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None, help="timed steps (default 20; 100 for resnet50_sgd)")
     ap.add_argument("--warmup", type=int, default=5)
@@ -603,32 +603,45 @@ def class_rate(name, c, peaks):
     return c["work_per_step"] / (c["ms_per_step"] * 1e-3) / 1e9, peaks["hbm"], "GB/s", "hbm"
 
 
-def kernel_source_digest():
-    """sha256 over the CUDA sources of libict.so (the kernels the counters describe)."""
+# CUDA sources of each kernel class's kernels: a committed DRAM-traffic figure is used
+# only while these files are unchanged since the counters were taken
+CLASS_SOURCES = {
+    "gemm": ["ict_gemm.cuh", "ict_device.cuh"],
+    "sgd": ["ict_elementwise.cuh", "ict_device.cuh"],
+    "align": ["ict_elementwise.cuh", "ict_device.cuh"],
+    "requant": ["ict_elementwise.cuh", "ict_device.cuh"],
+    "gelu": ["ict_elementwise.cuh", "ict_device.cuh"],
+    "estar": ["ict_elementwise.cuh", "ict_device.cuh"],
+    "other": ["ict_elementwise.cuh", "ict_device.cuh"],
+    "pointwise": ["ict_pointwise.cuh", "ict_elementwise.cuh", "ict_device.cuh"],
+}
+
+
+def class_source_digest(kernel_class):
+    """sha256 over the CUDA sources of one kernel class (file names and contents)."""
     import hashlib
 
     h = hashlib.sha256()
     src = os.path.join(ROOT, "integer_only_nn_02_b200", "csrc")
-    for name in sorted(os.listdir(src)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(src, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in CLASS_SOURCES[kernel_class]:
+        with open(os.path.join(src, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 
 def measured_traffic(config, kernel_class):
     """DRAM bytes per launch (read + write) of a kernel class in a configuration, from
-    the committed ncu summary, or None when the summary was taken on other kernel
-    sources or does not cover the class."""
+    the committed ncu summary, or None when the summary does not cover the class or was
+    taken on other sources of that class's kernels."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_sha256") != kernel_source_digest():
-        return None
     e = t.get("configs", {}).get(config, {}).get(kernel_class)
-    return None if e is None else e["dram_bytes_per_launch"]
+    if e is None or e.get("sources_sha256") != class_source_digest(kernel_class):
+        return None
+    return e["dram_bytes_per_launch"]
 
 
 def roofline(classes, peaks, config, gemm_bytes=0):
@@ -700,20 +713,75 @@ def side_int_mm(torch):
         return f"unavailable: {exc}"
 
 
-def side_measurements(ict, torch, peaks, flush, steps):
-    """The other configurations' step values (a few steps each), for context."""
+def measure(step, ict, torch, peaks, flush, config, steps, warmup, dist=None):
+    """Everything one configuration's line reports, for a constructed step: device time
+    of one graph replay per step (max over ranks), end-to-end time through host
+    buffers, host-launched time, the per-call and per-kernel-class breakdown, the
+    roofline of the dominant kernel class and the SM clocks during the timed region."""
+    step.run()
+    torch.cuda.synchronize()
+    code, raw = ict.ict_get_device_status()
+    if code != 0:
+        raise SystemExit(f"device status {code} ({raw:#x})")
+    graph = ict.StepGraph(step.run)
+    clocks = ClockSampler(torch.cuda.current_device())
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ms = time_graph(step, graph, steps, warmup, flush)
+    clk = clocks.stop()
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    eager_ms, _ = time_eager(step, steps, warmup, flush, backlogged=False)
+    _, per_call = time_eager(step, steps, warmup, flush, backlogged=True)
+    classes = time_classes(step, steps, flush)
+    e2e_ms, h2d, d2h = time_e2e(step, graph, steps, warmup)
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    code, raw = ict.ict_get_device_status()
+    if code != 0:
+        raise SystemExit(f"device status {code} ({raw:#x})")
+    world = dist.get_world_size() if dist else 1
+    agg = world if step.higher_is_better else 1  # rates add over independent replicas
+    out = {
+        "value": round(step.value_of(step.units, ms * 1e-3) * agg, 3), "unit": step.unit,
+        "ms_per_step": round(ms, 4),
+        "e2e": {"value": round(step.value_of(step.units, e2e_ms * 1e-3) * agg, 3), "unit": step.unit,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(graph.launches * steps),
+        "gpu_launches_per_step": graph.launches,
+        "launch": "one CUDA graph replay per step",
+        "eager_ms_per_step": round(eager_ms, 4),
+        "breakdown_ms": {n: round(float(v), 4) for (n, _), v in zip(step.calls, per_call)},
+        "kernel_classes": class_summary(classes, peaks),
+        "roofline": roofline(classes, peaks, config, step.gemm_bytes),
+        "clocks": clk,
+    }
+    del graph
+    return out
+
+
+def side_measurements(ict, torch, peaks, flush, steps, warmup, skip, with_cpu):
+    """The other configurations, each with its own value, roofline, e2e and oracle
+    baseline (a few steps each)."""
     out = {}
-    for name in ("vit_b_linear_trio", "resnet18_conv3x3", "resnet50_sgd", "single_linear"):
-        st = STEPS[name](ict, torch, 0)
-        graph = ict.StepGraph(st.run)
-        ms = time_graph(st, graph, steps, 3, flush)
-        _, per_call = time_eager(st, steps, 3, flush, backlogged=True)
-        classes = time_classes(st, steps, flush)
-        del graph
-        out[name] = {"value": round(st.value_of(st.units, ms * 1e-3), 2), "unit": st.unit,
-                     "ms_per_step": round(ms, 4),
-                     "breakdown_ms": {n: round(float(v), 4) for (n, _), v in zip(st.calls, per_call)},
-                     "kernel_classes": class_summary(classes, peaks)}
+    for name, cls in STEPS.items():
+        if name == skip:
+            continue
+        st = cls(ict, torch, 0)
+        k = 100 if name == "resnet50_sgd" else steps
+        entry = {"config": dict(cls.workload)}
+        entry.update(measure(st, ict, torch, peaks, flush, name, k, warmup))
+        entry["steps"] = k
+        if with_cpu:
+            entry["cpu_baseline"] = safe_cpu_baseline(cls)
+        out[name] = entry
         del st
         torch.cuda.empty_cache()
     out["torch_int_mm_8192_tops"] = side_int_mm(torch)
@@ -741,6 +809,13 @@ def cpu_baseline(step_cls):
     dt, units, sample = step_cls.oracle_step(step_cls.sample_arg)
     return {"value": step_cls.value_of(units, dt), "unit": step_cls.unit, "cores": oracle.num_threads(),
             "kind": "oracle", "sample": sample, "seconds": round(dt, 3)}
+
+
+def safe_cpu_baseline(step_cls):
+    try:
+        return cpu_baseline(step_cls)
+    except Exception as exc:  # pragma: no cover
+        return {"value": None, "unit": step_cls.unit, "cores": None, "kind": "oracle", "sample": f"failed: {exc}"}
 
 
 def run_reference(args):
@@ -787,69 +862,21 @@ def main():
     step_cls = STEPS[args.config]
     step = step_cls(ict, torch, rank)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    step.run()
-    torch.cuda.synchronize()
-    code, raw = ict.ict_get_device_status()
-    if code != 0:
-        raise SystemExit(f"device status {code} ({raw:#x})")
-
-    graph = ict.StepGraph(step.run)
-    clocks = ClockSampler(torch.cuda.current_device())
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    ms = time_graph(step, graph, args.steps, args.warmup, flush)
-    clk = clocks.stop()
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        dist.barrier()
-    eager_ms, _ = time_eager(step, args.steps, args.warmup, flush, backlogged=False)
-    _, per_call = time_eager(step, args.steps, args.warmup, flush, backlogged=True)
-    classes = time_classes(step, args.steps, flush)
-    e2e_ms, h2d, d2h = time_e2e(step, graph, args.steps, args.warmup)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    code, raw = ict.ict_get_device_status()
-    if code != 0:
-        raise SystemExit(f"device status {code} ({raw:#x})")
-
-    agg = world if step.higher_is_better else 1  # rates add over independent replicas
     line = base_line(args, step_cls, world)
-    line.update({
-        "value": round(step.value_of(step.units, ms * 1e-3) * agg, 3), "ms_per_step": round(ms, 4),
-        "e2e": {"value": round(step.value_of(step.units, e2e_ms * 1e-3) * agg, 3), "unit": step.unit,
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": int(graph.launches * args.steps),
-        "gpu_launches_per_step": graph.launches,
-        "launch": "one CUDA graph replay per step",
-        "eager_ms_per_step": round(eager_ms, 4),
-        "breakdown_ms": {n: round(float(v), 4) for (n, _), v in zip(step.calls, per_call)},
-        "kernel_classes": class_summary(classes, peaks),
-        "roofline": roofline(classes, peaks, args.config, step.gemm_bytes),
-        "clocks": clk,
-    })
+    line.update(measure(step, ict, torch, peaks, flush, args.config, args.steps, args.warmup, dist))
     if world > 1 and getattr(step, "exchanged_bytes", 0):
         line["allreduce_bytes_per_rank_per_step"] = int(step.exchanged_bytes)
-    if rank == 0 and world == 1 and not args.no_side and args.config == "vit_ti_mlp":
-        del graph, step
-        torch.cuda.empty_cache()
-        line["side"] = side_measurements(ict, torch, peaks, flush, max(5, args.steps // 2))
+    del step
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_side:
+        line["side"] = side_measurements(ict, torch, peaks, flush, max(5, args.steps // 2), args.warmup,
+                                         args.config, not args.no_cpu)
     if rank == 0:
         if not args.no_cpu and world == 1:
-            try:
-                line["cpu_baseline"] = cpu_baseline(step_cls)
-            except Exception as exc:  # pragma: no cover
-                line["cpu_baseline"] = {"value": None, "unit": step_cls.unit, "cores": None, "kind": "oracle",
-                                        "sample": f"failed: {exc}"}
+            line["cpu_baseline"] = safe_cpu_baseline(step_cls)
         print(json.dumps(line))
     if dist:
-        graph = None  # a CUDA graph holding NCCL calls goes before its process group
-        torch.cuda.synchronize()
+        torch.cuda.synchronize()  # every CUDA graph holding NCCL calls is gone by now
         dist.barrier()
         dist.destroy_process_group()
 

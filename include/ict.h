@@ -240,7 +240,10 @@ int32_t ict_linear_bwd_weight_partial(const ict_tensor *dY, const ict_tensor *X,
  *     ICT_NOALLOC_SCRATCH_BYTES are rejected with ICT_ERR_WORKSPACE before any launch.
  *   - It never calls cudaMalloc, cudaFree or any allocating routine.
  *   - The first call on a device looks up that device's copy of the array (with the
- *     device current); make that first call before any stream capture.
+ *     device current); make that first call before any stream capture.  The address is
+ *     kept with the CUDA context it belongs to: after a device reset (cudaDeviceReset,
+ *     or a framework that resets the device) the next call looks it up again, and is
+ *     then again a first call.
  *   - All calls share the one array and it keeps the last call's contents: calls that
  *     can overlap on the GPU (other streams, other threads) race on it and must be
  *     serialised by the caller. */
@@ -252,14 +255,19 @@ int32_t ict_linear_fwd_noalloc(const ict_tensor *X, const ict_tensor *W, ict_ten
 /*   dir FWD         a = X  [n*h*w][c], b = W [k][r*s*c] -> out = Y  [n*p*q][k]        */
 /*   dir BWD_DATA    a = dY [n*p*q][k], b = W [k][r*s*c] -> out = dX [n*h*w][c]        */
 /*   dir BWD_WEIGHT  a = dY [n*p*q][k], b = X [n*h*w][c] -> out = dW [k][r*s*c]        */
-/* Activation exponents must be uniform over pixels (g_rows >= rows); activation       */
-/* output groups likewise (g_rows >= rows, g_cols a multiple of 16); dW groups are     */
-/* per row.  The library supports square odd filters with "same" padding and stride 1 */
-/* (r = s, pad = (r - 1) / 2: 1x1, 3x3, 5x5, 7x7, ...), c and k multiples of 64 up to   */
-/* 256, w <= 128.  ict_conv_workspace() is an upper bound for the direction; for FWD   */
-/* and BWD_DATA it includes int32 sums of the whole output (4 bytes per element), used  */
-/* when the output groups span all pixels: one Product pass writes the sums and every  */
-/* group's largest need, a streaming pass rounds them.                                 */
+/* Activation exponents must be uniform over pixels (g_rows >= rows).  Output groups   */
+/* of FWD / BWD_DATA are pixel-local (g_rows = 1) or span all pixels (g_rows >= rows);  */
+/* their width g_cols is a multiple of 32 that divides the output tile width (64, 128,  */
+/* 192 or 256 channels, the smallest that holds out_c, else 256), or covers all out_c <= */
+/* 256 channels.  dW groups are per row.  The library supports square odd filters with   */
+/* "same" padding and stride 1 (r = s, pad = (r - 1) / 2: 1x1, 3x3, 5x5, 7x7, ...), c    */
+/* and k multiples of 64 up to 2048, w <= 128.  ict_conv_workspace() is an upper bound  */
+/* for the direction.  For FWD and BWD_DATA it includes, for output groups spanning all */
+/* pixels, int16 sums of the whole output (2 bytes per element) and one int32 need per  */
+/* output tile and group column: the Product pass rounds each exact sum to odd at an    */
+/* exponent 7 below its tile's largest need() (the int16 fits by construction) and      */
+/* raises every group's largest need; a streaming pass rounds to nearest even at the    */
+/* group exponent, a shift of at least 7 bits, which equals RNE of the exact sum.       */
 size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d);
 int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_tensor *a,
                                const ict_tensor *b, ict_tensor *out, void *ws,

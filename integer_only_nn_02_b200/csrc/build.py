@@ -9,8 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 LIB = os.path.join(PKG, "libict.so")
+INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 SOURCES = ["ict_api.cu"]
-HEADERS = ["ict_device.cuh", "ict_elementwise.cuh", "ict_gemm.cuh", "../../include/ict.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -20,12 +20,19 @@ FLAGS = [
 ]
 
 
+def dependencies() -> list:
+    """Every file the library is built from: the sources and headers in this directory,
+    the public headers, and this script."""
+    deps = [os.path.join(HERE, f) for f in sorted(os.listdir(HERE)) if f.endswith((".cu", ".cuh", ".h"))]
+    deps += [os.path.join(INCLUDE, f) for f in sorted(os.listdir(INCLUDE)) if f.endswith(".h")]
+    return deps + [os.path.abspath(__file__)]
+
+
 def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = SOURCES + HEADERS + [os.path.basename(__file__)]
-    return any(os.path.getmtime(os.path.join(HERE, f)) > t for f in deps)
+    return any(os.path.getmtime(f) > t for f in dependencies())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

@@ -31,6 +31,8 @@ std::mutex g_mu;
 DeviceInfo g_dev[64];
 uint64_t g_wait_ns = 2000000000ull;  // bound of every mbarrier wait inside a kernel
 const uint64_t kDrainNs = 1000000000ull;
+// largest channel count (contracted or produced) of the implicit-GEMM convolution
+constexpr int kConvMaxChannels = 2048;
 
 int device_info(int *sms) {
     int dev = 0;
@@ -379,7 +381,14 @@ int launch_requant_rows(RequantArgs a, cudaStream_t s) {
     const bool vec = !a.v64 && a.cs == 1 && G >= 64 && G <= 4096 && G % 4 == 0 && a.cols % 4 == 0 &&
                      a.ld % 4 == 0 && a.out_ld % 4 == 0 && a.split_stride % 4 == 0 &&
                      (reinterpret_cast<uintptr_t>(a.v32) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 3) == 0;
-    if (vec) {
+    const bool warp = vec && a.nsplit == 1 && G <= 1024 && (!a.col_exp || a.col_div == 1) &&
+                      (reinterpret_cast<uintptr_t>(a.col_exp) & 3) == 0;
+    if (warp) {
+        const unsigned b = (unsigned)cdiv64(groups, 8);
+        if (G <= 256) requant_warp_kernel<2><<<b, 256, 0, s>>>(a);
+        else if (G <= 512) requant_warp_kernel<4><<<b, 256, 0, s>>>(a);
+        else requant_warp_kernel<8><<<b, 256, 0, s>>>(a);
+    } else if (vec) {
         const unsigned b = (unsigned)groups;
         const bool wide = a.nsplit > 1;
 #define ICT_RQ_VEC(T_, V_)                                                      \
@@ -439,20 +448,24 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
         return launch_status();
     };
     constexpr int kB2 = GemmSmem<BN, BK, ST, 2>::kBytes;
-    if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, true>, 2, kB2);
+    if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_I32>, 2, kB2);
     if constexpr (LOAD == LOAD_CONV_WGRAD) {
         return ICT_ERR_LAYOUT;  // backward-weight writes int32 only
     } else {
+        if constexpr (LOAD == LOAD_CONV) {
+            if (p.epi == EPI_RO16) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_RO16>, 2, kB2);
+        }
+        if (p.epi != EPI_FIT_ROW) return ICT_ERR_LAYOUT;
         const int gt = p.G >= p.N ? BN : p.G;  // group width inside a tile
         if constexpr (LOAD == LOAD_2D && BN <= 128) {
             if (p.nwg == 4) {  // four epilogue warpgroups, four accumulators
                 constexpr int kB4 = GemmSmem<BN, BK, ST, 4>::kBytes;
-                if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, true, 4>, 4, kB4);
-                return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, false, 4>, 4, kB4);
+                if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, true, 4>, 4, kB4);
+                return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, false, 4>, 4, kB4);
             }
         }
-        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, true>, 2, kB2);
-        return run(gemm_ce_kernel<BN, BK, ST, LOAD, false, false>, 2, kB2);
+        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, true>, 2, kB2);
+        return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, false>, 2, kB2);
     }
 }
 
@@ -463,7 +476,7 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     // group straddles the halves
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
-    if (p.nwg != 4 || p.epi == EPI_I32) p.nwg = 2;
+    if (p.nwg != 4 || p.epi != EPI_FIT_ROW) p.nwg = 2;
     p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0));
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
     if (bn == BN_ && bk == BK_ && load == LOAD_) \
@@ -867,8 +880,10 @@ struct ConvPlan {
     bool global_groups;
     int32_t *gmax;
     int n_gcols;
-    int32_t *acc32;  // int32 sums of the one-pass global-group plan (else NULL)
-    int64_t acc_ld;
+    // groups spanning all pixels: int16 sums rounded to odd at a per-tile exponent
+    int16_t *ws16;
+    int64_t ws16_ld;
+    int32_t *tile_need;  // [m tiles][n_gcols]
 };
 
 int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_tensor *b,
@@ -880,7 +895,8 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
         d->stride < 1 || d->pad < 0)
         return ICT_ERR_INVALID_ARG;
     if (d->stride != 1 || d->r != d->s || 2 * d->pad != d->r - 1) return ICT_ERR_LAYOUT;
-    if (d->c % 64 || d->k % 64 || d->c > 256 || d->k > 256 || d->w > 128) return ICT_ERR_LAYOUT;
+    if (d->c % 64 || d->k % 64 || d->c > kConvMaxChannels || d->k > kConvMaxChannels || d->w > 128)
+        return ICT_ERR_LAYOUT;
     const int64_t npix = (int64_t)d->n * d->h * d->w, RS = (int64_t)d->r * d->s;
     if (dir != ICT_CONV_FWD && dir != ICT_CONV_BWD_DATA) return ICT_ERR_INVALID_ARG;
     const int64_t act_c = dir == ICT_CONV_FWD ? d->c : d->k;  // contracted channels
@@ -957,12 +973,15 @@ int plan_conv(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_te
     }
     cp->n_gcols = (int)n_grp_cols(out);
     cp->gmax = cp->global_groups ? (int32_t *)ws.take((size_t)cp->n_gcols * 4) : nullptr;
-    // groups spanning all pixels: one Product pass writes int32 sums and the groups'
-    // largest need; a streaming pass rounds (needs G a multiple of 16, at most 8 groups)
-    cp->acc32 = nullptr;
-    if (cp->global_groups && cp->n_gcols <= 8 && (G >= out_c || G % 16 == 0) && out_c % 16 == 0) {
-        cp->acc_ld = round_up(out_c, 32);
-        cp->acc32 = (int32_t *)ws.take((size_t)npix * cp->acc_ld * 4);
+    // groups spanning all pixels: one Product pass writes int16 sums rounded to odd at a
+    // per-tile exponent, every tile's need and every group's largest need; a streaming
+    // pass rounds them with the groups' exponents
+    cp->ws16 = nullptr;
+    cp->tile_need = nullptr;
+    if (cp->global_groups) {
+        cp->ws16_ld = round_up(out_c, 32);
+        cp->ws16 = (int16_t *)ws.take((size_t)npix * cp->ws16_ld * 2);
+        cp->tile_need = (int32_t *)ws.take((size_t)d->n * cp->tiles_per_img * cp->n_gcols * 4);
     }
     return ICT_OK;
 }
@@ -1041,41 +1060,34 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         }
         counted(1);
     }
-    if (cp.acc32) {
-        p.epi = EPI_I32;
-        p.ws32 = cp.acc32;
-        p.ws_ld = cp.acc_ld;
-        p.ws_split_stride = 0;
-        if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
-        if (!(phase & 2)) return ICT_OK;
-        GlobalRequantArgs r;
-        r.v = cp.acc32;
-        r.rows = cp.out_rows;
-        r.cols = cp.out_cols;
-        r.ld = cp.acc_ld;
-        r.eA = cp.eA;
-        r.eA_div = cp.eA_div;
-        r.eB = cp.eB;
-        r.eB_div = cp.eB_div;
-        r.gmax = cp.gmax;
-        r.G = p.G;
-        r.ngc = cp.n_gcols;
-        r.out = out->mant;
-        r.out_ld = out->ld;
-        r.out_exp = out->exp;
-        r.act = act;
-        const int64_t n = cp.out_rows * (cp.out_cols / 16);
-        KTimer kt(s, KC_REQUANT, 5.0 * (double)cp.out_rows * (double)cp.out_cols);
-        requant_global_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(r);
-        counted(1);
-        return launch_status();
-    }
-    p.epi = EPI_NEED_GLOBAL;  // the first pass is recompute: its work is not counted again
-    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, 0.0))) return st;
+    p.epi = EPI_RO16;
+    p.ws16 = cp.ws16;
+    p.ws16_ld = cp.ws16_ld;
+    p.tile_need = cp.tile_need;
+    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
     if (!(phase & 2)) return ICT_OK;
-    p.epi = EPI_FIT_GLOBAL;
-    if ((st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
-    return act == ACT_NONE ? ICT_OK : launch_clip(out, nullptr, act == ACT_RELU6, const_cast<ict_tensor *>(out), s);
+    Ro16RoundArgs r;
+    r.v = cp.ws16;
+    r.rows = cp.out_rows;
+    r.cols = cp.out_cols;
+    r.ld = cp.ws16_ld;
+    r.tile_need = cp.tile_need;
+    r.gmax = cp.gmax;
+    r.cv_W = d->w;
+    r.cv_P = d->h;
+    r.cv_rows = cp.rows_per_tile;
+    r.cv_tiles_per_img = cp.tiles_per_img;
+    r.G = p.G;
+    r.ngc = cp.n_gcols;
+    r.out = out->mant;
+    r.out_ld = out->ld;
+    r.out_exp = out->exp;
+    r.act = act;
+    const int64_t n = cp.out_rows * (cp.out_cols / 16);
+    KTimer kt(s, KC_REQUANT, 3.0 * (double)cp.out_rows * (double)cp.out_cols);
+    ro16_round_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(r);
+    counted(1);
+    return launch_status();
 }
 
 // ---- convolution backward-weight: dW[k][(r,s,c)] = sum over output pixels of
@@ -1316,21 +1328,47 @@ int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
 // ---- allocation-free forward Product: fixed scratch inside the library
 
 // One array per device that loads the library; host code must not pass its name to a
-// kernel (on the host it is only a stand-in), so its device address is looked up once
-// per device with cudaGetSymbolAddress.
+// kernel (on the host it is only a stand-in), so its device address is looked up with
+// cudaGetSymbolAddress, with the device current, and kept per device together with the
+// context it belongs to: after a device reset the module is loaded again (possibly at
+// another address) in a new context, and the next call looks the address up again.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[ICT_NOALLOC_SCRATCH_BYTES];
-void *g_noalloc_addr[64];
+struct NoallocSlot {
+    void *ctx;
+    void *addr;
+};
+NoallocSlot g_noalloc_slot[64];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (CtxGetCurrentFn)ptr;
+    }
+    return fn;
+}
 
 int noalloc_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ICT_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_noalloc_addr[dev]) {
-        void *p = nullptr;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return ICT_ERR_CUDA;
+    CUcontext ctx = nullptr;  // NULL until the runtime has made a context current on this thread
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return ICT_ERR_CUDA;
+    NoallocSlot &slot = g_noalloc_slot[dev];
+    if (!ctx || !slot.addr || slot.ctx != (void *)ctx) {
+        void *p = nullptr;  // the lookup makes the device's primary context current
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ICT_ERR_CUDA;
-        g_noalloc_addr[dev] = p;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return ICT_ERR_CUDA;
+        slot.ctx = (void *)ctx;
+        slot.addr = p;
     }
-    *out = g_noalloc_addr[dev];
+    *out = slot.addr;
     return ICT_OK;
 }
 
@@ -1691,8 +1729,11 @@ size_t ict_conv_workspace(int32_t dir, const ict_conv_desc *d) {
     w.take((size_t)std::max<int64_t>(d->k * RS * d->c, d->c * round_up(RS * d->k, 16)));
     w.take((size_t)std::max(d->k, d->c));
     w.take((size_t)std::max(d->k, d->c) * 4);
+    // groups spanning all pixels: int16 sums and the per-tile needs
     const int64_t out_c = dir == ICT_CONV_FWD ? d->k : d->c;
-    w.take((size_t)npix * round_up(out_c, 32) * 4);  // int32 sums for groups spanning all pixels
+    w.take((size_t)npix * round_up(out_c, 32) * 2);
+    const int64_t rows_per_tile = std::max(1, std::min(128 / std::max(d->w, 1), d->h));
+    w.take((size_t)d->n * cdiv64(d->h, rows_per_tile) * cdiv64(out_c, 16) * 4);
     return w.used;
 }
 

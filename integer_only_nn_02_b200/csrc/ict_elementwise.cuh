@@ -704,11 +704,55 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
     if (threadIdx.x == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
 }
 
-// FIT into groups that span all rows (a block of G columns over every row): the group
-// exponents are final in gmax (largest need over the whole group, from the Product's
-// epilogue), so every element is rounded independently.  16 columns per thread: four
-// 16-byte loads of int32 partial sums, one 16-byte store of mantissas.  Requires cols,
-// ld and out_ld multiples of 16.
+// FIT of row-local groups of one slice of int32 sums, one warp per group of at most
+// 128 V columns: each lane holds V 16-byte vectors (4 columns each), all loaded before
+// anything else, and the group's largest need is a warp reduction, so no block barrier
+// sits between the loads and the stores.  Requires cs = 1, col_div = 1 (or no column
+// exponents), G, cols, ld and out_ld multiples of 4.
+template <int V>
+__global__ void __launch_bounds__(256) requant_warp_kernel(const __grid_constant__ RequantArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gidx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (gidx >= a.rows * a.ngc) return;
+    const int64_t i = idiv(gidx, a.ngc), g = gidx - i * a.ngc;
+    const int64_t j0 = g * a.G;
+    const int glen = (int)min((int64_t)a.G, a.cols - j0);
+    const int re = a.base + (a.row_exp ? a.row_exp[idiv(i, a.row_div)] : 0);
+    int4 x[V];
+    uint32_t ce[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        const int jj = 4 * (lane + 32 * k);
+        x[k] = make_int4(0, 0, 0, 0);
+        ce[k] = 0;
+        if (jj < glen) {
+            x[k] = *reinterpret_cast<const int4 *>(a.v32 + i * a.ld + j0 + jj);
+            if (a.col_exp) ce[k] = *reinterpret_cast<const uint32_t *>(a.col_exp + j0 + jj);
+        }
+    }
+    int emax = kNoExp;
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        const int v[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            if (v[t]) emax = max(emax, re + sx8(ce[k], t) + need_off32((uint32_t)(v[t] < 0 ? -v[t] : v[t])));
+    }
+    const int e = finalize_exp(warp_max(emax));
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        const int jj = 4 * (lane + 32 * k);
+        if (jj < glen) {
+            const int v[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+            int o[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) o[t] = requant32(v[t], re + sx8(ce[k], t), e);
+            *reinterpret_cast<uint32_t *>(a.out + i * a.out_ld + j0 + jj) = pack4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    if (lane == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+}
+
 // ------------------------------------------------------------------ fused activations
 
 // ReLU6's clip bound in a group at exponent e, min(6 >> e, q_max) (Table 7): the integer
@@ -734,14 +778,22 @@ __device__ __forceinline__ uint4 apply_act(uint4 v, int act, int e) {
     return make_uint4(relu_word(v.x, hi), relu_word(v.y, hi), relu_word(v.z, hi), relu_word(v.w, hi));
 }
 
-struct GlobalRequantArgs {
-    const int32_t *v;
+// FIT into groups that span all rows of a convolution output, from the Product's int16
+// sums: t[i][j] is the exact sum rounded to odd at exponent e1 = tile_need - 7 of the
+// output tile holding pixel i (tile_need[tile][group], kNoExp when the tile's group is
+// all zero), and the group exponent e = finalize(gmax[group]) >= tile_need, so the
+// mantissa is RNE(t * 2^(e1 - e)), a right shift of at least 7 bits, which equals RNE of
+// the exact sum (Boldo and Melquiond, "Emulation of FMA and correctly rounded sums:
+// proved algorithms using rounding to odd", IEEE Trans. Computers 57(4), 2008).  Output
+// tiles are cv_rows image rows of width cv_W (cv_tiles_per_img per image of cv_P rows).
+// 16 columns per thread: two 16-byte loads, one 16-byte store; cols, ld and out_ld
+// multiples of 16, G a multiple of 16.
+struct Ro16RoundArgs {
+    const int16_t *v;
     int64_t rows, cols, ld;
-    const int8_t *eA;
-    int eA_div;
-    const int8_t *eB;
-    int eB_div;
-    const int32_t *gmax;
+    const int32_t *tile_need;  // [tiles][ngc]
+    const int32_t *gmax;       // [ngc]
+    int cv_W, cv_P, cv_rows, cv_tiles_per_img;
     int G;
     int64_t ngc;
     int8_t *out;
@@ -749,41 +801,49 @@ struct GlobalRequantArgs {
     int8_t *out_exp;
     int act;  // fused activation (ACT_*)
 };
-__global__ void __launch_bounds__(256) requant_global_kernel(GlobalRequantArgs a) {
+__global__ void __launch_bounds__(256) ro16_round_kernel(const __grid_constant__ Ro16RoundArgs a) {
     const int64_t cv = a.cols / 16;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= a.rows * cv) return;
     const int64_t i = idiv(t, cv), j0 = (t - i * cv) * 16;
-    const int ea = a.eA[idiv(i, a.eA_div)];
     const int64_t g = idiv(j0, a.G);  // 16 | G, so one group per thread
     const int e = finalize_exp(a.gmax[g]);
     if (i == 0 && j0 == g * a.G) a.out_exp[g] = (int8_t)e;
-    const int32_t *src = a.v + i * a.ld + j0;
-    int eb[16];
-    if (a.eB_div == 1 && (reinterpret_cast<uintptr_t>(a.eB) & 15) == 0) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(a.eB + j0);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int q = 0; q < 16; ++q) eb[q] = sx8(ww[q >> 2], q & 3);
-    } else {
-#pragma unroll
-        for (int q = 0; q < 16; ++q) eb[q] = a.eB[idiv(j0 + q, a.eB_div)];
-    }
-    // element exponent ea + eb[q]; mantissa = RNE(x * 2^-(e - ea - eb[q])): a right shift
-    // of at least 2 by high-half multiplies, anything else by the general routine
-    auto rq = [&](int32_t x, int q) {
-        const int sft = e - ea - eb[q];
-        if (sft >= 2 && sft < 32) {
-            const int m = 1 << (32 - sft), bias = (1 << (sft - 1)) - 1;
-            return __mulhi(x + bias + (__mulhi(x, m) & 1), m);
-        }
-        return requant32(x, ea + eb[q], e);
-    };
+    // output tile of pixel i
+    const int64_t prow = idiv(i, a.cv_W);               // image row over the whole batch
+    const int64_t img = idiv(prow, a.cv_P), h = prow - img * a.cv_P;
+    const int64_t tile = img * a.cv_tiles_per_img + idiv(h, a.cv_rows);
+    const int tn = a.tile_need[tile * a.ngc + g];
+    const int64_t s64 = (int64_t)e - ((int64_t)tn - 7);
+    const int s = (int)(s64 > 40 ? 40 : s64);
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.v + i * a.ld + j0);
+    const uint4 x0 = src[0], x1 = src[1];
+    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
     uint32_t o[4];
+    if (s >= 2 && s < 32) {
+        const int m = 1 << (32 - s), bias = (1 << (s - 1)) - 1;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int4 x = *reinterpret_cast<const int4 *>(src + 4 * q);
-        o[q] = pack4(rq(x.x, 4 * q), rq(x.y, 4 * q + 1), rq(x.z, 4 * q + 2), rq(x.w, 4 * q + 3));
+        for (int q = 0; q < 4; ++q) {
+            int y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int x = (int)(int16_t)(xw[2 * q + (k >> 1)] >> (16 * (k & 1)));
+                y[k] = __mulhi(x + bias + (__mulhi(x, m) & 1), m);
+            }
+            o[q] = pack4(y[0], y[1], y[2], y[3]);
+        }
+    } else if (s >= 32) {
+        o[0] = o[1] = o[2] = o[3] = 0u;  // |t| < 2^15: the value is below half a unit
+    } else {
+        // e below the tile's need only after an exponent overflow (status raised)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            int y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                y[k] = requant32((int)(int16_t)(xw[2 * q + (k >> 1)] >> (16 * (k & 1))), tn - 7, e);
+            o[q] = pack4(y[0], y[1], y[2], y[3]);
+        }
     }
     *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = apply_act(make_uint4(o[0], o[1], o[2], o[3]), a.act, e);
 }

@@ -32,10 +32,10 @@
 namespace ict {
 
 enum EpiMode : int {
-    EPI_FIT_ROW = 0,      // row-local groups (1, G) inside one tile -> int8 + exps
-    EPI_I32 = 1,          // raw int32 partials to a workspace slice (split-K / wide groups)
-    EPI_NEED_GLOBAL = 2,  // pass 1 of groups spanning all rows: max need per column group
-    EPI_FIT_GLOBAL = 3,   // pass 2: requantise with the global group exponents
+    EPI_FIT_ROW = 0,  // row-local groups (1, G) inside one tile -> int8 + exps
+    EPI_I32 = 1,      // raw int32 partials to a workspace slice (split-K)
+    EPI_RO16 = 2,     // groups spanning all rows: int16 sums rounded to odd at a per-tile
+                      // exponent, the tile's need and the group's running max need
 };
 // LOAD_2D         A, B: K-major rows from 2-D tensor maps (linear layers)
 // LOAD_CONV       A: one filter tap of NHWC activations per K block (4-D box), B: K-major
@@ -61,7 +61,14 @@ struct GemmParams {
     int64_t out_exp_ld;
     int32_t *ws32;
     int64_t ws_ld, ws_split_stride;
-    int32_t *gmax;  // [column groups] running max of need() (global groups)
+    // EPI_RO16 (output groups spanning all rows): t = RO(acc * 2^(eA + eB - e1)) as int16
+    // into ws16[row][ws16_ld], e1 = tile_need - 7 with tile_need the largest need() of the
+    // group's elements in the tile (tile_need[m tile][group column], kNoExp when all are
+    // zero), and the running max need of every group column in gmax
+    int16_t *ws16;
+    int64_t ws16_ld;
+    int32_t *tile_need;
+    int32_t *gmax;
     // implicit-GEMM convolution: output tile = cv_rows image rows of width cv_W
     int cv_W, cv_P, cv_rows, cv_tiles_per_img, cv_cblk, cv_S, cv_pad, cv_sign;
     // conv: every K block of the weight operand held in shared memory for the whole kernel
@@ -90,8 +97,8 @@ struct GemmSmem {
     static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 2 * NWG + 2) * 8 + 15) / 16 * 16;
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
-    static constexpr int kOffGacc = kOffCol + NWG * kColInts * 4;   // [8] group needs (I32 + global groups)
-    static constexpr int kBytes = kOffGacc + 8 * 4 + 1024;           // + alignment slack
+    static constexpr int kOffRed = kOffCol + NWG * kColInts * 4;  // [NWG][8 groups][4 warps] row-need maxima
+    static constexpr int kBytes = kOffRed + NWG * 32 * 4 + 1024;    // + alignment slack
     static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
                   "column tables are read as int4");
     static_assert(kABytes % 1024 == 0 && kBBytes % 512 == 0 && kOffB % 1024 == 0 && kABytes / 2 <= 16383 * 16,
@@ -118,7 +125,7 @@ __device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {
 // bit and the byte packing to the ALU pipe; TMEM is read once.
 template <bool MUL>  // MUL = false: every column of the group has the same exponent
 __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
-                                           bool valid, int ea, int64_t grow, int ncol, int gcol, int et) {
+                                           bool valid, int ea, int64_t grow, int ncol, int gcol) {
     uint32_t v[32];
     tmem_ld32(taddr, v);
     tmem_ld_wait();
@@ -139,12 +146,7 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     const int h = max(max(hi[0], hi[1]), max(hi[2], hi[3])), l = min(min(lo[0], lo[1]), min(lo[2], lo[3]));
     const int amax = valid ? max(h, -l) : 0;
     const int need = amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp;
-    if (p.epi == EPI_NEED_GLOBAL) {
-        const int m = warp_max(need);
-        if ((threadIdx.x & 31) == 0 && m > kNoExp && ncol < p.N) atomicMax(p.gmax + gcol, m);
-        return;
-    }
-    const int e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : need);
+    const int e = finalize_exp(need);
     // mantissa = RNE(y * 2^-S), S = e - ea - gm uniform over the row's group
     const int S = (e == kEZero) ? 0 : e - ea - gm;
     if (__any_sync(0xffffffffu, valid && S < 0)) {
@@ -172,10 +174,7 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
             v[q] = (uint32_t)((y + ((y >> 1) & 1)) >> 1);
         }
     }
-    if (ncol < p.N) {
-        if (p.epi == EPI_FIT_ROW && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
-        if (p.epi == EPI_FIT_GLOBAL && et == 0) p.out_exp[gcol] = (int8_t)e;
-    }
+    if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
     if (valid) {
         int8_t *dst = p.out + grow * p.out_ld + ncol;
 #pragma unroll
@@ -189,18 +188,20 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     }
 }
 
-// I32 (compile time): the kernel writes int32 partial sums (EPI_I32) and contains no FIT
-// code, and the FIT kernels contain no int32 path, so that each keeps a small code
-// footprint in the instruction cache.
+// OUTK (compile time, an EpiMode): which epilogue is compiled in -- the row-local FIT
+// (EPI_FIT_ROW), raw int32 partial sums (EPI_I32), or the int16 round-to-odd sums of
+// groups spanning all rows (EPI_RO16) -- so that each kernel keeps a small code footprint
+// in the instruction cache.
 // G32 (compile time, FIT kernels): output groups are 32 columns wide, so only the
 // 32-column fast path and the exact path are compiled in.
 // NWG (compile time): epilogue warpgroups, each owning one TMEM accumulator (2 or 4).
-template <int BN, int BK, int STAGES, int LOAD, bool I32, bool G32 = false, int NWG = 2>
+template <int BN, int BK, int STAGES, int LOAD, int OUTK, bool G32 = false, int NWG = 2>
 __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
     using L = GemmSmem<BN, BK, STAGES, NWG>;
     constexpr int NACC = NWG;
+    constexpr bool I32 = OUTK == EPI_I32, RO16 = OUTK == EPI_RO16;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(BK == 128 || BK == 64 || (BK == 256 && LOAD == LOAD_CONV_WGRAD), "BK");
     extern __shared__ uint8_t smem_raw[];
@@ -214,11 +215,10 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     const uint32_t bar_bres = bar_drain + 8;                // [1] resident weight operand landed
     volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
     int *sCol = (int *)(smem + L::kOffCol);  // per epilogue warpgroup column tables
-    int *gacc = (int *)(smem + L::kOffGacc);  // running max need per output group (I32 with gmax)
+    int *sRed = (int *)(smem + L::kOffRed);  // per warpgroup: [group][warp] row-need maxima (RO16)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    if (threadIdx.x < 8) gacc[threadIdx.x] = kNoExp;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
@@ -408,10 +408,11 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         // The exponents a tile needs (two column exponents and one row exponent per
         // thread) are loaded one tile ahead, so that their latency hides behind the
         // previous tile's epilogue.
-        int pf_e0 = kEZero, pf_e1 = kEZero, pf_ea = 0, pf_split = 0, pf_vr = 0, pf_n0 = 0;
+        int pf_e0 = kEZero, pf_e1 = kEZero, pf_ea = 0, pf_split = 0, pf_vr = 0, pf_n0 = 0, pf_mt = 0;
         int64_t pf_rb = 0;
         auto prefetch = [&](bool have) {
             if (!have) return;
+            pf_mt = c_mt;
             if (LOAD == LOAD_CONV) {
                 const int img = c_mt / p.cv_tiles_per_img;
                 const int h0 = (c_mt % p.cv_tiles_per_img) * p.cv_rows;
@@ -440,7 +441,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         for (int u = u0; u < p.num_units; u += u_step, it += it_step) {
             const int acc = it % NACC;
             const int64_t row_base = pf_rb;
-            const int valid_rows = pf_vr, n0 = pf_n0, split = pf_split;
+            const int valid_rows = pf_vr, n0 = pf_n0, split = pf_split, mt = pf_mt;
             const int e0 = pf_e0, e1 = pf_e1, ea_pf = pf_ea;
             prefetch(u + u_step < p.num_units);
             // column tables of this tile (independent of the accumulator: built before waiting)
@@ -500,19 +501,92 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                                 *reinterpret_cast<uint4 *>(dst + c + 4 * q) =
                                     make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
-                    if (p.gmax) {
-                        // groups spanning all rows: the largest need of each 32 columns,
-                        // exponent eA[m] + eB[n] per element, kept per CTA
-                        int emax = kNoExp;
-                        if (valid) {
-#pragma unroll 8
-                            for (int q = 0; q < 32; ++q) {
-                                const int32_t x = (int32_t)v[q];
-                                if (x) emax = max(emax, ea + colE[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
+                }
+            } else if constexpr (RO16) {
+                // Groups spanning all rows.  Pass A: the largest need() of each group over
+                // the tile's rows (row maxima, then warp maxima into sRed, then the four
+                // warps').  Pass B: every sum rounded to odd at e1 = tile need - 7, so that
+                // |t| < 127.5 * 2^7 fits int16 and the final rounding, a right shift by
+                // e_group - e1 >= 7 >= 2 bits, equals RNE of the exact sum (rounding to odd
+                // with two or more extra bits and then to nearest is correct rounding:
+                // Boldo and Melquiond, IEEE Trans. Computers 57(4), 2008).
+                int *red = sRed + wg * 32;
+                for (int g = g_lo; g < g_hi; ++g) {
+                    const int g0 = g * Gt, gf = gfast[g];
+                    int need = kNoExp;
+                    if (gf) {
+                        int ymax = 0, ymin = 0;
+                        for (int c = g0; c < g0 + Gt; c += 32) {
+                            tmem_ld32(taddr + c, v);
+                            tmem_ld_wait();
+                            if (valid) {
+#pragma unroll
+                                for (int q = 0; q < 32; q += 4) {
+                                    const int4 d4 = gf == 2 ? make_int4(1, 1, 1, 1) : *reinterpret_cast<const int4 *>(colD + c + q);
+                                    const int y0 = (int)v[q] * d4.x, y1 = (int)v[q + 1] * d4.y;
+                                    const int y2 = (int)v[q + 2] * d4.z, y3 = (int)v[q + 3] * d4.w;
+                                    ymax = max(ymax, max(max(y0, y1), max(y2, y3)));
+                                    ymin = min(ymin, min(min(y0, y1), min(y2, y3)));
+                                }
                             }
                         }
-                        emax = warp_max(emax);
-                        if (lane == 0 && emax > kNoExp) atomicMax(gacc + group_of(c) + gcol0, emax);
+                        const int amax = max(ymax, -ymin);
+                        if (amax) need = ea + gmin[g] + need_off32((uint32_t)amax);
+                    } else {
+                        for (int c = g0; c < g0 + Gt; c += 32) {
+                            tmem_ld32(taddr + c, v);
+                            tmem_ld_wait();
+                            if (valid) {
+#pragma unroll 8
+                                for (int q = 0; q < 32; ++q) {
+                                    const int32_t x = (int32_t)v[q];
+                                    if (x) need = max(need, ea + colE[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
+                                }
+                            }
+                        }
+                    }
+                    need = warp_max(need);
+                    if (lane == 0) red[g * 4 + wq] = need;
+                }
+                named_bar_sync(bar_id, 128);
+                for (int g = g_lo; g < g_hi; ++g) {
+                    const int g0 = g * Gt, gf = gfast[g], gcol = gcol0 + g;
+                    const int tneed = max(max(red[g * 4], red[g * 4 + 1]), max(red[g * 4 + 2], red[g * 4 + 3]));
+                    if (et == 0 && n0 + g0 < p.N) {
+                        p.tile_need[(int64_t)mt * p.out_exp_ld + gcol] = tneed;
+                        if (tneed > kNoExp) atomicMax(p.gmax + gcol, tneed);
+                    }
+                    const int e1 = tneed - 7;
+                    // round to odd: floor(y / 2^s) with the sticky bit ORed into the last place
+                    auto ro = [](int y, int s) {
+                        if (s <= 0) return y << min(-s, 31);
+                        s = min(s, 31);
+                        return (y >> s) | (int)((y & ((1 << s) - 1)) != 0);
+                    };
+                    for (int c = g0; c < g0 + Gt; c += 32) {
+                        tmem_ld32(taddr + c, v);
+                        tmem_ld_wait();
+                        if (!valid || n0 + c >= p.N) continue;
+                        uint32_t w[16];
+                        if (tneed <= kNoExp) {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) w[q] = 0u;
+                        } else if (gf) {
+                            const int s = e1 - ea - gmin[g];  // uniform over the row's group
+#pragma unroll
+                            for (int q = 0; q < 32; q += 2) {
+                                const int m0 = gf == 2 ? 1 : colD[c + q], m1 = gf == 2 ? 1 : colD[c + q + 1];
+                                w[q >> 1] = __byte_perm((uint32_t)ro((int)v[q] * m0, s), (uint32_t)ro((int)v[q + 1] * m1, s), 0x5410);
+                            }
+                        } else {
+#pragma unroll 4
+                            for (int q = 0; q < 32; q += 2)
+                                w[q >> 1] = __byte_perm((uint32_t)ro((int)v[q], e1 - ea - colE[c + q]),
+                                                        (uint32_t)ro((int)v[q + 1], e1 - ea - colE[c + q + 1]), 0x5410);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.ws16 + grow * p.ws16_ld + n0 + c);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                     }
                 }
             } else {
@@ -522,9 +596,9 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     const int gf = gfast[g];
                     if (G32 && gf) {
                         if (gf == 2)
-                            epi_fast32<false>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol, et);
+                            epi_fast32<false>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
                         else
-                            epi_fast32<true>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol, et);
+                            epi_fast32<true>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
                         continue;
                     }
                     const int gm = gmin[g];
@@ -547,13 +621,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                             }
                         }
                         const int amax = max(ymax, -ymin);
-                        const int need = amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp;
-                        if (p.epi == EPI_NEED_GLOBAL) {
-                            const int m = warp_max(need);
-                            if (lane == 0 && m > kNoExp && n0 + g0 < p.N) atomicMax(p.gmax + gcol, m);
-                            continue;
-                        }
-                        e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : need);
+                        e = finalize_exp(amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp);
                         // mantissa = RNE((x << d) * 2^-S), S = e - ea - gm uniform over the row
                         const int S = (e == kEZero) ? 0 : e - ea - gm;
                         const int ls = S < 0 ? -S : 0;
@@ -609,12 +677,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                                 }
                             }
                         }
-                        if (p.epi == EPI_NEED_GLOBAL) {
-                            const int m = warp_max(emax);
-                            if (lane == 0 && m > kNoExp && n0 + g0 < p.N) atomicMax(p.gmax + gcol, m);
-                            continue;
-                        }
-                        e = finalize_exp(p.epi == EPI_FIT_GLOBAL ? p.gmax[gcol] : emax);
+                        e = finalize_exp(emax);
                         for (int c = g0; c < g0 + Gt; c += 32) {
                             tmem_ld32(taddr + c, v);
                             tmem_ld_wait();
@@ -634,10 +697,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                             }
                         }
                     }
-                    if (n0 + g0 < p.N) {
-                        if (p.epi == EPI_FIT_ROW && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
-                        if (p.epi == EPI_FIT_GLOBAL && et == 0) p.out_exp[gcol] = (int8_t)e;
-                    }
+                    if (n0 + g0 < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
                 }
             }
             tc_fence_before();
@@ -649,8 +709,6 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (I32 && p.gmax && threadIdx.x < 8 && gacc[threadIdx.x] > kNoExp)
-        atomicMax(p.gmax + threadIdx.x, gacc[threadIdx.x]);
     if (warp == 2) tmem_dealloc(tmem_base, L::kTmemCols);
 }
 

@@ -180,6 +180,37 @@ def test_conv_fwd_and_bwd_data(ict, shape, global_groups):
     status_ok(ict)
 
 
+@pytest.mark.parametrize("n,h,w,c,k,G,wexp", [
+    (2, 7, 7, 256, 512, 32, (-10, -6)),    # 16 group columns (forward), 8 (backward-data); two N tiles
+    (2, 5, 12, 512, 128, 64, (-10, -6)),   # 512 contracted channels, 8 output groups backward
+    (1, 9, 20, 128, 320, 32, (-10, -6)),   # 320 = 256 + 64: a ragged N tile
+    (3, 6, 50, 64, 192, 192, (-10, -6)),   # one group over all channels, 100 of 128 tile rows
+    (2, 8, 8, 64, 128, 32, (-24, -6)),     # weight exponents 18 apart: exact per-element epilogue
+])
+def test_conv_all_pixel_groups(ict, n, h, w, c, k, G, wexp):
+    """Output groups spanning every pixel (Table 6 convolution, channel groups shared by
+    the whole batch): the Product's int16 round-to-odd sums, the per-tile needs and the
+    streaming rounding pass, forward and backward-data, with up to 16 group columns, two
+    N tiles, a ragged N tile, partial M tiles, all-zero groups and the exact epilogue."""
+    rng = np.random.default_rng(n * h + w + c + k + G)
+    npix = n * h * w
+    X = with_groups(np.where(rng.random((npix, c)) < 0.5, 0, rng.integers(1, 128, size=(npix, c))).astype(np.int8),
+                    npix, 32, lambda g: rng.integers(-8, -5, size=g))
+    W = rand_ce(rng, k, 9 * c, 1, 9 * c, elo=wexp[0], ehi=wexp[1])
+    W.mant[k - 32:] = 0          # the last forward group column is all zero: E_ZERO
+    W.exp[k - 32:] = E_ZERO
+    dY = with_groups(clipped_laplace(rng, (npix, k)), npix, 32, lambda g: rng.integers(-14, -11, size=g))
+    dY.mant[:, :32] = 0          # an all-zero input group: backward-data sums come from the others
+    dY.exp[0, 0] = E_ZERO
+    d = dict(n=n, h=h, w=w, c=c, k=k, r=3, s=3, stride=1, pad=1)
+    for direction, a, b, out_c in ((ict.CONV_FWD, X, W, k), (ict.CONV_BWD_DATA, dY, W, c)):
+        g = min(G, out_c)
+        ref = oracle.conv(direction, d, a, b, npix, g)
+        got = ict.conv(direction, d, ict.DevCE.from_host(a), ict.DevCE.from_host(b), npix, g).to_host()
+        same(got, ref, f"conv dir={direction} n{n} {h}x{w} c{c} k{k} G{g}")
+    status_ok(ict)
+
+
 # ------------------------------------------------------------------ GELU
 
 

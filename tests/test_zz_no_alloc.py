@@ -1,4 +1,4 @@
-"""The allocation-free forward Product against the workspace entry point.
+"""The allocation-free forward Product against the workspace entry point and the oracle.
 
 ict_linear_fwd_noalloc serves callers that cannot give the library a device workspace
 (host frameworks that reserve all device memory up front, statically budgeted
@@ -24,6 +24,7 @@ def _inputs(seed, M=1000, N=768, K=384):
 
 
 def test_noalloc_matches_workspace_entry_twice():
+    import oracle
     from integer_only_nn_02_b200 import ict
 
     for seed in (11, 12):  # two calls in a row share the scratch array
@@ -35,6 +36,9 @@ def test_noalloc_matches_workspace_entry_twice():
         ict.ict_linear_fwd_noalloc(dX, dW, Y)
         got = Y.to_host()
         assert np.array_equal(got.mant, ref.mant) and np.array_equal(got.exp, ref.exp), seed
+        # and, directly, against the CPU oracle
+        want = oracle.linear_fwd(X, W, 1, 64)
+        assert np.array_equal(got.mant, want.mant) and np.array_equal(got.exp, want.exp), seed
     code, raw = ict.ict_get_device_status()
     assert code == 0, (code, raw)
 
