@@ -102,6 +102,10 @@ def lib():
         L.oracle_rne_shift64.argtypes = [ctypes.c_int64, ctypes.c_int32]
         L.oracle_rne_shift64.restype = ctypes.c_int64
         L.oracle_fit_two_term.argtypes = [ctypes.c_int64] + [ctypes.c_void_p] * 5
+        L.oracle_softmax_ce.argtypes = [P(_OT), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, P(_OT)]
+        L.oracle_gelu_lut_fwd.argtypes = [P(_OT), ctypes.c_void_p, P(_OT)]
+        L.oracle_gelu_lut_bwd.argtypes = [P(_OT), P(_OT), ctypes.c_void_p, P(_OT)]
     return _lib
 
 
@@ -284,6 +288,43 @@ def gelu_fwd(H: CE) -> CE:
 
 def gelu_bwd(H: CE, dG: CE, g_rows=1, g_cols=32) -> CE:
     return _product("oracle_gelu_bwd", H, dG, H.rows, H.cols, g_rows, g_cols)
+
+
+# ------------------------------------------------------------------ lookup-table nonlinearities
+
+
+def softmax_ce(Z: CE, target: np.ndarray, g_rows: int = 1, g_cols: int = None):
+    """Output head through LUT_exp / LUT_log (Table 8): (loss per row as integers at
+    scale 2^-5, gradient of the summed loss as a (C,e) tensor in (g_rows, g_cols) groups)."""
+    from oracle import luts
+
+    t = luts.tables()
+    tgt = np.ascontiguousarray(target, dtype=np.int32)
+    loss = np.zeros(Z.rows, np.int32)
+    dZ = empty_ce(Z.rows, Z.cols, g_rows, g_cols or Z.cols)
+    _check(lib().oracle_softmax_ce(ctypes.byref(_ot(Z)), _ptr(tgt), _ptr(t["exp"]), _ptr(t["log"]), _ptr(loss),
+                                   ctypes.byref(_ot(dZ))), "softmax_ce")
+    return loss, dZ
+
+
+def gelu_lut_fwd(H: CE) -> CE:
+    """GELU forward through LUT_fwd (Table 7), exponents carried unchanged."""
+    from oracle import luts
+
+    out = empty_ce(H.rows, H.cols, H.g_rows, H.g_cols)
+    _check(lib().oracle_gelu_lut_fwd(ctypes.byref(_ot(H)), _ptr(luts.tables()["gelu_fwd"]), ctypes.byref(_ot(out))),
+           "gelu_lut_fwd")
+    return out
+
+
+def gelu_lut_bwd(H: CE, dY: CE, g_rows=1, g_cols=32) -> CE:
+    """GELU backward through LUT_bwd (Table 7): FIT(dY * LUT_bwd[e, C] * 2^-6)."""
+    from oracle import luts
+
+    out = empty_ce(H.rows, H.cols, g_rows, g_cols)
+    _check(lib().oracle_gelu_lut_bwd(ctypes.byref(_ot(H)), ctypes.byref(_ot(dY)), _ptr(luts.tables()["gelu_bwd"]),
+                                     ctypes.byref(_ot(out))), "gelu_lut_bwd")
+    return out
 
 
 def sum_(X: CE, Y: CE, g_rows: int, g_cols: int) -> CE:

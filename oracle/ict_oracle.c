@@ -1097,6 +1097,110 @@ int oracle_avgpool_bwd(const o_tensor *dY, int n, int h, int w, int K, o_tensor 
 /* ------------------------------------------------------------------------------------ */
 
 /* need() and RNE on int64 inputs, exported so the tests can pin them by brute force. */
+/* ------------------------------------------------------------------------------------ */
+/* Public: nonlinear-function primitive through lookup tables (Tables 7 and 8)          */
+/* ------------------------------------------------------------------------------------ */
+
+/* The tables are inputs (oracle/luts.py builds them from their defining formulas):
+ *   lut_exp [30][256] uint8, [e - LUT_E_LO][k + 255] = round(exp(k 2^e) 2^7), k in [-255, 0]
+ *   lut_log [256]     uint8, [p] = round(-log(p / 2^8) 2^5), p in [1, 254]
+ *   lut_gelu_fwd / _bwd [30][256] int8, [e - LUT_E_LO][C + 128]
+ * Rows cover e = -26 .. 3; every other exponent reads the nearest end row, which equals
+ * the formula's value there (see oracle/luts.py). */
+#define LUT_E_LO (-26)
+#define LUT_E_HI 3
+static int lut_row(int e) { return (e < LUT_E_LO ? LUT_E_LO : (e > LUT_E_HI ? LUT_E_HI : e)) - LUT_E_LO; }
+
+/* Output head: softmax and cross-entropy of one target class per row (Table 8: LUT_exp
+ * and LUT_log, B = 8).  Reading of the page's tables, step by step per row i:
+ *   1. the row's logits to one exponent e_i (ALIGN_MAX along the row, as before any sum);
+ *   2. k_j = C_j - max_j C_j, in [-254, 0];
+ *   3. E_j = LUT_exp[e_i][k_j], about exp(z_j - z_max) 2^7;
+ *   4. S = sum_j E_j (at least 128: the largest logit has k = 0);
+ *   5. p_j = round(E_j 2^8 / S), the exact quotient rounded half to even (probability
+ *      p_j / 2^8);
+ *   6. loss_i = LUT_log[clamp(p_t, 1, 254)], the cross-entropy at scale 2^-5;
+ *   7. gradient of the summed loss: g_j = p_j - 2^8 [j = t] at exponent -8, FIT into the
+ *      groups of dZ.
+ * loss[rows] receives the integers of step 6; target[i] must lie in [0, cols). */
+int oracle_softmax_ce(const o_tensor *Z, const int32_t *target, const uint8_t *lut_exp,
+                      const uint8_t *lut_log, int32_t *loss, o_tensor *dZ) {
+    int st = check_input(Z);
+    if (st) return st;
+    if ((st = check_output(dZ, Z->rows, Z->cols))) return st;
+    if (!target || !lut_exp || !lut_log || !loss) return ORC_ERR_ARG;
+    const int64_t R = Z->rows, K = Z->cols;
+    for (int64_t i = 0; i < R; i++)
+        if (target[i] < 0 || target[i] >= K) return ORC_ERR_ARG;
+    if (R == 0 || K == 0) return ORC_OK;
+    int8_t *m, *e;
+    if ((st = align_dense(Z, 1, &m, &e))) { free(m); free(e); return st; }
+    i128 *x = malloc(sizeof(i128) * R * K);
+    int *r = malloc(sizeof(int) * R * K);
+    for (int64_t i = 0; i < R; i++) {
+        const int8_t *c = m + i * K;
+        int cmax = c[0];
+        for (int64_t j = 1; j < K; j++) if (c[j] > cmax) cmax = c[j];
+        const uint8_t *row = lut_exp + (int64_t)lut_row(e[i]) * 256;
+        int64_t S = 0;
+        for (int64_t j = 0; j < K; j++) S += row[c[j] - cmax + 255];
+        int pt = 0;
+        for (int64_t j = 0; j < K; j++) {
+            int64_t num = (int64_t)row[c[j] - cmax + 255] << 8;
+            int64_t q = num / S, rem = num - q * S;
+            if (2 * rem > S || (2 * rem == S && (q & 1))) q++;
+            if (j == target[i]) pt = (int)q;
+            x[i * K + j] = q - (j == target[i] ? 256 : 0);
+            r[i * K + j] = -8;
+        }
+        loss[i] = lut_log[pt < 1 ? 1 : (pt > 254 ? 254 : pt)];
+    }
+    st = fit_matrix(x, r, dZ);
+    free(x); free(r); free(m); free(e);
+    return st;
+}
+
+/* GELU forward through its table (Table 7): out = LUT_fwd[e][C] with the exponent of
+ * every group carried unchanged (E_ZERO groups stay E_ZERO with zero mantissas).  out
+ * must have H's shape and group partition. */
+int oracle_gelu_lut_fwd(const o_tensor *H, const int8_t *lut_fwd, o_tensor *out) {
+    int st = check_input(H);
+    if (st) return st;
+    if ((st = check_output(out, H->rows, H->cols))) return st;
+    if (!lut_fwd || out->g_rows != H->g_rows || out->g_cols != H->g_cols) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < H->rows; i++)
+        for (int64_t j = 0; j < H->cols; j++) {
+            int e = exp_at(H, i, j), c = mant_at(H, i, j);
+            out->mant[i * out->ld + j] = e == E_ZERO ? 0 : lut_fwd[lut_row(e) * 256 + c + 128];
+        }
+    memcpy(out->exp, H->exp, (size_t)(n_grp_rows(H) * n_grp_cols(H)));
+    return ORC_OK;
+}
+
+/* GELU backward through its table (Table 7, "(dY * LUT_bwd[e, C]) >> B_G", B_G = 6):
+ * read as the exact product dY * LUT_bwd[e_H][C_H] at exponent e_dY - 6, requantised by
+ * FIT into the groups of dH like every other product. */
+int oracle_gelu_lut_bwd(const o_tensor *H, const o_tensor *dY, const int8_t *lut_bwd, o_tensor *dH) {
+    int st = check_input(H);
+    if (st || (st = check_input(dY))) return st;
+    if (dY->rows != H->rows || dY->cols != H->cols || !lut_bwd) return ORC_ERR_ARG;
+    if ((st = check_output(dH, H->rows, H->cols))) return st;
+    const int64_t n = H->rows * H->cols;
+    i128 *x = malloc(sizeof(i128) * (n + 1));
+    int *r = malloc(sizeof(int) * (n + 1));
+    for (int64_t i = 0; i < H->rows; i++)
+        for (int64_t j = 0; j < H->cols; j++) {
+            int eh = exp_at(H, i, j), ch = mant_at(H, i, j);
+            int ed = exp_at(dY, i, j), cd = mant_at(dY, i, j);
+            int slope = lut_bwd[lut_row(eh == E_ZERO ? 0 : eh) * 256 + ch + 128];
+            x[i * H->cols + j] = (i128)cd * slope;
+            r[i * H->cols + j] = ed == E_ZERO ? 0 : ed - 6;
+        }
+    st = fit_matrix(x, r, dH);
+    free(x); free(r);
+    return st;
+}
+
 int oracle_need64(int64_t x, int32_t r) { return x == 0 ? E_ZERO : need(x, r); }
 int64_t oracle_rne_shift64(int64_t x, int32_t k) { return (int64_t)rne_scale(x, k); }
 
