@@ -102,6 +102,8 @@ def lib():
         L.oracle_rne_shift64.argtypes = [ctypes.c_int64, ctypes.c_int32]
         L.oracle_rne_shift64.restype = ctypes.c_int64
         L.oracle_fit_two_term.argtypes = [ctypes.c_int64] + [ctypes.c_void_p] * 5
+        L.oracle_linear_bits.argtypes = [ctypes.c_int, P(_OT), P(_OT), P(_OT), ctypes.c_int32]
+        L.oracle_sgd_step_bits.argtypes = [P(_OT), P(_OT), P(_OT), P(_Sgd), ctypes.c_int32]
         L.oracle_softmax_ce.argtypes = [P(_OT), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, P(_OT)]
         L.oracle_gelu_lut_fwd.argtypes = [P(_OT), ctypes.c_void_p, P(_OT)]
@@ -277,6 +279,25 @@ def sgd_step(W: CE, V: CE, G: CE, mom=(230, 8), lr=(1, 4)):
     p = _Sgd(mom[0], mom[1], lr[0], lr[1])
     _check(lib().oracle_sgd_step(ctypes.byref(_ot(W2)), ctypes.byref(_ot(V2)), ctypes.byref(_ot(G)),
                                  ctypes.byref(p)), "sgd_step")
+    return W2, V2
+
+
+def linear_bits(op: int, a: CE, b: CE, bits: int, g_rows: int = 1, g_cols: int = 32) -> CE:
+    """A linear Product with B-bit outputs (op 0 forward, 1 backward-data, 2 backward-weight)."""
+    rows = a.cols if op == 2 else a.rows
+    cols = b.rows if op == 0 else b.cols
+    out = empty_ce(rows, cols, g_rows, g_cols)
+    _check(lib().oracle_linear_bits(op, ctypes.byref(_ot(a)), ctypes.byref(_ot(b)), ctypes.byref(_ot(out)),
+                                    int(bits)), "linear_bits")
+    return out
+
+
+def sgd_step_bits(W: CE, V: CE, G: CE, bits: int, mom=(230, 8), lr=(1, 4)):
+    """The momentum step with B-bit mantissas; returns new copies of (W, V)."""
+    W2, V2 = W.copy(), V.copy()
+    p = _Sgd(int(mom[0]), int(mom[1]), int(lr[0]), int(lr[1]))
+    _check(lib().oracle_sgd_step_bits(ctypes.byref(_ot(W2)), ctypes.byref(_ot(V2)), ctypes.byref(_ot(G)),
+                                      ctypes.byref(p), int(bits)), "sgd_step_bits")
     return W2, V2
 
 

@@ -435,28 +435,45 @@ int oracle_linear_bwd_weight_acc(const o_tensor *dY, const o_tensor *X, int64_t 
     return ORC_OK;
 }
 
-static int fit_acc(const int64_t *acc, const int32_t *r, o_tensor *out) {
+static int fit_acc_q(const int64_t *acc, const int32_t *r, o_tensor *out, int qmax) {
     int64_t n = out->rows * out->cols;
     i128 *v = malloc(sizeof(i128) * (n + 1));
     int *rr = malloc(sizeof(int) * (n + 1));
     for (int64_t i = 0; i < n; i++) { v[i] = acc[i]; rr[i] = r[i]; }
-    int st = fit_matrix(v, rr, out);
+    int st = fit_matrix_q(v, rr, out, qmax);
     free(v);
     free(rr);
     return st;
 }
 
+static int fit_acc(const int64_t *acc, const int32_t *r, o_tensor *out) { return fit_acc_q(acc, r, out, QMAX); }
+
 typedef int (*acc_fn)(const o_tensor *, const o_tensor *, int64_t *, int32_t *);
-static int product(acc_fn f, const o_tensor *a, const o_tensor *b, o_tensor *out,
-                   int64_t rows, int64_t cols) {
+static int product_q(acc_fn f, const o_tensor *a, const o_tensor *b, o_tensor *out,
+                     int64_t rows, int64_t cols, int qmax) {
     if (check_output(out, rows, cols)) return ORC_ERR_ARG;
     int64_t *acc = malloc(sizeof(int64_t) * (rows * cols + 1));
     int32_t *r = malloc(sizeof(int32_t) * (rows * cols + 1));
     int st = f(a, b, acc, r);
-    if (!st) st = fit_acc(acc, r, out);
+    if (!st) st = fit_acc_q(acc, r, out, qmax);
     free(acc);
     free(r);
     return st;
+}
+static int product(acc_fn f, const o_tensor *a, const o_tensor *b, o_tensor *out, int64_t rows, int64_t cols) {
+    return product_q(f, a, b, out, rows, cols, QMAX);
+}
+
+/* The three linear directions with B-bit outputs (Table 4: INT8 down to INT4): the same
+ * alignment and exact contraction, the FIT clipping at q_max = 2^(B-1) - 1.
+ * op 0: Y = X W^T (a = X, b = W); 1: dX = dY W (a = dY, b = W); 2: dW = dY^T X. */
+int oracle_linear_bits(int op, const o_tensor *a, const o_tensor *b, o_tensor *out, int32_t bits) {
+    if (bits < 2 || bits > 8 || !a || !b) return ORC_ERR_ARG;
+    const int q = (1 << (bits - 1)) - 1;
+    if (op == 0) return product_q(oracle_linear_fwd_acc, a, b, out, a->rows, b->rows, q);
+    if (op == 1) return product_q(oracle_linear_bwd_data_acc, a, b, out, a->rows, b->cols, q);
+    if (op == 2) return product_q(oracle_linear_bwd_weight_acc, a, b, out, a->cols, b->cols, q);
+    return ORC_ERR_ARG;
 }
 
 int oracle_linear_fwd(const o_tensor *X, const o_tensor *W, o_tensor *Y) {
@@ -741,7 +758,7 @@ int oracle_depthwise(int dir, const o_conv *d, const o_tensor *a, const o_tensor
  * multiply-shifts, each right-hand side an exact two-term Sum requantised once by FIT
  * into the group (so both exponents are chosen afresh every step).  W, V and G share
  * one group partition; W and V are updated in place. */
-int oracle_sgd_step(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p) {
+static int sgd_step_q(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p, int qmax) {
     int st;
     if (!p) return ORC_ERR_ARG;
     if ((st = check_input(W)) || (st = check_input(V)) || (st = check_input(G))) return st;
@@ -771,14 +788,14 @@ int oracle_sgd_step(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p)
                 for (int64_t j = j0; j < j1; j++, n++)
                     two_term((int64_t)p->mom_mul * mant_at(V, i, j), ev - p->mom_shift,
                              mant_at(G, i, j), eg, &x[n], &r[n]);
-            int ev2 = fit_group(n, x, r, cv);
+            int ev2 = fit_group_q(n, x, r, cv, qmax);
             /* weight: Cw * 2^ew - lr_mul * Cv' * 2^(ev' - lr_shift) */
             n = 0;
             for (int64_t i = i0; i < i1; i++)
                 for (int64_t j = j0; j < j1; j++, n++)
                     two_term(mant_at(W, i, j), ew, -(int64_t)p->lr_mul * cv[n],
                              ev2 - p->lr_shift, &x[n], &r[n]);
-            int ew2 = fit_group(n, x, r, cw);
+            int ew2 = fit_group_q(n, x, r, cw, qmax);
             if (ev2 > 127 || ew2 > 127) {
 #pragma omp atomic write
                 status = ORC_ERR_EXP_RANGE;
@@ -797,6 +814,17 @@ int oracle_sgd_step(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p)
         free(x); free(r); free(cv); free(cw);
     }
     return status;
+}
+int oracle_sgd_step(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p) {
+    return sgd_step_q(W, V, G, p, QMAX);
+}
+
+/* The same update with B-bit mantissas (Table 4 trains with INT8 down to INT4): both
+ * FITs clip at q_max = 2^(B-1) - 1 (Table 7's symmetric bound), 2 <= B <= 8; every other
+ * step is unchanged. */
+int oracle_sgd_step_bits(o_tensor *W, o_tensor *V, const o_tensor *G, const o_sgd *p, int32_t bits) {
+    if (bits < 2 || bits > 8) return ORC_ERR_ARG;
+    return sgd_step_q(W, V, G, p, (1 << (bits - 1)) - 1);
 }
 
 /* ------------------------------------------------------------------------------------ */

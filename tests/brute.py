@@ -45,14 +45,14 @@ def groups_of(rows, cols, g_rows, g_cols):
             yield gi, gj, cells
 
 
-def fit_matrix_brute(vals, g_rows, g_cols):
+def fit_matrix_brute(vals, g_rows, g_cols, qmax: int = 127):
     """vals: 2-D list of Fractions -> (mant 2-D list, exp grid 2-D list)."""
     rows, cols = len(vals), len(vals[0]) if vals else 0
     mant = [[0] * cols for _ in range(rows)]
     ng_r, ng_c = -(-rows // g_rows), -(-cols // g_cols)
     exps = [[E_ZERO] * ng_c for _ in range(ng_r)]
     for gi, gj, cells in groups_of(rows, cols, g_rows, g_cols):
-        c, e = fit_brute([vals[i][j] for i, j in cells])
+        c, e = fit_brute([vals[i][j] for i, j in cells], qmax)
         exps[gi][gj] = e
         for (i, j), cc in zip(cells, c):
             mant[i][j] = cc

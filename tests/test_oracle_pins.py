@@ -395,15 +395,15 @@ def test_sgd_golden():
     assert W2.mant.tolist() == g["W_new"]["mant"] and W2.exp.tolist() == g["W_new"]["exp"]
 
 
-def _sgd_brute(W, V, G, mom, lr):
+def _sgd_brute(W, V, G, mom, lr, qmax=127):
     wv, vv, gv = ce_values(W), ce_values(V), ce_values(G)
     rows, cols = W.rows, W.cols
     vnew = [[Fraction(mom[0]) * vv[i][j] / 2 ** mom[1] + gv[i][j] for j in range(cols)] for i in range(rows)]
-    vm, ve = fit_matrix_brute(vnew, W.g_rows, W.g_cols)
+    vm, ve = fit_matrix_brute(vnew, W.g_rows, W.g_cols, qmax)
     vq = [[value(vm[i][j], ve[i // W.g_rows][j // W.g_cols]) if ve[i // W.g_rows][j // W.g_cols] != E_ZERO
            else Fraction(0) for j in range(cols)] for i in range(rows)]
     wnew = [[wv[i][j] - Fraction(lr[0]) * vq[i][j] / 2 ** lr[1] for j in range(cols)] for i in range(rows)]
-    wm, we = fit_matrix_brute(wnew, W.g_rows, W.g_cols)
+    wm, we = fit_matrix_brute(wnew, W.g_rows, W.g_cols, qmax)
     return wm, we, vm, ve
 
 
@@ -748,3 +748,56 @@ def test_requant_bits_8_is_requant():
     x = rng.integers(-(2 ** 30), 2 ** 30, size=(9, 40)).astype(np.int64)
     a, b = oracle.requant_bits(x, 8, 1, 8, base_exp=3), oracle.requant(x, 1, 8, base_exp=3)
     assert (a.mant == b.mant).all() and (a.exp == b.exp).all()
+
+
+# --------------------------------------------------------------------- B-bit variants (Table 4)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+def test_linear_bits_match_bruteforce_fit(bits):
+    """B-bit linear Products: the pinned exact accumulators, then the brute-force FIT with
+    the clip bound q_max = 2^(B-1) - 1, on B-bit inputs."""
+    q = (1 << (bits - 1)) - 1
+    rng = np.random.default_rng(40 + bits)
+    M, N, K = 6, 5, 7
+    X = rand_ce(rng, M, K, 1, 3, mag=q)
+    W = rand_ce(rng, N, K, 1, K, mag=q)
+    dY = rand_ce(rng, M, N, 1, 2, mag=q)
+    for op, accfn, args, shape in ((0, oracle.linear_fwd_acc, (X, W), (M, N)),
+                                   (1, oracle.linear_bwd_data_acc, (dY, W), (M, K)),
+                                   (2, oracle.linear_bwd_weight_acc, (dY, X), (N, K))):
+        g = (1, max(1, shape[1] // 2))
+        out = oracle.linear_bits(op, *args, bits, *g)
+        acc, r = accfn(*args)
+        vals = [[value(int(acc[i, j]), int(r[i, j])) for j in range(shape[1])] for i in range(shape[0])]
+        mant, exps = fit_matrix_brute(vals, *g, qmax=q)
+        assert out.mant.tolist() == mant and out.exp.tolist() == exps, (bits, op)
+        assert np.abs(out.mant.astype(int)).max() <= q
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("erange", [(-16, -4), (-120, 0)])
+def test_sgd_bits_matches_bruteforce(bits, erange):
+    q = (1 << (bits - 1)) - 1
+    rng = np.random.default_rng(900 + bits + erange[0])
+    for trial in range(3):
+        W = rand_ce(rng, 5, 8, 1, 8, elo=erange[0], ehi=erange[1], zero_groups=0.1, mag=q)
+        V = rand_ce(rng, 5, 8, 1, 8, elo=erange[0], ehi=erange[1], zero_groups=0.3, mag=q)
+        G = rand_ce(rng, 5, 8, 1, 8, elo=erange[0], ehi=erange[1], zero_groups=0.1, mag=q)
+        mom, lr = (230, 8), [(1, 4), (205, 11), (3, 0)][trial]
+        wm, we, vm, ve = _sgd_brute(W, V, G, mom, lr, q)
+        if max(max(r) for r in we + ve) > 127:
+            continue
+        W2, V2 = oracle.sgd_step_bits(W, V, G, bits, mom, lr)
+        assert V2.mant.tolist() == vm and V2.exp.tolist() == ve, (bits, trial)
+        assert W2.mant.tolist() == wm and W2.exp.tolist() == we, (bits, trial)
+
+
+def test_bits_8_is_the_int8_path():
+    rng = np.random.default_rng(77)
+    X, W = rand_ce(rng, 20, 64, 1, 16), rand_ce(rng, 12, 64, 1, 32)
+    a, b = oracle.linear_bits(0, X, W, 8, 1, 4), oracle.linear_fwd(X, W, 1, 4)
+    assert np.array_equal(a.mant, b.mant) and np.array_equal(a.exp, b.exp)
+    V, G = rand_ce(rng, 12, 64, 1, 32), rand_ce(rng, 12, 64, 1, 32)
+    for x, y in zip(oracle.sgd_step_bits(W, V, G, 8), oracle.sgd_step(W, V, G)):
+        assert np.array_equal(x.mant, y.mant) and np.array_equal(x.exp, y.exp)
