@@ -227,6 +227,20 @@ int32_t ict_linear_bwd_weight_partial(const ict_tensor *dY, const ict_tensor *X,
                                       int32_t acc_bits, int64_t ld_acc, void *ws,
                                       size_t ws_bytes, void *stream);
 
+/* Mantissa width of the B-bit variants (Table 4 trains the same method with INT8 down to
+ * INT4 mantissas; Table 7's clip bound is q_max = 2^(B-1) - 1).  Process-wide, 2 <= B <= 8,
+ * default 8; read when an entry point is called.  With B < 8 every FIT of the linear
+ * Products (all three directions, the split-batch forms and ict_linear_fwd_noalloc),
+ * ict_requant and the SGD updates picks the smallest exponent at which the group fits
+ * [-q_max, q_max]; alignment, contraction and the two-term sums are unchanged (their
+ * results stay within the inputs' width).  Mantissas stay one per byte.  Entry points
+ * whose FIT is INT8-only (convolution, depthwise convolution, Sum, average pool, GELU
+ * backward, the output head, ReLU6) return ICT_ERR_LAYOUT while B < 8; ReLU, GELU
+ * forward and patch extraction never widen a mantissa and accept any B.
+ * ict_set_mantissa_bits returns ICT_ERR_INVALID_ARG outside [2, 8]. */
+int32_t ict_set_mantissa_bits(int32_t bits);
+int32_t ict_get_mantissa_bits(void);
+
 /* Allocation-free forward Product.  The paper has no counterpart to this entry point;
  * it exists for callers that cannot hand the library a device workspace: integrations
  * whose device memory is reserved up front by a host framework that exposes no
@@ -352,6 +366,41 @@ int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W,
 /*        partition.                                                                    */
 int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream);
 int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, void *stream);
+
+/* --------------------------------------------------------------------------------- */
+/* The nonlinear-function primitive through lookup tables.                             */
+/*   Table 7 (GELU): forward LUT_fwd[e, C], backward (dY * LUT_bwd[e, C]) >> B_G, INT8  */
+/*   [30, 256], the exponent carried unchanged.  Table 8 (output head): LUT_exp[e][k] = */
+/*   round(exp(k 2^e) 2^7), k in [-255, 0], [30, 256]; LUT_log[p] = round(-log(p / 2^8)*/
+/*   2^5), p in [1, 254], [256]; built once at initialization.                         */
+/* Readings (the page prints the entry formulas only): the 30 table exponents are       */
+/* e = -26 .. 3 and a lookup clamps e to them (the formulas give the end rows' values   */
+/* for every exponent beyond); "round" is half to even; GELU(x) = x Phi(x) with Phi the */
+/* standard normal CDF, LUT_fwd[e][C] = round(C Phi(C 2^e)), LUT_bwd[e][C] =            */
+/* round(GELU'(C 2^e) 2^6) (B_G = 6: the slope lies in about [-0.129, 1.129]).          */
+/* The library builds its tables once per process on the host.                          */
+/*                                                                                      */
+/* ict_lut_tables: host copies of the library's tables (any pointer may be NULL):        */
+/*   lut_exp [30][256] uint8 at [e + 26][k + 255];  lut_log [256] uint8 at [p] (entries  */
+/*   0 and 255 repeat 1 and 254);  gelu_fwd / gelu_bwd [30][256] int8 at [e + 26][C+128].*/
+/*   Host memory only; launches nothing.                                                */
+/* ict_gelu_lut_fwd: out mantissa = LUT_fwd[e][C]; out has H's shape and groups and      */
+/*   receives H's exponents.  cols, ld and g_cols multiples of 16 (or g_cols >= cols).  */
+/* ict_gelu_lut_bwd: dH = FIT(dY * LUT_bwd[e_H][C_H] * 2^-6), the exact product at       */
+/*   exponent e_dY - 6 requantised into dH's groups like every product; H, dY and dH     */
+/*   share one row-local group partition (g_rows = 1, g_cols a multiple of 16).          */
+/* ict_softmax_ce: the output head on logits Z [rows][classes] with one target class per */
+/*   row (target[rows], int32 in [0, classes), device memory).  Per row: the logits to  */
+/*   one exponent e (ALIGN_MAX along the row); k = C - max C; E = LUT_exp[e][k];        */
+/*   S = sum E; p = round(E 2^8 / S) (exact quotient, half to even); loss[row] =        */
+/*   LUT_log[clamp(p_target, 1, 254)] (int32, device memory, the cross-entropy at scale  */
+/*   2^-5); dZ = FIT(p - 2^8 [class = target]) at exponent -8 into dZ's row-local groups */
+/*   (the gradient of the summed loss).  Argument errors return before any launch.      */
+int32_t ict_lut_tables(uint8_t *lut_exp, uint8_t *lut_log, int8_t *gelu_fwd, int8_t *gelu_bwd);
+int32_t ict_gelu_lut_fwd(const ict_tensor *H, ict_tensor *out, void *stream);
+int32_t ict_gelu_lut_bwd(const ict_tensor *H, const ict_tensor *dY, ict_tensor *dH, void *stream);
+int32_t ict_softmax_ce(const ict_tensor *Z, const int32_t *target, int32_t *loss, ict_tensor *dZ,
+                       void *stream);
 
 /* --------------------------------------------------------------------------------- */
 /* ReLU / ReLU6, the Clip primitive (Table 6: "ReLU / ReLU6 -> Clip"; Table 7): integer  */

@@ -12,6 +12,7 @@
 #include "ict_device.cuh"
 #include "ict_elementwise.cuh"
 #include "ict_gemm.cuh"
+#include "ict_lut.cuh"
 #include "ict_pointwise.cuh"
 
 using namespace ict;
@@ -31,6 +32,11 @@ std::mutex g_mu;
 DeviceInfo g_dev[64];
 uint64_t g_wait_ns = 2000000000ull;  // bound of every mbarrier wait inside a kernel
 const uint64_t kDrainNs = 1000000000ull;
+// mantissa bits B of every FIT the linear Products, ict_requant and the SGD perform
+// (q_max = 2^(B-1) - 1; ict_set_mantissa_bits), process-wide
+std::atomic<int> g_mantissa_bits{8};
+// entry points whose FIT is written for INT8 only refuse other mantissa widths
+int int8_only() { return g_mantissa_bits.load(std::memory_order_relaxed) == 8 ? ICT_OK : ICT_ERR_LAYOUT; }
 // largest channel count (contracted or produced) of the implicit-GEMM convolution
 constexpr int kConvMaxChannels = 2048;
 
@@ -460,24 +466,77 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
         if constexpr (LOAD == LOAD_2D && BN <= 128) {
             if (p.nwg == 4) {  // four epilogue warpgroups, four accumulators
                 constexpr int kB4 = GemmSmem<BN, BK, ST, 4>::kBytes;
-                if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, true, 4>, 4, kB4);
-                return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, false, 4>, 4, kB4);
+                if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 1, 4>, 4, kB4);
+                return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 0, 4>, 4, kB4);
             }
         }
-        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, true>, 2, kB2);
-        return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, false>, 2, kB2);
+        if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 1>, 2, kB2);
+        if constexpr (LOAD == LOAD_2D) {
+            if (gt == 64) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 2>, 2, kB2);
+        }
+        return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 0>, 2, kB2);
     }
 }
 
+// Pairs of CTAs (clusters of two) on 256 x BN tiles: the grid is even and launched with
+// the cluster dimension; each CTA holds half of every B stage, so it has room for the
+// stages of a BN / 2 tile.
+template <int BN>
+int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid,
+                       cudaStream_t s) {
+    constexpr int ST = stages_for(BN / 2, 128);
+    auto run = [&](auto k, int smem_bytes, int nwg) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+            return (int)ICT_ERR_CUDA;
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        cfg.blockDim = dim3((unsigned)(128 + 128 * nwg), 1, 1);
+        cfg.dynamicSmemBytes = (size_t)smem_bytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, k, ta, tb, p) != cudaSuccess) return (int)ICT_ERR_CUDA;
+        counted(1);
+        return launch_status();
+    };
+    constexpr int kB = GemmSmem<BN, 128, ST, 2, true>::kBytes;
+    if (p.epi == EPI_I32) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_I32, 0, 2, true>, kB, 2);
+    if (p.epi != EPI_FIT_ROW) return ICT_ERR_LAYOUT;
+    const int gt = p.G >= p.N ? BN : p.G;
+    if constexpr (BN == 256) {
+        // 32- and 64-column groups on 256-wide tiles: four epilogue warpgroups, a quarter of
+        // the columns each
+        constexpr int kB4 = GemmSmem<BN, 128, ST, 4, true, 2>::kBytes;
+        if (gt == 32) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 1, 4, true, true>, kB4, 4);
+        if (gt == 64) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 3, 4, true, true>, kB4, 4);
+    }
+    if (gt == 32) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 1, 2, true>, kB, 2);
+    if (gt == 64) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 2, 2, true>, kB, 2);
+    return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 0, 2, true>, kB, 2);
+}
+
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
-                const GemmParams &p_in, int grid, cudaStream_t s, double ops) {
+                const GemmParams &p_in, int grid, cudaStream_t s, double ops, bool pair = false) {
     KTimer kt(s, KC_GEMM, ops);
     // both epilogue warpgroups take every tile (one column half each) when no output
     // group straddles the halves
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
-    if (p.nwg != 4 || p.epi != EPI_FIT_ROW) p.nwg = 2;
+    if (p.nwg != 4 || p.epi != EPI_FIT_ROW || pair) p.nwg = 2;
     p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0));
+    if (pair) {
+        if (load != LOAD_2D || bk != 128 || (grid & 1)) return ICT_ERR_LAYOUT;
+        if (bn == 128) return launch_gemm_pair_t<128>(ta, tb, p, grid, s);
+        if (bn == 192) return launch_gemm_pair_t<192>(ta, tb, p, grid, s);
+        if (bn == 256) return launch_gemm_pair_t<256>(ta, tb, p, grid, s);
+        return ICT_ERR_LAYOUT;
+    }
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
     if (bn == BN_ && bk == BK_ && load == LOAD_) \
         return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s);
@@ -566,6 +625,7 @@ Operand operand_cols(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
 struct ProductPlan {
     int bn, nwg, splits, kblk_per_split, n_kblk, n_mtiles, n_ntiles, units, grid;
     bool fused;
+    bool pair;  // clusters of two CTAs on 256-row tiles (tcgen05 cta_group::2)
     int32_t *ws32;
     int64_t ws_ld;
 };
@@ -577,19 +637,24 @@ ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out,
     ProductPlan pl;
     pl.bn = pick_bn_waves(M, N, out->g_cols, sms);
     pl.nwg = 2;
-    {   // short contractions are bound by the FIT epilogue: four epilogue warpgroups
-        // (four accumulators) on 128-wide tiles
+    {   // short contractions with 32-column output groups: four epilogue warpgroups (four
+        // accumulators) on 128-wide tiles.  64-column groups keep a whole group in
+        // registers, which leaves room for two warpgroups only; they split each tile.
         const int64_t G = out->g_cols;
-        if (K <= 1024 && N % 128 == 0 && G < N && G % 32 == 0 && 128 % G == 0) pl.bn = 128, pl.nwg = 4;
+        if (K <= 1024 && N % 128 == 0 && G == 32) pl.bn = 128, pl.nwg = 4;
     }
+    // large Products run on pairs of CTAs: a 256 x BN tile per pair halves the operand
+    // bytes each SM draws from L2 per multiply-add, which bounds 128-row tiles
+    pl.pair = pl.nwg == 2 && pl.bn >= 128 && pl.bn % 64 == 0 && M >= 2048 && sms >= 2;
+    const int units_per_wave = pl.pair ? sms / 2 : sms;
     pl.n_kblk = (int)cdiv64(K, 128);
-    pl.n_mtiles = (int)cdiv64(M, 128);
+    pl.n_mtiles = (int)cdiv64(M, pl.pair ? 256 : 128);
     pl.n_ntiles = (int)cdiv64(N, pl.bn);
     const int tiles = pl.n_mtiles * pl.n_ntiles;
     int splits = 1;
-    if (allow_split && tiles < sms && pl.n_kblk >= 8) {
+    if (allow_split && tiles < units_per_wave && pl.n_kblk >= 8) {
         // whole waves: as many K slices as fit next to the tiles on the SMs
-        splits = (int)std::min<int64_t>(sms / tiles, pl.n_kblk / 4);
+        splits = (int)std::min<int64_t>(units_per_wave / tiles, pl.n_kblk / 4);
         if (splits < 1) splits = 1;
     }
     // int32 partial sums stay exact: at most 2^17 products of magnitude <= 127^2 each
@@ -598,7 +663,7 @@ ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out,
     pl.kblk_per_split = (int)cdiv64(pl.n_kblk, splits);
     pl.splits = (int)cdiv64(pl.n_kblk, pl.kblk_per_split);
     pl.units = tiles * pl.splits;
-    pl.grid = std::min(pl.units, sms);
+    pl.grid = pl.pair ? 2 * std::min(pl.units, units_per_wave) : std::min(pl.units, sms);
     const int64_t G = out->g_cols;
     const bool groups_in_tile = (G >= N) ? (N <= pl.bn) : (pl.bn % G == 0 && G % 32 == 0);
     pl.fused = !raw && pl.splits == 1 && groups_in_tile;
@@ -628,7 +693,8 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     CUtensorMap ta, tb;
     int st;
     if ((st = tmap_2d(&ta, A.mant, K, M, A.ld, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return st;
-    if ((st = tmap_2d(&tb, B.mant, K, N, B.ld, 128, pl.bn, CU_TENSOR_MAP_SWIZZLE_128B))) return st;
+    if ((st = tmap_2d(&tb, B.mant, K, N, B.ld, 128, pl.pair ? pl.bn / 2 : pl.bn, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
     GemmParams p;
     memset(&p, 0, sizeof(p));
     p.M = (int)M;
@@ -652,17 +718,20 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     p.ws32 = pl.ws32;
     p.ws_ld = pl.ws_ld;
     p.ws_split_stride = M * pl.ws_ld;
-    p.stage_tx_bytes = (uint32_t)(128 * 128 + pl.bn * 128);
+    p.stage_tx_bytes = (uint32_t)(pl.pair ? 2 * (128 * 128 + (pl.bn / 2) * 128) : 128 * 128 + pl.bn * 128);
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     p.epi = pl.fused ? EPI_FIT_ROW : EPI_I32;
+    p.qb = g_mantissa_bits.load(std::memory_order_relaxed);
     p.nwg = pl.nwg;
-    if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K)))
+    if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K,
+                          pl.pair)))
         return st;
     if (pl.fused) return ICT_OK;
     if (raw_acc) return launch_sum_slices(pl, M, N, raw_acc, raw_bits, raw_ld, s);
     RequantArgs a;
     memset(&a, 0, sizeof(a));
+    a.qb = g_mantissa_bits.load(std::memory_order_relaxed);
     a.v32 = pl.ws32;
     a.nsplit = pl.splits;
     a.split_stride = M * pl.ws_ld;
@@ -1044,6 +1113,7 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     // the weight operand stays in shared memory when all its K blocks fit the B ring
     p.b_resident = p.n_ntiles == 1 && p.n_kblk <= stages_for(cp.bn, 64);
     p.stage_tx_bytes = (uint32_t)(64 * d->w * cp.rows_per_tile + (p.b_resident ? 0 : 64 * cp.bn));
+    p.qb = 8;
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
     const int grid = std::min(p.num_units, sms);
@@ -1204,6 +1274,7 @@ int run_wgrad(const ict_conv_desc *d, const ict_tensor *dY, const ict_tensor *X,
     if (sums_only) return ICT_OK;
     RequantArgs a;
     memset(&a, 0, sizeof(a));
+    a.qb = 8;  // convolution: INT8 only
     a.v64 = wp.sums64;
     a.nsplit = 1;
     a.rows = wp.N;
@@ -1383,6 +1454,7 @@ int conv_split(int dir, const ict_conv_desc *d, const ict_tensor *a, const ict_t
                int32_t *need, void *ws, size_t ws_bytes, void *stream, int phase) {
     int st, sms = 0;
     if ((st = device_info(&sms))) return st;
+    if ((st = int8_only())) return st;
     if ((dir != ICT_CONV_FWD && dir != ICT_CONV_BWD_DATA) || !need) return ICT_ERR_INVALID_ARG;
     if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
     Ws w = make_ws(ws, ws_bytes, false);
@@ -1575,6 +1647,13 @@ int32_t ict_set_wait_limit_ns(uint64_t ns) {
     return ICT_OK;
 }
 
+int32_t ict_set_mantissa_bits(int32_t bits) {
+    if (bits < 2 || bits > 8) return ICT_ERR_INVALID_ARG;
+    g_mantissa_bits.store(bits, std::memory_order_relaxed);
+    return ICT_OK;
+}
+int32_t ict_get_mantissa_bits(void) { return g_mantissa_bits.load(std::memory_order_relaxed); }
+
 int32_t ict_requant(const void *vals, int32_t val_bits, int64_t rows, int64_t cols, int64_t ld_vals,
                     int32_t base_exp, const int8_t *row_exp, const int8_t *col_exp,
                     ict_tensor *out, void *stream) {
@@ -1588,6 +1667,7 @@ int32_t ict_requant(const void *vals, int32_t val_bits, int64_t rows, int64_t co
     if (out->g_rows != 1 && rows > 1) return ICT_ERR_LAYOUT;
     RequantArgs a;
     memset(&a, 0, sizeof(a));
+    a.qb = g_mantissa_bits.load(std::memory_order_relaxed);
     a.v32 = val_bits == 32 ? (const int32_t *)vals : nullptr;
     a.v64 = val_bits == 64 ? (const int64_t *)vals : nullptr;
     a.nsplit = 1;
@@ -1742,6 +1822,7 @@ int32_t ict_conv_implicit_gemm(int32_t dir, const ict_conv_desc *d, const ict_te
                                void *stream) {
     int st, sms = 0;
     if ((st = device_info(&sms))) return st;
+    if ((st = int8_only())) return st;
     if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
     Ws w = make_ws(ws, ws_bytes, false);
     if (dir == ICT_CONV_BWD_WEIGHT) {
@@ -1761,6 +1842,7 @@ int32_t ict_conv_fwd_act(const ict_conv_desc *d, const ict_tensor *X, const ict_
                          int32_t act, void *ws, size_t ws_bytes, void *stream) {
     int st, sms = 0;
     if ((st = device_info(&sms))) return st;
+    if ((st = int8_only())) return st;
     if (act < ACT_NONE || act > ACT_RELU6) return ICT_ERR_INVALID_ARG;
     if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
     Ws w = make_ws(ws, ws_bytes, false);
@@ -1782,6 +1864,7 @@ int32_t ict_conv_bwd_weight_partial(const ict_conv_desc *d, const ict_tensor *dY
                                     size_t ws_bytes, void *stream) {
     int st, sms = 0;
     if ((st = device_info(&sms))) return st;
+    if ((st = int8_only())) return st;
     if (!d || !acc || !e_k || !e_rsc) return ICT_ERR_INVALID_ARG;
     if (ws && ((uintptr_t)ws & 255)) return ICT_ERR_WORKSPACE;
     const int64_t RSC = (int64_t)d->r * d->s * d->c;
@@ -1815,6 +1898,7 @@ int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W, ict
     if ((st = check_sgd_params(p))) return st;
     SgdArgs a;  // passed whole as the kernel's parameter block (about 12 KB)
     memset(&a, 0, sizeof(a));
+    a.qb = g_mantissa_bits.load(std::memory_order_relaxed);
     a.n = n_tensors;
     a.mom_mul = p->mom_mul;
     a.mom_shift = p->mom_shift;
@@ -1822,6 +1906,8 @@ int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W, ict
     a.lr_shift = p->lr_shift;
     a.cap_mom = 29 - bitlen_u64(127ull * (uint64_t)std::abs(p->mom_mul));
     a.cap_lr = 29 - bitlen_u64(127ull * (uint64_t)std::abs(p->lr_mul));
+    a.capf_mom = 23 - bitlen_u64(127ull * (uint64_t)std::abs(p->mom_mul));
+    a.capf_lr = 23 - bitlen_u64(127ull * (uint64_t)std::abs(p->lr_mul));
     int64_t total = 0;
     for (int i = 0; i < n_tensors; ++i) {
         if ((st = fill_sgd_tensor(W[i], V[i], G[i], &a.t[i]))) return st;
@@ -1867,6 +1953,7 @@ int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream) {
 int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
     if ((st = check_tensor(H)) || (st = check_tensor(dG)) || (st = check_tensor(dH))) return st;
     if (dG->rows != H->rows || dG->cols != H->cols || dH->rows != H->rows || dH->cols != H->cols)
         return ICT_ERR_INVALID_ARG;
@@ -1915,11 +2002,123 @@ int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, 
     return launch_status();
 }
 
+// ---- nonlinear functions through lookup tables (Tables 7 and 8)
+
+int32_t ict_lut_tables(uint8_t *lut_exp, uint8_t *lut_log, int8_t *gelu_fwd, int8_t *gelu_bwd) {
+    const LutTables &t = lut_tables();
+    if (lut_exp) memcpy(lut_exp, t.exp, sizeof(t.exp));
+    if (lut_log) memcpy(lut_log, t.log, sizeof(t.log));
+    if (gelu_fwd) memcpy(gelu_fwd, t.gelu_fwd, sizeof(t.gelu_fwd));
+    if (gelu_bwd) memcpy(gelu_bwd, t.gelu_bwd, sizeof(t.gelu_bwd));
+    return ICT_OK;
+}
+
+int32_t ict_gelu_lut_fwd(const ict_tensor *H, ict_tensor *out, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = check_tensor(H)) || (st = check_tensor(out))) return st;
+    if (out->rows != H->rows || out->cols != H->cols || out->g_rows != H->g_rows || out->g_cols != H->g_cols)
+        return ICT_ERR_INVALID_ARG;
+    if ((st = check_pointwise(H)) || (st = check_pointwise(out))) return st;
+    if (H->rows == 0 || H->cols == 0) return ICT_OK;
+    GeluLutArgs a;
+    memset(&a, 0, offsetof(GeluLutArgs, lut));
+    a.h = H->mant;
+    a.h_exp = H->exp;
+    a.out = out->mant;
+    a.rows = H->rows;
+    a.cols = H->cols;
+    a.ld_h = H->ld;
+    a.ld_out = out->ld;
+    a.g_rows = clamp_div(H->g_rows, H->rows);
+    a.g_cols = clamp_div(H->g_cols, H->cols);
+    a.ngc = n_grp_cols(H);
+    memcpy(a.lut, lut_tables().gelu_fwd, sizeof(a.lut));
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t ne = (size_t)(n_grp_rows(H) * n_grp_cols(H));
+    if (cudaMemcpyAsync(out->exp, H->exp, ne, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return ICT_ERR_CUDA;
+    KTimer kt(s, KC_GELU, 2.0 * (double)H->rows * (double)H->cols + 2.0 * (double)ne);
+    gelu_lut_fwd_kernel<<<(unsigned)cdiv64(H->rows * (H->cols / 16), 256), 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+int32_t ict_gelu_lut_bwd(const ict_tensor *H, const ict_tensor *dY, ict_tensor *dH, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
+    if ((st = check_tensor(H)) || (st = check_tensor(dY)) || (st = check_tensor(dH))) return st;
+    if (dY->rows != H->rows || dY->cols != H->cols || dH->rows != H->rows || dH->cols != H->cols)
+        return ICT_ERR_INVALID_ARG;
+    if ((H->g_rows != 1 || dY->g_rows != 1 || dH->g_rows != 1) && H->rows > 1) return ICT_ERR_LAYOUT;
+    if (H->g_cols != dY->g_cols || H->g_cols != dH->g_cols) return ICT_ERR_LAYOUT;
+    if ((st = check_pointwise(H)) || (st = check_pointwise(dY)) || (st = check_pointwise(dH))) return st;
+    if (H->rows == 0 || H->cols == 0) return ICT_OK;
+    GeluLutArgs a;
+    memset(&a, 0, offsetof(GeluLutArgs, lut));
+    a.h = H->mant;
+    a.h_exp = H->exp;
+    a.dy = dY->mant;
+    a.dy_exp = dY->exp;
+    a.out = dH->mant;
+    a.out_exp = dH->exp;
+    a.rows = H->rows;
+    a.cols = H->cols;
+    a.ld_h = H->ld;
+    a.ld_dy = dY->ld;
+    a.ld_out = dH->ld;
+    a.g_rows = 1;
+    a.g_cols = clamp_div(H->g_cols, H->cols);
+    a.ngc = n_grp_cols(H);
+    memcpy(a.lut, lut_tables().gelu_bwd, sizeof(a.lut));
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t groups = H->rows * a.ngc;
+    KTimer kt(s, KC_GELU, 3.0 * (double)H->rows * (double)H->cols + 3.0 * (double)groups);
+    gelu_lut_bwd_kernel<<<(unsigned)cdiv64(groups, 8), 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
+int32_t ict_softmax_ce(const ict_tensor *Z, const int32_t *target, int32_t *loss, ict_tensor *dZ, void *stream) {
+    int st;
+    if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
+    if ((st = check_tensor(Z)) || (st = check_tensor(dZ))) return st;
+    if (!target || !loss || dZ->rows != Z->rows || dZ->cols != Z->cols) return ICT_ERR_INVALID_ARG;
+    if (dZ->g_rows != 1 && dZ->rows > 1) return ICT_ERR_LAYOUT;
+    if (Z->rows == 0 || Z->cols == 0) return ICT_OK;
+    HeadArgs a;
+    memset(&a, 0, offsetof(HeadArgs, lut_exp));
+    a.z = Z->mant;
+    a.z_exp = Z->exp;
+    a.rows = Z->rows;
+    a.cols = Z->cols;
+    a.ld_z = Z->ld;
+    a.g_rows = clamp_div(Z->g_rows, Z->rows);
+    a.g_cols = clamp_div(Z->g_cols, Z->cols);
+    a.ngc = n_grp_cols(Z);
+    a.target = target;
+    a.loss = loss;
+    a.dz = dZ->mant;
+    a.dz_exp = dZ->exp;
+    a.ld_dz = dZ->ld;
+    a.gd = clamp_div(dZ->g_cols, dZ->cols);
+    a.ngd = n_grp_cols(dZ);
+    memcpy(a.lut_exp, lut_tables().exp, sizeof(a.lut_exp));
+    memcpy(a.lut_log, lut_tables().log, sizeof(a.lut_log));
+    cudaStream_t s = (cudaStream_t)stream;
+    KTimer kt(s, KC_OTHER, 2.0 * (double)Z->rows * (double)Z->cols + 8.0 * (double)Z->rows);
+    softmax_ce_kernel<<<(unsigned)cdiv64(Z->rows, 8), 256, 0, s>>>(a);
+    counted(1);
+    return launch_status();
+}
+
 int32_t ict_relu_fwd(const ict_tensor *X, int32_t six, ict_tensor *Z, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
     if ((st = check_pointwise(X)) || (st = check_pointwise(Z))) return st;
     if (six != 0 && six != 1) return ICT_ERR_INVALID_ARG;
+    if (six && (st = int8_only())) return st;  // ReLU6's bound min(6 >> e, q_max) is written for INT8
     if (Z->rows != X->rows || Z->cols != X->cols) return ICT_ERR_INVALID_ARG;
     if (!same_groups(X, Z)) return ICT_ERR_LAYOUT;
     return launch_clip(X, nullptr, six, Z, (cudaStream_t)stream);
@@ -1927,6 +2126,7 @@ int32_t ict_relu_fwd(const ict_tensor *X, int32_t six, ict_tensor *Z, void *stre
 int32_t ict_relu_bwd(const ict_tensor *X, const ict_tensor *dY, int32_t six, ict_tensor *dX, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if (six && (st = int8_only())) return st;
     if ((st = check_pointwise(X)) || (st = check_pointwise(dY)) || (st = check_pointwise(dX))) return st;
     if (six != 0 && six != 1) return ICT_ERR_INVALID_ARG;
     if (dY->rows != X->rows || dY->cols != X->cols || dX->rows != X->rows || dX->cols != X->cols)
@@ -1989,6 +2189,7 @@ int32_t ict_depthwise(int32_t dir, const ict_conv_desc *d, const ict_tensor *a, 
                       ict_tensor *out, void *ws, size_t ws_bytes, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
     if (!d || (st = check_tensor(a)) || (st = check_tensor(b)) || (st = check_tensor(out)))
         return d ? st : ICT_ERR_INVALID_ARG;
     if (d->n < 1 || d->h < 1 || d->w < 1 || d->c < 1 || d->k != d->c || d->r < 1 || d->s < 1 || d->stride < 1 ||
@@ -2050,6 +2251,7 @@ int sum_entry(const ict_tensor *X, int32_t x_mul, int32_t x_shift, const ict_ten
               int32_t y_shift, ict_tensor *Z, int act, void *ws, size_t ws_bytes, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
     if (x_mul < -512 || x_mul > 512 || y_mul < -512 || y_mul > 512 || x_shift < 0 || y_shift < 0 ||
         x_shift > 64 || y_shift > 64)
         return ICT_ERR_INVALID_ARG;
@@ -2121,6 +2323,7 @@ int32_t ict_avgpool_fwd(const ict_tensor *X, int32_t n, int32_t h, int32_t w, in
                         size_t ws_bytes, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
     PoolArgs a;
     if ((st = plan_pool(false, X, n, h, w, K, Y, &a))) return st;
     return run_pool(a, ws, ws_bytes, (cudaStream_t)stream);
@@ -2129,6 +2332,7 @@ int32_t ict_avgpool_bwd(const ict_tensor *dY, int32_t n, int32_t h, int32_t w, i
                         size_t ws_bytes, void *stream) {
     int st;
     if ((st = device_info(nullptr))) return st;
+    if ((st = int8_only())) return st;
     PoolArgs a;
     if ((st = plan_pool(true, dY, n, h, w, K, dX, &a))) return st;
     return run_pool(a, ws, ws_bytes, (cudaStream_t)stream);

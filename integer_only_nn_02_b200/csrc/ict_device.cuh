@@ -45,9 +45,22 @@ __device__ __forceinline__ int need_off32(uint32_t a) {
     if (s > 0 && (a >> (s - 1)) == 255u) s += 1;
     return s;
 }
+// The same for B-bit mantissas (|C| <= q_max = 2^(B-1) - 1, Table 4's INT8..INT4):
+// s = bitlen - (B - 1), plus one when the top B bits of a are all ones (a rounds to 2^(B-1)).
+__device__ __forceinline__ int need_off32q(uint32_t a, int bits) {
+    int s = (33 - bits) - __clz(a);
+    if (s > 0 && (a >> (s - 1)) == (1u << bits) - 1u) s += 1;
+    return s;
+}
 __device__ __forceinline__ int need_off64(uint64_t a) {
     int s = 57 - __clzll(a);
     if (s > 0 && (a >> (s - 1)) == 255ull) s += 1;
+    return s;
+}
+
+__device__ __forceinline__ int need_off64q(uint64_t a, int bits) {
+    int s = (65 - bits) - __clzll(a);
+    if (s > 0 && (a >> (s - 1)) == (1ull << bits) - 1ull) s += 1;
     return s;
 }
 
@@ -254,6 +267,67 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
         : "memory");
+}
+
+// ---- pairs of CTAs (a cluster of two) sharing one tcgen05.mma.cta_group::2 tile: CTA r
+// of the pair holds rows [r M/2, (r+1) M/2) of A and [r N/2, (r+1) N/2) of B in its own
+// shared memory and rows [r M/2, (r+1) M/2) of the accumulator in its own TMEM.  Every
+// copy is issued by the CTA that owns the destination, and every completion is signalled
+// on each CTA's barrier by its own arrive.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// arrive (release at cluster scope) on an mbarrier given by its shared::cluster address
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an mbarrier of
+// the pair's first CTA (bar_cluster: a shared::cluster address)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *m, uint32_t bar_cluster, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(m), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (both CTAs' TMEM) (+)= A * B^T for the pair, issued by one thread of the first CTA
+__device__ __forceinline__ void umma_i8_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on an mbarrier of either CTA of the pair (bar_cluster: a shared::cluster address)
+// once every tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+                 : "memory");
 }
 
 // 32 consecutive 32-bit TMEM columns of this thread's lane.

@@ -41,6 +41,10 @@ __device__ __forceinline__ TwoTerm two_term(int64_t a, int pa, int64_t b, int pb
 __device__ __forceinline__ int need64(int64_t x, int r) {
     return x == 0 ? kNoExp : r + need_off64((uint64_t)(x < 0 ? -x : x));
 }
+// the same for B-bit mantissas (q_max = 2^(B-1) - 1)
+__device__ __forceinline__ int need64q(int64_t x, int r, int bits) {
+    return x == 0 ? kNoExp : r + need_off64q((uint64_t)(x < 0 ? -x : x), bits);
+}
 
 template <int L>
 __device__ __forceinline__ int group_max(int v, unsigned mask) {
@@ -91,6 +95,7 @@ struct RequantArgs {
     int8_t *out_exp;
     int G;
     int64_t ngc;  // groups per row
+    int qb;       // mantissa bits B of the FIT (|C| <= 2^(B-1) - 1)
 };
 
 __device__ __forceinline__ int64_t rq_value(const RequantArgs &a, int64_t i, int64_t j) {
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(256) requant_rows_kernel(RequantArgs a) {
     int emax = kNoExp;
     for (int64_t j = j0 + lane; j < j1; j += 32) {
         const int64_t x = rq_value(a, i, j);
-        if (x) emax = max(emax, need64(x, re + (a.col_exp ? a.col_exp[idiv(j, a.col_div)] : 0)));
+        if (x) emax = max(emax, need64q(x, re + (a.col_exp ? a.col_exp[idiv(j, a.col_div)] : 0), a.qb));
     }
     const int e = finalize_exp(warp_max(emax));
     for (int64_t j = j0 + lane; j < j1; j += 32) {
@@ -604,7 +609,7 @@ __global__ void __launch_bounds__(T) requant_group_block_kernel(RequantArgs a) {
             const int64_t j = j0 + jj;
             x[k] = rq_value(a, i, j);
             r[k] = re + (a.col_exp ? a.col_exp[idiv(j, a.col_div)] : 0);
-            if (x[k]) emax = max(emax, need64(x[k], r[k]));
+            if (x[k]) emax = max(emax, need64q(x[k], r[k], a.qb));
         }
     }
     __shared__ int red[T / 32];
@@ -674,10 +679,10 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
                 if (WIDE) {
-                    if (x[k][t]) emax = max(emax, need64((int64_t)x[k][t], r[k][t]));
+                    if (x[k][t]) emax = max(emax, need64q((int64_t)x[k][t], r[k][t], a.qb));
                 } else {
                     const int32_t v = (int32_t)x[k][t];
-                    if (v) emax = max(emax, r[k][t] + need_off32((uint32_t)(v < 0 ? -v : v)));
+                    if (v) emax = max(emax, r[k][t] + need_off32q((uint32_t)(v < 0 ? -v : v), a.qb));
                 }
             }
         }
@@ -736,7 +741,7 @@ __global__ void __launch_bounds__(256) requant_warp_kernel(const __grid_constant
         const int v[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
 #pragma unroll
         for (int t = 0; t < 4; ++t)
-            if (v[t]) emax = max(emax, re + sx8(ce[k], t) + need_off32((uint32_t)(v[t] < 0 ? -v[t] : v[t])));
+            if (v[t]) emax = max(emax, re + sx8(ce[k], t) + need_off32q((uint32_t)(v[t] < 0 ? -v[t] : v[t]), a.qb));
     }
     const int e = finalize_exp(warp_max(emax));
 #pragma unroll
@@ -963,6 +968,10 @@ struct SgdArgs {
     // largest shift of each term at which |term| stays below 2^29 (so every two-term sum
     // is below 2^30): 29 - bitlen(127 |multiplier|)
     int cap_mom, cap_lr;
+    // the same for the fp32 fast path, whose integers must stay below 2^24:
+    // 24 - bitlen(127 |multiplier|)
+    int capf_mom, capf_lr;
+    int qb;  // mantissa bits B of both FITs (|C| <= 2^(B-1) - 1)
     SgdTensor t[kSgdMaxTensors];
 };
 
@@ -978,7 +987,7 @@ __device__ __forceinline__ void sgd_group(const SgdArgs &p, const SgdTensor &t, 
     int emax = kNoExp;
     for (int64_t j = j0 + lane; j < j1; j += 32) {
         const TwoTerm s = two_term((int64_t)p.mom_mul * t.v[i * t.ld + j], pv, t.g[i * t.ld + j], eg);
-        if (s.x) emax = max(emax, need64(s.x, s.r));
+        if (s.x) emax = max(emax, need64q(s.x, s.r, p.qb));
     }
     const int ev2 = finalize_exp(warp_max(emax));
     // weight (recompute the new velocity mantissas element by element)
@@ -988,7 +997,7 @@ __device__ __forceinline__ void sgd_group(const SgdArgs &p, const SgdTensor &t, 
         const TwoTerm s = two_term((int64_t)p.mom_mul * t.v[i * t.ld + j], pv, t.g[i * t.ld + j], eg);
         const int cv = requant64(s.x, s.r, ev2);
         const TwoTerm w = two_term(t.w[i * t.ld + j], ew, -(int64_t)p.lr_mul * cv, pu);
-        if (w.x) emax = max(emax, need64(w.x, w.r));
+        if (w.x) emax = max(emax, need64q(w.x, w.r, p.qb));
     }
     const int ew2 = finalize_exp(warp_max(emax));
     __syncwarp();
@@ -1032,7 +1041,7 @@ __device__ __forceinline__ void sgd_group_exact(const SgdArgs &p, const SgdTenso
     int emax = kNoExp;
     for (int j = li; j < glen; j += L) {
         const TwoTerm x = two_term((int64_t)p.mom_mul * t.v[row0 + j], pv, t.g[row0 + j], eg);
-        if (x.x) emax = max(emax, need64(x.x, x.r));
+        if (x.x) emax = max(emax, need64q(x.x, x.r, p.qb));
     }
     const int ev2 = finalize_exp(group_max<L>(emax, gmask));
     const int pu = ev2 - p.lr_shift;
@@ -1041,7 +1050,7 @@ __device__ __forceinline__ void sgd_group_exact(const SgdArgs &p, const SgdTenso
         const TwoTerm x = two_term((int64_t)p.mom_mul * t.v[row0 + j], pv, t.g[row0 + j], eg);
         const int cv = requant64(x.x, x.r, ev2);
         const TwoTerm w = two_term(t.w[row0 + j], ew, -(int64_t)p.lr_mul * cv, pu);
-        if (w.x) emax = max(emax, need64(w.x, w.r));
+        if (w.x) emax = max(emax, need64q(w.x, w.r, p.qb));
     }
     const int ew2 = finalize_exp(group_max<L>(emax, gmask));
     for (int j = li; j < glen; j += L) {
@@ -1161,7 +1170,7 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
                 lo = min(lo, x[e]);
             }
             const int amax = group_max<L>(max(hi, -lo), gmask);
-            ev2 = finalize_exp(amax ? r1 + need_off32((uint32_t)amax) : kNoExp);
+            ev2 = finalize_exp(amax ? r1 + need_off32q((uint32_t)amax, p.qb) : kNoExp);
             const Shift h = make_shift(ev2 == kEZero ? 0 : ev2 - r1);
             if (__any_sync(gmask, h.ls != 0)) {
 #pragma unroll
@@ -1199,7 +1208,7 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
                 lo = min(lo, y[e]);
             }
             const int amax = group_max<L>(max(hi, -lo), gmask);
-            ew2 = finalize_exp(amax ? r2 + need_off32((uint32_t)amax) : kNoExp);
+            ew2 = finalize_exp(amax ? r2 + need_off32q((uint32_t)amax, p.qb) : kNoExp);
             const Shift h = make_shift(ew2 == kEZero ? 0 : ew2 - r2);
             if (__any_sync(gmask, h.ls != 0)) {
 #pragma unroll
@@ -1249,12 +1258,60 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
 }
 
 // SGD over one dense tensor whose groups are whole rows of exactly 16 * L elements (a
-// parameter arena padded to its group width).  Same arithmetic as sgd_vec_kernel; the
-// next group's W, V, G chunks are loaded before the current group is computed, so each
-// warp keeps a load in flight while it computes.
+// parameter arena padded to its group width).  Each lane holds 16 elements of W, V and G;
+// the next group's chunks are loaded before the current group is computed.
+//
+// The two-term sums and their rounding run as exact integer arithmetic on the fp32 pipe
+// (twice the integer pipes' issue rate).  Per group the terms a * 2^pa and b * 2^pb sit
+// at the common exponent r0 = min(pa, pb); while |a| 2^(pa - r0) and |b| 2^(pb - r0) stay
+// below 2^23 each (shift caps from the multipliers' magnitudes), every sum is an integer
+// below 2^24, so the byte-built operands, the scalings by powers of two and the FMA that
+// adds the terms are all exact.  The group exponent then follows from the largest
+// magnitude (converted to int exactly), and RNE(x / 2^S) is one FMA onto 1.5 * 2^23: its
+// result lies in [2^23, 2^24), where fp32 rounds to the nearest integer with ties to
+// even, so the low byte of its bits is the int8 mantissa.  Groups beyond the caps take
+// the int64 path (sgd_group_exact).
+__device__ __forceinline__ float sx8f(uint32_t w_biased, int b) {
+    // byte b of w (stored with 0x80 added to every byte) as the float C: 2^23 + (C + 128) - (2^23 + 128)
+    return __uint_as_float(__byte_perm(w_biased, 0x4B000000u, 0x7650 | b)) - 8388736.0f;
+}
+// Plan of an exact fp32 two-term sum a * 2^pa + b * 2^pb (|a| < 2^(23 - cap_a),
+// |b| < 2^(23 - cap_b)): both terms at r0 = min(pa, pb), shifted by sa and sb (one of them
+// 0).  When the shifted term would exceed its cap, it is shifted by the cap only and the
+// other term is rounded to odd at 2^k first (k > 0, r0 raised by k): the sum then stays
+// below 2^24, and rounding that sum to nearest at an exponent at least 2 above r0 equals
+// rounding the exact sum (Boldo and Melquiond, IEEE Trans. Computers 57(4), 2008).  An
+// absent term (E_ZERO: all mantissas zero) takes the other's exponent.
+__device__ __forceinline__ void two_term_plan(int pa, bool za, int pb, bool zb, int cap_a, int cap_b, int &r0,
+                                              int &sa, int &sb, int &k) {
+    if (za) pa = pb;
+    if (zb) pb = pa;
+    r0 = min(pa, pb);
+    sa = pa - r0;
+    sb = pb - r0;
+    k = 0;
+    if (sa > cap_a) k = sa - cap_a, sa = cap_a;
+    if (sb > cap_b) k = sb - cap_b, sb = cap_b;
+    r0 += k;
+}
+// v / 2^k rounded to odd (floor, then the sticky bit ORed in), as a float; |v| < 2^22
+__device__ __forceinline__ float ro_float(int v, int k) {
+    k = min(k, 31);
+    const int q = (v >> k) | (int)((v & (int)((1u << k) - 1u)) != 0);
+    return __int_as_float(q + 0x4B400000) - 12582912.0f;
+}
+__device__ __forceinline__ float pow2f(int k) {  // 2^k for -126 <= k <= 127; 0 below
+    return k < -126 ? 0.0f : __int_as_float((k + 127) << 23);
+}
+__device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float d) {
+    return __byte_perm(__byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040),
+                       __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040), 0x5410);
+}
+
 template <int L>
 __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ SgdArgs p) {
     constexpr int GPW = 32 / L;
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
     const int lane = threadIdx.x & 31, sub = lane / L, li = lane % L;
     const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (sub * L));
     const SgdTensor &t0 = p.t[0];
@@ -1283,75 +1340,79 @@ __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ S
             ng4 = *reinterpret_cast<const uint4 *>(tg + at);
             nev = tve[rn], neg = tge[rn], new_ = twe[rn];
         }
-        const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w}, vv[4] = {cv.x, cv.y, cv.z, cv.w},
-                       gv[4] = {cg.x, cg.y, cg.z, cg.w};
-        // velocity
-        int r1, sa1, sb1;
-        bool small1;
-        common_exp(ev - p.mom_shift, ev == kEZero, eg, eg == kEZero, p.cap_mom, 22, r1, sa1, sb1, small1);
-        int r2 = 0, sa2 = 0, sb2 = 0, ev2 = kEZero;
-        bool small2 = false;
-        int x[16];
-        if (small1) {
-            const int ma = p.mom_mul << sa1, mb = 1 << sb1;
-            int hi = 0, lo = 0;
+        // velocity: v = mom * V 2^(ev - mom_shift) + G 2^eg
+        int r1, sa1, sb1, k1;
+        bool fit1;
+        two_term_plan(ev - p.mom_shift, ev == kEZero, eg, eg == kEZero, p.capf_mom, 16, r1, sa1, sb1, k1);
+        int r2 = 0, sa2 = 0, sb2 = 0, k2 = 0, ev2 = kEZero;
+        bool fit2 = false;
+        float vq[16];  // 1.5 * 2^23 + the new velocity mantissas
+        {
+            const uint32_t vb[4] = {cv.x ^ 0x80808080u, cv.y ^ 0x80808080u, cv.z ^ 0x80808080u, cv.w ^ 0x80808080u};
+            const uint32_t gb[4] = {cg.x ^ 0x80808080u, cg.y ^ 0x80808080u, cg.z ^ 0x80808080u, cg.w ^ 0x80808080u};
+            const float ma = (float)(p.mom_mul << sa1), mb = (float)(1 << sb1);
+            float x[16], amax = 0.0f;
+            if (k1 == 0) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                x[e] = sx8(vv[e >> 2], e & 3) * ma + sx8(gv[e >> 2], e & 3) * mb;
-                hi = max(hi, x[e]);
-                lo = min(lo, x[e]);
+                for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, sx8f(gb[e >> 2], e & 3) * mb);
+            } else if (sa1 == 0) {  // G 2^16 dominates: mom * V rounded to odd at 2^k1
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] = __fmaf_rn(sx8f(gb[e >> 2], e & 3), mb, ro_float(sx8(vb[e >> 2] ^ 0x80808080u, e & 3) * p.mom_mul, k1));
+            } else {  // mom * V 2^cap dominates: G rounded to odd at 2^k1
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, ro_float(sx8(gb[e >> 2] ^ 0x80808080u, e & 3), k1));
             }
-            const int amax = group_max<L>(max(hi, -lo), gmask);
-            ev2 = finalize_exp(amax ? r1 + need_off32((uint32_t)amax) : kNoExp);
-            const Shift h = make_shift(ev2 == kEZero ? 0 : ev2 - r1);
-            if (__any_sync(gmask, h.ls != 0)) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) x[e] <<= h.ls;
-            }
-            if (h.rs >= 2) {
-                const int m = 1 << (32 - h.rs);
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+            const int ia = group_max<L>((int)amax, gmask);
+            ev2 = finalize_exp(ia ? r1 + need_off32q((uint32_t)ia, p.qb) : kNoExp);
+            // with a rounded-to-odd term the final shift must be at least 2 bits (it is unless
+            // the dominant term's mantissas are all zero; then the exact path takes the group)
+            fit1 = k1 == 0 || ev2 == kEZero || ev2 - r1 >= 2;
+            const float sc = pow2f(ev2 == kEZero ? 0 : r1 - ev2);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) x[e] = __mulhi(x[e] + h.bias + (__mulhi(x[e], m) & 1), m);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) x[e] = (x[e] + h.bias + (int)bfe_u32((uint32_t)x[e], h.rs, h.om)) >> h.rs;
-            }
-            common_exp(ew, ew == kEZero, ev2 - p.lr_shift, ev2 == kEZero, 22, p.cap_lr, r2, sa2, sb2, small2);
+            for (int e = 0; e < 16; ++e) vq[e] = __fmaf_rn(x[e], sc, kMagic);
+            two_term_plan(ew, ew == kEZero, ev2 - p.lr_shift, ev2 == kEZero, 16, p.capf_lr, r2, sa2, sb2, k2);
         }
-        if (!(small1 && small2)) {
+        float y[16];
+        int ew2 = kEZero;
+        if (fit1) {
+            // weight: w = W 2^ew - lr * V' 2^(ev2 - lr_shift)
+            const uint32_t wb[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u, cw.w ^ 0x80808080u};
+            const float ma = (float)(1 << sa2), mb = (float)(-(p.lr_mul << sb2));
+            float amax = 0.0f;
+            if (k2 == 0) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(vq[e] - kMagic, mb, sx8f(wb[e >> 2], e & 3) * ma);
+            } else if (sa2 == 0) {  // lr * V' dominates: W rounded to odd at 2^k2
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    y[e] = __fmaf_rn(vq[e] - kMagic, mb, ro_float(sx8(wb[e >> 2] ^ 0x80808080u, e & 3), k2));
+            } else {  // W 2^16 dominates: -lr * V' rounded to odd at 2^k2
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    y[e] = __fmaf_rn(sx8f(wb[e >> 2], e & 3), ma,
+                                     ro_float(-p.lr_mul * (__float_as_int(vq[e]) - 0x4B400000), k2));
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(y[e]));
+            const int ia = group_max<L>((int)amax, gmask);
+            ew2 = finalize_exp(ia ? r2 + need_off32q((uint32_t)ia, p.qb) : kNoExp);
+            fit2 = k2 == 0 || ew2 == kEZero || ew2 - r2 >= 2;
+            const float sc = pow2f(ew2 == kEZero ? 0 : r2 - ew2);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(y[e], sc, kMagic);
+        }
+        if (!(fit1 && fit2)) {
             sgd_group_exact<L>(p, t0, r * (16 * L), r, 16 * L, li, gmask);
         } else {
-            const int ma = 1 << sa2, mb = -(p.lr_mul << sb2);
-            int y[16];
-            int hi = 0, lo = 0;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                y[e] = sx8(wv[e >> 2], e & 3) * ma + x[e] * mb;
-                hi = max(hi, y[e]);
-                lo = min(lo, y[e]);
-            }
-            const int amax = group_max<L>(max(hi, -lo), gmask);
-            const int ew2 = finalize_exp(amax ? r2 + need_off32((uint32_t)amax) : kNoExp);
-            const Shift h = make_shift(ew2 == kEZero ? 0 : ew2 - r2);
-            if (__any_sync(gmask, h.ls != 0)) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] <<= h.ls;
-            }
-            if (h.rs >= 2) {
-                const int m = 1 << (32 - h.rs);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = __mulhi(y[e] + h.bias + (__mulhi(y[e], m) & 1), m);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = (y[e] + h.bias + (int)bfe_u32((uint32_t)y[e], h.rs, h.om)) >> h.rs;
-            }
             uint32_t ov[4], ow[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                ov[q] = __byte_perm(__byte_perm(x[4 * q], x[4 * q + 1], 0x0040),
-                                    __byte_perm(x[4 * q + 2], x[4 * q + 3], 0x0040), 0x5410);
-                ow[q] = __byte_perm(__byte_perm(y[4 * q], y[4 * q + 1], 0x0040),
-                                    __byte_perm(y[4 * q + 2], y[4 * q + 3], 0x0040), 0x5410);
+                ov[q] = low_bytes4(vq[4 * q], vq[4 * q + 1], vq[4 * q + 2], vq[4 * q + 3]);
+                ow[q] = low_bytes4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
             }
             const int64_t at = r * (16 * L) + li * 16;
             *reinterpret_cast<uint4 *>(tv + at) = make_uint4(ov[0], ov[1], ov[2], ov[3]);

@@ -80,21 +80,22 @@ struct GemmParams {
     uint32_t stage_tx_bytes;
     uint64_t wait_ns, drain_ns;
     int epi;
+    int qb;         // mantissa bits B of the FIT (|C| <= 2^(B-1) - 1); 8 for INT8
     int epi_split;  // 1: both epilogue warpgroups share every tile, one half of its columns each
     int nwg;        // host only: epilogue warpgroups of the instantiation to launch (2 or 4)
 };
 
-template <int BN, int BK, int STAGES, int NWG = 2>
+template <int BN, int BK, int STAGES, int NWG = 2, bool PAIR = false, int NACC = NWG>
 struct GemmSmem {
     static constexpr int kABytes = 128 * BK;
-    static constexpr int kBBytes = BN * BK;
-    // one TMEM accumulator per epilogue warpgroup
-    static constexpr int kTmemCols = (NWG * BN <= 32) ? 32 : (NWG * BN <= 64) ? 64 : (NWG * BN <= 128) ? 128
-                                   : (NWG * BN <= 256) ? 256 : 512;
-    static_assert(NWG * BN <= 512, "accumulators must fit TMEM");
+    static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK;  // a pair's CTA holds half of B
+    // NACC TMEM accumulators of BN columns
+    static constexpr int kTmemCols = (NACC * BN <= 32) ? 32 : (NACC * BN <= 64) ? 64 : (NACC * BN <= 128) ? 128
+                                   : (NACC * BN <= 256) ? 256 : 512;
+    static_assert(NACC * BN <= 512, "accumulators must fit TMEM");
     static constexpr int kOffB = STAGES * kABytes;
-    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 2*NWG + 2 mbarriers
-    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 2 * NWG + 2) * 8 + 15) / 16 * 16;
+    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 2*NACC + 2 mbarriers
+    static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 2 * NACC + 2) * 8 + 15) / 16 * 16;
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
     static constexpr int kOffRed = kOffCol + NWG * kColInts * 4;  // [NWG][8 groups][4 warps] row-need maxima
@@ -118,21 +119,28 @@ __device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {
     return r;
 }
 
-// Fast epilogue of one output group of 32 columns of an accumulator row, the group on
-// the fast path: y = acc * 2^d_n (d_n = column shift inside the group, |y| < 2^30), the
-// group exponent from max |y|, then one RNE shift.  The multiplies and the high-half
-// multiplies of the rounding shift run on the FMA pipe, leaving compares, the rounding
-// bit and the byte packing to the ALU pipe; TMEM is read once.
-template <bool MUL>  // MUL = false: every column of the group has the same exponent
-__device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
-                                           bool valid, int ea, int64_t grow, int ncol, int gcol) {
-    uint32_t v[32];
-    tmem_ld32(taddr, v);
-    tmem_ld_wait();
+// Fast epilogue of one output group of NC x 32 columns of an accumulator row, the group
+// on the fast path: y = acc * 2^d_n (d_n = column shift inside the group, |y| < 2^30),
+// the group exponent from max |y|, then one RNE shift.  TMEM is read once (all NC chunks
+// issued before a single wait) and the group stays in registers from the largest
+// magnitude to the stores.  The multiplies and the high-half multiplies of the rounding
+// shift run on the FMA pipe, leaving compares, the rounding bit and the packing to the
+// ALU pipe.
+template <bool MUL, int NC>  // MUL = false: every column of the group has the same exponent
+__device__ __forceinline__ void epi_fast(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
+                                         bool valid, int ea, int64_t grow, int ncol, int gcol) {
+    uint32_t v[32 * NC];
+    if constexpr (NC == 2) {
+        tmem_ld64(taddr, *reinterpret_cast<uint32_t(*)[64]>(v));
+        tmem_ld_wait(*reinterpret_cast<uint32_t(*)[64]>(v));
+    } else {
+        tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld_wait();
+    }
     // four independent max / min chains, so that the reductions overlap
     int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int q = 0; q < 32; q += 4) {
+    for (int q = 0; q < 32 * NC; q += 4) {
         int y0 = (int)v[q], y1 = (int)v[q + 1], y2 = (int)v[q + 2], y3 = (int)v[q + 3];
         if (MUL) {
             const int4 m4 = *reinterpret_cast<const int4 *>(colM + q);
@@ -145,20 +153,20 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     }
     const int h = max(max(hi[0], hi[1]), max(hi[2], hi[3])), l = min(min(lo[0], lo[1]), min(lo[2], lo[3]));
     const int amax = valid ? max(h, -l) : 0;
-    const int need = amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp;
+    const int need = amax ? ea + gm + need_off32q((uint32_t)amax, p.qb) : kNoExp;
     const int e = finalize_exp(need);
     // mantissa = RNE(y * 2^-S), S = e - ea - gm uniform over the row's group
     const int S = (e == kEZero) ? 0 : e - ea - gm;
     if (__any_sync(0xffffffffu, valid && S < 0)) {
         const int lm = S < 0 ? (1 << min(-S, 30)) : 1;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = (uint32_t)((int)v[q] * lm);
+        for (int q = 0; q < 32 * NC; ++q) v[q] = (uint32_t)((int)v[q] * lm);
     }
     const int rs = S > 0 ? min(S, 31) : 0;
     if (rs >= 2) {
         const int m = 1 << (32 - rs), bias = (1 << (rs - 1)) - 1;
 #pragma unroll
-        for (int q = 0; q < 32; q += 8) {  // eight elements per stage, stage by stage
+        for (int q = 0; q < 32 * NC; q += 8) {  // eight elements per stage, stage by stage
             int t[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) t[k] = __mulhi((int)v[q + k], m);
@@ -169,7 +177,7 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
         }
     } else if (rs == 1) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 32 * NC; ++q) {
             const int y = (int)v[q];
             v[q] = (uint32_t)((y + ((y >> 1) & 1)) >> 1);
         }
@@ -178,7 +186,7 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     if (valid) {
         int8_t *dst = p.out + grow * p.out_ld + ncol;
 #pragma unroll
-        for (int q = 0; q < 32; q += 16)
+        for (int q = 0; q < 32 * NC; q += 16)
             if (ncol + q < p.N)
                 *reinterpret_cast<uint4 *>(dst + q) = make_uint4(
                     pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
@@ -188,19 +196,117 @@ __device__ __forceinline__ void epi_fast32(const GemmParams &p, uint32_t taddr, 
     }
 }
 
+// The same for a group of NCH x 32 columns read from TMEM twice, 32 columns at a time: the
+// first pass finds the largest magnitude, the second rounds and stores.  Half the
+// registers of the resident form, so that four epilogue warpgroups fit beside the
+// producer and MMA warps.
+template <bool MUL, int NCH>
+__device__ __forceinline__ void epi_two_pass(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
+                                             bool valid, int ea, int64_t grow, int ncol, int gcol) {
+    uint32_t v[32];
+    int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        tmem_ld32(taddr + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+            int y0 = (int)v[q], y1 = (int)v[q + 1], y2 = (int)v[q + 2], y3 = (int)v[q + 3];
+            if (MUL) {
+                const int4 m4 = *reinterpret_cast<const int4 *>(colM + 32 * c + q);
+                y0 *= m4.x, y1 *= m4.y, y2 *= m4.z, y3 *= m4.w;
+            }
+            const int k = (q >> 2) & 3;
+            hi[k] = max(hi[k], max(max(y0, y1), max(y2, y3)));
+            lo[k] = min(lo[k], min(min(y0, y1), min(y2, y3)));
+        }
+    }
+    const int h = max(max(hi[0], hi[1]), max(hi[2], hi[3])), l = min(min(lo[0], lo[1]), min(lo[2], lo[3]));
+    const int amax = valid ? max(h, -l) : 0;
+    const int e = finalize_exp(amax ? ea + gm + need_off32q((uint32_t)amax, p.qb) : kNoExp);
+    const int S = (e == kEZero) ? 0 : e - ea - gm;
+    const bool any_ls = __any_sync(0xffffffffu, valid && S < 0);
+    const int lm = S < 0 ? (1 << min(-S, 30)) : 1;
+    const int rs = S > 0 ? min(S, 31) : 0;
+    const int m = rs >= 2 ? 1 << (32 - rs) : 0, bias = rs ? (1 << (rs - 1)) - 1 : 0;
+    if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
+    int8_t *dst = p.out + grow * p.out_ld + ncol;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        tmem_ld32(taddr + 32 * c, v);
+        tmem_ld_wait();
+        if (MUL || any_ls) {
+#pragma unroll
+            for (int q = 0; q < 32; q += 4) {
+                int4 m4 = make_int4(lm, lm, lm, lm);
+                if (MUL) {
+                    const int4 c4 = *reinterpret_cast<const int4 *>(colM + 32 * c + q);
+                    m4 = make_int4(c4.x * lm, c4.y * lm, c4.z * lm, c4.w * lm);
+                }
+                v[q] = (uint32_t)((int)v[q] * m4.x), v[q + 1] = (uint32_t)((int)v[q + 1] * m4.y);
+                v[q + 2] = (uint32_t)((int)v[q + 2] * m4.z), v[q + 3] = (uint32_t)((int)v[q + 3] * m4.w);
+            }
+        }
+        if (rs >= 2) {
+#pragma unroll
+            for (int q = 0; q < 32; q += 8) {
+                int t[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) t[k] = __mulhi((int)v[q + k], m);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) t[k] = (int)v[q + k] + bias + (t[k] & 1);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[q + k] = (uint32_t)__mulhi(t[k], m);
+            }
+        } else if (rs == 1) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int y = (int)v[q];
+                v[q] = (uint32_t)((y + ((y >> 1) & 1)) >> 1);
+            }
+        }
+        if (valid) {
+#pragma unroll
+            for (int q = 0; q < 32; q += 16)
+                if (ncol + 32 * c + q < p.N)
+                    *reinterpret_cast<uint4 *>(dst + 32 * c + q) = make_uint4(
+                        pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
+                        pack4s((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
+                        pack4s((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
+                        pack4s((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+        }
+    }
+}
+
 // OUTK (compile time, an EpiMode): which epilogue is compiled in -- the row-local FIT
 // (EPI_FIT_ROW), raw int32 partial sums (EPI_I32), or the int16 round-to-odd sums of
 // groups spanning all rows (EPI_RO16) -- so that each kernel keeps a small code footprint
 // in the instruction cache.
-// G32 (compile time, FIT kernels): output groups are 32 columns wide, so only the
-// 32-column fast path and the exact path are compiled in.
+// GC (compile time, FIT kernels): 1 or 2 when output groups are 32 or 64 columns wide and
+// held in registers, 3 when 64-column groups are read from TMEM in two passes (fewer
+// registers), so that only that fast path and the exact path are compiled in; 0 for
+// other widths.
 // NWG (compile time): epilogue warpgroups, each owning one TMEM accumulator (2 or 4).
-template <int BN, int BK, int STAGES, int LOAD, int OUTK, bool G32 = false, int NWG = 2>
+// PAIR (compile time, LOAD_2D): a cluster of two CTAs computes 256 x BN tiles with
+// tcgen05.mma.cta_group::2.  CTA r of the pair loads rows [r 128, r 128 + 128) of the A
+// tile and [r BN/2, r BN/2 + BN/2) of the B tile into its own shared memory; both count
+// their copies on the first CTA's full barrier, whose MMA thread issues the pair's MMAs
+// and commits to both CTAs' barriers; each CTA's epilogue finishes its own 128 rows from
+// its own TMEM and arrives on the first CTA's accumulator-empty barrier.  Per SM this
+// halves the B bytes per multiply-add of a single-CTA 128 x BN tile.
+// Q4 (compile time): four epilogue warpgroups share every tile, one quarter of its columns
+// each, over two double-buffered accumulators (else one accumulator per warpgroup).
+template <int BN, int BK, int STAGES, int LOAD, int OUTK, int GC = 0, int NWG = 2, bool PAIR = false, bool Q4 = false>
 __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
-    using L = GemmSmem<BN, BK, STAGES, NWG>;
-    constexpr int NACC = NWG;
+    static_assert(!Q4 || NWG == 4, "Q4: four epilogue warpgroups");
+    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG>;
+    static_assert(!PAIR || (LOAD == LOAD_2D && BN % 64 == 0), "pairs: 2-D loads, BN a multiple of 64");
+    constexpr int TM = PAIR ? 256 : 128;  // rows of an output tile
+    constexpr int NACC = Q4 ? 2 : NWG;
+    // warpgroups sharing one tile (each takes a contiguous share of its columns)
+    const int wpt = Q4 ? 4 : (p.epi_split ? 2 : 1);
     constexpr bool I32 = OUTK == EPI_I32, RO16 = OUTK == EPI_RO16;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(BK == 128 || BK == 64 || (BK == 256 && LOAD == LOAD_CONV_WGRAD), "BK");
@@ -218,6 +324,11 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     int *sRed = (int *)(smem + L::kOffRed);  // per warpgroup: [group][warp] row-need maxima (RO16)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // pairs: this CTA's rank r and the pair's index; units advance pair by pair
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0;
+    const bool leader = rank == 0;
+    const int cta0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int ctas = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -226,7 +337,8 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         }
         for (int a = 0; a < NACC; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
-            mbar_init(bar_tempty + 8 * a, p.epi_split ? 256 : 128);
+            // pairs: one arrival per epilogue warpgroup of each CTA that handles the tile
+            mbar_init(bar_tempty + 8 * a, PAIR ? 2 * wpt : 128 * wpt);
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_bres, 1);
@@ -238,11 +350,17 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         prefetch_tmap(&tmB);
     }
     if (warp == 2) {
-        tmem_alloc(smem_u32((const void *)&misc[0]), L::kTmemCols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32((const void *)&misc[0]), L::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32((const void *)&misc[0]), L::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();  // both CTAs' barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = (uint32_t)misc[0];
     volatile int *abort_flag = &misc[1];
@@ -266,7 +384,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 for (int kb = 0; kb < p.n_kblk; ++kb)
                     tma_load_2d(sbase + L::kOffB + kb * L::kBBytes, &tmB, bar_bres, kb * BK, 0);
             }
-            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+            for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas) {
                 const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
                 const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
                 const int kb0 = split * p.kblk_per_split;
@@ -284,7 +402,14 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     const uint32_t fb = bar_full + 8 * stage;
                     const uint32_t sa = sbase + stage * L::kABytes;
                     const uint32_t sb = sbase + L::kOffB + stage * L::kBBytes;
-                    if (LOAD == LOAD_2D) {
+                    if (LOAD == LOAD_2D && PAIR) {
+                        // both CTAs' copies complete on the first CTA's full barrier, whose
+                        // one arrival (with the pair's byte count) comes from that CTA
+                        const uint32_t fb0 = mapa_shared(fb, 0);
+                        if (leader) mbar_expect_tx(fb, p.stage_tx_bytes);
+                        tma_load_2d_pair(sa, &tmA, fb0, kb * BK, mt * TM + (int)rank * 128);
+                        tma_load_2d_pair(sb, &tmB, fb0, kb * BK, nt * BN + (int)rank * (BN / 2));
+                    } else if (LOAD == LOAD_2D) {
                         mbar_expect_tx(fb, p.stage_tx_bytes);
                         tma_load_2d(sa, &tmA, fb, kb * BK, mt * 128);
                         tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
@@ -313,16 +438,20 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     if (++stage == STAGES) stage = 0, phase ^= 1;
                 }
             }
-            // drain: every issued copy must land before the CTA may exit
-            for (int s = 0; s < STAGES; ++s)
+            // drain: every issued copy must land before the CTA may exit (pairs: the first
+            // CTA's full barriers count both CTAs' copies, and the second CTA stays until
+            // the closing cluster barrier, which the first passes only after this drain)
+            for (int s = 0; s < STAGES && leader; ++s)
                 if (issued[s]) mbar_wait(bar_full + 8 * s, issued_phase[s], p.drain_ns, nullptr);
             if (bres && blockIdx.x < p.num_units) mbar_wait(bar_bres, 0, p.drain_ns, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && leader) {  // pairs: the first CTA issues the pair's MMAs
             constexpr bool kMN = LOAD == LOAD_CONV_WGRAD;  // both operands MN-major
-            constexpr uint32_t kIdesc = idesc_i8(128, BN, kMN, kMN);
+            constexpr uint32_t kIdesc = idesc_i8(TM, BN, kMN, kMN);
+            // pairs: the second CTA's barrier at the same offset, as a shared::cluster address
+            const uint32_t peer_off = PAIR ? mapa_shared(sbase, 1) - sbase : 0;
             const int kk_per_blk = kMN ? p.wg_kpix / 32 : BK / 32;
             int stage = 0;
             uint32_t phase = 0;
@@ -331,7 +460,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
             if (LOAD == LOAD_CONV && p.b_resident && blockIdx.x < p.num_units &&
                 !mbar_wait(bar_bres, 0, p.wait_ns, abort_flag))
                 fail();
-            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x, ++it) {
+            for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas, ++it) {
                 const int split = u / (p.n_mtiles * p.n_ntiles);
                 const int kb0 = split * p.kblk_per_split;
                 const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
@@ -361,18 +490,33 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         const int bslot = (LOAD == LOAD_CONV && p.b_resident) ? kb : stage;
                         const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + bslot * L::kBBytes, BK);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 32; ++kk)
-                            umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 32; ++kk) {
+                            if constexpr (PAIR)
+                                umma_i8_pair(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                            else
+                                umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     any = true;
-                    umma_commit(bar_empty + 8 * stage);
+                    if constexpr (PAIR) {  // both CTAs' stages are free once the MMAs are done
+                        umma_commit_pair(bar_empty + 8 * stage);
+                        umma_commit_pair(bar_empty + 8 * stage + peer_off);
+                    } else {
+                        umma_commit(bar_empty + 8 * stage);
+                    }
                     if (++stage == STAGES) stage = 0, phase ^= 1;
                 }
                 if (!ok) break;
-                umma_commit(bar_tfull + 8 * acc);
+                if constexpr (PAIR) {
+                    umma_commit_pair(bar_tfull + 8 * acc);
+                    umma_commit_pair(bar_tfull + 8 * acc + peer_off);
+                } else {
+                    umma_commit(bar_tfull + 8 * acc);
+                }
             }
             if (any) {  // drain: all issued MMAs complete before TMEM is released
-                umma_commit(bar_drain);
+                if constexpr (PAIR) umma_commit_pair(bar_drain);
+                else umma_commit(bar_drain);
                 mbar_wait(bar_drain, 0, p.drain_ns, nullptr);
             }
         }
@@ -388,18 +532,19 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         int *gfast = gmin + 8;                     // [8]  group takes the fast path
         const int Gt = p.G >= p.N ? BN : p.G;      // group width inside the tile
         const int ngroups = BN / Gt;
-        // split: every tile, groups [g_lo, g_hi) of it; else every other tile, all groups
-        const int g_lo = p.epi_split ? wg * (ngroups >> 1) : 0;
-        const int g_hi = p.epi_split ? g_lo + (ngroups >> 1) : ngroups;
-        const int c_lo = p.epi_split ? wg * (BN / 2) : 0, c_hi = p.epi_split ? c_lo + BN / 2 : BN;
-        const int u_step = p.epi_split ? gridDim.x : NWG * gridDim.x, it_step = p.epi_split ? 1 : NWG;
-        int it = p.epi_split ? 0 : wg;
+        // the warpgroups form NWG / wpt streams of tiles; within a stream each of the wpt
+        // warpgroups takes groups [g_lo, g_hi) (columns [c_lo, c_hi)) of every tile
+        const int streams = NWG / wpt, stream = wg / wpt, part = wg % wpt;
+        const int g_lo = part * (ngroups / wpt), g_hi = g_lo + ngroups / wpt;
+        const int c_lo = part * (BN / wpt), c_hi = c_lo + BN / wpt;
+        const int u_step = streams * ctas, it_step = streams;
+        int it = stream;
         // The loop never tests the abort flag on its own: the 128 threads decide together
         // through a barrier reduction, so none of them can be left waiting at a barrier.
         // Units are visited as u0, u0 + u_step, ...: their (split, m tile, n tile) advance
         // incrementally, with no division per tile.
         const int NT = p.n_ntiles, MT = p.n_mtiles, T = MT * NT;
-        const int u0 = blockIdx.x + (p.epi_split ? 0 : wg * gridDim.x);
+        const int u0 = cta0 + stream * ctas;
         const int d_split = u_step / T, d_m = (u_step % T) / NT, d_n = (u_step % T) % NT;
         int c_split = u0 / T, c_mt = (u0 % T) / NT, c_nt = (u0 % T) % NT;  // unit being prefetched
         // group of a tile column: shift for power-of-two widths (Gt == BN: always group 0)
@@ -419,8 +564,8 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 pf_rb = ((int64_t)img * p.cv_P + h0) * p.cv_W;
                 pf_vr = min(p.cv_rows, p.cv_P - h0) * p.cv_W;
             } else {
-                pf_rb = (int64_t)c_mt * 128;
-                pf_vr = min(128, p.M - c_mt * 128);
+                pf_rb = (int64_t)c_mt * TM + rank * 128;  // pairs: this CTA's half of the tile
+                pf_vr = max(0, min(128, p.M - (int)pf_rb));
             }
             pf_n0 = c_nt * BN;
             pf_split = c_split;
@@ -594,16 +739,24 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     const int g0 = g * Gt;
                     const int gcol = gcol0 + g;
                     const int gf = gfast[g];
-                    if (G32 && gf) {
+                    if (GC == 3 && gf) {  // 64-column groups, two passes over TMEM
                         if (gf == 2)
-                            epi_fast32<false>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                            epi_two_pass<false, 2>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
                         else
-                            epi_fast32<true>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                            epi_two_pass<true, 2>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                        continue;
+                    }
+                    if (GC && GC < 3 && gf) {
+                        constexpr int NC = GC > 0 && GC < 3 ? GC : 1;
+                        if (gf == 2)
+                            epi_fast<false, NC>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                        else
+                            epi_fast<true, NC>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
                         continue;
                     }
                     const int gm = gmin[g];
                     int e;
-                    if (!G32 && gf) {
+                    if (!GC && gf) {
                         // |x << d| < 2^30: the group exponent follows from the largest magnitude
                         int ymax = 0, ymin = 0;
                         for (int c = g0; c < g0 + Gt; c += 32) {
@@ -621,7 +774,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                             }
                         }
                         const int amax = max(ymax, -ymin);
-                        e = finalize_exp(amax ? ea + gm + need_off32((uint32_t)amax) : kNoExp);
+                        e = finalize_exp(amax ? ea + gm + need_off32q((uint32_t)amax, p.qb) : kNoExp);
                         // mantissa = RNE((x << d) * 2^-S), S = e - ea - gm uniform over the row
                         const int S = (e == kEZero) ? 0 : e - ea - gm;
                         const int ls = S < 0 ? -S : 0;
@@ -673,7 +826,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
 #pragma unroll
                                 for (int q = 0; q < 32; ++q) {
                                     const int32_t x = (int32_t)v[q];
-                                    if (x) emax = max(emax, ea + colE[c + q] + need_off32((uint32_t)(x < 0 ? -x : x)));
+                                    if (x) emax = max(emax, ea + colE[c + q] + need_off32q((uint32_t)(x < 0 ? -x : x), p.qb));
                                 }
                             }
                         }
@@ -701,15 +854,25 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(bar_tempty + 8 * acc);
-            named_bar_sync(bar_id, 128);  // the column tables are rewritten for the next tile
+            if constexpr (PAIR) {
+                // the warpgroup's TMEM reads are done; one thread tells the first CTA
+                named_bar_sync(bar_id, 128);
+                if (et == 0) mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
+            } else {
+                mbar_arrive(bar_tempty + 8 * acc);
+                named_bar_sync(bar_id, 128);  // the column tables are rewritten for the next tile
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();  // the first CTA's MMAs read this CTA's stages and write its TMEM
     tc_fence_after();
-    if (warp == 2) tmem_dealloc(tmem_base, L::kTmemCols);
+    if (warp == 2) {
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, L::kTmemCols);
+        else tmem_dealloc(tmem_base, L::kTmemCols);
+    }
 }
 
 }  // namespace ict

@@ -98,6 +98,12 @@ _SIGS = {
     "ict_depthwise": ([_i32, _P(ict_conv_desc)] + [_P(ict_tensor)] * 3 + [_vp, _sz, _vp], _i32),
     "ict_patchify": ([_P(ict_tensor), _i32, _i32, _i32, _i32, _P(ict_tensor), _vp], _i32),
     "ict_sum_scaled": ([_P(ict_tensor), _i32, _i32, _P(ict_tensor), _i32, _i32, _P(ict_tensor), _vp, _sz, _vp], _i32),
+    "ict_lut_tables": ([_vp, _vp, _vp, _vp], _i32),
+    "ict_set_mantissa_bits": ([_i32], _i32),
+    "ict_get_mantissa_bits": ([], _i32),
+    "ict_gelu_lut_fwd": ([_P(ict_tensor), _P(ict_tensor), _vp], _i32),
+    "ict_gelu_lut_bwd": ([_P(ict_tensor)] * 3 + [_vp], _i32),
+    "ict_softmax_ce": ([_P(ict_tensor), _vp, _vp, _P(ict_tensor), _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -359,6 +365,41 @@ def ict_gelu_bwd(H: DevCE, dG: DevCE, dH: DevCE, stream=None):
            "ict_gelu_bwd")
 
 
+def ict_set_mantissa_bits(bits: int):
+    _check(lib.ict_set_mantissa_bits(int(bits)), "ict_set_mantissa_bits")
+
+
+def ict_get_mantissa_bits() -> int:
+    return int(lib.ict_get_mantissa_bits())
+
+
+def ict_lut_tables():
+    """The library's own lookup tables (host memory): LUT_exp [30][256] uint8, LUT_log
+    [256] uint8, GELU forward and backward [30][256] int8."""
+    ex, lg = np.zeros((30, 256), np.uint8), np.zeros(256, np.uint8)
+    gf, gb = np.zeros((30, 256), np.int8), np.zeros((30, 256), np.int8)
+    _check(lib.ict_lut_tables(ex.ctypes.data, lg.ctypes.data, gf.ctypes.data, gb.ctypes.data), "ict_lut_tables")
+    return {"exp": ex, "log": lg, "gelu_fwd": gf, "gelu_bwd": gb}
+
+
+def ict_gelu_lut_fwd(H: DevCE, out: DevCE, stream=None):
+    ch, co = H.c(), out.c()
+    _check(lib.ict_gelu_lut_fwd(ctypes.byref(ch), ctypes.byref(co), _stream(stream)), "ict_gelu_lut_fwd")
+
+
+def ict_gelu_lut_bwd(H: DevCE, dY: DevCE, dH: DevCE, stream=None):
+    ch, cd, co = H.c(), dY.c(), dH.c()
+    _check(lib.ict_gelu_lut_bwd(ctypes.byref(ch), ctypes.byref(cd), ctypes.byref(co), _stream(stream)),
+           "ict_gelu_lut_bwd")
+
+
+def ict_softmax_ce(Z: DevCE, target: torch.Tensor, loss: torch.Tensor, dZ: DevCE, stream=None):
+    assert target.dtype == torch.int32 and loss.dtype == torch.int32 and target.is_cuda and loss.is_cuda
+    cz, cd = Z.c(), dZ.c()
+    _check(lib.ict_softmax_ce(ctypes.byref(cz), _ptr(target), _ptr(loss), ctypes.byref(cd), _stream(stream)),
+           "ict_softmax_ce")
+
+
 # ----------------------------------------------------------------- conveniences
 
 def ict_relu_fwd(X: DevCE, six: bool, Z: DevCE, stream=None):
@@ -459,6 +500,26 @@ def gelu_bwd(H: DevCE, dG: DevCE, stream=None) -> DevCE:
     dH = DevCE.empty(H.rows, H.cols, 1, H.g_cols)
     ict_gelu_bwd(H, dG, dH, stream)
     return dH
+
+
+def gelu_lut_fwd(H: DevCE, stream=None) -> DevCE:
+    out = DevCE.empty(H.rows, H.cols, H.g_rows, H.g_cols)
+    ict_gelu_lut_fwd(H, out, stream)
+    return out
+
+
+def gelu_lut_bwd(H: DevCE, dY: DevCE, stream=None) -> DevCE:
+    dH = DevCE.empty(H.rows, H.cols, 1, H.g_cols)
+    ict_gelu_lut_bwd(H, dY, dH, stream)
+    return dH
+
+
+def softmax_ce(Z: DevCE, target: torch.Tensor, g_cols: int | None = None, stream=None):
+    """(loss per row, int32 at scale 2^-5; gradient of the summed loss in (1, g_cols) groups)."""
+    loss = torch.empty(Z.rows, dtype=torch.int32, device="cuda")
+    dZ = DevCE.empty(Z.rows, Z.cols, 1, g_cols or Z.cols)
+    ict_softmax_ce(Z, target.to(device="cuda", dtype=torch.int32), loss, dZ, stream)
+    return loss, dZ
 
 
 def device_status(stream=None) -> int:

@@ -69,3 +69,15 @@ def test_conv_workspace():
     d = ict.conv_desc(dict(n=4, h=56, w=56, c=64, k=64, r=3, s=3, stride=1, pad=1))
     for direction in (0, 1, 2):
         assert ict.lib.ict_conv_workspace(direction, ctypes.byref(d)) > 0
+
+
+def test_library_lookup_tables_equal_the_oracles():
+    """The library builds its lookup tables (Tables 7 and 8) on the host, independently
+    of the oracle (long double libm against 90-digit decimals); every entry agrees."""
+    import numpy as np
+
+    from oracle import luts
+
+    mine, ref = ict.ict_lut_tables(), luts.tables()
+    for name in ("exp", "log", "gelu_fwd", "gelu_bwd"):
+        assert mine[name].shape == ref[name].shape and np.array_equal(mine[name], ref[name]), name
