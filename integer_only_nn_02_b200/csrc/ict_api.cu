@@ -449,7 +449,7 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
     auto run = [&](auto k, int nwg, int smem_bytes) {
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
             return (int)ICT_ERR_CUDA;
-        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, p);
+        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, tb, p);  // no staged output: tmY unused
         counted(1);
         return launch_status();
     };
@@ -482,9 +482,10 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
 // the cluster dimension; each CTA holds half of every B stage, so it has room for the
 // stages of a BN / 2 tile.
 template <int BN>
-int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid,
-                       cudaStream_t s) {
+int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, const GemmParams &p,
+                       int grid, cudaStream_t s) {
     constexpr int ST = stages_for(BN / 2, 128);
+    constexpr int ST4 = 5;  // four epilogue warpgroups stage 32 KB of output: one stage fewer
     auto run = [&](auto k, int smem_bytes, int nwg) {
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
             return (int)ICT_ERR_CUDA;
@@ -501,7 +502,7 @@ int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmP
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, k, ta, tb, p) != cudaSuccess) return (int)ICT_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, k, ta, tb, ty, p) != cudaSuccess) return (int)ICT_ERR_CUDA;
         counted(1);
         return launch_status();
     };
@@ -512,9 +513,9 @@ int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmP
     if constexpr (BN == 256) {
         // 32- and 64-column groups on 256-wide tiles: four epilogue warpgroups, a quarter of
         // the columns each
-        constexpr int kB4 = GemmSmem<BN, 128, ST, 4, true, 2>::kBytes;
-        if (gt == 32) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 1, 4, true, true>, kB4, 4);
-        if (gt == 64) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 3, 4, true, true>, kB4, 4);
+        constexpr int kB4 = GemmSmem<BN, 128, ST4, 4, true, 2, 128 * 64>::kBytes;
+        if (gt == 32) return run(gemm_ce_kernel<BN, 128, ST4, LOAD_2D, EPI_FIT_ROW, 1, 4, true, true>, kB4, 4);
+        if (gt == 64) return run(gemm_ce_kernel<BN, 128, ST4, LOAD_2D, EPI_FIT_ROW, 3, 4, true, true>, kB4, 4);
     }
     if (gt == 32) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 1, 2, true>, kB, 2);
     if (gt == 64) return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 2, 2, true>, kB, 2);
@@ -522,7 +523,8 @@ int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmP
 }
 
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
-                const GemmParams &p_in, int grid, cudaStream_t s, double ops, bool pair = false) {
+                const GemmParams &p_in, int grid, cudaStream_t s, double ops, bool pair = false,
+                const CUtensorMap *ty = nullptr) {
     KTimer kt(s, KC_GEMM, ops);
     // both epilogue warpgroups take every tile (one column half each) when no output
     // group straddles the halves
@@ -532,9 +534,10 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0));
     if (pair) {
         if (load != LOAD_2D || bk != 128 || (grid & 1)) return ICT_ERR_LAYOUT;
-        if (bn == 128) return launch_gemm_pair_t<128>(ta, tb, p, grid, s);
-        if (bn == 192) return launch_gemm_pair_t<192>(ta, tb, p, grid, s);
-        if (bn == 256) return launch_gemm_pair_t<256>(ta, tb, p, grid, s);
+        const CUtensorMap &y = ty ? *ty : tb;  // the output map, for staged stores
+        if (bn == 128) return launch_gemm_pair_t<128>(ta, tb, y, p, grid, s);
+        if (bn == 192) return launch_gemm_pair_t<192>(ta, tb, y, p, grid, s);
+        if (bn == 256) return launch_gemm_pair_t<256>(ta, tb, y, p, grid, s);
         return ICT_ERR_LAYOUT;
     }
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
@@ -695,6 +698,10 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     if ((st = tmap_2d(&ta, A.mant, K, M, A.ld, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return st;
     if ((st = tmap_2d(&tb, B.mant, K, N, B.ld, 128, pl.pair ? pl.bn / 2 : pl.bn, CU_TENSOR_MAP_SWIZZLE_128B)))
         return st;
+    // pairs with a fused FIT: the output as 64 x 128 boxes (64-byte swizzle) for staged stores
+    CUtensorMap ty;
+    const bool staged = pl.pair && pl.fused;
+    if (staged && (st = tmap_2d(&ty, out->mant, N, M, out->ld, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))) return st;
     GemmParams p;
     memset(&p, 0, sizeof(p));
     p.M = (int)M;
@@ -725,7 +732,7 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     p.qb = g_mantissa_bits.load(std::memory_order_relaxed);
     p.nwg = pl.nwg;
     if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K,
-                          pl.pair)))
+                          pl.pair, staged ? &ty : nullptr)))
         return st;
     if (pl.fused) return ICT_OK;
     if (raw_acc) return launch_sum_slices(pl, M, N, raw_acc, raw_bits, raw_ld, s);

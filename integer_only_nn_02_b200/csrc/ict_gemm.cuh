@@ -85,7 +85,7 @@ struct GemmParams {
     int nwg;        // host only: epilogue warpgroups of the instantiation to launch (2 or 4)
 };
 
-template <int BN, int BK, int STAGES, int NWG = 2, bool PAIR = false, int NACC = NWG>
+template <int BN, int BK, int STAGES, int NWG = 2, bool PAIR = false, int NACC = NWG, int STAGE = 0>
 struct GemmSmem {
     static constexpr int kABytes = 128 * BK;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK;  // a pair's CTA holds half of B
@@ -99,7 +99,9 @@ struct GemmSmem {
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
     static constexpr int kOffRed = kOffCol + NWG * kColInts * 4;  // [NWG][8 groups][4 warps] row-need maxima
-    static constexpr int kBytes = kOffRed + NWG * 32 * 4 + 1024;    // + alignment slack
+    // STAGE bytes per epilogue warpgroup of output staged for a TMA store (1024-aligned)
+    static constexpr int kOffStage = (kOffRed + NWG * 32 * 4 + 1023) / 1024 * 1024;
+    static constexpr int kBytes = kOffStage + NWG * STAGE + 1024;  // + alignment slack
     static_assert(kOffCol % 16 == 0 && (kColInts * 4) % 16 == 0 && (BN * 4) % 16 == 0,
                   "column tables are read as int4");
     static_assert(kABytes % 1024 == 0 && kBBytes % 512 == 0 && kOffB % 1024 == 0 && kABytes / 2 <= 16383 * 16,
@@ -126,9 +128,18 @@ __device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {
 // magnitude to the stores.  The multiplies and the high-half multiplies of the rounding
 // shift run on the FMA pipe, leaving compares, the rounding bit and the packing to the
 // ALU pipe.
-template <bool MUL, int NC>  // MUL = false: every column of the group has the same exponent
+// Output stores: straight to global memory, or (TS) into the warpgroup's staging rows,
+// 64 bytes per output row with the 16-byte chunks in the TMA store's 64-byte swizzle order
+// (chunk ^ ((row >> 1) & 3)), which also keeps the row-per-thread writes free of bank
+// conflicts.  scol: the chunk's first column within the warpgroup's 64.
+__device__ __forceinline__ void stage16(uint8_t *srow, int et, int scol, uint4 v) {
+    *reinterpret_cast<uint4 *>(srow + (((scol >> 4) ^ ((et >> 1) & 3)) << 4)) = v;
+}
+
+template <bool MUL, int NC, bool TS = false>  // MUL = false: every column of the group has the same exponent
 __device__ __forceinline__ void epi_fast(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
-                                         bool valid, int ea, int64_t grow, int ncol, int gcol) {
+                                         bool valid, int ea, int64_t grow, int ncol, int gcol,
+                                         uint8_t *srow = nullptr, int et = 0, int scol = 0) {
     uint32_t v[32 * NC];
     if constexpr (NC == 2) {
         tmem_ld64(taddr, *reinterpret_cast<uint32_t(*)[64]>(v));
@@ -183,16 +194,17 @@ __device__ __forceinline__ void epi_fast(const GemmParams &p, uint32_t taddr, co
         }
     }
     if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
-    if (valid) {
+    if (TS || valid) {
         int8_t *dst = p.out + grow * p.out_ld + ncol;
 #pragma unroll
-        for (int q = 0; q < 32 * NC; q += 16)
-            if (ncol + q < p.N)
-                *reinterpret_cast<uint4 *>(dst + q) = make_uint4(
-                    pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
-                    pack4s((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
-                    pack4s((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
-                    pack4s((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+        for (int q = 0; q < 32 * NC; q += 16) {
+            const uint4 w = make_uint4(pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
+                                       pack4s((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
+                                       pack4s((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
+                                       pack4s((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+            if (TS) stage16(srow, et, scol + q, w);
+            else if (ncol + q < p.N) *reinterpret_cast<uint4 *>(dst + q) = w;
+        }
     }
 }
 
@@ -200,9 +212,10 @@ __device__ __forceinline__ void epi_fast(const GemmParams &p, uint32_t taddr, co
 // first pass finds the largest magnitude, the second rounds and stores.  Half the
 // registers of the resident form, so that four epilogue warpgroups fit beside the
 // producer and MMA warps.
-template <bool MUL, int NCH>
+template <bool MUL, int NCH, bool TS = false>
 __device__ __forceinline__ void epi_two_pass(const GemmParams &p, uint32_t taddr, const int *colM, int gm,
-                                             bool valid, int ea, int64_t grow, int ncol, int gcol) {
+                                             bool valid, int ea, int64_t grow, int ncol, int gcol,
+                                             uint8_t *srow = nullptr, int et = 0, int scol = 0) {
     uint32_t v[32];
     int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -265,15 +278,16 @@ __device__ __forceinline__ void epi_two_pass(const GemmParams &p, uint32_t taddr
                 v[q] = (uint32_t)((y + ((y >> 1) & 1)) >> 1);
             }
         }
-        if (valid) {
+        if (TS || valid) {
 #pragma unroll
-            for (int q = 0; q < 32; q += 16)
-                if (ncol + 32 * c + q < p.N)
-                    *reinterpret_cast<uint4 *>(dst + 32 * c + q) = make_uint4(
-                        pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
-                        pack4s((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
-                        pack4s((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
-                        pack4s((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+            for (int q = 0; q < 32; q += 16) {
+                const uint4 w = make_uint4(pack4s((int)v[q], (int)v[q + 1], (int)v[q + 2], (int)v[q + 3]),
+                                           pack4s((int)v[q + 4], (int)v[q + 5], (int)v[q + 6], (int)v[q + 7]),
+                                           pack4s((int)v[q + 8], (int)v[q + 9], (int)v[q + 10], (int)v[q + 11]),
+                                           pack4s((int)v[q + 12], (int)v[q + 13], (int)v[q + 14], (int)v[q + 15]));
+                if (TS) stage16(srow, et, scol + 32 * c + q, w);
+                else if (ncol + 32 * c + q < p.N) *reinterpret_cast<uint4 *>(dst + 32 * c + q) = w;
+            }
         }
     }
 }
@@ -296,12 +310,18 @@ __device__ __forceinline__ void epi_two_pass(const GemmParams &p, uint32_t taddr
 // halves the B bytes per multiply-add of a single-CTA 128 x BN tile.
 // Q4 (compile time): four epilogue warpgroups share every tile, one quarter of its columns
 // each, over two double-buffered accumulators (else one accumulator per warpgroup).
+// With Q4 on pairs (TS), each epilogue warpgroup stages its 128 x 64 share of a tile's
+// int8 output in shared memory and one of its threads writes it with a TMA store through
+// tmY (the output, 64-byte swizzle, 64 x 128 boxes), instead of 16-byte stores that each
+// touch 32 rows.
 template <int BN, int BK, int STAGES, int LOAD, int OUTK, int GC = 0, int NWG = 2, bool PAIR = false, bool Q4 = false>
 __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmParams p) {
     static_assert(!Q4 || NWG == 4, "Q4: four epilogue warpgroups");
-    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG>;
+    constexpr bool TS = PAIR && Q4 && OUTK == EPI_FIT_ROW;
+    static_assert(!TS || BN == 256, "staged stores: 64 columns per warpgroup");
+    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * 64 : 0>;
     static_assert(!PAIR || (LOAD == LOAD_2D && BN % 64 == 0), "pairs: 2-D loads, BN a multiple of 64");
     constexpr int TM = PAIR ? 256 : 128;  // rows of an output tile
     constexpr int NACC = Q4 ? 2 : NWG;
@@ -322,6 +342,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     volatile int *misc = (volatile int *)(smem + L::kOffMisc);  // [0] tmem base, [1] abort
     int *sCol = (int *)(smem + L::kOffCol);  // per epilogue warpgroup column tables
     int *sRed = (int *)(smem + L::kOffRed);  // per warpgroup: [group][warp] row-need maxima (RO16)
+    uint8_t *sStage = smem + L::kOffStage;  // TS: per warpgroup, 128 rows x 64 bytes of output
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // pairs: this CTA's rank r and the pair's index; units advance pair by pair
@@ -348,6 +369,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        if (TS) prefetch_tmap(&tmY);
     }
     if (warp == 2) {
         if constexpr (PAIR) {
@@ -602,6 +624,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     if (BN > 128) cmin[4 + wq] = lo1, cmax[4 + wq] = hi1;
                 }
             }
+            if (TS && et == 0) bulk_wait_read();  // the previous tile's store has read the staging rows
             named_bar_sync(bar_id, 128);
             auto group_range = [&](int g, int &lo, int &hi) {
                 lo = 0x7fffffff, hi = kNoExp;
@@ -628,6 +651,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
             tc_fence_after();
 
             const bool valid = et < valid_rows;
+            uint8_t *srow = sStage + wg * (128 * 64) + et * 64;  // TS: this thread's staged output row
             const int64_t grow = row_base + et;
             const int ea = valid ? ea_pf : 0;
             const int gcol0 = n0 / p.G;  // output group of the tile's first column
@@ -741,17 +765,21 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     const int gf = gfast[g];
                     if (GC == 3 && gf) {  // 64-column groups, two passes over TMEM
                         if (gf == 2)
-                            epi_two_pass<false, 2>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                            epi_two_pass<false, 2, TS>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol,
+                                                       srow, et, g0 - c_lo);
                         else
-                            epi_two_pass<true, 2>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                            epi_two_pass<true, 2, TS>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol,
+                                                      srow, et, g0 - c_lo);
                         continue;
                     }
                     if (GC && GC < 3 && gf) {
                         constexpr int NC = GC > 0 && GC < 3 ? GC : 1;
                         if (gf == 2)
-                            epi_fast<false, NC>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                            epi_fast<false, NC, TS>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol,
+                                                    srow, et, g0 - c_lo);
                         else
-                            epi_fast<true, NC>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol);
+                            epi_fast<true, NC, TS>(p, taddr + g0, colD + g0, gmin[g], valid, ea, grow, n0 + g0, gcol,
+                                                   srow, et, g0 - c_lo);
                         continue;
                     }
                     const int gm = gmin[g];
@@ -834,7 +862,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         for (int c = g0; c < g0 + Gt; c += 32) {
                             tmem_ld32(taddr + c, v);
                             tmem_ld_wait();
-                            if (valid) {
+                            if (TS || valid) {
                                 uint32_t w[8];
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
@@ -842,11 +870,16 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                                                   requant32((int32_t)v[4 * q + 1], ea + colE[c + 4 * q + 1], e),
                                                   requant32((int32_t)v[4 * q + 2], ea + colE[c + 4 * q + 2], e),
                                                   requant32((int32_t)v[4 * q + 3], ea + colE[c + 4 * q + 3], e));
-                                int8_t *dst = p.out + grow * p.out_ld + n0 + c;
-                                if (n0 + c < p.N)
-                                    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-                                if (n0 + c + 16 < p.N)
-                                    *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                                if constexpr (TS) {
+                                    stage16(srow, et, c - c_lo, make_uint4(w[0], w[1], w[2], w[3]));
+                                    stage16(srow, et, c - c_lo + 16, make_uint4(w[4], w[5], w[6], w[7]));
+                                } else {
+                                    int8_t *dst = p.out + grow * p.out_ld + n0 + c;
+                                    if (n0 + c < p.N)
+                                        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                                    if (n0 + c + 16 < p.N)
+                                        *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                                }
                             }
                         }
                     }
@@ -854,15 +887,24 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 }
             }
             tc_fence_before();
+            if constexpr (TS) fence_proxy_async();  // the staged rows, for the TMA store
             if constexpr (PAIR) {
-                // the warpgroup's TMEM reads are done; one thread tells the first CTA
+                // the warpgroup's TMEM reads are done; one thread tells the first CTA (and,
+                // with staged output, stores the warpgroup's share of the tile)
                 named_bar_sync(bar_id, 128);
-                if (et == 0) mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
+                if (et == 0) {
+                    if (TS && valid_rows > 0) {
+                        tma_store_2d(&tmY, smem_u32(sStage + wg * (128 * 64)), n0 + c_lo, (int)row_base);
+                        bulk_commit();
+                    }
+                    mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
+                }
             } else {
                 mbar_arrive(bar_tempty + 8 * acc);
                 named_bar_sync(bar_id, 128);  // the column tables are rewritten for the next tile
             }
         }
+        if (TS && et == 0) bulk_wait_all();  // every staged store complete before the CTA exits
     }
 
     tc_fence_before();

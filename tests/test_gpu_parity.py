@@ -135,6 +135,35 @@ def test_linear_bwd_weight(ict, case, per_row):
     status_ok(ict)
 
 
+@pytest.mark.parametrize("M,N,K,G,wspan", [
+    (2600, 768, 256, 64, (-12, -6)),     # 128-wide pair tiles; the last tile's second CTA has no rows
+    (2100, 512, 1536, 32, (-12, -6)),    # 32-column groups, a long contraction
+    (2048, 704, 384, 64, (-12, -6)),     # a ragged last N tile
+    (3000, 512, 256, 128, (-12, -6)),    # 128-column groups (generic epilogue on pairs)
+    (2300, 512, 256, 64, (-40, -6)),     # column exponents far apart: the exact per-element path
+    (4200, 1024, 256, 64, (-12, -6)),    # 256-wide pair tiles, four epilogue warpgroups, TMA-store output
+    (4100, 1024, 1280, 32, (-12, -6)),   # the same with 32-column groups; ragged last M tile
+    (4160, 1024, 384, 64, (-40, -6)),    # staged output from the exact per-element path
+])
+def test_linear_pair_tiles(ict, M, N, K, G, wspan):
+    """Products large enough to run on pairs of CTAs (256-row tiles, tcgen05 cta_group::2)
+    against the oracle; on 256-wide tiles the FIT epilogue stages its output in shared
+    memory and writes it with TMA stores."""
+    rng = np.random.default_rng(M + N + K + G)
+    X = rand_ce(rng, M, K, 1, 64, elo=-10, ehi=-4, zero_groups=0.05)
+    W = rand_ce(rng, N, K, 1, K, elo=wspan[0], ehi=wspan[1], zero_groups=0.05)
+    dY = with_groups(clipped_laplace(rng, (M, N)), 1, 32, lambda g: rng.integers(-16, -10, size=g))
+    same(ict.linear_fwd(ict.DevCE.from_host(X), ict.DevCE.from_host(W), G).to_host(), oracle.linear_fwd(X, W, 1, G),
+         "pair fwd")
+    Wt = rand_ce(rng, N, K, 1, 64, elo=wspan[0], ehi=wspan[1])
+    same(ict.linear_bwd_data(ict.DevCE.from_host(dY), ict.DevCE.from_host(Wt), G).to_host(),
+         oracle.linear_bwd_data(dY, Wt, 1, G), "pair bwd-data")
+    # the weight gradient (N output rows: single CTAs, split-K) of the same operands
+    dW = ict.linear_bwd_weight(ict.DevCE.from_host(dY), ict.DevCE.from_host(X)).to_host()
+    same(dW, oracle.linear_bwd_weight(dY, X, 1, K), "bwd-weight")
+    status_ok(ict)
+
+
 def test_linear_long_contraction_int64(ict):
     """K far beyond 2^17 products of 127^2: split-K int32 partials, int64 combine."""
     rng = np.random.default_rng(77)
