@@ -252,6 +252,11 @@ AlignLaunch plan_align(const AlignJob &j, int sms) {
     a.out = j.out;
     a.out_ld = j.ld;
     a.e_star = j.e_star;
+    {
+        const int64_t gv = a.g_cols / 16;
+        if (a.ngc == 1) a.gv_shift1 = 32;
+        else if (a.g_cols % 16 == 0 && (gv & (gv - 1)) == 0) a.gv_shift1 = __builtin_ctzll((unsigned long long)gv) + 1;
+    }
     L.n_exp = n_grp_rows(in) * a.ngc;
     L.blocks = L.used = 0;
     if (j.given) {  // targets fixed by the caller: no e* pass, the shift kernel reads e_star
@@ -264,9 +269,10 @@ AlignLaunch plan_align(const AlignJob &j, int sms) {
     } else {
         // every thread of the scratch form keeps one group column: a stride that is a
         // multiple of ngc
-        L.blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(L.n_exp, 256 * 4), (int64_t)sms * 4));
-        L.used = (L.blocks * 256) / a.ngc * a.ngc;
-        L.estar = (j.col_max && a.ngc <= 8192 && L.used >= a.ngc) ? 2 : 3;
+        // one block per SM at most, each reducing a band of at least 32 group rows
+        L.blocks = std::max<int64_t>(1, std::min<int64_t>(cdiv64(n_grp_rows(in), 32), (int64_t)sms));
+        L.used = L.blocks * 256;
+        L.estar = (j.col_max && a.ngc <= 8192) ? 2 : 3;
         if (j.transpose && in->rows <= 4096 && a.g_cols >= 16) {
             L.estar = 0;  // few rows (a weight): each transposing block scans its columns' exponents
             a.col_scan = 1;
@@ -274,6 +280,70 @@ AlignLaunch plan_align(const AlignJob &j, int sms) {
         if (L.estar == 2) a.col_max = j.col_max;
     }
     return L;
+}
+
+// Tiles of the transposing kernels for the first n jobs of P (job 0's tiles first);
+// fills P.tiles0, P.tiles1 and P.ntc.
+unsigned transpose_tiles(AlignPair &P, int n) {
+    int64_t t[2];
+    for (int z = 0; z < 2; ++z) {
+        const int64_t tc = z < n ? cdiv64(P.a[z].cols, 128) : 1, tr = z < n ? cdiv64(P.a[z].rows, 128) : 0;
+        P.ntc[z] = (int)tc;
+        t[z] = tc * tr;
+    }
+    P.tiles0 = (int)t[0];
+    P.tiles1 = (int)t[1];
+    return (unsigned)(t[0] + t[1]);
+}
+
+// The transposing alignment of the first n jobs of P: persistent streaming blocks (three
+// per SM) unless a job scans its own column exponents, then one block per tile.
+void launch_align_transpose(AlignPair &P, int n, int sms, cudaStream_t s) {
+    const unsigned tiles = transpose_tiles(P, n);
+    const bool scan = P.a[0].col_scan || (n > 1 && P.a[1].col_scan);
+    if (scan)
+        align_transpose_kernel<<<tiles, 256, 0, s>>>(P);
+    else
+        align_transpose_stream_kernel<<<std::min<unsigned>(tiles, (unsigned)sms * 3), 256, 0, s>>>(P);
+}
+
+// Rows of 16-byte vectors, one row per segment of L lanes.  The narrowest segment whose
+// lanes hold at most six vectors each (the most bytes in flight per lane) and stay nine
+// tenths busy, else the busiest; NV = the row's vectors per lane rounded up to an
+// instantiated count.  Rows of more than 192 vectors or (computing e*) more than 2 L
+// groups, and 2^31 rows or more, go to the generic kernel.  Persistent grid: two blocks
+// per SM.
+int launch_align_rows(const AlignArgs &a, cudaStream_t s, int sms) {
+    const int64_t vpr = a.cols / 16;
+    const bool row_e = a.axis == 1 && a.row_estar;
+    int L = 0;
+    double best = -1.0;
+    for (int l : {8, 16, 32}) {
+        const int64_t per = cdiv64(vpr, l);
+        if (per > 6 || (row_e && a.ngc > 2 * l)) continue;
+        const double eff = (double)vpr / (double)(l * per);
+        if (eff >= 0.9) { L = l; break; }
+        if (eff > best + 1e-12) best = eff, L = l;
+    }
+    if (L == 0 || a.rows >= (1ll << 31)) {
+        align_rows_wide_kernel<<<dim3((unsigned)cdiv64(a.cols, 256), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);
+        return ICT_OK;
+    }
+    const int64_t per = cdiv64(vpr, L);
+    const int nv = per <= 2 ? 2 : per <= 3 ? 3 : per <= 4 ? 4 : 6;
+    const bool exact = a.axis == 1 && a.g_rows == 1 && a.gv_shift1 > 0 && vpr == (int64_t)L * nv;
+    const unsigned grid = (unsigned)std::min<int64_t>(cdiv64(a.rows, 256 / L), (int64_t)sms * 2);
+#define ICT_ALIGN_ROWS(L_, NV_)                                                             \
+    if (L == L_ && nv == NV_)                                                              \
+        return exact ? (align_rows_kernel<L_, NV_, true><<<grid, 256, 0, s>>>(a), ICT_OK) \
+                     : (align_rows_kernel<L_, NV_, false><<<grid, 256, 0, s>>>(a), ICT_OK);
+#define ICT_ALIGN_ROWS_L(L_) ICT_ALIGN_ROWS(L_, 2) ICT_ALIGN_ROWS(L_, 3) ICT_ALIGN_ROWS(L_, 4) ICT_ALIGN_ROWS(L_, 6)
+    ICT_ALIGN_ROWS_L(32)
+    ICT_ALIGN_ROWS_L(16)
+    ICT_ALIGN_ROWS_L(8)
+#undef ICT_ALIGN_ROWS_L
+#undef ICT_ALIGN_ROWS
+    return ICT_ERR_LAYOUT;
 }
 
 // One or two alignment jobs; two jobs must both be transposing column alignments with
@@ -297,8 +367,7 @@ int launch_align_n(const AlignJob *jobs, int n, cudaStream_t s) {
     int launches = 0;
     if (n == 2 && jobs[0].given && jobs[1].given && jobs[0].transpose && jobs[1].transpose) {
         KTimer kt(s, KC_ALIGN, align_work);
-        const int64_t cols = std::max(L[0].a.cols, L[1].a.cols), rows = std::max(L[0].a.rows, L[1].a.rows);
-        align_transpose_kernel<<<dim3((unsigned)cdiv64(cols, 128), (unsigned)cdiv64(rows, 128), 2), 256, 0, s>>>(P);
+        launch_align_transpose(P, 2, sms, s);
         counted(1);
         return launch_status();
     }
@@ -317,8 +386,7 @@ int launch_align_n(const AlignJob *jobs, int n, cudaStream_t s) {
                                         (size_t)ngc * 4, s>>>(P);
         }
         KTimer kt(s, KC_ALIGN, align_work);
-        const int64_t cols = std::max(L[0].a.cols, L[1].a.cols), rows = std::max(L[0].a.rows, L[1].a.rows);
-        align_transpose_kernel<<<dim3((unsigned)cdiv64(cols, 128), (unsigned)cdiv64(rows, 128), 2), 256, 0, s>>>(P);
+        launch_align_transpose(P, 2, sms, s);
         counted(2);
         return launch_status();
     }
@@ -340,9 +408,9 @@ int launch_align_n(const AlignJob *jobs, int n, cudaStream_t s) {
     }
     KTimer kt(s, KC_ALIGN, align_work);
     if (jobs[0].transpose)
-        align_transpose_kernel<<<dim3((unsigned)cdiv64(a.cols, 128), (unsigned)cdiv64(a.rows, 128)), 256, 0, s>>>(P);
-    else
-        align_rows_kernel<<<dim3((unsigned)cdiv64(a.cols, 256), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);
+        launch_align_transpose(P, 1, sms, s);
+    else if (int st = launch_align_rows(a, s, sms))
+        return st;
     counted(launches + 1);
     return launch_status();
 }

@@ -141,6 +141,8 @@ struct AlignArgs {
     const int32_t *col_max;   // axis 0 with scratch: max per group column (<= kNoExp: none)
     int row_estar;            // axis 1: the alignment kernel computes and stores e* itself
     int col_scan;             // axis 0, transposed: each block finds its columns' e* itself
+    int gv_shift1;            // log2(g_cols / 16) + 1 when that is a power of two, 32 for one
+                              // group across the row, 0: the group of a vector is a division
 };
 
 __device__ __forceinline__ int estar_of(int m) { return m <= kNoExp ? kEZero : m; }
@@ -178,74 +180,109 @@ __global__ void __launch_bounds__(256) estar_cols_kernel(AlignArgs a) {
     }
 }
 
-// e* per column with an int32 scratch (pre-set to 0x80808080): every thread keeps one
-// group column (the grid stride is a multiple of the group-column count), reduces its
-// strided slice of the exponent grid in a register, then one atomicMax in shared and
-// one in global memory.
+// e* per column with an int32 scratch (pre-set to 0x80808080): each block reduces a band
+// of group rows into a shared maximum per group column, then one atomicMax per group
+// column in global memory.
 // Up to two alignment jobs per launch (blockIdx.y or blockIdx.z selects the job), so that
 // both operands of a contraction are prepared by one launch of each kernel.
 struct AlignPair {
     AlignArgs a[2];
     int32_t *cm[2];
     int64_t used[2];
+    int tiles0, tiles1;  // transposing kernels: 128 x 128 tiles of job 0 and of job 1
+    int ntc[2];          // and tile columns of each job
 };
 
 __global__ void __launch_bounds__(256) estar_cols_scratch_kernel(const __grid_constant__ AlignPair P) {
     const AlignArgs &a = P.a[blockIdx.y];
     int32_t *const col_max = P.cm[blockIdx.y];
-    const int64_t used_threads = P.used[blockIdx.y];
     extern __shared__ int sm[];  // [ngc]
     for (int64_t g = threadIdx.x; g < a.ngc; g += blockDim.x) sm[g] = kNoExp;
     __syncthreads();
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t n = ((a.rows + a.g_rows - 1) / a.g_rows) * a.ngc;
-    if (tid < used_threads) {
-        int m = kNoExp;
-        int64_t idx = tid;
-        for (; idx + 3 * used_threads < n; idx += 4 * used_threads) {  // four loads in flight
-            const int e0 = a.in_exp[idx], e1 = a.in_exp[idx + used_threads];
-            const int e2 = a.in_exp[idx + 2 * used_threads], e3 = a.in_exp[idx + 3 * used_threads];
-            if (e0 != kEZero) m = max(m, e0);
-            if (e1 != kEZero) m = max(m, e1);
-            if (e2 != kEZero) m = max(m, e2);
-            if (e3 != kEZero) m = max(m, e3);
+    // a band of group rows per block
+    const int64_t ngr = (a.rows + a.g_rows - 1) / a.g_rows, ngc = a.ngc;
+    const int64_t band = (ngr + gridDim.x - 1) / gridDim.x, r0 = (int64_t)blockIdx.x * band;
+    const int64_t r1 = min(ngr, r0 + band);
+    const int W = (int)(ngc >> 2);
+    if (r0 < r1 && (ngc & 3) == 0 && W <= 256 && (reinterpret_cast<uintptr_t>(a.in_exp) & 3) == 0) {
+        // 4-byte words: thread (r, w) of the block takes word w of rows r0 + r, + per, ...
+        // keeping four byte-wise signed maxima.  E_ZERO (-128) is the smallest byte, so it
+        // only survives where every member is E_ZERO, and is dropped below.
+        const int per = 256 / W, w = (int)threadIdx.x % W, rr = (int)threadIdx.x / W;
+        if (rr < per) {
+            const uint32_t *e = reinterpret_cast<const uint32_t *>(a.in_exp);
+            uint32_t m = 0x80808080u;
+            int64_t r = r0 + rr;
+            for (; r + 3 * per < r1; r += 4 * per) {  // four loads in flight
+                const uint32_t x0 = e[r * W + w], x1 = e[(r + per) * W + w];
+                const uint32_t x2 = e[(r + 2 * per) * W + w], x3 = e[(r + 3 * per) * W + w];
+                m = __vmaxs4(__vmaxs4(m, x0), __vmaxs4(x1, __vmaxs4(x2, x3)));
+            }
+            for (; r < r1; r += per) m = __vmaxs4(m, e[r * W + w]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int v = (int)(int8_t)(m >> (8 * q));
+                if (v != kEZero) atomicMax(&sm[4 * w + q], v);
+            }
         }
-        for (; idx < n; idx += used_threads) {
+    } else if (r0 < r1) {
+        for (int64_t idx = r0 * ngc + threadIdx.x; idx < r1 * ngc; idx += blockDim.x) {
             const int e = a.in_exp[idx];
-            if (e != kEZero) m = max(m, e);
+            if (e != kEZero) atomicMax(&sm[idx % ngc], e);
         }
-        if (m > kNoExp) atomicMax(&sm[tid % a.ngc], m);
     }
     __syncthreads();
     for (int64_t g = threadIdx.x; g < a.ngc; g += blockDim.x)
         if (sm[g] > kNoExp) atomicMax(&col_max[g], sm[g]);
 }
 
-// RNE(C / 2^d) of 16 signed int8 mantissas (|C| <= 127), d >= 0.  d = 0 is a copy and
-// d >= 8 gives 0.  For 1 <= d <= 7 one fp32 FMA per byte computes it exactly:
-//   f = 2^23 + (C + 128)                      (bits 0x4B0000uu, uu = C ^ 0x80)
-//   f * 2^-d + (1.5 * 2^23 - 2^(23-d) - 2^(7-d)) = 1.5 * 2^23 + C * 2^-d
-// Every operand is exact in fp32.  The FMA rounds once, to the nearest integer with
-// ties to even, since its result lies in [2^23, 2^24) where the spacing is 1.  So the
-// low byte of the result's bits is RNE(C / 2^d) in two's complement.  The work runs on
-// the FMA pipe; the ALU only builds the operands and packs the bytes.
-__device__ __forceinline__ uint4 rne_shift16(uint4 raw, int d) {
-    if (d == 0) return raw;
-    if (d >= 8) return make_uint4(0, 0, 0, 0);
-    const float sc = __int_as_float((127 - d) << 23);
-    const float k = 12582912.0f - (float)(1 << (23 - d)) - (float)(1 << (7 - d));
+// RNE(C / 2^d) of 16 signed int8 mantissas (|C| <= 127), d >= 0; d >= 8 gives 0.  One
+// half-precision FMA rounds two bytes at once:
+//   h = 1024 + (C + 128)                     (fp16 bits 0x64uu, uu = C ^ 0x80)
+//   h * 2^-d + (1536 - 2^(10-d) - 2^(7-d)) = 1536 + C * 2^-d
+// The three operands are exact in fp16 and the fused multiply-add rounds once.  Its
+// result lies in [1024, 2048), where fp16 integers are spaced by 1, so the rounding is
+// to the nearest integer with ties to even, and the low byte of the result's bits
+// (1536 is 0x6600) is RNE(C / 2^d) in two's complement; d = 0 is exact (1536 + C).  Per
+// four bytes: one XOR, two byte permutes to build the halves, two f16x2 FMAs, one
+// permute to pack, and no branches, so lanes with different shifts stay together.
+__device__ __forceinline__ uint32_t fma_f16x2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+// The FMA's two constants for a shift d in [0, 7], and for index 8 (a shift of 8 or
+// more, or a zero group): multiplier 0 and addend 1536, which leaves every byte 0.
+struct RneK {
+    uint32_t sc, k;  // 2^-d and 1536 - 2^(10-d) - 2^(7-d) in both fp16 halves
+};
+__device__ __forceinline__ RneK rne_consts(int d) {
+    if (d >= 8) return RneK{0u, 0x66006600u};
+    const uint32_t kk = 1536u - (1024u >> d) - (128u >> d);  // an integer in [384, 1527]
+    const uint32_t kb = kk >= 1024u ? kk + 0x6000u : (kk >= 512u ? 2u * kk + 0x5C00u : 4u * kk + 0x5800u);
+    return RneK{(uint32_t)(15 - d) * 0x04000400u, kb * 0x10001u};
+}
+// Kernels that round many vectors keep the nine constant pairs in shared memory.
+__device__ __forceinline__ void rne_table_init(RneK *t) {
+    if (threadIdx.x < 9) t[threadIdx.x] = rne_consts(threadIdx.x);
+}
+// Table index of a vector with group exponent eg aligned to es: the shift, 8 for 8 or
+// more and for a zero group.  A target below eg (never asked for) also maps to 8.
+__device__ __forceinline__ int rne_index(int es, int eg) {
+    return eg == kEZero ? 8 : (int)min((unsigned)(es - eg), 8u);
+}
+__device__ __forceinline__ uint4 rne_shift16_k(uint4 raw, RneK c) {
     const uint32_t src[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
     uint32_t o[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        uint32_t r[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-            r[b] = __float_as_uint(__fmaf_rn(__uint_as_float(__byte_perm(src[q], 0x4B000000u, 0x7650 | b)), sc, k));
-        o[q] = __byte_perm(__byte_perm(r[0], r[1], 0x0040), __byte_perm(r[2], r[3], 0x0040), 0x5410);
+        const uint32_t lo = fma_f16x2(__byte_perm(src[q], 0x64646464u, 0x4140), c.sc, c.k);  // bytes 0, 1
+        const uint32_t hi = fma_f16x2(__byte_perm(src[q], 0x64646464u, 0x4342), c.sc, c.k);  // bytes 2, 3
+        o[q] = __byte_perm(lo, hi, 0x6420);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
+__device__ __forceinline__ uint4 rne_shift16(uint4 raw, int d) { return rne_shift16_k(raw, rne_consts(d)); }
 
 // Target exponent of the 16-byte vector at column j of row i (axis 1: per row; axis 0:
 // per column, from the column-max scratch or the e* vector).
@@ -255,14 +292,103 @@ __device__ __forceinline__ int align_target(const AlignArgs &a, int64_t i, int64
     return a.e_star[j];
 }
 
-// Aligned mantissas in place of layout, 64 x 256 tiles: four threads per row, each with
-// four 16-byte vectors (columns j, j + 64, j + 128, j + 192; cols are a multiple of 16,
-// g_cols a multiple of 16 or spanning all columns), loaded before the row's target is
-// known.
-// With axis 1 and no precomputed e*, the four threads of a row compute the row's e*
-// themselves (a quarter of its group exponents each, then two shuffles) and the first
-// of them stores it.
-__global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
+// Aligned mantissas in place of layout (cols a multiple of 16; g_cols a multiple of 16
+// or spanning all columns; rows below 2^31).  Each row is taken by a segment of L lanes
+// of a warp; lane lr holds the row's 16-byte vectors lr, lr + L, ..., NV of them, which
+// covers the row.  The blocks are persistent: a segment walks rows i, i + S, ... (S
+// segments in the grid) with two register buffers in turn, issuing every load of its
+// next row before it rounds and stores the current one, so that each SM keeps a row per
+// segment in flight.  With axis 1 and no given e*, the segment reduces the row's group
+// exponents (at most 2 L of them) to e* and its lane 0 stores it.  An E_ZERO exponent
+// (-128, the smallest byte) can take part in the max unchanged: it only wins when every
+// group is zero, and then e* is E_ZERO as well.
+template <int NV>
+struct RowBatch {
+    uint4 raw[NV];
+    int eg[NV];
+    int ep;  // axis 1: max of this lane's share of the row's group exponents, or the given e*
+};
+
+// EXACT: axis 1, one group row per row, g_cols / 16 a power of two and rows of exactly
+// L NV vectors, which drops every per-vector guard and division.
+template <int L, int NV, bool EXACT>
+__device__ __forceinline__ void align_row_load(const AlignArgs &a, int i, int gsh, bool row_e, RowBatch<NV> &b) {
+    const int lr = threadIdx.x % L;
+    const int8_t *erow = a.in_exp + (EXACT ? (int64_t)i : idiv(i, a.g_rows)) * a.ngc;
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.in + (int64_t)i * a.ld);
+#pragma unroll
+    for (int t = 0; t < NV; ++t) {
+        const int v = lr + L * t;
+        if (EXACT || v < (int)(a.cols >> 4)) {
+            b.raw[t] = src[v];
+            b.eg[t] = erow[EXACT || gsh >= 0 ? (v >> gsh) : (int)idiv(16 * (int64_t)v, a.g_cols)];
+        }
+    }
+    if (row_e) {
+        const int ngc = (int)a.ngc;
+        b.ep = max(lr < ngc ? (int)erow[lr] : kEZero, lr + L < ngc ? (int)erow[lr + L] : kEZero);
+    } else if (EXACT || a.axis == 1) {
+        b.ep = a.e_star[i];
+    }
+}
+
+template <int L, int NV, bool EXACT>
+__device__ __forceinline__ void align_row_store(const AlignArgs &a, int i, unsigned seg, bool row_e,
+                                                const RneK *tk, const RowBatch<NV> &b) {
+    const int lr = threadIdx.x % L;
+    int es = b.ep;
+    if (row_e) {
+#pragma unroll
+        for (int o = L / 2; o > 0; o >>= 1) es = max(es, __shfl_xor_sync(seg, es, o));
+        if (lr == 0) a.e_star[i] = (int8_t)es;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(a.out + (int64_t)i * a.out_ld);
+#pragma unroll
+    for (int t = 0; t < NV; ++t) {
+        const int v = lr + L * t;
+        if (!EXACT && v >= (int)(a.cols >> 4)) break;
+        int et = es;
+        if (!EXACT && a.axis == 0) {
+            et = align_target(a, i, 16 * (int64_t)v);
+            if (a.col_max && i == 0)
+                for (int q = 0; q < 16; ++q) a.e_star[16 * v + q] = (int8_t)et;
+        }
+        dst[v] = rne_shift16_k(b.raw[t], tk[rne_index(et, b.eg[t])]);
+    }
+}
+
+template <int L, int NV, bool EXACT>
+__global__ void __launch_bounds__(256, 2) align_rows_kernel(const __grid_constant__ AlignArgs a) {
+    constexpr int kSegs = 256 / L;
+    __shared__ RneK tk[9];
+    rne_table_init(tk);
+    __syncthreads();
+    const int rows = (int)a.rows, S = (int)gridDim.x * kSegs;
+    int i = (int)blockIdx.x * kSegs + (int)threadIdx.x / L;
+    if (i >= rows) return;  // whole segments leave together
+    const unsigned seg = (0xffffffffu >> (32 - L)) << ((threadIdx.x & 31) & ~(L - 1));
+    const bool row_e = a.axis == 1 && a.row_estar;
+    const int gsh = a.gv_shift1 - 1;
+    RowBatch<NV> ba, bb;
+    align_row_load<L, NV, EXACT>(a, i, gsh, row_e, ba);
+    while (true) {  // two rows per trip, one buffer each: no register copies
+        if (i + S < rows) align_row_load<L, NV, EXACT>(a, i + S, gsh, row_e, bb);
+        align_row_store<L, NV, EXACT>(a, i, seg, row_e, tk, ba);
+        if ((i += S) >= rows) break;
+        if (i + S < rows) align_row_load<L, NV, EXACT>(a, i + S, gsh, row_e, ba);
+        align_row_store<L, NV, EXACT>(a, i, seg, row_e, tk, bb);
+        if ((i += S) >= rows) break;
+    }
+}
+
+// The same for rows too wide for one batch per lane or with many groups: 64 x 256
+// tiles, four threads per row with four 16-byte vectors each (columns j, j + 64,
+// j + 128, j + 192), loaded before the row's target is known; with axis 1 and no given
+// e*, the four threads of a row reduce a quarter of its group exponents each.
+__global__ void __launch_bounds__(256) align_rows_wide_kernel(const __grid_constant__ AlignArgs a) {
+    __shared__ RneK tk[9];
+    rne_table_init(tk);
+    __syncthreads();
     const int64_t i = (int64_t)blockIdx.y * 64 + (threadIdx.x >> 2);
     const int64_t j0 = (int64_t)blockIdx.x * 256 + (threadIdx.x & 3) * 16;
     if (i >= a.rows) return;  // whole 4-thread row groups leave together
@@ -280,13 +406,11 @@ __global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
     const bool row_e = a.axis == 1 && a.row_estar;
     if (row_e) {
         const int8_t *e = a.in_exp + idiv(i, a.g_rows) * a.ngc;
-        int m = kNoExp;
-        for (int64_t g = threadIdx.x & 3; g < a.ngc; g += 4)
-            if (e[g] != kEZero) m = max(m, (int)e[g]);
+        int m = kEZero;
+        for (int64_t g = threadIdx.x & 3; g < a.ngc; g += 4) m = max(m, (int)e[g]);
         const unsigned quad = 0xfu << (threadIdx.x & 28);
         m = max(m, __shfl_xor_sync(quad, m, 1));
-        m = max(m, __shfl_xor_sync(quad, m, 2));
-        es_row = estar_of(m);
+        es_row = max(m, __shfl_xor_sync(quad, m, 2));
         if (blockIdx.x == 0 && (threadIdx.x & 3) == 0) a.e_star[i] = (int8_t)es_row;
     }
 #pragma unroll
@@ -295,26 +419,32 @@ __global__ void __launch_bounds__(256) align_rows_kernel(AlignArgs a) {
         if (j >= a.cols) continue;
         const int es = row_e ? es_row : align_target(a, i, j);
         if (a.axis == 0 && a.col_max && i == 0)
-            for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
-        *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) =
-            eg[v] == kEZero ? make_uint4(0, 0, 0, 0) : rne_shift16(raw[v], min(es - eg[v], 8));
+            for (int q = 0; q < 16; ++q) a.e_star[j + q] = (int8_t)es;
+        *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j) = rne_shift16_k(raw[v], tk[rne_index(es, eg[v])]);
     }
 }
 
-// Aligned and transposed, 128 x 128 tiles (rows and cols are multiples of 16).  Thread
-// (warp w, lane l) aligns rows 16 w + 4 (l & 3) .. + 3 at columns 16 (l >> 2) .. + 15,
-// transposes the 4 x 4 byte blocks in registers (8 byte permutes per 16 bytes) and
-// stores 32-bit words into a shared tile whose 16-byte chunks are XOR-swizzled by the
-// output row's 16-row band, so that both the word stores and the 16-byte reads that
-// feed the coalesced global stores are free of bank conflicts.
+// Aligned and transposed, 128 x 128 tiles (rows and cols are multiples of 16).  The
+// grid is one-dimensional over the tiles of both jobs (job 0's first, P.tiles0 of
+// them; P.ntc[z] tile columns per tile row).  Thread (warp w, lane l) aligns rows
+// 16 w + 4 (l & 3) .. + 3 at columns 16 (l >> 2) .. + 15, transposes the 4 x 4 byte
+// blocks in registers (8 byte permutes per 16 bytes) and stores 32-bit words into a
+// shared tile whose 16-byte chunks are XOR-swizzled by the output row's 16-row band, so
+// that both the word stores and the 16-byte reads that feed the coalesced global
+// stores are free of bank conflicts.
 __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_constant__ AlignPair P) {
-    const AlignArgs &a = P.a[blockIdx.z];
+    const int z = (int)blockIdx.x >= P.tiles0 ? 1 : 0;
+    const AlignArgs &a = P.a[z];
+    const int tile_id = (int)blockIdx.x - (z ? P.tiles0 : 0);
+    const int tr = tile_id / P.ntc[z], tcol = tile_id - tr * P.ntc[z];
     __shared__ uint4 tile[128][8];  // [output row = input column][16-byte chunk, swizzled]
+    __shared__ RneK tk[9];
+    __shared__ int gmx[16];  // col_scan: e* of the column groups of this block's 128 columns
+    rne_table_init(tk);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t r0 = (int64_t)blockIdx.y * 128, c0 = (int64_t)blockIdx.x * 128;
+    const int64_t r0 = (int64_t)tr * 128, c0 = (int64_t)tcol * 128;
     const int rq = 4 * warp + (lane & 3), cc = lane >> 2;  // row quad 0..31, column chunk 0..7
     const int64_t j = c0 + 16 * cc;
-    __shared__ int gmx[16];  // col_scan: e* of the column groups of this block's 128 columns
     int64_t g_first = 0;
     if (a.col_scan) {
         // a strip of at most 128 columns spans at most 9 groups (groups are >= 16 wide)
@@ -332,11 +462,11 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
             }
             if (m > kNoExp) atomicMax(&gmx[k], m);
         }
-        __syncthreads();
     }
+    __syncthreads();
     if (j < a.cols) {
         const int es_col = a.col_scan ? estar_of(gmx[idiv(j, a.g_cols) - g_first]) : 0;
-        if (a.axis == 0 && (a.col_max || a.col_scan) && blockIdx.y == 0 && rq == 0) {
+        if (a.axis == 0 && (a.col_max || a.col_scan) && tr == 0 && rq == 0) {
             const int es = a.col_scan ? es_col : align_target(a, 0, j);
             for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
         }
@@ -351,16 +481,18 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
             raw[t] = in ? *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j) : make_uint4(0, 0, 0, 0);
             eg[t] = in ? (int)a.in_exp[idiv(i, a.g_rows) * a.ngc + gcol] : kEZero;
         }
-        int es[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) es[t] = a.col_scan ? es_col : align_target(a, r0 + 4 * rq + t, j);
+        // axis 0: one target for the thread's 16 columns in all four rows
+        const int es_c = a.axis == 0 ? (a.col_scan ? es_col : align_target(a, 0, j)) : 0;
         uint4 v[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-            v[t] = eg[t] == kEZero ? make_uint4(0, 0, 0, 0) : rne_shift16(raw[t], min(es[t] - eg[t], 8));
+        for (int t = 0; t < 4; ++t) {
+            const int es = a.axis == 0 ? es_c : align_target(a, r0 + 4 * rq + t, j);
+            v[t] = rne_shift16_k(raw[t], tk[rne_index(es, eg[t])]);
+        }
         const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w}, {v[1].x, v[1].y, v[1].z, v[1].w},
                                   {v[2].x, v[2].y, v[2].z, v[2].w}, {v[3].x, v[3].y, v[3].z, v[3].w}};
         uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
+        const int chunk = (rq >> 2) ^ cc;  // swizzled 16-byte chunk
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // columns 16 cc + 4 q .. + 3
             const uint32_t t0 = __byte_perm(w[0][q], w[1][q], 0x5140), t1 = __byte_perm(w[0][q], w[1][q], 0x7362);
@@ -368,11 +500,7 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
             const uint32_t col[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
                                      __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632)};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int orow = 16 * cc + 4 * q + k;                 // output row in the tile
-                const int chunk = (rq >> 2) ^ cc;                     // swizzled 16-byte chunk
-                tw[orow * 32 + chunk * 4 + (rq & 3)] = col[k];
-            }
+            for (int k = 0; k < 4; ++k) tw[(16 * cc + 4 * q + k) * 32 + chunk * 4 + (rq & 3)] = col[k];
         }
     }
     __syncthreads();
@@ -382,6 +510,100 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
         const int64_t oi = c0 + orow, oj = r0 + 16 * m;
         if (oi < a.cols && oj < a.rows)
             *reinterpret_cast<uint4 *>(a.out + oi * a.out_ld + oj) = tile[orow][m ^ (orow >> 4)];
+    }
+}
+
+// The transposing alignment for jobs whose targets come from a column-max scratch or a
+// given e* (no block scans its columns' exponents): the same tiles and thread layout,
+// but persistent blocks that walk the tiles of both jobs with the grid's stride, issue
+// the loads of their next tile before they round and transpose the current one, and
+// alternate between two shared tiles, so that one barrier per tile suffices.
+struct TrTile {
+    uint4 raw[4];
+    int eg[4];
+    int es;  // axis 0: the target of the thread's 16 columns
+};
+
+__device__ __forceinline__ void tr_tile_decode(const AlignPair &P, int tile, int &z, int64_t &r0, int64_t &c0) {
+    z = tile >= P.tiles0 ? 1 : 0;
+    const int t = tile - (z ? P.tiles0 : 0);
+    const int tr = t / P.ntc[z];
+    r0 = (int64_t)tr * 128;
+    c0 = (int64_t)(t - tr * P.ntc[z]) * 128;
+}
+
+__device__ __forceinline__ void tr_tile_load(const AlignArgs &a, int64_t r0, int64_t j, int rq, TrTile &b) {
+    if (j >= a.cols) return;
+    const int64_t gcol = idiv(j, a.g_cols);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int64_t i = r0 + 4 * rq + t;
+        const bool in = i < a.rows;
+        b.raw[t] = in ? *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j) : make_uint4(0, 0, 0, 0);
+        b.eg[t] = in ? (int)a.in_exp[idiv(i, a.g_rows) * a.ngc + gcol] : kEZero;
+    }
+    b.es = a.axis == 0 ? align_target(a, 0, j) : 0;
+}
+
+__global__ void __launch_bounds__(256, 3) align_transpose_stream_kernel(const __grid_constant__ AlignPair P) {
+    __shared__ uint4 tile[2][128][8];  // [buffer][output row = input column][16-byte chunk, swizzled]
+    __shared__ RneK tk[9];
+    rne_table_init(tk);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rq = 4 * warp + (lane & 3), cc = lane >> 2;  // row quad 0..31, column chunk 0..7
+    const int total = P.tiles0 + P.tiles1;
+    int tile_id = blockIdx.x;
+    if (tile_id >= total) return;  // whole blocks
+    TrTile cur, nxt;
+    int z;
+    int64_t r0, c0;
+    tr_tile_decode(P, tile_id, z, r0, c0);
+    tr_tile_load(P.a[z], r0, c0 + 16 * cc, rq, cur);
+    for (int buf = 0; tile_id < total; tile_id += gridDim.x, buf ^= 1) {
+        const int next = tile_id + gridDim.x;
+        int zn = 0;
+        int64_t rn = 0, cn = 0;
+        if (next < total) {
+            tr_tile_decode(P, next, zn, rn, cn);
+            tr_tile_load(P.a[zn], rn, cn + 16 * cc, rq, nxt);
+        }
+        const AlignArgs &a = P.a[z];
+        const int64_t j = c0 + 16 * cc;
+        if (j < a.cols) {
+            if (a.axis == 0 && a.col_max && r0 == 0 && rq == 0)
+                for (int q = 0; q < 16; ++q) a.e_star[j + q] = (int8_t)cur.es;
+            uint4 v[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int es = a.axis == 0 ? cur.es : align_target(a, r0 + 4 * rq + t, j);
+                v[t] = rne_shift16_k(cur.raw[t], tk[rne_index(es, cur.eg[t])]);
+            }
+            const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w}, {v[1].x, v[1].y, v[1].z, v[1].w},
+                                      {v[2].x, v[2].y, v[2].z, v[2].w}, {v[3].x, v[3].y, v[3].z, v[3].w}};
+            uint32_t *tw = reinterpret_cast<uint32_t *>(tile[buf]);
+            const int chunk = (rq >> 2) ^ cc;  // swizzled 16-byte chunk
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {  // columns 16 cc + 4 q .. + 3
+                const uint32_t t0 = __byte_perm(w[0][q], w[1][q], 0x5140), t1 = __byte_perm(w[0][q], w[1][q], 0x7362);
+                const uint32_t t2 = __byte_perm(w[2][q], w[3][q], 0x5140), t3 = __byte_perm(w[2][q], w[3][q], 0x7362);
+                const uint32_t col[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
+                                         __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632)};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) tw[(16 * cc + 4 * q + k) * 32 + chunk * 4 + (rq & 3)] = col[k];
+            }
+        }
+        // one barrier per tile: the buffer written here was last read two tiles ago, and
+        // every thread has passed the barrier of the tile in between since then
+        __syncthreads();
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) {
+            const int orow = pass * 32 + (threadIdx.x >> 3), m = threadIdx.x & 7;
+            const int64_t oi = c0 + orow, oj = r0 + 16 * m;
+            if (oi < a.cols && oj < a.rows)
+                *reinterpret_cast<uint4 *>(a.out + oi * a.out_ld + oj) = tile[buf][orow][m ^ (orow >> 4)];
+        }
+        if (next < total) cur = nxt, z = zn, r0 = rn, c0 = cn;
     }
 }
 
