@@ -129,6 +129,14 @@ __device__ __forceinline__ int sx8(uint32_t w, int byte) {
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));
     return (int)r;
 }
+// Four values already within [-127, 127] packed into bytes in two conversion
+// instructions (each packs two values; the second merges the first's word).
+__device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {
+    uint32_t t, r;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(t) : "r"(d), "r"(c));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(b), "r"(a), "r"(t));
+    return r;
+}
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
            ((uint32_t)(d & 0xff) << 24);

@@ -812,6 +812,23 @@ __global__ void __launch_bounds__(256) gelu_bwd_vec_kernel(const __grid_constant
 
 // FIT of row-local groups wider than a warp can hold: one block of T threads per group,
 // EPT elements per thread kept in registers between the max and the rounding pass.
+// Fast FIT of a group's int32 values x with value exponents r (row + column exponent),
+// for groups whose nonzero values have exponents within [rmin, rmax] and
+// (rmax - rmin) + bitlen(max |x|) <= 30: with y = x * 2^(r - rmin) (exact, |y| < 2^30),
+// the group exponent is e = rmin + need_off(max |y|), since need_off(|x| 2^d) =
+// need_off(|x|) + d and need_off is monotone, and every mantissa is RNE(y / 2^(e - rmin)),
+// one multiply-high rounding per value (floor((y + 2^(S-1) - 1 + lsb) / 2^S)).
+__device__ __forceinline__ int fit_fast_shift(int y, int S, int m, int bias) {
+    if (S <= 0) return y << -S;
+    if (S == 1) return (y + ((y >> 1) & 1)) >> 1;
+    const int t = __mulhi(y, m);
+    return __mulhi(y + bias + (t & 1), m);
+}
+__device__ __forceinline__ bool fit_fast_ok(int rmin, int rmax, uint32_t amax) {
+    return amax == 0 || (rmax - rmin) + (32 - __clz(amax)) <= 30;
+}
+__device__ __forceinline__ uint32_t uabs32(int v) { return v < 0 ? 0u - (uint32_t)v : (uint32_t)v; }
+
 template <int T, int EPT>
 __global__ void __launch_bounds__(T) requant_group_block_kernel(RequantArgs a) {
     const int64_t gidx = blockIdx.x;
@@ -898,24 +915,98 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
 #pragma unroll
                 for (int t = 0; t < 4; ++t) r[k][t] = re + a.col_exp[(j0 + jj + t) / a.col_div];
             }
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                if (WIDE) {
-                    if (x[k][t]) emax = max(emax, need64q((int64_t)x[k][t], r[k][t], a.qb));
-                } else {
-                    const int32_t v = (int32_t)x[k][t];
-                    if (v) emax = max(emax, r[k][t] + need_off32q((uint32_t)(v < 0 ? -v : v), a.qb));
-                }
-            }
         }
     }
-    __shared__ int red[T / 32];
-    emax = warp_max(emax);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = emax;
-    __syncthreads();
-    int m = red[0];
+    __shared__ int red[4][T / 32];
+    const int wid = threadIdx.x >> 5;
+    if constexpr (!WIDE) {
+        // the fast exact FIT (see fit_fast_shift) when the group's value exponents are close
+        int rmin = 0x7fffffff, rmax = -0x7fffffff;
+        uint32_t amax = 0;
 #pragma unroll
-    for (int w = 1; w < T / 32; ++w) m = max(m, red[w]);
+        for (int k = 0; k < V; ++k) {
+            if (4 * (threadIdx.x + k * T) < glen)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) rmin = min(rmin, r[k][t]), rmax = max(rmax, r[k][t]);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) amax = max(amax, uabs32((int)x[k][t]));
+        }
+        rmin = __reduce_min_sync(0xffffffffu, rmin), rmax = __reduce_max_sync(0xffffffffu, rmax);
+        amax = __reduce_max_sync(0xffffffffu, amax);
+        if ((threadIdx.x & 31) == 0) red[0][wid] = rmin, red[1][wid] = rmax, red[2][wid] = (int)amax;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < T / 32; ++w)
+            rmin = min(rmin, red[0][w]), rmax = max(rmax, red[1][w]), amax = max(amax, (uint32_t)red[2][w]);
+        if (fit_fast_ok(rmin, rmax, amax)) {
+            const bool spread = rmax != rmin;
+            uint32_t ymax = amax;
+            if (spread) {  // y = x 2^(r - rmin) in place (exact: fewer than 31 bits)
+                ymax = 0;
+#pragma unroll
+                for (int k = 0; k < V; ++k)
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        x[k][t] = (int)x[k][t] << ((r[k][t] - rmin) & 31);
+                        ymax = max(ymax, uabs32((int)x[k][t]));
+                    }
+                ymax = __reduce_max_sync(0xffffffffu, ymax);
+                if ((threadIdx.x & 31) == 0) red[3][wid] = (int)ymax;
+                __syncthreads();
+#pragma unroll
+                for (int w = 0; w < T / 32; ++w) ymax = max(ymax, (uint32_t)red[3][w]);
+            }
+            const int e_raw = amax ? rmin + need_off32q(ymax, a.qb) : kNoExp;
+            if (e_raw <= 127) {  // a capped exponent takes the saturating exact path below
+                const int e = finalize_exp(e_raw);
+                const int S = e == kEZero ? 0 : min(e - rmin, 31);
+                const int m = S >= 2 ? 1 << (32 - S) : 0, bias = S >= 2 ? (1 << (S - 1)) - 1 : 0;
+#pragma unroll
+                for (int k = 0; k < V; ++k) {
+                    const int jj = 4 * (threadIdx.x + k * T);
+                    if (jj < glen) {
+                        int o[4];
+                        if (S >= 2) {
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int v = (int)x[k][t];
+                                o[t] = __mulhi(v + bias + (__mulhi(v, m) & 1), m);
+                            }
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) o[t] = fit_fast_shift((int)x[k][t], S, 0, 0);
+                        }
+                        *reinterpret_cast<uint32_t *>(a.out + i * a.out_ld + j0 + jj) = pack4s(o[0], o[1], o[2], o[3]);
+                    }
+                }
+                if (threadIdx.x == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
+                return;
+            }
+            if (spread)  // undo the in-place scaling for the exact path
+#pragma unroll
+                for (int k = 0; k < V; ++k)
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) x[k][t] = (int)x[k][t] >> ((r[k][t] - rmin) & 31);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < V; ++k)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if (WIDE) {
+                if (x[k][t]) emax = max(emax, need64q((int64_t)x[k][t], r[k][t], a.qb));
+            } else {
+                const int32_t v = (int32_t)x[k][t];
+                if (v) emax = max(emax, r[k][t] + need_off32q((uint32_t)(v < 0 ? -v : v), a.qb));
+            }
+        }
+    emax = warp_max(emax);
+    __syncthreads();  // the fast path's reductions may still read red[0]
+    if ((threadIdx.x & 31) == 0) red[0][wid] = emax;
+    __syncthreads();
+    int m = red[0][0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) m = max(m, red[0][w]);
     const int e = finalize_exp(m);
 #pragma unroll
     for (int k = 0; k < V; ++k) {
@@ -936,6 +1027,7 @@ __global__ void __launch_bounds__(T) requant_vec_kernel(RequantArgs a) {
 // anything else, and the group's largest need is a warp reduction, so no block barrier
 // sits between the loads and the stores.  Requires cs = 1, col_div = 1 (or no column
 // exponents), G, cols, ld and out_ld multiples of 4.
+
 template <int V>
 __global__ void __launch_bounds__(256) requant_warp_kernel(const __grid_constant__ RequantArgs a) {
     const int lane = threadIdx.x & 31;
@@ -957,25 +1049,91 @@ __global__ void __launch_bounds__(256) requant_warp_kernel(const __grid_constant
             if (a.col_exp) ce[k] = *reinterpret_cast<const uint32_t *>(a.col_exp + j0 + jj);
         }
     }
-    int emax = kNoExp;
+    // the group's column-exponent range (per-byte extremes of this lane's words, then the
+    // warp's) and its largest magnitude
+    uint32_t cmn = 0x7f7f7f7fu, cmx = 0x80808080u, amax = 0;
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-        const int v[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-            if (v[t]) emax = max(emax, re + sx8(ce[k], t) + need_off32q((uint32_t)(v[t] < 0 ? -v[t] : v[t]), a.qb));
+        if (4 * (lane + 32 * k) < glen) cmn = __vmins4(cmn, ce[k]), cmx = __vmaxs4(cmx, ce[k]);
+        amax = max(max(uabs32(x[k].x), uabs32(x[k].y)), max(max(uabs32(x[k].z), uabs32(x[k].w)), amax));
     }
-    const int e = finalize_exp(warp_max(emax));
+    int rmin = min(min(sx8(cmn, 0), sx8(cmn, 1)), min(sx8(cmn, 2), sx8(cmn, 3)));
+    int rmax = max(max(sx8(cmx, 0), sx8(cmx, 1)), max(sx8(cmx, 2), sx8(cmx, 3)));
+    rmin = __reduce_min_sync(0xffffffffu, rmin), rmax = __reduce_max_sync(0xffffffffu, rmax);
+    amax = __reduce_max_sync(0xffffffffu, amax);
+    uint32_t packed[V];
+    int e = kEZero;
+    bool fast = fit_fast_ok(rmin, rmax, amax);
+    const bool spread = rmax != rmin;
+    if (fast) {
+        uint32_t ymax = amax;
+        if (spread) {  // y = x 2^(ce - rmin) in place (exact: fewer than 31 bits)
+            ymax = 0;
 #pragma unroll
-    for (int k = 0; k < V; ++k) {
-        const int jj = 4 * (lane + 32 * k);
-        if (jj < glen) {
+            for (int k = 0; k < V; ++k) {
+                int *v = reinterpret_cast<int *>(&x[k]);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) v[t] <<= (sx8(ce[k], t) - rmin) & 31, ymax = max(ymax, uabs32(v[t]));
+            }
+            ymax = __reduce_max_sync(0xffffffffu, ymax);
+        }
+        const int e_raw = amax ? re + rmin + need_off32q(ymax, a.qb) : kNoExp;
+        fast = e_raw <= 127;  // a capped exponent takes the saturating exact path
+        if (fast) {
+            e = finalize_exp(e_raw);
+            const int S = e == kEZero ? 0 : min(e - re - rmin, 31);
+            if (S >= 2) {
+                const int m = 1 << (32 - S), bias = (1 << (S - 1)) - 1;
+#pragma unroll
+                for (int k = 0; k < V; ++k) {
+                    int *v = reinterpret_cast<int *>(&x[k]);
+                    int o[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) o[t] = __mulhi(v[t] + bias + (__mulhi(v[t], m) & 1), m);
+                    packed[k] = pack4s(o[0], o[1], o[2], o[3]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < V; ++k) {
+                    int *v = reinterpret_cast<int *>(&x[k]);
+                    int o[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) o[t] = fit_fast_shift(v[t], S, 0, 0);
+                    packed[k] = pack4s(o[0], o[1], o[2], o[3]);
+                }
+            }
+        } else if (spread) {  // undo the in-place scaling for the exact path
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                int *v = reinterpret_cast<int *>(&x[k]);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) v[t] >>= (sx8(ce[k], t) - rmin) & 31;
+            }
+        }
+    }
+    if (!fast) {
+        int emax = kNoExp;
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int v[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                if (v[t]) emax = max(emax, re + sx8(ce[k], t) + need_off32q((uint32_t)(v[t] < 0 ? -v[t] : v[t]), a.qb));
+        }
+        e = finalize_exp(warp_max(emax));
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
             const int v[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
             int o[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) o[t] = requant32(v[t], re + sx8(ce[k], t), e);
-            *reinterpret_cast<uint32_t *>(a.out + i * a.out_ld + j0 + jj) = pack4(o[0], o[1], o[2], o[3]);
+            packed[k] = pack4(o[0], o[1], o[2], o[3]);
         }
+    }
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        const int jj = 4 * (lane + 32 * k);
+        if (jj < glen) *reinterpret_cast<uint32_t *>(a.out + i * a.out_ld + j0 + jj) = packed[k];
     }
     if (lane == 0) a.out_exp[i * a.ngc + g] = (int8_t)e;
 }

@@ -112,14 +112,6 @@ struct GemmSmem {
 __device__ __forceinline__ uint32_t pack4b(int a, int b, int c, int d) {
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
-// The same packing for values already within [-127, 127], in two conversion
-// instructions (each packs two values into bytes; the second merges the first's word).
-__device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {
-    uint32_t t, r;
-    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(t) : "r"(d), "r"(c));
-    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(b), "r"(a), "r"(t));
-    return r;
-}
 
 // Fast epilogue of one output group of NC x 32 columns of an accumulator row, the group
 // on the fast path: y = acc * 2^d_n (d_n = column shift inside the group, |y| < 2^30),
