@@ -1432,22 +1432,30 @@ int run_sgd(SgdArgs &a, int sms, cudaStream_t s) {
               aligned16(a.t[i].g);
     vec = vec && G % 16 == 0 && G <= 2048;
     const SgdTensor &t0 = a.t[0];
-    // one dense tensor, one group per row of 16 * L elements: the prefetching kernel
+    // one dense tensor, one group per row of 16 L CPL elements: the prefetching kernel,
+    // two chunks per lane where the group allows (groups of 32 to 1024 elements)
     const int Lr = G / 16;
     if (vec && a.n == 1 && t0.ngc == 1 && t0.cols == t0.G && t0.ld == t0.G && Lr >= 1 && Lr <= 32 &&
         (Lr & (Lr - 1)) == 0) {
-        const int L = Lr;
+        const int CPL = (Lr >= 2 && Lr <= 64) ? 2 : 1, L = Lr / CPL;
         const int64_t gpb = 8 * (32 / L);
         const unsigned blocks = (unsigned)std::min<int64_t>(cdiv64(a.total_groups, gpb), (int64_t)sms * 8);
         bool done = true;
-        switch (L) {
-            case 1: sgd_rows_kernel<1><<<blocks, 256, 0, s>>>(a); break;
-            case 2: sgd_rows_kernel<2><<<blocks, 256, 0, s>>>(a); break;
-            case 4: sgd_rows_kernel<4><<<blocks, 256, 0, s>>>(a); break;
-            case 8: sgd_rows_kernel<8><<<blocks, 256, 0, s>>>(a); break;
-            case 16: sgd_rows_kernel<16><<<blocks, 256, 0, s>>>(a); break;
-            case 32: sgd_rows_kernel<32><<<blocks, 256, 0, s>>>(a); break;
-            default: done = false;
+        if (CPL == 2) {
+            switch (L) {
+                case 1: sgd_rows_kernel<1, 2><<<blocks, 256, 0, s>>>(a); break;
+                case 2: sgd_rows_kernel<2, 2><<<blocks, 256, 0, s>>>(a); break;
+                case 4: sgd_rows_kernel<4, 2><<<blocks, 256, 0, s>>>(a); break;
+                case 8: sgd_rows_kernel<8, 2><<<blocks, 256, 0, s>>>(a); break;
+                case 16: sgd_rows_kernel<16, 2><<<blocks, 256, 0, s>>>(a); break;
+                default: done = false;
+            }
+        } else {
+            switch (L) {
+                case 1: sgd_rows_kernel<1, 1><<<blocks, 256, 0, s>>>(a); break;
+                case 32: sgd_rows_kernel<32, 1><<<blocks, 256, 0, s>>>(a); break;
+                default: done = false;
+            }
         }
         if (done) {
             counted(1);

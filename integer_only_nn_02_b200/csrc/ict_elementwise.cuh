@@ -1637,9 +1637,9 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
     }
 }
 
-// SGD over one dense tensor whose groups are whole rows of exactly 16 * L elements (a
-// parameter arena padded to its group width).  Each lane holds 16 elements of W, V and G;
-// the next group's chunks are loaded before the current group is computed.
+// SGD over one dense tensor whose groups are whole rows of exactly 16 L CPL elements (a
+// parameter arena padded to its group width).  Each lane holds 16 CPL elements of W, V
+// and G; the next group's chunks are loaded before the current group is computed.
 //
 // The two-term sums and their rounding run as exact integer arithmetic on the fp32 pipe
 // (twice the integer pipes' issue rate).  Per group the terms a * 2^pa and b * 2^pb sit
@@ -1688,9 +1688,13 @@ __device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float 
                        __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040), 0x5410);
 }
 
-template <int L>
+// L lanes per group, CPL 16-byte chunks per lane (a group is 16 L CPL elements; chunk k
+// of lane li sits at element (k L + li) 16 of the group, so that each chunk index is a
+// coalesced row of the warp): more chunks per lane spread the per-group work (targets,
+// reductions, exponents, branches) over more elements.
+template <int L, int CPL>
 __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ SgdArgs p) {
-    constexpr int GPW = 32 / L;
+    constexpr int GPW = 32 / L, E = 16 * CPL, G = 16 * L * CPL;
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
     const int lane = threadIdx.x & 31, sub = lane / L, li = lane % L;
     const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (sub * L));
@@ -1700,24 +1704,30 @@ __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ S
     const int64_t rows = t0.rows;
     const int64_t step = (int64_t)gridDim.x * 8 * GPW;
     int64_t r = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * GPW + sub;
-    uint4 cw = make_uint4(0, 0, 0, 0), cv = cw, cg = cw;
+    uint4 cw[CPL], cv[CPL], cg[CPL];
     int ev = 0, eg = 0, ew = 0;
     if (r < rows) {
-        const int64_t at = r * (16 * L) + li * 16;
-        cw = *reinterpret_cast<const uint4 *>(tw + at);
-        cv = *reinterpret_cast<const uint4 *>(tv + at);
-        cg = *reinterpret_cast<const uint4 *>(tg + at);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            const int64_t at = r * G + (k * L + li) * 16;
+            cw[k] = *reinterpret_cast<const uint4 *>(tw + at);
+            cv[k] = *reinterpret_cast<const uint4 *>(tv + at);
+            cg[k] = *reinterpret_cast<const uint4 *>(tg + at);
+        }
         ev = tve[r], eg = tge[r], ew = twe[r];
     }
     for (; r < rows; r += step) {
         const int64_t rn = r + step;
-        uint4 nw4 = make_uint4(0, 0, 0, 0), nv4 = nw4, ng4 = nw4;
+        uint4 nw4[CPL], nv4[CPL], ng4[CPL];
         int nev = 0, neg = 0, new_ = 0;
         if (rn < rows) {  // prefetch the next group
-            const int64_t at = rn * (16 * L) + li * 16;
-            nw4 = *reinterpret_cast<const uint4 *>(tw + at);
-            nv4 = *reinterpret_cast<const uint4 *>(tv + at);
-            ng4 = *reinterpret_cast<const uint4 *>(tg + at);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                const int64_t at = rn * G + (k * L + li) * 16;
+                nw4[k] = *reinterpret_cast<const uint4 *>(tw + at);
+                nv4[k] = *reinterpret_cast<const uint4 *>(tv + at);
+                ng4[k] = *reinterpret_cast<const uint4 *>(tg + at);
+            }
             nev = tve[rn], neg = tge[rn], new_ = twe[rn];
         }
         // velocity: v = mom * V 2^(ev - mom_shift) + G 2^eg
@@ -1726,26 +1736,33 @@ __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ S
         two_term_plan(ev - p.mom_shift, ev == kEZero, eg, eg == kEZero, p.capf_mom, 16, r1, sa1, sb1, k1);
         int r2 = 0, sa2 = 0, sb2 = 0, k2 = 0, ev2 = kEZero;
         bool fit2 = false;
-        float vq[16];  // 1.5 * 2^23 + the new velocity mantissas
+        float vq[E];  // 1.5 * 2^23 + the new velocity mantissas
+        float y[E];   // the velocity sums, then the weight sums
         {
-            const uint32_t vb[4] = {cv.x ^ 0x80808080u, cv.y ^ 0x80808080u, cv.z ^ 0x80808080u, cv.w ^ 0x80808080u};
-            const uint32_t gb[4] = {cg.x ^ 0x80808080u, cg.y ^ 0x80808080u, cg.z ^ 0x80808080u, cg.w ^ 0x80808080u};
+            uint32_t vb[4 * CPL], gb[4 * CPL];
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                vb[4 * k] = cv[k].x ^ 0x80808080u, vb[4 * k + 1] = cv[k].y ^ 0x80808080u;
+                vb[4 * k + 2] = cv[k].z ^ 0x80808080u, vb[4 * k + 3] = cv[k].w ^ 0x80808080u;
+                gb[4 * k] = cg[k].x ^ 0x80808080u, gb[4 * k + 1] = cg[k].y ^ 0x80808080u;
+                gb[4 * k + 2] = cg[k].z ^ 0x80808080u, gb[4 * k + 3] = cg[k].w ^ 0x80808080u;
+            }
             const float ma = (float)(p.mom_mul << sa1), mb = (float)(1 << sb1);
-            float x[16], amax = 0.0f;
+            float amax = 0.0f;
             if (k1 == 0) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, sx8f(gb[e >> 2], e & 3) * mb);
+                for (int e = 0; e < E; ++e) y[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, sx8f(gb[e >> 2], e & 3) * mb);
             } else if (sa1 == 0) {  // G 2^16 dominates: mom * V rounded to odd at 2^k1
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    x[e] = __fmaf_rn(sx8f(gb[e >> 2], e & 3), mb, ro_float(sx8(vb[e >> 2] ^ 0x80808080u, e & 3) * p.mom_mul, k1));
+                for (int e = 0; e < E; ++e)
+                    y[e] = __fmaf_rn(sx8f(gb[e >> 2], e & 3), mb, ro_float(sx8(vb[e >> 2] ^ 0x80808080u, e & 3) * p.mom_mul, k1));
             } else {  // mom * V 2^cap dominates: G rounded to odd at 2^k1
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    x[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, ro_float(sx8(gb[e >> 2] ^ 0x80808080u, e & 3), k1));
+                for (int e = 0; e < E; ++e)
+                    y[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, ro_float(sx8(gb[e >> 2] ^ 0x80808080u, e & 3), k1));
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+            for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
             const int ia = group_max<L>((int)amax, gmask);
             ev2 = finalize_exp(ia ? r1 + need_off32q((uint32_t)ia, p.qb) : kNoExp);
             // with a rounded-to-odd term the final shift must be at least 2 bits (it is unless
@@ -1753,56 +1770,65 @@ __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ S
             fit1 = k1 == 0 || ev2 == kEZero || ev2 - r1 >= 2;
             const float sc = pow2f(ev2 == kEZero ? 0 : r1 - ev2);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) vq[e] = __fmaf_rn(x[e], sc, kMagic);
+            for (int e = 0; e < E; ++e) vq[e] = __fmaf_rn(y[e], sc, kMagic);
             two_term_plan(ew, ew == kEZero, ev2 - p.lr_shift, ev2 == kEZero, 16, p.capf_lr, r2, sa2, sb2, k2);
         }
-        float y[16];
         int ew2 = kEZero;
         if (fit1) {
             // weight: w = W 2^ew - lr * V' 2^(ev2 - lr_shift)
-            const uint32_t wb[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u, cw.w ^ 0x80808080u};
+            uint32_t wb[4 * CPL];
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                wb[4 * k] = cw[k].x ^ 0x80808080u, wb[4 * k + 1] = cw[k].y ^ 0x80808080u;
+                wb[4 * k + 2] = cw[k].z ^ 0x80808080u, wb[4 * k + 3] = cw[k].w ^ 0x80808080u;
+            }
             const float ma = (float)(1 << sa2), mb = (float)(-(p.lr_mul << sb2));
             float amax = 0.0f;
             if (k2 == 0) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(vq[e] - kMagic, mb, sx8f(wb[e >> 2], e & 3) * ma);
+                for (int e = 0; e < E; ++e) y[e] = __fmaf_rn(vq[e] - kMagic, mb, sx8f(wb[e >> 2], e & 3) * ma);
             } else if (sa2 == 0) {  // lr * V' dominates: W rounded to odd at 2^k2
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
+                for (int e = 0; e < E; ++e)
                     y[e] = __fmaf_rn(vq[e] - kMagic, mb, ro_float(sx8(wb[e >> 2] ^ 0x80808080u, e & 3), k2));
             } else {  // W 2^16 dominates: -lr * V' rounded to odd at 2^k2
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
+                for (int e = 0; e < E; ++e)
                     y[e] = __fmaf_rn(sx8f(wb[e >> 2], e & 3), ma,
                                      ro_float(-p.lr_mul * (__float_as_int(vq[e]) - 0x4B400000), k2));
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(y[e]));
+            for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
             const int ia = group_max<L>((int)amax, gmask);
             ew2 = finalize_exp(ia ? r2 + need_off32q((uint32_t)ia, p.qb) : kNoExp);
             fit2 = k2 == 0 || ew2 == kEZero || ew2 - r2 >= 2;
             const float sc = pow2f(ew2 == kEZero ? 0 : r2 - ew2);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) y[e] = __fmaf_rn(y[e], sc, kMagic);
+            for (int e = 0; e < E; ++e) y[e] = __fmaf_rn(y[e], sc, kMagic);
         }
         if (!(fit1 && fit2)) {
-            sgd_group_exact<L>(p, t0, r * (16 * L), r, 16 * L, li, gmask);
+            sgd_group_exact<L>(p, t0, r * G, r, G, li, gmask);
         } else {
-            uint32_t ov[4], ow[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                ov[q] = low_bytes4(vq[4 * q], vq[4 * q + 1], vq[4 * q + 2], vq[4 * q + 3]);
-                ow[q] = low_bytes4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+            for (int k = 0; k < CPL; ++k) {
+                uint32_t ov[4], ow[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int e = 16 * k + 4 * q;
+                    ov[q] = low_bytes4(vq[e], vq[e + 1], vq[e + 2], vq[e + 3]);
+                    ow[q] = low_bytes4(y[e], y[e + 1], y[e + 2], y[e + 3]);
+                }
+                const int64_t at = r * G + (k * L + li) * 16;
+                *reinterpret_cast<uint4 *>(tv + at) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+                *reinterpret_cast<uint4 *>(tw + at) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
             }
-            const int64_t at = r * (16 * L) + li * 16;
-            *reinterpret_cast<uint4 *>(tv + at) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-            *reinterpret_cast<uint4 *>(tw + at) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
             if (li == 0) {
                 tve[r] = (int8_t)ev2;
                 twe[r] = (int8_t)ew2;
             }
         }
-        cw = nw4, cv = nv4, cg = ng4;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) cw[k] = nw4[k], cv[k] = nv4[k], cg[k] = ng4[k];
         ev = nev, eg = neg, ew = new_;
     }
 }
