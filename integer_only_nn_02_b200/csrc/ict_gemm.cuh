@@ -885,11 +885,13 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 // with staged output, stores the warpgroup's share of the tile)
                 named_bar_sync(bar_id, 128);
                 if (et == 0) {
+                    // the accumulator is free first: issuing the store can wait on the
+                    // SM's TMA unit, which the next tile's MMAs must not
+                    mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
                     if (TS && valid_rows > 0) {
                         tma_store_2d(&tmY, smem_u32(sStage + wg * (128 * 64)), n0 + c_lo, (int)row_base);
                         bulk_commit();
                     }
-                    mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
                 }
             } else {
                 mbar_arrive(bar_tempty + 8 * acc);
