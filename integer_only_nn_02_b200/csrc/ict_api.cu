@@ -297,21 +297,33 @@ unsigned transpose_tiles(AlignPair &P, int n) {
 }
 
 // The transposing alignment of the first n jobs of P: persistent streaming blocks (three
-// per SM) unless a job scans its own column exponents, then one block per tile.
+// per SM) unless a job scans its own column exponents, then one block per tile.  The
+// streaming kernel's exact form serves jobs aligned per column from the column-max
+// scratch with one group row per row and power-of-two group widths.
 void launch_align_transpose(AlignPair &P, int n, int sms, cudaStream_t s) {
     const unsigned tiles = transpose_tiles(P, n);
     const bool scan = P.a[0].col_scan || (n > 1 && P.a[1].col_scan);
-    if (scan)
+    if (scan) {
         align_transpose_kernel<<<tiles, 256, 0, s>>>(P);
+        return;
+    }
+    bool exact = true;
+    for (int z = 0; z < n; ++z) {
+        const AlignArgs &a = P.a[z];
+        exact = exact && a.axis == 0 && a.col_max && a.g_rows == 1 && a.gv_shift1 > 0;
+    }
+    const unsigned grid = std::min<unsigned>(tiles, (unsigned)sms * 3);
+    if (exact)
+        align_transpose_stream_kernel<true><<<grid, 256, 0, s>>>(P);
     else
-        align_transpose_stream_kernel<<<std::min<unsigned>(tiles, (unsigned)sms * 3), 256, 0, s>>>(P);
+        align_transpose_stream_kernel<false><<<grid, 256, 0, s>>>(P);
 }
 
 // Rows of 16-byte vectors, one row per segment of L lanes.  The narrowest segment whose
 // lanes hold at most six vectors each (the most bytes in flight per lane) and stay nine
 // tenths busy, else the busiest; NV = the row's vectors per lane rounded up to an
-// instantiated count.  Rows of more than 192 vectors or (computing e*) more than 2 L
-// groups, and 2^31 rows or more, go to the generic kernel.  Persistent grid: two blocks
+// instantiated count.  Rows of fewer than 8 or more than 192 vectors or (computing e*)
+// more than 2 L groups, and 2^31 rows or more, go to the generic kernel.  Persistent grid: two blocks
 // per SM.
 int launch_align_rows(const AlignArgs &a, cudaStream_t s, int sms) {
     const int64_t vpr = a.cols / 16;
@@ -325,7 +337,7 @@ int launch_align_rows(const AlignArgs &a, cudaStream_t s, int sms) {
         if (eff >= 0.9) { L = l; break; }
         if (eff > best + 1e-12) best = eff, L = l;
     }
-    if (L == 0 || a.rows >= (1ll << 31)) {
+    if (L == 0 || vpr < 8 || a.rows >= (1ll << 31)) {  // narrow rows: four threads per row
         align_rows_wide_kernel<<<dim3((unsigned)cdiv64(a.cols, 256), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);
         return ICT_OK;
     }

@@ -532,19 +532,25 @@ __device__ __forceinline__ void tr_tile_decode(const AlignPair &P, int tile, int
     c0 = (int64_t)(t - tr * P.ntc[z]) * 128;
 }
 
+// EXACT: every job aligns per column from a column-max scratch, with one group row per
+// row and g_cols / 16 a power of two (or one group across the row): the group column
+// is a shift and no division or target branch remains in the loop.
+template <bool EXACT>
 __device__ __forceinline__ void tr_tile_load(const AlignArgs &a, int64_t r0, int64_t j, int rq, TrTile &b) {
     if (j >= a.cols) return;
-    const int64_t gcol = idiv(j, a.g_cols);
+    const int64_t gcol = EXACT ? (j >> (a.gv_shift1 + 3)) : idiv(j, a.g_cols);
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
         const int64_t i = r0 + 4 * rq + t;
         const bool in = i < a.rows;
         b.raw[t] = in ? *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j) : make_uint4(0, 0, 0, 0);
-        b.eg[t] = in ? (int)a.in_exp[idiv(i, a.g_rows) * a.ngc + gcol] : kEZero;
+        b.eg[t] = in ? (int)a.in_exp[(EXACT ? i : idiv(i, a.g_rows)) * a.ngc + gcol] : kEZero;
     }
-    b.es = a.axis == 0 ? align_target(a, 0, j) : 0;
+    if (EXACT) b.es = estar_of(a.col_max[gcol]);
+    else b.es = a.axis == 0 ? align_target(a, 0, j) : 0;
 }
 
+template <bool EXACT>
 __global__ void __launch_bounds__(256, 3) align_transpose_stream_kernel(const __grid_constant__ AlignPair P) {
     __shared__ uint4 tile[2][128][8];  // [buffer][output row = input column][16-byte chunk, swizzled]
     __shared__ RneK tk[9];
@@ -559,24 +565,24 @@ __global__ void __launch_bounds__(256, 3) align_transpose_stream_kernel(const __
     int z;
     int64_t r0, c0;
     tr_tile_decode(P, tile_id, z, r0, c0);
-    tr_tile_load(P.a[z], r0, c0 + 16 * cc, rq, cur);
+    tr_tile_load<EXACT>(P.a[z], r0, c0 + 16 * cc, rq, cur);
     for (int buf = 0; tile_id < total; tile_id += gridDim.x, buf ^= 1) {
         const int next = tile_id + gridDim.x;
         int zn = 0;
         int64_t rn = 0, cn = 0;
         if (next < total) {
             tr_tile_decode(P, next, zn, rn, cn);
-            tr_tile_load(P.a[zn], rn, cn + 16 * cc, rq, nxt);
+            tr_tile_load<EXACT>(P.a[zn], rn, cn + 16 * cc, rq, nxt);
         }
         const AlignArgs &a = P.a[z];
         const int64_t j = c0 + 16 * cc;
         if (j < a.cols) {
-            if (a.axis == 0 && a.col_max && r0 == 0 && rq == 0)
+            if ((EXACT || (a.axis == 0 && a.col_max)) && r0 == 0 && rq == 0)
                 for (int q = 0; q < 16; ++q) a.e_star[j + q] = (int8_t)cur.es;
             uint4 v[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                const int es = a.axis == 0 ? cur.es : align_target(a, r0 + 4 * rq + t, j);
+                const int es = EXACT || a.axis == 0 ? cur.es : align_target(a, r0 + 4 * rq + t, j);
                 v[t] = rne_shift16_k(cur.raw[t], tk[rne_index(es, cur.eg[t])]);
             }
             const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w}, {v[1].x, v[1].y, v[1].z, v[1].w},
