@@ -615,7 +615,6 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     if (pair) {
         if (load != LOAD_2D || bk != 128 || (grid & 1)) return ICT_ERR_LAYOUT;
         const CUtensorMap &y = ty ? *ty : tb;  // the output map, for staged stores
-        if (bn == 128) return launch_gemm_pair_t<128>(ta, tb, y, p, grid, s);
         if (bn == 192) return launch_gemm_pair_t<192>(ta, tb, y, p, grid, s);
         if (bn == 256) return launch_gemm_pair_t<256>(ta, tb, y, p, grid, s);
         return ICT_ERR_LAYOUT;
@@ -726,9 +725,10 @@ ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out,
         const int64_t G = out->g_cols;
         if (K <= 1024 && N % 128 == 0 && G == 32) pl.bn = 128, pl.nwg = 4;
     }
-    // large Products run on pairs of CTAs: a 256 x BN tile per pair halves the operand
-    // bytes each SM draws from L2 per multiply-add, which bounds 128-row tiles
-    pl.pair = pl.nwg == 2 && pl.bn >= 128 && pl.bn % 64 == 0 && M >= 2048 && sms >= 2;
+    // large Products with wide tiles run on pairs of CTAs: a 256 x BN tile per pair halves
+    // the B bytes each SM draws per multiply-add.  128-wide tiles stay on single CTAs,
+    // whose 128 x 128 steps measured faster than the pair's 256 x 128 ones.
+    pl.pair = pl.nwg == 2 && pl.bn >= 192 && pl.bn % 64 == 0 && M >= 2048 && sms >= 2;
     const int units_per_wave = pl.pair ? sms / 2 : sms;
     pl.n_kblk = (int)cdiv64(K, 128);
     pl.n_mtiles = (int)cdiv64(M, pl.pair ? 256 : 128);

@@ -136,11 +136,10 @@ def test_linear_bwd_weight(ict, case, per_row):
 
 
 @pytest.mark.parametrize("M,N,K,G,wspan", [
-    (2600, 768, 256, 64, (-12, -6)),     # 128-wide pair tiles; the last tile's second CTA has no rows
-    (2100, 512, 1536, 32, (-12, -6)),    # 32-column groups, a long contraction
-    (2048, 704, 384, 64, (-12, -6)),     # a ragged last N tile
-    (3000, 512, 256, 128, (-12, -6)),    # 128-column groups (generic epilogue on pairs)
-    (2300, 512, 256, 64, (-40, -6)),     # column exponents far apart: the exact per-element path
+    (12000, 576, 256, 64, (-12, -6)),    # 192-wide pair tiles, ragged last M tile
+    (12000, 576, 256, 64, (-40, -6)),    # the same with column exponents far apart: the exact per-element path
+    (2600, 768, 256, 64, (-12, -6)),     # 128-wide tiles on single CTAs
+    (3000, 512, 256, 128, (-12, -6)),    # 128-column groups (generic epilogue)
     (4200, 1024, 256, 64, (-12, -6)),    # 256-wide pair tiles, four epilogue warpgroups, TMA-store output
     (4100, 1024, 1280, 32, (-12, -6)),   # the same with 32-column groups; ragged last M tile
     (4160, 1024, 384, 64, (-40, -6)),    # staged output from the exact per-element path
