@@ -350,8 +350,9 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         }
         for (int a = 0; a < NACC; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
-            // pairs: one arrival per epilogue warpgroup of each CTA that handles the tile
-            mbar_init(bar_tempty + 8 * a, PAIR ? 2 * wpt : 128 * wpt);
+            // pairs: one local arrival per epilogue warpgroup that handles the tile, and on
+            // the first CTA one more, forwarded from the second CTA's barrier
+            mbar_init(bar_tempty + 8 * a, PAIR ? (leader ? wpt + 1 : wpt) : 128 * wpt);
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_bres, 1);
@@ -532,6 +533,22 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 if constexpr (PAIR) umma_commit_pair(bar_drain);
                 else umma_commit(bar_drain);
                 mbar_wait(bar_drain, 0, p.drain_ns, nullptr);
+            }
+        }
+    } else if (PAIR && warp == 3) {
+        // ------------------------------------------------------------ release forwarder
+        // second CTA of a pair: once all of its epilogue warpgroups have released an
+        // accumulator (its local barrier's phase for that tile), one remote arrival tells
+        // the first CTA, whose MMA thread waits for it with its own warpgroups' arrivals
+        if (!leader && lane == 0) {
+            int it = 0;
+            for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas, ++it) {
+                const int acc = it % NACC;
+                if (!mbar_wait(bar_tempty + 8 * acc, (it / NACC) & 1, p.wait_ns, abort_flag)) {
+                    fail();
+                    break;
+                }
+                mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
             }
         }
     } else if (warp >= 4) {
@@ -886,8 +903,10 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 named_bar_sync(bar_id, 128);
                 if (et == 0) {
                     // the accumulator is free first: issuing the store can wait on the
-                    // SM's TMA unit, which the next tile's MMAs must not
-                    mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * acc, 0));
+                    // SM's TMA unit, which the next tile's MMAs must not.  The arrival is
+                    // local (a remote one takes about a thousand cycles); the second CTA's
+                    // warp 3 forwards its barrier's phases to the first CTA.
+                    mbar_arrive(bar_tempty + 8 * acc);
                     if (TS && valid_rows > 0) {
                         tma_store_2d(&tmY, smem_u32(sStage + wg * (128 * 64)), n0 + c_lo, (int)row_base);
                         bulk_commit();
