@@ -541,6 +541,9 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
         if constexpr (LOAD == LOAD_CONV) {
             if (p.epi == EPI_RO16) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_RO16>, 2, kB2);
         }
+        if constexpr (LOAD == LOAD_2D) {
+            if (p.epi == EPI_RO16R) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_RO16R>, 2, kB2);
+        }
         if (p.epi != EPI_FIT_ROW) return ICT_ERR_LAYOUT;
         const int gt = p.G >= p.N ? BN : p.G;  // group width inside a tile
         if constexpr (LOAD == LOAD_2D && BN <= 128) {
@@ -611,7 +614,7 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
     if (p.nwg != 4 || p.epi != EPI_FIT_ROW || pair) p.nwg = 2;
-    p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || (gt < bn && (bn / 2) % gt == 0));
+    p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || p.epi == EPI_RO16R || (gt < bn && (bn / 2) % gt == 0));
     if (pair) {
         if (load != LOAD_2D || bk != 128 || (grid & 1)) return ICT_ERR_LAYOUT;
         const CUtensorMap &y = ty ? *ty : tb;  // the output map, for staged stores
@@ -707,9 +710,13 @@ Operand operand_cols(const ict_tensor *t, Ws &ws, AlignJob *jobs, int *njobs) {
 struct ProductPlan {
     int bn, nwg, splits, kblk_per_split, n_kblk, n_mtiles, n_ntiles, units, grid;
     bool fused;
-    bool pair;  // clusters of two CTAs on 256-row tiles (tcgen05 cta_group::2)
+    bool pair;   // clusters of two CTAs on 256-row tiles (tcgen05 cta_group::2)
+    bool ro16r;  // one output group per row across tiles: int16 rounded-to-odd sums + a round pass
     int32_t *ws32;
     int64_t ws_ld;
+    int16_t *ws16;
+    int64_t ws16_ld, tn_ld;
+    int32_t *tneed;
 };
 
 // Tiling of D[M][N] = A[M][K] B[N][K]^T with FIT into the row-local groups of `out`.
@@ -750,8 +757,19 @@ ProductPlan plan_product(int64_t M, int64_t N, int64_t K, const ict_tensor *out,
     const int64_t G = out->g_cols;
     const bool groups_in_tile = (G >= N) ? (N <= pl.bn) : (pl.bn % G == 0 && G % 32 == 0);
     pl.fused = !raw && pl.splits == 1 && groups_in_tile;
+    // one group per row spanning several tiles, no split: each (row, tile half) rounds its
+    // sums to odd into int16 with its own need; a streaming pass rounds to the row's group
+    pl.ro16r = !raw && !pl.fused && pl.splits == 1 && G >= N && !pl.pair && pl.nwg == 2 && N % 16 == 0 &&
+               out->ld % 16 == 0 && (reinterpret_cast<uintptr_t>(out->mant) & 15) == 0;
     pl.ws_ld = round_up(N, 32);
-    pl.ws32 = pl.fused ? nullptr : (int32_t *)ws.take((size_t)pl.splits * M * pl.ws_ld * 4);
+    pl.ws32 = (pl.fused || pl.ro16r) ? nullptr : (int32_t *)ws.take((size_t)pl.splits * M * pl.ws_ld * 4);
+    pl.ws16 = nullptr, pl.tneed = nullptr, pl.ws16_ld = pl.tn_ld = 0;
+    if (pl.ro16r) {
+        pl.ws16_ld = round_up(N, 32);  // the epilogue writes 32-column chunks
+        pl.ws16 = (int16_t *)ws.take((size_t)M * pl.ws16_ld * 2);
+        pl.tn_ld = (int64_t)pl.n_ntiles * 2;
+        pl.tneed = (int32_t *)ws.take((size_t)M * pl.tn_ld * 4);
+    }
     return pl;
 }
 
@@ -808,14 +826,37 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     p.stage_tx_bytes = (uint32_t)(pl.pair ? 2 * (128 * 128 + (pl.bn / 2) * 128) : 128 * 128 + pl.bn * 128);
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
-    p.epi = pl.fused ? EPI_FIT_ROW : EPI_I32;
+    p.epi = pl.fused ? EPI_FIT_ROW : (pl.ro16r ? EPI_RO16R : EPI_I32);
     p.qb = g_mantissa_bits.load(std::memory_order_relaxed);
     p.nwg = pl.nwg;
+    p.ws16 = pl.ws16;
+    p.ws16_ld = pl.ws16_ld;
+    p.tile_need = pl.tneed;
+    p.tn_ld = pl.tn_ld;
     if ((st = launch_gemm(pl.bn, 128, LOAD_2D, ta, tb, p, pl.grid, s, 2.0 * (double)M * (double)N * (double)K,
                           pl.pair, staged ? &ty : nullptr)))
         return st;
     if (pl.fused) return ICT_OK;
     if (raw_acc) return launch_sum_slices(pl, M, N, raw_acc, raw_bits, raw_ld, s);
+    if (pl.ro16r) {
+        Ro16RowsArgs r;
+        memset(&r, 0, sizeof(r));
+        r.v = pl.ws16;
+        r.rows = M;
+        r.cols = N;
+        r.ld = pl.ws16_ld;
+        r.need = pl.tneed;
+        r.tn_ld = pl.tn_ld;
+        r.part_cols = pl.bn / 2;
+        r.out = out->mant;
+        r.out_ld = out->ld;
+        r.out_exp = out->exp;
+        r.out_exp_ld = n_grp_cols(out);
+        KTimer kt(s, KC_REQUANT, 3.0 * (double)M * (double)N);
+        ro16_rows_round_kernel<<<(unsigned)cdiv64(M, 8), 256, 0, s>>>(r);
+        counted(1);
+        return launch_status();
+    }
     RequantArgs a;
     memset(&a, 0, sizeof(a));
     a.qb = g_mantissa_bits.load(std::memory_order_relaxed);

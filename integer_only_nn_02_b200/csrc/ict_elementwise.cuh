@@ -1192,6 +1192,71 @@ struct Ro16RoundArgs {
     int8_t *out_exp;
     int act;  // fused activation (ACT_*)
 };
+// The round pass of the Product's EPI_RO16R output (one group per row spanning tiles):
+// the row's group exponent e = finalize(max of its parts' needs), and every int16 t of
+// part k (rounded to odd at need_k - 7) becomes RNE(t * 2^(need_k - 7 - e)), a right shift
+// of at least 7 bits, which equals RNE of the exact sum (the same lemma as above).  One
+// warp per row, 16 columns per lane step (part_cols a multiple of 16).
+struct Ro16RowsArgs {
+    const int16_t *v;
+    int64_t rows, cols, ld;
+    const int32_t *need;  // [rows][tn_ld]: need of (row, part), kNoExp when all zero
+    int64_t tn_ld;
+    int part_cols;
+    int8_t *out;
+    int64_t out_ld;
+    int8_t *out_exp;
+    int64_t out_exp_ld;
+};
+__device__ __forceinline__ uint4 ro16_round16(const int16_t *src, int tn, int e) {
+    const int64_t s64 = (int64_t)e - ((int64_t)tn - 7);
+    const int s = (int)(s64 > 40 ? 40 : s64);
+    const uint4 x0 = reinterpret_cast<const uint4 *>(src)[0], x1 = reinterpret_cast<const uint4 *>(src)[1];
+    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint32_t o[4];
+    if (s >= 2 && s < 32) {
+        const int m = 1 << (32 - s), bias = (1 << (s - 1)) - 1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            int y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int x = (int)(int16_t)(xw[2 * q + (k >> 1)] >> (16 * (k & 1)));
+                y[k] = __mulhi(x + bias + (__mulhi(x, m) & 1), m);
+            }
+            o[q] = pack4(y[0], y[1], y[2], y[3]);
+        }
+    } else if (s >= 32) {
+        o[0] = o[1] = o[2] = o[3] = 0u;  // |t| < 2^15: below half a unit
+    } else {
+        // e below the part's need only after an exponent overflow (status raised)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            int y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                y[k] = requant32((int)(int16_t)(xw[2 * q + (k >> 1)] >> (16 * (k & 1))), tn - 7, e);
+            o[q] = pack4(y[0], y[1], y[2], y[3]);
+        }
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+__global__ void __launch_bounds__(256) ro16_rows_round_kernel(const __grid_constant__ Ro16RowsArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t i = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (i >= a.rows) return;
+    const int32_t *nrow = a.need + i * a.tn_ld;
+    int m = kNoExp;
+    for (int64_t k = lane; k < a.tn_ld; k += 32) m = max(m, nrow[k]);
+    const int e = finalize_exp(warp_max(m));
+    if (lane == 0) a.out_exp[i * a.out_exp_ld] = (int8_t)e;
+    const int64_t nchunk = a.cols / 16;
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        const int64_t j0 = 16 * c;
+        *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = ro16_round16(a.v + i * a.ld + j0, nrow[j0 / a.part_cols], e);
+    }
+}
+
 __global__ void __launch_bounds__(256) ro16_round_kernel(const __grid_constant__ Ro16RoundArgs a) {
     const int64_t cv = a.cols / 16;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;

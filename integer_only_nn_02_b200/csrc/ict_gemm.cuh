@@ -36,6 +36,8 @@ enum EpiMode : int {
     EPI_I32 = 1,      // raw int32 partials to a workspace slice (split-K)
     EPI_RO16 = 2,     // groups spanning all rows: int16 sums rounded to odd at a per-tile
                       // exponent, the tile's need and the group's running max need
+    EPI_RO16R = 3,    // one group per row spanning tiles: int16 sums rounded to odd at the
+                      // exponent of the (row, tile part)'s need, and that need
 };
 // LOAD_2D         A, B: K-major rows from 2-D tensor maps (linear layers)
 // LOAD_CONV       A: one filter tap of NHWC activations per K block (4-D box), B: K-major
@@ -69,6 +71,9 @@ struct GemmParams {
     int64_t ws16_ld;
     int32_t *tile_need;
     int32_t *gmax;
+    // EPI_RO16R: the same int16 form for one group per row spanning several tiles, with the
+    // need of each (row, tile part) in tile_need[row * tn_ld + n tile * parts + part]
+    int64_t tn_ld;
     // implicit-GEMM convolution: output tile = cv_rows image rows of width cv_W
     int cv_W, cv_P, cv_rows, cv_tiles_per_img, cv_cblk, cv_S, cv_pad, cv_sign;
     // conv: every K block of the weight operand held in shared memory for the whole kernel
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     constexpr int NACC = Q4 ? 2 : NWG;
     // warpgroups sharing one tile (each takes a contiguous share of its columns)
     const int wpt = Q4 ? 4 : (p.epi_split ? 2 : 1);
-    constexpr bool I32 = OUTK == EPI_I32, RO16 = OUTK == EPI_RO16;
+    constexpr bool I32 = OUTK == EPI_I32, RO16 = OUTK == EPI_RO16, RO16R = OUTK == EPI_RO16R;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(BK == 128 || BK == 64 || (BK == 256 && LOAD == LOAD_CONV_WGRAD), "BK");
     extern __shared__ uint8_t smem_raw[];
@@ -679,6 +684,71 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                                 *reinterpret_cast<uint4 *>(dst + c + 4 * q) =
                                     make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
+                }
+            } else if constexpr (RO16R) {
+                // One group per row spanning several tiles.  Pass A: the row's largest
+                // need() over this warpgroup's columns of the tile (thread-local: the thread
+                // owns the row).  Pass B: every sum rounded to odd at e1 = that need - 7 as
+                // int16 (|t| < 127.5 * 2^7); the streaming pass takes the row's largest need
+                // over all parts as the group exponent e >= e1 + 7, and its RNE by e - e1 >= 2
+                // bits equals RNE of the exact sum (Boldo and Melquiond, as for RO16).
+                const int gf = gfast[0];
+                int need = kNoExp;
+                for (int c = c_lo; c < c_hi; c += 32) {
+                    tmem_ld32(taddr + c, v);
+                    tmem_ld_wait();
+                    if (!valid || n0 + c >= p.N) continue;
+                    if (gf) {
+                        int ymax = 0, ymin = 0;
+#pragma unroll
+                        for (int q = 0; q < 32; q += 4) {
+                            const int4 d4 = gf == 2 ? make_int4(1, 1, 1, 1) : *reinterpret_cast<const int4 *>(colD + c + q);
+                            const int y0 = (int)v[q] * d4.x, y1 = (int)v[q + 1] * d4.y;
+                            const int y2 = (int)v[q + 2] * d4.z, y3 = (int)v[q + 3] * d4.w;
+                            ymax = max(ymax, max(max(y0, y1), max(y2, y3)));
+                            ymin = min(ymin, min(min(y0, y1), min(y2, y3)));
+                        }
+                        const int amax = max(ymax, -ymin);
+                        if (amax) need = max(need, ea + gmin[0] + need_off32q((uint32_t)amax, p.qb));
+                    } else {
+#pragma unroll 8
+                        for (int q = 0; q < 32; ++q) {
+                            const int32_t x = (int32_t)v[q];
+                            if (x) need = max(need, ea + colE[c + q] + need_off32q((uint32_t)(x < 0 ? -x : x), p.qb));
+                        }
+                    }
+                }
+                if (valid) p.tile_need[grow * p.tn_ld + (n0 / BN) * wpt + part] = need;
+                const int e1 = need - 7;
+                auto ro = [](int y, int s) {  // floor(y / 2^s) with the sticky bit ORed in
+                    if (s <= 0) return y << min(-s, 31);
+                    s = min(s, 31);
+                    return (y >> s) | (int)((y & ((1 << s) - 1)) != 0);
+                };
+                for (int c = c_lo; c < c_hi; c += 32) {
+                    tmem_ld32(taddr + c, v);
+                    tmem_ld_wait();
+                    if (!valid || n0 + c >= p.N) continue;
+                    uint32_t w[16];
+                    if (need <= kNoExp) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) w[q] = 0u;
+                    } else if (gf) {
+                        const int s = e1 - ea - gmin[0];  // uniform over the row
+#pragma unroll
+                        for (int q = 0; q < 32; q += 2) {
+                            const int m0 = gf == 2 ? 1 : colD[c + q], m1 = gf == 2 ? 1 : colD[c + q + 1];
+                            w[q >> 1] = __byte_perm((uint32_t)ro((int)v[q] * m0, s), (uint32_t)ro((int)v[q + 1] * m1, s), 0x5410);
+                        }
+                    } else {
+#pragma unroll 4
+                        for (int q = 0; q < 32; q += 2)
+                            w[q >> 1] = __byte_perm((uint32_t)ro((int)v[q], e1 - ea - colE[c + q]),
+                                                    (uint32_t)ro((int)v[q + 1], e1 - ea - colE[c + q + 1]), 0x5410);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.ws16 + grow * p.ws16_ld + n0 + c);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                 }
             } else if constexpr (RO16) {
                 // Groups spanning all rows.  Pass A: the largest need() of each group over

@@ -135,6 +135,25 @@ def test_linear_bwd_weight(ict, case, per_row):
     status_ok(ict)
 
 
+@pytest.mark.parametrize("M,N,K,xg,xspan", [
+    (700, 400, 336, 64, (-10, -4)),     # dW 400 x 336: rows span 3 tiles, a 16-column overhang
+    (896, 256, 528, 16, (-10, -4)),     # 16-column X groups: column exponents differ within a tile
+    (500, 320, 640, 16, (-40, -4)),     # column exponents far apart: the exact per-element path
+    (64, 144, 1024, 64, (-10, -4)),     # a 144-row dW with every row spanning 8 tiles
+])
+def test_linear_bwd_weight_row_groups_across_tiles(ict, M, N, K, xg, xspan):
+    """dW = dY^T X with one output group per row spanning several tiles and no split K:
+    the Product's int16 round-to-odd output with a need per (row, tile half), then the
+    streaming pass that rounds each row to its group exponent, against the oracle."""
+    rng = np.random.default_rng(M + N + K + xg)
+    X = rand_ce(rng, M, K, 1, xg, elo=xspan[0], ehi=xspan[1], zero_groups=0.05)
+    dY = with_groups(clipped_laplace(rng, (M, N)), 1, 32, lambda g: rng.integers(-16, -10, size=g))
+    ref = oracle.linear_bwd_weight(dY, X, 1, K)
+    got = ict.linear_bwd_weight(ict.DevCE.from_host(dY), ict.DevCE.from_host(X), K).to_host()
+    same(got, ref, "bwd-weight, row groups across tiles")
+    status_ok(ict)
+
+
 @pytest.mark.parametrize("M,N,K,G,wspan", [
     (12000, 576, 256, 64, (-12, -6)),    # 192-wide pair tiles, ragged last M tile
     (12000, 576, 256, 64, (-40, -6)),    # the same with column exponents far apart: the exact per-element path
