@@ -445,6 +445,20 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
     const int64_t r0 = (int64_t)tr * 128, c0 = (int64_t)tcol * 128;
     const int rq = 4 * warp + (lane & 3), cc = lane >> 2;  // row quad 0..31, column chunk 0..7
     const int64_t j = c0 + 16 * cc;
+    // the tile's loads first (rows beyond the tensor read nothing): they do not depend on
+    // the targets, so their latency overlaps the column scan
+    uint4 raw[4];
+    int eg[4];
+    if (j < a.cols) {
+        const int64_t gcol = idiv(j, a.g_cols);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int64_t i = r0 + 4 * rq + t;
+            const bool in = i < a.rows;
+            raw[t] = in ? *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j) : make_uint4(0, 0, 0, 0);
+            eg[t] = in ? (int)a.in_exp[idiv(i, a.g_rows) * a.ngc + gcol] : kEZero;
+        }
+    }
     int64_t g_first = 0;
     if (a.col_scan) {
         // a strip of at most 128 columns spans at most 9 groups (groups are >= 16 wide)
@@ -455,12 +469,19 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
         const int64_t ngr = idiv(a.rows + a.g_rows - 1, a.g_rows);
         const int k = threadIdx.x % ng, per = 256 / ng;
         if (threadIdx.x < per * ng) {
-            int m = kNoExp;
-            for (int64_t r = threadIdx.x / ng; r < ngr; r += per) {
-                const int e = a.in_exp[r * a.ngc + g_first + k];
-                if (e != kEZero) m = max(m, e);
+            // E_ZERO (-128) is the smallest byte: it only wins where every member is zero
+            int m0 = kEZero, m1 = kEZero, m2 = kEZero, m3 = kEZero;
+            const int8_t *e = a.in_exp + g_first + k;
+            int64_t r = threadIdx.x / ng;
+            for (; r + 3 * per < ngr; r += 4 * per) {  // four loads in flight
+                m0 = max(m0, (int)e[r * a.ngc]);
+                m1 = max(m1, (int)e[(r + per) * a.ngc]);
+                m2 = max(m2, (int)e[(r + 2 * per) * a.ngc]);
+                m3 = max(m3, (int)e[(r + 3 * per) * a.ngc]);
             }
-            if (m > kNoExp) atomicMax(&gmx[k], m);
+            for (; r < ngr; r += per) m0 = max(m0, (int)e[r * a.ngc]);
+            const int m = max(max(m0, m1), max(m2, m3));
+            if (m != kEZero) atomicMax(&gmx[k], m);
         }
     }
     __syncthreads();
@@ -469,17 +490,6 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
         if (a.axis == 0 && (a.col_max || a.col_scan) && tr == 0 && rq == 0) {
             const int es = a.col_scan ? es_col : align_target(a, 0, j);
             for (int b = 0; b < 16; ++b) a.e_star[j + b] = (int8_t)es;
-        }
-        // all loads first (rows beyond the tensor read nothing), then the shifts
-        uint4 raw[4];
-        int eg[4];
-        const int64_t gcol = idiv(j, a.g_cols);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int64_t i = r0 + 4 * rq + t;
-            const bool in = i < a.rows;
-            raw[t] = in ? *reinterpret_cast<const uint4 *>(a.in + i * a.ld + j) : make_uint4(0, 0, 0, 0);
-            eg[t] = in ? (int)a.in_exp[idiv(i, a.g_rows) * a.ngc + gcol] : kEZero;
         }
         // axis 0: one target for the thread's 16 columns in all four rows
         const int es_c = a.axis == 0 ? (a.col_scan ? es_col : align_target(a, 0, j)) : 0;
@@ -1208,10 +1218,9 @@ struct Ro16RowsArgs {
     int8_t *out_exp;
     int64_t out_exp_ld;
 };
-__device__ __forceinline__ uint4 ro16_round16(const int16_t *src, int tn, int e) {
+__device__ __forceinline__ uint4 ro16_round16(uint4 x0, uint4 x1, int tn, int e) {
     const int64_t s64 = (int64_t)e - ((int64_t)tn - 7);
     const int s = (int)(s64 > 40 ? 40 : s64);
-    const uint4 x0 = reinterpret_cast<const uint4 *>(src)[0], x1 = reinterpret_cast<const uint4 *>(src)[1];
     const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
     uint32_t o[4];
     if (s >= 2 && s < 32) {
@@ -1246,14 +1255,30 @@ __global__ void __launch_bounds__(256) ro16_rows_round_kernel(const __grid_const
     const int64_t i = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (i >= a.rows) return;
     const int32_t *nrow = a.need + i * a.tn_ld;
+    const int16_t *vrow = a.v + i * a.ld;
+    int8_t *orow = a.out + i * a.out_ld;
+    const int64_t nchunk = a.cols / 16;
+    // the first four chunks of this lane are loaded before the row's exponent is known
+    constexpr int P = 4;
+    uint4 x[P][2];
+#pragma unroll
+    for (int u = 0; u < P; ++u) {
+        const int64_t c = lane + 32 * u;
+        if (c < nchunk) x[u][0] = reinterpret_cast<const uint4 *>(vrow + 16 * c)[0], x[u][1] = reinterpret_cast<const uint4 *>(vrow + 16 * c)[1];
+    }
     int m = kNoExp;
     for (int64_t k = lane; k < a.tn_ld; k += 32) m = max(m, nrow[k]);
     const int e = finalize_exp(warp_max(m));
     if (lane == 0) a.out_exp[i * a.out_exp_ld] = (int8_t)e;
-    const int64_t nchunk = a.cols / 16;
-    for (int64_t c = lane; c < nchunk; c += 32) {
-        const int64_t j0 = 16 * c;
-        *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = ro16_round16(a.v + i * a.ld + j0, nrow[j0 / a.part_cols], e);
+#pragma unroll
+    for (int u = 0; u < P; ++u) {
+        const int64_t c = lane + 32 * u;
+        if (c < nchunk)
+            *reinterpret_cast<uint4 *>(orow + 16 * c) = ro16_round16(x[u][0], x[u][1], nrow[(16 * c) / a.part_cols], e);
+    }
+    for (int64_t c = lane + 32 * P; c < nchunk; c += 32) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(vrow + 16 * c);
+        *reinterpret_cast<uint4 *>(orow + 16 * c) = ro16_round16(src[0], src[1], nrow[(16 * c) / a.part_cols], e);
     }
 }
 
