@@ -118,6 +118,27 @@ __device__ __forceinline__ uint32_t pack4b(int a, int b, int c, int d) {
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
+// RNE(y * 2^-S) on the fp32 pipe, for |y| < 2^22 and 0 <= S <= 22.  The bit pattern
+// 0x4B400000 + y is the float 1.5 * 2^23 + y exactly (the sum stays in the binade of unit
+// spacing); one FMA by 2^-S with the addend 1.5 * 2^23 * (1 - 2^-S) (exact for S <= 22)
+// gives 1.5 * 2^23 + y * 2^-S rounded once, to nearest even, at the unit.  The low byte of
+// the result's bit pattern is then the rounded value in two's complement (|value| <= 128).
+struct RneF32 {
+    float sc, add;
+};
+__device__ __forceinline__ RneF32 rne_f32_consts(int S) {
+    const float sc = __int_as_float((127 - S) << 23);
+    return {sc, __fmaf_rn(-12582912.f, sc, 12582912.f)};
+}
+__device__ __forceinline__ uint32_t rne_f32(int y, RneF32 k) {
+    return __float_as_uint(__fmaf_rn(__int_as_float(0x4B400000 + y), k.sc, k.add));
+}
+// the group may take the fp32 rounding: every magnitude below 2^22, a right shift of at
+// most 22 bits, and an exponent that was not capped (a capped one saturates instead)
+__device__ __forceinline__ bool rne_f32_ok(bool valid, int amax, int S, int need) {
+    return !valid || (amax < (1 << 22) && S >= 0 && S <= 22 && need <= 127);
+}
+
 // Fast epilogue of one output group of NC x 32 columns of an accumulator row, the group
 // on the fast path: y = acc * 2^d_n (d_n = column shift inside the group, |y| < 2^30),
 // the group exponent from max |y|, then one RNE shift.  TMEM is read once (all NC chunks
@@ -165,6 +186,24 @@ __device__ __forceinline__ void epi_fast(const GemmParams &p, uint32_t taddr, co
     const int e = finalize_exp(need);
     // mantissa = RNE(y * 2^-S), S = e - ea - gm uniform over the row's group
     const int S = (e == kEZero) ? 0 : e - ea - gm;
+    if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
+    if (__all_sync(0xffffffffu, rne_f32_ok(valid, amax, S, need))) {
+        const RneF32 k = rne_f32_consts(S);
+        if (TS || valid) {
+            int8_t *dst = p.out + grow * p.out_ld + ncol;
+#pragma unroll
+            for (int q = 0; q < 32 * NC; q += 16) {
+                uint32_t r[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) r[t] = rne_f32((int)v[q + t], k);
+                const uint4 w = make_uint4(pack4b(r[0], r[1], r[2], r[3]), pack4b(r[4], r[5], r[6], r[7]),
+                                           pack4b(r[8], r[9], r[10], r[11]), pack4b(r[12], r[13], r[14], r[15]));
+                if (TS) stage16(srow, et, scol + q, w);
+                else if (ncol + q < p.N) *reinterpret_cast<uint4 *>(dst + q) = w;
+            }
+        }
+        return;
+    }
     if (__any_sync(0xffffffffu, valid && S < 0)) {
         const int lm = S < 0 ? (1 << min(-S, 30)) : 1;
 #pragma unroll
@@ -190,7 +229,6 @@ __device__ __forceinline__ void epi_fast(const GemmParams &p, uint32_t taddr, co
             v[q] = (uint32_t)((y + ((y >> 1) & 1)) >> 1);
         }
     }
-    if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
     if (TS || valid) {
         int8_t *dst = p.out + grow * p.out_ld + ncol;
 #pragma unroll
@@ -233,14 +271,40 @@ __device__ __forceinline__ void epi_two_pass(const GemmParams &p, uint32_t taddr
     }
     const int h = max(max(hi[0], hi[1]), max(hi[2], hi[3])), l = min(min(lo[0], lo[1]), min(lo[2], lo[3]));
     const int amax = valid ? max(h, -l) : 0;
-    const int e = finalize_exp(amax ? ea + gm + need_off32q((uint32_t)amax, p.qb) : kNoExp);
+    const int need = amax ? ea + gm + need_off32q((uint32_t)amax, p.qb) : kNoExp;
+    const int e = finalize_exp(need);
     const int S = (e == kEZero) ? 0 : e - ea - gm;
+    if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
+    int8_t *dst = p.out + grow * p.out_ld + ncol;
+    if (__all_sync(0xffffffffu, rne_f32_ok(valid, amax, S, need))) {
+        const RneF32 k = rne_f32_consts(S);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            tmem_ld32(taddr + 32 * c, v);
+            tmem_ld_wait();
+            if (TS || valid) {
+#pragma unroll
+                for (int q = 0; q < 32; q += 16) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int t = 0; t < 16; t += 4) {
+                        int4 m4 = make_int4(1, 1, 1, 1);
+                        if (MUL) m4 = *reinterpret_cast<const int4 *>(colM + 32 * c + q + t);
+                        w4[t >> 2] = pack4b(rne_f32((int)v[q + t] * m4.x, k), rne_f32((int)v[q + t + 1] * m4.y, k),
+                                            rne_f32((int)v[q + t + 2] * m4.z, k), rne_f32((int)v[q + t + 3] * m4.w, k));
+                    }
+                    const uint4 w = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    if (TS) stage16(srow, et, scol + 32 * c + q, w);
+                    else if (ncol + 32 * c + q < p.N) *reinterpret_cast<uint4 *>(dst + 32 * c + q) = w;
+                }
+            }
+        }
+        return;
+    }
     const bool any_ls = __any_sync(0xffffffffu, valid && S < 0);
     const int lm = S < 0 ? (1 << min(-S, 30)) : 1;
     const int rs = S > 0 ? min(S, 31) : 0;
     const int m = rs >= 2 ? 1 << (32 - rs) : 0, bias = rs ? (1 << (rs - 1)) - 1 : 0;
-    if (ncol < p.N && valid) p.out_exp[grow * p.out_exp_ld + gcol] = (int8_t)e;
-    int8_t *dst = p.out + grow * p.out_ld + ncol;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
         tmem_ld32(taddr + 32 * c, v);
