@@ -2042,8 +2042,6 @@ int32_t ict_sgd_momentum_step_multi(int32_t n_tensors, ict_tensor *const *W, ict
     a.lr_shift = p->lr_shift;
     a.cap_mom = 29 - bitlen_u64(127ull * (uint64_t)std::abs(p->mom_mul));
     a.cap_lr = 29 - bitlen_u64(127ull * (uint64_t)std::abs(p->lr_mul));
-    a.capf_mom = 23 - bitlen_u64(127ull * (uint64_t)std::abs(p->mom_mul));
-    a.capf_lr = 23 - bitlen_u64(127ull * (uint64_t)std::abs(p->lr_mul));
     int64_t total = 0;
     for (int i = 0; i < n_tensors; ++i) {
         if ((st = fill_sgd_tensor(W[i], V[i], G[i], &a.t[i]))) return st;

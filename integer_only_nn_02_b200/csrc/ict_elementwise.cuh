@@ -1444,9 +1444,6 @@ struct SgdArgs {
     // largest shift of each term at which |term| stays below 2^29 (so every two-term sum
     // is below 2^30): 29 - bitlen(127 |multiplier|)
     int cap_mom, cap_lr;
-    // the same for the fp32 fast path, whose integers must stay below 2^24:
-    // 24 - bitlen(127 |multiplier|)
-    int capf_mom, capf_lr;
     int qb;  // mantissa bits B of both FITs (|C| <= 2^(B-1) - 1)
     SgdTensor t[kSgdMaxTensors];
 };
@@ -1737,44 +1734,20 @@ __global__ void __launch_bounds__(256) sgd_vec_kernel(const __grid_constant__ Sg
 // parameter arena padded to its group width).  Each lane holds 16 CPL elements of W, V
 // and G; the next group's chunks are loaded before the current group is computed.
 //
-// The two-term sums and their rounding run as exact integer arithmetic on the fp32 pipe
-// (twice the integer pipes' issue rate).  Per group the terms a * 2^pa and b * 2^pb sit
-// at the common exponent r0 = min(pa, pb); while |a| 2^(pa - r0) and |b| 2^(pb - r0) stay
-// below 2^23 each (shift caps from the multipliers' magnitudes), every sum is an integer
-// below 2^24, so the byte-built operands, the scalings by powers of two and the FMA that
-// adds the terms are all exact.  The group exponent then follows from the largest
-// magnitude (converted to int exactly), and RNE(x / 2^S) is one FMA onto 1.5 * 2^23: its
-// result lies in [2^23, 2^24), where fp32 rounds to the nearest integer with ties to
-// even, so the low byte of its bits is the int8 mantissa.  Groups beyond the caps take
-// the int64 path (sgd_group_exact).
+// The two-term sums and their rounding run on the fp32 pipe, one code path for every
+// group (so that the groups of a warp never split it).  Per group the sum is taken at the
+// unit of one term (its mantissas are exact floats built from the bytes) with the other
+// term's multiplier a float power-of-two multiple of mom or lr; one pair of directed FMAs
+// gives each sum rounded to odd at 24 bits (ro_fma).  The group exponent follows from the
+// largest magnitude's bit pattern (need_rel_f32), and RNE(x / 2^S) is one FMA onto
+// 1.5 * 2^23: its result lies in [2^23, 2^24), where fp32 rounds to the nearest integer
+// with ties to even, so the low byte of its bits is the int8 mantissa; since that
+// rounding sits at least 16 bits above the sums' last places it equals rounding the exact
+// sums.  Groups whose exponents lie more than kSgdGap apart, or whose exponent leaves the
+// range, take the int64 path (sgd_group_exact).
 __device__ __forceinline__ float sx8f(uint32_t w_biased, int b) {
     // byte b of w (stored with 0x80 added to every byte) as the float C: 2^23 + (C + 128) - (2^23 + 128)
     return __uint_as_float(__byte_perm(w_biased, 0x4B000000u, 0x7650 | b)) - 8388736.0f;
-}
-// Plan of an exact fp32 two-term sum a * 2^pa + b * 2^pb (|a| < 2^(23 - cap_a),
-// |b| < 2^(23 - cap_b)): both terms at r0 = min(pa, pb), shifted by sa and sb (one of them
-// 0).  When the shifted term would exceed its cap, it is shifted by the cap only and the
-// other term is rounded to odd at 2^k first (k > 0, r0 raised by k): the sum then stays
-// below 2^24, and rounding that sum to nearest at an exponent at least 2 above r0 equals
-// rounding the exact sum (Boldo and Melquiond, IEEE Trans. Computers 57(4), 2008).  An
-// absent term (E_ZERO: all mantissas zero) takes the other's exponent.
-__device__ __forceinline__ void two_term_plan(int pa, bool za, int pb, bool zb, int cap_a, int cap_b, int &r0,
-                                              int &sa, int &sb, int &k) {
-    if (za) pa = pb;
-    if (zb) pb = pa;
-    r0 = min(pa, pb);
-    sa = pa - r0;
-    sb = pb - r0;
-    k = 0;
-    if (sa > cap_a) k = sa - cap_a, sa = cap_a;
-    if (sb > cap_b) k = sb - cap_b, sb = cap_b;
-    r0 += k;
-}
-// v / 2^k rounded to odd (floor, then the sticky bit ORed in), as a float; |v| < 2^22
-__device__ __forceinline__ float ro_float(int v, int k) {
-    k = min(k, 31);
-    const int q = (v >> k) | (int)((v & (int)((1u << k) - 1u)) != 0);
-    return __int_as_float(q + 0x4B400000) - 12582912.0f;
 }
 __device__ __forceinline__ float pow2f(int k) {  // 2^k for -126 <= k <= 127; 0 below
     return k < -126 ? 0.0f : __int_as_float((k + 127) << 23);
@@ -1783,6 +1756,26 @@ __device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float 
     return __byte_perm(__byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040),
                        __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040), 0x5410);
 }
+// a * b + c rounded to odd at fp32's 24 bits: rounded down and rounded up, the two
+// results are equal when the sum is exact and are neighbours otherwise, and the one whose
+// last significand bit is set is the round-to-odd result (for either sign).  Rounding
+// that to nearest even at a position at least two bits above its last place equals
+// rounding the exact sum (Boldo and Melquiond, IEEE Trans. Computers 57(4), 2008).
+__device__ __forceinline__ float ro_fma(float a, float b, float c) {
+    const float lo = __fmaf_rd(a, b, c), hi = __fmaf_ru(a, b, c);
+    return (__float_as_uint(lo) & 1u) ? lo : hi;
+}
+// need() of a positive normal float x (its bit pattern): the least S with
+// RNE(x 2^-S) <= 2^(B-1) - 1, i.e. x < (2^(B-1) - 1/2) 2^S: S = E - (B - 2) for
+// x = 1.f 2^E, plus one when 1.f >= 2 - 2^(1-B) (the significand field at or above
+// 2^23 - 2^(24-B)).  A value rounded to odd at 24 bits gives the same S as the exact one,
+// since the bound has at most B significant bits.
+__device__ __forceinline__ int need_rel_f32(uint32_t xb, int qb) {
+    return (int)(xb >> 23) - 127 - (qb - 2) + ((xb & 0x7FFFFFu) >= 0x800000u - (1u << (24 - qb)) ? 1 : 0);
+}
+// largest exponent gap between the two terms that the fp32 path takes: their multipliers
+// stay normal floats and far from overflow
+constexpr int kSgdGap = 100;
 
 // L lanes per group, CPL 16-byte chunks per lane (a group is 16 L CPL elements; chunk k
 // of lane li sits at element (k L + li) 16 of the group, so that each chunk index is a
@@ -1826,14 +1819,16 @@ __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ S
             }
             nev = tve[rn], neg = tge[rn], new_ = twe[rn];
         }
-        // velocity: v = mom * V 2^(ev - mom_shift) + G 2^eg
-        int r1, sa1, sb1, k1;
-        bool fit1;
-        two_term_plan(ev - p.mom_shift, ev == kEZero, eg, eg == kEZero, p.capf_mom, 16, r1, sa1, sb1, k1);
-        int r2 = 0, sa2 = 0, sb2 = 0, k2 = 0, ev2 = kEZero;
-        bool fit2 = false;
+        // velocity: v = mom * V 2^(ev - mom_shift) + G 2^eg, at the unit 2^pb (the G term
+        // unscaled, the other term's multiplier mom 2^(pa - pb) a float)
+        int pa = ev - p.mom_shift, pb = eg;
+        if (ev == kEZero) pa = pb;  // an absent term takes the other's exponent
+        if (eg == kEZero) pb = pa;
+        const int d1 = pa - pb;
+        bool fast = d1 >= -kSgdGap && d1 <= kSgdGap;
+        int ev2 = kEZero, ew2 = kEZero;
         float vq[E];  // 1.5 * 2^23 + the new velocity mantissas
-        float y[E];   // the velocity sums, then the weight sums
+        float y[E];   // the velocity sums, then the weight sums (rounded to odd at 24 bits)
         {
             uint32_t vb[4 * CPL], gb[4 * CPL];
 #pragma unroll
@@ -1843,65 +1838,52 @@ __global__ void __launch_bounds__(256) sgd_rows_kernel(const __grid_constant__ S
                 gb[4 * k] = cg[k].x ^ 0x80808080u, gb[4 * k + 1] = cg[k].y ^ 0x80808080u;
                 gb[4 * k + 2] = cg[k].z ^ 0x80808080u, gb[4 * k + 3] = cg[k].w ^ 0x80808080u;
             }
-            const float ma = (float)(p.mom_mul << sa1), mb = (float)(1 << sb1);
+            const float ma = (float)p.mom_mul * pow2f(fast ? d1 : 0);
             float amax = 0.0f;
-            if (k1 == 0) {
 #pragma unroll
-                for (int e = 0; e < E; ++e) y[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, sx8f(gb[e >> 2], e & 3) * mb);
-            } else if (sa1 == 0) {  // G 2^16 dominates: mom * V rounded to odd at 2^k1
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    y[e] = __fmaf_rn(sx8f(gb[e >> 2], e & 3), mb, ro_float(sx8(vb[e >> 2] ^ 0x80808080u, e & 3) * p.mom_mul, k1));
-            } else {  // mom * V 2^cap dominates: G rounded to odd at 2^k1
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    y[e] = __fmaf_rn(sx8f(vb[e >> 2], e & 3), ma, ro_float(sx8(gb[e >> 2] ^ 0x80808080u, e & 3), k1));
+            for (int e = 0; e < E; ++e) {
+                y[e] = ro_fma(sx8f(vb[e >> 2], e & 3), ma, sx8f(gb[e >> 2], e & 3));
+                amax = fmaxf(amax, fabsf(y[e]));
             }
-#pragma unroll
-            for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
-            const int ia = group_max<L>((int)amax, gmask);
-            ev2 = finalize_exp(ia ? r1 + need_off32q((uint32_t)ia, p.qb) : kNoExp);
-            // with a rounded-to-odd term the final shift must be at least 2 bits (it is unless
-            // the dominant term's mantissas are all zero; then the exact path takes the group)
-            fit1 = k1 == 0 || ev2 == kEZero || ev2 - r1 >= 2;
-            const float sc = pow2f(ev2 == kEZero ? 0 : r1 - ev2);
+            const uint32_t ia = (uint32_t)group_max<L>((int)__float_as_uint(amax), gmask);
+            const int need = pb + need_rel_f32(ia, p.qb);
+            ev2 = ia ? finalize_exp(need) : kEZero;
+            const int sh = ia ? ev2 - pb : 0;
+            fast = fast && (ia == 0u || (ia >= 0x00800000u && need <= 127 && sh >= -126 && sh <= 126));
+            const float sc = pow2f(fast ? -sh : 0);
 #pragma unroll
             for (int e = 0; e < E; ++e) vq[e] = __fmaf_rn(y[e], sc, kMagic);
-            two_term_plan(ew, ew == kEZero, ev2 - p.lr_shift, ev2 == kEZero, 16, p.capf_lr, r2, sa2, sb2, k2);
         }
-        int ew2 = kEZero;
-        if (fit1) {
-            // weight: w = W 2^ew - lr * V' 2^(ev2 - lr_shift)
+        if (fast) {
+            // weight: w = W 2^ew - lr * V' 2^(ev2 - lr_shift), at the unit 2^ew
+            int pw = ew, pv = ev2 - p.lr_shift;
+            if (ew == kEZero) pw = pv;
+            if (ev2 == kEZero) pv = pw;
+            const int d2 = pv - pw;
+            fast = d2 >= -kSgdGap && d2 <= kSgdGap;
             uint32_t wb[4 * CPL];
 #pragma unroll
             for (int k = 0; k < CPL; ++k) {
                 wb[4 * k] = cw[k].x ^ 0x80808080u, wb[4 * k + 1] = cw[k].y ^ 0x80808080u;
                 wb[4 * k + 2] = cw[k].z ^ 0x80808080u, wb[4 * k + 3] = cw[k].w ^ 0x80808080u;
             }
-            const float ma = (float)(1 << sa2), mb = (float)(-(p.lr_mul << sb2));
+            const float mb = -(float)p.lr_mul * pow2f(fast ? d2 : 0);
             float amax = 0.0f;
-            if (k2 == 0) {
 #pragma unroll
-                for (int e = 0; e < E; ++e) y[e] = __fmaf_rn(vq[e] - kMagic, mb, sx8f(wb[e >> 2], e & 3) * ma);
-            } else if (sa2 == 0) {  // lr * V' dominates: W rounded to odd at 2^k2
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    y[e] = __fmaf_rn(vq[e] - kMagic, mb, ro_float(sx8(wb[e >> 2] ^ 0x80808080u, e & 3), k2));
-            } else {  // W 2^16 dominates: -lr * V' rounded to odd at 2^k2
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    y[e] = __fmaf_rn(sx8f(wb[e >> 2], e & 3), ma,
-                                     ro_float(-p.lr_mul * (__float_as_int(vq[e]) - 0x4B400000), k2));
+            for (int e = 0; e < E; ++e) {
+                y[e] = ro_fma(vq[e] - kMagic, mb, sx8f(wb[e >> 2], e & 3));
+                amax = fmaxf(amax, fabsf(y[e]));
             }
-#pragma unroll
-            for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
-            const int ia = group_max<L>((int)amax, gmask);
-            ew2 = finalize_exp(ia ? r2 + need_off32q((uint32_t)ia, p.qb) : kNoExp);
-            fit2 = k2 == 0 || ew2 == kEZero || ew2 - r2 >= 2;
-            const float sc = pow2f(ew2 == kEZero ? 0 : r2 - ew2);
+            const uint32_t ia = (uint32_t)group_max<L>((int)__float_as_uint(amax), gmask);
+            const int need = pw + need_rel_f32(ia, p.qb);
+            ew2 = ia ? finalize_exp(need) : kEZero;
+            const int sh = ia ? ew2 - pw : 0;
+            fast = fast && (ia == 0u || (ia >= 0x00800000u && need <= 127 && sh >= -126 && sh <= 126));
+            const float sc = pow2f(fast ? -sh : 0);
 #pragma unroll
             for (int e = 0; e < E; ++e) y[e] = __fmaf_rn(y[e], sc, kMagic);
         }
+        const bool fit1 = fast, fit2 = fast;
         if (!(fit1 && fit2)) {
             sgd_group_exact<L>(p, t0, r * G, r, G, li, gmask);
         } else {
