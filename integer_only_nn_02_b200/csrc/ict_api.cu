@@ -2079,7 +2079,17 @@ int32_t ict_gelu_fwd(const ict_tensor *H, ict_tensor *out, void *stream) {
         return ICT_ERR_CUDA;
     const int64_t vecs = H->rows * (H->cols / 16);
     KTimer kt(s, KC_GELU, 2.0 * (double)H->rows * (double)H->cols + 2.0 * (double)ne);
-    gelu_fwd_kernel<<<(unsigned)cdiv64(vecs, 256), 256, 0, s>>>(a);
+    const int G = (int)a.g_cols;
+    if (a.g_rows == 1 && (G == 16 || G == 32 || G == 64)) {  // one thread per group
+        int sms = 148;
+        device_info(&sms);
+        const unsigned blocks = (unsigned)std::min<int64_t>(cdiv64(H->rows * a.ngc, 256), (int64_t)sms * 4);
+        if (G == 16) gelu_fwd_thread_kernel<1><<<blocks, 256, 0, s>>>(a);
+        else if (G == 32) gelu_fwd_thread_kernel<2><<<blocks, 256, 0, s>>>(a);
+        else gelu_fwd_thread_kernel<4><<<blocks, 256, 0, s>>>(a);
+    } else {
+        gelu_fwd_kernel<<<(unsigned)cdiv64(vecs, 256), 256, 0, s>>>(a);
+    }
     counted(1);
     return launch_status();
 }
@@ -2116,7 +2126,14 @@ int32_t ict_gelu_bwd(const ict_tensor *H, const ict_tensor *dG, ict_tensor *dH, 
     KTimer kt(s, KC_GELU, 3.0 * (double)H->rows * (double)H->cols + 3.0 * (double)groups);
     const bool vec = check_vec(H) == ICT_OK && check_vec(dG) == ICT_OK && check_vec(dH) == ICT_OK &&
                      G % 16 == 0 && G <= 512 && ((G / 16) & (G / 16 - 1)) == 0;
-    if (vec) {
+    if (vec && (G == 16 || G == 32 || G == 64)) {  // one thread per group
+        int sms = 148;
+        device_info(&sms);
+        const unsigned blocks = (unsigned)std::min<int64_t>(cdiv64(groups, 256), (int64_t)sms * 4);
+        if (G == 16) gelu_bwd_thread_kernel<1><<<blocks, 256, 0, s>>>(a);
+        else if (G == 32) gelu_bwd_thread_kernel<2><<<blocks, 256, 0, s>>>(a);
+        else gelu_bwd_thread_kernel<4><<<blocks, 256, 0, s>>>(a);
+    } else if (vec) {
         int sms = 148;
         device_info(&sms);
         const int L = G / 16, gpb = 8 * (32 / L);

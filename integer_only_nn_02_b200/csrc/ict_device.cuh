@@ -129,6 +129,32 @@ __device__ __forceinline__ int sx8(uint32_t w, int byte) {
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));
     return (int)r;
 }
+// The low bytes of four words packed into one (three byte permutes).
+__device__ __forceinline__ uint32_t pack4b(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// RNE(y * 2^-S) on the fp32 pipe, for |y| < 2^22 and 0 <= S <= 22.  The bit pattern
+// 0x4B400000 + y is the float 1.5 * 2^23 + y exactly (the sum stays in the binade of unit
+// spacing); one FMA by 2^-S with the addend 1.5 * 2^23 * (1 - 2^-S) (exact for S <= 22)
+// gives 1.5 * 2^23 + y * 2^-S rounded once, to nearest even, at the unit.  The low byte of
+// the result's bit pattern is then the rounded value in two's complement (|value| <= 128).
+struct RneF32 {
+    float sc, add;
+};
+__device__ __forceinline__ RneF32 rne_f32_consts(int S) {
+    const float sc = __int_as_float((127 - S) << 23);
+    return {sc, __fmaf_rn(-12582912.f, sc, 12582912.f)};
+}
+__device__ __forceinline__ uint32_t rne_f32(int y, RneF32 k) {
+    return __float_as_uint(__fmaf_rn(__int_as_float(0x4B400000 + y), k.sc, k.add));
+}
+// the group may take the fp32 rounding: every magnitude below 2^22, a right shift of at
+// most 22 bits, and an exponent that was not capped (a capped one saturates instead)
+__device__ __forceinline__ bool rne_f32_ok(bool valid, int amax, int S, int need) {
+    return !valid || (amax < (1 << 22) && S >= 0 && S <= 22 && need <= 127);
+}
+
 // Four values already within [-127, 127] packed into bytes in two conversion
 // instructions (each packs two values; the second merges the first's word).
 __device__ __forceinline__ uint32_t pack4s(int a, int b, int c, int d) {

@@ -824,6 +824,173 @@ __global__ void __launch_bounds__(256) gelu_bwd_vec_kernel(const __grid_constant
     }
 }
 
+// The same with one thread per group of V 16-byte vectors (G = 16 V columns, rows of
+// whole vectors): the thread owns the group's H and dG mantissas, so the group's largest
+// magnitude is a register reduction with no shuffles; groups run in row-major order over
+// the grid's threads (consecutive threads, consecutive groups of a row), the next
+// group's vectors and exponents are loaded before the current group is computed, and the
+// row / group cursor advances without a division.  Rounding: on the fp32 pipe when the
+// group's magnitudes are below 2^22 (rne_f32), else by the integer shift.
+template <int V>
+__global__ void __launch_bounds__(256) gelu_bwd_thread_kernel(const __grid_constant__ GeluArgs a) {
+    constexpr int E = 16 * V;
+    const int64_t total = a.rows * a.ngc;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    int64_t gw = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gw >= total) return;
+    int64_t i = gw / a.ngc, g = gw - i * a.ngc;
+    const int64_t di = step / a.ngc, dg = step - di * a.ngc;
+    uint4 h[V], d[V];
+    int eh = 0, ed = 0, nv = 0;
+    auto load = [&](int64_t ii, int64_t gg, uint4(&hh)[V], uint4(&dd)[V], int &e_h, int &e_d, int &n) {
+        const int64_t j0 = gg * E;
+        n = (int)min((int64_t)V, (a.cols - j0) >> 4);
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            hh[v] = v < n ? *reinterpret_cast<const uint4 *>(a.h + ii * a.ld_h + j0 + 16 * v) : make_uint4(0, 0, 0, 0);
+            dd[v] = v < n ? *reinterpret_cast<const uint4 *>(a.dg + ii * a.ld_dg + j0 + 16 * v) : make_uint4(0, 0, 0, 0);
+        }
+        e_h = a.h_exp[ii * a.ngc + gg];
+        e_d = a.dg_exp[ii * a.ngc + gg];
+    };
+    load(i, g, h, d, eh, ed, nv);
+    while (true) {
+        // the next group's cursor and loads first
+        int64_t ni = i + di, ng = g + dg;
+        if (ng >= a.ngc) ng -= a.ngc, ++ni;
+        const bool more = ni < a.rows;
+        uint4 h2[V], d2[V];
+        int eh2 = 0, ed2 = 0, nv2 = 0;
+        if (more) load(ni, ng, h2, d2, eh2, ed2, nv2);
+        const int64_t j0 = g * E;
+        const int sh = (eh < 0 && eh != kEZero) ? -eh : 0;
+        if (sh > 21) {
+            gelu_bwd_group_exact<1>(a, i, g, 16 * nv, 0, 0u);
+        } else {
+            // |C_h| < T is the interior; e_h >= 1 (or E_ZERO) leaves only C_h = 0 inside
+            const int T = (eh >= 1 || eh == kEZero) ? 1 : (1 - eh >= 8 ? 256 : (1 << (1 - eh)));
+            int xv[E];
+            int amax = 0;
+#pragma unroll
+            for (int b = 0; b < E; ++b) {
+                const uint4 &hv = h[b >> 4], &dv = d[b >> 4];
+                const uint32_t hw = (b & 15) < 4 ? hv.x : (b & 15) < 8 ? hv.y : (b & 15) < 12 ? hv.z : hv.w;
+                const uint32_t dw = (b & 15) < 4 ? dv.x : (b & 15) < 8 ? dv.y : (b & 15) < 12 ? dv.z : dv.w;
+                const int ch = sx8(hw, b & 3), cd = sx8(dw, b & 3);
+                const bool inside = ch > -T && ch < T;
+                const int hi = ch <= -T ? 0 : (inside ? cd : 2 * cd);
+                const int x = (hi << sh) + (inside ? cd * ch : 0);
+                xv[b] = x;
+                amax = max(amax, abs(x));
+            }
+            const int r0 = ed - 1 - sh;
+            const int need = amax ? r0 + need_off32((uint32_t)amax) : kNoExp;
+            const int e = finalize_exp(need);
+            const int S = e == kEZero ? 0 : e - r0;
+            uint32_t o[4 * V];
+            if (rne_f32_ok(true, amax, S, need)) {
+                const RneF32 k = rne_f32_consts(S);
+#pragma unroll
+                for (int q = 0; q < 4 * V; ++q)
+                    o[q] = pack4b(rne_f32(xv[4 * q], k), rne_f32(xv[4 * q + 1], k), rne_f32(xv[4 * q + 2], k),
+                                  rne_f32(xv[4 * q + 3], k));
+            } else {
+                const Shift hs = make_shift(S);
+#pragma unroll
+                for (int q = 0; q < 4 * V; ++q)
+                    o[q] = pack4(apply_shift(xv[4 * q], hs), apply_shift(xv[4 * q + 1], hs),
+                                 apply_shift(xv[4 * q + 2], hs), apply_shift(xv[4 * q + 3], hs));
+            }
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+                if (v < nv)
+                    *reinterpret_cast<uint4 *>(a.out + i * a.ld_out + j0 + 16 * v) =
+                        make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            a.out_exp[i * a.ngc + g] = (int8_t)e;
+        }
+        if (!more) break;
+        i = ni, g = ng, eh = eh2, ed = ed2, nv = nv2;
+#pragma unroll
+        for (int v = 0; v < V; ++v) h[v] = h2[v], d[v] = d2[v];
+    }
+}
+
+// GELU forward with one thread per group of V 16-byte vectors, the same traversal: the
+// group exponent fixes the curve's thresholds and the interior rounding shift for all 16 V
+// mantissas (the exponent is carried unchanged).
+template <int V>
+__global__ void __launch_bounds__(256) gelu_fwd_thread_kernel(const __grid_constant__ GeluArgs a) {
+    constexpr int E = 16 * V;
+    const int64_t total = a.rows * a.ngc;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    int64_t gw = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gw >= total) return;
+    int64_t i = gw / a.ngc, g = gw - i * a.ngc;
+    const int64_t di = step / a.ngc, dg = step - di * a.ngc;
+    uint4 h[V];
+    int eh = 0, nv = 0;
+    auto load = [&](int64_t ii, int64_t gg, uint4(&hh)[V], int &e_h, int &n) {
+        const int64_t j0 = gg * E;
+        n = (int)min((int64_t)V, (a.cols - j0) >> 4);
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+            hh[v] = v < n ? *reinterpret_cast<const uint4 *>(a.h + ii * a.ld_h + j0 + 16 * v) : make_uint4(0, 0, 0, 0);
+        e_h = a.h_exp[ii * a.ngc + gg];
+    };
+    load(i, g, h, eh, nv);
+    while (true) {
+        int64_t ni = i + di, ng = g + dg;
+        if (ng >= a.ngc) ng -= a.ngc, ++ni;
+        const bool more = ni < a.rows;
+        uint4 h2[V];
+        int eh2 = 0, nv2 = 0;
+        if (more) load(ni, ng, h2, eh2, nv2);
+        uint32_t o[4 * V];
+        if (eh == kEZero) {
+#pragma unroll
+            for (int q = 0; q < 4 * V; ++q) o[q] = 0u;
+        } else if (eh >= 2) {  // |x| >= 4 for every nonzero C: h(x) = max(x, 0)
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const uint32_t src[4] = {h[v].x, h[v].y, h[v].z, h[v].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) o[4 * v + q] = __vmaxs4(src[q], 0u);
+            }
+        } else {
+            const int s = 2 - eh;                              // interior: RNE(C (C + T) / 2^s)
+            const int t = s - 1 >= 8 ? 256 : (1 << (s - 1));  // T = 2^(1-e); |C| < 256
+            const int T = s <= 24 ? 1 << (s - 1) : 0;
+            const Shift hs = make_shift(s);
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const uint32_t src[4] = {h[v].x, h[v].y, h[v].z, h[v].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    int r[4];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const int c = sx8(src[q], b);
+                        // C^2 / 2^s < 1/2 beyond s = 24: RNE(C / 2 + a positive tiny term) = floor((C + 1) / 2)
+                        const int in = s <= 24 ? apply_shift(c * (c + T), hs) : (c + 1) >> 1;
+                        r[b] = c <= -t ? 0 : (c >= t ? c : in);
+                    }
+                    o[4 * v + q] = pack4(r[0], r[1], r[2], r[3]);
+                }
+            }
+        }
+        const int64_t j0 = g * E;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+            if (v < nv)
+                *reinterpret_cast<uint4 *>(a.out + i * a.ld_out + j0 + 16 * v) =
+                    make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        if (!more) break;
+        i = ni, g = ng, eh = eh2, nv = nv2;
+#pragma unroll
+        for (int v = 0; v < V; ++v) h[v] = h2[v];
+    }
+}
+
 // ------------------------------------------------------------------ requant, wide groups
 
 // FIT of row-local groups wider than a warp can hold: one block of T threads per group,
