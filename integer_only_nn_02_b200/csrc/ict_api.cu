@@ -539,6 +539,12 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
         return ICT_ERR_LAYOUT;  // backward-weight writes int32 only
     } else {
         if constexpr (LOAD == LOAD_CONV) {
+            if constexpr (BN <= 128) {
+                // four epilogue warpgroups on alternate tiles (four accumulators): the
+                // per-tile rounding to odd is latency-bound, more warps hide it
+                constexpr int kB4 = GemmSmem<BN, BK, ST, 4>::kBytes;
+                if (p.epi == EPI_RO16 && p.nwg == 4) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_RO16, 0, 4>, 4, kB4);
+            }
             if (p.epi == EPI_RO16) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_RO16>, 2, kB2);
         }
         if constexpr (LOAD == LOAD_2D) {
@@ -613,7 +619,8 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     // group straddles the halves
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
-    if (p.nwg != 4 || p.epi != EPI_FIT_ROW || pair) p.nwg = 2;
+    const bool nwg4_ok = p.epi == EPI_FIT_ROW || (p.epi == EPI_RO16 && load == LOAD_CONV);
+    if (p.nwg != 4 || !nwg4_ok || pair) p.nwg = 2;
     p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || p.epi == EPI_RO16R || (gt < bn && (bn / 2) % gt == 0));
     if (pair) {
         if (load != LOAD_2D || bk != 128 || (grid & 1)) return ICT_ERR_LAYOUT;
@@ -1259,6 +1266,7 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         counted(1);
     }
     p.epi = EPI_RO16;
+    p.nwg = cp.bn <= 128 ? 4 : 2;
     p.ws16 = cp.ws16;
     p.ws16_ld = cp.ws16_ld;
     p.tile_need = cp.tile_need;
