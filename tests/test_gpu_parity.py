@@ -140,11 +140,14 @@ def test_linear_bwd_weight(ict, case, per_row):
     (896, 256, 528, 16, (-10, -4)),     # 16-column X groups: column exponents differ within a tile
     (500, 320, 640, 16, (-40, -4)),     # column exponents far apart: the exact per-element path
     (64, 144, 1024, 64, (-10, -4)),     # a 144-row dW with every row spanning 8 tiles
+    (256, 4096, 768, 64, (-10, -4)),    # 192 tiles, more than the SMs: the int16 form and its row pass
+    (300, 3312, 768, 16, (-40, -4)),    # the same with a ragged last tile and the per-element path
 ])
 def test_linear_bwd_weight_row_groups_across_tiles(ict, M, N, K, xg, xspan):
     """dW = dY^T X with one output group per row spanning several tiles and no split K:
     the Product's int16 round-to-odd output with a need per (row, tile half), then the
-    streaming pass that rounds each row to its group exponent, against the oracle."""
+    streaming pass that rounds each row to its group exponent, against the oracle (one
+    tile per SM, and more tiles than SMs)."""
     rng = np.random.default_rng(M + N + K + xg)
     X = rand_ce(rng, M, K, 1, xg, elo=xspan[0], ehi=xspan[1], zero_groups=0.05)
     dY = with_groups(clipped_laplace(rng, (M, N)), 1, 32, lambda g: rng.integers(-16, -10, size=g))
