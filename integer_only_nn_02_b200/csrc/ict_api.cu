@@ -524,12 +524,12 @@ constexpr int stages_for(int bn, int bk) {
 
 template <int BN, int BK, int LOAD>
 int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid,
-                  cudaStream_t s) {
+                  cudaStream_t s, const CUtensorMap *ty = nullptr) {
     constexpr int ST = stages_for(BN, BK);
     auto run = [&](auto k, int nwg, int smem_bytes) {
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
             return (int)ICT_ERR_CUDA;
-        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, tb, p);  // no staged output: tmY unused
+        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, ty ? *ty : tb, p);  // tmY: staged output only
         counted(1);
         return launch_status();
     };
@@ -555,6 +555,14 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
         if constexpr (LOAD == LOAD_2D && BN <= 128) {
             if (p.nwg == 4) {  // four epilogue warpgroups, four accumulators
                 constexpr int kB4 = GemmSmem<BN, BK, ST, 4>::kBytes;
+                if constexpr (BN == 128) {
+                    // 32-column groups with the output staged per warpgroup (128 x 128) and
+                    // written by TMA stores: four stages leave room for the staging rows
+                    constexpr int ST4 = 4;
+                    constexpr int kB4s = GemmSmem<BN, BK, ST4, 4, false, 4, 128 * 128>::kBytes;
+                    if (gt == 32 && ty)
+                        return run(gemm_ce_kernel<BN, BK, ST4, LOAD, EPI_FIT_ROW, 1, 4, false, false, true>, 4, kB4s);
+                }
                 if (gt == 32) return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 1, 4>, 4, kB4);
                 return run(gemm_ce_kernel<BN, BK, ST, LOAD, EPI_FIT_ROW, 0, 4>, 4, kB4);
             }
@@ -631,7 +639,7 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     }
 #define ICT_GEMM_CASE(BN_, BK_, LOAD_)          \
     if (bn == BN_ && bk == BK_ && load == LOAD_) \
-        return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s);
+        return launch_gemm_t<BN_, BK_, LOAD_>(ta, tb, p, grid, s, ty);
     ICT_GEMM_CASE(64, 128, LOAD_2D)
     ICT_GEMM_CASE(128, 128, LOAD_2D)
     ICT_GEMM_CASE(192, 128, LOAD_2D)
@@ -803,9 +811,11 @@ int run_product(const Operand &A, const Operand &B, const ict_tensor *out, const
     if ((st = tmap_2d(&ta, A.mant, K, M, A.ld, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))) return st;
     if ((st = tmap_2d(&tb, B.mant, K, N, B.ld, 128, pl.pair ? pl.bn / 2 : pl.bn, CU_TENSOR_MAP_SWIZZLE_128B)))
         return st;
-    // pairs with a fused FIT: the output as 64 x 128 boxes (64-byte swizzle) for staged stores
+    // pairs with a fused FIT, and single CTAs with four epilogue warpgroups on 128-wide tiles
+    // of 32-column groups: the output as 64 x 128 boxes (64-byte swizzle) for staged stores
     CUtensorMap ty;
-    const bool staged = pl.pair && pl.fused;
+    const bool staged = pl.fused && (pl.pair || (pl.nwg == 4 && pl.bn == 128 && out->g_cols == 32 &&
+                                                 N % 128 == 0 && aligned16(out->mant) && out->ld % 16 == 0));
     if (staged && (st = tmap_2d(&ty, out->mant, N, M, out->ld, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))) return st;
     GemmParams p;
     memset(&p, 0, sizeof(p));

@@ -468,7 +468,18 @@ __global__ void __launch_bounds__(256) align_transpose_kernel(const __grid_const
         __syncthreads();
         const int64_t ngr = idiv(a.rows + a.g_rows - 1, a.g_rows);
         const int k = threadIdx.x % ng, per = 256 / ng;
-        if (threadIdx.x < per * ng) {
+        if (a.ngc == 1 && (reinterpret_cast<uintptr_t>(a.in_exp) & 3) == 0) {
+            // one group column (one exponent per row group, consecutive bytes): four
+            // exponents per load and every load issued before the first maximum
+            const uint32_t *e4 = reinterpret_cast<const uint32_t *>(a.in_exp);
+            const int64_t nw = ngr >> 2;
+            uint32_t m4 = 0x80808080u;  // E_ZERO (-128) in every byte: the smallest
+#pragma unroll 4
+            for (int64_t w = threadIdx.x; w < nw; w += 256) m4 = __vmaxs4(m4, e4[w]);
+            int m = max(max(sx8(m4, 0), sx8(m4, 1)), max(sx8(m4, 2), sx8(m4, 3)));
+            for (int64_t r = 4 * nw + threadIdx.x; r < ngr; r += 256) m = max(m, (int)a.in_exp[r]);
+            if (m != kEZero) atomicMax(&gmx[0], m);
+        } else if (threadIdx.x < per * ng) {
             // E_ZERO (-128) is the smallest byte: it only wins where every member is zero
             int m0 = kEZero, m1 = kEZero, m2 = kEZero, m3 = kEZero;
             const int8_t *e = a.in_exp + g_first + k;

@@ -125,9 +125,10 @@ struct GemmSmem {
 // Output stores: straight to global memory, or (TS) into the warpgroup's staging rows,
 // 64 bytes per output row with the 16-byte chunks in the TMA store's 64-byte swizzle order
 // (chunk ^ ((row >> 1) & 3)), which also keeps the row-per-thread writes free of bank
-// conflicts.  scol: the chunk's first column within the warpgroup's 64.
+// conflicts.  scol: the chunk's first column within the warpgroup's staged columns (64, or
+// 128 as two 128 x 64 blocks, one TMA store each).
 __device__ __forceinline__ void stage16(uint8_t *srow, int et, int scol, uint4 v) {
-    *reinterpret_cast<uint4 *>(srow + (((scol >> 4) ^ ((et >> 1) & 3)) << 4)) = v;
+    *reinterpret_cast<uint4 *>(srow + (scol >> 6) * (128 * 64) + ((((scol >> 4) & 3) ^ ((et >> 1) & 3)) << 4)) = v;
 }
 
 template <bool MUL, int NC, bool TS = false>  // MUL = false: every column of the group has the same exponent
@@ -350,15 +351,23 @@ __device__ __forceinline__ void epi_two_pass(const GemmParams &p, uint32_t taddr
 // With Q4 on pairs (TS), each epilogue warpgroup stages its 128 x 64 share of a tile's
 // int8 output in shared memory and one of its threads writes it with a TMA store through
 // tmY (the output, 64-byte swizzle, 64 x 128 boxes), instead of 16-byte stores that each
-// touch 32 rows.
-template <int BN, int BK, int STAGES, int LOAD, int OUTK, int GC = 0, int NWG = 2, bool PAIR = false, bool Q4 = false>
+// touch 32 rows.  STG: the same for single CTAs with four warpgroups on alternate 128-wide
+// tiles, each staging its whole 128 x 128 tile as two such boxes.
+template <int BN, int BK, int STAGES, int LOAD, int OUTK, int GC = 0, int NWG = 2, bool PAIR = false, bool Q4 = false,
+          bool STG = false>
 __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmParams p) {
     static_assert(!Q4 || NWG == 4, "Q4: four epilogue warpgroups");
-    constexpr bool TS = PAIR && Q4 && OUTK == EPI_FIT_ROW;
-    static_assert(!TS || BN == 256, "staged stores: 64 columns per warpgroup");
-    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * 64 : 0>;
+    // staged output: pairs with Q4 (64 columns per warpgroup), and single CTAs with four
+    // warpgroups on alternate 128-wide tiles of 32-column groups (128 columns per warpgroup)
+    constexpr bool TS1 = STG;
+    static_assert(!STG || (!PAIR && !Q4 && NWG == 4 && BN == 128 && GC == 1 && LOAD == LOAD_2D && OUTK == EPI_FIT_ROW),
+                  "staged single-CTA output: four warpgroups, 128-wide tiles of 32-column groups");
+    constexpr bool TS = (PAIR && Q4 && OUTK == EPI_FIT_ROW) || TS1;
+    constexpr int SCOLS = TS1 ? 128 : 64;  // staged columns per warpgroup
+    static_assert(!TS || BN == 256 || TS1, "staged stores: 64 columns per warpgroup");
+    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * SCOLS : 0>;
     static_assert(!PAIR || (LOAD == LOAD_2D && BN % 64 == 0), "pairs: 2-D loads, BN a multiple of 64");
     constexpr int TM = PAIR ? 256 : 128;  // rows of an output tile
     constexpr int NACC = Q4 ? 2 : NWG;
@@ -705,7 +714,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
             tc_fence_after();
 
             const bool valid = et < valid_rows;
-            uint8_t *srow = sStage + wg * (128 * 64) + et * 64;  // TS: this thread's staged output row
+            uint8_t *srow = sStage + wg * (128 * SCOLS) + et * 64;  // TS: this thread's staged output row
             const int64_t grow = row_base + et;
             const int ea = valid ? ea_pf : 0;
             const int gcol0 = n0 / p.G;  // output group of the tile's first column
@@ -1021,6 +1030,18 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         tma_store_2d(&tmY, smem_u32(sStage + wg * (128 * 64)), n0 + c_lo, (int)row_base);
                         bulk_commit();
                     }
+                }
+            } else if constexpr (TS) {
+                // every row staged and every TMEM read done: the accumulator is released, then
+                // one thread stores the warpgroup's tile, one TMA store per 64 columns
+                named_bar_sync(bar_id, 128);
+                mbar_arrive(bar_tempty + 8 * acc);
+                if (et == 0 && valid_rows > 0) {
+#pragma unroll
+                    for (int b = 0; b < SCOLS / 64; ++b)
+                        tma_store_2d(&tmY, smem_u32(sStage + wg * (128 * SCOLS) + b * (128 * 64)), n0 + c_lo + 64 * b,
+                                     (int)row_base);
+                    bulk_commit();
                 }
             } else {
                 mbar_arrive(bar_tempty + 8 * acc);

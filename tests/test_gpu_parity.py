@@ -157,6 +157,28 @@ def test_linear_bwd_weight_row_groups_across_tiles(ict, M, N, K, xg, xspan):
     status_ok(ict)
 
 
+@pytest.mark.parametrize("M,N,K,wspan", [
+    (1000, 256, 192, (-12, -6)),    # ragged last M tile, two 128-wide tiles per row band
+    (300, 768, 768, (-40, -6)),     # column exponents far apart: the exact per-element path, staged
+    (64, 128, 64, (-12, -6)),       # fewer rows than one tile
+    (2000, 384, 1024, (-12, -9)),   # the longest contraction on this plan
+])
+def test_linear_staged_single_cta(ict, M, N, K, wspan):
+    """Short contractions with 32-column output groups: four epilogue warpgroups on
+    alternate 128-wide tiles of single CTAs, each staging its 128 x 128 output tile in
+    shared memory for two TMA stores, against the oracle (forward and backward-data)."""
+    rng = np.random.default_rng(M + N + K)
+    X = rand_ce(rng, M, K, 1, 64 if K % 64 == 0 else K, elo=-10, ehi=-4, zero_groups=0.05)
+    W = rand_ce(rng, N, K, 1, K, elo=wspan[0], ehi=wspan[1], zero_groups=0.05)
+    same(ict.linear_fwd(ict.DevCE.from_host(X), ict.DevCE.from_host(W), 32).to_host(), oracle.linear_fwd(X, W, 1, 32),
+         "staged fwd")
+    dY = with_groups(clipped_laplace(rng, (M, K)), 1, 32, lambda g: rng.integers(-16, -10, size=g))
+    Wt = rand_ce(rng, K, N, 1, 64, elo=wspan[0], ehi=wspan[1])
+    same(ict.linear_bwd_data(ict.DevCE.from_host(dY), ict.DevCE.from_host(Wt), 32).to_host(),
+         oracle.linear_bwd_data(dY, Wt, 1, 32), "staged bwd-data")
+    status_ok(ict)
+
+
 @pytest.mark.parametrize("M,N,K,G,wspan", [
     (12000, 576, 256, 64, (-12, -6)),    # 192-wide pair tiles, ragged last M tile
     (12000, 576, 256, 64, (-40, -6)),    # the same with column exponents far apart: the exact per-element path
