@@ -568,32 +568,95 @@ def time_classes(step, K, flush):
 
 
 def time_e2e(step, graph, K, W):
-    """The same step through the public API with host buffers: pinned H2D copies of the
-    step's inputs, the step's graph, D2H copies of its results, all inside the timed
-    region."""
+    """The same step through the public API with host buffers: every step's inputs are
+    copied from pinned host memory and its results read back into pinned host memory,
+    all inside the timed region.  The copies are pipelined with the compute, as a
+    training loop's input prefetch does.  The step's inputs travel as one packed pinned
+    buffer into one of two device staging buffers (one host call per step, on a copy
+    stream) while the previous step computes; two CUDA graphs, one per staging buffer,
+    each scatter their staging buffer into the step's input tensors, run the step and
+    gather its results into a packed output staging buffer, which a second copy stream
+    reads back (one host call) while the next step computes.  Returns the time per step
+    and the host bytes moved each way per step."""
     torch = step.torch
-    host_in = [(t.cpu().pin_memory(), t) for t in step.h2d]
-    host_out = [(torch.empty_like(t, device="cpu").pin_memory(), t) for t in step.d2h]
-    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
-    d2h = sum(h.numel() * h.element_size() for h, _ in host_out)
+    ict = step.ict
 
-    def one():
-        for h, d in host_in:
-            d.copy_(h, non_blocking=True)
-        graph.replay()
-        for h, d in host_out:
-            h.copy_(d, non_blocking=True)
+    def layout(ts):
+        offs, off = [], 0
+        for t in ts:
+            offs.append(off)
+            off += (t.numel() * t.element_size() + 255) // 256 * 256
+        return offs, max(off, 256)
 
-    for _ in range(W):
-        one()
+    def view(buf, off, t):
+        n = t.numel() * t.element_size()
+        return buf[off:off + n].view(t.dtype).view(t.shape)
+
+    ins, outs = list(step.h2d), list(step.d2h)
+    in_off, in_bytes = layout(ins)
+    out_off, out_bytes = layout(outs)
+    h2d = sum(t.numel() * t.element_size() for t in ins)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    host_in = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+    host_out = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+    for t, o in zip(ins, in_off):
+        view(host_in, o, t).copy_(t.cpu())
+    stage_in = [torch.empty(in_bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    stage_out = [torch.empty(out_bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+
+    def graph_fn(b):
+        def fn():
+            for t, o in zip(ins, in_off):
+                t.copy_(view(stage_in[b], o, t))
+            step.run()
+            for t, o in zip(outs, out_off):
+                view(stage_out[b], o, t).copy_(t)
+        return fn
+
+    for b in range(2):  # the staging buffers' first contents: the inputs themselves
+        stage_in[b].copy_(host_in)
+    graphs = [ict.StepGraph(graph_fn(b)) for b in range(2)]
+    cur = torch.cuda.current_stream()
+    cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
+    landed = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]
+
+    def prefetch(b):  # host -> staging b, once the graph that last read it has finished
+        cs_in.wait_event(done[b])
+        with torch.cuda.stream(cs_in):
+            stage_in[b].copy_(host_in, non_blocking=True)
+            landed[b].record(cs_in)
+
+    def run(n):
+        for b in range(2):
+            done[b].record(cur)
+            read[b].record(cs_out)
+        prefetch(0)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:
+                prefetch(b ^ 1)  # overlaps this step's compute
+            cur.wait_event(landed[b])
+            cur.wait_event(read[b])  # the read-back of two steps ago has left stage_out[b]
+            graphs[b].replay()
+            done[b].record(cur)
+            cs_out.wait_event(done[b])
+            with torch.cuda.stream(cs_out):
+                host_out.copy_(stage_out[b], non_blocking=True)
+                read[b].record(cs_out)
+        cur.wait_stream(cs_out)
+        cur.wait_stream(cs_in)
+
+    run(W)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for _ in range(K):
-        one()
-    b.record()
+    run(K)
+    b_.record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / K, h2d, d2h
+    del graphs  # released here, before any process-group teardown (they may hold collectives)
+    return a.elapsed_time(b_) / K, h2d, d2h
 
 
 def class_rate(name, c, peaks):
@@ -753,7 +816,9 @@ def measure(step, ict, torch, peaks, flush, config, steps, warmup, dist=None):
         "value": round(step.value_of(step.units, ms * 1e-3) * agg, 3), "unit": step.unit,
         "ms_per_step": round(ms, 4),
         "e2e": {"value": round(step.value_of(step.units, e2e_ms * 1e-3) * agg, 3), "unit": step.unit,
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "copies": "one packed pinned buffer each way per step; step i+1's inputs copied in and step i's "
+                          "results read back on two copy streams while step i computes (device staging buffers)"},
         "gpu_launches": int(graph.launches * steps),
         "gpu_launches_per_step": graph.launches,
         "launch": "one CUDA graph replay per step",
