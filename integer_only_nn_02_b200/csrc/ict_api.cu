@@ -619,6 +619,20 @@ int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     return run(gemm_ce_kernel<BN, 128, ST, LOAD_2D, EPI_FIT_ROW, 0, 2, true>, kB, 2);
 }
 
+// Convolution Products on halo tiles (RO16 epilogue, four warpgroups, three stages of
+// three 16 KB box slots, the nine weight blocks resident).
+template <int BN>
+int launch_gemm_halo(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid, cudaStream_t s) {
+    constexpr int ST = 3;
+    constexpr int kB = GemmSmem<BN, 64, ST, 4, false, 4, 0, 3 * kHaloSlot, 9>::kBytes;
+    auto k = gemm_ce_kernel<BN, 64, ST, LOAD_CONV_HALO, EPI_RO16, 0, 4>;
+    if (p.epi != EPI_RO16 || p.nwg != 4 || p.n_ntiles != 1 || p.cv_bkblk > 9) return ICT_ERR_LAYOUT;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kB) != cudaSuccess) return ICT_ERR_CUDA;
+    k<<<grid, 128 + 128 * 4, kB, s>>>(ta, tb, tb, p);
+    counted(1);
+    return launch_status();
+}
+
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
                 const GemmParams &p_in, int grid, cudaStream_t s, double ops, bool pair = false,
                 const CUtensorMap *ty = nullptr) {
@@ -627,9 +641,15 @@ int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorM
     // group straddles the halves
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
-    const bool nwg4_ok = p.epi == EPI_FIT_ROW || (p.epi == EPI_RO16 && load == LOAD_CONV);
+    const bool nwg4_ok = p.epi == EPI_FIT_ROW || (p.epi == EPI_RO16 && (load == LOAD_CONV || load == LOAD_CONV_HALO));
     if (p.nwg != 4 || !nwg4_ok || pair) p.nwg = 2;
     p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || p.epi == EPI_RO16R || (gt < bn && (bn / 2) % gt == 0));
+    if (load == LOAD_CONV_HALO) {
+        if (bk != 64 || pair) return ICT_ERR_LAYOUT;
+        if (bn == 64) return launch_gemm_halo<64>(ta, tb, p, grid, s);
+        if (bn == 128) return launch_gemm_halo<128>(ta, tb, p, grid, s);
+        return ICT_ERR_LAYOUT;
+    }
     if (pair) {
         if (load != LOAD_2D || bk != 128 || (grid & 1)) return ICT_ERR_LAYOUT;
         const CUtensorMap &y = ty ? *ty : tb;  // the output map, for staged stores
@@ -1222,7 +1242,14 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         if ((st = launch_status())) return st;
     }
     CUtensorMap ta, tb;
-    if ((st = tmap_nhwc(&ta, cp.a_mant, d->n, d->h, d->w, cp.a_c, cp.rows_per_tile))) return st;
+    // halo tiles: 3 x 3 filters, 64 contracted channels (the nine weight blocks resident),
+    // image rows a multiple of 8 pixels (each row shift a whole number of swizzle atoms), a
+    // box of rows + 2 image rows plus the MMA's overhang inside one 16 KB slot, all-pixel
+    // output groups on one N tile (the four-warpgroup RO16 epilogue)
+    const bool halo = cp.global_groups && d->r == 3 && d->s == 3 && d->pad == 1 && cp.a_c == 64 && d->w % 8 == 0 &&
+                      (int64_t)(cp.rows_per_tile + 2) * d->w * 64 <= kHaloSlot &&
+                      (int64_t)2 * d->w * 64 + 128 * 64 <= kHaloSlot && cp.bn <= 128 && cp.out_cols <= cp.bn;
+    if ((st = tmap_nhwc(&ta, cp.a_mant, d->n, d->h, d->w, cp.a_c, cp.rows_per_tile + (halo ? 2 : 0)))) return st;
     const int64_t ktot = (int64_t)d->r * d->s * cp.a_c;
     if ((st = tmap_2d(&tb, cp.b_mant, ktot, cp.out_cols, cp.b_ld, 64, cp.bn, CU_TENSOR_MAP_SWIZZLE_64B)))
         return st;
@@ -1258,6 +1285,13 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     // the weight operand stays in shared memory when all its K blocks fit the B ring
     p.b_resident = p.n_ntiles == 1 && p.n_kblk <= stages_for(cp.bn, 64);
     p.stage_tx_bytes = (uint32_t)(64 * d->w * cp.rows_per_tile + (p.b_resident ? 0 : 64 * cp.bn));
+    if (halo) {  // one stage per 64-channel block: three boxes of rows + 2 image rows
+        p.cv_bkblk = p.n_kblk;
+        p.n_kblk = p.cv_cblk;
+        p.kblk_per_split = p.n_kblk;
+        p.b_resident = 1;
+        p.stage_tx_bytes = (uint32_t)(3 * 64 * d->w * (cp.rows_per_tile + 2));
+    }
     p.qb = 8;
     p.wait_ns = g_wait_ns;
     p.drain_ns = kDrainNs;
@@ -1280,7 +1314,8 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     p.ws16 = cp.ws16;
     p.ws16_ld = cp.ws16_ld;
     p.tile_need = cp.tile_need;
-    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, LOAD_CONV, ta, tb, p, grid, s, ops))) return st;
+    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, halo ? LOAD_CONV_HALO : LOAD_CONV, ta, tb, p, grid, s, ops)))
+        return st;
     if (!(phase & 2)) return ICT_OK;
     Ro16RoundArgs r;
     r.v = cp.ws16;

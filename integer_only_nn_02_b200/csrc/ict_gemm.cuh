@@ -45,7 +45,14 @@ enum EpiMode : int {
 // LOAD_CONV_WGRAD A: two (tap, 64-channel) slices of the shifted NHWC input X, B: 64
 //                 channels of dY, both MN-major with output pixels as K (convolution
 //                 backward-weight); BK is the largest number of pixels per K block
-enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1, LOAD_CONV_WGRAD = 2 };
+enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1, LOAD_CONV_WGRAD = 2, LOAD_CONV_HALO = 3 };
+// LOAD_CONV_HALO  3 x 3 "same" convolutions whose image width is a multiple of 8: per tile
+//                 and 64-channel block, three 4-D boxes (one per column shift of the
+//                 filter), each holding the tile's rows and one halo row above and below;
+//                 every tap's operand is a window of one box starting a whole number of
+//                 image rows in (a multiple of the 8-row swizzle atom), so nine taps take
+//                 three copies instead of nine.  The weight operand stays resident.
+constexpr int kHaloSlot = 16384;  // bytes per box slot (256 rows of 64 bytes)
 
 struct GemmParams {
     int M, N;       // output rows (MMA M side) and columns (MMA N side)
@@ -79,6 +86,9 @@ struct GemmParams {
     // conv: every K block of the weight operand held in shared memory for the whole kernel
     // (block kb at the B ring's slot kb; needs n_kblk <= STAGES); stage_tx_bytes is then A only
     int b_resident;
+    // LOAD_CONV_HALO: the weight's K blocks held resident (taps x channel blocks); n_kblk
+    // counts the channel blocks, one stage each
+    int cv_bkblk;
     // backward-weight: K block = wg_hrows image rows of every image (wg_kpix pixels), M rows
     // (tap, channel) in 64-row atoms (wg_atoms in total)
     int wg_hrows, wg_hblk, wg_kpix, wg_atoms;
@@ -90,16 +100,18 @@ struct GemmParams {
     int nwg;        // host only: epilogue warpgroups of the instantiation to launch (2 or 4)
 };
 
-template <int BN, int BK, int STAGES, int NWG = 2, bool PAIR = false, int NACC = NWG, int STAGE = 0>
+template <int BN, int BK, int STAGES, int NWG = 2, bool PAIR = false, int NACC = NWG, int STAGE = 0, int AB = 0,
+          int BSLOTS = 0>
 struct GemmSmem {
-    static constexpr int kABytes = 128 * BK;
+    static constexpr int kABytes = AB ? AB : 128 * BK;  // A bytes per stage
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK;  // a pair's CTA holds half of B
     // NACC TMEM accumulators of BN columns
     static constexpr int kTmemCols = (NACC * BN <= 32) ? 32 : (NACC * BN <= 64) ? 64 : (NACC * BN <= 128) ? 128
                                    : (NACC * BN <= 256) ? 256 : 512;
     static_assert(NACC * BN <= 512, "accumulators must fit TMEM");
     static constexpr int kOffB = STAGES * kABytes;
-    static constexpr int kOffBar = kOffB + STAGES * kBBytes;  // 2*STAGES + 2*NACC + 2 mbarriers
+    static constexpr int kBSlots = BSLOTS > STAGES ? BSLOTS : STAGES;  // B slots (a resident weight may need more)
+    static constexpr int kOffBar = kOffB + kBSlots * kBBytes;  // 2*STAGES + 2*NACC + 2 mbarriers
     static constexpr int kOffMisc = (kOffBar + (2 * STAGES + 2 * NACC + 2) * 8 + 15) / 16 * 16;
     static constexpr int kColInts = 2 * BN + 32;               // per epilogue warpgroup
     static constexpr int kOffCol = kOffMisc + 16;              // read with 16-byte vectors
@@ -367,7 +379,10 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     constexpr bool TS = (PAIR && Q4 && OUTK == EPI_FIT_ROW) || TS1;
     constexpr int SCOLS = TS1 ? 128 : 64;  // staged columns per warpgroup
     static_assert(!TS || BN == 256 || TS1, "staged stores: 64 columns per warpgroup");
-    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * SCOLS : 0>;
+    constexpr bool HALO = LOAD == LOAD_CONV_HALO;
+    static_assert(!HALO || (BK == 64 && !PAIR), "halo tiles: 64-byte channel rows, single CTAs");
+    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * SCOLS : 0, HALO ? 3 * kHaloSlot : 0,
+                       HALO ? 9 : 0>;
     static_assert(!PAIR || (LOAD == LOAD_2D && BN % 64 == 0), "pairs: 2-D loads, BN a multiple of 64");
     constexpr int TM = PAIR ? 256 : 128;  // rows of an output tile
     constexpr int NACC = Q4 ? 2 : NWG;
@@ -447,10 +462,11 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
             int issued[STAGES];
             uint32_t issued_phase[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = 0, issued_phase[s] = 0;
-            const bool bres = LOAD == LOAD_CONV && p.b_resident;
+            const bool bres = (LOAD == LOAD_CONV || HALO) && p.b_resident;
             if (bres && blockIdx.x < p.num_units) {  // the weight operand, once
-                mbar_expect_tx(bar_bres, (uint32_t)(p.n_kblk * L::kBBytes));
-                for (int kb = 0; kb < p.n_kblk; ++kb)
+                const int nb = HALO ? p.cv_bkblk : p.n_kblk;
+                mbar_expect_tx(bar_bres, (uint32_t)(nb * L::kBBytes));
+                for (int kb = 0; kb < nb; ++kb)
                     tma_load_2d(sbase + L::kOffB + kb * L::kBBytes, &tmB, bar_bres, kb * BK, 0);
             }
             for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas) {
@@ -459,7 +475,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 const int kb0 = split * p.kblk_per_split;
                 const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
                 int img = 0, h0 = 0;
-                if (LOAD == LOAD_CONV) {
+                if (LOAD == LOAD_CONV || HALO) {
                     img = mt / p.cv_tiles_per_img;
                     h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
                 }
@@ -482,6 +498,13 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         mbar_expect_tx(fb, p.stage_tx_bytes);
                         tma_load_2d(sa, &tmA, fb, kb * BK, mt * 128);
                         tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
+                    } else if (HALO) {
+                        // three boxes (column shifts s - pad) of rows [hs, hs + rows + 2): every
+                        // row shift r - pad is a window of them (the MMA's descriptor offset)
+                        mbar_expect_tx(fb, p.stage_tx_bytes);
+                        const int hs = p.cv_sign > 0 ? h0 - p.cv_pad : h0 + p.cv_pad - (p.cv_S - 1);
+                        for (int s2 = 0; s2 < p.cv_S; ++s2)
+                            tma_load_4d(sa + s2 * kHaloSlot, &tmA, fb, kb * 64, p.cv_sign * (s2 - p.cv_pad), hs, img);
                     } else if (LOAD == LOAD_CONV) {
                         mbar_expect_tx(fb, p.stage_tx_bytes);
                         const int tap = kb / p.cv_cblk, cb = kb % p.cv_cblk;
@@ -526,7 +549,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
             uint32_t phase = 0;
             int it = 0;
             bool any = false;
-            if (LOAD == LOAD_CONV && p.b_resident && blockIdx.x < p.num_units &&
+            if ((LOAD == LOAD_CONV || HALO) && p.b_resident && blockIdx.x < p.num_units &&
                 !mbar_wait(bar_bres, 0, p.wait_ns, abort_flag))
                 fail();
             for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas, ++it) {
@@ -548,7 +571,23 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         break;
                     }
                     tc_fence_after();
-                    if constexpr (kMN) {
+                    if constexpr (HALO) {
+                        // tap (r, s): box s, starting (r or R - 1 - r) image rows in; B block
+                        // (tap, channel block kb) of the resident weight
+                        const uint32_t sa0 = sbase + stage * L::kABytes;
+                        for (int r = 0; r < p.cv_S; ++r) {
+                            const int rr = p.cv_sign > 0 ? r : p.cv_S - 1 - r;
+                            for (int s2 = 0; s2 < p.cv_S; ++s2) {
+                                const uint64_t da = smem_desc_kmajor(sa0 + s2 * kHaloSlot + rr * p.cv_W * 64, BK);
+                                const int bkb = (r * p.cv_S + s2) * p.cv_cblk + kb;
+                                const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + bkb * L::kBBytes, BK);
+#pragma unroll
+                                for (int kk = 0; kk < BK / 32; ++kk)
+                                    umma_i8(tmem_d, da + 2 * kk, db + 2 * kk, kIdesc,
+                                            (kb > kb0 || r > 0 || s2 > 0 || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                    } else if constexpr (kMN) {
                         // 32 pixels per MMA = four 8-row atoms of 64 bytes = 2048 bytes
                         const uint64_t da = smem_desc_mnmajor64(sbase + stage * L::kABytes, L::kABytes / 2);
                         const uint64_t db = smem_desc_mnmajor64(sbase + L::kOffB + stage * L::kBBytes, L::kABytes / 2);
@@ -643,7 +682,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         auto prefetch = [&](bool have) {
             if (!have) return;
             pf_mt = c_mt;
-            if (LOAD == LOAD_CONV) {
+            if (LOAD == LOAD_CONV || HALO) {
                 const int img = c_mt / p.cv_tiles_per_img;
                 const int h0 = (c_mt % p.cv_tiles_per_img) * p.cv_rows;
                 pf_rb = ((int64_t)img * p.cv_P + h0) * p.cv_W;
