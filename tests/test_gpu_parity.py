@@ -236,7 +236,9 @@ def _conv_inputs(seed, n, h, w, c, k, gx=32):
 @pytest.mark.parametrize("shape", [(2, 8, 8, 64, 64), (3, 7, 56, 64, 64), (1, 9, 20, 128, 64),
                                    (2, 5, 12, 64, 128),
                                    # halo tiles with a one-row last tile; and with a box filling its slot
-                                   (2, 9, 16, 64, 64), (1, 6, 64, 64, 64)])
+                                   (2, 9, 16, 64, 64), (1, 6, 64, 64, 64),
+                                   # backward-data on halo tiles with 128 output channels (128-wide tiles)
+                                   (2, 6, 16, 128, 64)])
 @pytest.mark.parametrize("global_groups", [True, False])
 def test_conv_fwd_and_bwd_data(ict, shape, global_groups):
     X, W, dY, d = _conv_inputs(sum(shape), *shape)
