@@ -529,7 +529,7 @@ int launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams
     auto run = [&](auto k, int nwg, int smem_bytes) {
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
             return (int)ICT_ERR_CUDA;
-        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, ty ? *ty : tb, p);  // tmY: staged output only
+        k<<<grid, 128 + 128 * nwg, smem_bytes, s>>>(ta, tb, ty ? *ty : tb, tb, p);  // tmY: staged output only
         counted(1);
         return launch_status();
     };
@@ -599,7 +599,7 @@ int launch_gemm_pair_t(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, k, ta, tb, ty, p) != cudaSuccess) return (int)ICT_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, k, ta, tb, ty, tb, p) != cudaSuccess) return (int)ICT_ERR_CUDA;
         counted(1);
         return launch_status();
     };
@@ -628,22 +628,41 @@ int launch_gemm_halo(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPar
     auto k = gemm_ce_kernel<BN, 64, ST, LOAD_CONV_HALO, EPI_RO16, 0, 4>;
     if (p.epi != EPI_RO16 || p.nwg != 4 || p.n_ntiles != 1 || p.cv_bkblk > 9) return ICT_ERR_LAYOUT;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kB) != cudaSuccess) return ICT_ERR_CUDA;
-    k<<<grid, 128 + 128 * 4, kB, s>>>(ta, tb, tb, p);
+    k<<<grid, 128 + 128 * 4, kB, s>>>(ta, tb, tb, tb, p);
+    counted(1);
+    return launch_status();
+}
+
+// The ring form (64-wide tiles): four stages over three rings of image rows; tm2 is the map
+// of the continuing tiles' boxes, tmz the int16 sums' map for the staged stores.
+int launch_gemm_ring(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tm2, const CUtensorMap &tmz,
+                     const GemmParams &p, int grid, cudaStream_t s) {
+    constexpr int ST = 4;
+    constexpr int kB = GemmSmem<64, 64, ST, 4, false, 4, 128 * 128, 3 * kRingBox / ST, 9>::kBytes;
+    auto k = gemm_ce_kernel<64, 64, ST, LOAD_CONV_RING, EPI_RO16, 0, 4>;
+    if (p.epi != EPI_RO16 || p.nwg != 4 || p.n_ntiles != 1 || p.splits != 1 || p.cv_bkblk > 9) return ICT_ERR_LAYOUT;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kB) != cudaSuccess) return ICT_ERR_CUDA;
+    k<<<grid, 128 + 128 * 4, kB, s>>>(ta, tb, tm2, tmz, p);
     counted(1);
     return launch_status();
 }
 
 int launch_gemm(int bn, int bk, int load, const CUtensorMap &ta, const CUtensorMap &tb,
                 const GemmParams &p_in, int grid, cudaStream_t s, double ops, bool pair = false,
-                const CUtensorMap *ty = nullptr) {
+                const CUtensorMap *ty = nullptr, const CUtensorMap *tz = nullptr) {
     KTimer kt(s, KC_GEMM, ops);
     // both epilogue warpgroups take every tile (one column half each) when no output
     // group straddles the halves
     GemmParams p = p_in;
     const int gt = p.G >= p.N ? bn : p.G;
-    const bool nwg4_ok = p.epi == EPI_FIT_ROW || (p.epi == EPI_RO16 && (load == LOAD_CONV || load == LOAD_CONV_HALO));
+    const bool nwg4_ok = p.epi == EPI_FIT_ROW ||
+                         (p.epi == EPI_RO16 && (load == LOAD_CONV || load == LOAD_CONV_HALO || load == LOAD_CONV_RING));
     if (p.nwg != 4 || !nwg4_ok || pair) p.nwg = 2;
     p.epi_split = p.nwg == 2 && (p.epi == EPI_I32 || p.epi == EPI_RO16R || (gt < bn && (bn / 2) % gt == 0));
+    if (load == LOAD_CONV_RING) {
+        if (bk != 64 || pair || bn != 64 || !ty || !tz) return ICT_ERR_LAYOUT;
+        return launch_gemm_ring(ta, tb, *ty, *tz, p, grid, s);
+    }
     if (load == LOAD_CONV_HALO) {
         if (bk != 64 || pair) return ICT_ERR_LAYOUT;
         if (bn == 64) return launch_gemm_halo<64>(ta, tb, p, grid, s);
@@ -1249,7 +1268,16 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     const bool halo = cp.global_groups && d->r == 3 && d->s == 3 && d->pad == 1 && cp.a_c == 64 && d->w % 8 == 0 &&
                       (int64_t)(cp.rows_per_tile + 2) * d->w * 64 <= kHaloSlot &&
                       (int64_t)2 * d->w * 64 + 128 * 64 <= kHaloSlot && cp.bn <= 128 && cp.out_cols <= cp.bn;
+    // the ring form: 64-wide tiles (the weight's nine blocks and three 56 KB rings fit), a ring
+    // that holds a restarting tile's rows and windows
+    const int ring_rows = (int)(kRingBox / ((int64_t)d->w * 64)), ring_span = 2 + (int)cdiv64(128, d->w);
+    const bool ring = halo && cp.bn == 64 && ring_span <= ring_rows;
+    CUtensorMap ta2, tz;  // ring: the continuing tiles' boxes (the tile's own rows only), the int16 sums
     if ((st = tmap_nhwc(&ta, cp.a_mant, d->n, d->h, d->w, cp.a_c, cp.rows_per_tile + (halo ? 2 : 0)))) return st;
+    if (ring && (st = tmap_nhwc(&ta2, cp.a_mant, d->n, d->h, d->w, cp.a_c, cp.rows_per_tile))) return st;
+    if (ring && (st = tmap_2d(&tz, cp.ws16, (uint64_t)cp.out_cols * 2, (uint64_t)cp.out_rows, (uint64_t)cp.ws16_ld * 2,
+                              128, (uint32_t)(cp.rows_per_tile * d->w), CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
     const int64_t ktot = (int64_t)d->r * d->s * cp.a_c;
     if ((st = tmap_2d(&tb, cp.b_mant, ktot, cp.out_cols, cp.b_ld, 64, cp.bn, CU_TENSOR_MAP_SWIZZLE_64B)))
         return st;
@@ -1291,6 +1319,8 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
         p.kblk_per_split = p.n_kblk;
         p.b_resident = 1;
         p.stage_tx_bytes = (uint32_t)(3 * 64 * d->w * (cp.rows_per_tile + 2));
+        p.cv_ring_rows = ring_rows;
+        p.cv_ring_span = ring_span;
     }
     p.qb = 8;
     p.wait_ns = g_wait_ns;
@@ -1314,7 +1344,8 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     p.ws16 = cp.ws16;
     p.ws16_ld = cp.ws16_ld;
     p.tile_need = cp.tile_need;
-    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, halo ? LOAD_CONV_HALO : LOAD_CONV, ta, tb, p, grid, s, ops)))
+    if ((phase & 1) && (st = launch_gemm(cp.bn, 64, ring ? LOAD_CONV_RING : (halo ? LOAD_CONV_HALO : LOAD_CONV), ta, tb,
+                                         p, grid, s, ops, false, ring ? &ta2 : nullptr, ring ? &tz : nullptr)))
         return st;
     if (!(phase & 2)) return ICT_OK;
     Ro16RoundArgs r;

@@ -45,7 +45,7 @@ enum EpiMode : int {
 // LOAD_CONV_WGRAD A: two (tap, 64-channel) slices of the shifted NHWC input X, B: 64
 //                 channels of dY, both MN-major with output pixels as K (convolution
 //                 backward-weight); BK is the largest number of pixels per K block
-enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1, LOAD_CONV_WGRAD = 2, LOAD_CONV_HALO = 3 };
+enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1, LOAD_CONV_WGRAD = 2, LOAD_CONV_HALO = 3, LOAD_CONV_RING = 4 };
 // LOAD_CONV_HALO  3 x 3 "same" convolutions whose image width is a multiple of 8: per tile
 //                 and 64-channel block, three 4-D boxes (one per column shift of the
 //                 filter), each holding the tile's rows and one halo row above and below;
@@ -53,6 +53,14 @@ enum LoadMode : int { LOAD_2D = 0, LOAD_CONV = 1, LOAD_CONV_WGRAD = 2, LOAD_CONV
 //                 image rows in (a multiple of the 8-row swizzle atom), so nine taps take
 //                 three copies instead of nine.  The weight operand stays resident.
 constexpr int kHaloSlot = 16384;  // bytes per box slot (256 rows of 64 bytes)
+// LOAD_CONV_RING  the halo form with each CTA taking a contiguous run of tiles (in image
+//                 order): the three boxes' image rows live in three rings of kRingBox
+//                 bytes; a tile that continues the previous one (same image, next rows)
+//                 loads only its new rows after the previous tile's, whose last two rows
+//                 are its halo above, and a tile that does not, or that would pass the
+//                 ring's end, restarts at the ring's start once the previous tile's MMAs
+//                 are done.  Windows read past a tile's rows only for invalid output rows.
+constexpr int kRingBox = 36864;
 
 struct GemmParams {
     int M, N;       // output rows (MMA M side) and columns (MMA N side)
@@ -89,6 +97,11 @@ struct GemmParams {
     // LOAD_CONV_HALO: the weight's K blocks held resident (taps x channel blocks); n_kblk
     // counts the channel blocks, one stage each
     int cv_bkblk;
+    // LOAD_CONV_RING: image rows a ring holds, and the rows a tile's windows span from its
+    // first row (2 + ceil(128 / W)); tmY is then the map of the continuing tiles' boxes,
+    // and tmZ the int16 sums as bytes (128-byte rows, 128-byte swizzle, boxes of a full
+    // tile's cv_rows * cv_W rows) for the staged RO16 stores
+    int cv_ring_rows, cv_ring_span;
     // backward-weight: K block = wg_hrows image rows of every image (wg_kpix pixels), M rows
     // (tap, channel) in 64-row atoms (wg_atoms in total)
     int wg_hrows, wg_hblk, wg_kpix, wg_atoms;
@@ -369,7 +382,8 @@ template <int BN, int BK, int STAGES, int LOAD, int OUTK, int GC = 0, int NWG = 
           bool STG = false>
 __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     gemm_ce_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmZ,
+                   const __grid_constant__ GemmParams p) {
     static_assert(!Q4 || NWG == 4, "Q4: four epilogue warpgroups");
     // staged output: pairs with Q4 (64 columns per warpgroup), and single CTAs with four
     // warpgroups on alternate 128-wide tiles of 32-column groups (128 columns per warpgroup)
@@ -379,10 +393,15 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     constexpr bool TS = (PAIR && Q4 && OUTK == EPI_FIT_ROW) || TS1;
     constexpr int SCOLS = TS1 ? 128 : 64;  // staged columns per warpgroup
     static_assert(!TS || BN == 256 || TS1, "staged stores: 64 columns per warpgroup");
-    constexpr bool HALO = LOAD == LOAD_CONV_HALO;
+    constexpr bool RING = LOAD == LOAD_CONV_RING;
+    constexpr bool HALO = LOAD == LOAD_CONV_HALO || RING;
     static_assert(!HALO || (BK == 64 && !PAIR), "halo tiles: 64-byte channel rows, single CTAs");
-    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * SCOLS : 0, HALO ? 3 * kHaloSlot : 0,
-                       HALO ? 9 : 0>;
+    static_assert(!RING || (3 * kRingBox) % STAGES == 0, "ring: the A region split evenly over the stages");
+    // RING with RO16: each epilogue warpgroup stages its tile's int16 sums (128 rows of 128
+    // bytes, 128-byte swizzle) for one TMA store instead of row-per-thread 16-byte stores
+    constexpr bool TS16 = RING && OUTK == EPI_RO16 && NWG == 4 && BN == 64;
+    using L = GemmSmem<BN, BK, STAGES, NWG, PAIR, Q4 ? 2 : NWG, TS ? 128 * SCOLS : (TS16 ? 128 * 128 : 0),
+                       RING ? 3 * kRingBox / STAGES : (HALO ? 3 * kHaloSlot : 0), HALO ? 9 : 0>;
     static_assert(!PAIR || (LOAD == LOAD_2D && BN % 64 == 0), "pairs: 2-D loads, BN a multiple of 64");
     constexpr int TM = PAIR ? 256 : 128;  // rows of an output tile
     constexpr int NACC = Q4 ? 2 : NWG;
@@ -411,6 +430,16 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     const bool leader = rank == 0;
     const int cta0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
     const int ctas = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    // RING: the k-th unit of this CTA (u = cta0 + k ctas) is tile ring0 + k, so that its
+    // tiles are contiguous (the same count of units as the strided walk)
+    const int ring0 = RING ? cta0 * (p.num_units / ctas) + min(cta0, p.num_units % ctas) : 0;
+    // ring position of a tile given the previous tile's (the same walk in producer and MMA)
+    auto ring_pos = [&](int mt, int &pos, int &pimg, int &ph0, bool &cont) {
+        const int img = mt / p.cv_tiles_per_img, h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
+        cont = img == pimg && h0 == ph0 + p.cv_rows && pos + p.cv_rows + p.cv_ring_span <= p.cv_ring_rows;
+        pos = cont ? pos + p.cv_rows : 0;
+        pimg = img, ph0 = h0;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -431,7 +460,8 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (TS) prefetch_tmap(&tmY);
+        if (TS || RING) prefetch_tmap(&tmY);
+        if (TS16) prefetch_tmap(&tmZ);
     }
     if (warp == 2) {
         if constexpr (PAIR) {
@@ -469,8 +499,11 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 for (int kb = 0; kb < nb; ++kb)
                     tma_load_2d(sbase + L::kOffB + kb * L::kBBytes, &tmB, bar_bres, kb * BK, 0);
             }
+            int r_pos = 0, r_img = -1, r_h0 = -1000000, prev_stage = -1;
+            uint32_t prev_phase = 0;
             for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas) {
-                const int tile = u % (p.n_mtiles * p.n_ntiles), split = u / (p.n_mtiles * p.n_ntiles);
+                const int tile = RING ? ring0 + (u - cta0) / ctas : u % (p.n_mtiles * p.n_ntiles);
+                const int split = RING ? 0 : u / (p.n_mtiles * p.n_ntiles);
                 const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
                 const int kb0 = split * p.kblk_per_split;
                 const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
@@ -478,6 +511,17 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 if (LOAD == LOAD_CONV || HALO) {
                     img = mt / p.cv_tiles_per_img;
                     h0 = (mt % p.cv_tiles_per_img) * p.cv_rows;
+                }
+                bool r_cont = false;
+                if constexpr (RING) {
+                    ring_pos(mt, r_pos, r_img, r_h0, r_cont);
+                    // a restart overwrites rows that earlier tiles read: wait until the
+                    // previous tile's MMAs (and so all earlier ones) are done
+                    if (!r_cont && prev_stage >= 0 &&
+                        !mbar_wait(bar_empty + 8 * prev_stage, prev_phase, p.wait_ns, abort_flag)) {
+                        fail();
+                        break;
+                    }
                 }
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, p.wait_ns, abort_flag)) {
@@ -498,6 +542,15 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         mbar_expect_tx(fb, p.stage_tx_bytes);
                         tma_load_2d(sa, &tmA, fb, kb * BK, mt * 128);
                         tma_load_2d(sb, &tmB, fb, kb * BK, nt * BN);
+                    } else if (RING) {
+                        // rows h0 - 1 .. h0 + rows at ring rows r_pos .. (a restart), or only the
+                        // new rows h0 + 1 .. h0 + rows after the previous tile's (a continuation)
+                        const int nrows = r_cont ? p.cv_rows : p.cv_rows + 2;
+                        const int drow = r_cont ? r_pos + 2 : r_pos, hsrc = r_cont ? h0 + 1 : h0 - 1;
+                        mbar_expect_tx(fb, (uint32_t)(3 * nrows * p.cv_W * 64));
+                        for (int s2 = 0; s2 < 3; ++s2)
+                            tma_load_4d(sbase + s2 * kRingBox + drow * p.cv_W * 64, r_cont ? &tmY : &tmA, fb, kb * 64,
+                                        p.cv_sign * (s2 - p.cv_pad), hsrc, img);
                     } else if (HALO) {
                         // three boxes (column shifts s - pad) of rows [hs, hs + rows + 2): every
                         // row shift r - pad is a window of them (the MMA's descriptor offset)
@@ -527,6 +580,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     }
                     issued[stage] = 1;
                     issued_phase[stage] = phase;
+                    prev_stage = stage, prev_phase = phase;
                     if (++stage == STAGES) stage = 0, phase ^= 1;
                 }
             }
@@ -552,8 +606,11 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
             if ((LOAD == LOAD_CONV || HALO) && p.b_resident && blockIdx.x < p.num_units &&
                 !mbar_wait(bar_bres, 0, p.wait_ns, abort_flag))
                 fail();
+            int r_pos = 0, r_img = -1, r_h0 = -1000000;
             for (int u = cta0; u < p.num_units && !*abort_flag; u += ctas, ++it) {
-                const int split = u / (p.n_mtiles * p.n_ntiles);
+                const int split = RING ? 0 : u / (p.n_mtiles * p.n_ntiles);
+                bool r_cont = false;
+                if constexpr (RING) ring_pos(ring0 + (u - cta0) / ctas, r_pos, r_img, r_h0, r_cont);
                 const int kb0 = split * p.kblk_per_split;
                 const int kb1 = min(p.n_kblk, kb0 + p.kblk_per_split);
                 const int acc = it % NACC;
@@ -574,11 +631,12 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     if constexpr (HALO) {
                         // tap (r, s): box s, starting (r or R - 1 - r) image rows in; B block
                         // (tap, channel block kb) of the resident weight
-                        const uint32_t sa0 = sbase + stage * L::kABytes;
+                        const uint32_t sa0 = RING ? sbase + r_pos * p.cv_W * 64 : sbase + stage * L::kABytes;
+                        const int slot = RING ? kRingBox : kHaloSlot;
                         for (int r = 0; r < p.cv_S; ++r) {
                             const int rr = p.cv_sign > 0 ? r : p.cv_S - 1 - r;
                             for (int s2 = 0; s2 < p.cv_S; ++s2) {
-                                const uint64_t da = smem_desc_kmajor(sa0 + s2 * kHaloSlot + rr * p.cv_W * 64, BK);
+                                const uint64_t da = smem_desc_kmajor(sa0 + s2 * slot + rr * p.cv_W * 64, BK);
                                 const int bkb = (r * p.cv_S + s2) * p.cv_cblk + kb;
                                 const uint64_t db = smem_desc_kmajor(sbase + L::kOffB + bkb * L::kBBytes, BK);
 #pragma unroll
@@ -669,8 +727,11 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         // incrementally, with no division per tile.
         const int NT = p.n_ntiles, MT = p.n_mtiles, T = MT * NT;
         const int u0 = cta0 + stream * ctas;
-        const int d_split = u_step / T, d_m = (u_step % T) / NT, d_n = (u_step % T) % NT;
-        int c_split = u0 / T, c_mt = (u0 % T) / NT, c_nt = (u0 % T) % NT;  // unit being prefetched
+        // RING (one N tile, no split): the walk's units are tiles ring0 + k
+        const int d_split = RING ? 0 : u_step / T, d_m = RING ? streams : (u_step % T) / NT;
+        const int d_n = RING ? 0 : (u_step % T) % NT;
+        int c_split = RING ? 0 : u0 / T, c_mt = RING ? ring0 + stream : (u0 % T) / NT;
+        int c_nt = RING ? 0 : (u0 % T) % NT;  // unit being prefetched
         // group of a tile column: shift for power-of-two widths (Gt == BN: always group 0)
         const int gsh = (Gt & (Gt - 1)) == 0 ? __ffs(Gt) - 1 : -1;
         auto group_of = [&](int j) { return gsh >= 0 ? j >> gsh : j / Gt; };
@@ -726,7 +787,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                     if (BN > 128) cmin[4 + wq] = lo1, cmax[4 + wq] = hi1;
                 }
             }
-            if (TS && et == 0) bulk_wait_read();  // the previous tile's store has read the staging rows
+            if ((TS || TS16) && et == 0) bulk_wait_read();  // the previous tile's store has read the staging rows
             named_bar_sync(bar_id, 128);
             auto group_range = [&](int g, int &lo, int &hi) {
                 lo = 0x7fffffff, hi = kNoExp;
@@ -847,6 +908,9 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 // with two or more extra bits and then to nearest is correct rounding:
                 // Boldo and Melquiond, IEEE Trans. Computers 57(4), 2008).
                 int *red = sRed + wg * 32;
+                // staged stores for whole tiles only: a box of cv_rows * cv_W rows must not reach
+                // the next tile's pixels
+                const bool st16 = TS16 && valid_rows == p.cv_rows * p.cv_W;
                 for (int g = g_lo; g < g_hi; ++g) {
                     const int g0 = g * Gt, gf = gfast[g];
                     int need = kNoExp;
@@ -920,9 +984,18 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                                 w[q >> 1] = __byte_perm((uint32_t)ro((int)v[q], e1 - ea - colE[c + q]),
                                                         (uint32_t)ro((int)v[q + 1], e1 - ea - colE[c + q + 1]), 0x5410);
                         }
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.ws16 + grow * p.ws16_ld + n0 + c);
+                        if (TS16 && st16) {  // 16-byte chunk k of the row at (k ^ (row & 7)) * 16
+                            uint8_t *srow16 = sStage + wg * (128 * 128) + et * 128;
+                            const int k0 = (c - c_lo) >> 3;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                            for (int q = 0; q < 4; ++q)
+                                *reinterpret_cast<uint4 *>(srow16 + (((k0 + q) ^ (et & 7)) << 4)) =
+                                    make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(p.ws16 + grow * p.ws16_ld + n0 + c);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                        }
                     }
                 }
             } else {
@@ -1070,6 +1143,16 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                         bulk_commit();
                     }
                 }
+            } else if constexpr (TS16) {
+                // every row staged (whole tiles) and every TMEM read done: release, then one
+                // thread stores the tile's int16 sums with one TMA store
+                if (valid_rows == p.cv_rows * p.cv_W) fence_proxy_async();
+                named_bar_sync(bar_id, 128);
+                mbar_arrive(bar_tempty + 8 * acc);
+                if (et == 0 && valid_rows == p.cv_rows * p.cv_W) {
+                    tma_store_2d(&tmZ, smem_u32(sStage + wg * (128 * 128)), n0 * 2, (int)row_base);
+                    bulk_commit();
+                }
             } else if constexpr (TS) {
                 // every row staged and every TMEM read done: the accumulator is released, then
                 // one thread stores the warpgroup's tile, one TMA store per 64 columns
@@ -1087,7 +1170,7 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
                 named_bar_sync(bar_id, 128);  // the column tables are rewritten for the next tile
             }
         }
-        if (TS && et == 0) bulk_wait_all();  // every staged store complete before the CTA exits
+        if ((TS || TS16) && et == 0) bulk_wait_all();  // every staged store complete before the CTA exits
     }
 
     tc_fence_before();
