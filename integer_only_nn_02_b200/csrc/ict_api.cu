@@ -1365,9 +1365,9 @@ int run_conv(int dir, const ict_conv_desc *d, const ict_tensor *out, const ConvP
     r.out_ld = out->ld;
     r.out_exp = out->exp;
     r.act = act;
-    const int64_t n = cp.out_rows * (cp.out_cols / 16);
+    const int64_t image_rows = cp.out_rows / d->w;  // one block per image row of the batch
     KTimer kt(s, KC_REQUANT, 3.0 * (double)cp.out_rows * (double)cp.out_cols);
-    ro16_round_kernel<<<(unsigned)cdiv64(n, 256), 256, 0, s>>>(r);
+    ro16_round_kernel<<<(unsigned)image_rows, 256, 0, s>>>(r);
     counted(1);
     return launch_status();
 }

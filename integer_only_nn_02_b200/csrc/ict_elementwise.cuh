@@ -1460,51 +1460,61 @@ __global__ void __launch_bounds__(256) ro16_rows_round_kernel(const __grid_const
     }
 }
 
+// One block per image row of the whole batch (the row's pixels share one output tile,
+// so its tile index is worked out once), threads over (pixel, 16-column chunk); the
+// rounding by s = e - (tile need - 7) bits runs on the fp32 pipe while s <= 22 (|t| < 2^15).
 __global__ void __launch_bounds__(256) ro16_round_kernel(const __grid_constant__ Ro16RoundArgs a) {
-    const int64_t cv = a.cols / 16;
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= a.rows * cv) return;
-    const int64_t i = idiv(t, cv), j0 = (t - i * cv) * 16;
-    const int64_t g = idiv(j0, a.G);  // 16 | G, so one group per thread
-    const int e = finalize_exp(a.gmax[g]);
-    if (i == 0 && j0 == g * a.G) a.out_exp[g] = (int8_t)e;
-    // output tile of pixel i
-    const int64_t prow = idiv(i, a.cv_W);               // image row over the whole batch
-    const int64_t img = idiv(prow, a.cv_P), h = prow - img * a.cv_P;
-    const int64_t tile = img * a.cv_tiles_per_img + idiv(h, a.cv_rows);
-    const int tn = a.tile_need[tile * a.ngc + g];
-    const int64_t s64 = (int64_t)e - ((int64_t)tn - 7);
-    const int s = (int)(s64 > 40 ? 40 : s64);
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.v + i * a.ld + j0);
-    const uint4 x0 = src[0], x1 = src[1];
-    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    uint32_t o[4];
-    if (s >= 2 && s < 32) {
-        const int m = 1 << (32 - s), bias = (1 << (s - 1)) - 1;
+    const int64_t prow = blockIdx.x;  // image row over the whole batch
+    const int64_t img = idiv(prow, a.cv_P);
+    const int h = (int)(prow - img * a.cv_P);
+    const int64_t tile = img * a.cv_tiles_per_img + h / a.cv_rows;
+    const int cv = (int)(a.cols / 16), per_row = a.cv_W * cv;
+    for (int t = threadIdx.x; t < per_row; t += blockDim.x) {
+        const int w = t / cv, c16 = t - w * cv;
+        const int64_t i = prow * a.cv_W + w, j0 = (int64_t)c16 * 16;
+        const int64_t g = idiv(j0, a.G);  // 16 | G, so one group per thread
+        const int e = finalize_exp(a.gmax[g]);
+        if (i == 0 && j0 == g * a.G) a.out_exp[g] = (int8_t)e;
+        const int tn = a.tile_need[tile * a.ngc + g];
+        const int64_t s64 = (int64_t)e - ((int64_t)tn - 7);
+        const int s = (int)(s64 > 40 ? 40 : s64);
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.v + i * a.ld + j0);
+        const uint4 x0 = src[0], x1 = src[1];
+        const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        uint32_t o[4];
+        if (s >= 2 && s <= 22) {
+            const RneF32 k = rne_f32_consts(s);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            int y[4];
+            for (int q = 0; q < 4; ++q)
+                o[q] = pack4b(rne_f32((int)(int16_t)xw[2 * q], k), rne_f32((int)xw[2 * q] >> 16, k),
+                              rne_f32((int)(int16_t)xw[2 * q + 1], k), rne_f32((int)xw[2 * q + 1] >> 16, k));
+        } else if (s >= 2 && s < 32) {
+            const int m = 1 << (32 - s), bias = (1 << (s - 1)) - 1;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int x = (int)(int16_t)(xw[2 * q + (k >> 1)] >> (16 * (k & 1)));
-                y[k] = __mulhi(x + bias + (__mulhi(x, m) & 1), m);
+            for (int q = 0; q < 4; ++q) {
+                int y[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int x = (int)(int16_t)(xw[2 * q + (kk >> 1)] >> (16 * (kk & 1)));
+                    y[kk] = __mulhi(x + bias + (__mulhi(x, m) & 1), m);
+                }
+                o[q] = pack4(y[0], y[1], y[2], y[3]);
             }
-            o[q] = pack4(y[0], y[1], y[2], y[3]);
-        }
-    } else if (s >= 32) {
-        o[0] = o[1] = o[2] = o[3] = 0u;  // |t| < 2^15: the value is below half a unit
-    } else {
-        // e below the tile's need only after an exponent overflow (status raised)
+        } else if (s >= 32) {
+            o[0] = o[1] = o[2] = o[3] = 0u;  // |t| < 2^15: the value is below half a unit
+        } else {
+            // e below the tile's need only after an exponent overflow (status raised)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            int y[4];
+            for (int q = 0; q < 4; ++q) {
+                int y[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                y[k] = requant32((int)(int16_t)(xw[2 * q + (k >> 1)] >> (16 * (k & 1))), tn - 7, e);
-            o[q] = pack4(y[0], y[1], y[2], y[3]);
+                for (int kk = 0; kk < 4; ++kk)
+                    y[kk] = requant32((int)(int16_t)(xw[2 * q + (kk >> 1)] >> (16 * (kk & 1))), tn - 7, e);
+                o[q] = pack4(y[0], y[1], y[2], y[3]);
+            }
         }
+        *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = apply_act(make_uint4(o[0], o[1], o[2], o[3]), a.act, e);
     }
-    *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + j0) = apply_act(make_uint4(o[0], o[1], o[2], o[3]), a.act, e);
 }
 
 // Sum of split-K int32 slices, transposed: out[c][r] = sum_s in[s][r][c] (int64, row
