@@ -322,9 +322,10 @@ void launch_align_transpose(AlignPair &P, int n, int sms, cudaStream_t s) {
 // Rows of 16-byte vectors, one row per segment of L lanes.  The narrowest segment whose
 // lanes hold at most six vectors each (the most bytes in flight per lane) and stay nine
 // tenths busy, else the busiest; NV = the row's vectors per lane rounded up to an
-// instantiated count.  Rows of fewer than 8 or more than 192 vectors or (computing e*)
-// more than 2 L groups, and 2^31 rows or more, go to the generic kernel.  Persistent grid: two blocks
-// per SM.
+// instantiated count.  Rows of at most four vectors along the rows (with at most four
+// groups when computing e*) take one thread per row; other rows of fewer than 8 or more
+// than 192 vectors or (computing e*) more than 2 L groups, and 2^31 rows or more, go to the
+// generic kernel.  Persistent grid: two blocks per SM.
 int launch_align_rows(const AlignArgs &a, cudaStream_t s, int sms) {
     const int64_t vpr = a.cols / 16;
     const bool row_e = a.axis == 1 && a.row_estar;
@@ -336,6 +337,11 @@ int launch_align_rows(const AlignArgs &a, cudaStream_t s, int sms) {
         const double eff = (double)vpr / (double)(l * per);
         if (eff >= 0.9) { L = l; break; }
         if (eff > best + 1e-12) best = eff, L = l;
+    }
+    if (a.axis == 1 && vpr <= 4 && (!a.row_estar || a.ngc <= 4) && a.rows < (1ll << 31)) {  // thin rows
+        const unsigned grid = (unsigned)std::min<int64_t>(cdiv64(a.rows, 256), (int64_t)sms * 8);
+        align_rows_thin_kernel<<<grid, 256, 0, s>>>(a);
+        return ICT_OK;
     }
     if (L == 0 || vpr < 8 || a.rows >= (1ll << 31)) {  // narrow rows: four threads per row
         align_rows_wide_kernel<<<dim3((unsigned)cdiv64(a.cols, 256), (unsigned)cdiv64(a.rows, 64)), 256, 0, s>>>(a);

@@ -381,6 +381,43 @@ __global__ void __launch_bounds__(256, 2) align_rows_kernel(const __grid_constan
     }
 }
 
+// Rows of at most four 16-byte vectors and (computing e*) at most four groups, such as the
+// 64-channel pixel rows of a convolution, along the rows: one thread per row, every vector
+// and group exponent of the row loaded at once (64 bytes in flight per thread); the row's
+// e* is the largest of its group exponents (E_ZERO, the smallest byte, only when every
+// group is zero).
+__global__ void __launch_bounds__(256) align_rows_thin_kernel(const __grid_constant__ AlignArgs a) {
+    __shared__ RneK tk[9];
+    rne_table_init(tk);
+    __syncthreads();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int nv = (int)(a.cols >> 4);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.rows; i += stride) {
+        const int8_t *e = a.in_exp + idiv(i, a.g_rows) * a.ngc;
+        uint4 raw[4];
+        int eg[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            if (v < nv) {
+                raw[v] = *reinterpret_cast<const uint4 *>(a.in + i * a.ld + 16 * v);
+                eg[v] = e[idiv(16 * v, a.g_cols)];
+            }
+        }
+        int es;
+        if (a.row_estar) {
+            es = kEZero;
+            for (int g = 0; g < (int)a.ngc; ++g) es = max(es, (int)e[g]);
+            a.e_star[i] = (int8_t)es;
+        } else {
+            es = a.e_star[i];
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            if (v < nv)
+                *reinterpret_cast<uint4 *>(a.out + i * a.out_ld + 16 * v) = rne_shift16_k(raw[v], tk[rne_index(es, eg[v])]);
+    }
+}
+
 // The same for rows too wide for one batch per lane or with many groups: 64 x 256
 // tiles, four threads per row with four 16-byte vectors each (columns j, j + 64,
 // j + 128, j + 192), loaded before the row's target is known; with axis 1 and no given
